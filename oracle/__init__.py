@@ -1,0 +1,209 @@
+"""fp64 CPU oracle for the selective scan (S6) and its scalar-A (SSD) form.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``, ``smoke()`` in
+``__graft_entry__.py`` and the CPU-baseline / reference leg of ``bench.py``
+import this package.  It shares no code with the CUDA path and never imports
+it; the product path never imports this package.
+
+The arithmetic lives in ``selscan_oracle.c`` (plain single-threaded loops in
+double precision, each routine citing the page passage it follows).  This
+module only compiles that file with gcc and marshals numpy arrays into it.
+
+Pinned by ``tests/test_oracle_pins.py`` against: a brute-force unrolled sum,
+the time-invariant (LTI) special case as a causal convolution, the closed
+form of a one-state geometric series (``tests/golden``), the Delta = 0 and
+large-Delta gate invariants, linearity in the input, decode-step == scan,
+scalar-A == diagonal scan with broadcast A, and the SSD chunked form ==
+recurrence for several chunk lengths.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "selscan_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call([
+        "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+        "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        common = [_i64] * 5
+        lib.oracle_selscan.argtypes = common + [
+            _dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp,
+            _dp, _dp, _i64, _i64]
+        lib.oracle_selscan_step.argtypes = [_i64] * 4 + [
+            _dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
+        scal = [_i64] * 6 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp,
+                             _dp, _dp, _dp, _dp, _dp]
+        lib.oracle_selscan_scalarA.argtypes = scal + [_i64, _i64]
+        lib.oracle_ssd_chunked.argtypes = scal + [_i64]
+        for f in (lib.oracle_selscan, lib.oracle_selscan_step,
+                  lib.oracle_selscan_scalarA, lib.oracle_ssd_chunked):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None, None
+    arr = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    return arr, arr.ctypes.data_as(_dp)
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (code {rc})")
+
+
+def _bc4(B, batch):
+    """B/C given as (batch, N, L) are one group: view as (batch, 1, N, L)."""
+    B = np.asarray(B)
+    if B.ndim == 3:
+        B = B.reshape(batch, 1, B.shape[1], B.shape[2])
+    return B
+
+
+def selscan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+            delta_softplus=True, h0=None, channels=None):
+    """Diagonal-A selective scan in fp64.
+
+    u, delta, z: (batch, dim, L); A: (dim, N); B, C: (batch, N, L) or
+    (batch, G, N, L); D, delta_bias: (dim,); h0: (batch, dim, N).
+    ``channels`` = (begin, end) restricts the computation to those channels
+    (the returned arrays then hold only those rows).
+    Returns (y, last_state) as float64 arrays.
+    """
+    u = np.asarray(u)
+    batch, dim, L = u.shape
+    A = np.asarray(A)
+    N = A.shape[1]
+    B4, C4 = _bc4(B, batch), _bc4(C, batch)
+    G = B4.shape[1]
+    d0, d1 = (0, dim) if channels is None else channels
+    keep = []
+    uu, up = _f64(u); keep.append(uu)
+    dd, dp_ = _f64(delta); keep.append(dd)
+    bb, bp = _f64(delta_bias); keep.append(bb)
+    aa, ap = _f64(A); keep.append(aa)
+    BB, Bp = _f64(B4); keep.append(BB)
+    CC, Cp = _f64(C4); keep.append(CC)
+    DD, Dp = _f64(D); keep.append(DD)
+    zz, zp = _f64(z); keep.append(zz)
+    hh, hp = _f64(h0); keep.append(hh)
+    y = np.zeros((batch, dim, L), dtype=np.float64)
+    hs = np.zeros((batch, dim, N), dtype=np.float64)
+    rc = _load().oracle_selscan(
+        batch, dim, N, L, G, up, dp_, bp, int(bool(delta_softplus)), ap, Bp,
+        Cp, Dp, zp, hp, y.ctypes.data_as(_dp), hs.ctypes.data_as(_dp), d0, d1)
+    _check(rc)
+    return y[:, d0:d1], hs[:, d0:d1]
+
+
+def selscan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                 delta_softplus=True):
+    """One decode step.  state: (batch, dim, N) (not modified; a new state is
+    returned); u, delta, z: (batch, dim); B, C: (batch, N) or (batch, G, N).
+    Returns (y, new_state)."""
+    st = np.array(state, dtype=np.float64, copy=True, order="C")
+    batch, dim, N = st.shape
+    B = np.asarray(B)
+    C = np.asarray(C)
+    if B.ndim == 2:
+        B = B.reshape(batch, 1, N)
+        C = C.reshape(batch, 1, N)
+    G = B.shape[1]
+    keep = []
+    uu, up = _f64(u); keep.append(uu)
+    dd, dp_ = _f64(delta); keep.append(dd)
+    bb, bp = _f64(delta_bias); keep.append(bb)
+    aa, ap = _f64(A); keep.append(aa)
+    BB, Bp = _f64(B); keep.append(BB)
+    CC, Cp = _f64(C); keep.append(CC)
+    DD, Dp = _f64(D); keep.append(DD)
+    zz, zp = _f64(z); keep.append(zz)
+    y = np.zeros((batch, dim), dtype=np.float64)
+    rc = _load().oracle_selscan_step(
+        batch, dim, N, G, up, dp_, bp, int(bool(delta_softplus)), ap, Bp, Cp,
+        Dp, zp, st.ctypes.data_as(_dp), y.ctypes.data_as(_dp))
+    _check(rc)
+    return y, st
+
+
+def _scalar_args(x, dt, A, B, C, D, z, dt_bias, h0, headdim):
+    x = np.asarray(x)
+    batch, dim, L = x.shape
+    nheads = np.asarray(A).shape[0]
+    if dim != nheads * headdim:
+        raise ValueError("x.shape[1] must equal nheads * headdim")
+    B4, C4 = _bc4(B, batch), _bc4(C, batch)
+    G, N = B4.shape[1], B4.shape[2]
+    keep = []
+    ptrs = []
+    for a in (x, dt, dt_bias):
+        arr, p = _f64(a); keep.append(arr); ptrs.append(p)
+    rest = []
+    for a in (A, B4, C4, D, z, h0):
+        arr, p = _f64(a); keep.append(arr); rest.append(p)
+    return (batch, nheads, headdim, N, L, G), ptrs, rest, keep
+
+
+def selscan_scalarA(x, dt, A, B, C, headdim, D=None, z=None, dt_bias=None,
+                    dt_softplus=False, h0=None, heads=None):
+    """Scalar-A scan, recurrent form.  x, z: (batch, H*P, L); dt: (batch, H, L);
+    A, D, dt_bias: (H,); B, C: (batch, G, N, L) or (batch, N, L);
+    h0: (batch, H, P, N).  ``heads`` = (begin, end) restricts the heads
+    computed (returned arrays hold only those heads' channels/states).
+    Returns (y, last_state) in float64."""
+    dims, ptrs, rest, keep = _scalar_args(x, dt, A, B, C, D, z, dt_bias, h0,
+                                          headdim)
+    batch, nheads, P, N, L, G = dims
+    h0_, h1_ = (0, nheads) if heads is None else heads
+    y = np.zeros((batch, nheads * P, L), dtype=np.float64)
+    hs = np.zeros((batch, nheads, P, N), dtype=np.float64)
+    rc = _load().oracle_selscan_scalarA(
+        *dims, ptrs[0], ptrs[1], ptrs[2], int(bool(dt_softplus)), *rest,
+        y.ctypes.data_as(_dp), hs.ctypes.data_as(_dp), h0_, h1_)
+    _check(rc)
+    return y[:, h0_ * P:h1_ * P], hs[:, h0_:h1_]
+
+
+def ssd_chunked(x, dt, A, B, C, headdim, chunk, D=None, z=None, dt_bias=None,
+                dt_softplus=False, h0=None):
+    """Scalar-A scan in the chunked SSD matrix form (same arguments as
+    ``selscan_scalarA`` plus the chunk length).  Returns (y, last_state)."""
+    dims, ptrs, rest, keep = _scalar_args(x, dt, A, B, C, D, z, dt_bias, h0,
+                                          headdim)
+    batch, nheads, P, N, L, G = dims
+    y = np.zeros((batch, nheads * P, L), dtype=np.float64)
+    hs = np.zeros((batch, nheads, P, N), dtype=np.float64)
+    rc = _load().oracle_ssd_chunked(
+        *dims, ptrs[0], ptrs[1], ptrs[2], int(bool(dt_softplus)), *rest,
+        y.ctypes.data_as(_dp), hs.ctypes.data_as(_dp), int(chunk))
+    _check(rc)
+    return y, hs
