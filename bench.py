@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the selective-scan forward (S6) on B200.
+
+Default workload: the Mamba-2.8B-like layer scan -- batch 4, d_inner 5120,
+d_state 16, L 4096, bf16 u/delta/z/B/C, fp32 A/D/state, softplus on delta,
+D skip and silu(z) gate.  A "step" is one selscan_fwd call over that batch
+(the whole hot path: softplus, discretisation, scan, output contraction,
+gate, final state).  Throughput is elements (batch * d_inner * L) per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, timed
+
+For N > 1 (launched with torch.distributed.run) each rank scans its own
+independent shard of the same shape (the path has no exchange step), so the
+scaling is weak; the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "selective-scan Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU"
+HBM_FALLBACK_GBS = 6650.0
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": 1590.0}, "fallback"
+
+
+# ------------------------------------------------------------ byte counts
+def algorithmic_bytes(cfg: dict) -> int:
+    """Bytes one call must move at minimum: every input read once, every
+    output written once (the expanded state is never stored)."""
+    es = 2 if cfg["dtype"] == "bf16" else 4
+    b, L = cfg["batch"], cfg["L"]
+    if cfg["kind"] == "diag":
+        dim, N = cfg["dim"], cfg["N"]
+        stream = (3 if cfg["gate"] else 2) * es + es           # u, delta, (z) + y
+        total = b * dim * L * stream
+        total += 2 * b * N * L * es                             # B, C
+        total += dim * N * 4 + dim * 4 * (2 if cfg["D"] else 1)  # A, bias, D
+        total += b * dim * N * 4                                 # last_state
+        return total
+    H, P, N, G = cfg["nheads"], cfg["headdim"], cfg["N"], cfg["ngroups"]
+    dim = H * P
+    total = b * dim * L * es * (3 if cfg["gate"] else 2)        # x, (z), y
+    total += b * H * L * 4                                       # dt
+    total += 2 * b * G * N * L * es                              # B, C
+    total += H * 4 * 3                                           # A, D, bias
+    total += b * H * P * N * 4                                   # last_state
+    return total
+
+
+def ssd_flops(cfg: dict) -> float:
+    """Tensor-core FLOPs of the chunked SSD form per call (C.B^T once per
+    batch and chunk since heads share B/C; per head the intra-chunk product,
+    the chunk state and the carried-in term)."""
+    b, L, Q = cfg["batch"], cfg["L"], cfg["chunk"]
+    H, P, N = cfg["nheads"], cfg["headdim"], cfg["N"]
+    nch = (L + Q - 1) // Q
+    per_chunk = 2 * Q * Q * N + H * (2 * Q * Q * P + 2 * N * Q * P + 2 * Q * N * P)
+    return float(b * nch * per_chunk)
+
+
+# ------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._pump, daemon=True)
+        self.t.start()
+        time.sleep(0.3)  # let nvidia-smi start reporting
+
+    def _pump(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0: float, t1: float) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [l for (ts, l) in self.lines if t0 <= ts <= t1] or [l for (_, l) in self.lines]
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [p.strip() for p in r.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def physical_gpu_index(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids) and ids[local].isdigit():
+            return int(ids[local])
+    return local
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample(cfg_idx: int, inp: dict, seconds: float = 10.0):
+    """Time the fp64 oracle on a bounded sample of the workload: whole
+    channels (all tokens, all batches) of the first d_inner rows, grown
+    until about `seconds` of single-threaded CPU work."""
+    import oracle
+    cfg = synthetic.CONFIGS[cfg_idx]
+    L, b = cfg["L"], cfg["batch"]
+    n = 1
+    spent = 0.0
+    done_elems = 0
+    while True:
+        t0 = time.perf_counter()
+        if cfg["kind"] == "diag":
+            oracle.selscan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                           z=inp["z"], delta_bias=inp["delta_bias"],
+                           delta_softplus=inp["softplus"], channels=(0, n))
+            elems = b * n * L
+            unit = f"{n} channel(s)"
+        else:
+            P = cfg["headdim"]
+            h = max(1, n // P)
+            oracle.selscan_scalarA(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], P,
+                                   D=inp["D"], z=inp["z"], heads=(0, h))
+            elems = b * h * P * L
+            unit = f"{h} head(s)"
+        dt = time.perf_counter() - t0
+        spent, done_elems = dt, elems
+        if dt >= seconds * 0.5 or n >= (cfg.get("dim") or cfg["nheads"] * cfg["headdim"]):
+            break
+        grow = max(2.0, min(16.0, seconds / max(dt, 1e-3)))
+        n = int(min(n * grow, cfg.get("dim") or cfg["nheads"] * cfg["headdim"]))
+    return {"value": done_elems / spent / 1e9, "unit": "Gelem/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{unit} x batch {b} x L {L} = {done_elems} elements, "
+                      f"{spent:.1f} s single-threaded fp64"}
+
+
+def run_reference(args, rank: int, world: int):
+    """Reference arm: the fp64 oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    cfg = synthetic.CONFIGS[args.config]
+    inp = synthetic.make_config(args.config)
+    import oracle
+    # one step = one whole channel (all batches, all tokens) of the workload;
+    # grow to several channels if that is too fast to time
+    per_step_channels = 1
+    L, b = cfg["L"], cfg["batch"]
+
+    def step(i):
+        if cfg["kind"] == "diag":
+            c0 = (i * per_step_channels) % cfg["dim"]
+            oracle.selscan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                           z=inp["z"], delta_bias=inp["delta_bias"],
+                           delta_softplus=inp["softplus"], channels=(c0, c0 + per_step_channels))
+            return b * per_step_channels * L
+        P = cfg["headdim"]
+        h = i % cfg["nheads"]
+        oracle.selscan_scalarA(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], P,
+                               D=inp["D"], z=inp["z"], heads=(h, h + 1))
+        return b * P * L
+
+    budget = 150.0  # keep the whole reference run within a few minutes
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    elems = 0
+    steps_done = 0
+    for i in range(args.steps):
+        elems += step(i)
+        steps_done += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    dt = time.perf_counter() - t0
+    val = elems / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "Gelem/s",
+        "n_gpus": world, "steps": steps_done, "warmup": args.warmup,
+        "ms_per_step": dt / steps_done * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg["name"], "sample_per_step": "one channel (all batches, all tokens)"
+                   if cfg["kind"] == "diag" else "one head"},
+        "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{steps_done} steps x {elems // max(steps_done, 1)} elements"},
+        "e2e": {"value": val, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ GPU arm
+def to_dev(a, dtype, torch):
+    if a is None:
+        return None
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return (t.to(torch.bfloat16) if dtype == "bf16" else t.float()).cuda()
+
+
+def run_gpu(args, rank: int, world: int, local: int):
+    import torch
+    import selective_state_space_selscan_b200 as ss
+    torch.cuda.set_device(local)
+    cfg = synthetic.CONFIGS[args.config]
+    inp = synthetic.make_config(args.config)
+    dt = cfg["dtype"]
+    stream = torch.cuda.current_stream()
+    if cfg["kind"] == "diag":
+        dev = {k: to_dev(inp[k], dt, torch) for k in ("u", "delta", "B", "C", "z")}
+        dev.update({k: to_dev(inp[k], "f32", torch) for k in ("A", "D", "delta_bias")})
+        y = torch.empty_like(dev["u"])
+        hs = torch.empty((cfg["batch"], cfg["dim"], cfg["N"]), dtype=torch.float32,
+                         device="cuda")
+
+        def call():
+            ss.selscan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
+                           z=dev["z"], delta_bias=dev["delta_bias"], delta_softplus=True,
+                           out=y, last_state=hs)
+        host_in = ("u", "delta", "B", "C", "z", "A", "D", "delta_bias")
+        kernels_per_step = 1
+    else:
+        dev = {k: to_dev(inp[k], dt, torch) for k in ("x", "B", "C", "z")}
+        dev.update({k: to_dev(inp[k], "f32", torch) for k in ("dt", "A", "D")})
+        y = torch.empty_like(dev["x"])
+        hs = torch.empty((cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["N"]),
+                         dtype=torch.float32, device="cuda")
+
+        def call():
+            ss.selscan_fwd_scalarA(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"],
+                                   cfg["headdim"], D=dev["D"], z=dev["z"], out=y,
+                                   last_state=hs)
+        host_in = ("x", "dt", "B", "C", "z", "A", "D")
+        kernels_per_step = ss_kernels_per_step_scalarA()
+
+    elems = synthetic.elements(args.config)
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    ss.check()
+    barrier()
+    torch.cuda.synchronize()
+
+    # timed region: K steps, per-launch events on the launching stream
+    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    ss.check()
+    total_ms = start.elapsed_time(end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    clock_info = clocks.stop(t_wall0, t_wall1) if clocks else None
+    if dist:
+        t = torch.tensor([total_ms, statistics.mean(launch_ms)], device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms, avg_launch_ms = float(t[0]), float(t[1])
+    else:
+        avg_launch_ms = statistics.mean(launch_ms)
+    ms_per_step = total_ms / args.steps
+    value = world * elems / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host inputs -> device,
+    # scan, result back to the host, every step
+    pinned = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(
+        torch.bfloat16 if (dt == "bf16" and k not in ("A", "D", "delta_bias", "dt")) else
+        torch.float32).pin_memory() for k in host_in if inp.get(k) is not None}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    hs_host = torch.empty(hs.shape, dtype=hs.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = y_host.numel() * y_host.element_size() + hs_host.numel() * hs_host.element_size()
+    e2e_steps = max(1, min(args.steps, 10))
+
+    def e2e_step():
+        for k, t in pinned.items():
+            dev[k].copy_(t, non_blocking=True)
+        call()
+        y_host.copy_(y, non_blocking=True)
+        hs_host.copy_(hs, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    barrier()
+    if rank != 0:
+        return
+
+    peaks, peaks_src = measured_peaks()
+    nbytes = algorithmic_bytes(cfg)
+    achieved = nbytes / (avg_launch_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": args.traffic,
+            "peak_source": f"{peaks_src} HBM copy bandwidth",
+            "bytes_per_launch": nbytes, "avg_launch_ms": avg_launch_ms}
+    if cfg["kind"] == "scalarA":
+        fl = ssd_flops(cfg)
+        roof["tensor"] = {"flops_per_launch": fl,
+                          "achieved_tflops": fl / (avg_launch_ms * 1e-3) / 1e12,
+                          "peak_tflops": peaks.get("bf16_tflops"),
+                          "frac": fl / (avg_launch_ms * 1e-3) / 1e12 / peaks.get("bf16_tflops", 1590.0)}
+    line = {
+        "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dt, "data": "synthetic",
+        "config": {"workload": cfg["name"], "batch": cfg["batch"],
+                   "d_inner": cfg.get("dim") or cfg["nheads"] * cfg["headdim"],
+                   "d_state": cfg["N"], "seq_len": cfg["L"], "seed": cfg["seed"],
+                   "global_batch": cfg["batch"] * world,
+                   "l2": "inputs larger than L2 (no flush)" if nbytes > 126e6 else
+                         "inputs smaller than L2",
+                   "parallelism": f"dp{world} (independent shards, no collective)"},
+        "roofline": roof,
+        "e2e": {"value": world * elems / (e2e_ms * 1e-3) / 1e9, "unit": "Gelem/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clock_info,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(args.config, inp, seconds=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def ss_kernels_per_step_scalarA() -> int:
+    import selective_state_space_selscan_b200 as ss
+    return getattr(ss, "SCALARA_KERNELS_PER_CALL", 1)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch from an ncu capture of this kernel")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+    try:
+        run_gpu(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

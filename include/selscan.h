@@ -1,0 +1,157 @@
+/*
+ * selscan.h -- C ABI of libselscan, the selective-scan (S6) forward pass for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed (diagonal A).  For every batch b, channel d and token t,
+ * following "03 -- Modelos de espacio de estados: RWKV, S4, Mamba y el
+ * selective scan" (sections "El mecanismo selectivo de Mamba",
+ * "Discretizacion", "Parallel scan") and "P20 -- Mamba" (section 5,
+ * "Matematica minima"):
+ *
+ *   delta_t = softplus(delta[b,d,t] + delta_bias[d])   (softplus optional)
+ *   h_t[n]  = exp(delta_t * A[d,n]) * h_{t-1}[n] + delta_t * B[b,n,t] * u[b,d,t]
+ *   y[b,d,t] = (sum_n C[b,n,t] * h_t[n] + D[d] * u[b,d,t]) * silu(z[b,d,t])
+ *
+ * with h_{-1} = 0 (or the given initial state), A fixed and diagonal, and
+ * B, C, delta depending on the token.  The expanded state (batch, d, L, N)
+ * never reaches device memory ("P20 -- Mamba", section 3: the
+ * hardware-aware algorithm does not materialise the expanded state in slow
+ * memory); only y and the final state are written.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers of the current CUDA device, owned by
+ *     the caller.  The library keeps no pointer after a call returns.
+ *   - Calls are asynchronous on `stream`.  Scratch memory the kernels need
+ *     (look-back carries, flags) is taken with cudaMallocAsync on `stream`
+ *     and released with cudaFreeAsync on the same stream.
+ *   - Tensors are described by selscan_tensor: element type, rank, shape and
+ *     strides in ELEMENTS.  The last (time) dimension must have stride 1.
+ *     Other strides may be anything that keeps rows 16-byte aligned (they
+ *     are multiples of 16 bytes) and the base pointer 16-byte aligned; this
+ *     is what the bulk tensor copies (TMA) require.  For a contiguous bf16
+ *     tensor that means L % 8 == 0; for fp32, L % 4 == 0.
+ *   - Validation errors are returned synchronously and nothing is launched.
+ *     A failed launch returns SELSCAN_ERR_CUDA.  A device-side wait that ran
+ *     out of its iteration limit is recorded on the device and reported by
+ *     the next selscan_check().
+ *   - There is no CPU fallback: every step runs in this library's kernels.
+ */
+#ifndef SELSCAN_H
+#define SELSCAN_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SELSCAN_VERSION 10000 /* 1.0.0 */
+
+#if defined(__GNUC__)
+#define SELSCAN_API __attribute__((visibility("default")))
+#else
+#define SELSCAN_API
+#endif
+
+typedef enum {
+    SELSCAN_OK = 0,
+    SELSCAN_ERR_NULL = 1,        /* a required pointer is NULL            */
+    SELSCAN_ERR_SHAPE = 2,       /* ranks or sizes disagree              */
+    SELSCAN_ERR_STRIDE = 3,      /* time stride != 1, or bad layout      */
+    SELSCAN_ERR_DTYPE = 4,       /* element type not allowed here        */
+    SELSCAN_ERR_ALIGN = 5,       /* pointer / row stride not 16B aligned */
+    SELSCAN_ERR_UNSUPPORTED = 6, /* valid but not built (e.g. N != 16)   */
+    SELSCAN_ERR_CUDA = 7,        /* a CUDA runtime call failed           */
+    SELSCAN_ERR_TIMEOUT = 8      /* a device-side wait gave up           */
+} selscan_status;
+
+typedef enum { SELSCAN_F32 = 0, SELSCAN_BF16 = 1 } selscan_dtype;
+
+typedef struct {
+    void *data;        /* device pointer (NULL allowed only where noted) */
+    int32_t dtype;     /* selscan_dtype                                  */
+    int32_t ndim;      /* 1..4                                           */
+    int64_t shape[4];  /* sizes, outermost first                         */
+    int64_t stride[4]; /* strides in elements                            */
+} selscan_tensor;
+
+/*
+ * selscan_fwd -- diagonal-A selective scan forward.
+ *
+ *   u          (batch, D, L)   F32 or BF16; the input x of the pages
+ *   delta      (batch, D, L)   same dtype as u; raw step size Delta
+ *   delta_bias (D)             F32, contiguous; may be NULL
+ *   delta_softplus             nonzero: delta_t = softplus(delta + bias)
+ *   A          (D, N)          F32, contiguous; should be < 0 (not checked)
+ *   B, C       (batch, N, L) or (batch, 1, N, L)  same dtype as u
+ *   D          (D)             F32, contiguous; may be NULL (no skip term)
+ *   z          (batch, D, L)   same dtype as u; may be NULL (no gate)
+ *   y          (batch, D, L)   same dtype as u; written
+ *   last_state (batch, D, N)   F32, contiguous; may be NULL; written
+ *
+ * N must be 16.  batch, D or L may be 0 (nothing is launched; when L == 0
+ * last_state is zero-filled).  Internal arithmetic is fp32; y is rounded to
+ * u's dtype (round to nearest even).
+ */
+SELSCAN_API selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
+                           const selscan_tensor *delta_bias, int delta_softplus,
+                           const selscan_tensor *A, const selscan_tensor *B,
+                           const selscan_tensor *C, const selscan_tensor *D,
+                           const selscan_tensor *z, selscan_tensor *y,
+                           selscan_tensor *last_state, cudaStream_t stream);
+
+/*
+ * selscan_fwd_scalarA -- scalar-A (Mamba-2 / SSD) selective scan forward.
+ * The transition is one scalar per head times the identity ("Mamba-3: un
+ * modelo de espacio de estados centrado en la inferencia", first section),
+ * so the scan can be evaluated in the chunked matrix form of structured
+ * state-space duality ("Mamba-2 y state-space models", section 4.2) on the
+ * tensor cores.  Channel d = h * headdim + p belongs to head h.
+ *
+ *   x          (batch, H*P, L)  BF16
+ *   dt         (batch, H, L)    F32; per-head step size
+ *   dt_bias    (H)              F32; may be NULL
+ *   dt_softplus                 nonzero: step = softplus(dt + dt_bias)
+ *   A          (H)              F32 (< 0)
+ *   B, C       (batch, G, N, L) BF16; head h reads group h / (H / G)
+ *   D          (H)              F32; may be NULL
+ *   z          (batch, H*P, L)  BF16; may be NULL (no gate)
+ *   headdim    P
+ *   y          (batch, H*P, L)  BF16; written
+ *   last_state (batch, H, P, N) F32, contiguous; may be NULL; written
+ *
+ * Built for N = 128, P = 64, G = 1; other sizes return
+ * SELSCAN_ERR_UNSUPPORTED.
+ */
+SELSCAN_API selscan_status selscan_fwd_scalarA(const selscan_tensor *x,
+                                   const selscan_tensor *dt,
+                                   const selscan_tensor *dt_bias,
+                                   int dt_softplus, const selscan_tensor *A,
+                                   const selscan_tensor *B,
+                                   const selscan_tensor *C,
+                                   const selscan_tensor *D,
+                                   const selscan_tensor *z, int64_t headdim,
+                                   selscan_tensor *y,
+                                   selscan_tensor *last_state,
+                                   cudaStream_t stream);
+
+/*
+ * selscan_check -- synchronise `stream` and report device-side errors that
+ * earlier calls recorded (a bounded wait that gave up returns
+ * SELSCAN_ERR_TIMEOUT; the record is then cleared).  Returns
+ * SELSCAN_ERR_CUDA if the synchronisation itself failed.
+ */
+SELSCAN_API selscan_status selscan_check(cudaStream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+SELSCAN_API const char *selscan_strerror(selscan_status status);
+
+/* SELSCAN_VERSION of the built library. */
+SELSCAN_API int selscan_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SELSCAN_H */

@@ -1,0 +1,29 @@
+/*
+ * selscan_debug.h -- test hooks of libselscan.  Not needed by normal
+ * callers; they exist so that the failure paths of the device-side bounded
+ * waits can be exercised without faulting or hanging a GPU.
+ */
+#ifndef SELSCAN_DEBUG_H
+#define SELSCAN_DEBUG_H
+
+#include "selscan.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * Withhold the carry flag of work unit `unit` in subsequent selscan_fwd
+ * calls (-1 switches the hook off).  The unit that waits for that carry
+ * gives up after its time limit (SELSCAN_WAIT_TIMEOUT_MS, default 2000 ms),
+ * continues from a zero state and records the event; the next
+ * selscan_check() returns SELSCAN_ERR_TIMEOUT.  Work units are numbered
+ * segment-major: unit = segment * tiles + tile.
+ */
+SELSCAN_API void selscan_debug_withhold_carry(int unit);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SELSCAN_DEBUG_H */

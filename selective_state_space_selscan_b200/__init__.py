@@ -1,0 +1,176 @@
+"""libselscan: selective-scan (S6) forward for NVIDIA B200 (sm_100a).
+
+This package is a thin ctypes binding over the C ABI in ``include/selscan.h``
+(built in-tree as ``libselscan.so`` by ``build.py``).  It only marshals
+arguments: every step of the scan runs in the library's CUDA kernels.  There
+is no CPU fallback; if the shared library is missing the functions raise.
+
+PyTorch is used for device memory and streams only: tensors are passed by
+pointer, shape and strides.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libselscan.so")
+
+SELSCAN_F32 = 0
+SELSCAN_BF16 = 1
+
+STATUS = {
+    0: "SELSCAN_OK", 1: "SELSCAN_ERR_NULL", 2: "SELSCAN_ERR_SHAPE",
+    3: "SELSCAN_ERR_STRIDE", 4: "SELSCAN_ERR_DTYPE", 5: "SELSCAN_ERR_ALIGN",
+    6: "SELSCAN_ERR_UNSUPPORTED", 7: "SELSCAN_ERR_CUDA", 8: "SELSCAN_ERR_TIMEOUT",
+}
+STATUS_CODE = {v: k for k, v in STATUS.items()}
+
+# entry points declared in include/selscan.h
+EXPORTS = ("selscan_fwd", "selscan_fwd_scalarA", "selscan_check",
+           "selscan_strerror", "selscan_version")
+
+
+class SelscanError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        self.name = STATUS.get(status, f"status {status}")
+        super().__init__(f"{where}: {self.name} ({_strerror(status)})")
+
+
+class SelscanTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32),
+                ("ndim", ctypes.c_int32), ("shape", ctypes.c_int64 * 4),
+                ("stride", ctypes.c_int64 * 4)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libselscan.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m selective_state_space_selscan_b200.build` "
+                "(there is no fallback implementation)")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(SelscanTensor)
+        L.selscan_fwd.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, P, P, P,
+                                  ctypes.c_void_p]
+        L.selscan_fwd_scalarA.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, P,
+                                          ctypes.c_int64, P, P, ctypes.c_void_p]
+        L.selscan_check.argtypes = [ctypes.c_void_p]
+        L.selscan_strerror.argtypes = [ctypes.c_int]
+        L.selscan_strerror.restype = ctypes.c_char_p
+        L.selscan_version.argtypes = []
+        for f in (L.selscan_fwd, L.selscan_fwd_scalarA, L.selscan_check,
+                  L.selscan_version):
+            f.restype = ctypes.c_int
+        L.selscan_debug_withhold_carry.argtypes = [ctypes.c_int]
+        L.selscan_debug_withhold_carry.restype = None
+        _lib = L
+    return _lib
+
+
+def _strerror(status: int) -> str:
+    try:
+        return lib().selscan_strerror(int(status)).decode()
+    except Exception:  # pragma: no cover - only when the library is absent
+        return STATUS.get(status, "unknown")
+
+
+def version() -> int:
+    return lib().selscan_version()
+
+
+def describe(t, dtype_code=None) -> SelscanTensor | None:
+    """selscan_tensor for a torch tensor (None stays None -> NULL)."""
+    if t is None:
+        return None
+    import torch
+    d = SelscanTensor()
+    d.data = t.data_ptr()
+    if dtype_code is None:
+        dtype_code = {torch.float32: SELSCAN_F32,
+                      torch.bfloat16: SELSCAN_BF16}.get(t.dtype, -1)
+    d.dtype = dtype_code
+    d.ndim = t.dim()
+    for i in range(t.dim()):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _ref(d):
+    return None if d is None else ctypes.byref(d)
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def selscan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                delta_softplus=True, out=None, last_state=None,
+                return_last_state=True, stream=None):
+    """Diagonal-A selective scan forward through the C ABI.
+
+    u, delta, z: (batch, D, L) bf16 or fp32 CUDA tensors (time stride 1);
+    A: (D, N=16) fp32; B, C: (batch, N, L) same dtype as u; D, delta_bias:
+    (D,) fp32.  Returns (y, last_state); last_state is None unless requested.
+    """
+    import torch
+    y = out if out is not None else torch.empty_like(u, memory_format=torch.contiguous_format)
+    if last_state is None and return_last_state:
+        last_state = torch.empty((u.shape[0], u.shape[1], A.shape[1]),
+                                 dtype=torch.float32, device=u.device)
+    descs = [describe(t) for t in (u, delta, delta_bias, A, B, C, D, z, y, last_state)]
+    rc = lib().selscan_fwd(_ref(descs[0]), _ref(descs[1]), _ref(descs[2]),
+                           int(bool(delta_softplus)), _ref(descs[3]),
+                           _ref(descs[4]), _ref(descs[5]), _ref(descs[6]),
+                           _ref(descs[7]), _ref(descs[8]), _ref(descs[9]),
+                           _stream_handle(stream))
+    if rc != 0:
+        raise SelscanError(rc, "selscan_fwd")
+    return y, last_state
+
+
+def selscan_fwd_scalarA(x, dt, A, B, C, headdim, D=None, z=None, dt_bias=None,
+                        dt_softplus=False, out=None, last_state=None,
+                        return_last_state=True, stream=None):
+    """Scalar-A (Mamba-2 / SSD) scan forward through the C ABI.
+
+    x, z: (batch, H*P, L) bf16; dt: (batch, H, L) fp32; A, D, dt_bias: (H,)
+    fp32; B, C: (batch, G, N, L) bf16.  Returns (y, last_state (batch, H, P, N)).
+    """
+    import torch
+    y = out if out is not None else torch.empty_like(x, memory_format=torch.contiguous_format)
+    if last_state is None and return_last_state:
+        last_state = torch.empty((x.shape[0], A.shape[0], headdim, B.shape[2]),
+                                 dtype=torch.float32, device=x.device)
+    descs = [describe(t) for t in (x, dt, dt_bias, A, B, C, D, z, y, last_state)]
+    rc = lib().selscan_fwd_scalarA(_ref(descs[0]), _ref(descs[1]), _ref(descs[2]),
+                                   int(bool(dt_softplus)), _ref(descs[3]),
+                                   _ref(descs[4]), _ref(descs[5]), _ref(descs[6]),
+                                   _ref(descs[7]), int(headdim), _ref(descs[8]),
+                                   _ref(descs[9]), _stream_handle(stream))
+    if rc != 0:
+        raise SelscanError(rc, "selscan_fwd_scalarA")
+    return y, last_state
+
+
+def check(stream=None) -> None:
+    """Synchronise ``stream`` and raise if a device-side wait timed out."""
+    rc = lib().selscan_check(_stream_handle(stream))
+    if rc != 0:
+        raise SelscanError(rc, "selscan_check")
+
+
+def debug_withhold_carry(unit: int) -> None:
+    """Test hook: withhold the carry flag of work unit ``unit`` (-1: off)."""
+    lib().selscan_debug_withhold_carry(int(unit))

@@ -1,0 +1,497 @@
+// selscan_api.cu -- C ABI of libselscan (see include/selscan.h): argument
+// validation, tensor-map encoding, stream-ordered scratch memory and kernel
+// launch for the diagonal-A scan and the scalar-A (SSD) scan.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+#include <algorithm>
+
+#include "selscan.h"
+#include "selscan_debug.h"
+#include "scan_diag.cuh"
+#include "ssd_scalarA.cuh"
+
+using namespace selscan;
+
+// Device-side error word: bounded waits that give up OR a bit in here.
+__device__ unsigned int g_selscan_err = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sm_count = 0;
+    unsigned int *err = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+unsigned long long default_timeout_ns()
+{
+    // Upper bound for any single wait inside a kernel.  Normal waits last
+    // microseconds; the bound only matters if something is broken.
+    static unsigned long long v = [] {
+        const char *e = std::getenv("SELSCAN_WAIT_TIMEOUT_MS");
+        unsigned long long ms = e ? std::strtoull(e, nullptr, 10) : 2000ull;
+        if (ms == 0)
+            ms = 2000ull;
+        return ms * 1000000ull;
+    }();
+    return v;
+}
+
+selscan_status device_setup(int *dev_out, DeviceInfo **info_out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return SELSCAN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &di = g_dev[dev];
+    if (!di.ready) {
+        if (cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess)
+            return SELSCAN_ERR_CUDA;
+        if (cudaGetSymbolAddress(reinterpret_cast<void **>(&di.err), g_selscan_err) !=
+            cudaSuccess)
+            return SELSCAN_ERR_CUDA;
+        di.ready = true;
+    }
+    if (!g_encode) {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return SELSCAN_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *dev_out = dev;
+    *info_out = &di;
+    return SELSCAN_OK;
+}
+
+size_t elem_size(int32_t dt) { return dt == SELSCAN_BF16 ? 2 : 4; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t numel(const selscan_tensor *t)
+{
+    int64_t n = 1;
+    for (int i = 0; i < t->ndim && i < 4; ++i)
+        n *= t->shape[i];
+    return n;
+}
+
+// Present: non-NULL descriptor whose data is non-NULL, or that holds no
+// element at all (frameworks hand out NULL data for empty tensors).
+bool present(const selscan_tensor *t)
+{
+    return t && (t->data || (t->ndim >= 1 && t->ndim <= 4 && numel(t) == 0));
+}
+
+// A "sequence" tensor: rank 3 (outer0, outer1, L) with time stride 1 and
+// 16-byte aligned rows, as the bulk tensor copies need.
+selscan_status check_seq(const selscan_tensor *t, int64_t d0, int64_t d1, int64_t L,
+                         int32_t dtype)
+{
+    if (!present(t))
+        return SELSCAN_ERR_NULL;
+    if (t->ndim != 3 || t->shape[0] != d0 || t->shape[1] != d1 || t->shape[2] != L)
+        return SELSCAN_ERR_SHAPE;
+    if (t->dtype != dtype)
+        return SELSCAN_ERR_DTYPE;
+    if (L > 1 && t->stride[2] != 1)
+        return SELSCAN_ERR_STRIDE;
+    if (t->stride[0] < 0 || t->stride[1] < 0)
+        return SELSCAN_ERR_STRIDE;
+    const int64_t es = int64_t(elem_size(dtype));
+    if (!aligned16(t->data) || ((t->stride[0] * es) & 15) || ((t->stride[1] * es) & 15))
+        return SELSCAN_ERR_ALIGN;
+    return SELSCAN_OK;
+}
+
+// A small fp32 parameter tensor with the given shape, contiguous.
+selscan_status check_param(const selscan_tensor *t, int ndim, const int64_t *shape,
+                           bool nullable)
+{
+    if (!t || !t->data) {
+        if (nullable)
+            return SELSCAN_OK;
+        if (!present(t))
+            return SELSCAN_ERR_NULL;
+    }
+    if (t->ndim != ndim)
+        return SELSCAN_ERR_SHAPE;
+    int64_t expect = 1;
+    for (int i = ndim - 1; i >= 0; --i) {
+        if (t->shape[i] != shape[i])
+            return SELSCAN_ERR_SHAPE;
+        if (shape[i] > 1 && t->stride[i] != expect)
+            return SELSCAN_ERR_STRIDE;
+        expect *= shape[i];
+    }
+    if (t->dtype != SELSCAN_F32)
+        return SELSCAN_ERR_DTYPE;
+    if ((reinterpret_cast<uintptr_t>(t->data) & 3u) != 0)
+        return SELSCAN_ERR_ALIGN;
+    return SELSCAN_OK;
+}
+
+const void *opt_data(const selscan_tensor *t) { return (t && t->data) ? t->data : nullptr; }
+
+// 3-D tiled map over (L, rows, outer): box (box_t, box_rows, 1), 128-byte
+// swizzle, zero fill outside the tensor.
+bool encode_3d(CUtensorMap *m, const void *ptr, int32_t dtype, int64_t L, int64_t rows,
+               int64_t outer, int64_t row_stride, int64_t outer_stride, int box_t,
+               int box_rows)
+{
+    const size_t es = elem_size(dtype);
+    cuuint64_t dims[3] = {cuuint64_t(L), cuuint64_t(rows), cuuint64_t(outer)};
+    // strides must be non-zero multiples of 16 even where the extent is 1
+    int64_t rs = row_stride * int64_t(es), os = outer_stride * int64_t(es);
+    if (rows <= 1 && rs == 0)
+        rs = 16 * ((L * int64_t(es) + 15) / 16);
+    if (outer <= 1 && os == 0)
+        os = 16 * ((rows * rs + 15) / 16);
+    cuuint64_t strides[2] = {cuuint64_t(rs), cuuint64_t(os)};
+    cuuint32_t box[3] = {cuuint32_t(box_t), cuuint32_t(box_rows), 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = g_encode(m,
+                          dtype == SELSCAN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          3, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int g_dbg_skip_publish = -1;  // test hook, see selscan_debug_withhold_carry
+
+// ----------------------------------------------------- diagonal-A launch
+template <typename T, int CH, int STAGES, bool GATE>
+selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
+                           const selscan_tensor *B, const selscan_tensor *C,
+                           const selscan_tensor *z, selscan_tensor *y, DiagParams prm,
+                           int sm_count, cudaStream_t stream)
+{
+    using Lay = DiagLayout<T, CH, STAGES, GATE>;
+    constexpr int TC = DiagShape<T>::kChunk;
+    constexpr int CW = CH * 2 / 32;
+    const int32_t dt = u->dtype;
+    const int64_t batch = prm.batch, dim = prm.dim, L = prm.L;
+    const int64_t Bn = kDiagN;
+    // B/C may be rank 3 (batch, N, L) or rank 4 (batch, 1, N, L)
+    auto bc_strides = [](const selscan_tensor *t, int64_t &rs, int64_t &bs) {
+        if (t->ndim == 3) {
+            rs = t->stride[1];
+            bs = t->stride[0];
+        } else {
+            rs = t->stride[2];
+            bs = t->stride[0];
+        }
+    };
+    CUtensorMap tm_u, tm_d, tm_z, tm_B, tm_C, tm_y;
+    int64_t brs, bbs, crs, cbs;
+    bc_strides(B, brs, bbs);
+    bc_strides(C, crs, cbs);
+    bool ok = encode_3d(&tm_u, u->data, dt, L, dim, batch, u->stride[1], u->stride[0], TC, CH) &&
+              encode_3d(&tm_d, delta->data, dt, L, dim, batch, delta->stride[1],
+                        delta->stride[0], TC, CH) &&
+              encode_3d(&tm_B, B->data, dt, L, Bn, batch, brs, bbs, TC, kDiagN) &&
+              encode_3d(&tm_C, C->data, dt, L, Bn, batch, crs, cbs, TC, kDiagN) &&
+              encode_3d(&tm_y, y->data, dt, L, dim, batch, y->stride[1], y->stride[0], TC, CH);
+    if (ok && GATE)
+        ok = encode_3d(&tm_z, z->data, dt, L, dim, batch, z->stride[1], z->stride[0], TC, CH);
+    else
+        tm_z = tm_u;
+    if (!ok)
+        return SELSCAN_ERR_ALIGN;
+
+    // Work decomposition: tiles of CH channels, segments of seg_len tokens.
+    const int tpb = int((dim + CH - 1) / CH);
+    const int G = int(batch) * tpb;
+    const int ctas_max = sm_count;  // one persistent CTA per SM
+    const int64_t chunks = (L + TC - 1) / TC;
+    // aim for about 8 units per CTA so the tail is short, segments >= 4 chunks
+    int64_t want_units = 8ll * ctas_max;
+    int64_t S = (want_units + G - 1) / G;
+    S = std::max<int64_t>(1, std::min<int64_t>(S, (chunks + 3) / 4));
+    int64_t seg_chunks = (chunks + S - 1) / S;
+    S = (chunks + seg_chunks - 1) / seg_chunks;
+    prm.tiles_per_batch = tpb;
+    prm.num_tiles = G;
+    prm.seg_len = int(seg_chunks * TC);
+    prm.num_segs = int(S);
+    const int64_t units = int64_t(G) * S;
+    if (units > 0x7fffffffll)
+        return SELSCAN_ERR_UNSUPPORTED;
+    prm.total_units = int(units);
+
+    // scratch: ticket | flags[units][CW] | carry[units][CH][16]
+    const size_t head = 256;
+    const size_t flag_bytes = ((size_t(units) * CW * 4 + 255) / 256) * 256;
+    const size_t carry_bytes = size_t(units) * CH * kDiagN * 4;
+    const size_t ws_bytes = head + flag_bytes + carry_bytes;
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess)
+        return SELSCAN_ERR_CUDA;
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    if (cudaMemsetAsync(wsb, 0, head + flag_bytes, stream) != cudaSuccess) {
+        cudaFreeAsync(ws, stream);
+        return SELSCAN_ERR_CUDA;
+    }
+    prm.ticket = reinterpret_cast<unsigned int *>(wsb);
+    prm.flags = reinterpret_cast<unsigned int *>(wsb + head);
+    prm.carry = reinterpret_cast<float *>(wsb + head + flag_bytes);
+    prm.dbg_skip_publish = g_dbg_skip_publish;
+
+    auto kern = scan_diag_kernel<T, CH, STAGES, GATE>;
+    static bool attr_set[kMaxDevices] = {};  // per instantiation and device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Lay::kAlloc) != cudaSuccess) {
+            cudaFreeAsync(ws, stream);
+            return SELSCAN_ERR_CUDA;
+        }
+        attr_set[dev] = true;
+    }
+    const int grid = int(std::min<int64_t>(ctas_max, units));
+    kern<<<grid, CH * 2 + 32, Lay::kAlloc, stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, prm);
+    const cudaError_t le = cudaGetLastError();
+    cudaFreeAsync(ws, stream);
+    return le == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *selscan_strerror(selscan_status s)
+{
+    switch (s) {
+    case SELSCAN_OK: return "ok";
+    case SELSCAN_ERR_NULL: return "required pointer is NULL";
+    case SELSCAN_ERR_SHAPE: return "tensor ranks or sizes disagree";
+    case SELSCAN_ERR_STRIDE: return "unsupported strides (time stride must be 1)";
+    case SELSCAN_ERR_DTYPE: return "unsupported element type";
+    case SELSCAN_ERR_ALIGN: return "pointer or row stride not 16-byte aligned";
+    case SELSCAN_ERR_UNSUPPORTED: return "valid arguments, but this size is not built";
+    case SELSCAN_ERR_CUDA: return "CUDA runtime error";
+    case SELSCAN_ERR_TIMEOUT: return "a device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+int selscan_version(void) { return SELSCAN_VERSION; }
+
+// Test hook (not part of the public header's stable surface): withhold the
+// carry flag of one work unit so that its successor's bounded wait expires.
+// -1 switches it off.
+void selscan_debug_withhold_carry(int unit) { g_dbg_skip_publish = unit; }
+
+selscan_status selscan_check(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return SELSCAN_ERR_CUDA;
+    unsigned int err = 0;
+    if (cudaMemcpyFromSymbol(&err, g_selscan_err, sizeof(err)) != cudaSuccess)
+        return SELSCAN_ERR_CUDA;
+    if (err) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_selscan_err, &zero, sizeof(zero));
+        return SELSCAN_ERR_TIMEOUT;
+    }
+    return SELSCAN_OK;
+}
+
+selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
+                           const selscan_tensor *delta_bias, int delta_softplus,
+                           const selscan_tensor *A, const selscan_tensor *B,
+                           const selscan_tensor *C, const selscan_tensor *D,
+                           const selscan_tensor *z, selscan_tensor *y,
+                           selscan_tensor *last_state, cudaStream_t stream)
+{
+    // ---- validation (no CUDA call before it passes)
+    if (!present(u) || !delta || !A || !B || !C || !y)
+        return SELSCAN_ERR_NULL;
+    if (u->ndim != 3)
+        return SELSCAN_ERR_SHAPE;
+    const int32_t dt = u->dtype;
+    if (dt != SELSCAN_F32 && dt != SELSCAN_BF16)
+        return SELSCAN_ERR_DTYPE;
+    const int64_t batch = u->shape[0], dim = u->shape[1], L = u->shape[2];
+    if (batch < 0 || dim < 0 || L < 0)
+        return SELSCAN_ERR_SHAPE;
+    if (!present(A))
+        return SELSCAN_ERR_NULL;
+    if (A->ndim != 2 || A->shape[0] != dim)
+        return SELSCAN_ERR_SHAPE;
+    const int64_t N = A->shape[1];
+    selscan_status st;
+    if ((st = check_seq(u, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    if ((st = check_seq(delta, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    if ((st = check_seq(y, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    if (z && z->data && (st = check_seq(z, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    {
+        const int64_t ashape[2] = {dim, N};
+        if ((st = check_param(A, 2, ashape, false)) != SELSCAN_OK) return st;
+        const int64_t vshape[1] = {dim};
+        if ((st = check_param(delta_bias, 1, vshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(D, 1, vshape, true)) != SELSCAN_OK) return st;
+        const int64_t sshape[3] = {batch, dim, N};
+        if ((st = check_param(last_state, 3, sshape, true)) != SELSCAN_OK) return st;
+    }
+    for (const selscan_tensor *t : {B, C}) {
+        if (!present(t))
+            return SELSCAN_ERR_NULL;
+        if (t->ndim == 4) {
+            if (t->shape[1] != 1)
+                return SELSCAN_ERR_UNSUPPORTED;  // one group of B/C
+            selscan_tensor v = *t;
+            v.ndim = 3;
+            v.shape[1] = t->shape[2];
+            v.shape[2] = t->shape[3];
+            v.stride[1] = t->stride[2];
+            v.stride[2] = t->stride[3];
+            if ((st = check_seq(&v, batch, N, L, dt)) != SELSCAN_OK) return st;
+        } else {
+            if ((st = check_seq(t, batch, N, L, dt)) != SELSCAN_OK) return st;
+        }
+    }
+    if (N != kDiagN)
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch > 65535 || dim > (int64_t(1) << 30) || L > (int64_t(1) << 31) - 1024)
+        return SELSCAN_ERR_UNSUPPORTED;
+
+    // ---- empty problems: nothing to launch
+    if (batch == 0 || dim == 0)
+        return SELSCAN_OK;
+    if (L == 0) {
+        if (last_state && last_state->data)
+            return cudaMemsetAsync(last_state->data, 0, size_t(batch * dim * N) * 4, stream) ==
+                           cudaSuccess
+                       ? SELSCAN_OK
+                       : SELSCAN_ERR_CUDA;
+        return SELSCAN_OK;
+    }
+
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    if ((st = device_setup(&dev, &di)) != SELSCAN_OK)
+        return st;
+
+    DiagParams prm{};
+    prm.batch = int(batch);
+    prm.dim = int(dim);
+    prm.L = int(L);
+    prm.A = static_cast<const float *>(A->data);
+    prm.delta_bias = static_cast<const float *>(opt_data(delta_bias));
+    prm.Dskip = static_cast<const float *>(opt_data(D));
+    prm.h0 = nullptr;
+    prm.last_state = static_cast<float *>(last_state ? last_state->data : nullptr);
+    prm.softplus = delta_softplus ? 1 : 0;
+    prm.timeout_ns = default_timeout_ns();
+    prm.err = di->err;
+
+    const bool gate = z && z->data;
+    if (dt == SELSCAN_BF16) {
+        return gate ? launch_diag<__nv_bfloat16, 64, 4, true>(u, delta, B, C, z, y, prm,
+                                                              di->sm_count, stream)
+                    : launch_diag<__nv_bfloat16, 64, 4, false>(u, delta, B, C, z, y, prm,
+                                                               di->sm_count, stream);
+    }
+    return gate ? launch_diag<float, 64, 4, true>(u, delta, B, C, z, y, prm, di->sm_count,
+                                                  stream)
+                : launch_diag<float, 64, 4, false>(u, delta, B, C, z, y, prm, di->sm_count,
+                                                   stream);
+}
+
+selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor *dt,
+                                   const selscan_tensor *dt_bias, int dt_softplus,
+                                   const selscan_tensor *A, const selscan_tensor *B,
+                                   const selscan_tensor *C, const selscan_tensor *D,
+                                   const selscan_tensor *z, int64_t headdim, selscan_tensor *y,
+                                   selscan_tensor *last_state, cudaStream_t stream)
+{
+    if (!present(x) || !dt || !A || !B || !C || !y)
+        return SELSCAN_ERR_NULL;
+    if (x->ndim != 3 || !present(A) || A->ndim != 1 || headdim <= 0)
+        return SELSCAN_ERR_SHAPE;
+    if (x->dtype != SELSCAN_BF16)
+        return SELSCAN_ERR_DTYPE;
+    const int64_t batch = x->shape[0], dim = x->shape[1], L = x->shape[2];
+    const int64_t H = A->shape[0];
+    if (batch < 0 || L < 0 || H <= 0 || dim != H * headdim)
+        return SELSCAN_ERR_SHAPE;
+    selscan_status st;
+    if ((st = check_seq(x, batch, dim, L, SELSCAN_BF16)) != SELSCAN_OK) return st;
+    if ((st = check_seq(y, batch, dim, L, SELSCAN_BF16)) != SELSCAN_OK) return st;
+    if (z && z->data && (st = check_seq(z, batch, dim, L, SELSCAN_BF16)) != SELSCAN_OK)
+        return st;
+    if ((st = check_seq(dt, batch, H, L, SELSCAN_F32)) != SELSCAN_OK) return st;
+    for (const selscan_tensor *t : {B, C}) {
+        if (!present(t))
+            return SELSCAN_ERR_NULL;
+        if (t->ndim != 4 || t->shape[0] != batch || t->shape[3] != L)
+            return SELSCAN_ERR_SHAPE;
+        if (t->dtype != SELSCAN_BF16)
+            return SELSCAN_ERR_DTYPE;
+    }
+    const int64_t G = B->shape[1], N = B->shape[2];
+    if (C->shape[1] != G || C->shape[2] != N || G <= 0 || H % G != 0)
+        return SELSCAN_ERR_SHAPE;
+    for (const selscan_tensor *t : {B, C}) {
+        selscan_tensor v = *t;  // view (batch, G*N, L) needs G*N rows evenly strided
+        if (t->stride[1] != t->shape[2] * t->stride[2] && G > 1)
+            return SELSCAN_ERR_STRIDE;
+        v.ndim = 3;
+        v.shape[1] = G * N;
+        v.shape[2] = L;
+        v.stride[1] = t->stride[2];
+        v.stride[2] = t->stride[3];
+        if ((st = check_seq(&v, batch, G * N, L, SELSCAN_BF16)) != SELSCAN_OK) return st;
+    }
+    {
+        const int64_t hshape[1] = {H};
+        if ((st = check_param(A, 1, hshape, false)) != SELSCAN_OK) return st;
+        if ((st = check_param(dt_bias, 1, hshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(D, 1, hshape, true)) != SELSCAN_OK) return st;
+        const int64_t sshape[4] = {batch, H, headdim, N};
+        if ((st = check_param(last_state, 4, sshape, true)) != SELSCAN_OK) return st;
+    }
+    if (N != kSsdN || headdim != kSsdP || G != 1)
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch > 65535 || L > (int64_t(1) << 31) - 1024)
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch == 0)
+        return SELSCAN_OK;
+    if (L == 0) {
+        if (last_state && last_state->data)
+            return cudaMemsetAsync(last_state->data, 0,
+                                   size_t(batch * H * headdim * N) * 4, stream) == cudaSuccess
+                       ? SELSCAN_OK
+                       : SELSCAN_ERR_CUDA;
+        return SELSCAN_OK;
+    }
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    if ((st = device_setup(&dev, &di)) != SELSCAN_OK)
+        return st;
+    (void)dt_softplus;
+    (void)stream;
+    return SELSCAN_ERR_UNSUPPORTED;  // kernel added separately
+}
+
+}  // extern "C"

@@ -1,0 +1,134 @@
+"""CPU tests of the C ABI boundary: the library loads, exports every entry
+point the headers declare, and rejects malformed arguments synchronously
+(before any CUDA call) with the documented status codes.
+
+Every call here uses placeholder pointers and is INVALID in at least one
+way, so validation stops it before anything reaches a device.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import selective_state_space_selscan_b200 as ss
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names.update(re.findall(r"SELSCAN_API\s+[\w\s\*]+?\b(selscan_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_symbols()
+    assert {"selscan_fwd", "selscan_fwd_scalarA", "selscan_check",
+            "selscan_strerror", "selscan_version"} <= names
+    lib = ctypes.CDLL(ss.LIB_PATH)
+    for n in sorted(names):
+        assert hasattr(lib, n), f"{n} declared but not exported"
+
+
+def test_version_and_strerror():
+    assert ss.version() == 10000
+    for code in range(9):
+        assert ss._strerror(code)
+    assert "unknown" in ss._strerror(99)
+
+
+FAKE = 0x7f0000000000  # 16-byte aligned placeholder, never dereferenced
+
+
+def _t(shape, dtype=ss.SELSCAN_BF16, strides=None, data=FAKE):
+    d = ss.SelscanTensor()
+    d.data = data
+    d.dtype = dtype
+    d.ndim = len(shape)
+    if strides is None:
+        strides, acc = [], 1
+        for s in reversed(shape):
+            strides.insert(0, acc)
+            acc *= s
+    for i, (s, st) in enumerate(zip(shape, strides)):
+        d.shape[i] = s
+        d.stride[i] = st
+    return d
+
+
+def _fwd(**over):
+    b, D, N, L = 2, 64, 16, 128
+    args = dict(u=_t((b, D, L)), delta=_t((b, D, L)), bias=_t((D,), ss.SELSCAN_F32),
+                A=_t((D, N), ss.SELSCAN_F32), B=_t((b, N, L)), C=_t((b, N, L)),
+                Dv=_t((D,), ss.SELSCAN_F32), z=_t((b, D, L)), y=_t((b, D, L)),
+                hs=_t((b, D, N), ss.SELSCAN_F32))
+    args.update(over)
+    r = lambda x: None if x is None else ctypes.byref(x)
+    return ss.lib().selscan_fwd(r(args["u"]), r(args["delta"]), r(args["bias"]), 1,
+                                r(args["A"]), r(args["B"]), r(args["C"]), r(args["Dv"]),
+                                r(args["z"]), r(args["y"]), r(args["hs"]), None)
+
+
+C = ss.STATUS_CODE
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(u=None), "SELSCAN_ERR_NULL"),
+    (dict(y=None), "SELSCAN_ERR_NULL"),
+    (dict(B=_t((2, 16, 128), data=0)), "SELSCAN_ERR_NULL"),
+    (dict(delta=_t((2, 64, 127))), "SELSCAN_ERR_SHAPE"),
+    (dict(A=_t((63, 16), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(hs=_t((2, 64, 8), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(z=_t((2, 64, 128), ss.SELSCAN_F32)), "SELSCAN_ERR_DTYPE"),
+    (dict(bias=_t((64,), ss.SELSCAN_BF16)), "SELSCAN_ERR_DTYPE"),
+    (dict(u=_t((2, 64, 128), dtype=7)), "SELSCAN_ERR_DTYPE"),
+    (dict(u=_t((2, 64, 128), strides=(8192, 128, 2))), "SELSCAN_ERR_STRIDE"),
+    (dict(A=_t((64, 16), ss.SELSCAN_F32, strides=(1, 64))), "SELSCAN_ERR_STRIDE"),
+    (dict(u=_t((2, 64, 128), data=FAKE + 8)), "SELSCAN_ERR_ALIGN"),
+    (dict(y=_t((2, 64, 128), strides=(8192, 124, 1))), "SELSCAN_ERR_ALIGN"),
+    (dict(B=_t((2, 2, 16, 128))), "SELSCAN_ERR_UNSUPPORTED"),
+])
+def test_fwd_rejects(over, expect):
+    assert _fwd(**over) == C[expect]
+
+
+def test_fwd_rejects_state_size_other_than_16():
+    b, D, N, L = 1, 32, 8, 64
+    rc = _fwd(A=_t((D, N), ss.SELSCAN_F32), u=_t((b, D, L)), delta=_t((b, D, L)),
+              B=_t((b, N, L)), C=_t((b, N, L)), y=_t((b, D, L)), z=None,
+              bias=_t((D,), ss.SELSCAN_F32), Dv=_t((D,), ss.SELSCAN_F32),
+              hs=_t((b, D, N), ss.SELSCAN_F32), )
+    assert rc == C["SELSCAN_ERR_UNSUPPORTED"]
+
+
+def _scal(**over):
+    b, H, P, N, L, G = 2, 4, 64, 128, 256, 1
+    args = dict(x=_t((b, H * P, L)), dt=_t((b, H, L), ss.SELSCAN_F32), bias=None,
+                A=_t((H,), ss.SELSCAN_F32), B=_t((b, G, N, L)), C=_t((b, G, N, L)),
+                Dv=_t((H,), ss.SELSCAN_F32), z=None, P=P, y=_t((b, H * P, L)),
+                hs=_t((b, H, P, N), ss.SELSCAN_F32))
+    args.update(over)
+    r = lambda x: None if x is None else ctypes.byref(x)
+    return ss.lib().selscan_fwd_scalarA(r(args["x"]), r(args["dt"]), r(args["bias"]), 0,
+                                        r(args["A"]), r(args["B"]), r(args["C"]),
+                                        r(args["Dv"]), r(args["z"]), args["P"], r(args["y"]),
+                                        r(args["hs"]), None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(x=None), "SELSCAN_ERR_NULL"),
+    (dict(P=32), "SELSCAN_ERR_SHAPE"),
+    (dict(x=_t((2, 256, 256), ss.SELSCAN_F32)), "SELSCAN_ERR_DTYPE"),
+    (dict(dt=_t((2, 4, 256))), "SELSCAN_ERR_DTYPE"),
+    (dict(B=_t((2, 1, 128, 255))), "SELSCAN_ERR_SHAPE"),
+    (dict(hs=_t((2, 4, 64, 64), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(x=_t((2, 256, 256), data=FAKE + 4)), "SELSCAN_ERR_ALIGN"),
+    (dict(B=_t((2, 2, 64, 256)), C=_t((2, 2, 64, 256)),
+          hs=_t((2, 4, 64, 64), ss.SELSCAN_F32)), "SELSCAN_ERR_UNSUPPORTED"),
+])
+def test_scalarA_rejects(over, expect):
+    assert _scal(**over) == C[expect]
