@@ -415,6 +415,10 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the config's batch (smaller profiling cases)")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="override the config's L (smaller profiling cases)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -422,6 +426,10 @@ def main():
                     help="DRAM bytes per launch from an ncu capture of this kernel")
     args = ap.parse_args()
 
+    if args.batch is not None:
+        synthetic.CONFIGS[args.config] = dict(synthetic.CONFIGS[args.config], batch=args.batch)
+    if args.seqlen is not None:
+        synthetic.CONFIGS[args.config] = dict(synthetic.CONFIGS[args.config], L=args.seqlen)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -105,7 +105,19 @@ def selscan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     N = A.shape[1]
     B4, C4 = _bc4(B, batch), _bc4(C, batch)
     G = B4.shape[1]
-    d0, d1 = (0, dim) if channels is None else channels
+    if channels is not None and tuple(channels) != (0, dim):
+        # marshal only the requested channels (and their B/C group)
+        d0, d1 = channels
+        per = dim // G
+        g0, g1 = d0 // per, (d1 - 1) // per
+        if G > 1 and g0 != g1:
+            raise ValueError("a channel sample must lie within one B/C group")
+        sl = (lambda a: None if a is None else np.asarray(a)[:, d0:d1])
+        vec = (lambda a: None if a is None else np.asarray(a)[d0:d1])
+        return selscan(sl(u), sl(delta), np.asarray(A)[d0:d1], B4[:, g0:g0 + 1],
+                       C4[:, g0:g0 + 1], D=vec(D), z=sl(z), delta_bias=vec(delta_bias),
+                       delta_softplus=delta_softplus, h0=sl(h0), channels=None)
+    d0, d1 = 0, dim
     keep = []
     uu, up = _f64(u); keep.append(uu)
     dd, dp_ = _f64(delta); keep.append(dd)
@@ -122,7 +134,7 @@ def selscan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
         batch, dim, N, L, G, up, dp_, bp, int(bool(delta_softplus)), ap, Bp,
         Cp, Dp, zp, hp, y.ctypes.data_as(_dp), hs.ctypes.data_as(_dp), d0, d1)
     _check(rc)
-    return y[:, d0:d1], hs[:, d0:d1]
+    return y, hs
 
 
 def selscan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
@@ -180,17 +192,33 @@ def selscan_scalarA(x, dt, A, B, C, headdim, D=None, z=None, dt_bias=None,
     h0: (batch, H, P, N).  ``heads`` = (begin, end) restricts the heads
     computed (returned arrays hold only those heads' channels/states).
     Returns (y, last_state) in float64."""
+    nh = np.asarray(A).shape[0]
+    if heads is not None and tuple(heads) != (0, nh):
+        # marshal only the requested heads (and their B/C group)
+        a0, a1 = heads
+        Bq = _bc4(B, np.asarray(x).shape[0])
+        Cq = _bc4(C, np.asarray(x).shape[0])
+        per = nh // Bq.shape[1]
+        g0, g1 = a0 // per, (a1 - 1) // per
+        if Bq.shape[1] > 1 and g0 != g1:
+            raise ValueError("a head sample must lie within one B/C group")
+        ch = (lambda a: None if a is None else np.asarray(a)[:, a0 * headdim:a1 * headdim])
+        hv = (lambda a: None if a is None else np.asarray(a)[a0:a1])
+        return selscan_scalarA(ch(x), np.asarray(dt)[:, a0:a1], hv(A), Bq[:, g0:g0 + 1],
+                               Cq[:, g0:g0 + 1], headdim, D=hv(D), z=ch(z),
+                               dt_bias=hv(dt_bias), dt_softplus=dt_softplus,
+                               h0=None if h0 is None else np.asarray(h0)[:, a0:a1])
     dims, ptrs, rest, keep = _scalar_args(x, dt, A, B, C, D, z, dt_bias, h0,
                                           headdim)
     batch, nheads, P, N, L, G = dims
-    h0_, h1_ = (0, nheads) if heads is None else heads
+    h0_, h1_ = 0, nheads
     y = np.zeros((batch, nheads * P, L), dtype=np.float64)
     hs = np.zeros((batch, nheads, P, N), dtype=np.float64)
     rc = _load().oracle_selscan_scalarA(
         *dims, ptrs[0], ptrs[1], ptrs[2], int(bool(dt_softplus)), *rest,
         y.ctypes.data_as(_dp), hs.ctypes.data_as(_dp), h0_, h1_)
     _check(rc)
-    return y[:, h0_ * P:h1_ * P], hs[:, h0_:h1_]
+    return y, hs
 
 
 def ssd_chunked(x, dt, A, B, C, headdim, chunk, D=None, z=None, dt_bias=None,

@@ -1,0 +1,630 @@
+// scan_diag_bf16.cuh -- fast diagonal-A selective scan for bf16 inputs
+// (fp32 state), sm_100a.
+//
+// Same contract and work decomposition as scan_diag.cuh (persistent grid,
+// atomic ticket in segment-major order, one producer warp streaming chunks
+// with bulk tensor copies, carries linked by gpu-scope release/acquire
+// flags), with an inner loop laid out for the B200 SM:
+//
+//  * One consumer lane per channel for everything that is per token
+//    (softplus, delta*u, the decay base, gate, D skip, output): its row of
+//    the input tile is read with 16-byte shared loads, 8 tokens at a time.
+//  * The 16 states of a PAIR of channels are split between the two lanes of
+//    a lane pair by parity: lane p keeps states n = p, p+2, ..., p+14 of both
+//    channels.  B and C of one token therefore serve two channels per load,
+//    which halves the shared-memory traffic per element; they are staged
+//    once per chunk as packed bf16 pairs and widened in registers.
+//  * The state is kept rescaled, g = h / w with w = delta * u, so that the
+//    input term needs no multiply:  g_t = (w_{t-1}/w_t) exp(delta_t A) g_{t-1}
+//    + B_t and y_t = w_t (C_t . g_t).  |w| is kept >= 2^-64 so that the
+//    rescaling stays finite (a zero input then contributes 2^-64 * B, far
+//    below fp32 resolution of any non-trivial state).
+//  * For S4D-real A (A[d,n] = (n+1) A[d,0], checked per channel at run time)
+//    the decays are powers r^(n+1) of r = exp(delta A[d,0]); lane p needs
+//    the odd (p=0) or even (p=1) powers, i.e. base * s^j with s = r^2,
+//    computed with packed f32x2 multiplies.  Other A use one ex2 per state.
+//  * Packed f32x2 FMAs (sm_100) update two states per instruction.
+//  * The token-wise prologue of the next 8-token block is computed before
+//    the state updates of the current one so its special-function latency
+//    overlaps the FMA work.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+#include <type_traits>
+
+#include "ptx.cuh"
+#include "scan_diag.cuh"
+
+namespace selscan {
+
+__device__ __forceinline__ uint64_t pk2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ float lo2(uint64_t v)
+{
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo;
+}
+
+__device__ __forceinline__ float hi2(uint64_t v)
+{
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return hi;
+}
+
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// bf16 pair (lo, hi halves of a 32-bit word) -> packed fp32 pair
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w)
+{
+    return pk2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__device__ __forceinline__ void unpack8_bf16(uint4 v, float (&f)[8])
+{
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xffff0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xffff0000u);
+    f[4] = __uint_as_float(v.z << 16);
+    f[5] = __uint_as_float(v.z & 0xffff0000u);
+    f[6] = __uint_as_float(v.w << 16);
+    f[7] = __uint_as_float(v.w & 0xffff0000u);
+}
+
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+constexpr float kWMin = 5.421010862427522e-20f;  // 2^-64
+
+template <int CH, int STAGES, bool GATE>
+struct DiagFastLayout {
+    static constexpr int kChunk = 64;                    // tokens per stage
+    static constexpr int kTile = CH * 128;               // bf16 [CH][64]
+    static constexpr int kBCTile = kDiagN * 128;         // bf16 [16][64]
+    static constexpr int kStage = (2 + (GATE ? 1 : 0)) * kTile + 2 * kBCTile;
+    static constexpr int kStagesOff = 0;
+    static constexpr int kBCPOff = STAGES * kStage;      // fp32 B/C [2][64][128 B]
+    static constexpr int kYOff = kBCPOff + 2 * kChunk * 128;
+    static constexpr int kBarOff = kYOff + 2 * kTile;
+    static constexpr int kInfoOff = kBarOff + 2 * STAGES * 8;
+    static constexpr int kAbortOff = kInfoOff + STAGES * 16;
+    static constexpr int kBytes = kAbortOff + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+// Per-token values of one 8-token block for this lane's own channel.
+struct Prologue {
+    float r[8];   // decay base (POW) or delta (general)
+    float c[8];   // w_{t-1} / w_t
+    float w[8];   // rescale factor w_t = delta_t u_t (clamped)
+    float u[8];
+    float z[8];
+};
+
+template <bool POW, bool SOFTPLUS, bool GATE, bool TAIL>
+__device__ __forceinline__ void fast_prologue(Prologue &P, const uint8_t *u_row,
+                                              const uint8_t *dl_row, const uint8_t *z_row,
+                                              int off, int t_base, int L, float bias,
+                                              float a0, float &wprev)
+{
+    float dv[8];
+    unpack8_bf16(*reinterpret_cast<const uint4 *>(u_row + off), P.u);
+    unpack8_bf16(*reinterpret_cast<const uint4 *>(dl_row + off), dv);
+    if (GATE)
+        unpack8_bf16(*reinterpret_cast<const uint4 *>(z_row + off), P.z);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float x = dv[i] + bias;
+        float dt = SOFTPLUS ? softplus_fast(x) : x;
+        if (TAIL)
+            dt = (t_base + i < L) ? dt : 0.f;  // padding: identity step
+        const float wr = dt * P.u[i];
+        const float w = copysignf(fmaxf(fabsf(wr), kWMin), wr);
+        P.r[i] = POW ? ex2_approx(dt * a0) : dt;
+        P.c[i] = wprev * rcp_approx(w);
+        P.w[i] = w;
+        wprev = w;
+    }
+}
+
+template <bool POW>
+__device__ __forceinline__ void decay_pairs(uint64_t (&V)[4], float r, float c, int p,
+                                            const uint64_t (&apair)[4])
+{
+    if (POW) {
+        // powers r^(n+1) for n = p, p+2, ..., p+14 : base * s^j, s = r^2
+        const float s = r * r;
+        const float base = c * (p ? s : r);
+        V[0] = pk2(base, base * s);
+        const float s2 = s * s;
+        const uint64_t S2 = pk2(s2, s2);
+        V[1] = mul2(V[0], S2);
+        V[2] = mul2(V[1], S2);
+        V[3] = mul2(V[2], S2);
+    } else {
+        // general A: r holds delta; apair holds A*log2(e) of this lane's states
+        const uint64_t RR = pk2(r, r), CC = pk2(c, c);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const uint64_t X = mul2(RR, apair[jj]);
+            V[jj] = mul2(CC, pk2(ex2_approx(lo2(X)), ex2_approx(hi2(X))));
+        }
+    }
+}
+
+// 8 tokens of the scan for this lane's state parity of both channels.
+template <bool POW>
+__device__ __forceinline__ void scan_block8(uint64_t (&gown)[4], uint64_t (&goth)[4],
+                                            const float *bcb_blk, int pp, const Prologue &P,
+                                            const float (&ro)[8], const float (&co)[8],
+                                            const uint64_t (&aown)[4],
+                                            const uint64_t (&aoth)[4], float (&yown)[8],
+                                            float (&yoth)[8])
+{
+    uint64_t Vo[4], Vx[4];
+    decay_pairs<POW>(Vo, P.r[0], P.c[0], pp, aown);
+    decay_pairs<POW>(Vx, ro[0], co[0], pp, aoth);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const ulonglong2 *bq = reinterpret_cast<const ulonglong2 *>(bcb_blk + i * 32 + pp * 16);
+        const ulonglong2 b01 = bq[0], b23 = bq[1], c01 = bq[2], c23 = bq[3];
+        uint64_t Von[4], Vxn[4];
+        if (i + 1 < 8) {
+            decay_pairs<POW>(Von, P.r[i + 1], P.c[i + 1], pp, aown);
+            decay_pairs<POW>(Vxn, ro[i + 1], co[i + 1], pp, aoth);
+        }
+        gown[0] = fma2(Vo[0], gown[0], b01.x);
+        goth[0] = fma2(Vx[0], goth[0], b01.x);
+        gown[1] = fma2(Vo[1], gown[1], b01.y);
+        goth[1] = fma2(Vx[1], goth[1], b01.y);
+        gown[2] = fma2(Vo[2], gown[2], b23.x);
+        goth[2] = fma2(Vx[2], goth[2], b23.x);
+        gown[3] = fma2(Vo[3], gown[3], b23.y);
+        goth[3] = fma2(Vx[3], goth[3], b23.y);
+        uint64_t Yao = mul2(c01.x, gown[0]);
+        uint64_t Yax = mul2(c01.x, goth[0]);
+        uint64_t Ybo = mul2(c01.y, gown[1]);
+        uint64_t Ybx = mul2(c01.y, goth[1]);
+        Yao = fma2(c23.x, gown[2], Yao);
+        Yax = fma2(c23.x, goth[2], Yax);
+        Ybo = fma2(c23.y, gown[3], Ybo);
+        Ybx = fma2(c23.y, goth[3], Ybx);
+        const uint64_t Yo = add2(Yao, Ybo), Yx = add2(Yax, Ybx);
+        yown[i] = lo2(Yo) + hi2(Yo);
+        yoth[i] = lo2(Yx) + hi2(Yx);
+        if (i + 1 < 8) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                Vo[jj] = Von[jj];
+                Vx[jj] = Vxn[jj];
+            }
+        }
+    }
+}
+
+template <int CH, int STAGES, bool GATE, bool SOFTPLUS>
+__global__ void __launch_bounds__(CH + 32, 1)
+scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
+                      const __grid_constant__ CUtensorMap tm_delta,
+                      const __grid_constant__ CUtensorMap tm_z,
+                      const __grid_constant__ CUtensorMap tm_B,
+                      const __grid_constant__ CUtensorMap tm_C,
+                      const __grid_constant__ CUtensorMap tm_y,
+                      const DiagParams p)
+{
+    using Lay = DiagFastLayout<CH, STAGES, GATE>;
+    constexpr int TC = Lay::kChunk;
+    constexpr int CONS = CH;      // one consumer lane per channel
+    constexpr int CW = CONS / 32;
+    constexpr int TILE = Lay::kTile;
+    static_assert(CONS % 32 == 0, "consumer threads must fill warps");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *stages = smem + Lay::kStagesOff;
+    float *bcp = reinterpret_cast<float *>(smem + Lay::kBCPOff);
+    uint8_t *ytile = smem + Lay::kYOff;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Lay::kBarOff);
+    uint64_t *empty = full + STAGES;
+    int4 *info = reinterpret_cast<int4 *>(smem + Lay::kInfoOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kAbortOff);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], CW);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int G = p.num_tiles;
+
+    if (warp == CW) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_u);
+            prefetch_tmap(&tm_delta);
+            if (GATE)
+                prefetch_tmap(&tm_z);
+            prefetch_tmap(&tm_B);
+            prefetch_tmap(&tm_C);
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            while (ok) {
+                const unsigned int tk = atomicAdd(p.ticket, 1u);
+                if (tk >= unsigned(p.total_units))
+                    break;
+                const int k = int(tk) / G, g = int(tk) - k * G;
+                const int b = g / p.tiles_per_batch;
+                const int d0 = (g - b * p.tiles_per_batch) * CH;
+                const int tb = k * p.seg_len;
+                const int te = min(p.L, tb + p.seg_len);
+                const int nch = (te - tb + TC - 1) / TC;
+                for (int c = 0; c < nch; ++c) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const int t0 = tb + c * TC;
+                    info[s] = make_int4(int(tk), t0,
+                                        (c == 0 ? kInfoFirst : 0) |
+                                            (c == nch - 1 ? kInfoLast : 0),
+                                        0);
+                    uint8_t *st = stages + s * Lay::kStage;
+                    mbar_arrive_expect_tx(&full[s], Lay::kStage);
+                    tma_load_3d(st, &tm_u, &full[s], t0, d0, b);
+                    tma_load_3d(st + TILE, &tm_delta, &full[s], t0, d0, b);
+                    if (GATE)
+                        tma_load_3d(st + 2 * TILE, &tm_z, &full[s], t0, d0, b);
+                    uint8_t *bct = st + (GATE ? 3 : 2) * TILE;
+                    tma_load_3d(bct, &tm_B, &full[s], t0, 0, b);
+                    tma_load_3d(bct + Lay::kBCTile, &tm_C, &full[s], t0, 0, b);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (ok && mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns)) {
+                info[s] = make_int4(-1, 0, kInfoEnd, 0);
+                mbar_arrive(&full[s]);
+            } else {
+                atomicOr(p.err, kErrTimeoutPipe);
+                *abort_flag = 1;
+                __nanosleep(100000);  // let copies already issued land
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int ch = tid;          // this lane's own channel within the tile
+    const int pp = tid & 1;      // state parity handled by this lane
+    const int swz = ch & 7;      // 128-byte swizzle phase of this row
+    uint64_t gown[4], goth[4];   // rescaled states, parity pp, own / partner channel
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        gown[jj] = pk2(0.f, 0.f);
+        goth[jj] = pk2(0.f, 0.f);
+    }
+    uint64_t aown[4], aoth[4];   // A*log2e of this lane's states, paired (general path)
+    float a0 = 0.f, bias = 0.f, dsk = 0.f, wprev = 1.f;
+    bool pow_path = true;
+    int unit = -1, k = 0, b = 0, d0 = 0, d = 0;
+    int prev_t0 = 0, prev_d0 = 0, prev_b = 0;
+    int s = 0, it = 0;
+    uint32_t ph = 0;
+
+    for (;;) {
+        const bool arrived = mbar_wait(&full[s], ph, p.timeout_ns) && !*abort_flag;
+        int4 inf = make_int4(-1, 0, 0, 0);
+        if (arrived) {
+            inf = info[s];  // ordered after the barrier wait (acquire)
+            if (inf.z & kInfoEnd)
+                break;  // every consumer reads the same marker
+        }
+
+        if (arrived && (inf.z & kInfoFirst)) {
+            unit = inf.x;
+            k = unit / G;
+            const int g = unit - k * G;
+            b = g / p.tiles_per_batch;
+            d0 = (g - b * p.tiles_per_batch) * CH;
+            d = d0 + ch;
+            const int dpart = d0 + (ch ^ 1);
+            const bool live = d < p.dim, live_o = dpart < p.dim;
+            const float *arow = p.A + size_t(live ? d : 0) * kDiagN;
+            const float *orow = p.A + size_t(live_o ? dpart : 0) * kDiagN;
+            const float A0 = arow[0], O0 = orow[0];
+            bool ok = true;
+            float al[8], ol[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int n = 2 * j + pp;  // this lane's states
+                const float an = arow[n], on = orow[n];
+                ok = ok && (an == float(n + 1) * A0) && (on == float(n + 1) * O0);
+                al[j] = an * kLog2e;
+                ol[j] = on * kLog2e;
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                aown[jj] = pk2(al[2 * jj], al[2 * jj + 1]);
+                aoth[jj] = pk2(ol[2 * jj], ol[2 * jj + 1]);
+            }
+            // every lane also needs its own channel's full row structure
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int n = 2 * j + (pp ^ 1);
+                ok = ok && (arow[n] == float(n + 1) * A0);
+            }
+            a0 = A0 * kLog2e;
+            pow_path = __all_sync(0xffffffffu, ok);
+            bias = (p.delta_bias && live) ? p.delta_bias[d] : 0.f;
+            dsk = (p.Dskip && live) ? p.Dskip[d] : 0.f;
+            wprev = 1.f;  // g starts as h_in (w_{-1} := 1)
+            float hown[8], hoth[8];
+            if (k == 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int n = 2 * j + pp;
+                    hown[j] = (p.h0 && live) ? p.h0[(size_t(b) * p.dim + d) * kDiagN + n] : 0.f;
+                    hoth[j] = (p.h0 && live_o)
+                                  ? p.h0[(size_t(b) * p.dim + dpart) * kDiagN + n] : 0.f;
+                }
+            } else {
+                const int prev = unit - G;
+                const uint32_t *flag = p.flags + size_t(prev) * CW + warp;
+                bool got = true;
+                if (lane == 0)
+                    got = spin_flag(flag, 1u, p.timeout_ns);
+                got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                if (!got) {
+                    if (lane == 0)
+                        atomicOr(p.err, kErrTimeoutCarry);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        hown[j] = hoth[j] = 0.f;
+                } else {
+                    (void)ld_acquire_gpu(flag);
+                    // carry layout: [unit][channel][parity][8]
+                    const float4 *so = reinterpret_cast<const float4 *>(
+                        p.carry + (size_t(prev) * CH + ch) * kDiagN + pp * 8);
+                    const float4 *sx = reinterpret_cast<const float4 *>(
+                        p.carry + (size_t(prev) * CH + (ch ^ 1)) * kDiagN + pp * 8);
+                    const float4 o0 = __ldcg(so), o1 = __ldcg(so + 1);
+                    const float4 x0 = __ldcg(sx), x1 = __ldcg(sx + 1);
+                    hown[0] = o0.x; hown[1] = o0.y; hown[2] = o0.z; hown[3] = o0.w;
+                    hown[4] = o1.x; hown[5] = o1.y; hown[6] = o1.z; hown[7] = o1.w;
+                    hoth[0] = x0.x; hoth[1] = x0.y; hoth[2] = x0.z; hoth[3] = x0.w;
+                    hoth[4] = x1.x; hoth[5] = x1.y; hoth[6] = x1.z; hoth[7] = x1.w;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                gown[jj] = pk2(hown[2 * jj], hown[2 * jj + 1]);
+                goth[jj] = pk2(hoth[2 * jj], hoth[2 * jj + 1]);
+            }
+        }
+
+        uint8_t *st = stages + s * Lay::kStage;
+        const uint8_t *Bt = st + (GATE ? 3 : 2) * TILE;
+        const uint8_t *Ct = Bt + Lay::kBCTile;
+        float *bcb = bcp + (it & 1) * TC * 32;
+        // B, C -> fp32, token-major: [t][parity p][B: X[p], X[p+2], ..., X[p+14]][C: same]
+        for (int q = tid; arrived && q < TC * 32; q += CONS) {
+            const int t = q >> 5, rest = q & 31;
+            const int par = rest >> 4, isC = (rest >> 3) & 1, k8 = rest & 7;
+            const int n = 2 * k8 + par;
+            const uint8_t *src = isC ? Ct : Bt;
+            const int chunk = (t * 2) >> 4, within = (t * 2) & 15;
+            const uint16_t v = *reinterpret_cast<const uint16_t *>(
+                src + n * 128 + ((chunk ^ (n & 7)) << 4) + within);
+            bcb[q] = __uint_as_float(uint32_t(v) << 16);
+        }
+        if (tid == 0)
+            bulk_wait_read<0>();  // y tile (it & 1) free again
+        if (named_bar_any(1, CONS, !arrived)) {
+            if (tid == 0)
+                atomicOr(p.err, kErrTimeoutPipe);
+            *abort_flag = 1;
+            break;
+        }
+        if (tid == 0 && it > 0) {
+            tma_store_3d(&tm_y, ytile + ((it - 1) & 1) * TILE, prev_t0, prev_d0, prev_b);
+            bulk_commit();
+        }
+
+        const uint8_t *u_row = st + ch * 128;
+        const uint8_t *dl_row = st + TILE + ch * 128;
+        const uint8_t *z_row = st + 2 * TILE + ch * 128;
+        uint8_t *y_row = ytile + (it & 1) * TILE + ch * 128;
+        const int t0 = inf.y;
+
+        auto run = [&](auto pow_tag) {
+            constexpr bool POWC = decltype(pow_tag)::value;
+#pragma unroll 1
+            for (int j = 0; j < TC / 8; ++j) {
+                const int off = (j ^ swz) << 4;
+                const int tb = t0 + j * 8;
+                const uint4 uq = *reinterpret_cast<const uint4 *>(u_row + off);
+                const uint4 dq = *reinterpret_cast<const uint4 *>(dl_row + off);
+                uint4 zq = make_uint4(0, 0, 0, 0);
+                if (GATE)
+                    zq = *reinterpret_cast<const uint4 *>(z_row + off);
+                const int nvalid = p.L - tb;  // tokens of this block inside the sequence
+                uint32_t ypk[4];
+                const float *bcb_blk = bcb + j * 8 * 32;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    // token-wise prologue for this lane's own channel
+                    const uint32_t uw = (i < 2 ? uq.x : i < 4 ? uq.y : i < 6 ? uq.z : uq.w);
+                    const uint32_t dw = (i < 2 ? dq.x : i < 4 ? dq.y : i < 6 ? dq.z : dq.w);
+                    const float uv = __uint_as_float((i & 1) ? (uw & 0xffff0000u) : (uw << 16));
+                    const float dv = __uint_as_float((i & 1) ? (dw & 0xffff0000u) : (dw << 16));
+                    const float x = dv + bias;
+                    float dt = SOFTPLUS ? softplus_fast(x) : x;
+                    dt = (i < nvalid) ? dt : 0.f;  // padding past L: identity step
+                    const float wr = dt * uv;
+                    const float w = copysignf(fmaxf(fabsf(wr), kWMin), wr);
+                    const float r = POWC ? ex2_approx(dt * a0) : dt;
+                    const float c = wprev * rcp_approx(w);
+                    wprev = w;
+                    const float ro = __shfl_xor_sync(0xffffffffu, r, 1);
+                    const float co = __shfl_xor_sync(0xffffffffu, c, 1);
+                    // scan step for this lane's state parity of both channels
+                    const ulonglong2 *bq =
+                        reinterpret_cast<const ulonglong2 *>(bcb_blk + i * 32 + pp * 16);
+                    const ulonglong2 b01 = bq[0], b23 = bq[1], c01 = bq[2], c23 = bq[3];
+                    uint64_t Vo[4], Vx[4];
+                    decay_pairs<POWC>(Vo, r, c, pp, aown);
+                    decay_pairs<POWC>(Vx, ro, co, pp, aoth);
+                    gown[0] = fma2(Vo[0], gown[0], b01.x);
+                    goth[0] = fma2(Vx[0], goth[0], b01.x);
+                    gown[1] = fma2(Vo[1], gown[1], b01.y);
+                    goth[1] = fma2(Vx[1], goth[1], b01.y);
+                    gown[2] = fma2(Vo[2], gown[2], b23.x);
+                    goth[2] = fma2(Vx[2], goth[2], b23.x);
+                    gown[3] = fma2(Vo[3], gown[3], b23.y);
+                    goth[3] = fma2(Vx[3], goth[3], b23.y);
+                    uint64_t Yao = mul2(c01.x, gown[0]);
+                    uint64_t Yax = mul2(c01.x, goth[0]);
+                    uint64_t Ybo = mul2(c01.y, gown[1]);
+                    uint64_t Ybx = mul2(c01.y, goth[1]);
+                    Yao = fma2(c23.x, gown[2], Yao);
+                    Yax = fma2(c23.x, goth[2], Yax);
+                    Ybo = fma2(c23.y, gown[3], Ybo);
+                    Ybx = fma2(c23.y, goth[3], Ybx);
+                    const uint64_t Yo = add2(Yao, Ybo), Yx = add2(Yax, Ybx);
+                    // own channel output: own half + partner's half for this channel
+                    const float part = __shfl_xor_sync(0xffffffffu, lo2(Yx) + hi2(Yx), 1);
+                    float v = (lo2(Yo) + hi2(Yo) + part) * w;
+                    v = fmaf(dsk, uv, v);
+                    if (GATE) {
+                        const uint32_t zw = (i < 2 ? zq.x : i < 4 ? zq.y : i < 6 ? zq.z : zq.w);
+                        const float zv =
+                            __uint_as_float((i & 1) ? (zw & 0xffff0000u) : (zw << 16));
+                        v *= silu_fast(zv);
+                    }
+                    const uint32_t hv = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
+                    if (i & 1)
+                        ypk[i >> 1] |= hv << 16;
+                    else
+                        ypk[i >> 1] = hv;
+                }
+                *reinterpret_cast<uint4 *>(y_row + off) = make_uint4(ypk[0], ypk[1], ypk[2], ypk[3]);
+            }
+        };
+        if (pow_path)
+            run(std::true_type{});
+        else
+            run(std::false_type{});
+
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[s]);
+
+        if (inf.z & kInfoLast) {
+            // back to h = w_last * g; the partner's w arrives by shuffle
+            const float wo = __shfl_xor_sync(0xffffffffu, wprev, 1);
+            float hown[8], hoth[8];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                hown[2 * jj] = lo2(gown[jj]) * wprev;
+                hown[2 * jj + 1] = hi2(gown[jj]) * wprev;
+                hoth[2 * jj] = lo2(goth[jj]) * wo;
+                hoth[2 * jj + 1] = hi2(goth[jj]) * wo;
+            }
+            // continue from h with w_{-1} := 1
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                gown[jj] = pk2(hown[2 * jj], hown[2 * jj + 1]);
+                goth[jj] = pk2(hoth[2 * jj], hoth[2 * jj + 1]);
+            }
+            wprev = 1.f;
+            if (k < p.num_segs - 1) {
+                // [unit][channel][parity][8]: this lane writes parity pp of both channels
+                float4 *dst = reinterpret_cast<float4 *>(
+                    p.carry + (size_t(unit) * CH + ch) * kDiagN + pp * 8);
+                float4 *dsx = reinterpret_cast<float4 *>(
+                    p.carry + (size_t(unit) * CH + (ch ^ 1)) * kDiagN + pp * 8);
+                dst[0] = make_float4(hown[0], hown[1], hown[2], hown[3]);
+                dst[1] = make_float4(hown[4], hown[5], hown[6], hown[7]);
+                dsx[0] = make_float4(hoth[0], hoth[1], hoth[2], hoth[3]);
+                dsx[1] = make_float4(hoth[4], hoth[5], hoth[6], hoth[7]);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0 && unit != p.dbg_skip_publish)
+                    st_release_gpu(p.flags + size_t(unit) * CW + warp, 1u);
+            } else if (p.last_state && d < p.dim) {
+                // natural layout (batch, dim, 16): this lane's parity of its own channel
+                float *dst = p.last_state + (size_t(b) * p.dim + d) * kDiagN;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    dst[2 * j + pp] = hown[j];
+                const int dpart = d0 + (ch ^ 1);
+                if (dpart < p.dim) {
+                    float *dsx = p.last_state + (size_t(b) * p.dim + dpart) * kDiagN;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dsx[2 * j + pp] = hoth[j];
+                }
+            }
+        }
+        prev_t0 = inf.y;
+        prev_d0 = d0;
+        prev_b = b;
+        ++it;
+        if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+        }
+    }
+
+    named_bar_sync(1, CONS);
+    if (tid == 0) {
+        if (it > 0 && !*abort_flag) {
+            tma_store_3d(&tm_y, ytile + ((it - 1) & 1) * TILE, prev_t0, prev_d0, prev_b);
+            bulk_commit();
+        }
+        bulk_wait_all<0>();
+    }
+}
+
+}  // namespace selscan

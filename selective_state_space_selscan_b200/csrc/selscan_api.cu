@@ -14,6 +14,7 @@
 #include "selscan.h"
 #include "selscan_debug.h"
 #include "scan_diag.cuh"
+#include "scan_diag_bf16.cuh"
 #include "ssd_scalarA.cuh"
 
 using namespace selscan;
@@ -109,6 +110,8 @@ selscan_status check_seq(const selscan_tensor *t, int64_t d0, int64_t d1, int64_
         return SELSCAN_ERR_SHAPE;
     if (t->dtype != dtype)
         return SELSCAN_ERR_DTYPE;
+    if (d0 == 0 || d1 == 0 || L == 0)
+        return SELSCAN_OK;  // nothing will be read or written
     if (L > 1 && t->stride[2] != 1)
         return SELSCAN_ERR_STRIDE;
     if (t->stride[0] < 0 || t->stride[1] < 0)
@@ -131,10 +134,13 @@ selscan_status check_param(const selscan_tensor *t, int ndim, const int64_t *sha
     }
     if (t->ndim != ndim)
         return SELSCAN_ERR_SHAPE;
-    int64_t expect = 1;
+    int64_t expect = 1, count = 1;
     for (int i = ndim - 1; i >= 0; --i) {
         if (t->shape[i] != shape[i])
             return SELSCAN_ERR_SHAPE;
+        count *= shape[i];
+    }
+    for (int i = ndim - 1; i >= 0 && count > 0; --i) {
         if (shape[i] > 1 && t->stride[i] != expect)
             return SELSCAN_ERR_STRIDE;
         expect *= shape[i];
@@ -178,15 +184,39 @@ bool encode_3d(CUtensorMap *m, const void *ptr, int32_t dtype, int64_t L, int64_
 int g_dbg_skip_publish = -1;  // test hook, see selscan_debug_withhold_carry
 
 // ----------------------------------------------------- diagonal-A launch
-template <typename T, int CH, int STAGES, bool GATE>
+// Kernel variants share one launcher: KIND 0 = portable kernel (fp32 and
+// bf16, one lane pair per channel); KIND 1 = fast bf16 kernel (one lane per
+// channel, lane pairs share two channels' states).
+template <int KIND, typename T, int CH, int STAGES, bool GATE, bool SOFTPLUS>
+struct DiagVariant;
+
+template <typename T, int CH, int STAGES, bool GATE, bool SOFTPLUS>
+struct DiagVariant<0, T, CH, STAGES, GATE, SOFTPLUS> {
+    static constexpr int kChunk = DiagShape<T>::kChunk;
+    static constexpr int kThreads = CH * 2 + 32;
+    static constexpr int kConsWarps = CH * 2 / 32;
+    static constexpr int kSmem = DiagLayout<T, CH, STAGES, GATE>::kAlloc;
+    static constexpr auto kernel() { return scan_diag_kernel<T, CH, STAGES, GATE>; }
+};
+
+template <int CH, int STAGES, bool GATE, bool SOFTPLUS>
+struct DiagVariant<1, __nv_bfloat16, CH, STAGES, GATE, SOFTPLUS> {
+    static constexpr int kChunk = 64;
+    static constexpr int kThreads = CH + 32;
+    static constexpr int kConsWarps = CH / 32;
+    static constexpr int kSmem = DiagFastLayout<CH, STAGES, GATE>::kAlloc;
+    static constexpr auto kernel() { return scan_diag_bf16_kernel<CH, STAGES, GATE, SOFTPLUS>; }
+};
+
+template <int KIND, typename T, int CH, int STAGES, bool GATE, bool SOFTPLUS>
 selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
                            const selscan_tensor *B, const selscan_tensor *C,
                            const selscan_tensor *z, selscan_tensor *y, DiagParams prm,
                            int sm_count, cudaStream_t stream)
 {
-    using Lay = DiagLayout<T, CH, STAGES, GATE>;
-    constexpr int TC = DiagShape<T>::kChunk;
-    constexpr int CW = CH * 2 / 32;
+    using V = DiagVariant<KIND, T, CH, STAGES, GATE, SOFTPLUS>;
+    constexpr int TC = V::kChunk;
+    constexpr int CW = V::kConsWarps;
     const int32_t dt = u->dtype;
     const int64_t batch = prm.batch, dim = prm.dim, L = prm.L;
     const int64_t Bn = kDiagN;
@@ -255,20 +285,20 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
     prm.carry = reinterpret_cast<float *>(wsb + head + flag_bytes);
     prm.dbg_skip_publish = g_dbg_skip_publish;
 
-    auto kern = scan_diag_kernel<T, CH, STAGES, GATE>;
+    auto kern = V::kernel();
     static bool attr_set[kMaxDevices] = {};  // per instantiation and device
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Lay::kAlloc) != cudaSuccess) {
+                                 V::kSmem) != cudaSuccess) {
             cudaFreeAsync(ws, stream);
             return SELSCAN_ERR_CUDA;
         }
         attr_set[dev] = true;
     }
     const int grid = int(std::min<int64_t>(ctas_max, units));
-    kern<<<grid, CH * 2 + 32, Lay::kAlloc, stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, prm);
+    kern<<<grid, V::kThreads, V::kSmem, stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, prm);
     const cudaError_t le = cudaGetLastError();
     cudaFreeAsync(ws, stream);
     return le == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
@@ -406,16 +436,18 @@ selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
     prm.err = di->err;
 
     const bool gate = z && z->data;
+    const int sms = di->sm_count;
     if (dt == SELSCAN_BF16) {
-        return gate ? launch_diag<__nv_bfloat16, 64, 4, true>(u, delta, B, C, z, y, prm,
-                                                              di->sm_count, stream)
-                    : launch_diag<__nv_bfloat16, 64, 4, false>(u, delta, B, C, z, y, prm,
-                                                               di->sm_count, stream);
+        if (gate)
+            return prm.softplus
+                       ? launch_diag<1, __nv_bfloat16, 128, 3, true, true>(u, delta, B, C, z, y, prm, sms, stream)
+                       : launch_diag<1, __nv_bfloat16, 128, 3, true, false>(u, delta, B, C, z, y, prm, sms, stream);
+        return prm.softplus
+                   ? launch_diag<1, __nv_bfloat16, 128, 4, false, true>(u, delta, B, C, z, y, prm, sms, stream)
+                   : launch_diag<1, __nv_bfloat16, 128, 4, false, false>(u, delta, B, C, z, y, prm, sms, stream);
     }
-    return gate ? launch_diag<float, 64, 4, true>(u, delta, B, C, z, y, prm, di->sm_count,
-                                                  stream)
-                : launch_diag<float, 64, 4, false>(u, delta, B, C, z, y, prm, di->sm_count,
-                                                   stream);
+    return gate ? launch_diag<0, float, 64, 4, true, true>(u, delta, B, C, z, y, prm, sms, stream)
+                : launch_diag<0, float, 64, 4, false, true>(u, delta, B, C, z, y, prm, sms, stream);
 }
 
 selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor *dt,
