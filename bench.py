@@ -68,11 +68,12 @@ def algorithmic_bytes(cfg: dict) -> int:
     return total
 
 
-def ssd_flops(cfg: dict) -> float:
-    """Tensor-core FLOPs of the chunked SSD form per call (C.B^T once per
-    batch and chunk since heads share B/C; per head the intra-chunk product,
-    the chunk state and the carried-in term)."""
-    b, L, Q = cfg["batch"], cfg["L"], cfg["chunk"]
+def ssd_flops(cfg: dict, Q: int = 128) -> float:
+    """Tensor-core FLOPs of the chunked SSD form per call at chunk length Q
+    (the kernel's Q = 128): C.B^T once per batch and chunk since heads share
+    B/C; per head the intra-chunk product, the chunk state and the
+    carried-in term."""
+    b, L = cfg["batch"], cfg["L"]
     H, P, N = cfg["nheads"], cfg["headdim"], cfg["N"]
     nch = (L + Q - 1) // Q
     per_chunk = 2 * Q * Q * N + H * (2 * Q * Q * P + 2 * N * Q * P + 2 * Q * N * P)

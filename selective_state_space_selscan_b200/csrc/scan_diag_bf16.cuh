@@ -40,24 +40,12 @@ namespace selscan {
 
 __device__ __forceinline__ uint64_t pk2(float lo, float hi)
 {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
+    return (uint64_t(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
 }
 
-__device__ __forceinline__ float lo2(uint64_t v)
-{
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return lo;
-}
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float(uint32_t(v)); }
 
-__device__ __forceinline__ float hi2(uint64_t v)
-{
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return hi;
-}
+__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float(uint32_t(v >> 32)); }
 
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
 {

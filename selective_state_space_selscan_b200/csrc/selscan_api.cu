@@ -521,9 +521,52 @@ selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor
     DeviceInfo *di = nullptr;
     if ((st = device_setup(&dev, &di)) != SELSCAN_OK)
         return st;
-    (void)dt_softplus;
-    (void)stream;
-    return SELSCAN_ERR_UNSUPPORTED;  // kernel added separately
+
+    // B/C (batch, 1, N, L) -> 3-D maps over (L, N, batch); x over (L, H*P, batch)
+    CUtensorMap tm_C, tm_B, tm_X;
+    if (!encode_3d(&tm_C, C->data, SELSCAN_BF16, L, N, batch, C->stride[2], C->stride[0], 64,
+                   kSsdN) ||
+        !encode_3d(&tm_B, B->data, SELSCAN_BF16, L, N, batch, B->stride[2], B->stride[0], 64,
+                   kSsdN) ||
+        !encode_3d(&tm_X, x->data, SELSCAN_BF16, L, dim, batch, x->stride[1], x->stride[0], 64,
+                   kSsdP))
+        return SELSCAN_ERR_ALIGN;
+    SsdParams prm{};
+    prm.batch = int(batch);
+    prm.H = int(H);
+    prm.L = int(L);
+    prm.nchunks = int((L + kSsdQ - 1) / kSsdQ);
+    prm.dt = static_cast<const float *>(dt->data);
+    prm.dt_bs = dt->stride[0];
+    prm.dt_hs = dt->stride[1];
+    prm.dt_bias = static_cast<const float *>(opt_data(dt_bias));
+    prm.softplus = dt_softplus ? 1 : 0;
+    prm.A = static_cast<const float *>(A->data);
+    prm.Dskip = static_cast<const float *>(opt_data(D));
+    const bool gate = z && z->data;
+    prm.z = gate ? static_cast<const __nv_bfloat16 *>(z->data) : nullptr;
+    prm.z_bs = gate ? z->stride[0] : 0;
+    prm.z_cs = gate ? z->stride[1] : 0;
+    prm.y = static_cast<__nv_bfloat16 *>(y->data);
+    prm.y_bs = y->stride[0];
+    prm.y_cs = y->stride[1];
+    prm.last_state = static_cast<float *>(last_state ? last_state->data : nullptr);
+    prm.timeout_ns = default_timeout_ns();
+    prm.err = di->err;
+
+    auto kern = gate ? ssd_scalarA_kernel<true> : ssd_scalarA_kernel<false>;
+    static bool attr_set[2][kMaxDevices] = {};
+    if (!attr_set[gate][dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SsdLayout::kAlloc) != cudaSuccess)
+            return SELSCAN_ERR_CUDA;
+        attr_set[gate][dev] = true;
+    }
+    const int64_t grid = batch * H;
+    if (grid > 0x7fffffffll)
+        return SELSCAN_ERR_UNSUPPORTED;
+    kern<<<unsigned(grid), 128, SsdLayout::kAlloc, stream>>>(tm_C, tm_B, tm_X, prm);
+    return cudaGetLastError() == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
 }
 
 }  // extern "C"
