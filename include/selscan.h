@@ -137,6 +137,41 @@ SELSCAN_API selscan_status selscan_fwd_scalarA(const selscan_tensor *x,
                                    cudaStream_t stream);
 
 /*
+ * selscan_fwd_noalloc -- selscan_fwd for callers that cannot allocate device
+ * memory during a call.  The paper has no counterpart; this entry point
+ * exists for deployments such as fixed-footprint inference servers or
+ * real-time loops that reserve all memory at start-up and forbid allocation
+ * afterwards, and for systems where the stream-ordered allocator (memory
+ * pools, which selscan_fwd uses for its scratch) is unavailable.
+ *
+ * Same arguments, layouts and results as selscan_fwd; the caller passes all
+ * inputs and outputs.  Instead of cudaMallocAsync, the look-back scratch
+ * (ticket, carry flags, segment carries) lives in one file-scope device
+ * array of SELSCAN_NOALLOC_SCRATCH_BYTES per GPU, which every GPU that loads
+ * the library holds until the process exits.  The call makes no
+ * cudaMalloc / cudaFree / allocating call; it clears the part of the array
+ * that must start at zero with cudaMemsetAsync on `stream`.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents: calls that overlap on the GPU (different streams, no
+ *     ordering between them) race on it.  Serialise them.
+ *   - A launch whose scratch would exceed the array returns
+ *     SELSCAN_ERR_UNSUPPORTED and launches nothing.  The scratch is
+ *     256 bytes plus (segments - 1) * tiles * (flags + 128 or 64 carried
+ *     channels * 64 bytes); the library's scheduling keeps
+ *     (segments - 1) * tiles below 8 * SM count, about 9.7 MiB on a
+ *     148-SM B200.
+ */
+#define SELSCAN_NOALLOC_SCRATCH_BYTES (16u << 20)
+SELSCAN_API selscan_status selscan_fwd_noalloc(
+    const selscan_tensor *u, const selscan_tensor *delta, const selscan_tensor *delta_bias,
+    int delta_softplus, const selscan_tensor *A, const selscan_tensor *B,
+    const selscan_tensor *C, const selscan_tensor *D, const selscan_tensor *z,
+    selscan_tensor *y, selscan_tensor *last_state, cudaStream_t stream);
+
+/*
  * selscan_check -- synchronise `stream` and report device-side errors that
  * earlier calls recorded (a bounded wait that gave up returns
  * SELSCAN_ERR_TIMEOUT; the record is then cleared).  Returns

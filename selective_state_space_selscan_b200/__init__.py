@@ -69,6 +69,9 @@ def lib() -> ctypes.CDLL:
         for f in (L.selscan_fwd, L.selscan_fwd_scalarA, L.selscan_check,
                   L.selscan_version):
             f.restype = ctypes.c_int
+        L.selscan_fwd_noalloc.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, P, P, P,
+                                          ctypes.c_void_p]
+        L.selscan_fwd_noalloc.restype = ctypes.c_int
         L.selscan_debug_withhold_carry.argtypes = [ctypes.c_int]
         L.selscan_debug_withhold_carry.restype = None
         _lib = L
@@ -138,6 +141,30 @@ def selscan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     if rc != 0:
         raise SelscanError(rc, "selscan_fwd")
     return y, last_state
+
+
+def selscan_fwd_noalloc(u, delta, A, B, C, out, D=None, z=None, delta_bias=None,
+                        delta_softplus=True, last_state=None, stream=None):
+    """selscan_fwd for callers that cannot allocate device memory during a
+    call (fixed-footprint servers or real-time loops that reserve memory at
+    start-up, or systems without the stream-ordered allocator that
+    selscan_fwd uses for its scratch).  The library keeps the scratch in one
+    static device array per GPU, shared by all calls: calls that overlap on
+    the GPU race, so serialise them, and make the first call on a device
+    before any stream capture (it looks up the array's address).
+
+    ``out`` (the y buffer) and the optional ``last_state`` must be passed;
+    nothing is allocated here either.  Returns (out, last_state).
+    """
+    descs = [describe(t) for t in (u, delta, delta_bias, A, B, C, D, z, out, last_state)]
+    rc = lib().selscan_fwd_noalloc(_ref(descs[0]), _ref(descs[1]), _ref(descs[2]),
+                                   int(bool(delta_softplus)), _ref(descs[3]),
+                                   _ref(descs[4]), _ref(descs[5]), _ref(descs[6]),
+                                   _ref(descs[7]), _ref(descs[8]), _ref(descs[9]),
+                                   _stream_handle(stream))
+    if rc != 0:
+        raise SelscanError(rc, "selscan_fwd_noalloc")
+    return out, last_state
 
 
 def selscan_fwd_scalarA(x, dt, A, B, C, headdim, D=None, z=None, dt_bias=None,

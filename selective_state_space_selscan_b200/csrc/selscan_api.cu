@@ -570,3 +570,221 @@ selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// selscan_fwd_noalloc: the same scan with its scratch in a static device
+// array instead of stream-ordered allocations (see include/selscan.h).
+// ---------------------------------------------------------------------------
+
+// One array per GPU that loads this library, held until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SELSCAN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+uint8_t *g_noalloc_ptr[kMaxDevices] = {};  // device address of the array
+
+// Once per device, with that device current: the array's device address.
+// (In host code the symbol name is only a stand-in, not a device address.)
+selscan_status noalloc_setup(int dev, uint8_t **out)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+            return SELSCAN_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<uint8_t *>(ptr);
+    }
+    *out = g_noalloc_ptr[dev];
+    return SELSCAN_OK;
+}
+
+template <int KIND, typename T, int CH, int STAGES, bool GATE, bool SOFTPLUS>
+selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor *delta,
+                                   const selscan_tensor *B, const selscan_tensor *C,
+                                   const selscan_tensor *z, selscan_tensor *y, DiagParams prm,
+                                   int sm_count, uint8_t *scratch, cudaStream_t stream)
+{
+    using V = DiagVariant<KIND, T, CH, STAGES, GATE, SOFTPLUS>;
+    constexpr int TC = V::kChunk;
+    constexpr int CW = V::kConsWarps;
+    const int32_t dt = u->dtype;
+    const int64_t batch = prm.batch, dim = prm.dim, L = prm.L;
+    auto bc_strides = [](const selscan_tensor *t, int64_t &rs, int64_t &bs) {
+        rs = t->ndim == 3 ? t->stride[1] : t->stride[2];
+        bs = t->stride[0];
+    };
+    CUtensorMap tm_u, tm_d, tm_z, tm_B, tm_C, tm_y;
+    int64_t brs, bbs, crs, cbs;
+    bc_strides(B, brs, bbs);
+    bc_strides(C, crs, cbs);
+    bool ok = encode_3d(&tm_u, u->data, dt, L, dim, batch, u->stride[1], u->stride[0], TC, CH) &&
+              encode_3d(&tm_d, delta->data, dt, L, dim, batch, delta->stride[1],
+                        delta->stride[0], TC, CH) &&
+              encode_3d(&tm_B, B->data, dt, L, kDiagN, batch, brs, bbs, TC, kDiagN) &&
+              encode_3d(&tm_C, C->data, dt, L, kDiagN, batch, crs, cbs, TC, kDiagN) &&
+              encode_3d(&tm_y, y->data, dt, L, dim, batch, y->stride[1], y->stride[0], TC, CH);
+    if (ok && GATE)
+        ok = encode_3d(&tm_z, z->data, dt, L, dim, batch, z->stride[1], z->stride[0], TC, CH);
+    else
+        tm_z = tm_u;
+    if (!ok)
+        return SELSCAN_ERR_ALIGN;
+
+    // same work decomposition as selscan_fwd
+    const int tpb = int((dim + CH - 1) / CH);
+    const int G = int(batch) * tpb;
+    const int ctas_max = sm_count;
+    const int64_t chunks = (L + TC - 1) / TC;
+    int64_t S = (8ll * ctas_max + G - 1) / G;
+    S = std::max<int64_t>(1, std::min<int64_t>(S, (chunks + 3) / 4));
+    const int64_t seg_chunks = (chunks + S - 1) / S;
+    S = (chunks + seg_chunks - 1) / seg_chunks;
+    const int64_t units = int64_t(G) * S;
+    if (units > 0x7fffffffll)
+        return SELSCAN_ERR_UNSUPPORTED;
+    // Only units of the first S-1 segments publish a carry and a flag.
+    const int64_t linked = int64_t(G) * (S - 1);
+    const size_t head = 256;
+    const size_t flag_bytes = ((size_t(linked) * CW * 4 + 255) / 256) * 256;
+    const size_t carry_bytes = size_t(linked) * CH * kDiagN * 4;
+    if (head + flag_bytes + carry_bytes > size_t(SELSCAN_NOALLOC_SCRATCH_BYTES))
+        return SELSCAN_ERR_UNSUPPORTED;  // the static array is too small for this launch
+    prm.tiles_per_batch = tpb;
+    prm.num_tiles = G;
+    prm.seg_len = int(seg_chunks * TC);
+    prm.num_segs = int(S);
+    prm.total_units = int(units);
+    // the previous call's ticket and flags must not leak into this one
+    if (cudaMemsetAsync(scratch, 0, head + flag_bytes, stream) != cudaSuccess)
+        return SELSCAN_ERR_CUDA;
+    prm.ticket = reinterpret_cast<unsigned int *>(scratch);
+    prm.flags = reinterpret_cast<unsigned int *>(scratch + head);
+    prm.carry = reinterpret_cast<float *>(scratch + head + flag_bytes);
+    prm.dbg_skip_publish = -1;
+
+    auto kern = V::kernel();
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 V::kSmem) != cudaSuccess)
+            return SELSCAN_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    const int grid = int(std::min<int64_t>(ctas_max, units));
+    kern<<<grid, V::kThreads, V::kSmem, stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, prm);
+    return cudaGetLastError() == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" selscan_status selscan_fwd_noalloc(
+    const selscan_tensor *u, const selscan_tensor *delta, const selscan_tensor *delta_bias,
+    int delta_softplus, const selscan_tensor *A, const selscan_tensor *B,
+    const selscan_tensor *C, const selscan_tensor *D, const selscan_tensor *z,
+    selscan_tensor *y, selscan_tensor *last_state, cudaStream_t stream)
+{
+    // ---- validation, identical rules to selscan_fwd (no CUDA call before it)
+    if (!present(u) || !delta || !A || !B || !C || !y)
+        return SELSCAN_ERR_NULL;
+    if (u->ndim != 3)
+        return SELSCAN_ERR_SHAPE;
+    const int32_t dt = u->dtype;
+    if (dt != SELSCAN_F32 && dt != SELSCAN_BF16)
+        return SELSCAN_ERR_DTYPE;
+    const int64_t batch = u->shape[0], dim = u->shape[1], L = u->shape[2];
+    if (batch < 0 || dim < 0 || L < 0)
+        return SELSCAN_ERR_SHAPE;
+    if (!present(A))
+        return SELSCAN_ERR_NULL;
+    if (A->ndim != 2 || A->shape[0] != dim)
+        return SELSCAN_ERR_SHAPE;
+    const int64_t N = A->shape[1];
+    selscan_status st;
+    if ((st = check_seq(u, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    if ((st = check_seq(delta, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    if ((st = check_seq(y, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    if (z && z->data && (st = check_seq(z, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    {
+        const int64_t ashape[2] = {dim, N};
+        if ((st = check_param(A, 2, ashape, false)) != SELSCAN_OK) return st;
+        const int64_t vshape[1] = {dim};
+        if ((st = check_param(delta_bias, 1, vshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(D, 1, vshape, true)) != SELSCAN_OK) return st;
+        const int64_t sshape[3] = {batch, dim, N};
+        if ((st = check_param(last_state, 3, sshape, true)) != SELSCAN_OK) return st;
+    }
+    for (const selscan_tensor *t : {B, C}) {
+        if (!present(t))
+            return SELSCAN_ERR_NULL;
+        if (t->ndim == 4) {
+            if (t->shape[1] != 1)
+                return SELSCAN_ERR_UNSUPPORTED;
+            selscan_tensor v = *t;
+            v.ndim = 3;
+            v.shape[1] = t->shape[2];
+            v.shape[2] = t->shape[3];
+            v.stride[1] = t->stride[2];
+            v.stride[2] = t->stride[3];
+            if ((st = check_seq(&v, batch, N, L, dt)) != SELSCAN_OK) return st;
+        } else {
+            if ((st = check_seq(t, batch, N, L, dt)) != SELSCAN_OK) return st;
+        }
+    }
+    if (N != kDiagN)
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch > 65535 || dim > (int64_t(1) << 30) || L > (int64_t(1) << 31) - 1024)
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch == 0 || dim == 0)
+        return SELSCAN_OK;
+    if (L == 0) {
+        if (last_state && last_state->data)
+            return cudaMemsetAsync(last_state->data, 0, size_t(batch * dim * N) * 4, stream) ==
+                           cudaSuccess
+                       ? SELSCAN_OK
+                       : SELSCAN_ERR_CUDA;
+        return SELSCAN_OK;
+    }
+
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    if ((st = device_setup(&dev, &di)) != SELSCAN_OK)
+        return st;
+    uint8_t *scratch = nullptr;
+    if ((st = noalloc_setup(dev, &scratch)) != SELSCAN_OK)
+        return st;
+
+    DiagParams prm{};
+    prm.batch = int(batch);
+    prm.dim = int(dim);
+    prm.L = int(L);
+    prm.A = static_cast<const float *>(A->data);
+    prm.delta_bias = static_cast<const float *>(opt_data(delta_bias));
+    prm.Dskip = static_cast<const float *>(opt_data(D));
+    prm.h0 = nullptr;
+    prm.last_state = static_cast<float *>(last_state ? last_state->data : nullptr);
+    prm.softplus = delta_softplus ? 1 : 0;
+    prm.timeout_ns = default_timeout_ns();
+    prm.err = di->err;
+
+    const bool gate = z && z->data;
+    const int sms = di->sm_count;
+    if (dt == SELSCAN_BF16) {
+        if (gate)
+            return prm.softplus
+                       ? launch_diag_noalloc<1, __nv_bfloat16, 128, 3, true, true>(
+                             u, delta, B, C, z, y, prm, sms, scratch, stream)
+                       : launch_diag_noalloc<1, __nv_bfloat16, 128, 3, true, false>(
+                             u, delta, B, C, z, y, prm, sms, scratch, stream);
+        return prm.softplus
+                   ? launch_diag_noalloc<1, __nv_bfloat16, 128, 4, false, true>(
+                         u, delta, B, C, z, y, prm, sms, scratch, stream)
+                   : launch_diag_noalloc<1, __nv_bfloat16, 128, 4, false, false>(
+                         u, delta, B, C, z, y, prm, sms, scratch, stream);
+    }
+    return gate ? launch_diag_noalloc<0, float, 64, 4, true, true>(u, delta, B, C, z, y, prm, sms,
+                                                                    scratch, stream)
+                : launch_diag_noalloc<0, float, 64, 4, false, true>(u, delta, B, C, z, y, prm,
+                                                                     sms, scratch, stream);
+}
