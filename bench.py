@@ -32,7 +32,21 @@ sys.path.insert(0, ROOT)
 
 import synthetic  # noqa: E402
 
+BASE_CONFIGS = {k: dict(v) for k, v in synthetic.CONFIGS.items()}
+
 METRIC = "selective-scan Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU"
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+# ncu captures summarised in profiles/, keyed by config and the kernel they
+# were taken on; reported as roofline.traffic only for that kernel.
+NCU_TRAFFIC = {
+    # config 2 captured at L = 2048 (320 MB), scaled by tokens to L = 4096
+    2: ("scan_diag_bf16_kernel streaming v1", 640.0e6),
+    4: ("ssd_scalarA_kernel v1", 109.0e6),
+}
+KERNEL_TAG = {2: "scan_diag_bf16_kernel streaming v1", 1: "scan_diag_bf16_kernel streaming v1",
+              3: "scan_diag_bf16_kernel streaming v1", 0: "scan_diag_kernel fp32 v1",
+              4: "ssd_scalarA_kernel v1"}
 HBM_FALLBACK_GBS = 6650.0
 
 
@@ -371,8 +385,13 @@ def run_gpu(args, rank: int, world: int, local: int):
     peaks, peaks_src = measured_peaks()
     nbytes = algorithmic_bytes(cfg)
     achieved = nbytes / (avg_launch_ms * 1e-3) / 1e9
+    traffic = args.traffic
+    if traffic is None and args.config in NCU_TRAFFIC and \
+            NCU_TRAFFIC[args.config][0] == KERNEL_TAG.get(args.config) and \
+            synthetic.CONFIGS[args.config] == BASE_CONFIGS[args.config]:
+        traffic = NCU_TRAFFIC[args.config][1]
     roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / peaks["hbm_gbs"], "traffic": args.traffic,
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
             "peak_source": f"{peaks_src} HBM copy bandwidth",
             "bytes_per_launch": nbytes, "avg_launch_ms": avg_launch_ms}
     if cfg["kind"] == "scalarA":
