@@ -40,12 +40,12 @@ METRIC = "selective-scan Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU"
 # ncu captures summarised in profiles/, keyed by config and the kernel they
 # were taken on; reported as roofline.traffic only for that kernel.
 NCU_TRAFFIC = {
-    # config 2 captured at L = 2048 (320 MB), scaled by tokens to L = 4096
-    2: ("scan_diag_bf16_kernel streaming v1", 640.0e6),
+    # config 2 captured at L = 2048, scaled by tokens to L = 4096 (see profiles/)
+    2: ("scan_diag_bf16_kernel pairs v3", None),
     4: ("ssd_scalarA_kernel v1", 109.0e6),
 }
-KERNEL_TAG = {2: "scan_diag_bf16_kernel streaming v1", 1: "scan_diag_bf16_kernel streaming v1",
-              3: "scan_diag_bf16_kernel streaming v1", 0: "scan_diag_kernel fp32 v1",
+KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v3", 1: "scan_diag_bf16_kernel pairs v3",
+              3: "scan_diag_bf16_kernel pairs v3", 0: "scan_diag_kernel fp32 v1",
               4: "ssd_scalarA_kernel v1"}
 HBM_FALLBACK_GBS = 6650.0
 

@@ -6,14 +6,15 @@
 // with bulk tensor copies, carries linked by gpu-scope release/acquire
 // flags), with an inner loop laid out for the B200 SM:
 //
-//  * One consumer lane per channel for everything that is per token
-//    (softplus, delta*u, the decay base, gate, D skip, output): its row of
-//    the input tile is read with 16-byte shared loads, 8 tokens at a time.
-//  * The 16 states of a PAIR of channels are split between the two lanes of
-//    a lane pair by parity: lane p keeps states n = p, p+2, ..., p+14 of both
-//    channels.  B and C of one token therefore serve two channels per load,
-//    which halves the shared-memory traffic per element; they are staged
-//    once per chunk as packed bf16 pairs and widened in registers.
+//  * Two consumer lanes per channel (a lane pair), 128 channels per CTA, so
+//    that each scheduler runs two consumer warps.  Lane p keeps the states of
+//    parity p (n = p, p+2, ..., p+14) in registers and prepares the per-token
+//    values (softplus, w = delta*u, the decay base, 1/w) of half of each
+//    8-token block; the pair swaps them with warp shuffles, runs the 8 steps,
+//    and reduce-scatters the two partial outputs so each lane finishes four
+//    tokens (D skip, gate, bf16 store).  B and C of a chunk are staged once
+//    per CTA as fp32, token-major, parity-split, so every lane reads its 8 B
+//    and 8 C values of a token with four 16-byte broadcast loads.
 //  * The state is kept rescaled, g = h / w with w = delta * u, so that the
 //    input term needs no multiply:  g_t = (w_{t-1}/w_t) exp(delta_t A) g_{t-1}
 //    + B_t and y_t = w_t (C_t . g_t).  |w| is kept >= 2^-64 so that the
@@ -24,9 +25,6 @@
 //    the odd (p=0) or even (p=1) powers, i.e. base * s^j with s = r^2,
 //    computed with packed f32x2 multiplies.  Other A use one ex2 per state.
 //  * Packed f32x2 FMAs (sm_100) update two states per instruction.
-//  * The token-wise prologue of the next 8-token block is computed before
-//    the state updates of the current one so its special-function latency
-//    overlaps the FMA work.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -110,41 +108,6 @@ struct DiagFastLayout {
     static constexpr int kAlloc = kBytes + 1024;
 };
 
-// Per-token values of one 8-token block for this lane's own channel.
-struct Prologue {
-    float r[8];   // decay base (POW) or delta (general)
-    float c[8];   // w_{t-1} / w_t
-    float w[8];   // rescale factor w_t = delta_t u_t (clamped)
-    float u[8];
-    float z[8];
-};
-
-template <bool POW, bool SOFTPLUS, bool GATE, bool TAIL>
-__device__ __forceinline__ void fast_prologue(Prologue &P, const uint8_t *u_row,
-                                              const uint8_t *dl_row, const uint8_t *z_row,
-                                              int off, int t_base, int L, float bias,
-                                              float a0, float &wprev)
-{
-    float dv[8];
-    unpack8_bf16(*reinterpret_cast<const uint4 *>(u_row + off), P.u);
-    unpack8_bf16(*reinterpret_cast<const uint4 *>(dl_row + off), dv);
-    if (GATE)
-        unpack8_bf16(*reinterpret_cast<const uint4 *>(z_row + off), P.z);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float x = dv[i] + bias;
-        float dt = SOFTPLUS ? softplus_fast(x) : x;
-        if (TAIL)
-            dt = (t_base + i < L) ? dt : 0.f;  // padding: identity step
-        const float wr = dt * P.u[i];
-        const float w = copysignf(fmaxf(fabsf(wr), kWMin), wr);
-        P.r[i] = POW ? ex2_approx(dt * a0) : dt;
-        P.c[i] = wprev * rcp_approx(w);
-        P.w[i] = w;
-        wprev = w;
-    }
-}
-
 template <bool POW>
 __device__ __forceinline__ void decay_pairs(uint64_t (&V)[4], float r, float c, int p,
                                             const uint64_t (&apair)[4])
@@ -170,58 +133,8 @@ __device__ __forceinline__ void decay_pairs(uint64_t (&V)[4], float r, float c, 
     }
 }
 
-// 8 tokens of the scan for this lane's state parity of both channels.
-template <bool POW>
-__device__ __forceinline__ void scan_block8(uint64_t (&gown)[4], uint64_t (&goth)[4],
-                                            const float *bcb_blk, int pp, const Prologue &P,
-                                            const float (&ro)[8], const float (&co)[8],
-                                            const uint64_t (&aown)[4],
-                                            const uint64_t (&aoth)[4], float (&yown)[8],
-                                            float (&yoth)[8])
-{
-    uint64_t Vo[4], Vx[4];
-    decay_pairs<POW>(Vo, P.r[0], P.c[0], pp, aown);
-    decay_pairs<POW>(Vx, ro[0], co[0], pp, aoth);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const ulonglong2 *bq = reinterpret_cast<const ulonglong2 *>(bcb_blk + i * 32 + pp * 16);
-        const ulonglong2 b01 = bq[0], b23 = bq[1], c01 = bq[2], c23 = bq[3];
-        uint64_t Von[4], Vxn[4];
-        if (i + 1 < 8) {
-            decay_pairs<POW>(Von, P.r[i + 1], P.c[i + 1], pp, aown);
-            decay_pairs<POW>(Vxn, ro[i + 1], co[i + 1], pp, aoth);
-        }
-        gown[0] = fma2(Vo[0], gown[0], b01.x);
-        goth[0] = fma2(Vx[0], goth[0], b01.x);
-        gown[1] = fma2(Vo[1], gown[1], b01.y);
-        goth[1] = fma2(Vx[1], goth[1], b01.y);
-        gown[2] = fma2(Vo[2], gown[2], b23.x);
-        goth[2] = fma2(Vx[2], goth[2], b23.x);
-        gown[3] = fma2(Vo[3], gown[3], b23.y);
-        goth[3] = fma2(Vx[3], goth[3], b23.y);
-        uint64_t Yao = mul2(c01.x, gown[0]);
-        uint64_t Yax = mul2(c01.x, goth[0]);
-        uint64_t Ybo = mul2(c01.y, gown[1]);
-        uint64_t Ybx = mul2(c01.y, goth[1]);
-        Yao = fma2(c23.x, gown[2], Yao);
-        Yax = fma2(c23.x, goth[2], Yax);
-        Ybo = fma2(c23.y, gown[3], Ybo);
-        Ybx = fma2(c23.y, goth[3], Ybx);
-        const uint64_t Yo = add2(Yao, Ybo), Yx = add2(Yax, Ybx);
-        yown[i] = lo2(Yo) + hi2(Yo);
-        yoth[i] = lo2(Yx) + hi2(Yx);
-        if (i + 1 < 8) {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                Vo[jj] = Von[jj];
-                Vx[jj] = Vxn[jj];
-            }
-        }
-    }
-}
-
 template <int CH, int STAGES, bool GATE, bool SOFTPLUS>
-__global__ void __launch_bounds__(CH + 32, 1)
+__global__ void __launch_bounds__(2 * CH + 32, 1)
 scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                       const __grid_constant__ CUtensorMap tm_delta,
                       const __grid_constant__ CUtensorMap tm_z,
@@ -232,7 +145,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
 {
     using Lay = DiagFastLayout<CH, STAGES, GATE>;
     constexpr int TC = Lay::kChunk;
-    constexpr int CONS = CH;      // one consumer lane per channel
+    constexpr int CONS = 2 * CH;  // two consumer lanes per channel
     constexpr int CW = CONS / 32;
     constexpr int TILE = Lay::kTile;
     static_assert(CONS % 32 == 0, "consumer threads must fill warps");
@@ -322,16 +235,14 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
     }
 
     // ---------------------------------------------------------- consumers
-    const int ch = tid;          // this lane's own channel within the tile
-    const int pp = tid & 1;      // state parity handled by this lane
+    const int ch = tid >> 1;     // channel within the tile
+    const int pp = tid & 1;      // state parity held by this lane; token half it prepares
     const int swz = ch & 7;      // 128-byte swizzle phase of this row
-    uint64_t gown[4], goth[4];   // rescaled states, parity pp, own / partner channel
+    uint64_t g[4];               // rescaled states n = pp, pp+2, ..., pp+14 (pairs)
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-        gown[jj] = pk2(0.f, 0.f);
-        goth[jj] = pk2(0.f, 0.f);
-    }
-    uint64_t aown[4], aoth[4];   // A*log2e of this lane's states, paired (general path)
+    for (int jj = 0; jj < 4; ++jj)
+        g[jj] = pk2(0.f, 0.f);
+    uint64_t apair[4];           // A*log2e of this lane's states, paired (general path)
     float a0 = 0.f, bias = 0.f, dsk = 0.f, wprev = 1.f;
     bool pow_path = true;
     int unit = -1, k = 0, b = 0, d0 = 0, d = 0;
@@ -351,50 +262,36 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
         if (arrived && (inf.z & kInfoFirst)) {
             unit = inf.x;
             k = unit / G;
-            const int g = unit - k * G;
-            b = g / p.tiles_per_batch;
-            d0 = (g - b * p.tiles_per_batch) * CH;
+            const int gg = unit - k * G;
+            b = gg / p.tiles_per_batch;
+            d0 = (gg - b * p.tiles_per_batch) * CH;
             d = d0 + ch;
-            const int dpart = d0 + (ch ^ 1);
-            const bool live = d < p.dim, live_o = dpart < p.dim;
+            const bool live = d < p.dim;
             const float *arow = p.A + size_t(live ? d : 0) * kDiagN;
-            const float *orow = p.A + size_t(live_o ? dpart : 0) * kDiagN;
-            const float A0 = arow[0], O0 = orow[0];
+            const float A0 = arow[0];
             bool ok = true;
-            float al[8], ol[8];
+            float al[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int n = 2 * j + pp;  // this lane's states
-                const float an = arow[n], on = orow[n];
-                ok = ok && (an == float(n + 1) * A0) && (on == float(n + 1) * O0);
+                const float an = arow[n];
+                ok = ok && (an == float(n + 1) * A0);
                 al[j] = an * kLog2e;
-                ol[j] = on * kLog2e;
             }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                aown[jj] = pk2(al[2 * jj], al[2 * jj + 1]);
-                aoth[jj] = pk2(ol[2 * jj], ol[2 * jj + 1]);
-            }
-            // every lane also needs its own channel's full row structure
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int n = 2 * j + (pp ^ 1);
-                ok = ok && (arow[n] == float(n + 1) * A0);
-            }
+            for (int jj = 0; jj < 4; ++jj)
+                apair[jj] = pk2(al[2 * jj], al[2 * jj + 1]);
             a0 = A0 * kLog2e;
             pow_path = __all_sync(0xffffffffu, ok);
             bias = (p.delta_bias && live) ? p.delta_bias[d] : 0.f;
             dsk = (p.Dskip && live) ? p.Dskip[d] : 0.f;
             wprev = 1.f;  // g starts as h_in (w_{-1} := 1)
-            float hown[8], hoth[8];
+            float hv[8];
             if (k == 0) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int n = 2 * j + pp;
-                    hown[j] = (p.h0 && live) ? p.h0[(size_t(b) * p.dim + d) * kDiagN + n] : 0.f;
-                    hoth[j] = (p.h0 && live_o)
-                                  ? p.h0[(size_t(b) * p.dim + dpart) * kDiagN + n] : 0.f;
-                }
+                for (int j = 0; j < 8; ++j)
+                    hv[j] = (p.h0 && live) ? p.h0[(size_t(b) * p.dim + d) * kDiagN + 2 * j + pp]
+                                           : 0.f;
             } else {
                 const int prev = unit - G;
                 const uint32_t *flag = p.flags + size_t(prev) * CW + warp;
@@ -407,27 +304,20 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                         atomicOr(p.err, kErrTimeoutCarry);
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        hown[j] = hoth[j] = 0.f;
+                        hv[j] = 0.f;
                 } else {
                     (void)ld_acquire_gpu(flag);
                     // carry layout: [unit][channel][parity][8]
                     const float4 *so = reinterpret_cast<const float4 *>(
                         p.carry + (size_t(prev) * CH + ch) * kDiagN + pp * 8);
-                    const float4 *sx = reinterpret_cast<const float4 *>(
-                        p.carry + (size_t(prev) * CH + (ch ^ 1)) * kDiagN + pp * 8);
                     const float4 o0 = __ldcg(so), o1 = __ldcg(so + 1);
-                    const float4 x0 = __ldcg(sx), x1 = __ldcg(sx + 1);
-                    hown[0] = o0.x; hown[1] = o0.y; hown[2] = o0.z; hown[3] = o0.w;
-                    hown[4] = o1.x; hown[5] = o1.y; hown[6] = o1.z; hown[7] = o1.w;
-                    hoth[0] = x0.x; hoth[1] = x0.y; hoth[2] = x0.z; hoth[3] = x0.w;
-                    hoth[4] = x1.x; hoth[5] = x1.y; hoth[6] = x1.z; hoth[7] = x1.w;
+                    hv[0] = o0.x; hv[1] = o0.y; hv[2] = o0.z; hv[3] = o0.w;
+                    hv[4] = o1.x; hv[5] = o1.y; hv[6] = o1.z; hv[7] = o1.w;
                 }
             }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                gown[jj] = pk2(hown[2 * jj], hown[2 * jj + 1]);
-                goth[jj] = pk2(hoth[2 * jj], hoth[2 * jj + 1]);
-            }
+            for (int jj = 0; jj < 4; ++jj)
+                g[jj] = pk2(hv[2 * jj], hv[2 * jj + 1]);
         }
 
         uint8_t *st = stages + s * Lay::kStage;
@@ -468,74 +358,80 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             constexpr bool POWC = decltype(pow_tag)::value;
 #pragma unroll 1
             for (int j = 0; j < TC / 8; ++j) {
-                const int off = (j ^ swz) << 4;
-                const int tb = t0 + j * 8;
-                const uint4 uq = *reinterpret_cast<const uint4 *>(u_row + off);
-                const uint4 dq = *reinterpret_cast<const uint4 *>(dl_row + off);
-                uint4 zq = make_uint4(0, 0, 0, 0);
+                // this lane prepares tokens 4pp .. 4pp+3 of the 8-token block
+                const int off = ((j ^ swz) << 4) + pp * 8;
+                const uint2 uq = *reinterpret_cast<const uint2 *>(u_row + off);
+                const uint2 dq = *reinterpret_cast<const uint2 *>(dl_row + off);
+                uint2 zq = make_uint2(0, 0);
                 if (GATE)
-                    zq = *reinterpret_cast<const uint4 *>(z_row + off);
-                const int nvalid = p.L - tb;  // tokens of this block inside the sequence
-                uint32_t ypk[4];
-                const float *bcb_blk = bcb + j * 8 * 32;
+                    zq = *reinterpret_cast<const uint2 *>(z_row + off);
+                const int tmine = t0 + j * 8 + pp * 4;
+                float uv[4], rv[4], wv[4], rwv[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    // token-wise prologue for this lane's own channel
-                    const uint32_t uw = (i < 2 ? uq.x : i < 4 ? uq.y : i < 6 ? uq.z : uq.w);
-                    const uint32_t dw = (i < 2 ? dq.x : i < 4 ? dq.y : i < 6 ? dq.z : dq.w);
-                    const float uv = __uint_as_float((i & 1) ? (uw & 0xffff0000u) : (uw << 16));
-                    const float dv = __uint_as_float((i & 1) ? (dw & 0xffff0000u) : (dw << 16));
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t uw = kk < 2 ? uq.x : uq.y, dw = kk < 2 ? dq.x : dq.y;
+                    uv[kk] = __uint_as_float((kk & 1) ? (uw & 0xffff0000u) : (uw << 16));
+                    const float dv = __uint_as_float((kk & 1) ? (dw & 0xffff0000u) : (dw << 16));
                     const float x = dv + bias;
                     float dt = SOFTPLUS ? softplus_fast(x) : x;
-                    dt = (i < nvalid) ? dt : 0.f;  // padding past L: identity step
-                    const float wr = dt * uv;
-                    const float w = copysignf(fmaxf(fabsf(wr), kWMin), wr);
-                    const float r = POWC ? ex2_approx(dt * a0) : dt;
-                    const float c = wprev * rcp_approx(w);
-                    wprev = w;
-                    const float ro = __shfl_xor_sync(0xffffffffu, r, 1);
-                    const float co = __shfl_xor_sync(0xffffffffu, c, 1);
-                    // scan step for this lane's state parity of both channels
-                    const ulonglong2 *bq =
-                        reinterpret_cast<const ulonglong2 *>(bcb_blk + i * 32 + pp * 16);
+                    dt = (tmine + kk < p.L) ? dt : 0.f;  // padding past L: identity step
+                    const float wr = dt * uv[kk];
+                    wv[kk] = copysignf(fmaxf(fabsf(wr), kWMin), wr);
+                    rwv[kk] = rcp_approx(wv[kk]);
+                    rv[kk] = POWC ? ex2_approx(dt * a0) : dt;
+                }
+                // both lanes need r, w, 1/w of all 8 tokens
+                float r8[8], w8[8], rw8[8];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const float ro = __shfl_xor_sync(0xffffffffu, rv[kk], 1);
+                    const float wo = __shfl_xor_sync(0xffffffffu, wv[kk], 1);
+                    const float rwo = __shfl_xor_sync(0xffffffffu, rwv[kk], 1);
+                    r8[kk] = pp ? ro : rv[kk];
+                    r8[4 + kk] = pp ? rv[kk] : ro;
+                    w8[kk] = pp ? wo : wv[kk];
+                    w8[4 + kk] = pp ? wv[kk] : wo;
+                    rw8[kk] = pp ? rwo : rwv[kk];
+                    rw8[4 + kk] = pp ? rwv[kk] : rwo;
+                }
+                float yp[8];
+                const float *bcb_blk = bcb + j * 8 * 32 + pp * 16;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float c = (i == 0 ? wprev : w8[i - 1]) * rw8[i];
+                    const ulonglong2 *bq = reinterpret_cast<const ulonglong2 *>(bcb_blk + i * 32);
                     const ulonglong2 b01 = bq[0], b23 = bq[1], c01 = bq[2], c23 = bq[3];
-                    uint64_t Vo[4], Vx[4];
-                    decay_pairs<POWC>(Vo, r, c, pp, aown);
-                    decay_pairs<POWC>(Vx, ro, co, pp, aoth);
-                    gown[0] = fma2(Vo[0], gown[0], b01.x);
-                    goth[0] = fma2(Vx[0], goth[0], b01.x);
-                    gown[1] = fma2(Vo[1], gown[1], b01.y);
-                    goth[1] = fma2(Vx[1], goth[1], b01.y);
-                    gown[2] = fma2(Vo[2], gown[2], b23.x);
-                    goth[2] = fma2(Vx[2], goth[2], b23.x);
-                    gown[3] = fma2(Vo[3], gown[3], b23.y);
-                    goth[3] = fma2(Vx[3], goth[3], b23.y);
-                    uint64_t Yao = mul2(c01.x, gown[0]);
-                    uint64_t Yax = mul2(c01.x, goth[0]);
-                    uint64_t Ybo = mul2(c01.y, gown[1]);
-                    uint64_t Ybx = mul2(c01.y, goth[1]);
-                    Yao = fma2(c23.x, gown[2], Yao);
-                    Yax = fma2(c23.x, goth[2], Yax);
-                    Ybo = fma2(c23.y, gown[3], Ybo);
-                    Ybx = fma2(c23.y, goth[3], Ybx);
-                    const uint64_t Yo = add2(Yao, Ybo), Yx = add2(Yax, Ybx);
-                    // own channel output: own half + partner's half for this channel
-                    const float part = __shfl_xor_sync(0xffffffffu, lo2(Yx) + hi2(Yx), 1);
-                    float v = (lo2(Yo) + hi2(Yo) + part) * w;
-                    v = fmaf(dsk, uv, v);
+                    uint64_t V[4];
+                    decay_pairs<POWC>(V, r8[i], c, pp, apair);
+                    g[0] = fma2(V[0], g[0], b01.x);
+                    g[1] = fma2(V[1], g[1], b01.y);
+                    g[2] = fma2(V[2], g[2], b23.x);
+                    g[3] = fma2(V[3], g[3], b23.y);
+                    uint64_t Ya = mul2(c01.x, g[0]);
+                    uint64_t Yb = mul2(c01.y, g[1]);
+                    Ya = fma2(c23.x, g[2], Ya);
+                    Yb = fma2(c23.y, g[3], Yb);
+                    const uint64_t Y = add2(Ya, Yb);
+                    yp[i] = lo2(Y) + hi2(Y);
+                }
+                wprev = w8[7];
+                // reduce-scatter: this lane finishes tokens 4pp .. 4pp+3
+                float yo[4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const float send = pp ? yp[kk] : yp[4 + kk];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                    float v = ((pp ? yp[4 + kk] : yp[kk]) + recv) * wv[kk];
+                    v = fmaf(dsk, uv[kk], v);
                     if (GATE) {
-                        const uint32_t zw = (i < 2 ? zq.x : i < 4 ? zq.y : i < 6 ? zq.z : zq.w);
-                        const float zv =
-                            __uint_as_float((i & 1) ? (zw & 0xffff0000u) : (zw << 16));
+                        const uint32_t zw = kk < 2 ? zq.x : zq.y;
+                        const float zv = __uint_as_float((kk & 1) ? (zw & 0xffff0000u) : (zw << 16));
                         v *= silu_fast(zv);
                     }
-                    const uint32_t hv = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
-                    if (i & 1)
-                        ypk[i >> 1] |= hv << 16;
-                    else
-                        ypk[i >> 1] = hv;
+                    yo[kk] = v;
                 }
-                *reinterpret_cast<uint4 *>(y_row + off) = make_uint4(ypk[0], ypk[1], ypk[2], ypk[3]);
+                *reinterpret_cast<uint2 *>(y_row + off) =
+                    make_uint2(pack2_bf16(yo[0], yo[1]), pack2_bf16(yo[2], yo[3]));
             }
         };
         if (pow_path)
@@ -549,50 +445,29 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             mbar_arrive(&empty[s]);
 
         if (inf.z & kInfoLast) {
-            // back to h = w_last * g; the partner's w arrives by shuffle
-            const float wo = __shfl_xor_sync(0xffffffffu, wprev, 1);
-            float hown[8], hoth[8];
+            // back to h = w_last * g; continue from h with w_{-1} := 1
+            float hv[8];
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
-                hown[2 * jj] = lo2(gown[jj]) * wprev;
-                hown[2 * jj + 1] = hi2(gown[jj]) * wprev;
-                hoth[2 * jj] = lo2(goth[jj]) * wo;
-                hoth[2 * jj + 1] = hi2(goth[jj]) * wo;
-            }
-            // continue from h with w_{-1} := 1
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                gown[jj] = pk2(hown[2 * jj], hown[2 * jj + 1]);
-                goth[jj] = pk2(hoth[2 * jj], hoth[2 * jj + 1]);
+                hv[2 * jj] = lo2(g[jj]) * wprev;
+                hv[2 * jj + 1] = hi2(g[jj]) * wprev;
+                g[jj] = pk2(hv[2 * jj], hv[2 * jj + 1]);
             }
             wprev = 1.f;
             if (k < p.num_segs - 1) {
-                // [unit][channel][parity][8]: this lane writes parity pp of both channels
                 float4 *dst = reinterpret_cast<float4 *>(
                     p.carry + (size_t(unit) * CH + ch) * kDiagN + pp * 8);
-                float4 *dsx = reinterpret_cast<float4 *>(
-                    p.carry + (size_t(unit) * CH + (ch ^ 1)) * kDiagN + pp * 8);
-                dst[0] = make_float4(hown[0], hown[1], hown[2], hown[3]);
-                dst[1] = make_float4(hown[4], hown[5], hown[6], hown[7]);
-                dsx[0] = make_float4(hoth[0], hoth[1], hoth[2], hoth[3]);
-                dsx[1] = make_float4(hoth[4], hoth[5], hoth[6], hoth[7]);
+                dst[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+                dst[1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
                 __threadfence();
                 __syncwarp();
                 if (lane == 0 && unit != p.dbg_skip_publish)
                     st_release_gpu(p.flags + size_t(unit) * CW + warp, 1u);
             } else if (p.last_state && d < p.dim) {
-                // natural layout (batch, dim, 16): this lane's parity of its own channel
                 float *dst = p.last_state + (size_t(b) * p.dim + d) * kDiagN;
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    dst[2 * j + pp] = hown[j];
-                const int dpart = d0 + (ch ^ 1);
-                if (dpart < p.dim) {
-                    float *dsx = p.last_state + (size_t(b) * p.dim + dpart) * kDiagN;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        dsx[2 * j + pp] = hoth[j];
-                }
+                    dst[2 * j + pp] = hv[j];
             }
         }
         prev_t0 = inf.y;

@@ -202,8 +202,8 @@ struct DiagVariant<0, T, CH, STAGES, GATE, SOFTPLUS> {
 template <int CH, int STAGES, bool GATE, bool SOFTPLUS>
 struct DiagVariant<1, __nv_bfloat16, CH, STAGES, GATE, SOFTPLUS> {
     static constexpr int kChunk = 64;
-    static constexpr int kThreads = CH + 32;
-    static constexpr int kConsWarps = CH / 32;
+    static constexpr int kThreads = 2 * CH + 32;
+    static constexpr int kConsWarps = 2 * CH / 32;
     static constexpr int kSmem = DiagFastLayout<CH, STAGES, GATE>::kAlloc;
     static constexpr auto kernel() { return scan_diag_bf16_kernel<CH, STAGES, GATE, SOFTPLUS>; }
 };
