@@ -41,7 +41,7 @@ METRIC = "selective-scan Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU"
 # were taken on; reported as roofline.traffic only for that kernel.
 NCU_TRAFFIC = {
     # config 2 captured at L = 2048, scaled by tokens to L = 4096 (see profiles/)
-    2: ("scan_diag_bf16_kernel pairs v3", None),
+    2: ("scan_diag_bf16_kernel pairs v3", 647.2e6),
     4: ("ssd_scalarA_kernel v1", 109.0e6),
 }
 KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v3", 1: "scan_diag_bf16_kernel pairs v3",
