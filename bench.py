@@ -46,7 +46,7 @@ NCU_TRAFFIC = {
 }
 KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v3", 1: "scan_diag_bf16_kernel pairs v3",
               3: "scan_diag_bf16_kernel pairs v3", 0: "scan_diag_kernel fp32 v1",
-              4: "ssd_scalarA_kernel v1"}
+              4: "ssd_scalarA_kernel v2"}
 HBM_FALLBACK_GBS = 6650.0
 
 

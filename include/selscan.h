@@ -102,6 +102,24 @@ SELSCAN_API selscan_status selscan_fwd(const selscan_tensor *u, const selscan_te
                            selscan_tensor *last_state, cudaStream_t stream);
 
 /*
+ * selscan_fwd_h0 -- selscan_fwd continuing from a given state: h_{-1} = h0
+ * instead of zero (chunked prefill, or resuming a sequence from a saved
+ * state; "Mamba-2 y state-space models", section 4.3: the layer keeps a
+ * fixed-size state instead of a KV cache).  h0 (batch, D, N) F32,
+ * contiguous, may be NULL (then identical to selscan_fwd).  h0 may be the
+ * same buffer as last_state (in-place continuation): every channel's initial
+ * state is read before its final state is written.  With L == 0,
+ * last_state = h0.
+ */
+SELSCAN_API selscan_status selscan_fwd_h0(const selscan_tensor *u, const selscan_tensor *delta,
+                              const selscan_tensor *delta_bias, int delta_softplus,
+                              const selscan_tensor *A, const selscan_tensor *B,
+                              const selscan_tensor *C, const selscan_tensor *D,
+                              const selscan_tensor *z, const selscan_tensor *h0,
+                              selscan_tensor *y, selscan_tensor *last_state,
+                              cudaStream_t stream);
+
+/*
  * selscan_fwd_scalarA -- scalar-A (Mamba-2 / SSD) selective scan forward.
  * The transition is one scalar per head times the identity ("Mamba-3: un
  * modelo de espacio de estados centrado en la inferencia", first section),
@@ -135,6 +153,20 @@ SELSCAN_API selscan_status selscan_fwd_scalarA(const selscan_tensor *x,
                                    selscan_tensor *y,
                                    selscan_tensor *last_state,
                                    cudaStream_t stream);
+
+/*
+ * selscan_fwd_scalarA_h0 -- selscan_fwd_scalarA continuing from a given
+ * state h0 (batch, H, P, N) F32, contiguous (may be NULL: zero state; may be
+ * the same buffer as last_state).
+ */
+SELSCAN_API selscan_status selscan_fwd_scalarA_h0(const selscan_tensor *x,
+                                      const selscan_tensor *dt,
+                                      const selscan_tensor *dt_bias, int dt_softplus,
+                                      const selscan_tensor *A, const selscan_tensor *B,
+                                      const selscan_tensor *C, const selscan_tensor *D,
+                                      const selscan_tensor *z, int64_t headdim,
+                                      const selscan_tensor *h0, selscan_tensor *y,
+                                      selscan_tensor *last_state, cudaStream_t stream);
 
 /*
  * selscan_fwd_noalloc -- selscan_fwd for callers that cannot allocate device

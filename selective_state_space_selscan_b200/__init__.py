@@ -27,8 +27,8 @@ STATUS = {
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 # entry points declared in include/selscan.h
-EXPORTS = ("selscan_fwd", "selscan_fwd_scalarA", "selscan_check",
-           "selscan_strerror", "selscan_version")
+EXPORTS = ("selscan_fwd", "selscan_fwd_h0", "selscan_fwd_scalarA", "selscan_fwd_scalarA_h0",
+           "selscan_fwd_noalloc", "selscan_check", "selscan_strerror", "selscan_version")
 
 
 class SelscanError(RuntimeError):
@@ -69,6 +69,12 @@ def lib() -> ctypes.CDLL:
         for f in (L.selscan_fwd, L.selscan_fwd_scalarA, L.selscan_check,
                   L.selscan_version):
             f.restype = ctypes.c_int
+        L.selscan_fwd_h0.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, P, P, P, P,
+                                     ctypes.c_void_p]
+        L.selscan_fwd_h0.restype = ctypes.c_int
+        L.selscan_fwd_scalarA_h0.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, P,
+                                             ctypes.c_int64, P, P, P, ctypes.c_void_p]
+        L.selscan_fwd_scalarA_h0.restype = ctypes.c_int
         L.selscan_fwd_noalloc.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, P, P, P,
                                           ctypes.c_void_p]
         L.selscan_fwd_noalloc.restype = ctypes.c_int
@@ -120,12 +126,13 @@ def _stream_handle(stream):
 
 def selscan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                 delta_softplus=True, out=None, last_state=None,
-                return_last_state=True, stream=None):
+                return_last_state=True, stream=None, h0=None):
     """Diagonal-A selective scan forward through the C ABI.
 
     u, delta, z: (batch, D, L) bf16 or fp32 CUDA tensors (time stride 1);
     A: (D, N=16) fp32; B, C: (batch, N, L) same dtype as u; D, delta_bias:
-    (D,) fp32.  Returns (y, last_state); last_state is None unless requested.
+    (D,) fp32; h0: optional initial state (batch, D, N) fp32 (selscan_fwd_h0).
+    Returns (y, last_state); last_state is None unless requested.
     """
     import torch
     y = out if out is not None else torch.empty_like(u, memory_format=torch.contiguous_format)
@@ -133,13 +140,18 @@ def selscan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
         last_state = torch.empty((u.shape[0], u.shape[1], A.shape[1]),
                                  dtype=torch.float32, device=u.device)
     descs = [describe(t) for t in (u, delta, delta_bias, A, B, C, D, z, y, last_state)]
-    rc = lib().selscan_fwd(_ref(descs[0]), _ref(descs[1]), _ref(descs[2]),
-                           int(bool(delta_softplus)), _ref(descs[3]),
-                           _ref(descs[4]), _ref(descs[5]), _ref(descs[6]),
-                           _ref(descs[7]), _ref(descs[8]), _ref(descs[9]),
-                           _stream_handle(stream))
+    common = (_ref(descs[0]), _ref(descs[1]), _ref(descs[2]), int(bool(delta_softplus)),
+              _ref(descs[3]), _ref(descs[4]), _ref(descs[5]), _ref(descs[6]), _ref(descs[7]))
+    if h0 is None:
+        rc = lib().selscan_fwd(*common, _ref(descs[8]), _ref(descs[9]), _stream_handle(stream))
+        where = "selscan_fwd"
+    else:
+        hd = describe(h0)
+        rc = lib().selscan_fwd_h0(*common, _ref(hd), _ref(descs[8]), _ref(descs[9]),
+                                  _stream_handle(stream))
+        where = "selscan_fwd_h0"
     if rc != 0:
-        raise SelscanError(rc, "selscan_fwd")
+        raise SelscanError(rc, where)
     return y, last_state
 
 
@@ -169,7 +181,7 @@ def selscan_fwd_noalloc(u, delta, A, B, C, out, D=None, z=None, delta_bias=None,
 
 def selscan_fwd_scalarA(x, dt, A, B, C, headdim, D=None, z=None, dt_bias=None,
                         dt_softplus=False, out=None, last_state=None,
-                        return_last_state=True, stream=None):
+                        return_last_state=True, stream=None, h0=None):
     """Scalar-A (Mamba-2 / SSD) scan forward through the C ABI.
 
     x, z: (batch, H*P, L) bf16; dt: (batch, H, L) fp32; A, D, dt_bias: (H,)
@@ -181,13 +193,20 @@ def selscan_fwd_scalarA(x, dt, A, B, C, headdim, D=None, z=None, dt_bias=None,
         last_state = torch.empty((x.shape[0], A.shape[0], headdim, B.shape[2]),
                                  dtype=torch.float32, device=x.device)
     descs = [describe(t) for t in (x, dt, dt_bias, A, B, C, D, z, y, last_state)]
-    rc = lib().selscan_fwd_scalarA(_ref(descs[0]), _ref(descs[1]), _ref(descs[2]),
-                                   int(bool(dt_softplus)), _ref(descs[3]),
-                                   _ref(descs[4]), _ref(descs[5]), _ref(descs[6]),
-                                   _ref(descs[7]), int(headdim), _ref(descs[8]),
-                                   _ref(descs[9]), _stream_handle(stream))
+    common = (_ref(descs[0]), _ref(descs[1]), _ref(descs[2]), int(bool(dt_softplus)),
+              _ref(descs[3]), _ref(descs[4]), _ref(descs[5]), _ref(descs[6]), _ref(descs[7]),
+              int(headdim))
+    if h0 is None:
+        rc = lib().selscan_fwd_scalarA(*common, _ref(descs[8]), _ref(descs[9]),
+                                       _stream_handle(stream))
+        where = "selscan_fwd_scalarA"
+    else:
+        hd = describe(h0)
+        rc = lib().selscan_fwd_scalarA_h0(*common, _ref(hd), _ref(descs[8]), _ref(descs[9]),
+                                          _stream_handle(stream))
+        where = "selscan_fwd_scalarA_h0"
     if rc != 0:
-        raise SelscanError(rc, "selscan_fwd_scalarA")
+        raise SelscanError(rc, where)
     return y, last_state
 
 

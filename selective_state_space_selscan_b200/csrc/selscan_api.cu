@@ -346,12 +346,13 @@ selscan_status selscan_check(cudaStream_t stream)
     return SELSCAN_OK;
 }
 
-selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
-                           const selscan_tensor *delta_bias, int delta_softplus,
-                           const selscan_tensor *A, const selscan_tensor *B,
-                           const selscan_tensor *C, const selscan_tensor *D,
-                           const selscan_tensor *z, selscan_tensor *y,
-                           selscan_tensor *last_state, cudaStream_t stream)
+static selscan_status fwd_impl(const selscan_tensor *u, const selscan_tensor *delta,
+                               const selscan_tensor *delta_bias, int delta_softplus,
+                               const selscan_tensor *A, const selscan_tensor *B,
+                               const selscan_tensor *C, const selscan_tensor *D,
+                               const selscan_tensor *z, const selscan_tensor *h0,
+                               selscan_tensor *y, selscan_tensor *last_state,
+                               cudaStream_t stream)
 {
     // ---- validation (no CUDA call before it passes)
     if (!present(u) || !delta || !A || !B || !C || !y)
@@ -382,6 +383,7 @@ selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
         if ((st = check_param(D, 1, vshape, true)) != SELSCAN_OK) return st;
         const int64_t sshape[3] = {batch, dim, N};
         if ((st = check_param(last_state, 3, sshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(h0, 3, sshape, true)) != SELSCAN_OK) return st;
     }
     for (const selscan_tensor *t : {B, C}) {
         if (!present(t))
@@ -409,11 +411,16 @@ selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
     if (batch == 0 || dim == 0)
         return SELSCAN_OK;
     if (L == 0) {
-        if (last_state && last_state->data)
-            return cudaMemsetAsync(last_state->data, 0, size_t(batch * dim * N) * 4, stream) ==
-                           cudaSuccess
-                       ? SELSCAN_OK
-                       : SELSCAN_ERR_CUDA;
+        // nothing to scan: the final state is the initial one (zero if none)
+        if (last_state && last_state->data) {
+            const size_t bytes = size_t(batch * dim * N) * 4;
+            const cudaError_t e =
+                (h0 && h0->data)
+                    ? cudaMemcpyAsync(last_state->data, h0->data, bytes, cudaMemcpyDeviceToDevice,
+                                      stream)
+                    : cudaMemsetAsync(last_state->data, 0, bytes, stream);
+            return e == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+        }
         return SELSCAN_OK;
     }
 
@@ -429,7 +436,7 @@ selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
     prm.A = static_cast<const float *>(A->data);
     prm.delta_bias = static_cast<const float *>(opt_data(delta_bias));
     prm.Dskip = static_cast<const float *>(opt_data(D));
-    prm.h0 = nullptr;
+    prm.h0 = static_cast<const float *>(opt_data(h0));
     prm.last_state = static_cast<float *>(last_state ? last_state->data : nullptr);
     prm.softplus = delta_softplus ? 1 : 0;
     prm.timeout_ns = default_timeout_ns();
@@ -450,11 +457,34 @@ selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
                 : launch_diag<0, float, 64, 4, false, true>(u, delta, B, C, z, y, prm, sms, stream);
 }
 
-selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor *dt,
+selscan_status selscan_fwd(const selscan_tensor *u, const selscan_tensor *delta,
+                           const selscan_tensor *delta_bias, int delta_softplus,
+                           const selscan_tensor *A, const selscan_tensor *B,
+                           const selscan_tensor *C, const selscan_tensor *D,
+                           const selscan_tensor *z, selscan_tensor *y,
+                           selscan_tensor *last_state, cudaStream_t stream)
+{
+    return fwd_impl(u, delta, delta_bias, delta_softplus, A, B, C, D, z, nullptr, y, last_state,
+                    stream);
+}
+
+selscan_status selscan_fwd_h0(const selscan_tensor *u, const selscan_tensor *delta,
+                              const selscan_tensor *delta_bias, int delta_softplus,
+                              const selscan_tensor *A, const selscan_tensor *B,
+                              const selscan_tensor *C, const selscan_tensor *D,
+                              const selscan_tensor *z, const selscan_tensor *h0,
+                              selscan_tensor *y, selscan_tensor *last_state, cudaStream_t stream)
+{
+    return fwd_impl(u, delta, delta_bias, delta_softplus, A, B, C, D, z, h0, y, last_state,
+                    stream);
+}
+
+static selscan_status scalarA_impl(const selscan_tensor *x, const selscan_tensor *dt,
                                    const selscan_tensor *dt_bias, int dt_softplus,
                                    const selscan_tensor *A, const selscan_tensor *B,
                                    const selscan_tensor *C, const selscan_tensor *D,
-                                   const selscan_tensor *z, int64_t headdim, selscan_tensor *y,
+                                   const selscan_tensor *z, int64_t headdim,
+                                   const selscan_tensor *h0, selscan_tensor *y,
                                    selscan_tensor *last_state, cudaStream_t stream)
 {
     if (!present(x) || !dt || !A || !B || !C || !y)
@@ -502,6 +532,7 @@ selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor
         if ((st = check_param(D, 1, hshape, true)) != SELSCAN_OK) return st;
         const int64_t sshape[4] = {batch, H, headdim, N};
         if ((st = check_param(last_state, 4, sshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(h0, 4, sshape, true)) != SELSCAN_OK) return st;
     }
     if (N != kSsdN || headdim != kSsdP || G != 1)
         return SELSCAN_ERR_UNSUPPORTED;
@@ -510,11 +541,15 @@ selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor
     if (batch == 0)
         return SELSCAN_OK;
     if (L == 0) {
-        if (last_state && last_state->data)
-            return cudaMemsetAsync(last_state->data, 0,
-                                   size_t(batch * H * headdim * N) * 4, stream) == cudaSuccess
-                       ? SELSCAN_OK
-                       : SELSCAN_ERR_CUDA;
+        if (last_state && last_state->data) {
+            const size_t bytes = size_t(batch * H * headdim * N) * 4;
+            const cudaError_t e =
+                (h0 && h0->data)
+                    ? cudaMemcpyAsync(last_state->data, h0->data, bytes, cudaMemcpyDeviceToDevice,
+                                      stream)
+                    : cudaMemsetAsync(last_state->data, 0, bytes, stream);
+            return e == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+        }
         return SELSCAN_OK;
     }
     int dev = 0;
@@ -551,6 +586,7 @@ selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor
     prm.y_bs = y->stride[0];
     prm.y_cs = y->stride[1];
     prm.last_state = static_cast<float *>(last_state ? last_state->data : nullptr);
+    prm.h0 = static_cast<const float *>(opt_data(h0));
     prm.timeout_ns = default_timeout_ns();
     prm.err = di->err;
 
@@ -565,8 +601,31 @@ selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor
     const int64_t grid = batch * H;
     if (grid > 0x7fffffffll)
         return SELSCAN_ERR_UNSUPPORTED;
-    kern<<<unsigned(grid), 128, SsdLayout::kAlloc, stream>>>(tm_C, tm_B, tm_X, prm);
+    kern<<<unsigned(grid), 256, SsdLayout::kAlloc, stream>>>(tm_C, tm_B, tm_X, prm);
     return cudaGetLastError() == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+}
+
+selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor *dt,
+                                   const selscan_tensor *dt_bias, int dt_softplus,
+                                   const selscan_tensor *A, const selscan_tensor *B,
+                                   const selscan_tensor *C, const selscan_tensor *D,
+                                   const selscan_tensor *z, int64_t headdim, selscan_tensor *y,
+                                   selscan_tensor *last_state, cudaStream_t stream)
+{
+    return scalarA_impl(x, dt, dt_bias, dt_softplus, A, B, C, D, z, headdim, nullptr, y,
+                        last_state, stream);
+}
+
+selscan_status selscan_fwd_scalarA_h0(const selscan_tensor *x, const selscan_tensor *dt,
+                                      const selscan_tensor *dt_bias, int dt_softplus,
+                                      const selscan_tensor *A, const selscan_tensor *B,
+                                      const selscan_tensor *C, const selscan_tensor *D,
+                                      const selscan_tensor *z, int64_t headdim,
+                                      const selscan_tensor *h0, selscan_tensor *y,
+                                      selscan_tensor *last_state, cudaStream_t stream)
+{
+    return scalarA_impl(x, dt, dt_bias, dt_softplus, A, B, C, D, z, headdim, h0, y, last_state,
+                        stream);
 }
 
 }  // extern "C"

@@ -57,14 +57,15 @@ struct SsdParams {
     __nv_bfloat16 *y;          // (batch, H*P, L)
     int64_t y_bs, y_cs;
     float *last_state;         // (batch, H, P, N) or null
+    const float *h0;           // (batch, H, P, N) or null: initial state
     unsigned long long timeout_ns;
     unsigned int *err;
 };
 
 struct SsdLayout {
-    static constexpr int kC = 0;                   // [2 slabs][128 n][64 t]
-    static constexpr int kB = kC + 32768;          // [2 slabs][128 n][64 s]
-    static constexpr int kX = kB + 32768;          // 2 buffers x [2 slabs][64 p][64 s]
+    static constexpr int kC = 0;                   // 2 buffers x [2 slabs][128 n][64 t]
+    static constexpr int kB = kC + 2 * 32768;      // 2 buffers x [2 slabs][128 n][64 s]
+    static constexpr int kX = kB + 2 * 32768;      // 2 buffers x [2 slabs][64 p][64 s]
     static constexpr int kXw = kX + 2 * 16384;     // [2 slabs][64 p][64 s]
     static constexpr int kM = kXw + 16384;         // [2 slabs][128 t][64 s]
     static constexpr int kHs = kM + 32768;         // [128 n][64 p]
@@ -87,7 +88,7 @@ __device__ __forceinline__ float ssd_softplus(float x)
 }
 
 template <bool GATE>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                    const __grid_constant__ CUtensorMap tm_B,
                    const __grid_constant__ CUtensorMap tm_X, const SsdParams p)
@@ -98,21 +99,25 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ float s_delta[Q], s_S[Q], s_g[Q], s_wsum[4];
-    __shared__ uint64_t bar_tma, bar_mma;
+    __shared__ uint64_t bar_tma[2], bar_g, bar_yo, bar_mma;
     __shared__ uint32_t s_tbase;
 
+    // Two threads per row: r = row / token / state index, half = which half of
+    // the columns this thread handles.  Warp w reaches TMEM lanes 32*(w%4).
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = tid & 127, half = tid >> 7;
     const int b = blockIdx.x / p.H, hh = blockIdx.x - b * p.H;
-    const float a_nat = p.A[hh];
-    const float a_l2 = a_nat * 1.4426950408889634f;  // A in log2 units
+    const float a_l2 = p.A[hh] * 1.4426950408889634f;  // A in log2 units
     const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
     const float dsk = p.Dskip ? p.Dskip[hh] : 0.f;
     const uint32_t sbase = smem_addr(smem);
-    const uint32_t aC = sbase + Lay::kC, aB = sbase + Lay::kB, aXw = sbase + Lay::kXw;
-    const uint32_t aM = sbase + Lay::kM, aHs = sbase + Lay::kHs;
+    const uint32_t aXw = sbase + Lay::kXw, aM = sbase + Lay::kM, aHs = sbase + Lay::kHs;
 
     if (tid == 0) {
-        mbar_init(&bar_tma, 1);
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
+        mbar_init(&bar_g, 1);
+        mbar_init(&bar_yo, 1);
         mbar_init(&bar_mma, 1);
         fence_mbar_init();
         prefetch_tmap(&tm_C);
@@ -121,54 +126,101 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
     }
     if (warp == 0)
         tmem_alloc(&s_tbase, kSsdTmemCols);
-    // zero the bf16 copy of h_prev (row tid = state n)
+    // initial state h[n][p] (zero unless given): this thread's row n = r,
+    // columns p of its half; kept in fp32 for TMEM and in bf16 for C^T h
+    float h_init[32];
     {
-        uint4 *row = reinterpret_cast<uint4 *>(smem + Lay::kHs + tid * 128);
+        const float *h0row = p.h0 ? p.h0 + (int64_t(b) * p.H + hh) * P * N + r : nullptr;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            row[i] = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 32; ++i)
+            h_init[i] = h0row ? h0row[int64_t(half * 32 + i) * N] : 0.f;
+        uint8_t *hs = smem + Lay::kHs;
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+            uint4 pk;
+            pk.x = ssd_pack2(h_init[g8 * 8 + 0], h_init[g8 * 8 + 1]);
+            pk.y = ssd_pack2(h_init[g8 * 8 + 2], h_init[g8 * 8 + 3]);
+            pk.z = ssd_pack2(h_init[g8 * 8 + 4], h_init[g8 * 8 + 5]);
+            pk.w = ssd_pack2(h_init[g8 * 8 + 6], h_init[g8 * 8 + 7]);
+            *reinterpret_cast<uint4 *>(hs + sw128_offset(r, half * 32 + g8 * 8)) = pk;
+        }
     }
     fence_proxy_async_smem();
     tmem_fence_before_sync();
     __syncthreads();
     tmem_fence_after_sync();
     const uint32_t tb = s_tbase;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;  // this warp's TMEM lanes
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;  // this warp's TMEM lanes
+    const uint32_t colh = uint32_t(half * 32);                   // this thread's column half
     {
-        // h = 0 (the scan starts from the zero state)
-        float zero[16];
+        float v0[16], v1[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            zero[i] = 0.f;
-#pragma unroll
-        for (int c = 0; c < P; c += 16)
-            tmem_st16(tb + lane_off + kColH + c, zero);
+        for (int i = 0; i < 16; ++i) {
+            v0[i] = h_init[i];
+            v1[i] = h_init[16 + i];
+        }
+        tmem_st16(tb + lane_off + kColH + colh, v0);
+        tmem_st16(tb + lane_off + kColH + colh + 16, v1);
     }
 
     const float *dt_row = p.dt + int64_t(b) * p.dt_bs + int64_t(hh) * p.dt_hs;
-    bool ok = true;
-    auto issue_loads = [&](int c, int xb) {
-        const int t0 = c * Q;
-        mbar_arrive_expect_tx(&bar_tma, 32768 + 32768 + 16384);
-        tma_load_3d(smem + Lay::kC, &tm_C, &bar_tma, t0, 0, b);
-        tma_load_3d(smem + Lay::kC + 16384, &tm_C, &bar_tma, t0 + 64, 0, b);
-        tma_load_3d(smem + Lay::kB, &tm_B, &bar_tma, t0, 0, b);
-        tma_load_3d(smem + Lay::kB + 16384, &tm_B, &bar_tma, t0 + 64, 0, b);
-        uint8_t *xs = smem + Lay::kX + xb * 16384;
-        tma_load_3d(xs, &tm_X, &bar_tma, t0, hh * P, b);
-        tma_load_3d(xs + 8192, &tm_X, &bar_tma, t0 + 64, hh * P, b);
+    auto issue_loads = [&](int c) {
+        const int t0 = c * Q, buf = c & 1;
+        mbar_arrive_expect_tx(&bar_tma[buf], 32768 + 32768 + 16384);
+        uint8_t *cs = smem + Lay::kC + buf * 32768;
+        uint8_t *bs = smem + Lay::kB + buf * 32768;
+        uint8_t *xs = smem + Lay::kX + buf * 16384;
+        tma_load_3d(cs, &tm_C, &bar_tma[buf], t0, 0, b);
+        tma_load_3d(cs + 16384, &tm_C, &bar_tma[buf], t0 + 64, 0, b);
+        tma_load_3d(bs, &tm_B, &bar_tma[buf], t0, 0, b);
+        tma_load_3d(bs + 16384, &tm_B, &bar_tma[buf], t0 + 64, 0, b);
+        tma_load_3d(xs, &tm_X, &bar_tma[buf], t0, hh * P, b);
+        tma_load_3d(xs + 8192, &tm_X, &bar_tma[buf], t0 + 64, hh * P, b);
     };
-    if (tid == 0)
-        issue_loads(0, 0);
-    float dt_next = (tid < p.L) ? dt_row[tid] : 0.f;
-    uint32_t mma_phase = 0;
+    constexpr uint32_t idG = umma_idesc_bf16(128, 128, true, true);
+    constexpr uint32_t idYo = umma_idesc_bf16(128, 64, true, true);
+    constexpr uint32_t idYd = umma_idesc_bf16(128, 64, false, false);
+    auto issue_G = [&](int c) {
+        const uint32_t aC = sbase + Lay::kC + (c & 1) * 32768;
+        const uint32_t aB = sbase + Lay::kB + (c & 1) * 32768;
+#pragma unroll
+        for (int kk = 0; kk < N / 16; ++kk)
+            umma_bf16(tb + kColG, umma_desc_mnmajor(aC, N, kk), umma_desc_mnmajor(aB, N, kk),
+                      idG, kk > 0);
+        umma_commit(&bar_g);
+    };
+    bool ok = true;
+    if (tid == 0) {
+        issue_loads(0);
+        if (p.nchunks > 1)
+            issue_loads(1);
+        ok = mbar_wait(&bar_tma[0], 0u, p.timeout_ns) && ok;
+        tmem_fence_after_sync();
+        issue_G(0);
+    }
+    float dt_next = (half == 0 && r < p.L) ? dt_row[r] : 0.f;
 
     for (int c = 0; c < p.nchunks; ++c) {
-        const int xb = c & 1;
+        const int buf = c & 1;
+        const uint32_t ph = uint32_t(c & 1);        // bar_g / bar_yo / bar_mma phase
+        const uint32_t tph = uint32_t((c >> 1) & 1);  // bar_tma[buf] phase
         const int t0 = c * Q;
-        const int t = tid;  // this thread's token / row / state index
-        const bool valid = t0 + t < p.L;
-        // ---- step sizes and their cumulative sum over the chunk
+        const uint32_t aC = sbase + Lay::kC + buf * 32768;
+        const uint32_t aB = sbase + Lay::kB + buf * 32768;
+        const uint32_t aX = sbase + Lay::kX + buf * 16384;
+        // ---- carried-in term Yo = C^T h_prev (h_prev in bf16 from the last chunk)
+        if (tid == 0) {
+            if (c > 0)
+                ok = mbar_wait(&bar_tma[buf], tph, p.timeout_ns) && ok;
+            tmem_fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < N / 16; ++kk)
+                umma_bf16(tb + kColYo, umma_desc_mnmajor(aC, N, kk),
+                          umma_desc_mnmajor(aHs, N, kk), idYo, kk > 0);
+            umma_commit(&bar_yo);
+        }
+        // ---- step sizes and their cumulative sum over the chunk (first 128 threads)
+        const bool valid = t0 + r < p.L;
         float dl = dt_next + bias;
         if (p.softplus)
             dl = ssd_softplus(dl);
@@ -180,88 +232,75 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
             if (lane >= o)
                 S += v;
         }
-        if (lane == 31)
+        if (half == 0 && lane == 31)
             s_wsum[warp] = S;
         __syncthreads();
-        for (int w = 0; w < warp; ++w)
+        for (int w = 0; w < (warp & 3); ++w)
             S += s_wsum[w];
-        s_delta[t] = dl;
-        s_S[t] = S;
+        if (half == 0) {
+            s_delta[r] = dl;
+            s_S[r] = S;
+        }
         __syncthreads();
+        S = s_S[r];
+        dl = s_delta[r];
         const float S_end = s_S[Q - 1];
-        // column factor of the cross-block mask: exp(A (S_blockend - S_s)) delta_s
-        s_g[t] = ex2_approx(a_l2 * (s_S[(t | 31)] - S)) * dl;
-        __syncthreads();
+        if (half == 0)
+            s_g[r] = ex2_approx(a_l2 * (s_S[(r | 31)] - S)) * dl;
         const float w_state = ex2_approx(a_l2 * (S_end - S)) * dl;  // x scale for h
         const float e_row = ex2_approx(a_l2 * S);                     // Yo row scale
-        if (c + 1 < p.nchunks)
-            dt_next = (t0 + Q + t < p.L) ? dt_row[t0 + Q + t] : 0.f;
-
-        // ---- chunk inputs
-        ok = mbar_wait(&bar_tma, uint32_t(c & 1), p.timeout_ns) && ok;
-        // ---- G = C^T B and Yo = C^T h_prev on the tensor cores
-        if (tid == 0) {
-            tmem_fence_after_sync();
-            constexpr uint32_t idG = umma_idesc_bf16(128, 128, true, true);
-            constexpr uint32_t idYo = umma_idesc_bf16(128, 64, true, true);
-#pragma unroll
-            for (int kk = 0; kk < N / 16; ++kk)
-                umma_bf16(tb + kColG, umma_desc_mnmajor(aC, N, kk), umma_desc_mnmajor(aB, N, kk),
-                          idG, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < N / 16; ++kk)
-                umma_bf16(tb + kColYo, umma_desc_mnmajor(aC, N, kk),
-                          umma_desc_mnmajor(aHs, N, kk), idYo, kk > 0);
-            umma_commit(&bar_mma);
-        }
-        // ---- meanwhile: x * w for the state product, and h *= exp(A S_end)
+        if (half == 0 && c + 1 < p.nchunks)
+            dt_next = (t0 + Q + r < p.L) ? dt_row[t0 + Q + r] : 0.f;
+        __syncthreads();
+        // every thread reads this chunk's x below
+        ok = mbar_wait(&bar_tma[buf], tph, p.timeout_ns) && ok;
+        // ---- x * w for the state product (rows p of this half), h *= exp(A S_end)
         {
-            const uint8_t *xs = smem + Lay::kX + xb * 16384;
+            const uint8_t *xs = smem + Lay::kX + buf * 16384;
             uint8_t *xw = smem + Lay::kXw;
-            const uint32_t slab = uint32_t(t >> 6) * 8192u;
-#pragma unroll 8
-            for (int pp = 0; pp < P; ++pp) {
-                const uint32_t off = slab + sw128_offset(pp, t & 63);
+            const uint32_t slab = uint32_t(r >> 6) * 8192u;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int pp = half * 32 + i;
+                const uint32_t off = slab + sw128_offset(pp, r & 63);
                 const float xv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xs + off));
                 *reinterpret_cast<__nv_bfloat16 *>(xw + off) = __float2bfloat16_rn(xv * w_state);
             }
             const float dec = ex2_approx(a_l2 * S_end);
 #pragma unroll
-            for (int cc = 0; cc < P; cc += 16) {
+            for (int cc = 0; cc < 32; cc += 16) {
                 float v[16];
-                tmem_ld16(tb + lane_off + kColH + cc, v);
+                tmem_ld16(tb + lane_off + kColH + colh + cc, v);
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     v[i] *= dec;
-                tmem_st16(tb + lane_off + kColH + cc, v);
+                tmem_st16(tb + lane_off + kColH + colh + cc, v);
             }
         }
-        // ---- M = G masked by the decays (row t = this thread)
-        ok = mbar_wait(&bar_mma, mma_phase, p.timeout_ns) && ok;
-        mma_phase ^= 1u;
+        // ---- M = G masked by the decays: row t = r, pieces 4*half .. 4*half+3
+        ok = mbar_wait(&bar_g, ph, p.timeout_ns) && ok;
         tmem_fence_after_sync();
         {
-            const int bi = warp;  // 32-token block of this row
-            float fr[4];          // exp(A (S_t - S_{end of block j})) for blocks j < bi
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                fr[j] = (j < bi) ? ex2_approx(a_l2 * (S - s_S[32 * j + 31])) : 0.f;
+            const int bi = warp & 3;  // 32-token block of this row
             uint8_t *mrow = smem + Lay::kM;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {  // 16-column pieces of the row
+            for (int qq = 0; qq < 4; ++qq) {
+                const int q = half * 4 + qq;  // 16-column piece of the row
                 float m[16];
-                if (q < 2 * (bi + 1)) {    // warp-uniform
-                    float g[16];
-                    tmem_ld16(tb + lane_off + kColG + q * 16, g);
+                if (q < 2 * (bi + 1)) {       // warp-uniform
+                    float gv[16];
+                    tmem_ld16(tb + lane_off + kColG + q * 16, gv);
                     const int bj = q >> 1;
+                    // exp(A (S_t - S_{end of block bj})) for a block before this row's
+                    const float fr = (bj < bi) ? ex2_approx(a_l2 * (S - s_S[32 * bj + 31])) : 0.f;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int s = q * 16 + i;
                         float v;
                         if (bj < bi)
-                            v = g[i] * fr[bj] * s_g[s];
+                            v = gv[i] * fr * s_g[s];
                         else
-                            v = (s <= t) ? g[i] * ex2_approx(a_l2 * (S - s_S[s])) * s_delta[s]
+                            v = (s <= r) ? gv[i] * ex2_approx(a_l2 * (S - s_S[s])) * s_delta[s]
                                          : 0.f;
                         m[i] = v;
                     }
@@ -270,7 +309,6 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                     for (int i = 0; i < 16; ++i)
                         m[i] = 0.f;
                 }
-                // 16 bf16 = two 16-byte chunks of row t in slab q/4
                 const uint32_t slab = uint32_t(q >> 2) * 16384u;
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -280,18 +318,16 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                     pk.y = ssd_pack2(m[h2 * 8 + 2], m[h2 * 8 + 3]);
                     pk.z = ssd_pack2(m[h2 * 8 + 4], m[h2 * 8 + 5]);
                     pk.w = ssd_pack2(m[h2 * 8 + 6], m[h2 * 8 + 7]);
-                    *reinterpret_cast<uint4 *>(mrow + slab + sw128_offset(t, col)) = pk;
+                    *reinterpret_cast<uint4 *>(mrow + slab + sw128_offset(r, col)) = pk;
                 }
             }
         }
         fence_proxy_async_smem();
         tmem_fence_before_sync();
         __syncthreads();
-        // ---- Yd = M x^T and h += B (x w)^T
+        // ---- Yd = M x^T, h += B (x w)^T, then the next chunk's C^T B
         if (tid == 0) {
             tmem_fence_after_sync();
-            constexpr uint32_t idYd = umma_idesc_bf16(128, 64, false, false);
-            const uint32_t aX = sbase + Lay::kX + xb * 16384;
 #pragma unroll
             for (int kk = 0; kk < Q / 16; ++kk)
                 umma_bf16(tb + kColYd, umma_desc_kmajor(aM, 128, kk), umma_desc_kmajor(aX, P, kk),
@@ -301,32 +337,32 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                 umma_bf16(tb + kColH, umma_desc_kmajor(aB, N, kk), umma_desc_kmajor(aXw, P, kk),
                           idYd, 1u);
             umma_commit(&bar_mma);
+            if (c + 1 < p.nchunks) {
+                ok = mbar_wait(&bar_tma[buf ^ 1], uint32_t(((c + 1) >> 1) & 1), p.timeout_ns) && ok;
+                tmem_fence_after_sync();
+                issue_G(c + 1);
+            }
         }
-        ok = mbar_wait(&bar_mma, mma_phase, p.timeout_ns) && ok;
-        mma_phase ^= 1u;
+        ok = mbar_wait(&bar_yo, ph, p.timeout_ns) && ok;
+        ok = mbar_wait(&bar_mma, ph, p.timeout_ns) && ok;
         tmem_fence_after_sync();
-        // C and B are free now: bring the next chunk in while the epilogue runs
-        if (tid == 0 && c + 1 < p.nchunks) {
-            fence_proxy_async_smem();
-            issue_loads(c + 1, xb ^ 1);
-        }
-        // ---- outputs of token t: y[p, t] = Yd + e_t Yo + D x
+        // ---- outputs of token t = r, columns p of this half
         {
-            const uint8_t *xs = smem + Lay::kX + xb * 16384;
-            const uint32_t slab = uint32_t(t >> 6) * 8192u;
-            __nv_bfloat16 *yrow = p.y + int64_t(b) * p.y_bs + int64_t(hh * P) * p.y_cs + t0 + t;
+            const uint8_t *xs = smem + Lay::kX + buf * 16384;
+            const uint32_t slab = uint32_t(r >> 6) * 8192u;
+            __nv_bfloat16 *yrow = p.y + int64_t(b) * p.y_bs + int64_t(hh * P) * p.y_cs + t0 + r;
             const __nv_bfloat16 *zrow =
-                GATE ? p.z + int64_t(b) * p.z_bs + int64_t(hh * P) * p.z_cs + t0 + t : nullptr;
+                GATE ? p.z + int64_t(b) * p.z_bs + int64_t(hh * P) * p.z_cs + t0 + r : nullptr;
 #pragma unroll
-            for (int cc = 0; cc < P; cc += 16) {
+            for (int cc = 0; cc < 32; cc += 16) {
                 float yd[16], yo[16];
-                tmem_ld16(tb + lane_off + kColYd + cc, yd);
-                tmem_ld16(tb + lane_off + kColYo + cc, yo);
+                tmem_ld16(tb + lane_off + kColYd + colh + cc, yd);
+                tmem_ld16(tb + lane_off + kColYo + colh + cc, yo);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int pp = cc + i;
+                    const int pp = half * 32 + cc + i;
                     const float xv = __bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16 *>(xs + slab + sw128_offset(pp, t & 63)));
+                        *reinterpret_cast<const __nv_bfloat16 *>(xs + slab + sw128_offset(pp, r & 63)));
                     float v = fmaf(e_row, yo[i], yd[i]);
                     v = fmaf(dsk, xv, v);
                     if (GATE && valid) {
@@ -337,15 +373,15 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                         yrow[int64_t(pp) * p.y_cs] = __float2bfloat16_rn(v);
                 }
             }
-            // h (state n = t) -> bf16 copy for the next chunk's Yo; final state out
+            // h (state n = r) -> bf16 copy for the next chunk's Yo; final state out
             uint8_t *hs = smem + Lay::kHs;
             float *ls = (p.last_state && c == p.nchunks - 1)
-                            ? p.last_state + (int64_t(b) * p.H + hh) * P * N + t
+                            ? p.last_state + (int64_t(b) * p.H + hh) * P * N + r
                             : nullptr;
 #pragma unroll
-            for (int cc = 0; cc < P; cc += 16) {
+            for (int cc = 0; cc < 32; cc += 16) {
                 float hv[16];
-                tmem_ld16(tb + lane_off + kColH + cc, hv);
+                tmem_ld16(tb + lane_off + kColH + colh + cc, hv);
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     uint4 pk;
@@ -353,20 +389,25 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                     pk.y = ssd_pack2(hv[h2 * 8 + 2], hv[h2 * 8 + 3]);
                     pk.z = ssd_pack2(hv[h2 * 8 + 4], hv[h2 * 8 + 5]);
                     pk.w = ssd_pack2(hv[h2 * 8 + 6], hv[h2 * 8 + 7]);
-                    *reinterpret_cast<uint4 *>(hs + sw128_offset(t, cc + h2 * 8)) = pk;
+                    *reinterpret_cast<uint4 *>(hs + sw128_offset(r, colh + cc + h2 * 8)) = pk;
                 }
                 if (ls) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        ls[int64_t(cc + i) * N] = hv[i];
+                        ls[int64_t(colh + cc + i) * N] = hv[i];
                 }
             }
         }
         fence_proxy_async_smem();
         tmem_fence_before_sync();
         __syncthreads();
+        // this chunk's C, B, x buffers are free: bring in chunk c + 2
+        if (tid == 0 && c + 2 < p.nchunks) {
+            fence_proxy_async_smem();
+            issue_loads(c + 2);
+        }
     }
-    if (!ok && tid == 0)
+    if (!ok)
         atomicOr(p.err, 4u);
     tmem_fence_after_sync();
     if (warp == 0)
