@@ -205,6 +205,9 @@ def run_reference(args, rank: int, world: int):
     """Reference arm: the fp64 oracle on the host cores (rank 0 only)."""
     if rank != 0:
         return
+    if args.op == "step":
+        run_reference_step(args, world)
+        return
     cfg = synthetic.CONFIGS[args.config]
     inp = synthetic.make_config(args.config)
     import oracle
@@ -252,6 +255,50 @@ def run_reference(args, rank: int, world: int):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_reference_step(args, world: int):
+    """Reference arm of ``--op step``: the oracle's decode step, each timed
+    step a bounded sample of batch rows of the same workload."""
+    base = synthetic.CONFIGS[args.config]
+    batch = args.batch or STEP_BATCH[base["kind"]]
+    cfg = step_workload(base, batch)
+    rows = min(batch, 8)  # rows per timed step
+    if cfg["kind"] == "diag":
+        inp = synthetic.make_diag(rows, cfg["dim"], cfg["N"], 1, dtype=cfg["dtype"],
+                                  seed=cfg["seed"], gate=cfg["gate"], D=cfg["D"])
+        shape = (rows, cfg["dim"], cfg["N"])
+    else:
+        inp = synthetic.make_scalarA(rows, cfg["nheads"], cfg["headdim"], cfg["N"], 1,
+                                     ngroups=cfg["ngroups"], dtype=cfg["dtype"],
+                                     seed=cfg["seed"], gate=cfg["gate"])
+        shape = (rows, cfg["nheads"], cfg["headdim"], cfg["N"])
+    state = np.random.default_rng(cfg["seed"] + 1000).standard_normal(shape, dtype=np.float32)
+    one = lambda: oracle_step_sample(dict(cfg, batch=rows), inp, state, seconds=0.0)
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(args.steps):
+        one()
+        done += 1
+        if time.perf_counter() - t0 > 150.0:
+            break
+    dt = time.perf_counter() - t0
+    val = done * rows / dt
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "selective-scan decode step, tokens/s (one token per batch row) and % of "
+                  "B200 HBM roofline, 1 GPU",
+        "value": val, "unit": "tokens/s", "n_gpus": world, "steps": done,
+        "warmup": args.warmup, "ms_per_step": dt / done * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": step_name(cfg), "sample_per_step": f"{rows} batch rows"},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{done} steps x {rows} batch rows"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
 
 
 # ------------------------------------------------------------ GPU arm
@@ -424,6 +471,227 @@ def run_gpu(args, rank: int, world: int, local: int):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ decode step
+STEP_BATCH = {"diag": 1024, "scalarA": 512}  # state 336 / 537 MB, far above L2
+# DRAM bytes per launch of the decode step at the default batch (ncu capture
+# summarised in profiles/step_kernel_decode.md), keyed by config
+STEP_NCU_TRAFFIC = {2: ("step_kernel v2", 660.0e6), 4: ("step_kernel v2", 1019.7e6)}
+STEP_KERNEL_TAG = "step_kernel v2"
+
+
+def step_workload(cfg: dict, batch: int) -> dict:
+    """The decode step of a config's layer: one token for ``batch`` rows."""
+    return dict(cfg, batch=batch, L=1)
+
+
+def step_name(cfg: dict) -> str:
+    if cfg["kind"] == "diag":
+        shape = f"D{cfg['dim']} N{cfg['N']}"
+    else:
+        shape = f"H{cfg['nheads']} P{cfg['headdim']} N{cfg['N']} G{cfg['ngroups']}"
+    extra = (", gate" if cfg["gate"] else "") + (", D skip" if cfg.get("D") else "")
+    return f"{cfg['kind']} decode step ({shape}, {cfg['dtype']}{extra}), batch {cfg['batch']}"
+
+
+def step_bytes(cfg: dict) -> int:
+    """Bytes one decode step must move: the fp32 state read and written, the
+    token's inputs and y, B and C, and the per-channel parameters."""
+    es = 2 if cfg["dtype"] == "bf16" else 4
+    b = cfg["batch"]
+    if cfg["kind"] == "diag":
+        dim, N, units = cfg["dim"], cfg["N"], cfg["dim"]
+        tok = b * dim * es * (4 if cfg["gate"] else 3)           # u, delta, (z), y
+        params = dim * N * 4 + units * 4 * (2 if cfg["D"] else 1)
+        bc = 2 * b * N * es
+    else:
+        units, P, N = cfg["nheads"], cfg["headdim"], cfg["N"]
+        dim = units * P
+        tok = b * dim * es * (3 if cfg["gate"] else 2) + b * units * 4  # x, (z), y, dt
+        params = units * 4 * 2
+        bc = 2 * b * cfg["ngroups"] * N * es
+    return b * dim * N * 4 * 2 + tok + bc + params
+
+
+def run_step(args, rank: int, world: int, local: int):
+    """Decode-step arm (``--op step``): selscan_step / selscan_step_scalarA
+    on the config's layer with ``--batch`` rows (default 512 diagonal, 256
+    scalar), the state resident on the device and updated in place."""
+    import torch
+    import selective_state_space_selscan_b200 as ss
+    torch.cuda.set_device(local)
+    base = synthetic.CONFIGS[args.config]
+    batch = args.batch or STEP_BATCH[base["kind"]]
+    cfg = step_workload(base, batch)
+    dt = cfg["dtype"]
+    stream = torch.cuda.current_stream()
+    rng = np.random.default_rng(cfg["seed"] + 1000 + rank)
+    if cfg["kind"] == "diag":
+        inp = synthetic.make_diag(batch, cfg["dim"], cfg["N"], 1, dtype=dt, seed=cfg["seed"] + rank,
+                                  gate=cfg["gate"], D=cfg["D"])
+        state_shape = (batch, cfg["dim"], cfg["N"])
+        tok_keys = ("u", "delta", "z", "B", "C")
+    else:
+        inp = synthetic.make_scalarA(batch, cfg["nheads"], cfg["headdim"], cfg["N"], 1,
+                                     ngroups=cfg["ngroups"], dtype=dt, seed=cfg["seed"] + rank,
+                                     gate=cfg["gate"])
+        state_shape = (batch, cfg["nheads"], cfg["headdim"], cfg["N"])
+        tok_keys = ("x", "dt", "z", "B", "C")
+    host = {k: inp[k][..., 0] for k in tok_keys if inp.get(k) is not None}
+    dev = {k: to_dev(v, "f32" if k == "dt" else dt, torch) for k, v in host.items()}
+    par = {k: to_dev(inp[k], "f32", torch) for k in ("A", "D", "delta_bias")
+           if inp.get(k) is not None}
+    state = torch.from_numpy(rng.standard_normal(state_shape, dtype=np.float32)).cuda()
+    first = dev["u"] if "u" in dev else dev["x"]
+    y = torch.empty(first.shape, dtype=first.dtype, device="cuda")
+
+    if cfg["kind"] == "diag":
+        def call():
+            ss.selscan_step(state, dev["u"], dev["delta"], par["A"], dev["B"], dev["C"],
+                            D=par.get("D"), z=dev.get("z"), delta_bias=par.get("delta_bias"),
+                            out=y)
+    else:
+        def call():
+            ss.selscan_step_scalarA(state, dev["x"], dev["dt"], par["A"], dev["B"], dev["C"],
+                                    cfg["headdim"], D=par.get("D"), z=dev.get("z"), out=y)
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    ss.check()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    ss.check()
+    total_ms = start.elapsed_time(end)
+    avg_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    clock_info = clocks.stop(t_wall0, t_wall1) if clocks else None
+    if dist:
+        t = torch.tensor([total_ms, avg_launch_ms], device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms, avg_launch_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    value = world * batch / (ms_per_step * 1e-3)
+
+    # end to end: the token's inputs from pinned host memory, y back; the
+    # state stays resident on the device, as a decoding server keeps it
+    pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(
+        torch.float32 if (k == "dt" or dt == "f32") else torch.bfloat16).pin_memory()
+        for k, v in host.items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = y_host.numel() * y_host.element_size()
+    e2e_steps = max(1, min(args.steps, 100))
+
+    def e2e_step():
+        for k, t in pinned.items():
+            dev[k].copy_(t, non_blocking=True)
+        call()
+        y_host.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    barrier()
+    if rank != 0:
+        return
+    peaks, peaks_src = measured_peaks()
+    nbytes = step_bytes(cfg)
+    traffic = args.traffic
+    if traffic is None and args.config in STEP_NCU_TRAFFIC and \
+            STEP_NCU_TRAFFIC[args.config][0] == STEP_KERNEL_TAG and \
+            batch == STEP_BATCH[cfg["kind"]] and base == BASE_CONFIGS[args.config]:
+        traffic = STEP_NCU_TRAFFIC[args.config][1]
+    achieved = nbytes / (avg_launch_ms * 1e-3) / 1e9
+    dim = cfg.get("dim") or cfg["nheads"] * cfg["headdim"]
+    line = {
+        "metric": "selective-scan decode step, tokens/s (one token per batch row) and % of "
+                  "B200 HBM roofline, 1 GPU",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dt, "data": "synthetic",
+        "config": {"workload": step_name(cfg), "batch": batch, "d_inner": dim, "d_state": cfg["N"],
+                   "global_batch": batch * world,
+                   "l2": "state larger than L2 (no flush)" if nbytes > 126e6 else
+                         "state smaller than L2",
+                   "parallelism": f"dp{world} (independent shards, no collective)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic, "peak_source": f"{peaks_src} HBM copy bandwidth",
+                     "bytes_per_launch": nbytes, "avg_launch_ms": avg_launch_ms},
+        "e2e": {"value": world * batch / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clock_info,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_step_sample(cfg, inp, state.cpu().numpy(),
+                                                  seconds=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def oracle_step_sample(cfg: dict, inp: dict, state: np.ndarray, seconds: float = 10.0):
+    """The fp64 oracle's decode step on the first rows of the batch, grown
+    until about `seconds` of single-threaded work; tokens/s."""
+    import oracle
+    rows, spent = 1, 0.0
+    while True:
+        t0 = time.perf_counter()
+        if cfg["kind"] == "diag":
+            oracle.selscan_step(state[:rows], inp["u"][:rows, :, 0], inp["delta"][:rows, :, 0],
+                                inp["A"], inp["B"][:rows, :, 0], inp["C"][:rows, :, 0],
+                                D=inp["D"], z=None if inp["z"] is None else inp["z"][:rows, :, 0],
+                                delta_bias=inp["delta_bias"])
+        else:
+            sl = lambda a: None if a is None else a[:rows]
+            oracle.selscan_scalarA(sl(inp["x"]), sl(inp["dt"]), inp["A"], sl(inp["B"]),
+                                   sl(inp["C"]), cfg["headdim"], D=inp["D"], z=sl(inp["z"]),
+                                   h0=state[:rows])
+        spent = time.perf_counter() - t0
+        if spent >= seconds * 0.5 or rows >= cfg["batch"]:
+            break
+        rows = int(min(cfg["batch"], rows * max(2.0, min(16.0, seconds / max(spent, 1e-3)))))
+    return {"value": rows / spent, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} batch row(s) of one decode step, {spent:.2f} s "
+                      "single-threaded fp64"}
+
+
 def ss_kernels_per_step_scalarA() -> int:
     import selective_state_space_selscan_b200 as ss
     return getattr(ss, "SCALARA_KERNELS_PER_CALL", 1)
@@ -442,11 +710,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="scan", choices=["scan", "step"],
+                    help="scan: the forward over the config's sequence (default); "
+                         "step: one decode step of the config's layer")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch from an ncu capture of this kernel")
     args = ap.parse_args()
 
-    if args.batch is not None:
+    if args.batch is not None and args.op == "scan":
         synthetic.CONFIGS[args.config] = dict(synthetic.CONFIGS[args.config], batch=args.batch)
     if args.seqlen is not None:
         synthetic.CONFIGS[args.config] = dict(synthetic.CONFIGS[args.config], L=args.seqlen)
@@ -464,7 +735,7 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local))
     try:
-        run_gpu(args, rank, world, local)
+        (run_step if args.op == "step" else run_gpu)(args, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as tdist

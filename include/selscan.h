@@ -204,6 +204,67 @@ SELSCAN_API selscan_status selscan_fwd_noalloc(
     selscan_tensor *y, selscan_tensor *last_state, cudaStream_t stream);
 
 /*
+ * selscan_step -- one decode step of the diagonal-A scan, state in place.
+ * "03 -- Modelos de espacio de estados: RWKV, S4, Mamba y el selective
+ * scan", section "Coste de inferencia": per token the layer updates a fixed
+ * state and reads it out, with no dependence on the length already seen.
+ * For every (b, d):
+ *
+ *   delta_t = softplus(delta[b,d] + delta_bias[d])   (softplus optional)
+ *   state[b,d,n] = exp(delta_t * A[d,n]) * state[b,d,n] + delta_t * B[b,g,n] * u[b,d]
+ *   y[b,d] = (sum_n C[b,g,n] * state[b,d,n] + D[d] * u[b,d]) * silu(z[b,d])
+ *
+ * which is one token of selscan_fwd_h0 with h0 = last_state = state.
+ *
+ *   state      (batch, D, N)  F32, contiguous, 16-byte aligned; read and
+ *                             overwritten with the new state
+ *   u, delta   (batch, D)     F32 or BF16 (same); any non-negative strides
+ *   delta_bias (D)            F32, contiguous; may be NULL
+ *   A          (D, N)         F32, contiguous, 16-byte aligned
+ *   B, C       (batch, N) or (batch, G, N)  same dtype as u, any strides;
+ *                             channel d reads group d / (D / G)
+ *   D          (D)            F32; may be NULL
+ *   z          (batch, D)     same dtype as u; may be NULL (no gate)
+ *   y          (batch, D)     same dtype as u; written; must not overlap an
+ *                             input other than u
+ *
+ * N must be 16, 32, 64 or 128.  The state must not overlap any other
+ * argument.  Arithmetic is fp32 with the library's exp.
+ */
+SELSCAN_API selscan_status selscan_step(selscan_tensor *state, const selscan_tensor *u,
+                            const selscan_tensor *delta, const selscan_tensor *delta_bias,
+                            int delta_softplus, const selscan_tensor *A,
+                            const selscan_tensor *B, const selscan_tensor *C,
+                            const selscan_tensor *D, const selscan_tensor *z,
+                            selscan_tensor *y, cudaStream_t stream);
+
+/*
+ * selscan_step_scalarA -- one decode step of the scalar-A (Mamba-2) scan,
+ * state in place: for channel d = h * headdim + p,
+ *
+ *   state[b,h,p,n] = exp(dt_t * A[h]) * state[b,h,p,n] + dt_t * B[b,g,n] * x[b,d]
+ *   y[b,d] = (sum_n C[b,g,n] * state[b,h,p,n] + D[h] * x[b,d]) * silu(z[b,d])
+ *
+ * with dt_t = softplus(dt[b,h] + dt_bias[h]) (softplus optional) and
+ * g = h / (H / G): one token of selscan_fwd_scalarA_h0.
+ *
+ *   state      (batch, H, P, N) F32, contiguous, 16-byte aligned; in place
+ *   x, z, y    (batch, H*P)     F32 or BF16 (same); any strides; z may be NULL
+ *   dt         (batch, H)       F32
+ *   dt_bias, D (H)              F32; may be NULL
+ *   A          (H)              F32
+ *   B, C       (batch, N) or (batch, G, N)  same dtype as x
+ *
+ * N must be 16, 32, 64 or 128; any headdim.
+ */
+SELSCAN_API selscan_status selscan_step_scalarA(selscan_tensor *state, const selscan_tensor *x,
+                                    const selscan_tensor *dt, const selscan_tensor *dt_bias,
+                                    int dt_softplus, const selscan_tensor *A,
+                                    const selscan_tensor *B, const selscan_tensor *C,
+                                    const selscan_tensor *D, const selscan_tensor *z,
+                                    int64_t headdim, selscan_tensor *y, cudaStream_t stream);
+
+/*
  * selscan_check -- synchronise `stream` and report device-side errors that
  * earlier calls recorded (a bounded wait that gave up returns
  * SELSCAN_ERR_TIMEOUT; the record is then cleared).  Returns

@@ -28,7 +28,8 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 # entry points declared in include/selscan.h
 EXPORTS = ("selscan_fwd", "selscan_fwd_h0", "selscan_fwd_scalarA", "selscan_fwd_scalarA_h0",
-           "selscan_fwd_noalloc", "selscan_check", "selscan_strerror", "selscan_version")
+           "selscan_fwd_noalloc", "selscan_step", "selscan_step_scalarA", "selscan_check",
+           "selscan_strerror", "selscan_version")
 
 
 class SelscanError(RuntimeError):
@@ -78,6 +79,12 @@ def lib() -> ctypes.CDLL:
         L.selscan_fwd_noalloc.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, P, P, P,
                                           ctypes.c_void_p]
         L.selscan_fwd_noalloc.restype = ctypes.c_int
+        L.selscan_step.argtypes = [P, P, P, P, ctypes.c_int, P, P, P, P, P, P,
+                                   ctypes.c_void_p]
+        L.selscan_step.restype = ctypes.c_int
+        L.selscan_step_scalarA.argtypes = [P, P, P, P, ctypes.c_int, P, P, P, P, P,
+                                           ctypes.c_int64, P, ctypes.c_void_p]
+        L.selscan_step_scalarA.restype = ctypes.c_int
         L.selscan_debug_withhold_carry.argtypes = [ctypes.c_int]
         L.selscan_debug_withhold_carry.restype = None
         _lib = L
@@ -208,6 +215,39 @@ def selscan_fwd_scalarA(x, dt, A, B, C, headdim, D=None, z=None, dt_bias=None,
     if rc != 0:
         raise SelscanError(rc, where)
     return y, last_state
+
+
+def selscan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                 delta_softplus=True, out=None, stream=None):
+    """One decode step of the diagonal-A scan; ``state`` (batch, D, N) fp32
+    is updated in place.  u, delta, z: (batch, D) bf16 or fp32 (any strides);
+    B, C: (batch, N) or (batch, G, N).  Returns y (batch, D)."""
+    import torch
+    y = out if out is not None else torch.empty(u.shape, dtype=u.dtype, device=u.device)
+    d = [describe(t) for t in (state, u, delta, delta_bias, A, B, C, D, z, y)]
+    rc = lib().selscan_step(_ref(d[0]), _ref(d[1]), _ref(d[2]), _ref(d[3]),
+                            int(bool(delta_softplus)), _ref(d[4]), _ref(d[5]), _ref(d[6]),
+                            _ref(d[7]), _ref(d[8]), _ref(d[9]), _stream_handle(stream))
+    if rc != 0:
+        raise SelscanError(rc, "selscan_step")
+    return y
+
+
+def selscan_step_scalarA(state, x, dt, A, B, C, headdim, D=None, z=None, dt_bias=None,
+                         dt_softplus=False, out=None, stream=None):
+    """One decode step of the scalar-A (Mamba-2) scan; ``state`` (batch, H,
+    P, N) fp32 is updated in place.  x, z: (batch, H*P); dt: (batch, H)
+    fp32; B, C: (batch, N) or (batch, G, N).  Returns y (batch, H*P)."""
+    import torch
+    y = out if out is not None else torch.empty(x.shape, dtype=x.dtype, device=x.device)
+    d = [describe(t) for t in (state, x, dt, dt_bias, A, B, C, D, z, y)]
+    rc = lib().selscan_step_scalarA(_ref(d[0]), _ref(d[1]), _ref(d[2]), _ref(d[3]),
+                                    int(bool(dt_softplus)), _ref(d[4]), _ref(d[5]),
+                                    _ref(d[6]), _ref(d[7]), _ref(d[8]), int(headdim),
+                                    _ref(d[9]), _stream_handle(stream))
+    if rc != 0:
+        raise SelscanError(rc, "selscan_step_scalarA")
+    return y
 
 
 def check(stream=None) -> None:

@@ -16,6 +16,7 @@
 #include "scan_diag.cuh"
 #include "scan_diag_bf16.cuh"
 #include "ssd_scalarA.cuh"
+#include "step.cuh"
 
 using namespace selscan;
 
@@ -846,4 +847,223 @@ extern "C" selscan_status selscan_fwd_noalloc(
                                                                     scratch, stream)
                 : launch_diag_noalloc<0, float, 64, 4, false, true>(u, delta, B, C, z, y, prm,
                                                                      sms, scratch, stream);
+}
+
+// ------------------------------------------------------------ decode step
+namespace {
+
+// A per-token tensor (d0, d1): any non-negative element strides, element-
+// aligned data.
+selscan_status check_tok(const selscan_tensor *t, int64_t d0, int64_t d1, int32_t dtype)
+{
+    if (!present(t))
+        return SELSCAN_ERR_NULL;
+    if (t->ndim != 2 || t->shape[0] != d0 || t->shape[1] != d1)
+        return SELSCAN_ERR_SHAPE;
+    if (t->dtype != dtype)
+        return SELSCAN_ERR_DTYPE;
+    if (d0 == 0 || d1 == 0)
+        return SELSCAN_OK;
+    if (t->stride[0] < 0 || t->stride[1] < 0)
+        return SELSCAN_ERR_STRIDE;
+    if (reinterpret_cast<uintptr_t>(t->data) % elem_size(dtype))
+        return SELSCAN_ERR_ALIGN;
+    return SELSCAN_OK;
+}
+
+// B or C of one token: (batch, N) or (batch, G, N); returns G through *G.
+selscan_status check_tok_bc(const selscan_tensor *t, int64_t batch, int64_t N, int32_t dtype,
+                            int64_t *G, int64_t s[3])
+{
+    if (!present(t))
+        return SELSCAN_ERR_NULL;
+    if (t->dtype != dtype)
+        return SELSCAN_ERR_DTYPE;
+    if (t->ndim == 2) {
+        if (t->shape[0] != batch || t->shape[1] != N)
+            return SELSCAN_ERR_SHAPE;
+        *G = 1;
+        s[0] = t->stride[0];
+        s[1] = 0;
+        s[2] = t->stride[1];
+    } else if (t->ndim == 3) {
+        if (t->shape[0] != batch || t->shape[2] != N || t->shape[1] <= 0)
+            return SELSCAN_ERR_SHAPE;
+        *G = t->shape[1];
+        s[0] = t->stride[0];
+        s[1] = t->stride[1];
+        s[2] = t->stride[2];
+    } else {
+        return SELSCAN_ERR_SHAPE;
+    }
+    if (s[0] < 0 || s[1] < 0 || s[2] < 0)
+        return SELSCAN_ERR_STRIDE;
+    if (numel(t) > 0 && reinterpret_cast<uintptr_t>(t->data) % elem_size(dtype))
+        return SELSCAN_ERR_ALIGN;
+    return SELSCAN_OK;
+}
+
+template <typename T, bool SCALAR>
+cudaError_t launch_step(const StepParams &prm, int64_t batch, int tpc, cudaStream_t stream)
+{
+    const int64_t inner = SCALAR ? prm.headdim : prm.dim;
+    const dim3 grid(unsigned((inner * tpc + 255) / 256), SCALAR ? unsigned(prm.units) : 1u,
+                    unsigned(batch));
+    switch (tpc) {
+    case 2: step_kernel<T, 2, SCALAR><<<grid, 256, 0, stream>>>(prm); break;
+    case 4: step_kernel<T, 4, SCALAR><<<grid, 256, 0, stream>>>(prm); break;
+    case 8: step_kernel<T, 8, SCALAR><<<grid, 256, 0, stream>>>(prm); break;
+    default: step_kernel<T, 16, SCALAR><<<grid, 256, 0, stream>>>(prm); break;
+    }
+    return cudaGetLastError();
+}
+
+// Shared by the diagonal and the scalar (Mamba-2) step.  `scalar` selects
+// per-head A / dt / bias / D and a (batch, H, P, N) state.
+selscan_status step_impl(bool scalar, selscan_tensor *state, const selscan_tensor *u,
+                         const selscan_tensor *delta, const selscan_tensor *delta_bias,
+                         int delta_softplus, const selscan_tensor *A, const selscan_tensor *B,
+                         const selscan_tensor *C, const selscan_tensor *D,
+                         const selscan_tensor *z, int64_t headdim, selscan_tensor *y,
+                         cudaStream_t stream)
+{
+    if (!present(state) || !present(u) || !present(delta) || !present(A) || !B || !C ||
+        !present(y))
+        return SELSCAN_ERR_NULL;
+    const int32_t dt = u->dtype;
+    if (dt != SELSCAN_F32 && dt != SELSCAN_BF16)
+        return SELSCAN_ERR_DTYPE;
+    if (u->ndim != 2)
+        return SELSCAN_ERR_SHAPE;
+    const int64_t batch = u->shape[0], dim = u->shape[1];
+    if (batch < 0 || dim < 0)
+        return SELSCAN_ERR_SHAPE;
+    int64_t units, N;
+    if (scalar) {
+        if (A->ndim != 1 || headdim <= 0 || state->ndim != 4)
+            return SELSCAN_ERR_SHAPE;
+        units = A->shape[0];
+        if (units <= 0 || dim != units * headdim)
+            return SELSCAN_ERR_SHAPE;
+        N = state->shape[3];
+    } else {
+        if (A->ndim != 2 || A->shape[0] != dim || state->ndim != 3)
+            return SELSCAN_ERR_SHAPE;
+        units = dim;
+        headdim = 1;
+        N = A->shape[1];
+    }
+    selscan_status st;
+    if ((st = check_tok(u, batch, dim, dt)) != SELSCAN_OK) return st;
+    if ((st = check_tok(y, batch, dim, dt)) != SELSCAN_OK) return st;
+    if (z && z->data && (st = check_tok(z, batch, dim, dt)) != SELSCAN_OK) return st;
+    if ((st = check_tok(delta, batch, units, scalar ? SELSCAN_F32 : dt)) != SELSCAN_OK)
+        return st;
+    int64_t G = 1, Gc = 1, sb[3], sc[3];
+    if ((st = check_tok_bc(B, batch, N, dt, &G, sb)) != SELSCAN_OK) return st;
+    if ((st = check_tok_bc(C, batch, N, dt, &Gc, sc)) != SELSCAN_OK) return st;
+    if (Gc != G || units % G != 0)
+        return SELSCAN_ERR_SHAPE;
+    {
+        const int64_t ushape[1] = {units};
+        if ((st = check_param(delta_bias, 1, ushape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(D, 1, ushape, true)) != SELSCAN_OK) return st;
+        if (scalar) {
+            if ((st = check_param(A, 1, ushape, false)) != SELSCAN_OK) return st;
+            const int64_t sshape[4] = {batch, units, headdim, N};
+            if ((st = check_param(state, 4, sshape, false)) != SELSCAN_OK) return st;
+        } else {
+            const int64_t ashape[2] = {dim, N};
+            if ((st = check_param(A, 2, ashape, false)) != SELSCAN_OK) return st;
+            if (!aligned16(A->data))
+                return SELSCAN_ERR_ALIGN;
+            const int64_t sshape[3] = {batch, dim, N};
+            if ((st = check_param(state, 3, sshape, false)) != SELSCAN_OK) return st;
+        }
+    }
+    if (N != 16 && N != 32 && N != 64 && N != 128)
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch == 0 || dim == 0)
+        return SELSCAN_OK;
+    if (!aligned16(state->data))
+        return SELSCAN_ERR_ALIGN;
+    const int tpc = int(N / 8);
+    if (batch > 65535 || dim * tpc > (int64_t(0x7fffffff) - 255) || units > 65535)
+        return SELSCAN_ERR_UNSUPPORTED;
+
+    StepParams prm{};
+    prm.dim = int(dim);
+    prm.headdim = int(headdim);
+    prm.units = int(units);
+    prm.per_group = int(units / G);
+    {
+        // B and C rows readable as aligned 4-element vectors
+        const int64_t es = int64_t(elem_size(dt));
+        auto vec_ok = [&](const selscan_tensor *t, const int64_t s[3]) {
+            return s[2] == 1 && s[0] % 4 == 0 && s[1] % 4 == 0 &&
+                   reinterpret_cast<uintptr_t>(t->data) % uintptr_t(4 * es) == 0;
+        };
+        prm.bc_vec = vec_ok(B, sb) && vec_ok(C, sc) ? 1 : 0;
+    }
+    prm.u = u->data;
+    prm.su0 = u->stride[0];
+    prm.su1 = u->stride[1];
+    prm.delta = delta->data;
+    prm.sd0 = delta->stride[0];
+    prm.sd1 = delta->stride[1];
+    const bool gate = z && z->data;
+    prm.z = gate ? z->data : nullptr;
+    prm.sz0 = gate ? z->stride[0] : 0;
+    prm.sz1 = gate ? z->stride[1] : 0;
+    prm.y = y->data;
+    prm.sy0 = y->stride[0];
+    prm.sy1 = y->stride[1];
+    prm.B = B->data;
+    prm.sb0 = sb[0];
+    prm.sb1 = sb[1];
+    prm.sb2 = sb[2];
+    prm.C = C->data;
+    prm.sc0 = sc[0];
+    prm.sc1 = sc[1];
+    prm.sc2 = sc[2];
+    prm.A = static_cast<const float *>(A->data);
+    prm.delta_bias = static_cast<const float *>(opt_data(delta_bias));
+    prm.Dskip = static_cast<const float *>(opt_data(D));
+    prm.state = static_cast<float *>(state->data);
+    prm.softplus = delta_softplus ? 1 : 0;
+
+    cudaError_t e;
+    if (dt == SELSCAN_BF16)
+        e = scalar ? launch_step<__nv_bfloat16, true>(prm, batch, tpc, stream)
+                   : launch_step<__nv_bfloat16, false>(prm, batch, tpc, stream);
+    else
+        e = scalar ? launch_step<float, true>(prm, batch, tpc, stream)
+                   : launch_step<float, false>(prm, batch, tpc, stream);
+    return e == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" selscan_status selscan_step(selscan_tensor *state, const selscan_tensor *u,
+                                       const selscan_tensor *delta,
+                                       const selscan_tensor *delta_bias, int delta_softplus,
+                                       const selscan_tensor *A, const selscan_tensor *B,
+                                       const selscan_tensor *C, const selscan_tensor *D,
+                                       const selscan_tensor *z, selscan_tensor *y,
+                                       cudaStream_t stream)
+{
+    return step_impl(false, state, u, delta, delta_bias, delta_softplus, A, B, C, D, z, 1, y,
+                     stream);
+}
+
+extern "C" selscan_status selscan_step_scalarA(selscan_tensor *state, const selscan_tensor *x,
+                                               const selscan_tensor *dt,
+                                               const selscan_tensor *dt_bias, int dt_softplus,
+                                               const selscan_tensor *A, const selscan_tensor *B,
+                                               const selscan_tensor *C, const selscan_tensor *D,
+                                               const selscan_tensor *z, int64_t headdim,
+                                               selscan_tensor *y, cudaStream_t stream)
+{
+    return step_impl(true, state, x, dt, dt_bias, dt_softplus, A, B, C, D, z, headdim, y,
+                     stream);
 }

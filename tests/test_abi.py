@@ -132,3 +132,52 @@ def _scal(**over):
 ])
 def test_scalarA_rejects(over, expect):
     assert _scal(**over) == C[expect]
+
+
+def _step(scalar=False, **over):
+    b, D, N = 2, 64, 16
+    if scalar:
+        H, P, N = 2, 32, 128
+        args = dict(state=_t((b, H, P, N), ss.SELSCAN_F32), u=_t((b, H * P)),
+                    delta=_t((b, H), ss.SELSCAN_F32), bias=None, A=_t((H,), ss.SELSCAN_F32),
+                    B=_t((b, N)), C=_t((b, N)), Dv=_t((H,), ss.SELSCAN_F32), z=None,
+                    y=_t((b, H * P)), P=P)
+    else:
+        args = dict(state=_t((b, D, N), ss.SELSCAN_F32), u=_t((b, D)), delta=_t((b, D)),
+                    bias=_t((D,), ss.SELSCAN_F32), A=_t((D, N), ss.SELSCAN_F32),
+                    B=_t((b, N)), C=_t((b, N)), Dv=_t((D,), ss.SELSCAN_F32), z=_t((b, D)),
+                    y=_t((b, D)))
+    args.update(over)
+    r = lambda x: None if x is None else ctypes.byref(x)
+    common = (r(args["state"]), r(args["u"]), r(args["delta"]), r(args["bias"]), 1,
+              r(args["A"]), r(args["B"]), r(args["C"]), r(args["Dv"]), r(args["z"]))
+    if scalar:
+        return ss.lib().selscan_step_scalarA(*common, args["P"], r(args["y"]), None)
+    return ss.lib().selscan_step(*common, r(args["y"]), None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(state=None), "SELSCAN_ERR_NULL"),
+    (dict(y=None), "SELSCAN_ERR_NULL"),
+    (dict(u=_t((2, 64, 1))), "SELSCAN_ERR_SHAPE"),
+    (dict(delta=_t((2, 64), ss.SELSCAN_F32)), "SELSCAN_ERR_DTYPE"),
+    (dict(state=_t((2, 64, 16), ss.SELSCAN_F32, data=FAKE + 4)), "SELSCAN_ERR_ALIGN"),
+    (dict(state=_t((2, 64, 16), ss.SELSCAN_F32, strides=(2048, 32, 1))), "SELSCAN_ERR_STRIDE"),
+    (dict(B=_t((2, 3, 16)), C=_t((2, 3, 16))), "SELSCAN_ERR_SHAPE"),
+    (dict(B=_t((2, 2, 16)), C=_t((2, 4, 16))), "SELSCAN_ERR_SHAPE"),
+    (dict(y=_t((2, 64), strides=(-64, 1))), "SELSCAN_ERR_STRIDE"),
+    (dict(A=_t((64, 8), ss.SELSCAN_F32), state=_t((2, 64, 8), ss.SELSCAN_F32),
+          B=_t((2, 8)), C=_t((2, 8))), "SELSCAN_ERR_UNSUPPORTED"),
+])
+def test_step_rejects(over, expect):
+    assert _step(**over) == C[expect]
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(P=48), "SELSCAN_ERR_SHAPE"),
+    (dict(delta=_t((2, 2))), "SELSCAN_ERR_DTYPE"),
+    (dict(state=_t((2, 2, 32, 64), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(A=_t((2, 1), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+])
+def test_step_scalarA_rejects(over, expect):
+    assert _step(scalar=True, **over) == C[expect]
