@@ -44,9 +44,9 @@ NCU_TRAFFIC = {
     2: ("scan_diag_bf16_kernel pairs v3", 647.2e6),
     4: ("ssd_scalarA_kernel v1", 109.0e6),
 }
-KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v3", 1: "scan_diag_bf16_kernel pairs v3",
-              3: "scan_diag_bf16_kernel pairs v3", 0: "scan_diag_kernel fp32 v1",
-              4: "ssd_scalarA_kernel v2"}
+KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v4", 1: "scan_diag_bf16_kernel pairs v4",
+              3: "scan_diag_bf16_kernel pairs v4", 0: "scan_diag_kernel fp32 v2",
+              4: "ssd_scalarA_kernel v3"}
 HBM_FALLBACK_GBS = 6650.0
 
 

@@ -275,8 +275,9 @@ scan_diag_kernel(const __grid_constant__ CUtensorMap tm_u,
     static_assert(CONS % 32 == 0, "consumer threads must fill warps");
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, offset from the shared array itself so that
+    // every pointer derived from it stays in the shared address space
+    uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem + Lay::kStagesOff;
     float *bc = reinterpret_cast<float *>(smem + Lay::kBCOff);
     uint8_t *ytile = smem + Lay::kYOff;

@@ -559,12 +559,15 @@ static selscan_status scalarA_impl(const selscan_tensor *x, const selscan_tensor
         return st;
 
     // B/C (batch, 1, N, L) -> 3-D maps over (L, N, batch); x over (L, H*P, batch)
-    CUtensorMap tm_C, tm_B, tm_X;
+    // y (batch, H*P, L) is written back through the same kind of map
+    CUtensorMap tm_C, tm_B, tm_X, tm_Y;
     if (!encode_3d(&tm_C, C->data, SELSCAN_BF16, L, N, batch, C->stride[2], C->stride[0], 64,
                    kSsdN) ||
         !encode_3d(&tm_B, B->data, SELSCAN_BF16, L, N, batch, B->stride[2], B->stride[0], 64,
                    kSsdN) ||
         !encode_3d(&tm_X, x->data, SELSCAN_BF16, L, dim, batch, x->stride[1], x->stride[0], 64,
+                   kSsdP) ||
+        !encode_3d(&tm_Y, y->data, SELSCAN_BF16, L, dim, batch, y->stride[1], y->stride[0], 64,
                    kSsdP))
         return SELSCAN_ERR_ALIGN;
     SsdParams prm{};
@@ -583,9 +586,6 @@ static selscan_status scalarA_impl(const selscan_tensor *x, const selscan_tensor
     prm.z = gate ? static_cast<const __nv_bfloat16 *>(z->data) : nullptr;
     prm.z_bs = gate ? z->stride[0] : 0;
     prm.z_cs = gate ? z->stride[1] : 0;
-    prm.y = static_cast<__nv_bfloat16 *>(y->data);
-    prm.y_bs = y->stride[0];
-    prm.y_cs = y->stride[1];
     prm.last_state = static_cast<float *>(last_state ? last_state->data : nullptr);
     prm.h0 = static_cast<const float *>(opt_data(h0));
     prm.timeout_ns = default_timeout_ns();
@@ -602,7 +602,8 @@ static selscan_status scalarA_impl(const selscan_tensor *x, const selscan_tensor
     const int64_t grid = batch * H;
     if (grid > 0x7fffffffll)
         return SELSCAN_ERR_UNSUPPORTED;
-    kern<<<unsigned(grid), 256, SsdLayout::kAlloc, stream>>>(tm_C, tm_B, tm_X, prm);
+    kern<<<unsigned(grid), kSsdWG * 128, SsdLayout::kAlloc, stream>>>(tm_C, tm_B, tm_X, tm_Y,
+                                                                       prm);
     return cudaGetLastError() == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
 }
 

@@ -6,35 +6,48 @@
 //
 // One CTA owns one (batch, head) and walks its chunks of Q = 128 tokens in
 // order, carrying the head's state h (N x P = 128 x 64, fp32) in tensor
-// memory.  For a chunk with cumulative step sum S_t (inclusive, from the
-// chunk start):
+// memory.  With cs_t = A log2(e) S_t, S_t the inclusive sum of the step
+// sizes from the chunk start:
 //
 //   G[t,s]   = sum_n C[n,t] B[n,s]                       (tcgen05, K = N)
-//   M[t,s]   = G[t,s] exp(A (S_t - S_s)) delta_s, s <= t  (CUDA cores)
+//   M[t,s]   = G[t,s] 2^(cs_t - cs_s) delta_s, s <= t     (CUDA cores)
 //   Yd[t,p]  = sum_s M[t,s] x[p,s]                        (tcgen05, K = Q)
 //   Yo[t,p]  = sum_n C[n,t] h_prev[n,p]                   (tcgen05, K = N)
-//   y[p,t]   = Yd[t,p] + exp(A S_t) Yo[t,p] + D x[p,t]    (then the gate)
-//   h[n,p]   = exp(A S_Q) h_prev[n,p]
-//            + sum_s B[n,s] exp(A (S_Q - S_s)) delta_s x[p,s]   (tcgen05)
+//   y[p,t]   = Yd[t,p] + 2^cs_t Yo[t,p] + D x[p,t]        (then the gate)
+//   h[n,p]   = 2^cs_Q h_prev[n,p]
+//            + sum_s B[n,s] 2^(cs_Q - cs_s) delta_s x[p,s]   (tcgen05)
 //
-// exp(A (S_t - S_s)) is the product of the per-token decays between s and
-// t, so this is the recurrence of the diagonal scan with A[d,n] = A_head.
-// The mask factors never overflow: inside a 32-token block the exponential
-// is taken per element; across blocks it is split at the end of the earlier
-// block, where both factors are <= 1.
+// 2^(cs_t - cs_s) is the product of the per-token decays between s and t, so
+// this is the recurrence of the diagonal scan with A[d,n] = A_head.  No
+// factor exceeds 1: below the diagonal 16 x 16 pieces of M the decay is split
+// at the last token e of the column piece, 2^(cs_t - cs_e) 2^(cs_e - cs_s)
+// (one exponential per row and piece, one per column), and in the pieces
+// that hold a warp's diagonal it is taken per element.
+//
+// Per chunk c, in order (all threads unless noted):
+//   1. x * w for the state product (needs chunk c's x);
+//   2. M from G (tensor memory) and the decays (needs G(c));
+//   3. one thread issues Yd(c), the state product and G(c + 1);
+//   4. the first warpgroup prepares the step sizes of chunk c + 1;
+//   5. y = Yd + 2^cs_t Yo + D x (+ gate), staged in shared memory and written
+//      back by one bulk tensor store;
+//   6. state: h -> bf16 copy for Yo(c + 1), last_state, h *= 2^cs_Q(c + 1);
+//   7. one thread issues Yo(c + 1) and the loads of chunk c + 2.
 //
 // Operands (bf16, 128-byte swizzle) in shared memory:
 //   C chunk [n][t] and B chunk [n][s] as loaded by the bulk tensor copy,
 //   used MN-major (C^T as A of G and Yo; B as B of G) and K-major (B as A of
 //   the state product); x chunk [p][s] (K-major B of Yd); x * w [p][s]
 //   (K-major B of the state product); M [t][s] (K-major A of Yd); h_prev in
-//   bf16 [n][p] (MN-major B of Yo).  Accumulators in tensor memory (fp32):
-//   G (128 columns), Yd (64), Yo (64), h (64).
+//   bf16 [n][p] (MN-major B of Yo).  The y tile [p][t] is staged in the M
+//   buffer once Yd has read it.  Accumulators in tensor memory (fp32): G (128
+//   columns), Yd (64), Yo (64), h (64).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "f32x2.cuh"
 #include "ptx.cuh"
 #include "umma.cuh"
 
@@ -43,6 +56,7 @@ namespace selscan {
 constexpr int kSsdN = 128;  // state size built
 constexpr int kSsdP = 64;   // head dimension built
 constexpr int kSsdQ = 128;  // chunk length
+constexpr int kSsdWG = 4;   // warpgroups per CTA
 
 struct SsdParams {
     int batch, H, L, nchunks;
@@ -54,8 +68,6 @@ struct SsdParams {
     const float *Dskip;        // (H) or null
     const __nv_bfloat16 *z;    // (batch, H*P, L) or null
     int64_t z_bs, z_cs;
-    __nv_bfloat16 *y;          // (batch, H*P, L)
-    int64_t y_bs, y_cs;
     float *last_state;         // (batch, H, P, N) or null
     const float *h0;           // (batch, H, P, N) or null: initial state
     unsigned long long timeout_ns;
@@ -67,7 +79,7 @@ struct SsdLayout {
     static constexpr int kB = kC + 2 * 32768;      // 2 buffers x [2 slabs][128 n][64 s]
     static constexpr int kX = kB + 2 * 32768;      // 2 buffers x [2 slabs][64 p][64 s]
     static constexpr int kXw = kX + 2 * 16384;     // [2 slabs][64 p][64 s]
-    static constexpr int kM = kXw + 16384;         // [2 slabs][128 t][64 s]
+    static constexpr int kM = kXw + 16384;         // [2 slabs][128 t][64 s]; y tile [2][64 p][64 t]
     static constexpr int kHs = kM + 32768;         // [128 n][64 p]
     static constexpr int kBytes = kHs + 16384;
     static constexpr int kAlloc = kBytes + 1024;
@@ -76,94 +88,74 @@ struct SsdLayout {
 constexpr uint32_t kSsdTmemCols = 512;
 constexpr uint32_t kColG = 0, kColYd = 128, kColYo = 192, kColH = 256;
 
-__device__ __forceinline__ uint32_t ssd_pack2(float a, float b)
-{
-    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
 __device__ __forceinline__ float ssd_softplus(float x)
 {
     return x > 20.f ? x : log1pf(__expf(x));
 }
 
+// 16 consecutive fp32 from shared memory (16-byte aligned).
+__device__ __forceinline__ void lds16(const float *src, float (&v)[16])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 q = reinterpret_cast<const float4 *>(src)[i];
+        v[4 * i] = q.x;
+        v[4 * i + 1] = q.y;
+        v[4 * i + 2] = q.z;
+        v[4 * i + 3] = q.w;
+    }
+}
+
+// 16 values -> bf16, stored as two 16-byte swizzle units at byte offsets o0, o1.
+__device__ __forceinline__ void sts16_bf16(uint8_t *base, uint32_t o0, uint32_t o1,
+                                           const float (&m)[16])
+{
+    uint4 a, c;
+    a.x = pack2_bf16(m[0], m[1]);
+    a.y = pack2_bf16(m[2], m[3]);
+    a.z = pack2_bf16(m[4], m[5]);
+    a.w = pack2_bf16(m[6], m[7]);
+    c.x = pack2_bf16(m[8], m[9]);
+    c.y = pack2_bf16(m[10], m[11]);
+    c.z = pack2_bf16(m[12], m[13]);
+    c.w = pack2_bf16(m[14], m[15]);
+    *reinterpret_cast<uint4 *>(base + o0) = a;
+    *reinterpret_cast<uint4 *>(base + o1) = c;
+}
+
 template <bool GATE>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kSsdWG * 128, 1)
 ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                    const __grid_constant__ CUtensorMap tm_B,
-                   const __grid_constant__ CUtensorMap tm_X, const SsdParams p)
+                   const __grid_constant__ CUtensorMap tm_X,
+                   const __grid_constant__ CUtensorMap tm_Y, const SsdParams p)
 {
     using Lay = SsdLayout;
-    constexpr int Q = kSsdQ, P = kSsdP, N = kSsdN;
+    constexpr int Q = kSsdQ, P = kSsdP, N = kSsdN, NWG = kSsdWG, NT = NWG * 128;
+    constexpr int PW = P / NWG;    // p columns per thread in the epilogue / state pass
+    constexpr int QPW = 8 / NWG;   // 16-column pieces of M per thread
+    static_assert(PW % 16 == 0 && QPW % 2 == 0, "column split");
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ float s_delta[Q], s_S[Q], s_g[Q], s_wsum[4];
-    __shared__ uint64_t bar_tma[2], bar_g, bar_yo, bar_mma;
+    // 1024-byte aligned base, offset from the shared array itself so that
+    // every pointer derived from it stays in the shared address space
+    uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    // per-token values of the chunk being prepared (see cumsum below)
+    __shared__ __align__(16) float s_cs[Q], s_n2[Q], s_sg[Q];
+    __shared__ float s_wsum[4];
+    __shared__ uint64_t bar_tma[2], bar_g, bar_yo, bar_yd, bar_st;
     __shared__ uint32_t s_tbase;
 
-    // Two threads per row: r = row / token / state index, half = which half of
-    // the columns this thread handles.  Warp w reaches TMEM lanes 32*(w%4).
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r = tid & 127, half = tid >> 7;
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // TMEM lane: token t or state n of this thread
     const int b = blockIdx.x / p.H, hh = blockIdx.x - b * p.H;
     const float a_l2 = p.A[hh] * 1.4426950408889634f;  // A in log2 units
     const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
     const float dsk = p.Dskip ? p.Dskip[hh] : 0.f;
     const uint32_t sbase = smem_addr(smem);
     const uint32_t aXw = sbase + Lay::kXw, aM = sbase + Lay::kM, aHs = sbase + Lay::kHs;
-
-    if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(&bar_g, 1);
-        mbar_init(&bar_yo, 1);
-        mbar_init(&bar_mma, 1);
-        fence_mbar_init();
-        prefetch_tmap(&tm_C);
-        prefetch_tmap(&tm_B);
-        prefetch_tmap(&tm_X);
-    }
-    if (warp == 0)
-        tmem_alloc(&s_tbase, kSsdTmemCols);
-    // initial state h[n][p] (zero unless given): this thread's row n = r,
-    // columns p of its half; kept in fp32 for TMEM and in bf16 for C^T h
-    float h_init[32];
-    {
-        const float *h0row = p.h0 ? p.h0 + (int64_t(b) * p.H + hh) * P * N + r : nullptr;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            h_init[i] = h0row ? h0row[int64_t(half * 32 + i) * N] : 0.f;
-        uint8_t *hs = smem + Lay::kHs;
-#pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-            uint4 pk;
-            pk.x = ssd_pack2(h_init[g8 * 8 + 0], h_init[g8 * 8 + 1]);
-            pk.y = ssd_pack2(h_init[g8 * 8 + 2], h_init[g8 * 8 + 3]);
-            pk.z = ssd_pack2(h_init[g8 * 8 + 4], h_init[g8 * 8 + 5]);
-            pk.w = ssd_pack2(h_init[g8 * 8 + 6], h_init[g8 * 8 + 7]);
-            *reinterpret_cast<uint4 *>(hs + sw128_offset(r, half * 32 + g8 * 8)) = pk;
-        }
-    }
-    fence_proxy_async_smem();
-    tmem_fence_before_sync();
-    __syncthreads();
-    tmem_fence_after_sync();
-    const uint32_t tb = s_tbase;
-    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;  // this warp's TMEM lanes
-    const uint32_t colh = uint32_t(half * 32);                   // this thread's column half
-    {
-        float v0[16], v1[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            v0[i] = h_init[i];
-            v1[i] = h_init[16 + i];
-        }
-        tmem_st16(tb + lane_off + kColH + colh, v0);
-        tmem_st16(tb + lane_off + kColH + colh + 16, v1);
-    }
-
     const float *dt_row = p.dt + int64_t(b) * p.dt_bs + int64_t(hh) * p.dt_hs;
+
     auto issue_loads = [&](int c) {
         const int t0 = c * Q, buf = c & 1;
         mbar_arrive_expect_tx(&bar_tma[buf], 32768 + 32768 + 16384);
@@ -177,6 +169,92 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
         tma_load_3d(xs, &tm_X, &bar_tma[buf], t0, hh * P, b);
         tma_load_3d(xs + 8192, &tm_X, &bar_tma[buf], t0 + 64, hh * P, b);
     };
+
+    if (tid == 0) {
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
+        mbar_init(&bar_g, 1);
+        mbar_init(&bar_yo, 1);
+        mbar_init(&bar_yd, 1);
+        mbar_init(&bar_st, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_C);
+        prefetch_tmap(&tm_B);
+        prefetch_tmap(&tm_X);
+        prefetch_tmap(&tm_Y);
+        issue_loads(0);
+        if (p.nchunks > 1)
+            issue_loads(1);
+    }
+    if (warp == 0)
+        tmem_alloc(&s_tbase, kSsdTmemCols);
+
+    // Step sizes of chunk cc (first warpgroup, token r): delta, its inclusive
+    // sum in log2-decay units cs, and per token
+    //   s_n2[s] = log2(delta_s) - cs_s        (pieces on a warp's diagonal)
+    //   s_sg[s] = 2^(cs_e - cs_s) delta_s     (e = last token of s's piece)
+    auto cumsum = [&](int cc, float dtv) {
+        if (wg != 0)
+            return;
+        float dl = dtv + bias;
+        if (p.softplus)
+            dl = ssd_softplus(dl);
+        dl = (cc * Q + r < p.L) ? dl : 0.f;
+        float S = dl;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, S, o);
+            if (lane >= o)
+                S += v;
+        }
+        if (lane == 31)
+            s_wsum[quarter] = S;
+        named_bar_sync(1, 128);
+        for (int w = 0; w < quarter; ++w)
+            S += s_wsum[w];
+        const float cs = a_l2 * S;
+        const float cse = __shfl_sync(0xffffffffu, cs, lane | 15);
+        s_cs[r] = cs;
+        s_n2[r] = lg2_approx(dl) - cs;  // -inf for delta = 0, and 2^-inf = 0
+        s_sg[r] = ex2_approx(cse - cs) * dl;
+    };
+
+    // initial state h[n][p] (zero unless given): row n = r, columns p of this
+    // warpgroup's slice
+    float h_init[PW];
+    {
+        const float *h0row = p.h0 ? p.h0 + (int64_t(b) * p.H + hh) * P * N + r : nullptr;
+#pragma unroll
+        for (int i = 0; i < PW; ++i)
+            h_init[i] = h0row ? h0row[int64_t(wg * PW + i) * N] : 0.f;
+    }
+    cumsum(0, (wg == 0 && r < p.L) ? dt_row[r] : 0.f);
+    float dt_next = (wg == 0 && Q + r < p.L) ? dt_row[Q + r] : 0.f;
+    __syncthreads();  // s_cs of chunk 0, TMEM address
+    tmem_fence_after_sync();
+    const uint32_t tb = s_tbase;
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;  // this warp's TMEM lanes
+    {
+        const float alpha0 = ex2_approx(s_cs[Q - 1]);
+        uint8_t *hs = smem + Lay::kHs;
+#pragma unroll
+        for (int cc = 0; cc < PW; cc += 16) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                v[i] = h_init[cc + i];
+            const uint32_t col = uint32_t(wg * PW + cc);
+            sts16_bf16(hs, sw128_offset(r, col), sw128_offset(r, col + 8), v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                v[i] *= alpha0;
+            tmem_st16(tb + lane_off + kColH + col, v);
+        }
+    }
+    fence_proxy_async_smem();
+    tmem_fence_before_sync();
+    __syncthreads();
+
     constexpr uint32_t idG = umma_idesc_bf16(128, 128, true, true);
     constexpr uint32_t idYo = umma_idesc_bf16(128, 64, true, true);
     constexpr uint32_t idYd = umma_idesc_bf16(128, 64, false, false);
@@ -189,224 +267,236 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                       idG, kk > 0);
         umma_commit(&bar_g);
     };
+    auto issue_Yo = [&](int c) {
+        const uint32_t aC = sbase + Lay::kC + (c & 1) * 32768;
+#pragma unroll
+        for (int kk = 0; kk < N / 16; ++kk)
+            umma_bf16(tb + kColYo, umma_desc_mnmajor(aC, N, kk), umma_desc_mnmajor(aHs, N, kk),
+                      idYo, kk > 0);
+        umma_commit(&bar_yo);
+    };
     bool ok = true;
     if (tid == 0) {
-        issue_loads(0);
-        if (p.nchunks > 1)
-            issue_loads(1);
-        ok = mbar_wait(&bar_tma[0], 0u, p.timeout_ns) && ok;
         tmem_fence_after_sync();
+        ok = mbar_wait(&bar_tma[0], 0u, p.timeout_ns) && ok;
+        issue_Yo(0);
         issue_G(0);
     }
-    float dt_next = (half == 0 && r < p.L) ? dt_row[r] : 0.f;
+
+    // byte offsets of x[p][t] / y[p][t] (t = r) in a [2 slabs][64 p][64 t]
+    // tile for p = 8k + j: slab + p*128 + ((t%64/8 ^ j) << 4) + (t%8)*2
+    uint32_t off8[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        off8[j] = uint32_t(r >> 6) * 8192u + ((((uint32_t(r) & 63u) >> 3) ^ uint32_t(j)) << 4) +
+                  (uint32_t(r) & 7u) * 2u;
 
     for (int c = 0; c < p.nchunks; ++c) {
         const int buf = c & 1;
-        const uint32_t ph = uint32_t(c & 1);        // bar_g / bar_yo / bar_mma phase
-        const uint32_t tph = uint32_t((c >> 1) & 1);  // bar_tma[buf] phase
+        const uint32_t ph = uint32_t(c & 1);          // bar_g / bar_yo / bar_yd / bar_st
+        const uint32_t tph = uint32_t((c >> 1) & 1);  // bar_tma[buf]
         const int t0 = c * Q;
-        const uint32_t aC = sbase + Lay::kC + buf * 32768;
         const uint32_t aB = sbase + Lay::kB + buf * 32768;
         const uint32_t aX = sbase + Lay::kX + buf * 16384;
-        // ---- carried-in term Yo = C^T h_prev (h_prev in bf16 from the last chunk)
-        if (tid == 0) {
-            if (c > 0)
-                ok = mbar_wait(&bar_tma[buf], tph, p.timeout_ns) && ok;
-            tmem_fence_after_sync();
-#pragma unroll
-            for (int kk = 0; kk < N / 16; ++kk)
-                umma_bf16(tb + kColYo, umma_desc_mnmajor(aC, N, kk),
-                          umma_desc_mnmajor(aHs, N, kk), idYo, kk > 0);
-            umma_commit(&bar_yo);
-        }
-        // ---- step sizes and their cumulative sum over the chunk (first 128 threads)
-        const bool valid = t0 + r < p.L;
-        float dl = dt_next + bias;
-        if (p.softplus)
-            dl = ssd_softplus(dl);
-        dl = valid ? dl : 0.f;
-        float S = dl;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, S, o);
-            if (lane >= o)
-                S += v;
-        }
-        if (half == 0 && lane == 31)
-            s_wsum[warp] = S;
-        __syncthreads();
-        for (int w = 0; w < (warp & 3); ++w)
-            S += s_wsum[w];
-        if (half == 0) {
-            s_delta[r] = dl;
-            s_S[r] = S;
-        }
-        __syncthreads();
-        S = s_S[r];
-        dl = s_delta[r];
-        const float S_end = s_S[Q - 1];
-        if (half == 0)
-            s_g[r] = ex2_approx(a_l2 * (s_S[(r | 31)] - S)) * dl;
-        const float w_state = ex2_approx(a_l2 * (S_end - S)) * dl;  // x scale for h
-        const float e_row = ex2_approx(a_l2 * S);                     // Yo row scale
-        if (half == 0 && c + 1 < p.nchunks)
-            dt_next = (t0 + Q + r < p.L) ? dt_row[t0 + Q + r] : 0.f;
-        __syncthreads();
-        // every thread reads this chunk's x below
+        const uint8_t *xs = smem + Lay::kX + buf * 16384;
+
+        // ---- 1. x * w for the state product, w_s = 2^(cs_Q - cs_s) delta_s
+        //         = 2^(cs_Q - cs_e) s_sg[s]; units of (p, 8 tokens)
         ok = mbar_wait(&bar_tma[buf], tph, p.timeout_ns) && ok;
-        // ---- x * w for the state product (rows p of this half), h *= exp(A S_end)
         {
-            const uint8_t *xs = smem + Lay::kX + buf * 16384;
+            const float csQ = s_cs[Q - 1];
             uint8_t *xw = smem + Lay::kXw;
-            const uint32_t slab = uint32_t(r >> 6) * 8192u;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int pp = half * 32 + i;
-                const uint32_t off = slab + sw128_offset(pp, r & 63);
-                const float xv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xs + off));
-                *reinterpret_cast<__nv_bfloat16 *>(xw + off) = __float2bfloat16_rn(xv * w_state);
-            }
-            const float dec = ex2_approx(a_l2 * S_end);
-#pragma unroll
-            for (int cc = 0; cc < 32; cc += 16) {
-                float v[16];
-                tmem_ld16(tb + lane_off + kColH + colh + cc, v);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    v[i] *= dec;
-                tmem_st16(tb + lane_off + kColH + colh + cc, v);
+            for (int k = 0; k < 1024 / NT; ++k) {
+                const int u = tid + k * NT;
+                const int pp = u & 63, g = u >> 6;  // g: 8-token group 0..15
+                const float pf = ex2_approx(csQ - s_cs[(g >> 1) * 16 + 15]);
+                const float4 w0 = reinterpret_cast<const float4 *>(s_sg + g * 8)[0];
+                const float4 w1 = reinterpret_cast<const float4 *>(s_sg + g * 8)[1];
+                const uint32_t off = uint32_t(g >> 3) * 8192u + uint32_t(pp) * 128u +
+                                     ((uint32_t(g & 7) ^ uint32_t(pp & 7)) << 4);
+                const uint4 xv = *reinterpret_cast<const uint4 *>(xs + off);
+                const uint64_t PF = pk2(pf, pf);
+                const uint64_t s01 = mul2(pk2(w0.x, w0.y), PF), s23 = mul2(pk2(w0.z, w0.w), PF);
+                const uint64_t s45 = mul2(pk2(w1.x, w1.y), PF), s67 = mul2(pk2(w1.z, w1.w), PF);
+                const uint64_t x01 = mul2(bf2_to_f2(xv.x), s01), x23 = mul2(bf2_to_f2(xv.y), s23);
+                const uint64_t x45 = mul2(bf2_to_f2(xv.z), s45), x67 = mul2(bf2_to_f2(xv.w), s67);
+                uint4 o;
+                o.x = pack2_bf16(lo2(x01), hi2(x01));
+                o.y = pack2_bf16(lo2(x23), hi2(x23));
+                o.z = pack2_bf16(lo2(x45), hi2(x45));
+                o.w = pack2_bf16(lo2(x67), hi2(x67));
+                *reinterpret_cast<uint4 *>(xw + off) = o;
             }
         }
-        // ---- M = G masked by the decays: row t = r, pieces 4*half .. 4*half+3
+        // ---- 2. M: row t = r, pieces q = wg + NWG * j of 16 columns
+        const float cs_t = s_cs[r];
+        const float ey = ex2_approx(cs_t);  // Yo row scale, used in step 5
         ok = mbar_wait(&bar_g, ph, p.timeout_ns) && ok;
         tmem_fence_after_sync();
         {
-            const int bi = warp & 3;  // 32-token block of this row
-            uint8_t *mrow = smem + Lay::kM;
+            uint8_t *mt = smem + Lay::kM;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int q = half * 4 + qq;  // 16-column piece of the row
-                float m[16];
-                if (q < 2 * (bi + 1)) {       // warp-uniform
-                    float gv[16];
-                    tmem_ld16(tb + lane_off + kColG + q * 16, gv);
-                    const int bj = q >> 1;
-                    // exp(A (S_t - S_{end of block bj})) for a block before this row's
-                    const float fr = (bj < bi) ? ex2_approx(a_l2 * (S - s_S[32 * bj + 31])) : 0.f;
+            for (int j0 = 0; j0 < QPW; j0 += 2) {
+                float gv[2][16];
+                tmem_ld16x2(tb + lane_off + kColG + (wg + NWG * j0) * 16, gv[0],
+                            tb + lane_off + kColG + (wg + NWG * (j0 + 1)) * 16, gv[1]);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int s = q * 16 + i;
-                        float v;
-                        if (bj < bi)
-                            v = gv[i] * fr * s_g[s];
-                        else
-                            v = (s <= r) ? gv[i] * ex2_approx(a_l2 * (S - s_S[s])) * s_delta[s]
-                                         : 0.f;
-                        m[i] = v;
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int q = wg + NWG * (j0 + jj);
+                    float m[16];
+                    if (q < 2 * quarter) {
+                        // every row of this warp is past piece q: split decay
+                        float sg[16];
+                        lds16(s_sg + q * 16, sg);
+                        const float fr = ex2_approx(cs_t - s_cs[q * 16 + 15]);
+                        const uint64_t FR = pk2(fr, fr);
+#pragma unroll
+                        for (int i = 0; i < 16; i += 2) {
+                            const uint64_t v = mul2(
+                                mul2(pk2(gv[jj][i], gv[jj][i + 1]), pk2(sg[i], sg[i + 1])), FR);
+                            m[i] = lo2(v);
+                            m[i + 1] = hi2(v);
+                        }
+                    } else if (q <= 2 * quarter + 1) {
+                        // pieces holding this warp's diagonal: per element, masked
+                        float n2[16];
+                        lds16(s_n2 + q * 16, n2);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float e = ex2_approx(cs_t + n2[i]);
+                            m[i] = (q * 16 + i <= r) ? gv[jj][i] * e : 0.f;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            m[i] = 0.f;
                     }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        m[i] = 0.f;
-                }
-                const uint32_t slab = uint32_t(q >> 2) * 16384u;
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int col = (q & 3) * 16 + h2 * 8;
-                    uint4 pk;
-                    pk.x = ssd_pack2(m[h2 * 8 + 0], m[h2 * 8 + 1]);
-                    pk.y = ssd_pack2(m[h2 * 8 + 2], m[h2 * 8 + 3]);
-                    pk.z = ssd_pack2(m[h2 * 8 + 4], m[h2 * 8 + 5]);
-                    pk.w = ssd_pack2(m[h2 * 8 + 6], m[h2 * 8 + 7]);
-                    *reinterpret_cast<uint4 *>(mrow + slab + sw128_offset(r, col)) = pk;
+                    const uint32_t slab = uint32_t(q >> 2) * 16384u;
+                    const uint32_t col = uint32_t(q & 3) * 16u;
+                    sts16_bf16(mt, slab + sw128_offset(r, col), slab + sw128_offset(r, col + 8),
+                               m);
                 }
             }
         }
         fence_proxy_async_smem();
         tmem_fence_before_sync();
         __syncthreads();
-        // ---- Yd = M x^T, h += B (x w)^T, then the next chunk's C^T B
+        // ---- 3. Yd = M x^T; h += B (x w)^T; then the next chunk's C^T B
         if (tid == 0) {
             tmem_fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < Q / 16; ++kk)
                 umma_bf16(tb + kColYd, umma_desc_kmajor(aM, 128, kk), umma_desc_kmajor(aX, P, kk),
                           idYd, kk > 0);
+            umma_commit(&bar_yd);
 #pragma unroll
             for (int kk = 0; kk < Q / 16; ++kk)
                 umma_bf16(tb + kColH, umma_desc_kmajor(aB, N, kk), umma_desc_kmajor(aXw, P, kk),
                           idYd, 1u);
-            umma_commit(&bar_mma);
+            umma_commit(&bar_st);
             if (c + 1 < p.nchunks) {
-                ok = mbar_wait(&bar_tma[buf ^ 1], uint32_t(((c + 1) >> 1) & 1), p.timeout_ns) && ok;
+                ok = mbar_wait(&bar_tma[buf ^ 1], uint32_t(((c + 1) >> 1) & 1), p.timeout_ns) &&
+                     ok;
                 tmem_fence_after_sync();
                 issue_G(c + 1);
             }
         }
+        // ---- 4. step sizes of the next chunk (the per-token arrays are free
+        //         once every thread has passed the barrier above)
+        if (c + 1 < p.nchunks) {
+            cumsum(c + 1, dt_next);
+            if (wg == 0)
+                dt_next = (t0 + 2 * Q + r < p.L) ? dt_row[t0 + 2 * Q + r] : 0.f;
+        }
+        // ---- 5. y for token t = r, columns p of this warpgroup's slice
         ok = mbar_wait(&bar_yo, ph, p.timeout_ns) && ok;
-        ok = mbar_wait(&bar_mma, ph, p.timeout_ns) && ok;
+        ok = mbar_wait(&bar_yd, ph, p.timeout_ns) && ok;
         tmem_fence_after_sync();
-        // ---- outputs of token t = r, columns p of this half
         {
-            const uint8_t *xs = smem + Lay::kX + buf * 16384;
-            const uint32_t slab = uint32_t(r >> 6) * 8192u;
-            __nv_bfloat16 *yrow = p.y + int64_t(b) * p.y_bs + int64_t(hh * P) * p.y_cs + t0 + r;
+            uint8_t *ys = smem + Lay::kM;  // Yd has finished reading M
+            const bool valid = t0 + r < p.L;
             const __nv_bfloat16 *zrow =
                 GATE ? p.z + int64_t(b) * p.z_bs + int64_t(hh * P) * p.z_cs + t0 + r : nullptr;
 #pragma unroll
-            for (int cc = 0; cc < 32; cc += 16) {
+            for (int cc = 0; cc < PW; cc += 16) {
+                const int pbase = wg * PW + cc;
                 float yd[16], yo[16];
-                tmem_ld16(tb + lane_off + kColYd + colh + cc, yd);
-                tmem_ld16(tb + lane_off + kColYo + colh + cc, yo);
+                tmem_ld16x2(tb + lane_off + kColYd + pbase, yd, tb + lane_off + kColYo + pbase, yo);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int pp = half * 32 + cc + i;
-                    const float xv = __bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16 *>(xs + slab + sw128_offset(pp, r & 63)));
-                    float v = fmaf(e_row, yo[i], yd[i]);
+                    const uint32_t off = off8[i & 7] + uint32_t(pbase + i) * 128u;
+                    const float xv = __uint_as_float(
+                        uint32_t(*reinterpret_cast<const uint16_t *>(xs + off)) << 16);
+                    float v = fmaf(ey, yo[i], yd[i]);
                     v = fmaf(dsk, xv, v);
-                    if (GATE && valid) {
-                        const float zv = __bfloat162float(zrow[int64_t(pp) * p.z_cs]);
+                    if (GATE) {
+                        const float zv =
+                            valid ? __bfloat162float(zrow[int64_t(pbase + i) * p.z_cs]) : 0.f;
                         v *= zv / (1.f + __expf(-zv));
                     }
-                    if (valid)
-                        yrow[int64_t(pp) * p.y_cs] = __float2bfloat16_rn(v);
+                    *reinterpret_cast<__nv_bfloat16 *>(ys + off) = __float2bfloat16_rn(v);
                 }
             }
-            // h (state n = r) -> bf16 copy for the next chunk's Yo; final state out
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_3d(&tm_Y, smem + Lay::kM, t0, hh * P, b);
+            if (t0 + 64 < p.L)
+                tma_store_3d(&tm_Y, smem + Lay::kM + 8192, t0 + 64, hh * P, b);
+            bulk_commit();
+        }
+        // ---- 6. state n = r: bf16 copy for Yo(c+1), final state, decay into chunk c+1
+        ok = mbar_wait(&bar_st, ph, p.timeout_ns) && ok;
+        tmem_fence_after_sync();
+        {
             uint8_t *hs = smem + Lay::kHs;
-            float *ls = (p.last_state && c == p.nchunks - 1)
+            const bool last = c == p.nchunks - 1;
+            const float alpha = last ? 1.f : ex2_approx(s_cs[Q - 1]);  // chunk c+1's decay
+            float *ls = (p.last_state && last)
                             ? p.last_state + (int64_t(b) * p.H + hh) * P * N + r
                             : nullptr;
 #pragma unroll
-            for (int cc = 0; cc < 32; cc += 16) {
+            for (int cc = 0; cc < PW; cc += 16) {
+                const uint32_t col = uint32_t(wg * PW + cc);
                 float hv[16];
-                tmem_ld16(tb + lane_off + kColH + colh + cc, hv);
+                tmem_ld16(tb + lane_off + kColH + col, hv);
+                if (!last) {
+                    sts16_bf16(hs, sw128_offset(r, col), sw128_offset(r, col + 8), hv);
+                    const uint64_t AL = pk2(alpha, alpha);
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint4 pk;
-                    pk.x = ssd_pack2(hv[h2 * 8 + 0], hv[h2 * 8 + 1]);
-                    pk.y = ssd_pack2(hv[h2 * 8 + 2], hv[h2 * 8 + 3]);
-                    pk.z = ssd_pack2(hv[h2 * 8 + 4], hv[h2 * 8 + 5]);
-                    pk.w = ssd_pack2(hv[h2 * 8 + 6], hv[h2 * 8 + 7]);
-                    *reinterpret_cast<uint4 *>(hs + sw128_offset(r, colh + cc + h2 * 8)) = pk;
-                }
-                if (ls) {
+                    for (int i = 0; i < 16; i += 2) {
+                        const uint64_t v = mul2(pk2(hv[i], hv[i + 1]), AL);
+                        hv[i] = lo2(v);
+                        hv[i + 1] = hi2(v);
+                    }
+                    tmem_st16(tb + lane_off + kColH + col, hv);
+                } else if (ls) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        ls[int64_t(colh + cc + i) * N] = hv[i];
+                        ls[int64_t(col + i) * N] = hv[i];
                 }
             }
         }
         fence_proxy_async_smem();
         tmem_fence_before_sync();
+        if (tid == 0)
+            bulk_wait_read<0>();  // the y tile has left the M buffer
         __syncthreads();
-        // this chunk's C, B, x buffers are free: bring in chunk c + 2
-        if (tid == 0 && c + 2 < p.nchunks) {
-            fence_proxy_async_smem();
-            issue_loads(c + 2);
+        // ---- 7. Yo(c+1) from the new bf16 state; chunk c+2 into this buffer
+        if (tid == 0) {
+            tmem_fence_after_sync();
+            if (c + 1 < p.nchunks)
+                issue_Yo(c + 1);
+            if (c + 2 < p.nchunks) {
+                fence_proxy_async_smem();
+                issue_loads(c + 2);
+            }
         }
     }
+    if (tid == 0)
+        bulk_wait_all<0>();
     if (!ok)
         atomicOr(p.err, 4u);
     tmem_fence_after_sync();
