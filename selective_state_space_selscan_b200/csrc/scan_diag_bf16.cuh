@@ -302,19 +302,22 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
         uint8_t *y_row = ytile + (it & 1) * TILE + ch * 128;
         const int t0 = inf.y;
 
+        // The 8-token blocks are software-pipelined: while block j runs its
+        // eight steps, the same basic block prepares block j + 1 (softplus,
+        // w, 1/w, decay base: special-function latency) and finishes block
+        // j - 1 (reduce-scatter, D skip, gate, store), so the latencies of
+        // those two phases hide under the step arithmetic.
         auto run = [&](auto pow_tag) {
             constexpr bool POWC = decltype(pow_tag)::value;
-#pragma unroll 1
-            for (int j = 0; j < TC / 8; ++j) {
-                // this lane prepares tokens 4pp .. 4pp+3 of the 8-token block
-                const int off = ((j ^ swz) << 4) + pp * 8;
+            float rv[4], wv[4], rwv[4], uv[4];  // prepared block (this lane's 4 tokens)
+            uint2 zq = make_uint2(0, 0);
+            auto prep = [&](int jb) {
+                const int off = ((jb ^ swz) << 4) + pp * 8;
                 const uint2 uq = *reinterpret_cast<const uint2 *>(u_row + off);
                 const uint2 dq = *reinterpret_cast<const uint2 *>(dl_row + off);
-                uint2 zq = make_uint2(0, 0);
                 if (GATE)
                     zq = *reinterpret_cast<const uint2 *>(z_row + off);
-                const int tmine = t0 + j * 8 + pp * 4;
-                float uv[4], rv[4], wv[4], rwv[4];
+                const int tmine = t0 + jb * 8 + pp * 4;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint32_t uw = kk < 2 ? uq.x : uq.y, dw = kk < 2 ? dq.x : dq.y;
@@ -328,7 +331,34 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                     rwv[kk] = rcp_approx(wv[kk]);
                     rv[kk] = POWC ? ex2_approx(dt * a0) : dt;
                 }
-                // both lanes need r, w, 1/w of all 8 tokens
+            };
+            // finished-block state carried into the next iteration
+            float yp_prev[8], w_prev4[4], u_prev4[4];
+            uint2 z_prev = make_uint2(0, 0);
+            int off_prev = 0;
+            auto finish = [&]() {
+                // reduce-scatter: this lane finishes tokens 4pp .. 4pp+3
+                float yo[4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const float send = pp ? yp_prev[kk] : yp_prev[4 + kk];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                    float v = ((pp ? yp_prev[4 + kk] : yp_prev[kk]) + recv) * w_prev4[kk];
+                    v = fmaf(dsk, u_prev4[kk], v);
+                    if (GATE) {
+                        const uint32_t zw = kk < 2 ? z_prev.x : z_prev.y;
+                        const float zv = __uint_as_float((kk & 1) ? (zw & 0xffff0000u) : (zw << 16));
+                        v *= silu_fast(zv);
+                    }
+                    yo[kk] = v;
+                }
+                *reinterpret_cast<uint2 *>(y_row + off_prev) =
+                    make_uint2(pack2_bf16(yo[0], yo[1]), pack2_bf16(yo[2], yo[3]));
+            };
+            prep(0);
+#pragma unroll 2
+            for (int j = 0; j < TC / 8; ++j) {
+                // both lanes need r, w, 1/w of all 8 tokens of block j
                 float r8[8], w8[8], rw8[8];
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
@@ -342,6 +372,16 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                     rw8[kk] = pp ? rwo : rwv[kk];
                     rw8[4 + kk] = pp ? rwv[kk] : rwo;
                 }
+                float wmine[4], umine[4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    wmine[kk] = wv[kk];
+                    umine[kk] = uv[kk];
+                }
+                const uint2 zmine = zq;
+                if (j > 0)
+                    finish();            // block j - 1
+                prep((j + 1) & 7);       // block j + 1 (wraps harmlessly after the last)
                 float yp[8];
                 const float *bcb_blk = bcb + j * 8 * 32 + pp * 16;
 #pragma unroll
@@ -363,24 +403,18 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                     yp[i] = lo2(Y) + hi2(Y);
                 }
                 wprev = w8[7];
-                // reduce-scatter: this lane finishes tokens 4pp .. 4pp+3
-                float yo[4];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    yp_prev[i] = yp[i];
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const float send = pp ? yp[kk] : yp[4 + kk];
-                    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-                    float v = ((pp ? yp[4 + kk] : yp[kk]) + recv) * wv[kk];
-                    v = fmaf(dsk, uv[kk], v);
-                    if (GATE) {
-                        const uint32_t zw = kk < 2 ? zq.x : zq.y;
-                        const float zv = __uint_as_float((kk & 1) ? (zw & 0xffff0000u) : (zw << 16));
-                        v *= silu_fast(zv);
-                    }
-                    yo[kk] = v;
+                    w_prev4[kk] = wmine[kk];
+                    u_prev4[kk] = umine[kk];
                 }
-                *reinterpret_cast<uint2 *>(y_row + off) =
-                    make_uint2(pack2_bf16(yo[0], yo[1]), pack2_bf16(yo[2], yo[3]));
+                z_prev = zmine;
+                off_prev = ((j ^ swz) << 4) + pp * 8;
             }
+            finish();  // last block
         };
         if (pow_path)
             run(std::true_type{});
