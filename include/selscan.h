@@ -278,6 +278,15 @@ SELSCAN_API const char *selscan_strerror(selscan_status status);
 /* SELSCAN_VERSION of the built library. */
 SELSCAN_API int selscan_version(void);
 
+/*
+ * Number of kernels this library has launched in the calling process so far
+ * (all entry points, all devices).  A selscan_fwd call launches one kernel,
+ * or two when it uses the two-pass form (few channel tiles, long
+ * sequences); the other entry points launch one.  Benchmarks read it around
+ * a timed region to report how many of the library's kernels ran in it.
+ */
+SELSCAN_API unsigned long long selscan_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

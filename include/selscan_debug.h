@@ -22,6 +22,18 @@ extern "C" {
  */
 SELSCAN_API void selscan_debug_withhold_carry(int unit);
 
+/*
+ * Choose how the fast bf16 diagonal scan links the segments of a channel
+ * tile in subsequent selscan_fwd calls: 0 = one pass with carries chained
+ * from segment to segment; 1 = two passes (every segment's end state from
+ * zero and its sum of step sizes, then the output pass folding those into
+ * each segment's initial state); -1 (default) = the library's choice (two
+ * passes when there are at most half as many tiles as SMs).  Both forms
+ * compute the same recurrence; the hook lets tests cover both on the same
+ * inputs.  Single-segment launches are unaffected.
+ */
+SELSCAN_API void selscan_debug_diag_mode(int mode);
+
 #ifdef __cplusplus
 }
 #endif

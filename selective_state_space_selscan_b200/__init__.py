@@ -29,7 +29,7 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 # entry points declared in include/selscan.h
 EXPORTS = ("selscan_fwd", "selscan_fwd_h0", "selscan_fwd_scalarA", "selscan_fwd_scalarA_h0",
            "selscan_fwd_noalloc", "selscan_step", "selscan_step_scalarA", "selscan_check",
-           "selscan_strerror", "selscan_version")
+           "selscan_strerror", "selscan_version", "selscan_launch_count")
 
 
 class SelscanError(RuntimeError):
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.selscan_strerror.argtypes = [ctypes.c_int]
         L.selscan_strerror.restype = ctypes.c_char_p
         L.selscan_version.argtypes = []
+        L.selscan_launch_count.argtypes = []
+        L.selscan_launch_count.restype = ctypes.c_ulonglong
         for f in (L.selscan_fwd, L.selscan_fwd_scalarA, L.selscan_check,
                   L.selscan_version):
             f.restype = ctypes.c_int
@@ -87,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.selscan_step_scalarA.restype = ctypes.c_int
         L.selscan_debug_withhold_carry.argtypes = [ctypes.c_int]
         L.selscan_debug_withhold_carry.restype = None
+        L.selscan_debug_diag_mode.argtypes = [ctypes.c_int]
+        L.selscan_debug_diag_mode.restype = None
         _lib = L
     return _lib
 
@@ -100,6 +104,11 @@ def _strerror(status: int) -> str:
 
 def version() -> int:
     return lib().selscan_version()
+
+
+def launch_count() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(lib().selscan_launch_count())
 
 
 def describe(t, dtype_code=None) -> SelscanTensor | None:
@@ -255,6 +264,11 @@ def check(stream=None) -> None:
     rc = lib().selscan_check(_stream_handle(stream))
     if rc != 0:
         raise SelscanError(rc, "selscan_check")
+
+
+def debug_diag_mode(mode: int) -> None:
+    """Test hook: 0 = chained carries, 1 = two-pass form, -1 = automatic."""
+    lib().selscan_debug_diag_mode(int(mode))
 
 
 def debug_withhold_carry(unit: int) -> None:

@@ -52,6 +52,8 @@ struct DiagParams {
     const float *delta_bias;  // (dim) or null
     const float *Dskip;   // (dim) or null
     const float *h0;      // (batch, dim, 16) or null
+    float *agg;           // two-pass form: [units][CH][parity][8] segment end states
+    float *agg_sd;        // two-pass form: [units][CH] sums of step sizes
     float *last_state;    // (batch, dim, 16) or null
     int softplus;
     unsigned int *ticket;  // zeroed before launch

@@ -80,7 +80,13 @@ __device__ __forceinline__ void decay_pairs(uint64_t (&V)[4], float r, float c, 
     }
 }
 
-template <int CH, int STAGES, bool GATE, bool SOFTPLUS>
+// MODE 0: one pass, segments chained through published carries.
+// MODE 1: aggregate pass of the two-pass form: every segment scans from a
+//         zero state and records its end state and the sum of its step sizes
+//         (reads u, delta and B only; writes no y).
+// MODE 2: output pass of the two-pass form: every segment starts from the
+//         state folded from the aggregates of the segments before it.
+template <int CH, int STAGES, bool GATE, bool SOFTPLUS, int MODE = 0>
 __global__ void __launch_bounds__(2 * CH + 32, 1)
 scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                       const __grid_constant__ CUtensorMap tm_delta,
@@ -131,7 +137,8 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             if (GATE)
                 prefetch_tmap(&tm_z);
             prefetch_tmap(&tm_B);
-            prefetch_tmap(&tm_C);
+            if (MODE != 1)
+                prefetch_tmap(&tm_C);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -156,14 +163,16 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                                             (c == nch - 1 ? kInfoLast : 0),
                                         0);
                     uint8_t *st = stages + s * Lay::kStage;
-                    mbar_arrive_expect_tx(&full[s], Lay::kStage);
+                    mbar_arrive_expect_tx(&full[s], MODE == 1 ? 2 * TILE + Lay::kBCTile
+                                                              : Lay::kStage);
                     tma_load_3d(st, &tm_u, &full[s], t0, d0, b);
                     tma_load_3d(st + TILE, &tm_delta, &full[s], t0, d0, b);
-                    if (GATE)
+                    if (GATE && MODE != 1)
                         tma_load_3d(st + 2 * TILE, &tm_z, &full[s], t0, d0, b);
                     uint8_t *bct = st + (GATE ? 3 : 2) * TILE;
                     tma_load_3d(bct, &tm_B, &full[s], t0, 0, b);
-                    tma_load_3d(bct + Lay::kBCTile, &tm_C, &full[s], t0, 0, b);
+                    if (MODE != 1)
+                        tma_load_3d(bct + Lay::kBCTile, &tm_C, &full[s], t0, 0, b);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -192,6 +201,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
         g[jj] = pk2(0.f, 0.f);
     uint64_t apair[4];           // A*log2e of this lane's states, paired (general path)
     float a0 = 0.f, bias = 0.f, dsk = 0.f, wprev = 1.f;
+    float sdel = 0.f;            // this lane's sum of step sizes in the segment (MODE 1)
     bool pow_path = true;
     int unit = -1, k = 0, b = 0, d0 = 0, d = 0;
     int prev_t0 = 0, prev_d0 = 0, prev_b = 0;
@@ -234,12 +244,32 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             bias = (p.delta_bias && live) ? p.delta_bias[d] : 0.f;
             dsk = (p.Dskip && live) ? p.Dskip[d] : 0.f;
             wprev = 1.f;  // g starts as h_in (w_{-1} := 1)
+            sdel = 0.f;
             float hv[8];
-            if (k == 0) {
+            if (MODE == 1) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    hv[j] = 0.f;
+            } else if (k == 0 || MODE == 2) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     hv[j] = (p.h0 && live) ? p.h0[(size_t(b) * p.dim + d) * kDiagN + 2 * j + pp]
                                            : 0.f;
+                if (MODE == 2) {
+                    // h_in = fold over the earlier segments j of this tile:
+                    // h = exp(A * sum(delta_j)) h + E_j
+                    for (int jseg = 0; jseg < k; ++jseg) {
+                        const size_t uj = size_t(jseg) * G + gg;
+                        const float sd = __ldcg(p.agg_sd + uj * CH + ch);
+                        const float4 *e = reinterpret_cast<const float4 *>(
+                            p.agg + (uj * CH + ch) * kDiagN + pp * 8);
+                        const float4 e0 = __ldcg(e), e1 = __ldcg(e + 1);
+                        const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            hv[j] = fmaf(ex2_approx(al[j] * sd), hv[j], ev[j]);
+                    }
+                }
             } else {
                 const int prev = unit - G;
                 const uint32_t *flag = p.flags + size_t(prev) * CW + warp;
@@ -273,7 +303,12 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
         const uint8_t *Ct = Bt + Lay::kBCTile;
         float *bcb = bcp + (it & 1) * TC * 32;
         // B, C -> fp32, token-major: [t][parity p][B: X[p], X[p+2], ..., X[p+14]][C: same]
-        for (int q = tid; arrived && q < TC * 32; q += CONS) {
+        for (int q2 = tid; arrived && q2 < TC * (MODE == 1 ? 16 : 32); q2 += CONS) {
+            // MODE 1 stages B only: (token, parity, k8) -> its slot in the
+            // [t][parity][B 8 | C 8] row
+            const int q = MODE == 1
+                              ? ((q2 >> 4) << 5) + (((q2 >> 3) & 1) << 4) + (q2 & 7)
+                              : q2;
             const int t = q >> 5, rest = q & 31;
             const int par = rest >> 4, isC = (rest >> 3) & 1, k8 = rest & 7;
             const int n = 2 * k8 + par;
@@ -291,7 +326,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             *abort_flag = 1;
             break;
         }
-        if (tid == 0 && it > 0) {
+        if (MODE != 1 && tid == 0 && it > 0) {
             tma_store_3d(&tm_y, ytile + ((it - 1) & 1) * TILE, prev_t0, prev_d0, prev_b);
             bulk_commit();
         }
@@ -310,12 +345,13 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
         auto run = [&](auto pow_tag) {
             constexpr bool POWC = decltype(pow_tag)::value;
             float rv[4], wv[4], rwv[4], uv[4];  // prepared block (this lane's 4 tokens)
+            float dts[4];                       // its step sizes (aggregate pass)
             uint2 zq = make_uint2(0, 0);
             auto prep = [&](int jb) {
                 const int off = ((jb ^ swz) << 4) + pp * 8;
                 const uint2 uq = *reinterpret_cast<const uint2 *>(u_row + off);
                 const uint2 dq = *reinterpret_cast<const uint2 *>(dl_row + off);
-                if (GATE)
+                if (GATE && MODE != 1)
                     zq = *reinterpret_cast<const uint2 *>(z_row + off);
                 const int tmine = t0 + jb * 8 + pp * 4;
 #pragma unroll
@@ -326,6 +362,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                     const float x = dv + bias;
                     float dt = SOFTPLUS ? softplus_fast(x) : x;
                     dt = (tmine + kk < p.L) ? dt : 0.f;  // padding past L: identity step
+                    dts[kk] = dt;
                     const float wr = dt * uv[kk];
                     wv[kk] = copysignf(fmaxf(fabsf(wr), kWMin), wr);
                     rwv[kk] = rcp_approx(wv[kk]);
@@ -379,7 +416,9 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                     umine[kk] = uv[kk];
                 }
                 const uint2 zmine = zq;
-                if (j > 0)
+                if (MODE == 1)
+                    sdel += (dts[0] + dts[1]) + (dts[2] + dts[3]);
+                if (MODE != 1 && j > 0)
                     finish();            // block j - 1
                 prep((j + 1) & 7);       // block j + 1 (wraps harmlessly after the last)
                 float yp[8];
@@ -388,13 +427,18 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                 for (int i = 0; i < 8; ++i) {
                     const float c = (i == 0 ? wprev : w8[i - 1]) * rw8[i];
                     const ulonglong2 *bq = reinterpret_cast<const ulonglong2 *>(bcb_blk + i * 32);
-                    const ulonglong2 b01 = bq[0], b23 = bq[1], c01 = bq[2], c23 = bq[3];
+                    const ulonglong2 b01 = bq[0], b23 = bq[1];
                     uint64_t V[4];
                     decay_pairs<POWC>(V, r8[i], c, pp, apair);
                     g[0] = fma2(V[0], g[0], b01.x);
                     g[1] = fma2(V[1], g[1], b01.y);
                     g[2] = fma2(V[2], g[2], b23.x);
                     g[3] = fma2(V[3], g[3], b23.y);
+                    if (MODE == 1) {
+                        yp[i] = 0.f;
+                        continue;
+                    }
+                    const ulonglong2 c01 = bq[2], c23 = bq[3];
                     uint64_t Ya = mul2(c01.x, g[0]);
                     uint64_t Yb = mul2(c01.y, g[1]);
                     Ya = fma2(c23.x, g[2], Ya);
@@ -414,7 +458,8 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                 z_prev = zmine;
                 off_prev = ((j ^ swz) << 4) + pp * 8;
             }
-            finish();  // last block
+            if (MODE != 1)
+                finish();  // last block
         };
         if (pow_path)
             run(std::true_type{});
@@ -436,7 +481,16 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                 g[jj] = pk2(hv[2 * jj], hv[2 * jj + 1]);
             }
             wprev = 1.f;
-            if (k < p.num_segs - 1) {
+            if (MODE == 1) {
+                // aggregate of this segment: end state from zero, sum of steps
+                const size_t ua = size_t(unit) * CH + ch;
+                float4 *dst = reinterpret_cast<float4 *>(p.agg + ua * kDiagN + pp * 8);
+                __stcg(dst, make_float4(hv[0], hv[1], hv[2], hv[3]));
+                __stcg(dst + 1, make_float4(hv[4], hv[5], hv[6], hv[7]));
+                const float sd = sdel + __shfl_xor_sync(0xffffffffu, sdel, 1);
+                if (pp == 0)
+                    __stcg(p.agg_sd + ua, sd);
+            } else if (MODE == 0 && k < p.num_segs - 1) {
                 float4 *dst = reinterpret_cast<float4 *>(
                     p.carry + (size_t(unit) * CH + ch) * kDiagN + pp * 8);
                 dst[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
@@ -445,7 +499,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                 __syncwarp();
                 if (lane == 0 && unit != p.dbg_skip_publish)
                     st_release_gpu(p.flags + size_t(unit) * CW + warp, 1u);
-            } else if (p.last_state && d < p.dim) {
+            } else if (p.last_state && d < p.dim && k == p.num_segs - 1) {
                 float *dst = p.last_state + (size_t(b) * p.dim + d) * kDiagN;
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
@@ -464,7 +518,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
 
     named_bar_sync(1, CONS);
     if (tid == 0) {
-        if (it > 0 && !*abort_flag) {
+        if (MODE != 1 && it > 0 && !*abort_flag) {
             tma_store_3d(&tm_y, ytile + ((it - 1) & 1) * TILE, prev_t0, prev_d0, prev_b);
             bulk_commit();
         }

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <atomic>
 #include <mutex>
 #include <algorithm>
 
@@ -22,6 +23,18 @@ using namespace selscan;
 
 // Device-side error word: bounded waits that give up OR a bit in here.
 __device__ unsigned int g_selscan_err = 0;
+
+// Kernels launched by this library in this process (selscan_launch_count).
+static std::atomic<unsigned long long> g_launches{0};
+
+// Status of the launch just made; counts it when it succeeded.
+static cudaError_t counted_launch()
+{
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess)
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
 
 namespace {
 
@@ -207,7 +220,33 @@ struct DiagVariant<1, __nv_bfloat16, CH, STAGES, GATE, SOFTPLUS> {
     static constexpr int kConsWarps = 2 * CH / 32;
     static constexpr int kSmem = DiagFastLayout<CH, STAGES, GATE>::kAlloc;
     static constexpr auto kernel() { return scan_diag_bf16_kernel<CH, STAGES, GATE, SOFTPLUS>; }
+    // two-pass form: MODE 1 reads no z, MODE 2 is the full output pass
+    template <int MODE>
+    static constexpr auto kernel_mode()
+    {
+        return scan_diag_bf16_kernel<CH, STAGES, GATE && MODE != 1, SOFTPLUS, MODE>;
+    }
+    template <int MODE>
+    static constexpr int smem_mode()
+    {
+        return DiagFastLayout<CH, STAGES, GATE && MODE != 1>::kAlloc;
+    }
 };
+
+// Dynamic shared memory limit of a kernel, raised once per device.
+template <typename K>
+bool ensure_smem(K kern, int bytes, int dev, bool (&done)[kMaxDevices])
+{
+    if (done[dev])
+        return true;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return false;
+    done[dev] = true;
+    return true;
+}
+
+int g_dbg_diag_mode = -1;  // test hook, see selscan_debug_diag_mode
 
 template <int KIND, typename T, int CH, int STAGES, bool GATE, bool SOFTPLUS>
 selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
@@ -268,6 +307,65 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
         return SELSCAN_ERR_UNSUPPORTED;
     prm.total_units = int(units);
 
+    // Few tiles and several segments: a chain of carries would leave most
+    // SMs waiting, so use the two-pass form (aggregates, then output).
+    if constexpr (KIND == 1) {
+    const bool two_pass = g_dbg_diag_mode >= 0 ? (g_dbg_diag_mode == 1 && S > 1)
+                                               : (S > 1 && 2 * int64_t(G) <= sm_count);
+    if (two_pass) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const int64_t agg_units = int64_t(G) * (S - 1);  // the last segment needs none
+        // scratch: 2 tickets | agg[agg_units][CH][16] | agg_sd[agg_units][CH] | h0 copy
+        // Every output-pass segment reads the initial state, and segments no
+        // longer wait for one another, so they read a copy: the caller's h0
+        // may be the last_state buffer that the last segments overwrite.
+        const size_t head = 256;
+        const size_t agg_bytes = size_t(agg_units) * CH * kDiagN * 4;
+        const size_t sd_bytes = ((size_t(agg_units) * CH * 4 + 255) / 256) * 256;
+        const size_t h0_bytes = prm.h0 ? size_t(batch) * dim * kDiagN * 4 : 0;
+        void *ws = nullptr;
+        if (cudaMallocAsync(&ws, head + agg_bytes + sd_bytes + h0_bytes, stream) != cudaSuccess)
+            return SELSCAN_ERR_CUDA;
+        uint8_t *wsb = static_cast<uint8_t *>(ws);
+        if (cudaMemsetAsync(wsb, 0, head, stream) != cudaSuccess ||
+            (prm.h0 && cudaMemcpyAsync(wsb + head + agg_bytes + sd_bytes, prm.h0, h0_bytes,
+                                       cudaMemcpyDeviceToDevice, stream) != cudaSuccess)) {
+            cudaFreeAsync(ws, stream);
+            return SELSCAN_ERR_CUDA;
+        }
+        if (prm.h0)
+            prm.h0 = reinterpret_cast<const float *>(wsb + head + agg_bytes + sd_bytes);
+        prm.flags = nullptr;
+        prm.carry = nullptr;
+        prm.agg = reinterpret_cast<float *>(wsb + head);
+        prm.agg_sd = reinterpret_cast<float *>(wsb + head + agg_bytes);
+        prm.dbg_skip_publish = -1;
+        DiagParams p1 = prm, p2 = prm;
+        p1.ticket = reinterpret_cast<unsigned int *>(wsb);
+        p1.total_units = int(agg_units);
+        p2.ticket = reinterpret_cast<unsigned int *>(wsb + 64);
+        auto k1 = V::template kernel_mode<1>();
+        auto k2 = V::template kernel_mode<2>();
+        static bool done1[kMaxDevices] = {}, done2[kMaxDevices] = {};
+        if (!ensure_smem(k1, V::template smem_mode<1>(), dev, done1) ||
+            !ensure_smem(k2, V::template smem_mode<2>(), dev, done2)) {
+            cudaFreeAsync(ws, stream);
+            return SELSCAN_ERR_CUDA;
+        }
+        k1<<<int(std::min<int64_t>(ctas_max, agg_units)), V::kThreads,
+             V::template smem_mode<1>(), stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, p1);
+        cudaError_t le = counted_launch();
+        if (le == cudaSuccess) {
+            k2<<<int(std::min<int64_t>(ctas_max, units)), V::kThreads,
+                 V::template smem_mode<2>(), stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, p2);
+            le = counted_launch();
+        }
+        cudaFreeAsync(ws, stream);
+        return le == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+    }
+    }
+
     // scratch: ticket | flags[units][CW] | carry[units][CH][16]
     const size_t head = 256;
     const size_t flag_bytes = ((size_t(units) * CW * 4 + 255) / 256) * 256;
@@ -300,7 +398,7 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
     }
     const int grid = int(std::min<int64_t>(ctas_max, units));
     kern<<<grid, V::kThreads, V::kSmem, stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, prm);
-    const cudaError_t le = cudaGetLastError();
+    const cudaError_t le = counted_launch();
     cudaFreeAsync(ws, stream);
     return le == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
 }
@@ -327,9 +425,16 @@ const char *selscan_strerror(selscan_status s)
 
 int selscan_version(void) { return SELSCAN_VERSION; }
 
+unsigned long long selscan_launch_count(void)
+{
+    return g_launches.load(std::memory_order_relaxed);
+}
+
 // Test hook (not part of the public header's stable surface): withhold the
 // carry flag of one work unit so that its successor's bounded wait expires.
 // -1 switches it off.
+void selscan_debug_diag_mode(int mode) { g_dbg_diag_mode = mode; }
+
 void selscan_debug_withhold_carry(int unit) { g_dbg_skip_publish = unit; }
 
 selscan_status selscan_check(cudaStream_t stream)
@@ -604,7 +709,7 @@ static selscan_status scalarA_impl(const selscan_tensor *x, const selscan_tensor
         return SELSCAN_ERR_UNSUPPORTED;
     kern<<<unsigned(grid), kSsdWG * 128, SsdLayout::kAlloc, stream>>>(tm_C, tm_B, tm_X, tm_Y,
                                                                        prm);
-    return cudaGetLastError() == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+    return counted_launch() == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
 }
 
 selscan_status selscan_fwd_scalarA(const selscan_tensor *x, const selscan_tensor *dt,
@@ -735,7 +840,7 @@ selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor
     }
     const int grid = int(std::min<int64_t>(ctas_max, units));
     kern<<<grid, V::kThreads, V::kSmem, stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, prm);
-    return cudaGetLastError() == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+    return counted_launch() == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
 }
 
 }  // namespace
@@ -916,7 +1021,7 @@ cudaError_t launch_step(const StepParams &prm, int64_t batch, int tpc, cudaStrea
     case 8: step_kernel<T, 8, SCALAR><<<grid, 256, 0, stream>>>(prm); break;
     default: step_kernel<T, 16, SCALAR><<<grid, 256, 0, stream>>>(prm); break;
     }
-    return cudaGetLastError();
+    return counted_launch();
 }
 
 // Shared by the diagonal and the scalar (Mamba-2) step.  `scalar` selects

@@ -200,3 +200,65 @@ def test_full_size_config_sampled(cfg):
     assert_parity(inp, np.concatenate(ys, 1), np.concatenate(hsl, 1),
                   np.concatenate(yr, 1), np.concatenate(hr, 1), f"config {cfg}")
     assert np.isfinite(y).all()
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_chained_and_two_pass_forms(mode):
+    """Two channel tiles, 32 segments: the carries chained from segment to
+    segment (mode 0) and the two-pass form (mode 1: segment aggregates, then
+    the output pass) both reproduce the oracle, with an initial state."""
+    import selective_state_space_selscan_b200 as ss
+    torch = _torch()
+    inp = synthetic.make_diag(1, 256, 16, 8192, dtype="bf16", seed=31)
+    h0 = np.random.default_rng(4).standard_normal((1, 256, 16)).astype(np.float32)
+    ss.debug_diag_mode(mode)
+    try:
+        y, hs = ss.selscan_fwd(dev(inp["u"], "bf16"), dev(inp["delta"], "bf16"), dev32(inp["A"]),
+                               dev(inp["B"], "bf16"), dev(inp["C"], "bf16"), D=dev32(inp["D"]),
+                               z=dev(inp["z"], "bf16"), delta_bias=dev32(inp["delta_bias"]),
+                               h0=torch.from_numpy(h0).cuda())
+        ss.check()
+    finally:
+        ss.debug_diag_mode(-1)
+    y_ref, hs_ref = oracle.selscan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                                   D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"], h0=h0)
+    assert_parity(inp, y.float().cpu().numpy(), hs.cpu().numpy(), y_ref, hs_ref, f"mode {mode}")
+
+
+def test_withheld_carry_times_out():
+    """Failure detection without a GPU fault: one work unit withholds its
+    carry flag, its successor gives up after the (short) wait limit, and
+    selscan_check reports SELSCAN_ERR_TIMEOUT; the next call runs clean.
+    Runs in a child process so that the short limit applies only there."""
+    import os
+    import subprocess
+    import sys
+    code = r'''
+import numpy as np, torch, sys
+sys.path.insert(0, sys.argv[1])
+import selective_state_space_selscan_b200 as ss, synthetic
+inp = synthetic.make_diag(1, 256, 16, 4096, dtype="bf16", seed=32)
+cv = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(torch.bfloat16)
+f = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda().float()
+args = (cv(inp["u"]), cv(inp["delta"]), f(inp["A"]), cv(inp["B"]), cv(inp["C"]))
+kw = dict(D=f(inp["D"]), z=cv(inp["z"]), delta_bias=f(inp["delta_bias"]))
+ss.debug_diag_mode(0)
+ss.debug_withhold_carry(3)      # unit 3 = segment 1 of tile 1 (two tiles)
+ss.selscan_fwd(*args, **kw)
+try:
+    ss.check()
+    print("NO_TIMEOUT")
+except ss.SelscanError as e:
+    print("STATUS", e.name)
+ss.debug_withhold_carry(-1)
+y, hs = ss.selscan_fwd(*args, **kw)
+ss.check()
+print("CLEAN", bool(torch.isfinite(y.float()).all()))
+'''
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SELSCAN_WAIT_TIMEOUT_MS="300")
+    r = subprocess.run([sys.executable, "-c", code, root], capture_output=True, text=True,
+                       env=env, timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert "STATUS SELSCAN_ERR_TIMEOUT" in r.stdout, r.stdout
+    assert "CLEAN True" in r.stdout, r.stdout
