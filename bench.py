@@ -40,12 +40,15 @@ METRIC = "selective-scan Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU"
 # ncu captures summarised in profiles/, keyed by config and the kernel they
 # were taken on; reported as roofline.traffic only for that kernel.
 NCU_TRAFFIC = {
-    # config 2 captured at L = 2048, scaled by tokens to L = 4096 (see profiles/)
-    2: ("scan_diag_bf16_kernel pairs v3", 647.2e6),
-    4: ("ssd_scalarA_kernel v1", 109.0e6),
+    # config 2 captured at L = 2048, scaled by tokens to L = 4096
+    2: ("scan_diag_bf16_kernel pairs v4", 642.3e6),
+    # config 3 (two-pass form, both kernels of one call) captured at
+    # L = 32768, scaled by tokens to L = 131072
+    3: ("scan_diag_bf16_kernel two-pass v1", 2679.6e6),
+    4: ("ssd_scalarA_kernel v3", 108.4e6),
 }
 KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v4", 1: "scan_diag_bf16_kernel pairs v4",
-              3: "scan_diag_bf16_kernel pairs v4", 0: "scan_diag_kernel fp32 v2",
+              3: "scan_diag_bf16_kernel two-pass v1", 0: "scan_diag_kernel fp32 v2",
               4: "ssd_scalarA_kernel v3"}
 HBM_FALLBACK_GBS = 6650.0
 
