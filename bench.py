@@ -97,6 +97,31 @@ def ssd_flops(cfg: dict, Q: int = 128) -> float:
     return float(b * nch * per_chunk)
 
 
+# ------------------------------------------------------------ ranks
+def max_over_ranks(values, device="cuda"):
+    """Element-wise max of a list of floats over all ranks of the default
+    process group (identity without one).  Every rank must call it with the
+    same number of values, in the same order."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def aggregate_rate(world: int, units_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own shard of the same
+    size each step, and the step takes the slowest rank's time."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
+def shard_seed(cfg: dict, rank: int) -> int:
+    """Seed of a rank's independent shard (rank 0 keeps the config's seed)."""
+    return int(cfg["seed"]) + 7919 * rank
+
+
 # ------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -317,7 +342,7 @@ def run_gpu(args, rank: int, world: int, local: int):
     import selective_state_space_selscan_b200 as ss
     torch.cuda.set_device(local)
     cfg = synthetic.CONFIGS[args.config]
-    inp = synthetic.make_config(args.config)
+    inp = synthetic.make_config(args.config, seed=shard_seed(cfg, rank))
     dt = cfg["dtype"]
     stream = torch.cuda.current_stream()
     if cfg["kind"] == "diag":
@@ -386,14 +411,9 @@ def run_gpu(args, rank: int, world: int, local: int):
     total_ms = start.elapsed_time(end)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     clock_info = clocks.stop(t_wall0, t_wall1) if clocks else None
-    if dist:
-        t = torch.tensor([total_ms, statistics.mean(launch_ms)], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms, avg_launch_ms = float(t[0]), float(t[1])
-    else:
-        avg_launch_ms = statistics.mean(launch_ms)
+    total_ms, avg_launch_ms = max_over_ranks([total_ms, statistics.mean(launch_ms)])
     ms_per_step = total_ms / args.steps
-    value = world * elems / (ms_per_step * 1e-3) / 1e9
+    value = aggregate_rate(world, elems, ms_per_step) / 1e9
 
     # end to end through the public API: pinned host inputs -> device,
     # scan, result back to the host, every step
@@ -423,11 +443,7 @@ def run_gpu(args, rank: int, world: int, local: int):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
     barrier()
     if rank != 0:
         return
@@ -467,7 +483,7 @@ def run_gpu(args, rank: int, world: int, local: int):
                          "inputs smaller than L2",
                    "parallelism": f"dp{world} (independent shards, no collective)"},
         "roofline": roof,
-        "e2e": {"value": world * elems / (e2e_ms * 1e-3) / 1e9, "unit": "Gelem/s",
+        "e2e": {"value": aggregate_rate(world, elems, e2e_ms) / 1e9, "unit": "Gelem/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": n_launch,
@@ -533,13 +549,13 @@ def run_step(args, rank: int, world: int, local: int):
     stream = torch.cuda.current_stream()
     rng = np.random.default_rng(cfg["seed"] + 1000 + rank)
     if cfg["kind"] == "diag":
-        inp = synthetic.make_diag(batch, cfg["dim"], cfg["N"], 1, dtype=dt, seed=cfg["seed"] + rank,
+        inp = synthetic.make_diag(batch, cfg["dim"], cfg["N"], 1, dtype=dt, seed=shard_seed(cfg, rank),
                                   gate=cfg["gate"], D=cfg["D"])
         state_shape = (batch, cfg["dim"], cfg["N"])
         tok_keys = ("u", "delta", "z", "B", "C")
     else:
         inp = synthetic.make_scalarA(batch, cfg["nheads"], cfg["headdim"], cfg["N"], 1,
-                                     ngroups=cfg["ngroups"], dtype=dt, seed=cfg["seed"] + rank,
+                                     ngroups=cfg["ngroups"], dtype=dt, seed=shard_seed(cfg, rank),
                                      gate=cfg["gate"])
         state_shape = (batch, cfg["nheads"], cfg["headdim"], cfg["N"])
         tok_keys = ("x", "dt", "z", "B", "C")
@@ -599,12 +615,9 @@ def run_step(args, rank: int, world: int, local: int):
     total_ms = start.elapsed_time(end)
     avg_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     clock_info = clocks.stop(t_wall0, t_wall1) if clocks else None
-    if dist:
-        t = torch.tensor([total_ms, avg_launch_ms], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms, avg_launch_ms = float(t[0]), float(t[1])
+    total_ms, avg_launch_ms = max_over_ranks([total_ms, avg_launch_ms])
     ms_per_step = total_ms / args.steps
-    value = world * batch / (ms_per_step * 1e-3)
+    value = aggregate_rate(world, batch, ms_per_step)
 
     # end to end: the token's inputs from pinned host memory, y back; the
     # state stays resident on the device, as a decoding server keeps it
@@ -632,11 +645,7 @@ def run_step(args, rank: int, world: int, local: int):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
     barrier()
     if rank != 0:
         return
@@ -664,7 +673,7 @@ def run_step(args, rank: int, world: int, local: int):
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": traffic, "peak_source": f"{peaks_src} HBM copy bandwidth",
                      "bytes_per_launch": nbytes, "avg_launch_ms": avg_launch_ms},
-        "e2e": {"value": world * batch / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": aggregate_rate(world, batch, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": n_launch,
         "clocks": clock_info,
