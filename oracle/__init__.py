@@ -62,8 +62,12 @@ def _load():
                              _dp, _dp, _dp, _dp, _dp]
         lib.oracle_selscan_scalarA.argtypes = scal + [_i64, _i64]
         lib.oracle_ssd_chunked.argtypes = scal + [_i64]
+        lib.oracle_selscan_bwd.argtypes = common + [
+            _dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp,
+            _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
         for f in (lib.oracle_selscan, lib.oracle_selscan_step,
-                  lib.oracle_selscan_scalarA, lib.oracle_ssd_chunked):
+                  lib.oracle_selscan_scalarA, lib.oracle_ssd_chunked,
+                  lib.oracle_selscan_bwd):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -135,6 +139,46 @@ def selscan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
         Cp, Dp, zp, hp, y.ctypes.data_as(_dp), hs.ctypes.data_as(_dp), d0, d1)
     _check(rc)
     return y, hs
+
+
+def selscan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                delta_softplus=True, h0=None, dlast=None):
+    """Gradients of the diagonal-A scan in fp64 for the loss
+    sum(dy * y) + sum(dlast * last_state).  Shapes as in selscan; dy like u;
+    dlast like h0.  Returns a dict with du, ddelta (like u), dA (like A),
+    dB, dC (like B), and dD, dz, ddelta_bias, dh0 (None where the input is
+    None)."""
+    u = np.asarray(u)
+    batch, dim, L = u.shape
+    A = np.asarray(A)
+    N = A.shape[1]
+    B_in = np.asarray(B)
+    B4, C4 = _bc4(B, batch), _bc4(C, batch)
+    G = B4.shape[1]
+    keep = []
+    ptr = []
+    for a in (u, delta, delta_bias, A, B4, C4, D, z, h0, dy, dlast):
+        arr, pp = _f64(a)
+        keep.append(arr)
+        ptr.append(pp)
+    out = {
+        "du": np.zeros((batch, dim, L)), "ddelta": np.zeros((batch, dim, L)),
+        "dA": np.zeros((dim, N)), "dB": np.zeros(B4.shape), "dC": np.zeros(C4.shape),
+        "dD": np.zeros(dim) if D is not None else None,
+        "dz": np.zeros((batch, dim, L)) if z is not None else None,
+        "ddelta_bias": np.zeros(dim) if delta_bias is not None else None,
+        "dh0": np.zeros((batch, dim, N)) if h0 is not None else None,
+    }
+    optr = lambda k: None if out[k] is None else out[k].ctypes.data_as(_dp)
+    rc = _load().oracle_selscan_bwd(
+        batch, dim, N, L, G, ptr[0], ptr[1], ptr[2], int(bool(delta_softplus)), ptr[3],
+        ptr[4], ptr[5], ptr[6], ptr[7], ptr[8], ptr[9], ptr[10],
+        optr("du"), optr("ddelta"), optr("dA"), optr("dB"), optr("dC"), optr("dD"),
+        optr("dz"), optr("ddelta_bias"), optr("dh0"))
+    _check(rc)
+    out["dB"] = out["dB"].reshape(B_in.shape)
+    out["dC"] = out["dC"].reshape(np.asarray(C).shape)
+    return out
 
 
 def selscan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,

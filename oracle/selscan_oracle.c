@@ -346,3 +346,128 @@ int oracle_ssd_chunked(int64_t batch, int64_t nheads, int64_t headdim,
     free(S); free(step); free(hprev); free(hnext);
     return ORACLE_OK;
 }
+
+/*
+ * Gradients of the diagonal-A selective scan (reverse-mode differentiation
+ * of oracle_selscan, step by step, in fp64).  The loss is
+ *     sum_{b,d,t} dy[b,d,t] y[b,d,t] + sum_{b,d,n} dlast[b,d,n] h_L[b,d,n]
+ * (dlast may be NULL: the final state is not an output of the loss).
+ *
+ * With delta_t the step size, abar_t[n] = exp(delta_t A[d,n]),
+ * h_t = abar_t h_{t-1} + delta_t B_t u_t, out_t = C_t . h_t + D u_t and
+ * y_t = out_t silu(z_t), walking t from L-1 down to 0 with
+ * g = dLoss/dh_t (starting from dlast):
+ *     dout   = dy_t silu(z_t)             dz_t += dy_t out_t silu'(z_t)
+ *     g     += dout C_t                   dC_t += dout h_t
+ *     du_t   = dout D + sum_n g delta_t B_t
+ *     dB_t  += g delta_t u_t              dD   += dout u_t
+ *     ddelta = sum_n g (A abar_t h_{t-1} + B_t u_t)
+ *     dA    += g delta_t abar_t h_{t-1}
+ *     g      = abar_t g                   (now dLoss/dh_{t-1})
+ *     dDelta_t = ddelta * sigmoid(Delta_t + bias) with the softplus (its
+ *     derivative), ddelta otherwise;  dbias += dDelta_t
+ * and after t = 0, dh0 = g.
+ *
+ * Shapes as in oracle_selscan; dy [batch][dim][L]; dlast, dh0
+ * [batch][dim][N].  Outputs du, ddelta, dz [batch][dim][L] are written;
+ * dA [dim][N], dB, dC [batch][ngroups][N][L], dD, dbias [dim] are
+ * ACCUMULATED (the caller zeroes them); dz, dD, dbias, dh0 may be NULL.
+ */
+int oracle_selscan_bwd(int64_t batch, int64_t dim, int64_t N, int64_t L,
+                       int64_t ngroups,
+                       const double *u, const double *delta,
+                       const double *delta_bias, int softplus_flag,
+                       const double *A, const double *B, const double *C,
+                       const double *D, const double *z, const double *h0,
+                       const double *dy, const double *dlast,
+                       double *du, double *ddelta, double *dA, double *dB,
+                       double *dC, double *dD, double *dz, double *dbias,
+                       double *dh0)
+{
+    if (batch < 0 || dim < 0 || N <= 0 || L < 0 || ngroups <= 0 || dim % ngroups != 0)
+        return ORACLE_ERR_ARG;
+    const int64_t per_group = dim / ngroups;
+    /* forward states h_t for t = -1 .. L-1 of one channel, and step sizes */
+    double *hs = (double *)malloc(sizeof(double) * (size_t)((L + 1) * N));
+    double *dts = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *g = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!hs || !dts || !g) {
+        free(hs);
+        free(dts);
+        free(g);
+        return ORACLE_ERR_NOMEM;
+    }
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t grp = d / per_group;
+            const double *Bg = B + (b * ngroups + grp) * N * L;
+            const double *Cg = C + (b * ngroups + grp) * N * L;
+            double *dBg = dB + (b * ngroups + grp) * N * L;
+            double *dCg = dC + (b * ngroups + grp) * N * L;
+            const int64_t row = (b * dim + d) * L;
+            const double bias = delta_bias ? delta_bias[d] : 0.0;
+            /* forward, keeping every state (hs[t+1] = h_t, hs[0] = h_{-1}) */
+            for (int64_t n = 0; n < N; ++n)
+                hs[n] = h0 ? h0[(b * dim + d) * N + n] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                double dt = delta[row + t] + bias;
+                if (softplus_flag)
+                    dt = oracle_softplus(dt);
+                dts[t] = dt;
+                for (int64_t n = 0; n < N; ++n)
+                    hs[(t + 1) * N + n] = exp(dt * A[d * N + n]) * hs[t * N + n]
+                                        + dt * Bg[n * L + t] * u[row + t];
+            }
+            /* backward */
+            for (int64_t n = 0; n < N; ++n)
+                g[n] = dlast ? dlast[(b * dim + d) * N + n] : 0.0;
+            for (int64_t t = L - 1; t >= 0; --t) {
+                const double dt = dts[t];
+                const double x = u[row + t];
+                const double *h_t = hs + (t + 1) * N;
+                const double *h_prev = hs + t * N;
+                double out = (D ? D[d] * x : 0.0);
+                for (int64_t n = 0; n < N; ++n)
+                    out += Cg[n * L + t] * h_t[n];
+                double dout = dy[row + t];
+                if (z) {
+                    const double zv = z[row + t];
+                    const double sg = 1.0 / (1.0 + exp(-zv));
+                    const double dsilu = sg * (1.0 + zv * (1.0 - sg));
+                    if (dz)
+                        dz[row + t] = dy[row + t] * out * dsilu;
+                    dout = dy[row + t] * zv * sg;
+                }
+                double dx = D ? dout * D[d] : 0.0;
+                if (dD)
+                    dD[d] += dout * x;
+                double ddt = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double a = A[d * N + n];
+                    const double abar = exp(dt * a);
+                    g[n] += dout * Cg[n * L + t];
+                    dCg[n * L + t] += dout * h_t[n];
+                    dx += g[n] * dt * Bg[n * L + t];
+                    dBg[n * L + t] += g[n] * dt * x;
+                    ddt += g[n] * (a * abar * h_prev[n] + Bg[n * L + t] * x);
+                    dA[d * N + n] += g[n] * dt * abar * h_prev[n];
+                    g[n] *= abar;
+                }
+                du[row + t] = dx;
+                double dDelta = ddt;
+                if (softplus_flag)
+                    dDelta = ddt / (1.0 + exp(-(delta[row + t] + bias)));
+                ddelta[row + t] = dDelta;
+                if (dbias)
+                    dbias[d] += dDelta;
+            }
+            if (dh0)
+                for (int64_t n = 0; n < N; ++n)
+                    dh0[(b * dim + d) * N + n] = g[n];
+        }
+    }
+    free(hs);
+    free(dts);
+    free(g);
+    return ORACLE_OK;
+}
