@@ -236,6 +236,9 @@ def run_reference(args, rank: int, world: int):
     if args.op == "step":
         run_reference_step(args, world)
         return
+    if args.op == "bwd":
+        run_reference_bwd(args, world)
+        return
     cfg = synthetic.CONFIGS[args.config]
     inp = synthetic.make_config(args.config)
     import oracle
@@ -325,6 +328,49 @@ def run_reference_step(args, world: int):
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": f"{done} steps x {rows} batch rows"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def run_reference_bwd(args, world: int):
+    """Reference arm of ``--op bwd``: the oracle's backward, each timed step
+    one whole channel (all batches, all tokens) of the workload."""
+    cfg = synthetic.CONFIGS[args.config]
+    inp = synthetic.make_config(args.config)
+    dy = np.random.default_rng(cfg["seed"] + 500).standard_normal(inp["u"].shape,
+                                                                     dtype=np.float32)
+    import oracle
+
+    def one(i):
+        c = i % cfg["dim"]
+        sl = lambda x: None if x is None else x[:, c:c + 1]
+        vec = lambda x: None if x is None else x[c:c + 1]
+        oracle.selscan_bwd(sl(inp["u"]), sl(inp["delta"]), inp["A"][c:c + 1], inp["B"],
+                           inp["C"], dy[:, c:c + 1], D=vec(inp["D"]), z=sl(inp["z"]),
+                           delta_bias=vec(inp["delta_bias"]))
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    done = 0
+    for i in range(args.steps):
+        one(i)
+        done += 1
+        if time.perf_counter() - t0 > 150.0:
+            break
+    dt = time.perf_counter() - t0
+    val = done * cfg["batch"] * cfg["L"] / dt / 1e9
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "selective-scan backward Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU",
+        "value": val, "unit": "Gelem/s", "n_gpus": world, "steps": done,
+        "warmup": args.warmup, "ms_per_step": dt / done * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "backward of " + cfg["name"],
+                   "sample_per_step": "one channel (all batches, all tokens)"},
+        "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{done} steps x one channel"},
+        "e2e": {"value": val, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -684,6 +730,168 @@ def run_step(args, rank: int, world: int, local: int):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ backward
+def bwd_bytes(cfg: dict) -> int:
+    """Bytes one backward call must move: u, delta, z, dy read and du,
+    ddelta, dz written once, B and C read and dB, dC (fp32) written once,
+    the per-channel parameters and their gradients."""
+    es = 2 if cfg["dtype"] == "bf16" else 4
+    b, dim, N, L = cfg["batch"], cfg["dim"], cfg["N"], cfg["L"]
+    per_elem = es * (3 if cfg["gate"] else 2) * 2 + es           # (u, delta, z) in+grad, dy
+    total = b * dim * L * per_elem
+    total += 2 * b * N * L * (es + 4)                               # B, C in; dB, dC out
+    total += 2 * dim * N * 4 + 4 * dim * 4                          # A, dA; D, dD, bias, dbias
+    return total
+
+
+def run_bwd(args, rank: int, world: int, local: int):
+    """Backward arm (``--op bwd``): selscan_bwd on the config's diagonal
+    workload with a seeded upstream gradient dy."""
+    import torch
+    import selective_state_space_selscan_b200 as ss
+    torch.cuda.set_device(local)
+    cfg = synthetic.CONFIGS[args.config]
+    if cfg["kind"] != "diag":
+        raise SystemExit("--op bwd runs the diagonal configs (0-3)")
+    inp = synthetic.make_config(args.config, seed=shard_seed(cfg, rank))
+    dt = cfg["dtype"]
+    stream = torch.cuda.current_stream()
+    rng = np.random.default_rng(shard_seed(cfg, rank) + 500)
+    dy_host = rng.standard_normal(inp["u"].shape, dtype=np.float32)
+    dev = {k: to_dev(inp[k], dt, torch) for k in ("u", "delta", "B", "C", "z")}
+    dev["dy"] = to_dev(dy_host, dt, torch)
+    par = {k: to_dev(inp[k], "f32", torch) for k in ("A", "D", "delta_bias")}
+
+    def call():
+        return ss.selscan_bwd(dev["u"], dev["delta"], par["A"], dev["B"], dev["C"], dev["dy"],
+                              D=par["D"], z=dev["z"], delta_bias=par["delta_bias"])
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    ss.check()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    n_launch0 = ss.launch_count()
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        grads = call()
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    n_launch = ss.launch_count() - n_launch0
+    ss.check()
+    total_ms = start.elapsed_time(end)
+    avg_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    clock_info = clocks.stop(t_wall0, t_wall1) if clocks else None
+    total_ms, avg_launch_ms = max_over_ranks([total_ms, avg_launch_ms])
+    ms_per_step = total_ms / args.steps
+    elems = cfg["batch"] * cfg["dim"] * cfg["L"]
+    value = aggregate_rate(world, elems, ms_per_step) / 1e9
+
+    # end to end: inputs and dy from pinned host memory in, every gradient out
+    host_keys = ("u", "delta", "B", "C", "z", "dy")
+    src = dict(inp, dy=dy_host)
+    pinned = {k: torch.from_numpy(np.ascontiguousarray(src[k])).to(
+        torch.bfloat16 if dt == "bf16" else torch.float32).pin_memory()
+        for k in host_keys if src.get(k) is not None}
+    outs = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
+            for k, v in grads.items() if v is not None}
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    e2e_steps = max(1, min(args.steps, 10))
+
+    def e2e_step():
+        for k, t in pinned.items():
+            dev[k].copy_(t, non_blocking=True)
+        g = call()
+        for k, t in outs.items():
+            t.copy_(g[k], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
+    barrier()
+    if rank != 0:
+        return
+    peaks, peaks_src = measured_peaks()
+    nbytes = bwd_bytes(cfg)
+    achieved = nbytes / (avg_launch_ms * 1e-3) / 1e9
+    line = {
+        "metric": "selective-scan backward Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU",
+        "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dt, "data": "synthetic",
+        "config": {"workload": "backward of " + cfg["name"], "batch": cfg["batch"],
+                   "d_inner": cfg["dim"], "d_state": cfg["N"], "seq_len": cfg["L"],
+                   "global_batch": cfg["batch"] * world,
+                   "l2": "inputs larger than L2 (no flush)" if nbytes > 126e6 else
+                         "inputs smaller than L2",
+                   "parallelism": f"dp{world} (independent shards, no collective)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": args.traffic, "peak_source": f"{peaks_src} HBM copy bandwidth",
+                     "bytes_per_launch": nbytes, "avg_launch_ms": avg_launch_ms,
+                     "kernels_per_call": n_launch / args.steps},
+        "e2e": {"value": aggregate_rate(world, elems, e2e_ms) / 1e9, "unit": "Gelem/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": n_launch,
+        "clocks": clock_info,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_bwd_sample(cfg, inp, dy_host, seconds=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def oracle_bwd_sample(cfg: dict, inp: dict, dy: np.ndarray, seconds: float = 10.0):
+    """The fp64 oracle's backward on whole channels of the workload (all
+    batches, all tokens), grown until about `seconds` of work; Gelem/s."""
+    import oracle
+    n, spent = 1, 0.0
+    b, L = cfg["batch"], cfg["L"]
+    while True:
+        sl = lambda x: None if x is None else x[:, :n]
+        vec = lambda x: None if x is None else x[:n]
+        t0 = time.perf_counter()
+        oracle.selscan_bwd(sl(inp["u"]), sl(inp["delta"]), inp["A"][:n], inp["B"], inp["C"],
+                           dy[:, :n], D=vec(inp["D"]), z=sl(inp["z"]),
+                           delta_bias=vec(inp["delta_bias"]))
+        spent = time.perf_counter() - t0
+        if spent >= seconds * 0.5 or n >= cfg["dim"]:
+            break
+        n = int(min(cfg["dim"], n * max(2.0, min(16.0, seconds / max(spent, 1e-3)))))
+    return {"value": b * n * L / spent / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} channel(s) x batch {b} x L {L}, {spent:.1f} s single-threaded fp64"}
+
+
 def oracle_step_sample(cfg: dict, inp: dict, state: np.ndarray, seconds: float = 10.0):
     """The fp64 oracle's decode step on the first rows of the batch, grown
     until about `seconds` of single-threaded work; tokens/s."""
@@ -723,14 +931,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="scan", choices=["scan", "step"],
+    ap.add_argument("--op", default="scan", choices=["scan", "step", "bwd"],
                     help="scan: the forward over the config's sequence (default); "
-                         "step: one decode step of the config's layer")
+                         "step: one decode step of the config's layer; "
+                         "bwd: the backward pass of the config's scan")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch from an ncu capture of this kernel")
     args = ap.parse_args()
 
-    if args.batch is not None and args.op == "scan":
+    if args.batch is not None and args.op != "step":
         synthetic.CONFIGS[args.config] = dict(synthetic.CONFIGS[args.config], batch=args.batch)
     if args.seqlen is not None:
         synthetic.CONFIGS[args.config] = dict(synthetic.CONFIGS[args.config], L=args.seqlen)
@@ -748,7 +957,7 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local))
     try:
-        (run_step if args.op == "step" else run_gpu)(args, rank, world, local)
+        {"step": run_step, "bwd": run_bwd}.get(args.op, run_gpu)(args, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as tdist

@@ -265,6 +265,45 @@ SELSCAN_API selscan_status selscan_step_scalarA(selscan_tensor *state, const sel
                                     int64_t headdim, selscan_tensor *y, cudaStream_t stream);
 
 /*
+ * selscan_bwd -- gradients of selscan_fwd_h0 (diagonal A) for the loss
+ *     sum(dy * y) + sum(dlast * last_state)
+ * (training differentiates the recurrence of the forward pass; "03 --
+ * Modelos de espacio de estados", sections "Discretizacion" and "Parallel
+ * scan").  Walking t from the last token down with g = dLoss/dh_t:
+ *   dout = dy silu(z), dz = dy out silu'(z) (out = C.h + D u before the gate),
+ *   g += dout C_t;  dC_t += dout h_t;  dB_t += g delta u;  dD += dout u
+ *   du = dout D + sum_n g delta B_t;  ddelta = sum_n g (A exp(delta A) h_{t-1} + B_t u)
+ *   dA += g delta exp(delta A) h_{t-1};  g = exp(delta A) g
+ *   d(Delta) = ddelta sigmoid(Delta + bias) with the softplus (ddelta without)
+ *   d(bias) = sum d(Delta);  dh0 = g after the first token.
+ *
+ * Forward inputs exactly as selscan_fwd_h0 (u, delta, delta_bias, softplus,
+ * A, B, C, D, z, h0; time stride 1, element-aligned rows; N = 16, one group).
+ *   dy         (batch, D, L)  same dtype as u: gradient of y
+ *   dlast      (batch, D, N)  F32, contiguous; may be NULL (zero)
+ * Outputs (all overwritten):
+ *   du, ddelta (batch, D, L)  same dtype as u
+ *   dz         (batch, D, L)  same dtype as u; required iff z is given
+ *   dA         (D, N)         F32, contiguous
+ *   dB, dC     (batch, N, L)  F32, contiguous (sums over the channels)
+ *   dD, ddelta_bias (D)       F32; may be NULL (not computed)
+ *   dh0        (batch, D, N)  F32; may be NULL (not computed)
+ * The expanded states are recomputed, never stored: a forward pass keeps h
+ * every 16 tokens in stream-ordered scratch (batch * D * ceil(L/16) * 64
+ * bytes), then the chunks are walked backwards.  Sums over channels and
+ * batch rows use fp32 atomics, so the last bits of dA, dB, dC, dD and
+ * ddelta_bias depend on the order of the additions.
+ */
+SELSCAN_API selscan_status selscan_bwd(
+    const selscan_tensor *u, const selscan_tensor *delta, const selscan_tensor *delta_bias,
+    int delta_softplus, const selscan_tensor *A, const selscan_tensor *B,
+    const selscan_tensor *C, const selscan_tensor *D, const selscan_tensor *z,
+    const selscan_tensor *h0, const selscan_tensor *dy, const selscan_tensor *dlast,
+    selscan_tensor *du, selscan_tensor *ddelta, selscan_tensor *dA, selscan_tensor *dB,
+    selscan_tensor *dC, selscan_tensor *dD, selscan_tensor *dz, selscan_tensor *ddelta_bias,
+    selscan_tensor *dh0, cudaStream_t stream);
+
+/*
  * selscan_check -- synchronise `stream` and report device-side errors that
  * earlier calls recorded (a bounded wait that gave up returns
  * SELSCAN_ERR_TIMEOUT; the record is then cleared).  Returns

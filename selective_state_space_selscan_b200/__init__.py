@@ -29,7 +29,7 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 # entry points declared in include/selscan.h
 EXPORTS = ("selscan_fwd", "selscan_fwd_h0", "selscan_fwd_scalarA", "selscan_fwd_scalarA_h0",
            "selscan_fwd_noalloc", "selscan_step", "selscan_step_scalarA", "selscan_check",
-           "selscan_strerror", "selscan_version", "selscan_launch_count")
+           "selscan_strerror", "selscan_version", "selscan_launch_count", "selscan_bwd")
 
 
 class SelscanError(RuntimeError):
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.selscan_step_scalarA.argtypes = [P, P, P, P, ctypes.c_int, P, P, P, P, P,
                                            ctypes.c_int64, P, ctypes.c_void_p]
         L.selscan_step_scalarA.restype = ctypes.c_int
+        L.selscan_bwd.argtypes = [P, P, P, ctypes.c_int] + [P] * 17 + [ctypes.c_void_p]
+        L.selscan_bwd.restype = ctypes.c_int
         L.selscan_debug_withhold_carry.argtypes = [ctypes.c_int]
         L.selscan_debug_withhold_carry.restype = None
         L.selscan_debug_diag_mode.argtypes = [ctypes.c_int]
@@ -257,6 +259,41 @@ def selscan_step_scalarA(state, x, dt, A, B, C, headdim, D=None, z=None, dt_bias
     if rc != 0:
         raise SelscanError(rc, "selscan_step_scalarA")
     return y
+
+
+def selscan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                delta_softplus=True, h0=None, dlast=None, need_dh0=None, stream=None):
+    """Gradients of selscan_fwd (diagonal A) for sum(dy * y) + sum(dlast *
+    last_state).  Returns a dict: du, ddelta (like u), dz (like u, or None),
+    dA (D, N), dB, dC (batch, N, L) fp32, dD, ddelta_bias (D) fp32 or None,
+    dh0 (batch, D, N) fp32 or None (computed when h0 is given or need_dh0)."""
+    import torch
+    dev = u.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    out = {
+        "du": torch.empty(u.shape, dtype=u.dtype, device=dev),
+        "ddelta": torch.empty(u.shape, dtype=u.dtype, device=dev),
+        "dz": torch.empty(u.shape, dtype=u.dtype, device=dev) if z is not None else None,
+        "dA": torch.empty((dim, N), **f32),
+        "dB": torch.empty((batch, N, L), **f32),
+        "dC": torch.empty((batch, N, L), **f32),
+        "dD": torch.empty((dim,), **f32) if D is not None else None,
+        "ddelta_bias": torch.empty((dim,), **f32) if delta_bias is not None else None,
+        "dh0": torch.empty((batch, dim, N), **f32)
+        if (h0 is not None or need_dh0) else None,
+    }
+    ins = [describe(t) for t in (u, delta, delta_bias)]
+    rest = [describe(t) for t in (A, B, C, D, z, h0, dy, dlast)]
+    outs = [describe(out[k]) for k in ("du", "ddelta", "dA", "dB", "dC", "dD", "dz",
+                                       "ddelta_bias", "dh0")]
+    rc = lib().selscan_bwd(_ref(ins[0]), _ref(ins[1]), _ref(ins[2]), int(bool(delta_softplus)),
+                           *[_ref(x) for x in rest], *[_ref(x) for x in outs],
+                           _stream_handle(stream))
+    if rc != 0:
+        raise SelscanError(rc, "selscan_bwd")
+    return out
 
 
 def check(stream=None) -> None:

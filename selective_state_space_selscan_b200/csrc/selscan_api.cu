@@ -18,6 +18,7 @@
 #include "scan_diag_bf16.cuh"
 #include "ssd_scalarA.cuh"
 #include "step.cuh"
+#include "bwd_diag.cuh"
 
 using namespace selscan;
 
@@ -1172,4 +1173,185 @@ extern "C" selscan_status selscan_step_scalarA(selscan_tensor *state, const sels
 {
     return step_impl(true, state, x, dt, dt_bias, dt_softplus, A, B, C, D, z, headdim, y,
                      stream);
+}
+
+// ------------------------------------------------------------ backward
+namespace {
+
+// A sequence tensor (d0, d1, L), time stride 1, element-aligned (the
+// backward reads it with plain loads, no bulk copies).
+selscan_status check_seq_plain(const selscan_tensor *t, int64_t d0, int64_t d1, int64_t L,
+                               int32_t dtype)
+{
+    if (!present(t))
+        return SELSCAN_ERR_NULL;
+    if (t->ndim != 3 || t->shape[0] != d0 || t->shape[1] != d1 || t->shape[2] != L)
+        return SELSCAN_ERR_SHAPE;
+    if (t->dtype != dtype)
+        return SELSCAN_ERR_DTYPE;
+    if (d0 == 0 || d1 == 0 || L == 0)
+        return SELSCAN_OK;
+    if ((L > 1 && t->stride[2] != 1) || t->stride[0] < 0 || t->stride[1] < 0)
+        return SELSCAN_ERR_STRIDE;
+    if (reinterpret_cast<uintptr_t>(t->data) % elem_size(dtype))
+        return SELSCAN_ERR_ALIGN;
+    return SELSCAN_OK;
+}
+
+}  // namespace
+
+extern "C" selscan_status selscan_bwd(
+    const selscan_tensor *u, const selscan_tensor *delta, const selscan_tensor *delta_bias,
+    int delta_softplus, const selscan_tensor *A, const selscan_tensor *B,
+    const selscan_tensor *C, const selscan_tensor *D, const selscan_tensor *z,
+    const selscan_tensor *h0, const selscan_tensor *dy, const selscan_tensor *dlast,
+    selscan_tensor *du, selscan_tensor *ddelta, selscan_tensor *dA, selscan_tensor *dB,
+    selscan_tensor *dC, selscan_tensor *dD, selscan_tensor *dz, selscan_tensor *ddelta_bias,
+    selscan_tensor *dh0, cudaStream_t stream)
+{
+    if (!present(u) || !present(A))
+        return SELSCAN_ERR_NULL;
+    if (u->ndim != 3 || A->ndim != 2)
+        return SELSCAN_ERR_SHAPE;
+    const int32_t dt = u->dtype;
+    if (dt != SELSCAN_F32 && dt != SELSCAN_BF16)
+        return SELSCAN_ERR_DTYPE;
+    const int64_t batch = u->shape[0], dim = u->shape[1], L = u->shape[2];
+    const int64_t N = A->shape[1];
+    if (batch < 0 || dim < 0 || L < 0 || A->shape[0] != dim)
+        return SELSCAN_ERR_SHAPE;
+    selscan_status st;
+    for (const selscan_tensor *t : {u, delta, dy, static_cast<const selscan_tensor *>(du),
+                                    static_cast<const selscan_tensor *>(ddelta)})
+        if ((st = check_seq_plain(t, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    const bool gate = z && z->data;
+    if (gate) {
+        if ((st = check_seq_plain(z, batch, dim, L, dt)) != SELSCAN_OK) return st;
+        if ((st = check_seq_plain(dz, batch, dim, L, dt)) != SELSCAN_OK) return st;
+    }
+    // B, C: (batch, N, L) or (batch, 1, N, L); dB, dC: (batch, N, L) fp32 contiguous
+    selscan_tensor Bv{}, Cv{};
+    for (int k = 0; k < 2; ++k) {
+        const selscan_tensor *t = k ? C : B;
+        if (!present(t))
+            return SELSCAN_ERR_NULL;
+        selscan_tensor v = *t;
+        if (t->ndim == 4) {
+            if (t->shape[1] != 1)
+                return SELSCAN_ERR_UNSUPPORTED;
+            v.ndim = 3;
+            v.shape[1] = t->shape[2];
+            v.shape[2] = t->shape[3];
+            v.stride[1] = t->stride[2];
+            v.stride[2] = t->stride[3];
+        }
+        if ((st = check_seq_plain(&v, batch, N, L, dt)) != SELSCAN_OK) return st;
+        (k ? Cv : Bv) = v;
+    }
+    {
+        const int64_t ashape[2] = {dim, N}, vshape[1] = {dim}, sshape[3] = {batch, dim, N};
+        const int64_t bcshape[3] = {batch, N, L};
+        if ((st = check_param(A, 2, ashape, false)) != SELSCAN_OK) return st;
+        if ((st = check_param(dA, 2, ashape, false)) != SELSCAN_OK) return st;
+        if ((st = check_param(delta_bias, 1, vshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(D, 1, vshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(dD, 1, vshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(ddelta_bias, 1, vshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(h0, 3, sshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(dlast, 3, sshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(dh0, 3, sshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(dB, 3, bcshape, false)) != SELSCAN_OK) return st;
+        if ((st = check_param(dC, 3, bcshape, false)) != SELSCAN_OK) return st;
+    }
+    if (N != kBwdN)
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch > 65535 || dim > (int64_t(1) << 30) || L > (int64_t(1) << 30))
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch == 0 || dim == 0)
+        return SELSCAN_OK;
+
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    if ((st = device_setup(&dev, &di)) != SELSCAN_OK)
+        return st;
+    auto zero = [&](selscan_tensor *t) {
+        return (!t || !t->data) ? cudaSuccess
+                                : cudaMemsetAsync(t->data, 0, size_t(numel(t)) * 4, stream);
+    };
+    if (zero(dA) != cudaSuccess || zero(dB) != cudaSuccess || zero(dC) != cudaSuccess ||
+        zero(dD) != cudaSuccess || zero(ddelta_bias) != cudaSuccess)
+        return SELSCAN_ERR_CUDA;
+    if (L == 0) {
+        // nothing to walk back through: the gradient of h0 is that of the final state
+        if (dh0 && dh0->data) {
+            const size_t bytes = size_t(batch * dim * N) * 4;
+            const cudaError_t e =
+                (dlast && dlast->data)
+                    ? cudaMemcpyAsync(dh0->data, dlast->data, bytes, cudaMemcpyDeviceToDevice,
+                                      stream)
+                    : cudaMemsetAsync(dh0->data, 0, bytes, stream);
+            return e == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+        }
+        return SELSCAN_OK;
+    }
+
+    BwdParams prm{};
+    prm.batch = int(batch);
+    prm.dim = int(dim);
+    prm.L = int(L);
+    prm.nchunks = int((L + kBwdT - 1) / kBwdT);
+    prm.u = u->data;
+    prm.u_bs = u->stride[0];
+    prm.u_ds = u->stride[1];
+    prm.delta = delta->data;
+    prm.dl_bs = delta->stride[0];
+    prm.dl_ds = delta->stride[1];
+    prm.z = gate ? z->data : nullptr;
+    prm.z_bs = gate ? z->stride[0] : 0;
+    prm.z_ds = gate ? z->stride[1] : 0;
+    prm.dy = dy->data;
+    prm.dy_bs = dy->stride[0];
+    prm.dy_ds = dy->stride[1];
+    prm.B = Bv.data;
+    prm.B_bs = Bv.stride[0];
+    prm.B_ns = Bv.stride[1];
+    prm.C = Cv.data;
+    prm.C_bs = Cv.stride[0];
+    prm.C_ns = Cv.stride[1];
+    prm.A = static_cast<const float *>(A->data);
+    prm.delta_bias = static_cast<const float *>(opt_data(delta_bias));
+    prm.Dskip = static_cast<const float *>(opt_data(D));
+    prm.h0 = static_cast<const float *>(opt_data(h0));
+    prm.dlast = static_cast<const float *>(opt_data(dlast));
+    prm.softplus = delta_softplus ? 1 : 0;
+    prm.du = du->data;
+    prm.du_bs = du->stride[0];
+    prm.du_ds = du->stride[1];
+    prm.ddelta = ddelta->data;
+    prm.dd_bs = ddelta->stride[0];
+    prm.dd_ds = ddelta->stride[1];
+    prm.dz = gate ? dz->data : nullptr;
+    prm.dz_bs = gate ? dz->stride[0] : 0;
+    prm.dz_ds = gate ? dz->stride[1] : 0;
+    prm.dA = static_cast<float *>(dA->data);
+    prm.dB = static_cast<float *>(dB->data);
+    prm.dC = static_cast<float *>(dC->data);
+    prm.dD = static_cast<float *>(dD ? dD->data : nullptr);
+    prm.dbias = static_cast<float *>(ddelta_bias ? ddelta_bias->data : nullptr);
+    prm.dh0 = static_cast<float *>(dh0 ? dh0->data : nullptr);
+
+    // checkpoints of h every kBwdT tokens: [batch][dim][nchunks][16] fp32
+    const size_t ck_bytes = size_t(batch) * dim * prm.nchunks * kBwdN * 4;
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, ck_bytes, stream) != cudaSuccess)
+        return SELSCAN_ERR_CUDA;
+    prm.ckpt = static_cast<float *>(ws);
+    const dim3 grid(unsigned((dim + 31) / 32), unsigned(batch));
+    if (dt == SELSCAN_BF16)
+        selscan_bwd_kernel<__nv_bfloat16><<<grid, 32, 0, stream>>>(prm);
+    else
+        selscan_bwd_kernel<float><<<grid, 32, 0, stream>>>(prm);
+    const cudaError_t le = counted_launch();
+    cudaFreeAsync(ws, stream);
+    return le == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
 }

@@ -181,3 +181,38 @@ def test_step_rejects(over, expect):
 ])
 def test_step_scalarA_rejects(over, expect):
     assert _step(scalar=True, **over) == C[expect]
+
+
+def _bwd(**over):
+    b, D, N, L = 2, 64, 16, 48
+    f32 = ss.SELSCAN_F32
+    args = dict(u=_t((b, D, L)), delta=_t((b, D, L)), bias=None, A=_t((D, N), f32),
+                B=_t((b, N, L)), C=_t((b, N, L)), Dv=None, z=None, h0=None, dy=_t((b, D, L)),
+                dlast=None, du=_t((b, D, L)), dd=_t((b, D, L)), dA=_t((D, N), f32),
+                dB=_t((b, N, L), f32), dC=_t((b, N, L), f32), dD=None, dz=None, dbias=None,
+                dh0=None)
+    args.update(over)
+    r = lambda x: None if x is None else ctypes.byref(x)
+    order = ("u", "delta", "bias")
+    rest = ("A", "B", "C", "Dv", "z", "h0", "dy", "dlast", "du", "dd", "dA", "dB", "dC",
+            "dD", "dz", "dbias", "dh0")
+    return ss.lib().selscan_bwd(r(args["u"]), r(args["delta"]), r(args["bias"]), 1,
+                                *[r(args[k]) for k in rest], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(u=None), "SELSCAN_ERR_NULL"),
+    (dict(dy=None), "SELSCAN_ERR_NULL"),
+    (dict(dA=None), "SELSCAN_ERR_NULL"),
+    (dict(dy=_t((2, 64, 47))), "SELSCAN_ERR_SHAPE"),
+    (dict(du=_t((2, 64, 48), ss.SELSCAN_F32)), "SELSCAN_ERR_DTYPE"),
+    (dict(dB=_t((2, 16, 48))), "SELSCAN_ERR_DTYPE"),
+    (dict(z=_t((2, 64, 48))), "SELSCAN_ERR_NULL"),          # gate given, dz missing
+    (dict(dh0=_t((2, 64, 8), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(delta=_t((2, 64, 48), strides=(64 * 96, 96, 2))), "SELSCAN_ERR_STRIDE"),
+    (dict(A=_t((64, 8), ss.SELSCAN_F32), dA=_t((64, 8), ss.SELSCAN_F32),
+          B=_t((2, 8, 48)), C=_t((2, 8, 48)), dB=_t((2, 8, 48), ss.SELSCAN_F32),
+          dC=_t((2, 8, 48), ss.SELSCAN_F32)), "SELSCAN_ERR_UNSUPPORTED"),
+])
+def test_bwd_rejects(over, expect):
+    assert _bwd(**over) == C[expect]
