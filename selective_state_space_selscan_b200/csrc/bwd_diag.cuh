@@ -12,16 +12,27 @@
 //   ddelta = sum_n g (A abar h_{t-1} + B_t u)       dA += g delta abar h_{t-1}
 //   g    = abar g;   dDelta = ddelta * sigmoid(Delta + bias) under softplus
 //
-// and dh0 = g after the first token.  The expanded states are never stored:
-// pass A runs the forward recurrence once and keeps h every kBwdT tokens;
-// pass B walks the chunks backwards, recomputes the chunk's states from its
-// checkpoint into shared memory and runs the reverse recurrence over them.
+// and dh0 = g after the first token.
 //
-// Work split: one warp per (batch row, 32 channels), one lane per channel
-// holding all 16 states.  dB and dC sum over the channels of a batch row:
-// each token's 32 per-lane values are reduced across the warp by a
-// butterfly (31 shuffles leave lane i with the sum of value i), then added
-// to global memory atomically (one add per lane and token).  dA, dD and the
+// Work units are (32 channels of one batch row, one time segment), one warp
+// each, one lane per channel holding all 16 states.  Both recurrences are
+// linear, so segments need not wait for one another:
+//   * bwd_agg_kernel scans every segment forward from a zero state (its end
+//     state E) and backward from a zero gradient (its start gradient G:
+//     g_{t-1} = abar_t (g_t + dout_t C_t) needs no forward state), and sums
+//     its step sizes S;
+//   * selscan_bwd_kernel starts segment k from
+//       h_in  = fold_{j<k}  h <- exp(A S_j) h + E_j      (from h0)
+//       g_end = fold_{j>k, last first} g <- exp(A S_j) g + G_j  (from dlast)
+//     then keeps h every 8 tokens (pass A), and walks the 8-token chunks
+//     backwards (pass B): the chunk's states are recomputed from their
+//     checkpoint into shared memory and the reverse step runs over them.
+// The expanded states (batch, D, L, N) are never stored.
+//
+// dB and dC sum over the channels of a batch row: each token's 32 per-lane
+// values are reduced across the warp by a butterfly (31 shuffles leave lane i
+// with the sum of value i); a lane keeps its sums for the chunk's 8 tokens
+// and adds them to global memory with two 16-byte atomics.  dA, dD and the
 // bias gradient sum over batch rows and tokens: registers, then atomics.
 #pragma once
 
@@ -29,19 +40,22 @@
 #include <cstdint>
 #include <type_traits>
 
+#include "f32x2.cuh"
 #include "ptx.cuh"
 #include "scan_diag.cuh"
 
 namespace selscan {
 
 constexpr int kBwdN = 16;  // states per channel
-constexpr int kBwdT = 16;  // tokens per checkpoint chunk
+constexpr int kBwdT = 8;   // tokens per checkpoint chunk
 
 struct BwdParams {
-    int batch, dim, L, nchunks;
-    const void *u, *delta, *z, *dy;  // (batch, dim, L), time stride 1
+    int batch, dim, L, nchunks;      // nchunks = ceil(L / kBwdT)
+    int tiles, segs, seg_chunks;     // units = tiles * segs; tile = (batch row, 32 channels)
+    int tiles_per_batch;
+    const void *u, *delta, *z, *dy;  // (batch, dim, L), time stride 1, 16-byte aligned rows
     int64_t u_bs, u_ds, dl_bs, dl_ds, z_bs, z_ds, dy_bs, dy_ds;
-    const void *B, *C;               // (batch, 16, L), time stride 1
+    const void *B, *C;               // (batch, 16, L), same alignment
     int64_t B_bs, B_ns, C_bs, C_ns;
     const float *A;                  // (dim, 16)
     const float *delta_bias, *Dskip; // (dim) or null
@@ -54,58 +68,296 @@ struct BwdParams {
     float *dD, *dbias;               // (dim) or null, accumulated
     float *dh0;                      // (batch, dim, 16) or null, written
     float *ckpt;                     // [batch][dim][nchunks][16] scratch
+    float *aggE, *aggG, *aggS;       // [units][32][16], [units][32][16], [units][32]
 };
 
-__device__ __forceinline__ float bwd_ld(const void *p, int64_t off, const float *)
+// 8 consecutive elements of a row (16-byte aligned start) as fp32; elements
+// at or past `valid` read as zero.
+__device__ __forceinline__ void bwd_ld8(const void *base, int64_t off, int valid, float (&v)[8],
+                                        const __nv_bfloat16 *)
 {
-    return static_cast<const float *>(p)[off];
-}
-
-__device__ __forceinline__ float bwd_ld(const void *p, int64_t off, const __nv_bfloat16 *)
-{
-    return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[off]);
-}
-
-__device__ __forceinline__ void bwd_st(void *p, int64_t off, float v, const float *)
-{
-    static_cast<float *>(p)[off] = v;
-}
-
-__device__ __forceinline__ void bwd_st(void *p, int64_t off, float v, const __nv_bfloat16 *)
-{
-    static_cast<__nv_bfloat16 *>(p)[off] = __float2bfloat16_rn(v);
-}
-
-// exp(delta * A[n]) for the 16 states: r^(n+1) for S4D-real A
-// (A[n] = (n+1) A[0], checked per channel), else one exponential per state.
-template <bool FAST>
-__device__ __forceinline__ void bwd_decays(float dt, const float (&al)[kBwdN], bool pow_path,
-                                           float (&a)[kBwdN])
-{
-    if (pow_path) {
-        const float r = FAST ? ex2_approx(dt * al[0]) : exp2f(dt * al[0]);
-        a[0] = r;
-#pragma unroll
-        for (int n = 1; n < kBwdN; ++n)
-            a[n] = a[n - 1] * r;
+    const __nv_bfloat16 *p = static_cast<const __nv_bfloat16 *>(base) + off;
+    if (valid >= 8) {
+        const uint4 q = *reinterpret_cast<const uint4 *>(p);
+        unpack8_bf16(q, v);
     } else {
 #pragma unroll
-        for (int n = 0; n < kBwdN; ++n)
-            a[n] = FAST ? ex2_approx(dt * al[n]) : exp2f(dt * al[n]);
+        for (int i = 0; i < 8; ++i)
+            v[i] = i < valid ? __bfloat162float(p[i]) : 0.f;
     }
 }
 
+__device__ __forceinline__ void bwd_ld8(const void *base, int64_t off, int valid, float (&v)[8],
+                                        const float *)
+{
+    const float *p = static_cast<const float *>(base) + off;
+    if (valid >= 8) {
+        const float4 a = reinterpret_cast<const float4 *>(p)[0];
+        const float4 b = reinterpret_cast<const float4 *>(p)[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            v[i] = i < valid ? p[i] : 0.f;
+    }
+}
+
+__device__ __forceinline__ void bwd_st8(void *base, int64_t off, int valid, const float (&v)[8],
+                                        const __nv_bfloat16 *)
+{
+    __nv_bfloat16 *p = static_cast<__nv_bfloat16 *>(base) + off;
+    if (valid >= 8) {
+        uint4 q;
+        q.x = pack2_bf16(v[0], v[1]);
+        q.y = pack2_bf16(v[2], v[3]);
+        q.z = pack2_bf16(v[4], v[5]);
+        q.w = pack2_bf16(v[6], v[7]);
+        *reinterpret_cast<uint4 *>(p) = q;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i < valid)
+                p[i] = __float2bfloat16_rn(v[i]);
+    }
+}
+
+__device__ __forceinline__ void bwd_st8(void *base, int64_t off, int valid, const float (&v)[8],
+                                        const float *)
+{
+    float *p = static_cast<float *>(base) + off;
+    if (valid >= 8) {
+        reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i < valid)
+                p[i] = v[i];
+    }
+}
+
+// exp(delta * A[n]) for the 16 states as 8 pairs: r^(n+1) for S4D-real A
+// (A[n] = (n+1) A[0], checked per channel), else one exponential per state.
+template <bool FAST>
+__device__ __forceinline__ void bwd_decays(float dt, const float (&al)[kBwdN], bool pow_path,
+                                           uint64_t (&a2)[8])
+{
+    if (pow_path) {
+        const float r = FAST ? ex2_approx(dt * al[0]) : exp2f(dt * al[0]);
+        const float r2 = r * r;
+        const uint64_t R2 = pk2(r2, r2);
+        a2[0] = pk2(r, r2);
+#pragma unroll
+        for (int j = 1; j < 8; ++j)
+            a2[j] = mul2(a2[j - 1], R2);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            a2[j] = FAST ? pk2(ex2_approx(dt * al[2 * j]), ex2_approx(dt * al[2 * j + 1]))
+                         : pk2(exp2f(dt * al[2 * j]), exp2f(dt * al[2 * j + 1]));
+    }
+}
+
+template <bool FAST>
+__device__ __forceinline__ float bwd_step(float raw, int softplus)
+{
+    if (!softplus)
+        return raw;
+    return FAST ? softplus_fast(raw) : softplus_exact(raw);
+}
+
+// Per-warp shared memory: B and C of the chunk (fp32, [token][n]) and the
+// recomputed states of the chunk ([token][n][lane]).
+struct BwdSmem {
+    float bc[kBwdT][2][kBwdN];
+    float h[kBwdT][kBwdN][32];
+};
+
+// Stage B (and C) of tokens [t0, t0 + valid) of batch row b as fp32.
 template <typename T>
-__device__ __forceinline__ float bwd_step_size(const BwdParams &p, int64_t row_dl, int t,
-                                               float bias, float *raw)
+__device__ __forceinline__ void bwd_stage_bc(const BwdParams &p, BwdSmem &sm, int b, int t0,
+                                             int valid, bool withC, int lane)
+{
+    const T *tag = nullptr;
+    if (lane < kBwdN || withC) {
+        const int n = lane & 15;
+        const bool isC = lane >= kBwdN;
+        float v[8];
+        bwd_ld8(isC ? p.C : p.B,
+                int64_t(b) * (isC ? p.C_bs : p.B_bs) + int64_t(n) * (isC ? p.C_ns : p.B_ns) + t0,
+                valid, v, tag);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            sm.bc[i][isC][n] = v[i];
+    }
+    __syncwarp();
+}
+
+template <typename T>
+struct BwdChannel {
+    float al[kBwdN];
+    uint64_t An2[8];
+    bool pow_path;
+    float bias, dsk;
+    int64_t row_u, row_dl, row_z, row_dy, row_du, row_dd, row_dz;
+
+    __device__ __forceinline__ void init(const BwdParams &p, int b, int dd)
+    {
+        float An[kBwdN];
+        pow_path = true;
+#pragma unroll
+        for (int n = 0; n < kBwdN; ++n) {
+            An[n] = p.A[int64_t(dd) * kBwdN + n];
+            al[n] = An[n] * kLog2e;
+            pow_path = pow_path && (An[n] == float(n + 1) * An[0]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            An2[j] = pk2(An[2 * j], An[2 * j + 1]);
+        bias = p.delta_bias ? p.delta_bias[dd] : 0.f;
+        dsk = p.Dskip ? p.Dskip[dd] : 0.f;
+        row_u = int64_t(b) * p.u_bs + int64_t(dd) * p.u_ds;
+        row_dl = int64_t(b) * p.dl_bs + int64_t(dd) * p.dl_ds;
+        row_z = int64_t(b) * p.z_bs + int64_t(dd) * p.z_ds;
+        row_dy = int64_t(b) * p.dy_bs + int64_t(dd) * p.dy_ds;
+        row_du = int64_t(b) * p.du_bs + int64_t(dd) * p.du_ds;
+        row_dd = int64_t(b) * p.dd_bs + int64_t(dd) * p.dd_ds;
+        row_dz = int64_t(b) * p.dz_bs + int64_t(dd) * p.dz_ds;
+    }
+};
+
+// Forward over [t0, t0 + valid): h <- abar h + delta u B, token by token;
+// when `keep` is set the state after each token goes to shared memory.
+template <typename T, bool KEEP>
+__device__ __forceinline__ void bwd_forward_chunk(const BwdParams &p, const BwdChannel<T> &ch,
+                                                  BwdSmem &sm, int t0, int valid,
+                                                  uint64_t (&h2)[8], int lane)
 {
     constexpr bool FAST = !std::is_same<T, float>::value;
     const T *tag = nullptr;
-    const float x = bwd_ld(p.delta, row_dl + t, tag) + bias;
-    *raw = x;
-    if (!p.softplus)
-        return x;
-    return FAST ? softplus_fast(x) : softplus_exact(x);
+    float uv[8], dv[8];
+    bwd_ld8(p.u, ch.row_u + t0, valid, uv, tag);
+    bwd_ld8(p.delta, ch.row_dl + t0, valid, dv, tag);
+#pragma unroll
+    for (int i = 0; i < kBwdT; ++i) {
+        if (i >= valid)
+            break;
+        const float dt = bwd_step<FAST>(dv[i] + ch.bias, p.softplus);
+        const float dx = dt * uv[i];
+        const uint64_t DX = pk2(dx, dx);
+        uint64_t a2[8];
+        bwd_decays<FAST>(dt, ch.al, ch.pow_path, a2);
+        const float4 *bq = reinterpret_cast<const float4 *>(sm.bc[i][0]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 bb = bq[q];
+            h2[2 * q] = fma2(a2[2 * q], h2[2 * q], mul2(DX, pk2(bb.x, bb.y)));
+            h2[2 * q + 1] = fma2(a2[2 * q + 1], h2[2 * q + 1], mul2(DX, pk2(bb.z, bb.w)));
+        }
+        if (KEEP) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                sm.h[i][2 * j][lane] = lo2(h2[j]);
+                sm.h[i][2 * j + 1][lane] = hi2(h2[j]);
+            }
+        }
+    }
+}
+
+// Segment aggregates: E (end state from zero), G (start gradient from a zero
+// end gradient), S (sum of step sizes) of every (tile, segment) unit but the
+// ones that no other unit needs (E of the last segment, G of the first).
+template <typename T>
+__global__ void __launch_bounds__(32)
+bwd_agg_kernel(const BwdParams p)
+{
+    constexpr bool FAST = !std::is_same<T, float>::value;
+    const T *tag = nullptr;
+    __shared__ __align__(16) BwdSmem sm;
+    const int lane = threadIdx.x;
+    const int unit = blockIdx.x;
+    const int seg = unit / p.tiles, tile = unit - seg * p.tiles;
+    const int b = tile / p.tiles_per_batch;
+    const int d = (tile - b * p.tiles_per_batch) * 32 + lane;
+    const bool live = d < p.dim;
+    BwdChannel<T> ch;
+    ch.init(p, b, live ? d : 0);
+    const int c0 = seg * p.seg_chunks, c1 = min(p.nchunks, c0 + p.seg_chunks);
+
+    // forward from zero: end state and the sum of step sizes
+    uint64_t h2[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        h2[j] = pk2(0.f, 0.f);
+    float ssum = 0.f;
+    if (seg < p.segs - 1) {
+        for (int c = c0; c < c1; ++c) {
+            const int t0 = c * kBwdT, valid = min(kBwdT, p.L - t0);
+            bwd_stage_bc<T>(p, sm, b, t0, valid, false, lane);
+            bwd_forward_chunk<T, false>(p, ch, sm, t0, valid, h2, lane);
+            __syncwarp();
+        }
+    }
+    {
+        // the sum of step sizes (every segment but the first is folded over)
+        for (int c = c0; c < c1; ++c) {
+            const int t0 = c * kBwdT, valid = min(kBwdT, p.L - t0);
+            float dv[8];
+            bwd_ld8(p.delta, ch.row_dl + t0, valid, dv, tag);
+#pragma unroll
+            for (int i = 0; i < kBwdT; ++i)
+                if (i < valid)
+                    ssum += bwd_step<FAST>(dv[i] + ch.bias, p.softplus);
+        }
+    }
+    // backward from zero: g_{t-1} = abar_t (g_t + dout_t C_t)
+    uint64_t g2[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        g2[j] = pk2(0.f, 0.f);
+    if (seg > 0) {
+        for (int c = c1 - 1; c >= c0; --c) {
+            const int t0 = c * kBwdT, valid = min(kBwdT, p.L - t0);
+            bwd_stage_bc<T>(p, sm, b, t0, valid, true, lane);
+            float dv[8], yv[8], zv[8];
+            bwd_ld8(p.delta, ch.row_dl + t0, valid, dv, tag);
+            bwd_ld8(p.dy, ch.row_dy + t0, valid, yv, tag);
+            if (p.z)
+                bwd_ld8(p.z, ch.row_z + t0, valid, zv, tag);
+#pragma unroll
+            for (int i = kBwdT - 1; i >= 0; --i) {
+                if (i >= valid)
+                    continue;
+                const float dt = bwd_step<FAST>(dv[i] + ch.bias, p.softplus);
+                float dout = live ? yv[i] : 0.f;
+                if (p.z)
+                    dout *= zv[i] / (1.f + __expf(-zv[i]));
+                const uint64_t DO = pk2(dout, dout);
+                uint64_t a2[8];
+                bwd_decays<FAST>(dt, ch.al, ch.pow_path, a2);
+                const float4 *cq = reinterpret_cast<const float4 *>(sm.bc[i][1]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 cc = cq[q];
+                    g2[2 * q] = mul2(a2[2 * q], fma2(DO, pk2(cc.x, cc.y), g2[2 * q]));
+                    g2[2 * q + 1] = mul2(a2[2 * q + 1], fma2(DO, pk2(cc.z, cc.w), g2[2 * q + 1]));
+                }
+            }
+            __syncwarp();
+        }
+    }
+    if (live) {
+        const int64_t o = (int64_t(unit) * 32 + lane) * kBwdN;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            p.aggE[o + 2 * j] = lo2(h2[j]);
+            p.aggE[o + 2 * j + 1] = hi2(h2[j]);
+            p.aggG[o + 2 * j] = lo2(g2[j]);
+            p.aggG[o + 2 * j + 1] = hi2(g2[j]);
+        }
+        p.aggS[int64_t(unit) * 32 + lane] = ssum;
+    }
 }
 
 template <typename T>
@@ -115,151 +367,172 @@ selscan_bwd_kernel(const BwdParams p)
     constexpr int N = kBwdN, TC = kBwdT;
     constexpr bool FAST = !std::is_same<T, float>::value;
     const T *tag = nullptr;
-    __shared__ float s_h[TC][N][32];  // recomputed states of the chunk, lane-minor
+    __shared__ __align__(16) BwdSmem sm;
 
     const int lane = threadIdx.x;
-    const int b = blockIdx.y;
-    const int d = blockIdx.x * 32 + lane;
+    const int unit = blockIdx.x;
+    const int seg = unit / p.tiles, tile = unit - seg * p.tiles;
+    const int b = tile / p.tiles_per_batch;
+    const int d = (tile - b * p.tiles_per_batch) * 32 + lane;
     const bool live = d < p.dim;
-    const int dd = live ? d : 0;  // dead lanes mirror channel 0 and contribute zeros
-
-    const int64_t row_u = int64_t(b) * p.u_bs + int64_t(dd) * p.u_ds;
-    const int64_t row_dl = int64_t(b) * p.dl_bs + int64_t(dd) * p.dl_ds;
-    const int64_t row_z = int64_t(b) * p.z_bs + int64_t(dd) * p.z_ds;
-    const int64_t row_dy = int64_t(b) * p.dy_bs + int64_t(dd) * p.dy_ds;
-    const int64_t row_du = int64_t(b) * p.du_bs + int64_t(dd) * p.du_ds;
-    const int64_t row_dd = int64_t(b) * p.dd_bs + int64_t(dd) * p.dd_ds;
-    const int64_t row_dz = int64_t(b) * p.dz_bs + int64_t(dd) * p.dz_ds;
-    const int64_t bB = int64_t(b) * p.B_bs, bC = int64_t(b) * p.C_bs;
-    const float bias = p.delta_bias ? p.delta_bias[dd] : 0.f;
-    const float dsk = p.Dskip ? p.Dskip[dd] : 0.f;
-    float An[N], al[N];
-    bool pow_path = true;
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        An[n] = p.A[int64_t(dd) * N + n];
-        al[n] = An[n] * kLog2e;
-        pow_path = pow_path && (An[n] == float(n + 1) * An[0]);
-    }
+    const int dd = live ? d : 0;  // lanes past the last channel mirror channel 0, add zeros
+    BwdChannel<T> ch;
+    ch.init(p, b, dd);
+    const int c0 = seg * p.seg_chunks, c1 = min(p.nchunks, c0 + p.seg_chunks);
     float *ck = p.ckpt + (int64_t(b) * p.dim + dd) * p.nchunks * N;
 
-    // ---- pass A: forward recurrence, h at the start of every chunk
-    float h[N];
+    // ---- initial state of the segment and gradient at its end
+    uint64_t h2[8], g2[8];
+    {
+        float hv[N], gv[N];
 #pragma unroll
-    for (int n = 0; n < N; ++n)
-        h[n] = (p.h0 && live) ? p.h0[(int64_t(b) * p.dim + dd) * N + n] : 0.f;
-    for (int t = 0; t < p.L; ++t) {
-        if (t % TC == 0 && live) {
-            float4 *dst = reinterpret_cast<float4 *>(ck + (t / TC) * N);
+        for (int n = 0; n < N; ++n) {
+            hv[n] = (p.h0 && live) ? p.h0[(int64_t(b) * p.dim + dd) * N + n] : 0.f;
+            gv[n] = (p.dlast && live) ? p.dlast[(int64_t(b) * p.dim + dd) * N + n] : 0.f;
+        }
+        for (int j = 0; j < seg; ++j) {
+            const int64_t o = (int64_t(j) * p.tiles + tile) * 32 + lane;
+            const float s = __ldcg(p.aggS + o);
+#pragma unroll
+            for (int n = 0; n < N; ++n)
+                hv[n] = fmaf(ex2_approx(ch.al[n] * s), hv[n], __ldcg(p.aggE + o * N + n));
+        }
+        for (int j = p.segs - 1; j > seg; --j) {
+            const int64_t o = (int64_t(j) * p.tiles + tile) * 32 + lane;
+            const float s = __ldcg(p.aggS + o);
+#pragma unroll
+            for (int n = 0; n < N; ++n)
+                gv[n] = fmaf(ex2_approx(ch.al[n] * s), gv[n], __ldcg(p.aggG + o * N + n));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            h2[j] = live ? pk2(hv[2 * j], hv[2 * j + 1]) : pk2(0.f, 0.f);
+            g2[j] = live ? pk2(gv[2 * j], gv[2 * j + 1]) : pk2(0.f, 0.f);
+        }
+    }
+
+    // ---- pass A: forward over the segment, h at the start of every chunk
+    for (int c = c0; c < c1; ++c) {
+        const int t0 = c * TC, valid = min(TC, p.L - t0);
+        if (live) {
+            float4 *dst = reinterpret_cast<float4 *>(ck + c * N);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                dst[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+                dst[q] = make_float4(lo2(h2[2 * q]), hi2(h2[2 * q]), lo2(h2[2 * q + 1]),
+                                     hi2(h2[2 * q + 1]));
         }
-        float raw;
-        const float dt = bwd_step_size<T>(p, row_dl, t, bias, &raw);
-        const float dx = dt * bwd_ld(p.u, row_u + t, tag);
-        float a[N];
-        bwd_decays<FAST>(dt, al, pow_path, a);
-#pragma unroll
-        for (int n = 0; n < N; ++n)
-            h[n] = fmaf(a[n], h[n], dx * bwd_ld(p.B, bB + int64_t(n) * p.B_ns + t, tag));
+        bwd_stage_bc<T>(p, sm, b, t0, valid, false, lane);
+        bwd_forward_chunk<T, false>(p, ch, sm, t0, valid, h2, lane);
+        __syncwarp();
     }
-    __syncwarp();
 
     // ---- pass B: chunks backwards
-    float g[N], gA[N];
+    uint64_t gA2[8];
 #pragma unroll
-    for (int n = 0; n < N; ++n) {
-        g[n] = (p.dlast && live) ? p.dlast[(int64_t(b) * p.dim + dd) * N + n] : 0.f;
-        gA[n] = 0.f;
-    }
+    for (int j = 0; j < 8; ++j)
+        gA2[j] = pk2(0.f, 0.f);
     float gD = 0.f, gbias = 0.f;
-    for (int c = p.nchunks - 1; c >= 0; --c) {
-        const int t0 = c * TC;
-        const int tn = min(TC, p.L - t0);
-        float hc[N];  // state before the chunk
+    for (int c = c1 - 1; c >= c0; --c) {
+        const int t0 = c * TC, valid = min(TC, p.L - t0);
+        uint64_t hc2[8];  // state before the chunk
         {
             const float4 *src = reinterpret_cast<const float4 *>(ck + c * N);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 v = live ? src[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-                hc[4 * q] = v.x;
-                hc[4 * q + 1] = v.y;
-                hc[4 * q + 2] = v.z;
-                hc[4 * q + 3] = v.w;
+                hc2[2 * q] = pk2(v.x, v.y);
+                hc2[2 * q + 1] = pk2(v.z, v.w);
             }
         }
-        // recompute the chunk's states
+        bwd_stage_bc<T>(p, sm, b, t0, valid, true, lane);
         {
+            uint64_t hr[8];
 #pragma unroll
-            for (int n = 0; n < N; ++n)
-                h[n] = hc[n];
-            for (int i = 0; i < tn; ++i) {
-                const int t = t0 + i;
-                float raw;
-                const float dt = bwd_step_size<T>(p, row_dl, t, bias, &raw);
-                const float dx = dt * bwd_ld(p.u, row_u + t, tag);
-                float a[N];
-                bwd_decays<FAST>(dt, al, pow_path, a);
-#pragma unroll
-                for (int n = 0; n < N; ++n) {
-                    h[n] = fmaf(a[n], h[n], dx * bwd_ld(p.B, bB + int64_t(n) * p.B_ns + t, tag));
-                    s_h[i][n][lane] = h[n];
-                }
-            }
+            for (int j = 0; j < 8; ++j)
+                hr[j] = hc2[j];
+            bwd_forward_chunk<T, true>(p, ch, sm, t0, valid, hr, lane);
         }
         __syncwarp();
-        // reverse recurrence over the chunk
-        for (int i = tn - 1; i >= 0; --i) {
-            const int t = t0 + i;
-            float raw;
-            const float dt = bwd_step_size<T>(p, row_dl, t, bias, &raw);
-            const float x = bwd_ld(p.u, row_u + t, tag);
-            float a[N];
-            bwd_decays<FAST>(dt, al, pow_path, a);
-            float Bv[N], Cv[N], ht[N], hp[N];
+        float uv[8], dv[8], yv[8], zv[8];
+        bwd_ld8(p.u, ch.row_u + t0, valid, uv, tag);
+        bwd_ld8(p.delta, ch.row_dl + t0, valid, dv, tag);
+        bwd_ld8(p.dy, ch.row_dy + t0, valid, yv, tag);
+        if (p.z)
+            bwd_ld8(p.z, ch.row_z + t0, valid, zv, tag);
+        float o_du[8], o_dd[8], o_dz[8], red[8];
 #pragma unroll
-            for (int n = 0; n < N; ++n) {
-                Bv[n] = bwd_ld(p.B, bB + int64_t(n) * p.B_ns + t, tag);
-                Cv[n] = bwd_ld(p.C, bC + int64_t(n) * p.C_ns + t, tag);
-                ht[n] = s_h[i][n][lane];
-                hp[n] = i > 0 ? s_h[i - 1][n][lane] : hc[n];
+        for (int i = 0; i < TC; ++i) {
+            o_du[i] = o_dd[i] = o_dz[i] = red[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = TC - 1; i >= 0; --i) {
+            if (i >= valid)
+                continue;
+            uint64_t ht2[8], hp2[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                ht2[j] = pk2(sm.h[i][2 * j][lane], sm.h[i][2 * j + 1][lane]);
+                hp2[j] = i > 0 ? pk2(sm.h[i - 1][2 * j][lane], sm.h[i - 1][2 * j + 1][lane])
+                               : hc2[j];
             }
-            float out = dsk * x;
+            const float raw = dv[i] + ch.bias;
+            const float dt = bwd_step<FAST>(raw, p.softplus);
+            const float x = uv[i];
+            uint64_t a2[8];
+            bwd_decays<FAST>(dt, ch.al, ch.pow_path, a2);
+            uint64_t B2[8], C2[8];
+            {
+                const float4 *bq = reinterpret_cast<const float4 *>(sm.bc[i][0]);
+                const float4 *cq = reinterpret_cast<const float4 *>(sm.bc[i][1]);
 #pragma unroll
-            for (int n = 0; n < N; ++n)
-                out = fmaf(Cv[n], ht[n], out);
-            const float dyv = live ? bwd_ld(p.dy, row_dy + t, tag) : 0.f;
+                for (int q = 0; q < 4; ++q) {
+                    const float4 bb = bq[q], cc = cq[q];
+                    B2[2 * q] = pk2(bb.x, bb.y);
+                    B2[2 * q + 1] = pk2(bb.z, bb.w);
+                    C2[2 * q] = pk2(cc.x, cc.y);
+                    C2[2 * q + 1] = pk2(cc.z, cc.w);
+                }
+            }
+            uint64_t Y2 = mul2(C2[0], ht2[0]);
+#pragma unroll
+            for (int j = 1; j < 8; ++j)
+                Y2 = fma2(C2[j], ht2[j], Y2);
+            const float out = fmaf(ch.dsk, x, lo2(Y2) + hi2(Y2));
+            const float dyv = live ? yv[i] : 0.f;
             float dout = dyv;
             if (p.z) {
-                const float zv = bwd_ld(p.z, row_z + t, tag);
-                const float sg = 1.f / (1.f + __expf(-zv));
-                if (live)
-                    bwd_st(p.dz, row_dz + t, dyv * out * (sg * (1.f + zv * (1.f - sg))), tag);
-                dout = dyv * zv * sg;
+                const float zz = zv[i];
+                const float sg = 1.f / (1.f + __expf(-zz));
+                o_dz[i] = dyv * out * (sg * (1.f + zz * (1.f - sg)));
+                dout = dyv * zz * sg;
             }
-            float dx = dout * dsk, ddt = 0.f;
             gD = fmaf(dout, x, gD);
+            const uint64_t DO = pk2(dout, dout), DT = pk2(dt, dt), X = pk2(x, x);
+            uint64_t dx2 = pk2(0.f, 0.f), ddt2 = pk2(0.f, 0.f);
             float v[32];  // dB (states 0..15), dC (states 0..15) of this channel
 #pragma unroll
-            for (int n = 0; n < N; ++n) {
-                g[n] = fmaf(dout, Cv[n], g[n]);
-                v[N + n] = dout * ht[n];
-                v[n] = g[n] * dt * x;
-                dx = fmaf(g[n] * dt, Bv[n], dx);
-                const float ah = a[n] * hp[n];
-                ddt = fmaf(g[n], fmaf(An[n], ah, Bv[n] * x), ddt);
-                gA[n] = fmaf(g[n] * dt, ah, gA[n]);
-                g[n] *= a[n];
+            for (int j = 0; j < 8; ++j) {
+                g2[j] = fma2(DO, C2[j], g2[j]);
+                const uint64_t vc = mul2(DO, ht2[j]);
+                const uint64_t gdt = mul2(g2[j], DT);
+                const uint64_t vb = mul2(gdt, X);
+                v[2 * j] = lo2(vb);
+                v[2 * j + 1] = hi2(vb);
+                v[N + 2 * j] = lo2(vc);
+                v[N + 2 * j + 1] = hi2(vc);
+                dx2 = fma2(gdt, B2[j], dx2);
+                const uint64_t ah = mul2(a2[j], hp2[j]);
+                ddt2 = fma2(g2[j], fma2(ch.An2[j], ah, mul2(B2[j], X)), ddt2);
+                gA2[j] = fma2(gdt, ah, gA2[j]);
+                g2[j] = mul2(g2[j], a2[j]);
             }
-            float dDelta = ddt;
-            if (p.softplus)
-                dDelta = ddt / (1.f + __expf(-raw));
+            const float dx = fmaf(dout, ch.dsk, lo2(dx2) + hi2(dx2));
+            const float ddt = lo2(ddt2) + hi2(ddt2);
+            const float dDelta = p.softplus ? ddt / (1.f + __expf(-raw)) : ddt;
             gbias += dDelta;
-            if (live) {
-                bwd_st(p.du, row_du + t, dx, tag);
-                bwd_st(p.ddelta, row_dd + t, dDelta, tag);
-            } else {
+            o_du[i] = dx;
+            o_dd[i] = dDelta;
+            if (!live) {
 #pragma unroll
                 for (int k = 0; k < 32; ++k)
                     v[k] = 0.f;  // lanes past the last channel add exact zeros
@@ -276,21 +549,43 @@ selscan_bwd_kernel(const BwdParams p)
                     v[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
                 }
             }
-            float *dst = lane < N ? p.dB + (int64_t(b) * N + lane) * p.L + t
-                                  : p.dC + (int64_t(b) * N + (lane - N)) * p.L + t;
-            atomicAdd(dst, v[0]);
+            red[i] = v[0];
+        }
+        if (live) {
+            bwd_st8(p.du, ch.row_du + t0, valid, o_du, tag);
+            bwd_st8(p.ddelta, ch.row_dd + t0, valid, o_dd, tag);
+            if (p.z)
+                bwd_st8(p.dz, ch.row_dz + t0, valid, o_dz, tag);
+        }
+        {
+            float *dst = lane < N ? p.dB + (int64_t(b) * N + lane) * p.L + t0
+                                  : p.dC + (int64_t(b) * N + (lane - N)) * p.L + t0;
+            if (valid >= 8 && (p.L & 3) == 0) {  // rows of dB / dC 16-byte aligned
+                atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(red[0], red[1], red[2], red[3]));
+                atomicAdd(reinterpret_cast<float4 *>(dst) + 1,
+                          make_float4(red[4], red[5], red[6], red[7]));
+            } else {
+#pragma unroll
+                for (int i = 0; i < TC; ++i)
+                    if (i < valid)
+                        atomicAdd(dst + i, red[i]);
+            }
         }
         __syncwarp();
     }
     if (live) {
-        if (p.dh0) {
+        if (p.dh0 && seg == 0) {
 #pragma unroll
-            for (int n = 0; n < N; ++n)
-                p.dh0[(int64_t(b) * p.dim + d) * N + n] = g[n];
+            for (int j = 0; j < 8; ++j) {
+                p.dh0[(int64_t(b) * p.dim + d) * N + 2 * j] = lo2(g2[j]);
+                p.dh0[(int64_t(b) * p.dim + d) * N + 2 * j + 1] = hi2(g2[j]);
+            }
         }
 #pragma unroll
-        for (int n = 0; n < N; ++n)
-            atomicAdd(p.dA + int64_t(d) * N + n, gA[n]);
+        for (int j = 0; j < 8; ++j) {
+            atomicAdd(p.dA + int64_t(d) * N + 2 * j, lo2(gA2[j]));
+            atomicAdd(p.dA + int64_t(d) * N + 2 * j + 1, hi2(gA2[j]));
+        }
         if (p.dD)
             atomicAdd(p.dD + d, gD);
         if (p.dbias)

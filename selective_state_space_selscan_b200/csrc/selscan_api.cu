@@ -1178,26 +1178,6 @@ extern "C" selscan_status selscan_step_scalarA(selscan_tensor *state, const sels
 // ------------------------------------------------------------ backward
 namespace {
 
-// A sequence tensor (d0, d1, L), time stride 1, element-aligned (the
-// backward reads it with plain loads, no bulk copies).
-selscan_status check_seq_plain(const selscan_tensor *t, int64_t d0, int64_t d1, int64_t L,
-                               int32_t dtype)
-{
-    if (!present(t))
-        return SELSCAN_ERR_NULL;
-    if (t->ndim != 3 || t->shape[0] != d0 || t->shape[1] != d1 || t->shape[2] != L)
-        return SELSCAN_ERR_SHAPE;
-    if (t->dtype != dtype)
-        return SELSCAN_ERR_DTYPE;
-    if (d0 == 0 || d1 == 0 || L == 0)
-        return SELSCAN_OK;
-    if ((L > 1 && t->stride[2] != 1) || t->stride[0] < 0 || t->stride[1] < 0)
-        return SELSCAN_ERR_STRIDE;
-    if (reinterpret_cast<uintptr_t>(t->data) % elem_size(dtype))
-        return SELSCAN_ERR_ALIGN;
-    return SELSCAN_OK;
-}
-
 }  // namespace
 
 extern "C" selscan_status selscan_bwd(
@@ -1223,11 +1203,11 @@ extern "C" selscan_status selscan_bwd(
     selscan_status st;
     for (const selscan_tensor *t : {u, delta, dy, static_cast<const selscan_tensor *>(du),
                                     static_cast<const selscan_tensor *>(ddelta)})
-        if ((st = check_seq_plain(t, batch, dim, L, dt)) != SELSCAN_OK) return st;
+        if ((st = check_seq(t, batch, dim, L, dt)) != SELSCAN_OK) return st;
     const bool gate = z && z->data;
     if (gate) {
-        if ((st = check_seq_plain(z, batch, dim, L, dt)) != SELSCAN_OK) return st;
-        if ((st = check_seq_plain(dz, batch, dim, L, dt)) != SELSCAN_OK) return st;
+        if ((st = check_seq(z, batch, dim, L, dt)) != SELSCAN_OK) return st;
+        if ((st = check_seq(dz, batch, dim, L, dt)) != SELSCAN_OK) return st;
     }
     // B, C: (batch, N, L) or (batch, 1, N, L); dB, dC: (batch, N, L) fp32 contiguous
     selscan_tensor Bv{}, Cv{};
@@ -1245,7 +1225,7 @@ extern "C" selscan_status selscan_bwd(
             v.stride[1] = t->stride[2];
             v.stride[2] = t->stride[3];
         }
-        if ((st = check_seq_plain(&v, batch, N, L, dt)) != SELSCAN_OK) return st;
+        if ((st = check_seq(&v, batch, N, L, dt)) != SELSCAN_OK) return st;
         (k ? Cv : Bv) = v;
     }
     {
@@ -1340,18 +1320,61 @@ extern "C" selscan_status selscan_bwd(
     prm.dbias = static_cast<float *>(ddelta_bias ? ddelta_bias->data : nullptr);
     prm.dh0 = static_cast<float *>(dh0 ? dh0->data : nullptr);
 
-    // checkpoints of h every kBwdT tokens: [batch][dim][nchunks][16] fp32
+    // Units: (batch row, 32 channels) x time segments, one warp each.  As
+    // many segments as fit in one wave of resident warps (a second, partial
+    // wave would double the time of its units), at least 32 chunks each.
+    prm.tiles_per_batch = int((dim + 31) / 32);
+    prm.tiles = int(batch) * prm.tiles_per_batch;
+    {
+        int per_sm = 0;
+        const cudaError_t oe =
+            dt == SELSCAN_BF16
+                ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                      &per_sm, selscan_bwd_kernel<__nv_bfloat16>, 32, 0)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
+                                                                selscan_bwd_kernel<float>, 32, 0);
+        if (oe != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        const int64_t slots = int64_t(per_sm) * di->sm_count;
+        const int64_t want = std::max<int64_t>(1, slots / prm.tiles);
+        const int64_t max_segs = std::max<int64_t>(1, prm.nchunks / 32);
+        int64_t S = std::max<int64_t>(1, std::min(want, max_segs));
+        const int64_t seg_chunks = (prm.nchunks + S - 1) / S;
+        S = (prm.nchunks + seg_chunks - 1) / seg_chunks;
+        if (int64_t(prm.tiles) * S > 0x7fffffffll)
+            return SELSCAN_ERR_UNSUPPORTED;
+        prm.segs = int(S);
+        prm.seg_chunks = int(seg_chunks);
+    }
+    const int64_t units = int64_t(prm.tiles) * prm.segs;
+    // scratch: checkpoints of h every kBwdT tokens [batch][dim][nchunks][16],
+    // segment aggregates E, G [units][32][16] and S [units][32] (fp32)
     const size_t ck_bytes = size_t(batch) * dim * prm.nchunks * kBwdN * 4;
+    const size_t agg_bytes = prm.segs > 1 ? size_t(units) * 32 * kBwdN * 4 : 0;
+    const size_t s_bytes = prm.segs > 1 ? size_t(units) * 32 * 4 : 0;
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, ck_bytes, stream) != cudaSuccess)
+    if (cudaMallocAsync(&ws, ck_bytes + 2 * agg_bytes + s_bytes, stream) != cudaSuccess)
         return SELSCAN_ERR_CUDA;
-    prm.ckpt = static_cast<float *>(ws);
-    const dim3 grid(unsigned((dim + 31) / 32), unsigned(batch));
-    if (dt == SELSCAN_BF16)
-        selscan_bwd_kernel<__nv_bfloat16><<<grid, 32, 0, stream>>>(prm);
-    else
-        selscan_bwd_kernel<float><<<grid, 32, 0, stream>>>(prm);
-    const cudaError_t le = counted_launch();
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    prm.ckpt = reinterpret_cast<float *>(wsb);
+    prm.aggE = reinterpret_cast<float *>(wsb + ck_bytes);
+    prm.aggG = reinterpret_cast<float *>(wsb + ck_bytes + agg_bytes);
+    prm.aggS = reinterpret_cast<float *>(wsb + ck_bytes + 2 * agg_bytes);
+    cudaError_t le = cudaSuccess;
+    if (prm.segs > 1) {
+        if (dt == SELSCAN_BF16)
+            bwd_agg_kernel<__nv_bfloat16><<<unsigned(units), 32, 0, stream>>>(prm);
+        else
+            bwd_agg_kernel<float><<<unsigned(units), 32, 0, stream>>>(prm);
+        le = counted_launch();
+    }
+    if (le == cudaSuccess) {
+        if (dt == SELSCAN_BF16)
+            selscan_bwd_kernel<__nv_bfloat16><<<unsigned(units), 32, 0, stream>>>(prm);
+        else
+            selscan_bwd_kernel<float><<<unsigned(units), 32, 0, stream>>>(prm);
+        le = counted_launch();
+    }
     cudaFreeAsync(ws, stream);
     return le == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
 }

@@ -90,7 +90,12 @@ def test_bf16(gate, softplus):
         inp["delta"] = synthetic.round_bf16(np.abs(inp["delta"]) * 0.05)
         inp["delta_bias"] = None
     dy = _dy(inp, 85)
-    compare(run(inp, dy, "bf16", softplus=softplus), ref(inp, dy, softplus=softplus), "bf16")
+    # an initial state and a final-state gradient exercise the segment folds
+    rng = np.random.default_rng(86)
+    h0 = rng.standard_normal((2, 192, 16)).astype(np.float32) if gate else None
+    dlast = rng.standard_normal((2, 192, 16)).astype(np.float32) if gate else None
+    compare(run(inp, dy, "bf16", h0, dlast, softplus=softplus),
+            ref(inp, dy, h0, dlast, softplus=softplus), "bf16")
 
 
 def test_general_A_no_bias():
