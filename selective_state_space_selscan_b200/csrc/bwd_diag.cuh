@@ -71,38 +71,6 @@ struct BwdParams {
     float *aggE, *aggG, *aggS;       // [units][32][16], [units][32][16], [units][32]
 };
 
-// 8 consecutive elements of a row (16-byte aligned start) as fp32; elements
-// at or past `valid` read as zero.
-__device__ __forceinline__ void bwd_ld8(const void *base, int64_t off, int valid, float (&v)[8],
-                                        const __nv_bfloat16 *)
-{
-    const __nv_bfloat16 *p = static_cast<const __nv_bfloat16 *>(base) + off;
-    if (valid >= 8) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(p);
-        unpack8_bf16(q, v);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            v[i] = i < valid ? __bfloat162float(p[i]) : 0.f;
-    }
-}
-
-__device__ __forceinline__ void bwd_ld8(const void *base, int64_t off, int valid, float (&v)[8],
-                                        const float *)
-{
-    const float *p = static_cast<const float *>(base) + off;
-    if (valid >= 8) {
-        const float4 a = reinterpret_cast<const float4 *>(p)[0];
-        const float4 b = reinterpret_cast<const float4 *>(p)[1];
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            v[i] = i < valid ? p[i] : 0.f;
-    }
-}
-
 __device__ __forceinline__ void bwd_st8(void *base, int64_t off, int valid, const float (&v)[8],
                                         const __nv_bfloat16 *)
 {
@@ -174,22 +142,103 @@ struct BwdSmem {
     float h[kBwdT][kBwdN][32];
 };
 
-// Stage B (and C) of tokens [t0, t0 + valid) of batch row b as fp32.
+// One chunk's raw inputs, copied asynchronously: per lane its channel's 8
+// tokens of u, delta, dy, z (KV 16-byte vectors each), one row of B (lanes
+// 0..15) or C (lanes 16..31), and its checkpoint.
+template <int KV>
+struct BwdStage {
+    uint4 u[KV][32], dl[KV][32], dy[KV][32], z[KV][32], bc[KV][32];
+    float4 ck[4][32];
+};
+
+constexpr int kLdU = 1, kLdDl = 2, kLdDy = 4, kLdZ = 8, kLdB = 16, kLdC = 32, kLdCk = 64;
+
 template <typename T>
-__device__ __forceinline__ void bwd_stage_bc(const BwdParams &p, BwdSmem &sm, int b, int t0,
-                                             int valid, bool withC, int lane)
+constexpr int bwd_kv() { return int(sizeof(T)) * kBwdT / 16; }
+
+// Issue the copies of tokens [t0, t0 + valid) of this lane's rows (`what` is
+// a mask of kLd*); the caller commits the group.
+template <typename T, int KV>
+__device__ __forceinline__ void bwd_issue(const BwdParams &p, BwdStage<KV> &st, int64_t row_u,
+                                          int64_t row_dl, int64_t row_dy, int64_t row_z, int b,
+                                          int t0, int valid, int lane, int what, const float *ck)
 {
-    const T *tag = nullptr;
-    if (lane < kBwdN || withC) {
-        const int n = lane & 15;
+    constexpr int EPV = 16 / int(sizeof(T));  // elements per 16-byte vector
+    const T *base;
+#pragma unroll
+    for (int k = 0; k < KV; ++k) {
+        const int left = valid - k * EPV;
+        const uint32_t bytes = uint32_t(left <= 0 ? 0 : (left >= EPV ? 16 : left * int(sizeof(T))));
+        const int off = t0 + (left > 0 ? k * EPV : 0);
+        if (what & kLdU) {
+            base = static_cast<const T *>(p.u);
+            cp_async16(&st.u[k][lane], base + row_u + off, bytes);
+        }
+        if (what & kLdDl) {
+            base = static_cast<const T *>(p.delta);
+            cp_async16(&st.dl[k][lane], base + row_dl + off, bytes);
+        }
+        if (what & kLdDy) {
+            base = static_cast<const T *>(p.dy);
+            cp_async16(&st.dy[k][lane], base + row_dy + off, bytes);
+        }
+        if ((what & kLdZ) && p.z) {
+            base = static_cast<const T *>(p.z);
+            cp_async16(&st.z[k][lane], base + row_z + off, bytes);
+        }
         const bool isC = lane >= kBwdN;
+        if ((what & (isC ? kLdC : kLdB))) {
+            const int n = lane & 15;
+            base = static_cast<const T *>(isC ? p.C : p.B);
+            const int64_t row = int64_t(b) * (isC ? p.C_bs : p.B_bs) +
+                                int64_t(n) * (isC ? p.C_ns : p.B_ns);
+            cp_async16(&st.bc[k][lane], base + row + off, bytes);
+        }
+    }
+    if (what & kLdCk) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            cp_async16(&st.ck[q][lane], ck + 4 * q, 16);
+    }
+}
+
+__device__ __forceinline__ void bwd_unpack(const uint4 (&v)[1], float (&f)[8], const __nv_bfloat16 *)
+{
+    unpack8_bf16(v[0], f);
+}
+
+__device__ __forceinline__ void bwd_unpack(const uint4 (&v)[2], float (&f)[8], const float *)
+{
+    f[0] = __uint_as_float(v[0].x); f[1] = __uint_as_float(v[0].y);
+    f[2] = __uint_as_float(v[0].z); f[3] = __uint_as_float(v[0].w);
+    f[4] = __uint_as_float(v[1].x); f[5] = __uint_as_float(v[1].y);
+    f[6] = __uint_as_float(v[1].z); f[7] = __uint_as_float(v[1].w);
+}
+
+// This lane's 8 values of a staged tensor.
+template <typename T, int KV>
+__device__ __forceinline__ void bwd_vals(const uint4 (&src)[KV][32], int lane, float (&f)[8])
+{
+    uint4 v[KV];
+#pragma unroll
+    for (int k = 0; k < KV; ++k)
+        v[k] = src[k][lane];
+    const T *tag = nullptr;
+    bwd_unpack(v, f, tag);
+}
+
+// Staged B / C rows -> fp32 [token][n] for the whole warp.
+template <typename T, int KV>
+__device__ __forceinline__ void bwd_bc_to_smem(const BwdStage<KV> &st, BwdSmem &sm, int lane,
+                                               bool withC)
+{
+    if (lane < kBwdN || withC) {
         float v[8];
-        bwd_ld8(isC ? p.C : p.B,
-                int64_t(b) * (isC ? p.C_bs : p.B_bs) + int64_t(n) * (isC ? p.C_ns : p.B_ns) + t0,
-                valid, v, tag);
+        bwd_vals<T, KV>(st.bc, lane, v);
+        const int isC = lane >= kBwdN;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            sm.bc[i][isC][n] = v[i];
+            sm.bc[i][isC][lane & 15] = v[i];
     }
     __syncwarp();
 }
@@ -231,14 +280,11 @@ struct BwdChannel {
 // when `keep` is set the state after each token goes to shared memory.
 template <typename T, bool KEEP>
 __device__ __forceinline__ void bwd_forward_chunk(const BwdParams &p, const BwdChannel<T> &ch,
-                                                  BwdSmem &sm, int t0, int valid,
-                                                  uint64_t (&h2)[8], int lane)
+                                                  BwdSmem &sm, int valid, const float (&uv)[8],
+                                                  const float (&dv)[8], uint64_t (&h2)[8],
+                                                  int lane)
 {
     constexpr bool FAST = !std::is_same<T, float>::value;
-    const T *tag = nullptr;
-    float uv[8], dv[8];
-    bwd_ld8(p.u, ch.row_u + t0, valid, uv, tag);
-    bwd_ld8(p.delta, ch.row_dl + t0, valid, dv, tag);
 #pragma unroll
     for (int i = 0; i < kBwdT; ++i) {
         if (i >= valid)
@@ -273,7 +319,6 @@ __global__ void __launch_bounds__(32)
 bwd_agg_kernel(const BwdParams p)
 {
     constexpr bool FAST = !std::is_same<T, float>::value;
-    const T *tag = nullptr;
     __shared__ __align__(16) BwdSmem sm;
     const int lane = threadIdx.x;
     const int unit = blockIdx.x;
@@ -285,31 +330,45 @@ bwd_agg_kernel(const BwdParams p)
     ch.init(p, b, live ? d : 0);
     const int c0 = seg * p.seg_chunks, c1 = min(p.nchunks, c0 + p.seg_chunks);
 
-    // forward from zero: end state and the sum of step sizes
+    constexpr int KV = bwd_kv<T>();
+    __shared__ __align__(16) BwdStage<KV> st[2];
+
+    // forward from zero: end state (not needed for the last segment) and the
+    // sum of step sizes; chunk c+1's inputs are copied while c is computed
     uint64_t h2[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
         h2[j] = pk2(0.f, 0.f);
     float ssum = 0.f;
-    if (seg < p.segs - 1) {
-        for (int c = c0; c < c1; ++c) {
-            const int t0 = c * kBwdT, valid = min(kBwdT, p.L - t0);
-            bwd_stage_bc<T>(p, sm, b, t0, valid, false, lane);
-            bwd_forward_chunk<T, false>(p, ch, sm, t0, valid, h2, lane);
-            __syncwarp();
-        }
-    }
     {
-        // the sum of step sizes (every segment but the first is folded over)
+        const bool fwd = seg < p.segs - 1;
+        const int what = fwd ? (kLdU | kLdDl | kLdB) : kLdDl;
+        int buf = 0;
+        bwd_issue<T, KV>(p, st[0], ch.row_u, ch.row_dl, ch.row_dy, ch.row_z, b, c0 * kBwdT,
+                         min(kBwdT, p.L - c0 * kBwdT), lane, what, nullptr);
+        cp_async_commit();
         for (int c = c0; c < c1; ++c) {
             const int t0 = c * kBwdT, valid = min(kBwdT, p.L - t0);
-            float dv[8];
-            bwd_ld8(p.delta, ch.row_dl + t0, valid, dv, tag);
+            if (c + 1 < c1)
+                bwd_issue<T, KV>(p, st[buf ^ 1], ch.row_u, ch.row_dl, ch.row_dy, ch.row_z, b,
+                                 t0 + kBwdT, min(kBwdT, p.L - t0 - kBwdT), lane, what, nullptr);
+            cp_async_commit();
+            cp_async_wait<1>();
+            float uv[8], dv[8];
+            bwd_vals<T, KV>(st[buf].dl, lane, dv);
 #pragma unroll
             for (int i = 0; i < kBwdT; ++i)
                 if (i < valid)
                     ssum += bwd_step<FAST>(dv[i] + ch.bias, p.softplus);
+            if (fwd) {
+                bwd_vals<T, KV>(st[buf].u, lane, uv);
+                bwd_bc_to_smem<T, KV>(st[buf], sm, lane, false);
+                bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane);
+            }
+            __syncwarp();
+            buf ^= 1;
         }
+        cp_async_wait<0>();
     }
     // backward from zero: g_{t-1} = abar_t (g_t + dout_t C_t)
     uint64_t g2[8];
@@ -317,14 +376,27 @@ bwd_agg_kernel(const BwdParams p)
     for (int j = 0; j < 8; ++j)
         g2[j] = pk2(0.f, 0.f);
     if (seg > 0) {
+        const int what = kLdDl | kLdDy | kLdZ | kLdC;
+        int buf = 0;
+        {
+            const int cl = c1 - 1;
+            bwd_issue<T, KV>(p, st[0], ch.row_u, ch.row_dl, ch.row_dy, ch.row_z, b, cl * kBwdT,
+                             min(kBwdT, p.L - cl * kBwdT), lane, what, nullptr);
+        }
+        cp_async_commit();
         for (int c = c1 - 1; c >= c0; --c) {
             const int t0 = c * kBwdT, valid = min(kBwdT, p.L - t0);
-            bwd_stage_bc<T>(p, sm, b, t0, valid, true, lane);
+            if (c > c0)
+                bwd_issue<T, KV>(p, st[buf ^ 1], ch.row_u, ch.row_dl, ch.row_dy, ch.row_z, b,
+                                 t0 - kBwdT, kBwdT, lane, what, nullptr);
+            cp_async_commit();
+            cp_async_wait<1>();
+            bwd_bc_to_smem<T, KV>(st[buf], sm, lane, true);
             float dv[8], yv[8], zv[8];
-            bwd_ld8(p.delta, ch.row_dl + t0, valid, dv, tag);
-            bwd_ld8(p.dy, ch.row_dy + t0, valid, yv, tag);
+            bwd_vals<T, KV>(st[buf].dl, lane, dv);
+            bwd_vals<T, KV>(st[buf].dy, lane, yv);
             if (p.z)
-                bwd_ld8(p.z, ch.row_z + t0, valid, zv, tag);
+                bwd_vals<T, KV>(st[buf].z, lane, zv);
 #pragma unroll
             for (int i = kBwdT - 1; i >= 0; --i) {
                 if (i >= valid)
@@ -345,7 +417,9 @@ bwd_agg_kernel(const BwdParams p)
                 }
             }
             __syncwarp();
+            buf ^= 1;
         }
+        cp_async_wait<0>();
     }
     if (live) {
         const int64_t o = (int64_t(unit) * 32 + lane) * kBwdN;
@@ -411,18 +485,40 @@ selscan_bwd_kernel(const BwdParams p)
         }
     }
 
-    // ---- pass A: forward over the segment, h at the start of every chunk
-    for (int c = c0; c < c1; ++c) {
-        const int t0 = c * TC, valid = min(TC, p.L - t0);
-        if (live) {
-            float4 *dst = reinterpret_cast<float4 *>(ck + c * N);
+    constexpr int KV = bwd_kv<T>();
+    __shared__ __align__(16) BwdStage<KV> st[2];
+
+    // ---- pass A: forward over the segment, h at the start of every chunk;
+    //      chunk c+1's inputs are copied while c is computed
+    {
+        const int what = kLdU | kLdDl | kLdB;
+        int buf = 0;
+        bwd_issue<T, KV>(p, st[0], ch.row_u, ch.row_dl, ch.row_dy, ch.row_z, b, c0 * TC,
+                         min(TC, p.L - c0 * TC), lane, what, nullptr);
+        cp_async_commit();
+        for (int c = c0; c < c1; ++c) {
+            const int t0 = c * TC, valid = min(TC, p.L - t0);
+            if (c + 1 < c1)
+                bwd_issue<T, KV>(p, st[buf ^ 1], ch.row_u, ch.row_dl, ch.row_dy, ch.row_z, b,
+                                 t0 + TC, min(TC, p.L - t0 - TC), lane, what, nullptr);
+            cp_async_commit();
+            if (live) {
+                float4 *dst = reinterpret_cast<float4 *>(ck + c * N);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                dst[q] = make_float4(lo2(h2[2 * q]), hi2(h2[2 * q]), lo2(h2[2 * q + 1]),
-                                     hi2(h2[2 * q + 1]));
+                for (int q = 0; q < 4; ++q)
+                    dst[q] = make_float4(lo2(h2[2 * q]), hi2(h2[2 * q]), lo2(h2[2 * q + 1]),
+                                         hi2(h2[2 * q + 1]));
+            }
+            cp_async_wait<1>();
+            float uv[8], dv[8];
+            bwd_vals<T, KV>(st[buf].u, lane, uv);
+            bwd_vals<T, KV>(st[buf].dl, lane, dv);
+            bwd_bc_to_smem<T, KV>(st[buf], sm, lane, false);
+            bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane);
+            __syncwarp();
+            buf ^= 1;
         }
-        bwd_stage_bc<T>(p, sm, b, t0, valid, false, lane);
-        bwd_forward_chunk<T, false>(p, ch, sm, t0, valid, h2, lane);
+        cp_async_wait<0>();
         __syncwarp();
     }
 
@@ -432,33 +528,44 @@ selscan_bwd_kernel(const BwdParams p)
     for (int j = 0; j < 8; ++j)
         gA2[j] = pk2(0.f, 0.f);
     float gD = 0.f, gbias = 0.f;
+    const int whatB = kLdU | kLdDl | kLdDy | kLdZ | kLdB | kLdC | kLdCk;
+    int bufB = 0;
+    {
+        const int cl = c1 - 1;
+        bwd_issue<T, KV>(p, st[0], ch.row_u, ch.row_dl, ch.row_dy, ch.row_z, b, cl * TC,
+                         min(TC, p.L - cl * TC), lane, whatB, ck + cl * N);
+    }
+    cp_async_commit();
     for (int c = c1 - 1; c >= c0; --c) {
         const int t0 = c * TC, valid = min(TC, p.L - t0);
+        if (c > c0)
+            bwd_issue<T, KV>(p, st[bufB ^ 1], ch.row_u, ch.row_dl, ch.row_dy, ch.row_z, b,
+                             t0 - TC, TC, lane, whatB, ck + (c - 1) * N);
+        cp_async_commit();
+        cp_async_wait<1>();
+        const BwdStage<KV> &cur = st[bufB];
         uint64_t hc2[8];  // state before the chunk
-        {
-            const float4 *src = reinterpret_cast<const float4 *>(ck + c * N);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = live ? src[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-                hc2[2 * q] = pk2(v.x, v.y);
-                hc2[2 * q + 1] = pk2(v.z, v.w);
-            }
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = live ? cur.ck[q][lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+            hc2[2 * q] = pk2(v.x, v.y);
+            hc2[2 * q + 1] = pk2(v.z, v.w);
         }
-        bwd_stage_bc<T>(p, sm, b, t0, valid, true, lane);
+        float uv[8], dv[8], yv[8], zv[8];
+        bwd_vals<T, KV>(cur.u, lane, uv);
+        bwd_vals<T, KV>(cur.dl, lane, dv);
+        bwd_vals<T, KV>(cur.dy, lane, yv);
+        if (p.z)
+            bwd_vals<T, KV>(cur.z, lane, zv);
+        bwd_bc_to_smem<T, KV>(cur, sm, lane, true);
         {
             uint64_t hr[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 hr[j] = hc2[j];
-            bwd_forward_chunk<T, true>(p, ch, sm, t0, valid, hr, lane);
+            bwd_forward_chunk<T, true>(p, ch, sm, valid, uv, dv, hr, lane);
         }
         __syncwarp();
-        float uv[8], dv[8], yv[8], zv[8];
-        bwd_ld8(p.u, ch.row_u + t0, valid, uv, tag);
-        bwd_ld8(p.delta, ch.row_dl + t0, valid, dv, tag);
-        bwd_ld8(p.dy, ch.row_dy + t0, valid, yv, tag);
-        if (p.z)
-            bwd_ld8(p.z, ch.row_z + t0, valid, zv, tag);
         float o_du[8], o_dd[8], o_dz[8], red[8];
 #pragma unroll
         for (int i = 0; i < TC; ++i) {
@@ -572,7 +679,9 @@ selscan_bwd_kernel(const BwdParams p)
             }
         }
         __syncwarp();
+        bufB ^= 1;
     }
+    cp_async_wait<0>();
     if (live) {
         if (p.dh0 && seg == 0) {
 #pragma unroll

@@ -190,6 +190,26 @@ __device__ __forceinline__ bool spin_flag(const uint32_t *flag, uint32_t want,
     return true;
 }
 
+// ------------------------------------------- asynchronous 16-byte copies
+// global -> shared, `src_bytes` (0..16) read and the rest of the 16 bytes
+// zero-filled; completion tracked per thread by commit / wait groups.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(smem_addr(smem_dst)), "l"(gsrc), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory");
+}
+
 // ------------------------------------------- fast special functions
 __device__ __forceinline__ float ex2_approx(float x)
 {
