@@ -139,8 +139,8 @@ SELSCAN_API selscan_status selscan_fwd_h0(const selscan_tensor *u, const selscan
  *   y          (batch, H*P, L)  BF16; written
  *   last_state (batch, H, P, N) F32, contiguous; may be NULL; written
  *
- * Built for N = 128, P = 64, G = 1; other sizes return
- * SELSCAN_ERR_UNSUPPORTED.
+ * Built for N = 128, P = 64 and any number of groups G dividing H; other
+ * sizes return SELSCAN_ERR_UNSUPPORTED.
  */
 SELSCAN_API selscan_status selscan_fwd_scalarA(const selscan_tensor *x,
                                    const selscan_tensor *dt,

@@ -641,7 +641,7 @@ static selscan_status scalarA_impl(const selscan_tensor *x, const selscan_tensor
         if ((st = check_param(last_state, 4, sshape, true)) != SELSCAN_OK) return st;
         if ((st = check_param(h0, 4, sshape, true)) != SELSCAN_OK) return st;
     }
-    if (N != kSsdN || headdim != kSsdP || G != 1)
+    if (N != kSsdN || headdim != kSsdP)
         return SELSCAN_ERR_UNSUPPORTED;
     if (batch > 65535 || L > (int64_t(1) << 31) - 1024)
         return SELSCAN_ERR_UNSUPPORTED;
@@ -667,9 +667,10 @@ static selscan_status scalarA_impl(const selscan_tensor *x, const selscan_tensor
     // B/C (batch, 1, N, L) -> 3-D maps over (L, N, batch); x over (L, H*P, batch)
     // y (batch, H*P, L) is written back through the same kind of map
     CUtensorMap tm_C, tm_B, tm_X, tm_Y;
-    if (!encode_3d(&tm_C, C->data, SELSCAN_BF16, L, N, batch, C->stride[2], C->stride[0], 64,
+    // B/C (batch, G, N, L) viewed as (batch, G*N, L): head h loads rows g*N .. g*N+N-1
+    if (!encode_3d(&tm_C, C->data, SELSCAN_BF16, L, G * N, batch, C->stride[2], C->stride[0], 64,
                    kSsdN) ||
-        !encode_3d(&tm_B, B->data, SELSCAN_BF16, L, N, batch, B->stride[2], B->stride[0], 64,
+        !encode_3d(&tm_B, B->data, SELSCAN_BF16, L, G * N, batch, B->stride[2], B->stride[0], 64,
                    kSsdN) ||
         !encode_3d(&tm_X, x->data, SELSCAN_BF16, L, dim, batch, x->stride[1], x->stride[0], 64,
                    kSsdP) ||
@@ -681,6 +682,7 @@ static selscan_status scalarA_impl(const selscan_tensor *x, const selscan_tensor
     prm.H = int(H);
     prm.L = int(L);
     prm.nchunks = int((L + kSsdQ - 1) / kSsdQ);
+    prm.heads_per_group = int(H / G);
     prm.dt = static_cast<const float *>(dt->data);
     prm.dt_bs = dt->stride[0];
     prm.dt_hs = dt->stride[1];

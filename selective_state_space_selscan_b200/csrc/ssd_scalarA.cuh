@@ -60,6 +60,7 @@ constexpr int kSsdWG = 4;   // warpgroups per CTA
 
 struct SsdParams {
     int batch, H, L, nchunks;
+    int heads_per_group;       // head h reads B/C group h / heads_per_group
     const float *dt;           // (batch, H, L), time stride 1
     int64_t dt_bs, dt_hs;
     const float *dt_bias;      // (H) or null
@@ -162,10 +163,11 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
         uint8_t *cs = smem + Lay::kC + buf * 32768;
         uint8_t *bs = smem + Lay::kB + buf * 32768;
         uint8_t *xs = smem + Lay::kX + buf * 16384;
-        tma_load_3d(cs, &tm_C, &bar_tma[buf], t0, 0, b);
-        tma_load_3d(cs + 16384, &tm_C, &bar_tma[buf], t0 + 64, 0, b);
-        tma_load_3d(bs, &tm_B, &bar_tma[buf], t0, 0, b);
-        tma_load_3d(bs + 16384, &tm_B, &bar_tma[buf], t0 + 64, 0, b);
+        const int grow = (hh / p.heads_per_group) * N;  // first row of this head's group
+        tma_load_3d(cs, &tm_C, &bar_tma[buf], t0, grow, b);
+        tma_load_3d(cs + 16384, &tm_C, &bar_tma[buf], t0 + 64, grow, b);
+        tma_load_3d(bs, &tm_B, &bar_tma[buf], t0, grow, b);
+        tma_load_3d(bs + 16384, &tm_B, &bar_tma[buf], t0 + 64, grow, b);
         tma_load_3d(xs, &tm_X, &bar_tma[buf], t0, hh * P, b);
         tma_load_3d(xs + 8192, &tm_X, &bar_tma[buf], t0 + 64, hh * P, b);
     };

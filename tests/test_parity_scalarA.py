@@ -102,3 +102,13 @@ def test_full_size_config4_sampled():
     check(np.concatenate(ys, 1), np.concatenate(hl, 1), np.concatenate(yr, 1),
           np.concatenate(hr, 1), "config 4")
     assert np.isfinite(y).all()
+
+
+@pytest.mark.parametrize("G", [2, 4])
+def test_grouped_BC(G):
+    """Several B/C groups (Mamba-2 with ngroups > 1): head h reads group
+    h / (H / G)."""
+    inp = synthetic.make_scalarA(2, 4, 64, 128, 384, ngroups=G, seed=44 + G)
+    y, hs = run_gpu(inp)
+    y_ref, hs_ref = run_oracle(inp)
+    check(y, hs, y_ref, hs_ref, f"G={G}")
