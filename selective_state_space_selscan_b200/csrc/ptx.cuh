@@ -89,18 +89,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map,
         : "memory");
 }
 
-__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map,
-                                            uint64_t *bar, int c0, int c1,
-                                            int c2, int c3)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5}], [%6];"
-        :: "r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)),
-           "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_addr(bar))
-        : "memory");
-}
-
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map,
                                              const void *src, int c0, int c1, int c2)
 {
