@@ -45,11 +45,11 @@ NCU_TRAFFIC = {
     # config 3 (two-pass form, both kernels of one call) captured at
     # L = 32768, scaled by tokens to L = 131072
     3: ("scan_diag_bf16_kernel two-pass v1", 2679.6e6),
-    4: ("ssd_scalarA_kernel v3", 108.4e6),
+    4: ("ssd_scalarA_kernel v4", None),
 }
 KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v4", 1: "scan_diag_bf16_kernel pairs v4",
               3: "scan_diag_bf16_kernel two-pass v1", 0: "scan_diag_kernel fp32 v2",
-              4: "ssd_scalarA_kernel v3"}
+              4: "ssd_scalarA_kernel v4"}
 HBM_FALLBACK_GBS = 6650.0
 
 
@@ -744,6 +744,21 @@ def bwd_bytes(cfg: dict) -> int:
     return total
 
 
+# DRAM bytes per backward call (ncu, profiles/selscan_bwd_config2.md): captured
+# at L = 1024 on the B4 D5120 layer, scaled by tokens to L = 4096
+BWD_NCU_TRAFFIC = {2: ("selscan_bwd_kernel v2", 4 * 654.9e6)}
+BWD_KERNEL_TAG = "selscan_bwd_kernel v2"
+
+
+def bwd_traffic(args, cfg):
+    if args.traffic is not None:
+        return args.traffic
+    ent = BWD_NCU_TRAFFIC.get(args.config)
+    if ent and ent[0] == BWD_KERNEL_TAG and cfg == BASE_CONFIGS[args.config]:
+        return ent[1]
+    return None
+
+
 def run_bwd(args, rank: int, world: int, local: int):
     """Backward arm (``--op bwd``): selscan_bwd on the config's diagonal
     workload with a seeded upstream gradient dy."""
@@ -858,7 +873,7 @@ def run_bwd(args, rank: int, world: int, local: int):
                    "parallelism": f"dp{world} (independent shards, no collective)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": args.traffic, "peak_source": f"{peaks_src} HBM copy bandwidth",
+                     "traffic": bwd_traffic(args, cfg), "peak_source": f"{peaks_src} HBM copy bandwidth",
                      "bytes_per_launch": nbytes, "avg_launch_ms": avg_launch_ms,
                      "kernels_per_call": n_launch / args.steps},
         "e2e": {"value": aggregate_rate(world, elems, e2e_ms) / 1e9, "unit": "Gelem/s",

@@ -311,3 +311,26 @@ def test_round_bf16_matches_torch():
     ours = synthetic.round_bf16(a)
     ref = torch.from_numpy(a).to(torch.bfloat16).to(torch.float32).numpy()
     assert np.array_equal(ours, ref)
+
+
+def test_scalarA_groups_split_into_independent_problems():
+    """Scalar-A with G groups of B/C: heads of group g see only B[:, g],
+    C[:, g], so the result equals G single-group problems over the head
+    slices (structure of Mamba-2's grouped B/C; a wrong group index fails)."""
+    rng = np.random.default_rng(17)
+    batch, H, P, N, L, G = 2, 4, 3, 5, 9, 2
+    x = rng.standard_normal((batch, H * P, L))
+    dt = rng.uniform(0.01, 0.2, (batch, H, L))
+    A = -rng.uniform(0.5, 3.0, H)
+    B = rng.standard_normal((batch, G, N, L))
+    C = rng.standard_normal((batch, G, N, L))
+    D = rng.standard_normal(H)
+    y, hs = oracle.selscan_scalarA(x, dt, A, B, C, P, D=D)
+    per = H // G
+    for g in range(G):
+        hsl = slice(g * per, (g + 1) * per)
+        csl = slice(g * per * P, (g + 1) * per * P)
+        yg, hg = oracle.selscan_scalarA(x[:, csl], dt[:, hsl], A[hsl], B[:, g:g + 1],
+                                        C[:, g:g + 1], P, D=D[hsl])
+        np.testing.assert_allclose(y[:, csl], yg, rtol=0, atol=0)
+        np.testing.assert_allclose(hs[:, hsl], hg, rtol=0, atol=0)
