@@ -535,7 +535,7 @@ def run_gpu(args, rank: int, world: int, local: int):
         "gpu_launches": n_launch,
         "clocks": clock_info,
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:  # the oracle baseline: rank 0 at N = 1
         line["cpu_baseline"] = oracle_sample(args.config, inp, seconds=args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
@@ -724,7 +724,7 @@ def run_step(args, rank: int, world: int, local: int):
         "gpu_launches": n_launch,
         "clocks": clock_info,
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:  # the oracle baseline: rank 0 at N = 1
         line["cpu_baseline"] = oracle_step_sample(cfg, inp, state.cpu().numpy(),
                                                   seconds=args.cpu_seconds)
     print(json.dumps(line), flush=True)
@@ -881,7 +881,7 @@ def run_bwd(args, rank: int, world: int, local: int):
         "gpu_launches": n_launch,
         "clocks": clock_info,
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:  # the oracle baseline: rank 0 at N = 1
         line["cpu_baseline"] = oracle_bwd_sample(cfg, inp, dy_host, seconds=args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
