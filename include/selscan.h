@@ -1,6 +1,8 @@
 /*
- * selscan.h -- C ABI of libselscan, the selective-scan (S6) forward pass for
- * NVIDIA B200 (sm_100a).
+ * selscan.h -- C ABI of libselscan, the selective scan (S6) on NVIDIA B200
+ * (sm_100a): the forward pass over a sequence (diagonal A, and scalar A in
+ * the chunked matrix form on the tensor cores), the one-token decode step of
+ * both, and the backward pass of the diagonal form.
  *
  * What is computed (diagonal A).  For every batch b, channel d and token t,
  * following "03 -- Modelos de espacio de estados: RWKV, S4, Mamba y el
@@ -22,14 +24,16 @@
  *   - All pointers are DEVICE pointers of the current CUDA device, owned by
  *     the caller.  The library keeps no pointer after a call returns.
  *   - Calls are asynchronous on `stream`.  Scratch memory the kernels need
- *     (look-back carries, flags) is taken with cudaMallocAsync on `stream`
- *     and released with cudaFreeAsync on the same stream.
+ *     (segment carries and flags, segment aggregates, backward checkpoints)
+ *     is taken with cudaMallocAsync on `stream` and released with
+ *     cudaFreeAsync on the same stream (selscan_fwd_noalloc excepted).
  *   - Tensors are described by selscan_tensor: element type, rank, shape and
  *     strides in ELEMENTS.  The last (time) dimension must have stride 1.
  *     Other strides may be anything that keeps rows 16-byte aligned (they
  *     are multiples of 16 bytes) and the base pointer 16-byte aligned; this
  *     is what the bulk tensor copies (TMA) require.  For a contiguous bf16
- *     tensor that means L % 8 == 0; for fp32, L % 4 == 0.
+ *     tensor that means L % 8 == 0; for fp32, L % 4 == 0.  (The decode-step
+ *     entry points take per-token tensors with any strides; see there.)
  *   - Validation errors are returned synchronously and nothing is launched.
  *     A failed launch returns SELSCAN_ERR_CUDA.  A device-side wait that ran
  *     out of its iteration limit is recorded on the device and reported by
