@@ -25,10 +25,11 @@
 // that hold a warp's diagonal it is taken per element.
 //
 // Per chunk c, in order (all threads unless noted):
-//   1. x * w for the state product (needs chunk c's x);
+//   1. x * w for the state product (needs chunk c's x); one thread issues
+//      the state product, which runs during step 2;
 //   2. M from G (tensor memory) and the decays (needs G(c));
-//   3. one thread issues Yd(c), the state product and G(c + 1);
-//   4. the first warpgroup prepares the step sizes of chunk c + 1;
+//   3. one thread issues Yd(c) and G(c + 1);
+//   4. the second warpgroup prepares the step sizes of chunk c + 1;
 //   5. y = Yd + 2^cs_t Yo + D x (+ gate), staged in shared memory and written
 //      back by one bulk tensor store;
 //   6. state: h -> bf16 copy for Yo(c + 1), last_state, h *= 2^cs_Q(c + 1);
@@ -191,12 +192,13 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
     if (warp == 0)
         tmem_alloc(&s_tbase, kSsdTmemCols);
 
-    // Step sizes of chunk cc (first warpgroup, token r): delta, its inclusive
+    // Step sizes of chunk cc (second warpgroup, token r, so that the thread
+    // issuing the tensor-core work in warp 0 never delays it): delta, its inclusive
     // sum in log2-decay units cs, and per token
     //   s_n2[s] = log2(delta_s) - cs_s        (pieces on a warp's diagonal)
     //   s_sg[s] = 2^(cs_e - cs_s) delta_s     (e = last token of s's piece)
     auto cumsum = [&](int cc, float dtv) {
-        if (wg != 0)
+        if (wg != 1)
             return;
         float dl = dtv + bias;
         if (p.softplus)
@@ -230,8 +232,8 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
         for (int i = 0; i < PW; ++i)
             h_init[i] = h0row ? h0row[int64_t(wg * PW + i) * N] : 0.f;
     }
-    cumsum(0, (wg == 0 && r < p.L) ? dt_row[r] : 0.f);
-    float dt_next = (wg == 0 && Q + r < p.L) ? dt_row[Q + r] : 0.f;
+    cumsum(0, (wg == 1 && r < p.L) ? dt_row[r] : 0.f);
+    float dt_next = (wg == 1 && Q + r < p.L) ? dt_row[Q + r] : 0.f;
     __syncthreads();  // s_cs of chunk 0, TMEM address
     tmem_fence_after_sync();
     const uint32_t tb = s_tbase;
@@ -331,6 +333,18 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                 *reinterpret_cast<uint4 *>(xw + off) = o;
             }
         }
+        // the state product h += B (x w)^T runs while the mask is built
+        fence_proxy_async_smem();
+        tmem_fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tmem_fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < Q / 16; ++kk)
+                umma_bf16(tb + kColH, umma_desc_kmajor(aB, N, kk), umma_desc_kmajor(aXw, P, kk),
+                          idYd, 1u);
+            umma_commit(&bar_st);
+        }
         // ---- 2. M: row t = r, pieces q = wg + NWG * j of 16 columns
         const float cs_t = s_cs[r];
         const float ey = ex2_approx(cs_t);  // Yo row scale, used in step 5
@@ -384,7 +398,7 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
         fence_proxy_async_smem();
         tmem_fence_before_sync();
         __syncthreads();
-        // ---- 3. Yd = M x^T; h += B (x w)^T; then the next chunk's C^T B
+        // ---- 3. Yd = M x^T; then the next chunk's C^T B
         if (tid == 0) {
             tmem_fence_after_sync();
 #pragma unroll
@@ -392,11 +406,6 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                 umma_bf16(tb + kColYd, umma_desc_kmajor(aM, 128, kk), umma_desc_kmajor(aX, P, kk),
                           idYd, kk > 0);
             umma_commit(&bar_yd);
-#pragma unroll
-            for (int kk = 0; kk < Q / 16; ++kk)
-                umma_bf16(tb + kColH, umma_desc_kmajor(aB, N, kk), umma_desc_kmajor(aXw, P, kk),
-                          idYd, 1u);
-            umma_commit(&bar_st);
             if (c + 1 < p.nchunks) {
                 ok = mbar_wait(&bar_tma[buf ^ 1], uint32_t(((c + 1) >> 1) & 1), p.timeout_ns) &&
                      ok;
@@ -408,7 +417,7 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
         //         once every thread has passed the barrier above)
         if (c + 1 < p.nchunks) {
             cumsum(c + 1, dt_next);
-            if (wg == 0)
+            if (wg == 1)
                 dt_next = (t0 + 2 * Q + r < p.L) ? dt_row[t0 + 2 * Q + r] : 0.f;
         }
         // ---- 5. y for token t = r, columns p of this warpgroup's slice
