@@ -45,11 +45,11 @@ NCU_TRAFFIC = {
     # config 3 (two-pass form, both kernels of one call) captured at
     # L = 32768, scaled by tokens to L = 131072
     3: ("scan_diag_bf16_kernel two-pass v1", 2679.6e6),
-    4: ("ssd_scalarA_kernel v4", 107.3e6),
+    4: ("ssd_scalarA_kernel v5", None),
 }
 KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v4", 1: "scan_diag_bf16_kernel pairs v4",
               3: "scan_diag_bf16_kernel two-pass v1", 0: "scan_diag_kernel fp32 v2",
-              4: "ssd_scalarA_kernel v4"}
+              4: "ssd_scalarA_kernel v5"}
 HBM_FALLBACK_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # the HGX/DGX nominal figure, reported beside the measured peak
 
