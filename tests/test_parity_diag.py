@@ -262,3 +262,20 @@ print("CLEAN", bool(torch.isfinite(y.float()).all()))
     assert r.returncode == 0, r.stderr[-2000:]
     assert "STATUS SELSCAN_ERR_TIMEOUT" in r.stdout, r.stdout
     assert "CLEAN True" in r.stdout, r.stdout
+
+
+@pytest.mark.parametrize("gate", [False, True])
+def test_two_pass_without_softplus(gate):
+    """The two-pass form's instances without the softplus (raw positive step
+    sizes, no bias), with and without the gate."""
+    import selective_state_space_selscan_b200 as ss
+    inp = synthetic.make_diag(1, 256, 16, 2048, dtype="bf16", seed=33, gate=gate, bias=False)
+    inp["delta"] = synthetic.round_bf16(np.abs(inp["delta"]) * 0.05)
+    inp["softplus"] = False
+    ss.debug_diag_mode(1)
+    try:
+        y, hs = run_gpu(inp)
+    finally:
+        ss.debug_diag_mode(-1)
+    y_ref, hs_ref = run_oracle(inp)
+    assert_parity(inp, y, hs, y_ref, hs_ref, f"two-pass, no softplus, gate={gate}")
