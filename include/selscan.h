@@ -325,7 +325,9 @@ SELSCAN_API int selscan_version(void);
  * Number of kernels this library has launched in the calling process so far
  * (all entry points, all devices).  A selscan_fwd call launches one kernel,
  * or two when it uses the two-pass form (few channel tiles, long
- * sequences); the other entry points launch one.  Benchmarks read it around
+ * sequences); selscan_bwd launches two (three with time segments: the
+ * segment aggregates, the gradient walk, the sum of the dB / dC partial
+ * copies); the other entry points launch one.  Benchmarks read it around
  * a timed region to report how many of the library's kernels ran in it.
  */
 SELSCAN_API unsigned long long selscan_launch_count(void);

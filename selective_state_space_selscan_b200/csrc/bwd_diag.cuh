@@ -32,7 +32,8 @@
 // dB and dC sum over the channels of a batch row: each token's 32 per-lane
 // values are reduced across the warp by a butterfly (31 shuffles leave lane i
 // with the sum of value i); a lane keeps its sums for the chunk's 8 tokens
-// and adds them to global memory with two 16-byte atomics.  dA, dD and the
+// and adds them with two 16-byte atomics into one of kBwdCopies partial
+// copies, which bwd_reduce_bc sums at the end.  dA, dD and the
 // bias gradient sum over batch rows and tokens: registers, then atomics.
 #pragma once
 
@@ -48,6 +49,11 @@ namespace selscan {
 
 constexpr int kBwdN = 16;  // states per channel
 constexpr int kBwdT = 8;   // tokens per checkpoint chunk
+// dB / dC are accumulated into this many partial copies (tile i adds into
+// copy i % kBwdCopies) and summed afterwards: all tiles of a batch row walk
+// the same tokens at nearly the same time, so one copy would take every
+// tile's atomic add of a token at once.
+constexpr int kBwdCopies = 8;
 
 struct BwdParams {
     int batch, dim, L, nchunks;      // nchunks = ceil(L / kBwdT)
@@ -64,7 +70,8 @@ struct BwdParams {
     void *du, *ddelta, *dz;          // (batch, dim, L) like u; dz null without gate
     int64_t du_bs, du_ds, dd_bs, dd_ds, dz_bs, dz_ds;
     float *dA;                       // (dim, 16), accumulated
-    float *dB, *dC;                  // (batch, 16, L) contiguous, accumulated
+    float *dB, *dC;                  // (batch, 16, L) contiguous, written by bwd_reduce_bc
+    float *pB, *pC;                  // kBwdCopies partial sums of dB, dC, accumulated
     float *dD, *dbias;               // (dim) or null, accumulated
     float *dh0;                      // (batch, dim, 16) or null, written
     float *ckpt;                     // [batch][dim][nchunks][16] scratch
@@ -665,8 +672,9 @@ selscan_bwd_kernel(const BwdParams p)
                 bwd_st8(p.dz, ch.row_dz + t0, valid, o_dz, tag);
         }
         {
-            float *dst = lane < N ? p.dB + (int64_t(b) * N + lane) * p.L + t0
-                                  : p.dC + (int64_t(b) * N + (lane - N)) * p.L + t0;
+            const int64_t copy = int64_t(tile % kBwdCopies) * p.batch * N * p.L;
+            float *dst = lane < N ? p.pB + copy + (int64_t(b) * N + lane) * p.L + t0
+                                  : p.pC + copy + (int64_t(b) * N + (lane - N)) * p.L + t0;
             if (valid >= 8 && (p.L & 3) == 0) {  // rows of dB / dC 16-byte aligned
                 atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(red[0], red[1], red[2], red[3]));
                 atomicAdd(reinterpret_cast<float4 *>(dst) + 1,
@@ -699,6 +707,23 @@ selscan_bwd_kernel(const BwdParams p)
             atomicAdd(p.dD + d, gD);
         if (p.dbias)
             atomicAdd(p.dbias + d, gbias);
+    }
+}
+
+// dB, dC = sum of the kBwdCopies partial copies (n elements each).
+__global__ void __launch_bounds__(256)
+bwd_reduce_bc(const float *pB, const float *pC, float *dB, float *dC, int64_t n)
+{
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        float sb = 0.f, sc = 0.f;
+#pragma unroll
+        for (int k = 0; k < kBwdCopies; ++k) {
+            sb += pB[int64_t(k) * n + i];
+            sc += pC[int64_t(k) * n + i];
+        }
+        dB[i] = sb;
+        dC[i] = sc;
     }
 }
 

@@ -1249,19 +1249,23 @@ extern "C" selscan_status selscan_bwd(
         return SELSCAN_ERR_UNSUPPORTED;
     if (batch > 65535 || dim > (int64_t(1) << 30) || L > (int64_t(1) << 30))
         return SELSCAN_ERR_UNSUPPORTED;
-    if (batch == 0 || dim == 0)
+    auto zero = [&](selscan_tensor *t) {
+        return (!t || !t->data || numel(t) == 0)
+                   ? cudaSuccess
+                   : cudaMemsetAsync(t->data, 0, size_t(numel(t)) * 4, stream);
+    };
+    if (batch == 0)
         return SELSCAN_OK;
+    if (dim == 0)  // dB and dC sum over no channel
+        return zero(dB) == cudaSuccess && zero(dC) == cudaSuccess ? SELSCAN_OK
+                                                                  : SELSCAN_ERR_CUDA;
 
     int dev = 0;
     DeviceInfo *di = nullptr;
     if ((st = device_setup(&dev, &di)) != SELSCAN_OK)
         return st;
-    auto zero = [&](selscan_tensor *t) {
-        return (!t || !t->data) ? cudaSuccess
-                                : cudaMemsetAsync(t->data, 0, size_t(numel(t)) * 4, stream);
-    };
-    if (zero(dA) != cudaSuccess || zero(dB) != cudaSuccess || zero(dC) != cudaSuccess ||
-        zero(dD) != cudaSuccess || zero(ddelta_bias) != cudaSuccess)
+    // dB and dC are written whole by the final reduction (L > 0)
+    if (zero(dA) != cudaSuccess || zero(dD) != cudaSuccess || zero(ddelta_bias) != cudaSuccess)
         return SELSCAN_ERR_CUDA;
     if (L == 0) {
         // nothing to walk back through: the gradient of h0 is that of the final state
@@ -1353,15 +1357,24 @@ extern "C" selscan_status selscan_bwd(
     // segment aggregates E, G [units][32][16] and S [units][32] (fp32)
     const size_t ck_bytes = size_t(batch) * dim * prm.nchunks * kBwdN * 4;
     const size_t agg_bytes = prm.segs > 1 ? size_t(units) * 32 * kBwdN * 4 : 0;
-    const size_t s_bytes = prm.segs > 1 ? size_t(units) * 32 * 4 : 0;
+    const size_t s_bytes = prm.segs > 1 ? ((size_t(units) * 32 * 4 + 255) / 256) * 256 : 0;
+    const int64_t bc_n = batch * kBwdN * L;           // elements of dB (and of dC)
+    const size_t part_bytes = size_t(kBwdCopies) * bc_n * 4;
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, ck_bytes + 2 * agg_bytes + s_bytes, stream) != cudaSuccess)
+    if (cudaMallocAsync(&ws, ck_bytes + 2 * agg_bytes + s_bytes + 2 * part_bytes, stream) !=
+        cudaSuccess)
         return SELSCAN_ERR_CUDA;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     prm.ckpt = reinterpret_cast<float *>(wsb);
     prm.aggE = reinterpret_cast<float *>(wsb + ck_bytes);
     prm.aggG = reinterpret_cast<float *>(wsb + ck_bytes + agg_bytes);
     prm.aggS = reinterpret_cast<float *>(wsb + ck_bytes + 2 * agg_bytes);
+    prm.pB = reinterpret_cast<float *>(wsb + ck_bytes + 2 * agg_bytes + s_bytes);
+    prm.pC = prm.pB + size_t(kBwdCopies) * bc_n;
+    if (cudaMemsetAsync(prm.pB, 0, 2 * part_bytes, stream) != cudaSuccess) {
+        cudaFreeAsync(ws, stream);
+        return SELSCAN_ERR_CUDA;
+    }
     cudaError_t le = cudaSuccess;
     if (prm.segs > 1) {
         if (dt == SELSCAN_BF16)
@@ -1375,6 +1388,12 @@ extern "C" selscan_status selscan_bwd(
             selscan_bwd_kernel<__nv_bfloat16><<<unsigned(units), 32, 0, stream>>>(prm);
         else
             selscan_bwd_kernel<float><<<unsigned(units), 32, 0, stream>>>(prm);
+        le = counted_launch();
+    }
+    if (le == cudaSuccess) {
+        const int64_t blocks = std::min<int64_t>((bc_n + 255) / 256, 8ll * di->sm_count);
+        bwd_reduce_bc<<<unsigned(blocks), 256, 0, stream>>>(prm.pB, prm.pC, prm.dB, prm.dC,
+                                                            bc_n);
         le = counted_launch();
     }
     cudaFreeAsync(ws, stream);
