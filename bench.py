@@ -45,7 +45,7 @@ NCU_TRAFFIC = {
     # config 3 (two-pass form, both kernels of one call) captured at
     # L = 32768, scaled by tokens to L = 131072
     3: ("scan_diag_bf16_kernel two-pass v1", 2679.6e6),
-    4: ("ssd_scalarA_kernel v5", None),
+    4: ("ssd_scalarA_kernel v5", 107.9e6),
 }
 KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v4", 1: "scan_diag_bf16_kernel pairs v4",
               3: "scan_diag_bf16_kernel two-pass v1", 0: "scan_diag_kernel fp32 v2",
