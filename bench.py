@@ -17,6 +17,8 @@ scaling is weak; the step time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import contextlib
+import gc
 import json
 import os
 import statistics
@@ -99,6 +101,24 @@ def ssd_flops(cfg: dict, Q: int = 128) -> float:
 
 
 # ------------------------------------------------------------ ranks
+@contextlib.contextmanager
+def gc_paused(collect: bool = True):
+    """Keep Python's garbage collector off for a timed region (after a full
+    collection unless the caller just made one).  With torch loaded a full
+    collection pauses the host for tens to hundreds of milliseconds; inside
+    a timed loop of asynchronous calls that pause drains the GPU's queue
+    and is counted as device time."""
+    if collect:
+        gc.collect()
+    was_on = gc.isenabled()
+    gc.disable()
+    try:
+        yield
+    finally:
+        if was_on:
+            gc.enable()
+
+
 def max_over_ranks(values, device="cuda"):
     """Element-wise max of a list of floats over all ranks of the default
     process group (identity without one).  Every rank must call it with the
@@ -433,6 +453,7 @@ def run_gpu(args, rank: int, world: int, local: int):
     torch.cuda.synchronize()
 
     # timed region: K steps, per-launch events on the launching stream
+    gc.collect()  # before the clock samples start (see gc_paused)
     clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
     if clocks:
         clocks.start()
@@ -444,12 +465,13 @@ def run_gpu(args, rank: int, world: int, local: int):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     n_launch0 = ss.launch_count()
-    start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        call()
-        ev[i][1].record(stream)
-    end.record(stream)
+    with gc_paused(collect=False):
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        end.record(stream)
     torch.cuda.synchronize()
     barrier()
     t_wall1 = time.time()
@@ -485,10 +507,11 @@ def run_gpu(args, rank: int, world: int, local: int):
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    with gc_paused():
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
     barrier()
@@ -638,6 +661,7 @@ def run_step(args, rank: int, world: int, local: int):
     ss.check()
     barrier()
     torch.cuda.synchronize()
+    gc.collect()  # before the clock samples start (see gc_paused)
     clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
     if clocks:
         clocks.start()
@@ -649,12 +673,13 @@ def run_step(args, rank: int, world: int, local: int):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     n_launch0 = ss.launch_count()
-    start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        call()
-        ev[i][1].record(stream)
-    end.record(stream)
+    with gc_paused(collect=False):
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        end.record(stream)
     torch.cuda.synchronize()
     barrier()
     t_wall1 = time.time()
@@ -688,10 +713,11 @@ def run_step(args, rank: int, world: int, local: int):
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    with gc_paused():
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
     barrier()
@@ -797,6 +823,7 @@ def run_bwd(args, rank: int, world: int, local: int):
     ss.check()
     barrier()
     torch.cuda.synchronize()
+    gc.collect()  # before the clock samples start (see gc_paused)
     clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
     if clocks:
         clocks.start()
@@ -808,12 +835,13 @@ def run_bwd(args, rank: int, world: int, local: int):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     n_launch0 = ss.launch_count()
-    start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        grads = call()
-        ev[i][1].record(stream)
-    end.record(stream)
+    with gc_paused(collect=False):
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            grads = call()
+            ev[i][1].record(stream)
+        end.record(stream)
     torch.cuda.synchronize()
     barrier()
     t_wall1 = time.time()
@@ -851,10 +879,11 @@ def run_bwd(args, rank: int, world: int, local: int):
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    with gc_paused():
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
     barrier()

@@ -25,8 +25,10 @@
  *     the caller.  The library keeps no pointer after a call returns.
  *   - Calls are asynchronous on `stream`.  Scratch memory the kernels need
  *     (segment carries and flags, segment aggregates, backward checkpoints)
- *     is taken with cudaMallocAsync on `stream` and released with
- *     cudaFreeAsync on the same stream (selscan_fwd_noalloc excepted).
+ *     is taken on `stream` from a stream-ordered memory pool that the
+ *     library creates per device, and freed with cudaFreeAsync on the same
+ *     stream (selscan_fwd_noalloc excepted).  The pool keeps freed memory
+ *     for the next call; selscan_release_scratch() hands it back.
  *   - Tensors are described by selscan_tensor: element type, rank, shape and
  *     strides in ELEMENTS.  The last (time) dimension must have stride 1.
  *     Other strides may be anything that keeps rows 16-byte aligned (they
@@ -293,10 +295,11 @@ SELSCAN_API selscan_status selscan_step_scalarA(selscan_tensor *state, const sel
  *   dD, ddelta_bias (D)       F32; may be NULL (not computed)
  *   dh0        (batch, D, N)  F32; may be NULL (not computed)
  * The expanded states are recomputed, never stored: a forward pass keeps h
- * every 16 tokens in stream-ordered scratch (batch * D * ceil(L/16) * 64
+ * every 8 tokens in stream-ordered scratch (batch * D * ceil(L/8) * 64
  * bytes), then the chunks are walked backwards.  Sums over channels and
- * batch rows use fp32 atomics, so the last bits of dA, dB, dC, dD and
- * ddelta_bias depend on the order of the additions.
+ * batch rows use fp32 atomics (dB and dC into 8 partial copies that a
+ * last kernel adds), so the last bits of dA, dB, dC, dD and ddelta_bias
+ * depend on the order of the additions.
  */
 SELSCAN_API selscan_status selscan_bwd(
     const selscan_tensor *u, const selscan_tensor *delta, const selscan_tensor *delta_bias,
@@ -331,6 +334,16 @@ SELSCAN_API int selscan_version(void);
  * a timed region to report how many of the library's kernels ran in it.
  */
 SELSCAN_API unsigned long long selscan_launch_count(void);
+
+/*
+ * selscan_release_scratch -- return to the driver the scratch memory that
+ * the library's pools hold but no call is using (every device the process
+ * has called on).  Memory whose cudaFreeAsync has not yet run on its stream
+ * is kept; synchronise the streams first to release everything.  Calls
+ * after it allocate again as needed.  Returns SELSCAN_ERR_CUDA if a trim
+ * failed, else SELSCAN_OK.
+ */
+SELSCAN_API selscan_status selscan_release_scratch(void);
 
 #ifdef __cplusplus
 }

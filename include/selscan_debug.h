@@ -34,6 +34,16 @@ SELSCAN_API void selscan_debug_withhold_carry(int unit);
  */
 SELSCAN_API void selscan_debug_diag_mode(int mode);
 
+/*
+ * Number of time segments per channel tile in subsequent selscan_bwd calls
+ * (0, the default, = the library's choice: as many as fill one wave of
+ * resident warps, with at least 32 checkpoint chunks each).  Capped at the
+ * number of checkpoint chunks.  Every segment count computes the same
+ * gradients; the hook lets tests cover the segment folds on small inputs
+ * and lets the choice be timed.
+ */
+SELSCAN_API void selscan_debug_bwd_segments(int segs);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,7 +29,8 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 # entry points declared in include/selscan.h
 EXPORTS = ("selscan_fwd", "selscan_fwd_h0", "selscan_fwd_scalarA", "selscan_fwd_scalarA_h0",
            "selscan_fwd_noalloc", "selscan_step", "selscan_step_scalarA", "selscan_check",
-           "selscan_strerror", "selscan_version", "selscan_launch_count", "selscan_bwd")
+           "selscan_strerror", "selscan_version", "selscan_launch_count", "selscan_bwd",
+           "selscan_release_scratch")
 
 
 class SelscanError(RuntimeError):
@@ -89,10 +90,14 @@ def lib() -> ctypes.CDLL:
         L.selscan_step_scalarA.restype = ctypes.c_int
         L.selscan_bwd.argtypes = [P, P, P, ctypes.c_int] + [P] * 17 + [ctypes.c_void_p]
         L.selscan_bwd.restype = ctypes.c_int
+        L.selscan_release_scratch.argtypes = []
+        L.selscan_release_scratch.restype = ctypes.c_int
         L.selscan_debug_withhold_carry.argtypes = [ctypes.c_int]
         L.selscan_debug_withhold_carry.restype = None
         L.selscan_debug_diag_mode.argtypes = [ctypes.c_int]
         L.selscan_debug_diag_mode.restype = None
+        L.selscan_debug_bwd_segments.argtypes = [ctypes.c_int]
+        L.selscan_debug_bwd_segments.restype = None
         _lib = L
     return _lib
 
@@ -111,6 +116,14 @@ def version() -> int:
 def launch_count() -> int:
     """Kernels launched by the library in this process so far."""
     return int(lib().selscan_launch_count())
+
+
+def release_scratch() -> None:
+    """Hand back to the driver the scratch memory the library's pools keep
+    between calls (synchronise the streams first to release all of it)."""
+    st = lib().selscan_release_scratch()
+    if st != 0:
+        raise SelscanError(st, "selscan_release_scratch")
 
 
 def describe(t, dtype_code=None) -> SelscanTensor | None:
@@ -306,6 +319,11 @@ def check(stream=None) -> None:
 def debug_diag_mode(mode: int) -> None:
     """Test hook: 0 = chained carries, 1 = two-pass form, -1 = automatic."""
     lib().selscan_debug_diag_mode(int(mode))
+
+
+def debug_bwd_segments(segs: int) -> None:
+    """Test hook: time segments per channel tile in selscan_bwd (0: automatic)."""
+    lib().selscan_debug_bwd_segments(int(segs))
 
 
 def debug_withhold_carry(unit: int) -> None:

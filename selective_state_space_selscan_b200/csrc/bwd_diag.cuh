@@ -29,12 +29,14 @@
 //     checkpoint into shared memory and the reverse step runs over them.
 // The expanded states (batch, D, L, N) are never stored.
 //
-// dB and dC sum over the channels of a batch row: each token's 32 per-lane
-// values are reduced across the warp by a butterfly (31 shuffles leave lane i
-// with the sum of value i); a lane keeps its sums for the chunk's 8 tokens
-// and adds them with two 16-byte atomics into one of kBwdCopies partial
-// copies, which bwd_reduce_bc sums at the end.  dA, dD and the
-// bias gradient sum over batch rows and tokens: registers, then atomics.
+// dB and dC sum over the channels of a batch row.  Per chunk they are sums
+// over the warp's lanes of rows of shared memory: dC_t[n] of dout_t times the
+// recomputed states (before the reverse walk), dB_t[n] of the terms
+// g delta u that the walk writes over the states it has used.  Lane l sums
+// state n = l % 16 for four of the chunk's tokens and adds both results with
+// one 16-byte atomic each into one of kBwdCopies partial copies, which
+// bwd_reduce_bc sums at the end.  dA, dD and the bias gradient sum over batch
+// rows and tokens: registers, then atomics.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -142,12 +144,41 @@ __device__ __forceinline__ float bwd_step(float raw, int softplus)
     return FAST ? softplus_fast(raw) : softplus_exact(raw);
 }
 
-// Per-warp shared memory: B and C of the chunk (fp32, [token][n]) and the
-// recomputed states of the chunk ([token][n][lane]).
+// Per-warp shared memory: B and C of the chunk (fp32, [token][n]), the
+// recomputed states of the chunk ([token][n][lane]; the reverse walk puts
+// each lane's dB terms in their place once it has used them) and the output
+// gradient through the gate ([token][lane]).
 struct BwdSmem {
     float bc[kBwdT][2][kBwdN];
     float h[kBwdT][kBwdN][32];
+    float dout[kBwdT][32];
 };
+
+// Sum over the warp's 32 lanes of row (i, n) of sm.h, weighted by sm.dout[i]
+// when WEIGHTED.  Each lane starts at its own 16-byte column, so the eight
+// lanes of a quarter warp (eight rows of one token) read distinct banks.
+template <bool WEIGHTED>
+__device__ __forceinline__ float bwd_row_sum(const BwdSmem &sm, int i, int n, int lane)
+{
+    const float4 *hr = reinterpret_cast<const float4 *>(sm.h[i][n]);
+    const float4 *wr = reinterpret_cast<const float4 *>(sm.dout[i]);
+    uint64_t s0 = pk2(0.f, 0.f), s1 = pk2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int c = (k + lane) & 7;
+        const float4 h = hr[c];
+        if (WEIGHTED) {
+            const float4 w = wr[c];
+            s0 = fma2(pk2(w.x, w.y), pk2(h.x, h.y), s0);
+            s1 = fma2(pk2(w.z, w.w), pk2(h.z, h.w), s1);
+        } else {
+            s0 = add2(pk2(h.x, h.y), s0);
+            s1 = add2(pk2(h.z, h.w), s1);
+        }
+    }
+    const uint64_t s = add2(s0, s1);
+    return lo2(s) + hi2(s);
+}
 
 // One chunk's raw inputs, copied asynchronously: per lane its channel's 8
 // tokens of u, delta, dy, z (KV 16-byte vectors each), one row of B (lanes
@@ -573,22 +604,52 @@ selscan_bwd_kernel(const BwdParams p)
             bwd_forward_chunk<T, true>(p, ch, sm, valid, uv, dv, hr, lane);
         }
         __syncwarp();
-        float o_du[8], o_dd[8], o_dz[8], red[8];
+        // output gradient through the gate and the factor of dz, per token
+        float dov[8], fzv[8];
 #pragma unroll
         for (int i = 0; i < TC; ++i) {
-            o_du[i] = o_dd[i] = o_dz[i] = red[i] = 0.f;
+            const float dyv = (live && i < valid) ? yv[i] : 0.f;
+            float dout = dyv, f = 0.f;
+            if (p.z) {
+                const float zz = zv[i];
+                const float sg = 1.f / (1.f + __expf(-zz));
+                f = dyv * (sg * (1.f + zz * (1.f - sg)));
+                dout = dyv * zz * sg;
+            }
+            dov[i] = dout;
+            fzv[i] = f;
+            sm.dout[i][lane] = dout;
         }
+        __syncwarp();
+        // dC of the chunk: lane -> state rn, tokens ri .. ri + 3
+        const int rn = lane & (N - 1), ri = 4 * (lane >> 4);
+        float dCv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            dCv[r] = bwd_row_sum<true>(sm, ri + r, rn, lane);
+        __syncwarp();  // all rows read before the walk overwrites them
+        float o_du[8], o_dd[8], o_dz[8];
+#pragma unroll
+        for (int i = 0; i < TC; ++i)
+            o_du[i] = o_dd[i] = o_dz[i] = 0.f;
+        uint64_t ht2[8];  // state after token i, carried down from token i + 1
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            ht2[j] = pk2(0.f, 0.f);
 #pragma unroll
         for (int i = TC - 1; i >= 0; --i) {
             if (i >= valid)
                 continue;
-            uint64_t ht2[8], hp2[8];
+            if (i == valid - 1) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                ht2[j] = pk2(sm.h[i][2 * j][lane], sm.h[i][2 * j + 1][lane]);
+                for (int j = 0; j < 8; ++j)
+                    ht2[j] = pk2(sm.h[i][2 * j][lane], sm.h[i][2 * j + 1][lane]);
+            }
+            uint64_t hp2[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
                 hp2[j] = i > 0 ? pk2(sm.h[i - 1][2 * j][lane], sm.h[i - 1][2 * j + 1][lane])
                                : hc2[j];
-            }
             const float raw = dv[i] + ch.bias;
             const float dt = bwd_step<FAST>(raw, p.softplus);
             const float x = uv[i];
@@ -607,38 +668,30 @@ selscan_bwd_kernel(const BwdParams p)
                     C2[2 * q + 1] = pk2(cc.z, cc.w);
                 }
             }
-            uint64_t Y2 = mul2(C2[0], ht2[0]);
-#pragma unroll
-            for (int j = 1; j < 8; ++j)
-                Y2 = fma2(C2[j], ht2[j], Y2);
-            const float out = fmaf(ch.dsk, x, lo2(Y2) + hi2(Y2));
-            const float dyv = live ? yv[i] : 0.f;
-            float dout = dyv;
             if (p.z) {
-                const float zz = zv[i];
-                const float sg = 1.f / (1.f + __expf(-zz));
-                o_dz[i] = dyv * out * (sg * (1.f + zz * (1.f - sg)));
-                dout = dyv * zz * sg;
+                uint64_t Y2 = mul2(C2[0], ht2[0]);
+#pragma unroll
+                for (int j = 1; j < 8; ++j)
+                    Y2 = fma2(C2[j], ht2[j], Y2);
+                o_dz[i] = fzv[i] * fmaf(ch.dsk, x, lo2(Y2) + hi2(Y2));
             }
+            const float dout = dov[i];
             gD = fmaf(dout, x, gD);
             const uint64_t DO = pk2(dout, dout), DT = pk2(dt, dt), X = pk2(x, x);
             uint64_t dx2 = pk2(0.f, 0.f), ddt2 = pk2(0.f, 0.f);
-            float v[32];  // dB (states 0..15), dC (states 0..15) of this channel
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 g2[j] = fma2(DO, C2[j], g2[j]);
-                const uint64_t vc = mul2(DO, ht2[j]);
                 const uint64_t gdt = mul2(g2[j], DT);
                 const uint64_t vb = mul2(gdt, X);
-                v[2 * j] = lo2(vb);
-                v[2 * j + 1] = hi2(vb);
-                v[N + 2 * j] = lo2(vc);
-                v[N + 2 * j + 1] = hi2(vc);
+                sm.h[i][2 * j][lane] = lo2(vb);  // this lane's dB terms of token i
+                sm.h[i][2 * j + 1][lane] = hi2(vb);
                 dx2 = fma2(gdt, B2[j], dx2);
                 const uint64_t ah = mul2(a2[j], hp2[j]);
                 ddt2 = fma2(g2[j], fma2(ch.An2[j], ah, mul2(B2[j], X)), ddt2);
                 gA2[j] = fma2(gdt, ah, gA2[j]);
                 g2[j] = mul2(g2[j], a2[j]);
+                ht2[j] = hp2[j];
             }
             const float dx = fmaf(dout, ch.dsk, lo2(dx2) + hi2(dx2));
             const float ddt = lo2(ddt2) + hi2(ddt2);
@@ -646,25 +699,12 @@ selscan_bwd_kernel(const BwdParams p)
             gbias += dDelta;
             o_du[i] = dx;
             o_dd[i] = dDelta;
-            if (!live) {
-#pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    v[k] = 0.f;  // lanes past the last channel add exact zeros
-            }
-            // sum the 32 values over the warp's channels: lane i gets value i
-#pragma unroll
-            for (int lv = 0; lv < 5; ++lv) {
-                const int half = 16 >> lv;
-                const bool up = (lane & half) != 0;
-#pragma unroll
-                for (int k = 0; k < half; ++k) {
-                    const float send = up ? v[k] : v[k + half];
-                    const float keep = up ? v[k + half] : v[k];
-                    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-                }
-            }
-            red[i] = v[0];
         }
+        __syncwarp();
+        float dBv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            dBv[r] = bwd_row_sum<false>(sm, ri + r, rn, lane);
         if (live) {
             bwd_st8(p.du, ch.row_du + t0, valid, o_du, tag);
             bwd_st8(p.ddelta, ch.row_dd + t0, valid, o_dd, tag);
@@ -673,17 +713,20 @@ selscan_bwd_kernel(const BwdParams p)
         }
         {
             const int64_t copy = int64_t(tile % kBwdCopies) * p.batch * N * p.L;
-            float *dst = lane < N ? p.pB + copy + (int64_t(b) * N + lane) * p.L + t0
-                                  : p.pC + copy + (int64_t(b) * N + (lane - N)) * p.L + t0;
-            if (valid >= 8 && (p.L & 3) == 0) {  // rows of dB / dC 16-byte aligned
-                atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(red[0], red[1], red[2], red[3]));
-                atomicAdd(reinterpret_cast<float4 *>(dst) + 1,
-                          make_float4(red[4], red[5], red[6], red[7]));
+            const int64_t off = copy + (int64_t(b) * N + rn) * p.L + t0 + ri;
+            float *db = p.pB + off, *dc = p.pC + off;
+            if (ri + 4 <= valid && (p.L & 3) == 0) {  // rows of dB / dC 16-byte aligned
+                atomicAdd(reinterpret_cast<float4 *>(db),
+                          make_float4(dBv[0], dBv[1], dBv[2], dBv[3]));
+                atomicAdd(reinterpret_cast<float4 *>(dc),
+                          make_float4(dCv[0], dCv[1], dCv[2], dCv[3]));
             } else {
 #pragma unroll
-                for (int i = 0; i < TC; ++i)
-                    if (i < valid)
-                        atomicAdd(dst + i, red[i]);
+                for (int r = 0; r < 4; ++r)
+                    if (ri + r < valid) {
+                        atomicAdd(db + r, dBv[r]);
+                        atomicAdd(dc + r, dCv[r]);
+                    }
             }
         }
         __syncwarp();

@@ -49,6 +49,7 @@ struct DeviceInfo {
 
 std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
+cudaMemPool_t g_pool[kMaxDevices] = {};  // scratch pools, created on first use
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 unsigned long long default_timeout_ns()
@@ -93,6 +94,44 @@ selscan_status device_setup(int *dev_out, DeviceInfo **info_out)
     *dev_out = dev;
     *info_out = &di;
     return SELSCAN_OK;
+}
+
+// Stream-ordered scratch from a pool of the library's own on the current
+// device.  Its release threshold keeps freed memory mapped: the device's
+// default pool hands memory back to the driver at every synchronisation, so
+// the next call would map the backward checkpoints (hundreds of MB) again.
+// selscan_release_scratch() trims the pools.
+cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t stream)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    cudaMemPool_t pool = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!g_pool[dev]) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.handleTypes = cudaMemHandleTypeNone;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            cudaMemPool_t np = nullptr;
+            if ((e = cudaMemPoolCreate(&np, &props)) != cudaSuccess)
+                return e;
+            uint64_t keep = UINT64_MAX;
+            if ((e = cudaMemPoolSetAttribute(np, cudaMemPoolAttrReleaseThreshold, &keep)) !=
+                cudaSuccess) {
+                cudaMemPoolDestroy(np);
+                return e;
+            }
+            g_pool[dev] = np;
+        }
+        pool = g_pool[dev];
+    }
+    return cudaMallocFromPoolAsync(p, bytes, pool, stream);
 }
 
 size_t elem_size(int32_t dt) { return dt == SELSCAN_BF16 ? 2 : 4; }
@@ -248,6 +287,7 @@ bool ensure_smem(K kern, int bytes, int dev, bool (&done)[kMaxDevices])
 }
 
 int g_dbg_diag_mode = -1;  // test hook, see selscan_debug_diag_mode
+int g_dbg_bwd_segs = 0;     // test hook, see selscan_debug_bwd_segments
 
 template <int KIND, typename T, int CH, int STAGES, bool GATE, bool SOFTPLUS>
 selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
@@ -326,7 +366,7 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
         const size_t sd_bytes = ((size_t(agg_units) * CH * 4 + 255) / 256) * 256;
         const size_t h0_bytes = prm.h0 ? size_t(batch) * dim * kDiagN * 4 : 0;
         void *ws = nullptr;
-        if (cudaMallocAsync(&ws, head + agg_bytes + sd_bytes + h0_bytes, stream) != cudaSuccess)
+        if (scratch_alloc(&ws, head + agg_bytes + sd_bytes + h0_bytes, stream) != cudaSuccess)
             return SELSCAN_ERR_CUDA;
         uint8_t *wsb = static_cast<uint8_t *>(ws);
         if (cudaMemsetAsync(wsb, 0, head, stream) != cudaSuccess ||
@@ -373,7 +413,7 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
     const size_t carry_bytes = size_t(units) * CH * kDiagN * 4;
     const size_t ws_bytes = head + flag_bytes + carry_bytes;
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess)
+    if (scratch_alloc(&ws, ws_bytes, stream) != cudaSuccess)
         return SELSCAN_ERR_CUDA;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     if (cudaMemsetAsync(wsb, 0, head + flag_bytes, stream) != cudaSuccess) {
@@ -431,10 +471,21 @@ unsigned long long selscan_launch_count(void)
     return g_launches.load(std::memory_order_relaxed);
 }
 
+selscan_status selscan_release_scratch(void)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    for (int d = 0; d < kMaxDevices; ++d)
+        if (g_pool[d] && cudaMemPoolTrimTo(g_pool[d], 0) != cudaSuccess)
+            return SELSCAN_ERR_CUDA;
+    return SELSCAN_OK;
+}
+
 // Test hook (not part of the public header's stable surface): withhold the
 // carry flag of one work unit so that its successor's bounded wait expires.
 // -1 switches it off.
 void selscan_debug_diag_mode(int mode) { g_dbg_diag_mode = mode; }
+
+void selscan_debug_bwd_segments(int segs) { g_dbg_bwd_segs = segs < 0 ? 0 : segs; }
 
 void selscan_debug_withhold_carry(int unit) { g_dbg_skip_publish = unit; }
 
@@ -1326,9 +1377,13 @@ extern "C" selscan_status selscan_bwd(
     prm.dbias = static_cast<float *>(ddelta_bias ? ddelta_bias->data : nullptr);
     prm.dh0 = static_cast<float *>(dh0 ? dh0->data : nullptr);
 
-    // Units: (batch row, 32 channels) x time segments, one warp each.  As
-    // many segments as fit in one wave of resident warps (a second, partial
-    // wave would double the time of its units), at least 32 chunks each.
+    // Units: (batch row, 32 channels) x time segments, one warp each, at
+    // least 32 chunks per segment.  As many segments as fit in one wave of
+    // resident warps when that wave is at least three quarters full (a
+    // second, partial wave would double the time of its units); otherwise
+    // about four waves of short segments, which balance better than one
+    // sparse wave (B4 D5120 L4096 on 148 SMs: 5.28 ms with one segment,
+    // 5.0 ms with 6 to 12).
     prm.tiles_per_batch = int((dim + 31) / 32);
     prm.tiles = int(batch) * prm.tiles_per_batch;
     {
@@ -1342,9 +1397,13 @@ extern "C" selscan_status selscan_bwd(
         if (oe != cudaSuccess || per_sm < 1)
             per_sm = 1;
         const int64_t slots = int64_t(per_sm) * di->sm_count;
-        const int64_t want = std::max<int64_t>(1, slots / prm.tiles);
+        int64_t want = std::max<int64_t>(1, slots / prm.tiles);
+        if (4 * want * prm.tiles < 3 * slots)
+            want = std::max<int64_t>(2, 4 * slots / prm.tiles);
         const int64_t max_segs = std::max<int64_t>(1, prm.nchunks / 32);
         int64_t S = std::max<int64_t>(1, std::min(want, max_segs));
+        if (g_dbg_bwd_segs > 0)
+            S = std::min<int64_t>(g_dbg_bwd_segs, std::max(1, prm.nchunks));
         const int64_t seg_chunks = (prm.nchunks + S - 1) / S;
         S = (prm.nchunks + seg_chunks - 1) / seg_chunks;
         if (int64_t(prm.tiles) * S > 0x7fffffffll)
@@ -1361,7 +1420,7 @@ extern "C" selscan_status selscan_bwd(
     const int64_t bc_n = batch * kBwdN * L;           // elements of dB (and of dC)
     const size_t part_bytes = size_t(kBwdCopies) * bc_n * 4;
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, ck_bytes + 2 * agg_bytes + s_bytes + 2 * part_bytes, stream) !=
+    if (scratch_alloc(&ws, ck_bytes + 2 * agg_bytes + s_bytes + 2 * part_bytes, stream) !=
         cudaSuccess)
         return SELSCAN_ERR_CUDA;
     uint8_t *wsb = static_cast<uint8_t *>(ws);

@@ -34,6 +34,12 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, n), f"{n} declared but not exported"
 
 
+def test_release_scratch_without_pools():
+    """Before any call has allocated scratch there is nothing to trim, and
+    the call makes no CUDA request (so it also runs without a GPU)."""
+    ss.release_scratch()
+
+
 def test_version_and_strerror():
     assert ss.version() == 10000
     for code in range(9):

@@ -148,3 +148,17 @@ def test_empty_sequence():
     g = ss.selscan_bwd(u, u, A, BC, BC, u, dlast=dlast, need_dh0=True)
     ss.check()
     assert torch.equal(g["dh0"], dlast) and torch.all(g["dA"] == 0)
+
+
+def test_results_unchanged_after_release_scratch():
+    """The scratch pool handed back between two calls: the second call maps
+    fresh memory and still matches the oracle."""
+    import torch
+    import selective_state_space_selscan_b200 as ss
+    inp = synthetic.make_diag(1, 96, 16, 512, dtype="f32", seed=87)
+    dy = _dy(inp, 88)
+    want = ref(inp, dy)
+    compare(run(inp, dy, "f32"), want, "f32")
+    torch.cuda.synchronize()
+    ss.release_scratch()
+    compare(run(inp, dy, "f32"), want, "f32")
