@@ -30,12 +30,12 @@
 // The expanded states (batch, D, L, N) are never stored.
 //
 // dB and dC sum over the channels of a batch row.  Per chunk they are sums
-// over the warp's lanes of rows of shared memory: dC_t[n] of dout_t times the
+// over the warp's lanes of shared memory: dC_t[n] of dout_t times the
 // recomputed states (before the reverse walk), dB_t[n] of the terms
 // g delta u that the walk writes over the states it has used.  Lane l sums
-// state n = l % 16 for four of the chunk's tokens and adds both results with
-// one 16-byte atomic each into one of kBwdCopies partial copies, which
-// bwd_reduce_bc sums at the end.  dA, dD and the bias gradient sum over batch
+// states 4 (l % 4) .. 4 (l % 4) + 3 of token l / 4 and adds both results
+// with one 16-byte atomic each into one of kBwdCopies partial copies
+// (token-major, [batch][L][16]), which bwd_reduce_bc sums and transposes.  dA, dD and the bias gradient sum over batch
 // rows and tokens: registers, then atomics.
 #pragma once
 
@@ -73,7 +73,7 @@ struct BwdParams {
     int64_t du_bs, du_ds, dd_bs, dd_ds, dz_bs, dz_ds;
     float *dA;                       // (dim, 16), accumulated
     float *dB, *dC;                  // (batch, 16, L) contiguous, written by bwd_reduce_bc
-    float *pB, *pC;                  // kBwdCopies partial sums of dB, dC, accumulated
+    float *pB, *pC;                  // kBwdCopies partial sums [batch][L][16] of dB, dC
     float *dD, *dbias;               // (dim) or null, accumulated
     float *dh0;                      // (batch, dim, 16) or null, written
     float *ckpt;                     // [batch][dim][nchunks][16] scratch
@@ -145,39 +145,63 @@ __device__ __forceinline__ float bwd_step(float raw, int softplus)
 }
 
 // Per-warp shared memory: B and C of the chunk (fp32, [token][n]), the
-// recomputed states of the chunk ([token][n][lane]; the reverse walk puts
-// each lane's dB terms in their place once it has used them) and the output
-// gradient through the gate ([token][lane]).
+// recomputed states of the chunk ([token][lane] rows of 16 states in four
+// 16-byte pieces; the reverse walk puts each lane's dB terms in their place
+// once it has used them) and the output gradient through the gate
+// ([token][lane]).  Piece c of lane l's row sits at position
+// c ^ ((l >> 1) & 3): the eight lanes of a quarter warp that store or load
+// the same piece of their own rows then hit eight distinct bank groups.
 struct BwdSmem {
     float bc[kBwdT][2][kBwdN];
-    float h[kBwdT][kBwdN][32];
+    float4 h[kBwdT][32][4];
     float dout[kBwdT][32];
 };
 
-// Sum over the warp's 32 lanes of row (i, n) of sm.h, weighted by sm.dout[i]
-// when WEIGHTED.  Each lane starts at its own 16-byte column, so the eight
-// lanes of a quarter warp (eight rows of one token) read distinct banks.
-template <bool WEIGHTED>
-__device__ __forceinline__ float bwd_row_sum(const BwdSmem &sm, int i, int n, int lane)
+__device__ __forceinline__ int bwd_piece(int l, int c) { return c ^ ((l >> 1) & 3); }
+
+// This lane's 16 values of token i (8 pairs) into / out of sm.h.
+__device__ __forceinline__ void bwd_put_row(BwdSmem &sm, int i, int lane, const uint64_t (&v)[8])
 {
-    const float4 *hr = reinterpret_cast<const float4 *>(sm.h[i][n]);
-    const float4 *wr = reinterpret_cast<const float4 *>(sm.dout[i]);
-    uint64_t s0 = pk2(0.f, 0.f), s1 = pk2(0.f, 0.f);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int c = (k + lane) & 7;
-        const float4 h = hr[c];
+    for (int c = 0; c < 4; ++c)
+        sm.h[i][lane][bwd_piece(lane, c)] =
+            make_float4(lo2(v[2 * c]), hi2(v[2 * c]), lo2(v[2 * c + 1]), hi2(v[2 * c + 1]));
+}
+
+__device__ __forceinline__ void bwd_get_row(const BwdSmem &sm, int i, int lane, uint64_t (&v)[8])
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float4 q = sm.h[i][lane][bwd_piece(lane, c)];
+        v[2 * c] = pk2(q.x, q.y);
+        v[2 * c + 1] = pk2(q.z, q.w);
+    }
+}
+
+// Sum over the warp's 32 lanes of piece c (states 4c .. 4c + 3) of token i,
+// weighted by sm.dout[i] when WEIGHTED.  The lanes of token i start at row
+// i: a quarter warp (two consecutive tokens, four pieces each) then reads
+// eight distinct bank groups at every step, and the eight tokens' weights
+// lie in eight distinct banks.
+template <bool WEIGHTED>
+__device__ __forceinline__ float4 bwd_piece_sum(const BwdSmem &sm, int i, int c)
+{
+    uint64_t s0 = pk2(0.f, 0.f), s1 = pk2(0.f, 0.f);
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+        const int l = (k + i) & 31;
+        const float4 h = sm.h[i][l][bwd_piece(l, c)];
         if (WEIGHTED) {
-            const float4 w = wr[c];
-            s0 = fma2(pk2(w.x, w.y), pk2(h.x, h.y), s0);
-            s1 = fma2(pk2(w.z, w.w), pk2(h.z, h.w), s1);
+            const float w = sm.dout[i][l];
+            const uint64_t W = pk2(w, w);
+            s0 = fma2(W, pk2(h.x, h.y), s0);
+            s1 = fma2(W, pk2(h.z, h.w), s1);
         } else {
             s0 = add2(pk2(h.x, h.y), s0);
             s1 = add2(pk2(h.z, h.w), s1);
         }
     }
-    const uint64_t s = add2(s0, s1);
-    return lo2(s) + hi2(s);
+    return make_float4(lo2(s0), hi2(s0), lo2(s1), hi2(s1));
 }
 
 // One chunk's raw inputs, copied asynchronously: per lane its channel's 8
@@ -315,12 +339,13 @@ struct BwdChannel {
 };
 
 // Forward over [t0, t0 + valid): h <- abar h + delta u B, token by token;
-// when `keep` is set the state after each token goes to shared memory.
+// when KEEP is set the state after each token goes to shared memory and
+// the step sizes to dts.
 template <typename T, bool KEEP>
 __device__ __forceinline__ void bwd_forward_chunk(const BwdParams &p, const BwdChannel<T> &ch,
                                                   BwdSmem &sm, int valid, const float (&uv)[8],
                                                   const float (&dv)[8], uint64_t (&h2)[8],
-                                                  int lane)
+                                                  int lane, float (&dts)[8])
 {
     constexpr bool FAST = !std::is_same<T, float>::value;
 #pragma unroll
@@ -328,6 +353,8 @@ __device__ __forceinline__ void bwd_forward_chunk(const BwdParams &p, const BwdC
         if (i >= valid)
             break;
         const float dt = bwd_step<FAST>(dv[i] + ch.bias, p.softplus);
+        if (KEEP)
+            dts[i] = dt;
         const float dx = dt * uv[i];
         const uint64_t DX = pk2(dx, dx);
         uint64_t a2[8];
@@ -339,13 +366,8 @@ __device__ __forceinline__ void bwd_forward_chunk(const BwdParams &p, const BwdC
             h2[2 * q] = fma2(a2[2 * q], h2[2 * q], mul2(DX, pk2(bb.x, bb.y)));
             h2[2 * q + 1] = fma2(a2[2 * q + 1], h2[2 * q + 1], mul2(DX, pk2(bb.z, bb.w)));
         }
-        if (KEEP) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                sm.h[i][2 * j][lane] = lo2(h2[j]);
-                sm.h[i][2 * j + 1][lane] = hi2(h2[j]);
-            }
-        }
+        if (KEEP)
+            bwd_put_row(sm, i, lane, h2);
     }
 }
 
@@ -392,7 +414,7 @@ bwd_agg_kernel(const BwdParams p)
                                  t0 + kBwdT, min(kBwdT, p.L - t0 - kBwdT), lane, what, nullptr);
             cp_async_commit();
             cp_async_wait<1>();
-            float uv[8], dv[8];
+            float uv[8], dv[8], dts[8];  // dts unused (KEEP off)
             bwd_vals<T, KV>(st[buf].dl, lane, dv);
 #pragma unroll
             for (int i = 0; i < kBwdT; ++i)
@@ -401,7 +423,7 @@ bwd_agg_kernel(const BwdParams p)
             if (fwd) {
                 bwd_vals<T, KV>(st[buf].u, lane, uv);
                 bwd_bc_to_smem<T, KV>(st[buf], sm, lane, false);
-                bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane);
+                bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane, dts);
             }
             __syncwarp();
             buf ^= 1;
@@ -548,11 +570,11 @@ selscan_bwd_kernel(const BwdParams p)
                                          hi2(h2[2 * q + 1]));
             }
             cp_async_wait<1>();
-            float uv[8], dv[8];
+            float uv[8], dv[8], dts[8];  // dts unused (KEEP off)
             bwd_vals<T, KV>(st[buf].u, lane, uv);
             bwd_vals<T, KV>(st[buf].dl, lane, dv);
             bwd_bc_to_smem<T, KV>(st[buf], sm, lane, false);
-            bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane);
+            bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane, dts);
             __syncwarp();
             buf ^= 1;
         }
@@ -589,7 +611,7 @@ selscan_bwd_kernel(const BwdParams p)
             hc2[2 * q] = pk2(v.x, v.y);
             hc2[2 * q + 1] = pk2(v.z, v.w);
         }
-        float uv[8], dv[8], yv[8], zv[8];
+        float uv[8], dv[8], yv[8], zv[8], dts[8];
         bwd_vals<T, KV>(cur.u, lane, uv);
         bwd_vals<T, KV>(cur.dl, lane, dv);
         bwd_vals<T, KV>(cur.dy, lane, yv);
@@ -601,7 +623,7 @@ selscan_bwd_kernel(const BwdParams p)
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 hr[j] = hc2[j];
-            bwd_forward_chunk<T, true>(p, ch, sm, valid, uv, dv, hr, lane);
+            bwd_forward_chunk<T, true>(p, ch, sm, valid, uv, dv, hr, lane, dts);
         }
         __syncwarp();
         // output gradient through the gate and the factor of dz, per token
@@ -621,12 +643,9 @@ selscan_bwd_kernel(const BwdParams p)
             sm.dout[i][lane] = dout;
         }
         __syncwarp();
-        // dC of the chunk: lane -> state rn, tokens ri .. ri + 3
-        const int rn = lane & (N - 1), ri = 4 * (lane >> 4);
-        float dCv[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-            dCv[r] = bwd_row_sum<true>(sm, ri + r, rn, lane);
+        // dC of the chunk: lane -> token ri, states 4 rc .. 4 rc + 3
+        const int ri = lane >> 2, rc = lane & 3;
+        const float4 dCv = bwd_piece_sum<true>(sm, ri, rc);
         __syncwarp();  // all rows read before the walk overwrites them
         float o_du[8], o_dd[8], o_dz[8];
 #pragma unroll
@@ -640,18 +659,18 @@ selscan_bwd_kernel(const BwdParams p)
         for (int i = TC - 1; i >= 0; --i) {
             if (i >= valid)
                 continue;
-            if (i == valid - 1) {
+            if (i == valid - 1)
+                bwd_get_row(sm, i, lane, ht2);
+            uint64_t hp2[8];
+            if (i > 0) {
+                bwd_get_row(sm, i - 1, lane, hp2);
+            } else {
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    ht2[j] = pk2(sm.h[i][2 * j][lane], sm.h[i][2 * j + 1][lane]);
+                    hp2[j] = hc2[j];
             }
-            uint64_t hp2[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                hp2[j] = i > 0 ? pk2(sm.h[i - 1][2 * j][lane], sm.h[i - 1][2 * j + 1][lane])
-                               : hc2[j];
             const float raw = dv[i] + ch.bias;
-            const float dt = bwd_step<FAST>(raw, p.softplus);
+            const float dt = dts[i];
             const float x = uv[i];
             uint64_t a2[8];
             bwd_decays<FAST>(dt, ch.al, ch.pow_path, a2);
@@ -677,57 +696,44 @@ selscan_bwd_kernel(const BwdParams p)
             }
             const float dout = dov[i];
             gD = fmaf(dout, x, gD);
-            const uint64_t DO = pk2(dout, dout), DT = pk2(dt, dt), X = pk2(x, x);
-            uint64_t dx2 = pk2(0.f, 0.f), ddt2 = pk2(0.f, 0.f);
+            // with g after adding dout C:  du = dt sum g B + D dout,
+            // ddelta = sum g A abar h_prev + u sum g B,  dA += dt g abar h_prev
+            const uint64_t DO = pk2(dout, dout), DT = pk2(dt, dt);
+            const uint64_t DTX = pk2(dt * x, dt * x);
+            uint64_t gB2 = pk2(0.f, 0.f), gAh2 = pk2(0.f, 0.f), vb[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 g2[j] = fma2(DO, C2[j], g2[j]);
-                const uint64_t gdt = mul2(g2[j], DT);
-                const uint64_t vb = mul2(gdt, X);
-                sm.h[i][2 * j][lane] = lo2(vb);  // this lane's dB terms of token i
-                sm.h[i][2 * j + 1][lane] = hi2(vb);
-                dx2 = fma2(gdt, B2[j], dx2);
-                const uint64_t ah = mul2(a2[j], hp2[j]);
-                ddt2 = fma2(g2[j], fma2(ch.An2[j], ah, mul2(B2[j], X)), ddt2);
-                gA2[j] = fma2(gdt, ah, gA2[j]);
+                vb[j] = mul2(g2[j], DTX);
+                gB2 = fma2(g2[j], B2[j], gB2);
+                const uint64_t gah = mul2(g2[j], mul2(a2[j], hp2[j]));
+                gAh2 = fma2(ch.An2[j], gah, gAh2);
+                gA2[j] = fma2(DT, gah, gA2[j]);
                 g2[j] = mul2(g2[j], a2[j]);
                 ht2[j] = hp2[j];
             }
-            const float dx = fmaf(dout, ch.dsk, lo2(dx2) + hi2(dx2));
-            const float ddt = lo2(ddt2) + hi2(ddt2);
+            bwd_put_row(sm, i, lane, vb);  // this lane's dB terms of token i
+            const float gB = lo2(gB2) + hi2(gB2);
+            const float dx = fmaf(dout, ch.dsk, dt * gB);
+            const float ddt = fmaf(x, gB, lo2(gAh2) + hi2(gAh2));
             const float dDelta = p.softplus ? ddt / (1.f + __expf(-raw)) : ddt;
             gbias += dDelta;
             o_du[i] = dx;
             o_dd[i] = dDelta;
         }
         __syncwarp();
-        float dBv[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-            dBv[r] = bwd_row_sum<false>(sm, ri + r, rn, lane);
+        const float4 dBv = bwd_piece_sum<false>(sm, ri, rc);
         if (live) {
             bwd_st8(p.du, ch.row_du + t0, valid, o_du, tag);
             bwd_st8(p.ddelta, ch.row_dd + t0, valid, o_dd, tag);
             if (p.z)
                 bwd_st8(p.dz, ch.row_dz + t0, valid, o_dz, tag);
         }
-        {
-            const int64_t copy = int64_t(tile % kBwdCopies) * p.batch * N * p.L;
-            const int64_t off = copy + (int64_t(b) * N + rn) * p.L + t0 + ri;
-            float *db = p.pB + off, *dc = p.pC + off;
-            if (ri + 4 <= valid && (p.L & 3) == 0) {  // rows of dB / dC 16-byte aligned
-                atomicAdd(reinterpret_cast<float4 *>(db),
-                          make_float4(dBv[0], dBv[1], dBv[2], dBv[3]));
-                atomicAdd(reinterpret_cast<float4 *>(dc),
-                          make_float4(dCv[0], dCv[1], dCv[2], dCv[3]));
-            } else {
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    if (ri + r < valid) {
-                        atomicAdd(db + r, dBv[r]);
-                        atomicAdd(dc + r, dCv[r]);
-                    }
-            }
+        if (ri < valid) {
+            const int64_t off = ((int64_t(tile % kBwdCopies) * p.batch + b) * p.L + t0 + ri) * N +
+                                4 * rc;
+            atomicAdd(reinterpret_cast<float4 *>(p.pB + off), dBv);
+            atomicAdd(reinterpret_cast<float4 *>(p.pC + off), dCv);
         }
         __syncwarp();
         bufB ^= 1;
@@ -753,20 +759,37 @@ selscan_bwd_kernel(const BwdParams p)
     }
 }
 
-// dB, dC = sum of the kBwdCopies partial copies (n elements each).
+// dB, dC (batch, 16, L) = sum of the kBwdCopies partial copies, each
+// [batch][L][16] (`rows` = batch * L rows of 16).  One thread per row: it
+// reads its row's 64 bytes from every copy and writes state n to dB[b][n][t],
+// consecutive threads writing consecutive tokens.
 __global__ void __launch_bounds__(256)
-bwd_reduce_bc(const float *pB, const float *pC, float *dB, float *dC, int64_t n)
+bwd_reduce_bc(const float *pB, const float *pC, float *dB, float *dC, int64_t rows, int L)
 {
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += int64_t(gridDim.x) * blockDim.x) {
-        float sb = 0.f, sc = 0.f;
+    const int64_t copy = rows * kBwdN;  // floats per partial copy
+    for (int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; r < rows;
+         r += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t b = r / L, t = r - b * L;
+        float *ob = dB + b * kBwdN * L + t, *oc = dC + b * kBwdN * L + t;
 #pragma unroll
-        for (int k = 0; k < kBwdCopies; ++k) {
-            sb += pB[int64_t(k) * n + i];
-            sc += pC[int64_t(k) * n + i];
+        for (int q = 0; q < 4; ++q) {
+            float4 sb = make_float4(0.f, 0.f, 0.f, 0.f), sc = sb;
+#pragma unroll
+            for (int k = 0; k < kBwdCopies; ++k) {
+                const float4 vb = reinterpret_cast<const float4 *>(pB + k * copy + r * kBwdN)[q];
+                const float4 vc = reinterpret_cast<const float4 *>(pC + k * copy + r * kBwdN)[q];
+                sb.x += vb.x; sb.y += vb.y; sb.z += vb.z; sb.w += vb.w;
+                sc.x += vc.x; sc.y += vc.y; sc.z += vc.z; sc.w += vc.w;
+            }
+            ob[int64_t(4 * q) * L] = sb.x;
+            ob[int64_t(4 * q + 1) * L] = sb.y;
+            ob[int64_t(4 * q + 2) * L] = sb.z;
+            ob[int64_t(4 * q + 3) * L] = sb.w;
+            oc[int64_t(4 * q) * L] = sc.x;
+            oc[int64_t(4 * q + 1) * L] = sc.y;
+            oc[int64_t(4 * q + 2) * L] = sc.z;
+            oc[int64_t(4 * q + 3) * L] = sc.w;
         }
-        dB[i] = sb;
-        dC[i] = sc;
     }
 }
 

@@ -1450,9 +1450,10 @@ extern "C" selscan_status selscan_bwd(
         le = counted_launch();
     }
     if (le == cudaSuccess) {
-        const int64_t blocks = std::min<int64_t>((bc_n + 255) / 256, 8ll * di->sm_count);
+        const int64_t rows = batch * L;
+        const int64_t blocks = std::min<int64_t>((rows + 255) / 256, 8ll * di->sm_count);
         bwd_reduce_bc<<<unsigned(blocks), 256, 0, stream>>>(prm.pB, prm.pC, prm.dB, prm.dC,
-                                                            bc_n);
+                                                            rows, int(L));
         le = counted_launch();
     }
     cudaFreeAsync(ws, stream);
