@@ -121,13 +121,17 @@ __device__ __forceinline__ void bwd_decays(float dt, const float (&al)[kBwdN], b
                                            uint64_t (&a2)[8])
 {
     if (pow_path) {
+        // r^1 .. r^16 by a product tree (depth 4, not a chain of 7)
         const float r = FAST ? ex2_approx(dt * al[0]) : exp2f(dt * al[0]);
-        const float r2 = r * r;
-        const uint64_t R2 = pk2(r2, r2);
+        const float r2 = r * r, r4 = r2 * r2, r8 = r4 * r4;
+        const uint64_t R2 = pk2(r2, r2), R4 = pk2(r4, r4), R8 = pk2(r8, r8);
         a2[0] = pk2(r, r2);
+        a2[1] = mul2(a2[0], R2);
+        a2[2] = mul2(a2[0], R4);
+        a2[3] = mul2(a2[1], R4);
 #pragma unroll
-        for (int j = 1; j < 8; ++j)
-            a2[j] = mul2(a2[j - 1], R2);
+        for (int j = 4; j < 8; ++j)
+            a2[j] = mul2(a2[j - 4], R8);
     } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -144,15 +148,20 @@ __device__ __forceinline__ float bwd_step(float raw, int softplus)
     return FAST ? softplus_fast(raw) : softplus_exact(raw);
 }
 
-// Per-warp shared memory: B and C of the chunk (fp32, [token][n]), the
-// recomputed states of the chunk ([token][lane] rows of 16 states in four
-// 16-byte pieces; the reverse walk puts each lane's dB terms in their place
-// once it has used them) and the output gradient through the gate
-// ([token][lane]).  Piece c of lane l's row sits at position
-// c ^ ((l >> 1) & 3): the eight lanes of a quarter warp that store or load
-// the same piece of their own rows then hit eight distinct bank groups.
-struct BwdSmem {
+// B and C of the chunk (fp32, [token][n]): all the aggregate kernel keeps
+// in shared memory besides its copy stages, so it fits more warps per SM.
+struct BwdBC {
     float bc[kBwdT][2][kBwdN];
+};
+
+// Per-warp shared memory of the gradient walk: B and C, the recomputed
+// states of the chunk ([token][lane] rows of 16 states in four 16-byte
+// pieces; the reverse walk puts each lane's dB terms in their place once it
+// has used them) and the output gradient through the gate ([token][lane]).
+// Piece c of lane l's row sits at position c ^ ((l >> 1) & 3): the eight
+// lanes of a quarter warp that store or load the same piece of their own
+// rows then hit eight distinct bank groups.
+struct BwdSmem : BwdBC {
     float4 h[kBwdT][32][4];
     float dout[kBwdT][32];
 };
@@ -183,25 +192,32 @@ __device__ __forceinline__ void bwd_get_row(const BwdSmem &sm, int i, int lane, 
 // i: a quarter warp (two consecutive tokens, four pieces each) then reads
 // eight distinct bank groups at every step, and the eight tokens' weights
 // lie in eight distinct banks.
+// Four partial sums per half-piece keep the dependent chains 8 long.
 template <bool WEIGHTED>
 __device__ __forceinline__ float4 bwd_piece_sum(const BwdSmem &sm, int i, int c)
 {
-    uint64_t s0 = pk2(0.f, 0.f), s1 = pk2(0.f, 0.f);
-#pragma unroll 8
+    uint64_t s0[4], s1[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+        s0[a] = s1[a] = pk2(0.f, 0.f);
+#pragma unroll
     for (int k = 0; k < 32; ++k) {
         const int l = (k + i) & 31;
         const float4 h = sm.h[i][l][bwd_piece(l, c)];
+        const int a = k & 3;
         if (WEIGHTED) {
             const float w = sm.dout[i][l];
             const uint64_t W = pk2(w, w);
-            s0 = fma2(W, pk2(h.x, h.y), s0);
-            s1 = fma2(W, pk2(h.z, h.w), s1);
+            s0[a] = fma2(W, pk2(h.x, h.y), s0[a]);
+            s1[a] = fma2(W, pk2(h.z, h.w), s1[a]);
         } else {
-            s0 = add2(pk2(h.x, h.y), s0);
-            s1 = add2(pk2(h.z, h.w), s1);
+            s0[a] = add2(pk2(h.x, h.y), s0[a]);
+            s1[a] = add2(pk2(h.z, h.w), s1[a]);
         }
     }
-    return make_float4(lo2(s0), hi2(s0), lo2(s1), hi2(s1));
+    const uint64_t t0 = add2(add2(s0[0], s0[1]), add2(s0[2], s0[3]));
+    const uint64_t t1 = add2(add2(s1[0], s1[1]), add2(s1[2], s1[3]));
+    return make_float4(lo2(t0), hi2(t0), lo2(t1), hi2(t1));
 }
 
 // One chunk's raw inputs, copied asynchronously: per lane its channel's 8
@@ -291,7 +307,7 @@ __device__ __forceinline__ void bwd_vals(const uint4 (&src)[KV][32], int lane, f
 
 // Staged B / C rows -> fp32 [token][n] for the whole warp.
 template <typename T, int KV>
-__device__ __forceinline__ void bwd_bc_to_smem(const BwdStage<KV> &st, BwdSmem &sm, int lane,
+__device__ __forceinline__ void bwd_bc_to_smem(const BwdStage<KV> &st, BwdBC &sm, int lane,
                                                bool withC)
 {
     if (lane < kBwdN || withC) {
@@ -339,11 +355,11 @@ struct BwdChannel {
 };
 
 // Forward over [t0, t0 + valid): h <- abar h + delta u B, token by token;
-// when KEEP is set the state after each token goes to shared memory and
-// the step sizes to dts.
-template <typename T, bool KEEP>
+// when KEEP is set (SM = BwdSmem) the state after each token goes to shared
+// memory and the step sizes to dts.
+template <typename T, bool KEEP, typename SM>
 __device__ __forceinline__ void bwd_forward_chunk(const BwdParams &p, const BwdChannel<T> &ch,
-                                                  BwdSmem &sm, int valid, const float (&uv)[8],
+                                                  SM &sm, int valid, const float (&uv)[8],
                                                   const float (&dv)[8], uint64_t (&h2)[8],
                                                   int lane, float (&dts)[8])
 {
@@ -366,7 +382,7 @@ __device__ __forceinline__ void bwd_forward_chunk(const BwdParams &p, const BwdC
             h2[2 * q] = fma2(a2[2 * q], h2[2 * q], mul2(DX, pk2(bb.x, bb.y)));
             h2[2 * q + 1] = fma2(a2[2 * q + 1], h2[2 * q + 1], mul2(DX, pk2(bb.z, bb.w)));
         }
-        if (KEEP)
+        if constexpr (KEEP)
             bwd_put_row(sm, i, lane, h2);
     }
 }
@@ -379,7 +395,7 @@ __global__ void __launch_bounds__(32)
 bwd_agg_kernel(const BwdParams p)
 {
     constexpr bool FAST = !std::is_same<T, float>::value;
-    __shared__ __align__(16) BwdSmem sm;
+    __shared__ __align__(16) BwdBC sm;
     const int lane = threadIdx.x;
     const int unit = blockIdx.x;
     const int seg = unit / p.tiles, tile = unit - seg * p.tiles;

@@ -1378,12 +1378,13 @@ extern "C" selscan_status selscan_bwd(
     prm.dh0 = static_cast<float *>(dh0 ? dh0->data : nullptr);
 
     // Units: (batch row, 32 channels) x time segments, one warp each, at
-    // least 32 chunks per segment.  As many segments as fit in one wave of
-    // resident warps when that wave is at least three quarters full (a
-    // second, partial wave would double the time of its units); otherwise
-    // about four waves of short segments, which balance better than one
-    // sparse wave (B4 D5120 L4096 on 148 SMs: 5.28 ms with one segment,
-    // 5.0 ms with 6 to 12).
+    // least 32 chunks per segment.  A wave of resident warps ends with its
+    // slowest unit, so the time goes as ceil(units / slots) / S: choose S
+    // (at most four waves) within 2 % of the lowest such cost, the smallest
+    // one that gives at least 1.5 waves (shorter units balance better over
+    // the SMs; more segments cost more aggregate work).  On 148 SMs this
+    // picks 7 segments for B4 D5120 L4096 (4.05 ms; 6 or 8: 4.25-4.45 ms)
+    // and 6 for B8 D1536 L2048 (1.30 ms; 3: 1.37 ms).
     prm.tiles_per_batch = int((dim + 31) / 32);
     prm.tiles = int(batch) * prm.tiles_per_batch;
     {
@@ -1397,11 +1398,23 @@ extern "C" selscan_status selscan_bwd(
         if (oe != cudaSuccess || per_sm < 1)
             per_sm = 1;
         const int64_t slots = int64_t(per_sm) * di->sm_count;
-        int64_t want = std::max<int64_t>(1, slots / prm.tiles);
-        if (4 * want * prm.tiles < 3 * slots)
-            want = std::max<int64_t>(2, 4 * slots / prm.tiles);
-        const int64_t max_segs = std::max<int64_t>(1, prm.nchunks / 32);
-        int64_t S = std::max<int64_t>(1, std::min(want, max_segs));
+        const int64_t max_segs = std::max<int64_t>(
+            1, std::min<int64_t>(prm.nchunks / 32, 4 * slots / prm.tiles));
+        auto waves = [&](int64_t s) { return (prm.tiles * s + slots - 1) / slots; };
+        double best = 1e30;
+        for (int64_t s = 1; s <= max_segs; ++s)
+            best = std::min(best, double(waves(s)) / double(s));
+        int64_t S = 0, S_any = 0;
+        for (int64_t s = 1; s <= max_segs && !S; ++s) {
+            if (double(waves(s)) / double(s) > 1.02 * best)
+                continue;
+            if (!S_any)
+                S_any = s;
+            if (2 * prm.tiles * s >= 3 * slots)
+                S = s;
+        }
+        if (!S)
+            S = S_any;
         if (g_dbg_bwd_segs > 0)
             S = std::min<int64_t>(g_dbg_bwd_segs, std::max(1, prm.nchunks));
         const int64_t seg_chunks = (prm.nchunks + S - 1) / S;
