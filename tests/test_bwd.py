@@ -138,6 +138,35 @@ def test_larger_sampled_channels():
         compare(part, {k: want[k] for k in part}, "bf16")
 
 
+def test_full_size_config2_sampled():
+    """The benchmark's workload, B4 D5120 L4096 bf16 with gate, D and bias,
+    in the launch configuration it times.  Per-channel gradients are
+    checked on channels sampled at the start, middle and end of d_inner.
+    dB and dC sum over all channels, so a second call gets dy only on the
+    sampled channels: every other channel then has a zero gradient state
+    and adds exactly zero, and the oracle's sums over the sampled channels
+    are the whole answer."""
+    inp = synthetic.make_config(2)
+    dy = _dy(inp, 93)
+    dim = inp["u"].shape[1]
+    ranges = [(0, 4), (dim // 2 - 2, dim // 2 + 2), (dim - 4, dim)]
+    chans = np.concatenate([np.arange(a, b) for a, b in ranges])
+    sub = dict(inp, u=inp["u"][:, chans], delta=inp["delta"][:, chans], z=inp["z"][:, chans],
+               A=inp["A"][chans], D=inp["D"][chans], delta_bias=inp["delta_bias"][chans])
+    want = ref(sub, np.ascontiguousarray(dy[:, chans]))
+    got = run(inp, dy, "bf16")
+    part = {"du": got["du"][:, chans], "ddelta": got["ddelta"][:, chans],
+            "dz": got["dz"][:, chans], "dA": got["dA"][chans], "dD": got["dD"][chans],
+            "ddelta_bias": got["ddelta_bias"][chans], "dh0": None}
+    compare(part, {k: want[k] for k in part}, "bf16")
+    dy_masked = np.zeros_like(dy)
+    dy_masked[:, chans] = dy[:, chans]
+    got = run(inp, dy_masked, "bf16")
+    compare({"dB": got["dB"], "dC": got["dC"]}, {"dB": want["dB"], "dC": want["dC"]}, "bf16")
+    others = np.setdiff1d(np.arange(dim), chans)[::97]
+    assert not got["du"][:, others].any() and not got["dA"][others].any()
+
+
 def test_empty_sequence():
     import torch
     import selective_state_space_selscan_b200 as ss
