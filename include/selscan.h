@@ -183,7 +183,7 @@ SELSCAN_API selscan_status selscan_fwd_scalarA_h0(const selscan_tensor *x,
  * pools, which selscan_fwd uses for its scratch) is unavailable.
  *
  * Same arguments, layouts and results as selscan_fwd; the caller passes all
- * inputs and outputs.  Instead of cudaMallocAsync, the look-back scratch
+ * inputs and outputs.  Instead of the stream-ordered pool, the look-back scratch
  * (ticket, carry flags, segment carries) lives in one file-scope device
  * array of SELSCAN_NOALLOC_SCRATCH_BYTES per GPU, which every GPU that loads
  * the library holds until the process exits.  The call makes no
