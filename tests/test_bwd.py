@@ -167,6 +167,26 @@ def test_full_size_config2_sampled():
     assert not got["du"][:, others].any() and not got["dA"][others].any()
 
 
+@pytest.mark.parametrize("segs", [1, 3, 16])
+def test_forced_segment_counts(segs):
+    """The same gradients whatever the number of time segments per tile:
+    the segment folds (end states and start gradients of the earlier and
+    later segments) against the oracle, with h0 and a final-state gradient;
+    187 chunks, so the last segment is shorter than the others."""
+    import selective_state_space_selscan_b200 as ss
+    inp = synthetic.make_diag(2, 64, 16, 1496, dtype="bf16", seed=94)
+    rng = np.random.default_rng(95)
+    h0 = rng.standard_normal((2, 64, 16)).astype(np.float32)
+    dlast = rng.standard_normal((2, 64, 16)).astype(np.float32)
+    dy = _dy(inp, 96)
+    ss.debug_bwd_segments(segs)
+    try:
+        got = run(inp, dy, "bf16", h0, dlast)
+    finally:
+        ss.debug_bwd_segments(0)
+    compare(got, ref(inp, dy, h0, dlast), "bf16")
+
+
 def test_empty_sequence():
     import torch
     import selective_state_space_selscan_b200 as ss
