@@ -250,6 +250,38 @@ def oracle_sample(cfg_idx: int, inp: dict, seconds: float = 10.0):
                       f"{spent:.1f} s single-threaded fp64"}
 
 
+def scan_config(cfg: dict, world: int) -> dict:
+    """The ``config`` object of a forward-scan line (both arms)."""
+    return {"workload": cfg["name"], "batch": cfg["batch"],
+            "d_inner": cfg.get("dim") or cfg["nheads"] * cfg["headdim"],
+            "d_state": cfg["N"], "seq_len": cfg["L"], "seed": cfg["seed"],
+            "global_batch": cfg["batch"] * world,
+            "l2": "inputs larger than L2 (no flush)" if algorithmic_bytes(cfg) > 126e6 else
+                  "inputs smaller than L2",
+            "parallelism": f"dp{world} (independent shards, no collective)"}
+
+
+def step_config(cfg: dict, world: int) -> dict:
+    """The ``config`` object of a decode-step line (both arms); ``cfg`` is
+    the step workload (``step_workload``)."""
+    dim = cfg.get("dim") or cfg["nheads"] * cfg["headdim"]
+    return {"workload": step_name(cfg), "batch": cfg["batch"], "d_inner": dim,
+            "d_state": cfg["N"], "global_batch": cfg["batch"] * world,
+            "l2": "state larger than L2 (no flush)" if step_bytes(cfg) > 126e6 else
+                  "state smaller than L2",
+            "parallelism": f"dp{world} (independent shards, no collective)"}
+
+
+def bwd_config(cfg: dict, world: int) -> dict:
+    """The ``config`` object of a backward line (both arms)."""
+    return {"workload": "backward of " + cfg["name"], "batch": cfg["batch"],
+            "d_inner": cfg["dim"], "d_state": cfg["N"], "seq_len": cfg["L"],
+            "global_batch": cfg["batch"] * world,
+            "l2": "inputs larger than L2 (no flush)" if bwd_bytes(cfg) > 126e6 else
+                  "inputs smaller than L2",
+            "parallelism": f"dp{world} (independent shards, no collective)"}
+
+
 def run_reference(args, rank: int, world: int):
     """Reference arm: the fp64 oracle on the host cores (rank 0 only)."""
     if rank != 0:
@@ -299,8 +331,9 @@ def run_reference(args, rank: int, world: int):
         "n_gpus": world, "steps": steps_done, "warmup": args.warmup,
         "ms_per_step": dt / steps_done * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg["name"], "sample_per_step": "one channel (all batches, all tokens)"
-                   if cfg["kind"] == "diag" else "one head"},
+        "config": dict(scan_config(cfg, world),
+                       sample_per_step="one channel (all batches, all tokens)"
+                       if cfg["kind"] == "diag" else "one head"),
         "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
                          "sample": f"{steps_done} steps x {elems // max(steps_done, 1)} elements"},
         "e2e": {"value": val, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
@@ -345,7 +378,7 @@ def run_reference_step(args, world: int):
         "value": val, "unit": "tokens/s", "n_gpus": world, "steps": done,
         "warmup": args.warmup, "ms_per_step": dt / done * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": step_name(cfg), "sample_per_step": f"{rows} batch rows"},
+        "config": dict(step_config(cfg, world), sample_per_step=f"{rows} batch rows"),
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": f"{done} steps x {rows} batch rows"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -387,8 +420,8 @@ def run_reference_bwd(args, world: int):
         "value": val, "unit": "Gelem/s", "n_gpus": world, "steps": done,
         "warmup": args.warmup, "ms_per_step": dt / done * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "backward of " + cfg["name"],
-                   "sample_per_step": "one channel (all batches, all tokens)"},
+        "config": dict(bwd_config(cfg, world),
+                       sample_per_step="one channel (all batches, all tokens)"),
         "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
                          "sample": f"{done} steps x one channel"},
         "e2e": {"value": val, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
@@ -546,13 +579,7 @@ def run_gpu(args, rank: int, world: int, local: int):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": dt, "data": "synthetic",
-        "config": {"workload": cfg["name"], "batch": cfg["batch"],
-                   "d_inner": cfg.get("dim") or cfg["nheads"] * cfg["headdim"],
-                   "d_state": cfg["N"], "seq_len": cfg["L"], "seed": cfg["seed"],
-                   "global_batch": cfg["batch"] * world,
-                   "l2": "inputs larger than L2 (no flush)" if nbytes > 126e6 else
-                         "inputs smaller than L2",
-                   "parallelism": f"dp{world} (independent shards, no collective)"},
+        "config": scan_config(cfg, world),
         "roofline": roof,
         "e2e": {"value": aggregate_rate(world, elems, e2e_ms) / 1e9, "unit": "Gelem/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -738,11 +765,7 @@ def run_step(args, rank: int, world: int, local: int):
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": dt, "data": "synthetic",
-        "config": {"workload": step_name(cfg), "batch": batch, "d_inner": dim, "d_state": cfg["N"],
-                   "global_batch": batch * world,
-                   "l2": "state larger than L2 (no flush)" if nbytes > 126e6 else
-                         "state smaller than L2",
-                   "parallelism": f"dp{world} (independent shards, no collective)"},
+        "config": step_config(cfg, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "frac_nominal": achieved / NOMINAL_HBM_GBS,
@@ -897,12 +920,7 @@ def run_bwd(args, rank: int, world: int, local: int):
         "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": dt, "data": "synthetic",
-        "config": {"workload": "backward of " + cfg["name"], "batch": cfg["batch"],
-                   "d_inner": cfg["dim"], "d_state": cfg["N"], "seq_len": cfg["L"],
-                   "global_batch": cfg["batch"] * world,
-                   "l2": "inputs larger than L2 (no flush)" if nbytes > 126e6 else
-                         "inputs smaller than L2",
-                   "parallelism": f"dp{world} (independent shards, no collective)"},
+        "config": bwd_config(cfg, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "frac_nominal": achieved / NOMINAL_HBM_GBS,
