@@ -479,6 +479,12 @@ def run_gpu(args, rank: int, world: int, local: int):
         if dist:
             tdist.barrier()
 
+    # collect garbage and start the clock sampler first, so that the warm-up
+    # keeps the GPU busy (and its clocks up) until the timed region starts
+    gc.collect()
+    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
     for _ in range(max(3, args.warmup)):
         call()
     ss.check()
@@ -486,10 +492,6 @@ def run_gpu(args, rank: int, world: int, local: int):
     torch.cuda.synchronize()
 
     # timed region: K steps, per-launch events on the launching stream
-    gc.collect()  # before the clock samples start (see gc_paused)
-    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
-    if clocks:
-        clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     barrier()
@@ -683,15 +685,17 @@ def run_step(args, rank: int, world: int, local: int):
         if dist:
             tdist.barrier()
 
+    # collect garbage and start the clock sampler first, so that the warm-up
+    # keeps the GPU busy (and its clocks up) until the timed region starts
+    gc.collect()
+    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
     for _ in range(max(3, args.warmup)):
         call()
     ss.check()
     barrier()
     torch.cuda.synchronize()
-    gc.collect()  # before the clock samples start (see gc_paused)
-    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
-    if clocks:
-        clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     barrier()
@@ -841,15 +845,17 @@ def run_bwd(args, rank: int, world: int, local: int):
         if dist:
             tdist.barrier()
 
+    # collect garbage and start the clock sampler first, so that the warm-up
+    # keeps the GPU busy (and its clocks up) until the timed region starts
+    gc.collect()
+    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
     for _ in range(max(3, args.warmup)):
         call()
     ss.check()
     barrier()
     torch.cuda.synchronize()
-    gc.collect()  # before the clock samples start (see gc_paused)
-    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
-    if clocks:
-        clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     barrier()
