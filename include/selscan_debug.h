@@ -44,6 +44,15 @@ SELSCAN_API void selscan_debug_diag_mode(int mode);
  */
 SELSCAN_API void selscan_debug_bwd_segments(int segs);
 
+/*
+ * The number of time segments per channel tile that selscan_bwd would pick
+ * for `tiles` tiles of (batch row, 32 channels), `nchunks` 8-token
+ * checkpoint chunks and `slots` warps resident at once (blocks per SM x
+ * SMs), before rounding to whole chunks per segment.  Host arithmetic only:
+ * no CUDA call.  Lets the choice be tested without a GPU.
+ */
+SELSCAN_API long long selscan_debug_bwd_plan(long long tiles, long long nchunks, long long slots);
+
 #ifdef __cplusplus
 }
 #endif

@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.selscan_debug_diag_mode.restype = None
         L.selscan_debug_bwd_segments.argtypes = [ctypes.c_int]
         L.selscan_debug_bwd_segments.restype = None
+        L.selscan_debug_bwd_plan.argtypes = [ctypes.c_longlong] * 3
+        L.selscan_debug_bwd_plan.restype = ctypes.c_longlong
         _lib = L
     return _lib
 
@@ -324,6 +326,13 @@ def debug_diag_mode(mode: int) -> None:
 def debug_bwd_segments(segs: int) -> None:
     """Test hook: time segments per channel tile in selscan_bwd (0: automatic)."""
     lib().selscan_debug_bwd_segments(int(segs))
+
+
+def debug_bwd_plan(tiles: int, nchunks: int, slots: int) -> int:
+    """Test hook: the backward's segment count for ``tiles`` channel tiles,
+    ``nchunks`` checkpoint chunks and ``slots`` resident warps (host
+    arithmetic only, no GPU needed)."""
+    return int(lib().selscan_debug_bwd_plan(int(tiles), int(nchunks), int(slots)))
 
 
 def debug_withhold_carry(unit: int) -> None:

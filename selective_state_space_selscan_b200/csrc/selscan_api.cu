@@ -134,6 +134,37 @@ cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t stream)
     return cudaMallocFromPoolAsync(p, bytes, pool, stream);
 }
 
+// Time segments per channel tile of the backward pass: `tiles` units of
+// (batch row, 32 channels), `nchunks` checkpoint chunks, `slots` warps that
+// can be resident at once.  At least 32 chunks per segment.  A wave of
+// resident warps ends with its slowest unit, so the time goes as
+// ceil(tiles * S / slots) / S: take S (at most four waves) within 2 % of the
+// lowest such cost, the smallest that gives at least 1.5 waves (shorter
+// units balance better over the SMs; more segments cost more aggregate
+// work).  With 1184 slots (148 SMs) this picks 7 segments for B4 D5120
+// L4096 (4.05 ms; 6 or 8: 4.25-4.45 ms) and 6 for B8 D1536 L2048 (1.30 ms;
+// 3: 1.37 ms).
+int64_t bwd_segments(int64_t tiles, int64_t nchunks, int64_t slots)
+{
+    if (tiles < 1 || nchunks < 1 || slots < 1)
+        return 1;
+    const int64_t max_segs = std::max<int64_t>(1, std::min<int64_t>(nchunks / 32, 4 * slots / tiles));
+    auto waves = [&](int64_t s) { return (tiles * s + slots - 1) / slots; };
+    double best = 1e30;
+    for (int64_t s = 1; s <= max_segs; ++s)
+        best = std::min(best, double(waves(s)) / double(s));
+    int64_t S = 0, S_any = 0;
+    for (int64_t s = 1; s <= max_segs && !S; ++s) {
+        if (double(waves(s)) / double(s) > 1.02 * best)
+            continue;
+        if (!S_any)
+            S_any = s;
+        if (2 * tiles * s >= 3 * slots)
+            S = s;
+    }
+    return S ? S : S_any;
+}
+
 size_t elem_size(int32_t dt) { return dt == SELSCAN_BF16 ? 2 : 4; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -486,6 +517,11 @@ selscan_status selscan_release_scratch(void)
 void selscan_debug_diag_mode(int mode) { g_dbg_diag_mode = mode; }
 
 void selscan_debug_bwd_segments(int segs) { g_dbg_bwd_segs = segs < 0 ? 0 : segs; }
+
+long long selscan_debug_bwd_plan(long long tiles, long long nchunks, long long slots)
+{
+    return bwd_segments(tiles, nchunks, slots);
+}
 
 void selscan_debug_withhold_carry(int unit) { g_dbg_skip_publish = unit; }
 
@@ -1377,14 +1413,8 @@ extern "C" selscan_status selscan_bwd(
     prm.dbias = static_cast<float *>(ddelta_bias ? ddelta_bias->data : nullptr);
     prm.dh0 = static_cast<float *>(dh0 ? dh0->data : nullptr);
 
-    // Units: (batch row, 32 channels) x time segments, one warp each, at
-    // least 32 chunks per segment.  A wave of resident warps ends with its
-    // slowest unit, so the time goes as ceil(units / slots) / S: choose S
-    // (at most four waves) within 2 % of the lowest such cost, the smallest
-    // one that gives at least 1.5 waves (shorter units balance better over
-    // the SMs; more segments cost more aggregate work).  On 148 SMs this
-    // picks 7 segments for B4 D5120 L4096 (4.05 ms; 6 or 8: 4.25-4.45 ms)
-    // and 6 for B8 D1536 L2048 (1.30 ms; 3: 1.37 ms).
+    // Units: (batch row, 32 channels) x time segments, one warp each; the
+    // segment count comes from bwd_segments.
     prm.tiles_per_batch = int((dim + 31) / 32);
     prm.tiles = int(batch) * prm.tiles_per_batch;
     {
@@ -1398,25 +1428,9 @@ extern "C" selscan_status selscan_bwd(
         if (oe != cudaSuccess || per_sm < 1)
             per_sm = 1;
         const int64_t slots = int64_t(per_sm) * di->sm_count;
-        const int64_t max_segs = std::max<int64_t>(
-            1, std::min<int64_t>(prm.nchunks / 32, 4 * slots / prm.tiles));
-        auto waves = [&](int64_t s) { return (prm.tiles * s + slots - 1) / slots; };
-        double best = 1e30;
-        for (int64_t s = 1; s <= max_segs; ++s)
-            best = std::min(best, double(waves(s)) / double(s));
-        int64_t S = 0, S_any = 0;
-        for (int64_t s = 1; s <= max_segs && !S; ++s) {
-            if (double(waves(s)) / double(s) > 1.02 * best)
-                continue;
-            if (!S_any)
-                S_any = s;
-            if (2 * prm.tiles * s >= 3 * slots)
-                S = s;
-        }
-        if (!S)
-            S = S_any;
-        if (g_dbg_bwd_segs > 0)
-            S = std::min<int64_t>(g_dbg_bwd_segs, std::max(1, prm.nchunks));
+        int64_t S = g_dbg_bwd_segs > 0
+                        ? std::min<int64_t>(g_dbg_bwd_segs, std::max(1, prm.nchunks))
+                        : bwd_segments(prm.tiles, prm.nchunks, slots);
         const int64_t seg_chunks = (prm.nchunks + S - 1) / S;
         S = (prm.nchunks + seg_chunks - 1) / seg_chunks;
         if (int64_t(prm.tiles) * S > 0x7fffffffll)

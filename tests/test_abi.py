@@ -222,3 +222,24 @@ def _bwd(**over):
 ])
 def test_bwd_rejects(over, expect):
     assert _bwd(**over) == C[expect]
+
+
+def test_backward_segment_plan():
+    """The backward's choice of time segments (host arithmetic, no GPU):
+    ceil(units / slots) / S is minimised over at most four waves, with at
+    least 32 checkpoint chunks per segment, and among near-ties the
+    smallest S that gives 1.5 waves or more is taken.  1184 slots = 8
+    resident warps on each of 148 SMs."""
+    plan = ss.debug_bwd_plan
+    assert plan(640, 512, 1184) == 7       # B4 D5120 L4096: 4480 units, 3.8 waves
+    assert plan(384, 256, 1184) == 6       # B8 D1536 L2048: 2304 units, 1.95 waves
+    assert plan(64, 16384, 1184) == 37     # B1 D2048 L131072: 2368 units, 2 waves
+    assert plan(640, 128, 1184) == 3       # L = 1024: at most 4 segments of 32 chunks
+    assert plan(2, 31, 1184) == 1          # fewer than 32 chunks: one segment
+    assert plan(5000, 512, 1184) == 1      # more than four waves of tiles already
+    assert plan(0, 10, 10) == 1 and plan(10, 0, 10) == 1 and plan(10, 10, 0) == 1
+    for tiles in (1, 7, 100, 640, 3000):
+        for nchunks in (1, 40, 512, 16384):
+            s = plan(tiles, nchunks, 1184)
+            assert 1 <= s <= max(1, nchunks // 32)
+            assert s == 1 or tiles * s <= 4 * 1184
