@@ -35,8 +35,9 @@
 // g delta u that the walk writes over the states it has used.  Lane l sums
 // states 4 (l % 4) .. 4 (l % 4) + 3 of token l / 4 and adds both results
 // with one 16-byte atomic each into one of kBwdCopies partial copies
-// (token-major, [batch][L][16]), which bwd_reduce_bc sums and transposes.  dA, dD and the bias gradient sum over batch
-// rows and tokens: registers, then atomics.
+// (token-major, [batch][L][16]), which bwd_reduce_bc sums and transposes.
+// dA, dD and the bias gradient sum over batch rows and tokens: registers,
+// then atomics.
 #pragma once
 
 #include <cuda_bf16.h>
