@@ -219,6 +219,14 @@ def _bwd(**over):
     (dict(A=_t((64, 8), ss.SELSCAN_F32), dA=_t((64, 8), ss.SELSCAN_F32),
           B=_t((2, 8, 48)), C=_t((2, 8, 48)), dB=_t((2, 8, 48), ss.SELSCAN_F32),
           dC=_t((2, 8, 48), ss.SELSCAN_F32)), "SELSCAN_ERR_UNSUPPORTED"),
+    (dict(u=_t((2, 64, 48), dtype=7)), "SELSCAN_ERR_DTYPE"),
+    (dict(dy=_t((2, 64, 48), data=FAKE + 8)), "SELSCAN_ERR_ALIGN"),
+    (dict(du=_t((2, 64, 48), strides=(64 * 48, 44, 1))), "SELSCAN_ERR_ALIGN"),
+    (dict(dB=_t((2, 16, 48), ss.SELSCAN_F32, strides=(16 * 48, 1, 16))), "SELSCAN_ERR_STRIDE"),
+    (dict(dC=None), "SELSCAN_ERR_NULL"),
+    (dict(h0=_t((2, 64, 16))), "SELSCAN_ERR_DTYPE"),          # bf16 initial state
+    (dict(dlast=_t((2, 63, 16), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(B=_t((2, 2, 16, 48))), "SELSCAN_ERR_UNSUPPORTED"),  # groups of B / C
 ])
 def test_bwd_rejects(over, expect):
     assert _bwd(**over) == C[expect]
