@@ -129,10 +129,15 @@ def release_scratch() -> None:
 
 
 def describe(t, dtype_code=None) -> SelscanTensor | None:
-    """selscan_tensor for a torch tensor (None stays None -> NULL)."""
+    """selscan_tensor for a CUDA torch tensor (None stays None -> NULL).
+    Host tensors are refused: the C ABI takes device pointers only, and
+    there is no CPU implementation to fall back to."""
     if t is None:
         return None
     import torch
+    if not t.is_cuda:
+        raise ValueError(f"libselscan takes CUDA tensors only (got one on {t.device}); "
+                         "there is no CPU implementation")
     d = SelscanTensor()
     d.data = t.data_ptr()
     if dtype_code is None:
