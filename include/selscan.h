@@ -284,7 +284,8 @@ SELSCAN_API selscan_status selscan_step_scalarA(selscan_tensor *state, const sel
  *   d(bias) = sum d(Delta);  dh0 = g after the first token.
  *
  * Forward inputs exactly as selscan_fwd_h0 (u, delta, delta_bias, softplus,
- * A, B, C, D, z, h0; time stride 1, element-aligned rows; N = 16, one group).
+ * A, B, C, D, z, h0; time stride 1 and 16-byte aligned rows, as there; N =
+ * 16, one group of B / C).
  *   dy         (batch, D, L)  same dtype as u: gradient of y
  *   dlast      (batch, D, N)  F32, contiguous; may be NULL (zero)
  * Outputs (all overwritten):
@@ -296,7 +297,8 @@ SELSCAN_API selscan_status selscan_step_scalarA(selscan_tensor *state, const sel
  *   dh0        (batch, D, N)  F32; may be NULL (not computed)
  * The expanded states are recomputed, never stored: a forward pass keeps h
  * every 8 tokens in stream-ordered scratch (batch * D * ceil(L/8) * 64
- * bytes), then the chunks are walked backwards.  Sums over channels and
+ * bytes, plus 2 * 8 * batch * N * L * 4 bytes of dB / dC partial sums and
+ * small segment aggregates), then the chunks are walked backwards.  Sums over channels and
  * batch rows use fp32 atomics (dB and dC into 8 partial copies that a
  * last kernel adds), so the last bits of dA, dB, dC, dD and ddelta_bias
  * depend on the order of the additions.
