@@ -270,8 +270,8 @@ int g_dbg_skip_publish = -1;  // test hook, see selscan_debug_withhold_carry
 
 // ----------------------------------------------------- diagonal-A launch
 // Kernel variants share one launcher: KIND 0 = portable kernel (fp32 and
-// bf16, one lane pair per channel); KIND 1 = fast bf16 kernel (one lane per
-// channel, lane pairs share two channels' states).
+// bf16, one lane pair per channel); KIND 1 = fast bf16 kernel (its own
+// threads-per-channel constant, kFastLanesPerChannel).
 template <int KIND, typename T, int CH, int STAGES, bool GATE, bool SOFTPLUS>
 struct DiagVariant;
 
@@ -287,8 +287,8 @@ struct DiagVariant<0, T, CH, STAGES, GATE, SOFTPLUS> {
 template <int CH, int STAGES, bool GATE, bool SOFTPLUS>
 struct DiagVariant<1, __nv_bfloat16, CH, STAGES, GATE, SOFTPLUS> {
     static constexpr int kChunk = 64;
-    static constexpr int kThreads = 2 * CH + 32;
-    static constexpr int kConsWarps = 2 * CH / 32;
+    static constexpr int kThreads = kFastLanesPerChannel * CH + 32;
+    static constexpr int kConsWarps = kFastLanesPerChannel * CH / 32;
     static constexpr int kSmem = DiagFastLayout<CH, STAGES, GATE>::kAlloc;
     static constexpr auto kernel() { return scan_diag_bf16_kernel<CH, STAGES, GATE, SOFTPLUS>; }
     // two-pass form: MODE 1 reads no z, MODE 2 is the full output pass
@@ -378,6 +378,9 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
     if (units > 0x7fffffffll)
         return SELSCAN_ERR_UNSUPPORTED;
     prm.total_units = int(units);
+    prm.y = y->data;
+    prm.y_bs = y->stride[0];
+    prm.y_rs = y->stride[1];
 
     // Few tiles and several segments: a chain of carries would leave most
     // SMs waiting, so use the two-pass form (aggregates, then output).
@@ -910,6 +913,9 @@ selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor
     prm.seg_len = int(seg_chunks * TC);
     prm.num_segs = int(S);
     prm.total_units = int(units);
+    prm.y = y->data;
+    prm.y_bs = y->stride[0];
+    prm.y_rs = y->stride[1];
     // the previous call's ticket and flags must not leak into this one
     if (cudaMemsetAsync(scratch, 0, head + flag_bytes, stream) != cudaSuccess)
         return SELSCAN_ERR_CUDA;
@@ -1341,8 +1347,11 @@ extern "C" selscan_status selscan_bwd(
                    ? cudaSuccess
                    : cudaMemsetAsync(t->data, 0, size_t(numel(t)) * 4, stream);
     };
-    if (batch == 0)
-        return SELSCAN_OK;
+    if (batch == 0)  // dA, dD and d bias sum over no batch row: zero, not left as they were
+        return zero(dA) == cudaSuccess && zero(dD) == cudaSuccess &&
+                       zero(ddelta_bias) == cudaSuccess
+                   ? SELSCAN_OK
+                   : SELSCAN_ERR_CUDA;
     if (dim == 0)  // dB and dC sum over no channel
         return zero(dB) == cudaSuccess && zero(dC) == cudaSuccess ? SELSCAN_OK
                                                                   : SELSCAN_ERR_CUDA;

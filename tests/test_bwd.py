@@ -211,3 +211,31 @@ def test_results_unchanged_after_release_scratch():
     torch.cuda.synchronize()
     ss.release_scratch()
     compare(run(inp, dy, "f32"), want, "f32")
+
+
+def test_empty_batch_zeroes_parameter_gradients():
+    """batch = 0 with channels present: dA, dD and d bias are sums over no
+    batch row, so the call must write zeros into them, whatever the caller's
+    buffers held (here NaN), through the C ABI."""
+    import torch
+    import selective_state_space_selscan_b200 as ss
+    dev = "cuda"
+    dim, N, L = 32, 16, 64
+    u = torch.empty(0, dim, L, dtype=torch.bfloat16, device=dev)
+    BC = torch.empty(0, N, L, dtype=torch.bfloat16, device=dev)
+    A = -torch.arange(1, N + 1, dtype=torch.float32, device=dev).repeat(dim, 1)
+    Dv = torch.ones(dim, device=dev)
+    bias = torch.zeros(dim, device=dev)
+    nan = lambda *s: torch.full(s, float("nan"), device=dev)
+    dA, dD, dbias = nan(dim, N), nan(dim), nan(dim)
+    du = torch.empty_like(u)
+    dd = torch.empty_like(u)
+    dB = torch.empty(0, N, L, device=dev)
+    dC = torch.empty(0, N, L, device=dev)
+    r = lambda t: ss._ref(ss.describe(t))
+    rc = ss.lib().selscan_bwd(r(u), r(u), r(bias), 1, r(A), r(BC), r(BC), r(Dv), None, None,
+                              r(u), None, r(du), r(dd), r(dA), r(dB), r(dC), r(dD), None,
+                              r(dbias), None, ss._stream_handle(None))
+    assert rc == 0
+    ss.check()
+    assert torch.all(dA == 0) and torch.all(dD == 0) and torch.all(dbias == 0)
