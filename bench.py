@@ -49,9 +49,10 @@ NCU_TRAFFIC = {
     3: ("scan_diag_bf16_kernel two-pass v1", 2679.6e6),
     4: ("ssd_scalarA_kernel v5", 107.9e6),
 }
-KERNEL_TAG = {2: "scan_diag_bf16_kernel pairs v4", 1: "scan_diag_bf16_kernel pairs v4",
-              3: "scan_diag_bf16_kernel two-pass v1", 0: "scan_diag_kernel fp32 v2",
-              4: "ssd_scalarA_kernel v5"}
+KERNEL_TAG = {2: "scan_diag_bf16_kernel lane-per-channel v5",
+              1: "scan_diag_bf16_kernel lane-per-channel v5",
+              3: "scan_diag_bf16_kernel lane-per-channel two-pass v5",
+              0: "scan_diag_kernel fp32 v3", 4: "ssd_scalarA_kernel v5"}
 HBM_FALLBACK_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # the HGX/DGX nominal figure, reported beside the measured peak
 

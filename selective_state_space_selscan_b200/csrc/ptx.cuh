@@ -56,19 +56,52 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase
+// completes or `hint_ns` nanoseconds pass, instead of returning at once: a
+// waiting warp then issues no instructions (a polling loop would take issue
+// slots from the warps that share its scheduler).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of `bar` to complete, giving up after
 // `timeout_ns` nanoseconds (%globaltimer).  Returns false on time-out.  The
-// timer is only read once the barrier has been polled many times, so the
-// fast path is a bare try_wait.
+// fast path is a bare try_wait; after that the thread sleeps in the
+// hardware between checks (at most 20 us at a time) and reads the timer
+// after each wake-up.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           uint64_t timeout_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t start = global_timer_ns();
-    uint32_t spins = 0;
+    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
+        if (global_timer_ns() - start > timeout_ns)
+            return false;
+    }
+    return true;
+}
+
+// Wait for a slow event (the producer waiting for a stage to be released):
+// poll with a short sleep between tries, so that the waiting warp takes
+// almost no issue slots from the warps that share its scheduler.  Returns
+// false after `timeout_ns`.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t *bar, uint32_t parity,
+                                                  uint64_t timeout_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t start = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if ((++spins & 255u) == 0u && global_timer_ns() - start > timeout_ns)
+        __nanosleep(200);
+        if (global_timer_ns() - start > timeout_ns)
             return false;
     }
     return true;
@@ -210,6 +243,14 @@ __device__ __forceinline__ float lg2_approx(float x)
 {
     float y;
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// tanh on the special-function unit (maximum absolute error about 2^-11)
+__device__ __forceinline__ float tanh_approx(float x)
+{
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 

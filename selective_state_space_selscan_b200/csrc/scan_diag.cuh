@@ -55,6 +55,8 @@ struct DiagParams {
     float *agg;           // two-pass form: [units][CH][parity][8] segment end states
     float *agg_sd;        // two-pass form: [units][CH] sums of step sizes
     float *last_state;    // (batch, dim, 16) or null
+    void *y;              // output (batch, dim, L), element strides y_bs, y_rs (fast bf16 kernel)
+    long long y_bs, y_rs;
     int softplus;
     unsigned int *ticket;  // zeroed before launch
     unsigned int *flags;   // [total_units][consumer warps], zeroed
@@ -130,6 +132,16 @@ __device__ __forceinline__ float softplus_fast(float x)
 __device__ __forceinline__ float softplus_exact(float x)
 {
     return x > 20.f ? x + log1pf(expf(-x)) : log1pf(expf(x));
+}
+
+// exp(x) for the fp32 decay factors.  For small |x| (x is delta * A, often
+// -1e-3) the factor sits just below 1, and a long product of them is only as
+// good as the rounding of each: 1 + expm1f(x) is the correctly rounded value
+// up to one unbiased rounding, so products over thousands of tokens do not
+// drift.  Larger |x| take expf.
+__device__ __forceinline__ float exp_decay(float x)
+{
+    return fabsf(x) < 0.5f ? 1.f + expm1f(x) : expf(x);
 }
 
 __device__ __forceinline__ float silu_fast(float v)
@@ -231,7 +243,7 @@ __device__ __forceinline__ void diag_chunk_compute(
             } else {
 #pragma unroll
                 for (int n = 0; n < 8; ++n)
-                    dA[n] = kFast ? ex2_approx(q_all[i] * a[n]) : expf(q_all[i] * a[n]);
+                    dA[n] = kFast ? ex2_approx(q_all[i] * a[n]) : exp_decay(q_all[i] * a[n]);
             }
             float acc = 0.f;
 #pragma unroll

@@ -1,30 +1,42 @@
 // scan_diag_bf16.cuh -- fast diagonal-A selective scan for bf16 inputs
 // (fp32 state), sm_100a.
 //
-// Same contract and work decomposition as scan_diag.cuh (persistent grid,
-// atomic ticket in segment-major order, one producer warp streaming chunks
-// with bulk tensor copies, carries linked by gpu-scope release/acquire
-// flags), with an inner loop laid out for the B200 SM:
+// What it computes (per batch row b, channel d, token t; "03 -- Modelos de
+// espacio de estados", sections "El mecanismo selectivo de Mamba",
+// "Discretizacion", "Parallel scan"; "P20 -- Mamba", section 5):
+//   delta_t = softplus(Delta + bias)     h_t = exp(delta_t A) h_{t-1} + delta_t B_t u_t
+//   y_t     = (C_t . h_t + D u_t) * silu(z_t)
 //
-//  * Two consumer lanes per channel (a lane pair), 128 channels per CTA, so
-//    that each scheduler runs two consumer warps.  Lane p keeps the states of
-//    parity p (n = p, p+2, ..., p+14) in registers and prepares the per-token
-//    values (softplus, w = delta*u, the decay base, 1/w) of half of each
-//    8-token block; the pair swaps them with warp shuffles, runs the 8 steps,
-//    and reduce-scatters the two partial outputs so each lane finishes four
-//    tokens (D skip, gate, bf16 store).  B and C of a chunk are staged once
-//    per CTA as fp32, token-major, parity-split, so every lane reads its 8 B
-//    and 8 C values of a token with four 16-byte broadcast loads.
-//  * The state is kept rescaled, g = h / w with w = delta * u, so that the
-//    input term needs no multiply:  g_t = (w_{t-1}/w_t) exp(delta_t A) g_{t-1}
-//    + B_t and y_t = w_t (C_t . g_t).  |w| is kept >= 2^-64 so that the
-//    rescaling stays finite (a zero input then contributes 2^-64 * B, far
-//    below fp32 resolution of any non-trivial state).
+// Same contract and work decomposition as scan_diag.cuh (persistent grid,
+// atomic ticket in segment-major order, one producer warp streaming 64-token
+// chunks with bulk tensor copies, segments linked by gpu-scope
+// release/acquire flags), with an inner loop laid out for the B200 SM:
+//
+//  * One consumer thread per channel, all 16 states in registers (eight
+//    packed f32x2 pairs): no exchange between lanes at all.  128 channels per
+//    CTA, so each of the four schedulers runs one consumer warp; the chains
+//    of a channel are sequential in time, so what matters is how fast a
+//    single warp can issue.
+//  * The state is kept rescaled, g = h / s with s = delta * u * log2(e), so
+//    that the input term needs no multiply per state:
+//       g_t = (s_{t-1}/s_t) exp(delta_t A) g_{t-1} + ln2 * B_t,
+//       y_t = s_t (C_t . g_t) + D u_t.
+//    B is staged pre-multiplied by ln2.  When some |s_t| of an 8-token block
+//    is below 2^-64 (u = 0 padding, a zero step size, ...) the whole warp
+//    takes the exact form of that block instead: s_t is clamped to +-2^-64
+//    and the input term is scaled by s_t / clamp(s_t), which is 0 for a zero
+//    input, so no tiny or zero input is rounded up.
+//  * Per-token work that does not depend on the state index (softplus in
+//    log2 units, the decay base, 1/s, the D skip, the gate) runs on pairs of
+//    tokens with packed f32x2 instructions, and is software-pipelined: the
+//    next 8-token block is prepared and the previous one finished in the same
+//    basic block as the current block's eight steps.
 //  * For S4D-real A (A[d,n] = (n+1) A[d,0], checked per channel at run time)
-//    the decays are powers r^(n+1) of r = exp(delta A[d,0]); lane p needs
-//    the odd (p=0) or even (p=1) powers, i.e. base * s^j with s = r^2,
-//    computed with packed f32x2 multiplies.  Other A use one ex2 per state.
-//  * Packed f32x2 FMAs (sm_100) update two states per instruction.
+//    the decays are powers r^(n+1) of r = exp(delta A[d,0]): one ex2 per token
+//    and seven packed multiplies.  Other A take one ex2 per state.
+//  * B and C of a chunk are staged once per CTA as fp32, token-major
+//    ([t][B 16 | C 16]), so a thread reads a token's 32 values with eight
+//    16-byte broadcast loads.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -37,17 +49,20 @@
 
 namespace selscan {
 
-constexpr float kWMin = 5.421010862427522e-20f;  // 2^-64
+constexpr float kTau = 5.421010862427522e-20f;  // 2^-64: smallest |s| of the fast form
+constexpr float kSmallE = 0.015625f;            // below 2^-6 the log1p series is used
+
+constexpr int kFastLanesPerChannel = 1;  // consumer threads per channel
 
 template <int CH, int STAGES, bool GATE>
 struct DiagFastLayout {
     static constexpr int kChunk = 64;                    // tokens per stage
-    static constexpr int kTile = CH * 128;               // bf16 [CH][64]
+    static constexpr int kTile = CH * 128;               // bf16 [CH][64], 128-byte swizzled rows
     static constexpr int kBCTile = kDiagN * 128;         // bf16 [16][64]
     static constexpr int kStage = (2 + (GATE ? 1 : 0)) * kTile + 2 * kBCTile;
     static constexpr int kStagesOff = 0;
-    static constexpr int kBCPOff = STAGES * kStage;      // fp32 B/C [2][64][128 B]
-    static constexpr int kYOff = kBCPOff + 2 * kChunk * 128;
+    static constexpr int kBCFOff = STAGES * kStage;      // fp32 [2][64][32]
+    static constexpr int kYOff = kBCFOff + 2 * kChunk * 32 * 4;
     static constexpr int kBarOff = kYOff + 2 * kTile;
     static constexpr int kInfoOff = kBarOff + 2 * STAGES * 8;
     static constexpr int kAbortOff = kInfoOff + STAGES * 16;
@@ -55,29 +70,160 @@ struct DiagFastLayout {
     static constexpr int kAlloc = kBytes + 1024;
 };
 
-template <bool POW>
-__device__ __forceinline__ void decay_pairs(uint64_t (&V)[4], float r, float c, int p,
-                                            const uint64_t (&apair)[4])
+// Per-token values of one 8-token block, as pairs (tokens 2k, 2k+1).
+struct PrepBlock {
+    uint64_t R[4];   // decay base r = exp(delta A0) (S4D-real) or delta*log2e (general A)
+    uint64_t W[4];   // s = delta * log2e * u
+    uint64_t RS[4];  // 1 / s (fast form only)
+    uint64_t SD;     // sum of the block's step sizes, log2 units (aggregate pass)
+    bool tiny;       // some |s| < 2^-64 in the block
+};
+
+template <bool SOFTPLUS, bool POW, int MODE>
+__device__ __forceinline__ void prep8(PrepBlock &pb, const uint8_t *u_row, const uint8_t *dl_row,
+                                      int off, int tfirst, int L, uint64_t BL2E2, float a0)
 {
-    if (POW) {
-        // powers r^(n+1) for n = p, p+2, ..., p+14 : base * s^j, s = r^2
-        const float s = r * r;
-        const float base = c * (p ? s : r);
-        V[0] = pk2(base, base * s);
-        const float s2 = s * s;
-        const uint64_t S2 = pk2(s2, s2);
-        V[1] = mul2(V[0], S2);
-        V[2] = mul2(V[1], S2);
-        V[3] = mul2(V[2], S2);
-    } else {
-        // general A: r holds delta; apair holds A*log2(e) of this lane's states
-        const uint64_t RR = pk2(r, r), CC = pk2(c, c);
+    const uint4 uq = *reinterpret_cast<const uint4 *>(u_row + off);
+    const uint4 dq = *reinterpret_cast<const uint4 *>(dl_row + off);
+    const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+    const uint32_t dw[4] = {dq.x, dq.y, dq.z, dq.w};
+    const uint64_t L2E2 = pk2(kLog2e, kLog2e);
+    float mn = 3.0e38f;
+    uint64_t SD = pk2(0.f, 0.f);
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const uint64_t X = mul2(RR, apair[jj]);
-            V[jj] = mul2(CC, pk2(ex2_approx(lo2(X)), ex2_approx(hi2(X))));
+    for (int k = 0; k < 4; ++k) {
+        const uint64_t U = bf2_to_f2(uw[k]);
+        uint64_t D2 = fma2(bf2_to_f2(dw[k]), L2E2, BL2E2);  // (Delta + bias) log2e
+        if (SOFTPLUS) {
+            // delta log2e = log2(1 + 2^x): lg2 of 1 + e, or the log1p series
+            // (in log2 units) when e < 2^-6; x itself beyond 2^64.
+            const float xa = lo2(D2), xb = hi2(D2);
+            const uint64_t E = pk2(ex2_approx(fminf(xa, 64.f)), ex2_approx(fminf(xb, 64.f)));
+            const uint64_t T = add2(E, pk2(1.f, 1.f));
+            uint64_t Q = fma2(E, pk2(kLog2e / 3.f, kLog2e / 3.f),
+                              pk2(-0.5f * kLog2e, -0.5f * kLog2e));
+            Q = fma2(E, Q, L2E2);
+            Q = mul2(E, Q);
+            float da = lo2(E) < kSmallE ? lo2(Q) : lg2_approx(lo2(T));
+            float db = hi2(E) < kSmallE ? hi2(Q) : lg2_approx(hi2(T));
+            D2 = pk2(fmaxf(da, xa), fmaxf(db, xb));
+        }
+        if (tfirst + 8 > L) {
+            // tokens past the end of the sequence: identity steps
+            const int t = tfirst + 2 * k;
+            D2 = pk2(t < L ? lo2(D2) : 0.f, t + 1 < L ? hi2(D2) : 0.f);
+        }
+        if (MODE == 1)
+            SD = add2(SD, D2);
+        if (POW) {
+            const uint64_t X = mul2(D2, pk2(a0, a0));
+            pb.R[k] = pk2(ex2_approx(lo2(X)), ex2_approx(hi2(X)));
+        } else {
+            pb.R[k] = D2;
+        }
+        const uint64_t W = mul2(D2, U);
+        pb.W[k] = W;
+        mn = fminf(mn, fminf(fabsf(lo2(W)), fabsf(hi2(W))));
+        pb.RS[k] = pk2(rcp_approx(lo2(W)), rcp_approx(hi2(W)));
+    }
+    pb.SD = SD;
+    pb.tiny = mn < kTau;
+}
+
+// Eight recurrence steps of one block.  EXACT: the clamped form for blocks
+// with a tiny |s|.  OUT: also form the outputs (not in the aggregate pass).
+template <bool EXACT, bool POW, bool OUT>
+__device__ __forceinline__ void steps8(uint64_t (&g)[8], const PrepBlock &pb, float &s_prev,
+                                       const float *bct, float (&yp)[8], float (&se)[8],
+                                       const uint64_t (&apair)[8])
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int k = i >> 1;
+        const bool hi = (i & 1) != 0;
+        const float w = hi ? hi2(pb.W[k]) : lo2(pb.W[k]);
+        float s, rs;
+        if (EXACT) {
+            s = copysignf(fmaxf(fabsf(w), kTau), w);
+            rs = rcp_approx(s);
+        } else {
+            s = w;
+            rs = hi ? hi2(pb.RS[k]) : lo2(pb.RS[k]);
+        }
+        const float rho = s_prev * rs;
+        s_prev = s;
+        se[i] = s;
+        const float rr = hi ? hi2(pb.R[k]) : lo2(pb.R[k]);
+        uint64_t V[8];
+        if (POW) {
+            const float r2 = rr * rr;
+            V[0] = pk2(rho * rr, rho * r2);
+            const uint64_t SS = pk2(r2, r2);
+#pragma unroll
+            for (int kk = 1; kk < 8; ++kk)
+                V[kk] = mul2(V[kk - 1], SS);
+        } else {
+            const uint64_t DD = pk2(rr, rr), RR = pk2(rho, rho);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t X = mul2(DD, apair[kk]);
+                V[kk] = mul2(RR, pk2(ex2_approx(lo2(X)), ex2_approx(hi2(X))));
+            }
+        }
+        const ulonglong2 *q = reinterpret_cast<const ulonglong2 *>(bct + i * 32);
+        const ulonglong2 b01 = q[0], b23 = q[1], b45 = q[2], b67 = q[3];
+        uint64_t Bp[8] = {b01.x, b01.y, b23.x, b23.y, b45.x, b45.y, b67.x, b67.y};
+        if (EXACT) {
+            const float kap = w * rs;
+            const uint64_t KK = pk2(kap, kap);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                Bp[kk] = mul2(KK, Bp[kk]);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            g[kk] = fma2(V[kk], g[kk], Bp[kk]);
+        if (OUT) {
+            const ulonglong2 c01 = q[4], c23 = q[5], c45 = q[6], c67 = q[7];
+            uint64_t acc = mul2(c01.x, g[0]);
+            acc = fma2(c01.y, g[1], acc);
+            acc = fma2(c23.x, g[2], acc);
+            acc = fma2(c23.y, g[3], acc);
+            acc = fma2(c45.x, g[4], acc);
+            acc = fma2(c45.y, g[5], acc);
+            acc = fma2(c67.x, g[6], acc);
+            acc = fma2(c67.y, g[7], acc);
+            yp[i] = lo2(acc) + hi2(acc);
         }
     }
+}
+
+// Outputs of one block: y = s (C.g) + D u, times silu(z); bf16 into the y tile.
+template <bool GATE>
+__device__ __forceinline__ void finish8(const float (&yp)[8], const float (&se)[8],
+                                        const uint8_t *u_row, const uint8_t *z_row,
+                                        uint8_t *y_row, int off, float dsk)
+{
+    const uint4 uq = *reinterpret_cast<const uint4 *>(u_row + off);
+    uint4 zq = make_uint4(0, 0, 0, 0);
+    if (GATE)
+        zq = *reinterpret_cast<const uint4 *>(z_row + off);
+    const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+    const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint64_t DU = mul2(bf2_to_f2(uw[k]), pk2(dsk, dsk));
+        uint64_t Y = fma2(pk2(se[2 * k], se[2 * k + 1]), pk2(yp[2 * k], yp[2 * k + 1]), DU);
+        if (GATE) {
+            // silu(z) = z sigmoid(z) = (z/2) (1 + tanh(z/2))
+            const uint64_t HZ = mul2(bf2_to_f2(zw[k]), pk2(0.5f, 0.5f));
+            const uint64_t TH = pk2(tanh_approx(lo2(HZ)), tanh_approx(hi2(HZ)));
+            Y = mul2(Y, fma2(HZ, TH, HZ));
+        }
+        o[k] = pack2_bf16(lo2(Y), hi2(Y));
+    }
+    *reinterpret_cast<uint4 *>(y_row + off) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // MODE 0: one pass, segments chained through published carries.
@@ -87,7 +233,7 @@ __device__ __forceinline__ void decay_pairs(uint64_t (&V)[4], float r, float c, 
 // MODE 2: output pass of the two-pass form: every segment starts from the
 //         state folded from the aggregates of the segments before it.
 template <int CH, int STAGES, bool GATE, bool SOFTPLUS, int MODE = 0>
-__global__ void __launch_bounds__(2 * CH + 32, 1)
+__global__ void __launch_bounds__(CH + 32, 1)
 scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                       const __grid_constant__ CUtensorMap tm_delta,
                       const __grid_constant__ CUtensorMap tm_z,
@@ -98,17 +244,18 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
 {
     using Lay = DiagFastLayout<CH, STAGES, GATE>;
     constexpr int TC = Lay::kChunk;
-    constexpr int CONS = 2 * CH;  // two consumer lanes per channel
+    constexpr int CONS = CH;  // one consumer thread per channel
     constexpr int CW = CONS / 32;
     constexpr int TILE = Lay::kTile;
-    static_assert(CONS % 32 == 0, "consumer threads must fill warps");
+    constexpr bool OUT = MODE != 1;
+    static_assert(CONS % 32 == 0 && CW >= 1 && CW <= 8, "consumer threads must fill warps");
 
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, offset from the shared array itself so that
     // every pointer derived from it stays in the shared address space
     uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem + Lay::kStagesOff;
-    float *bcp = reinterpret_cast<float *>(smem + Lay::kBCPOff);
+    float *bcf = reinterpret_cast<float *>(smem + Lay::kBCFOff);
     uint8_t *ytile = smem + Lay::kYOff;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Lay::kBarOff);
     uint64_t *empty = full + STAGES;
@@ -137,7 +284,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             if (GATE)
                 prefetch_tmap(&tm_z);
             prefetch_tmap(&tm_B);
-            if (MODE != 1)
+            if (OUT)
                 prefetch_tmap(&tm_C);
             int s = 0;
             uint32_t ph = 0;
@@ -153,7 +300,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                 const int te = min(p.L, tb + p.seg_len);
                 const int nch = (te - tb + TC - 1) / TC;
                 for (int c = 0; c < nch; ++c) {
-                    if (!mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns)) {
+                    if (!mbar_wait_backoff(&empty[s], ph ^ 1u, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -163,15 +310,14 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                                             (c == nch - 1 ? kInfoLast : 0),
                                         0);
                     uint8_t *st = stages + s * Lay::kStage;
-                    mbar_arrive_expect_tx(&full[s], MODE == 1 ? 2 * TILE + Lay::kBCTile
-                                                              : Lay::kStage);
+                    mbar_arrive_expect_tx(&full[s], OUT ? Lay::kStage : 2 * TILE + Lay::kBCTile);
                     tma_load_3d(st, &tm_u, &full[s], t0, d0, b);
                     tma_load_3d(st + TILE, &tm_delta, &full[s], t0, d0, b);
-                    if (GATE && MODE != 1)
+                    if (GATE && OUT)
                         tma_load_3d(st + 2 * TILE, &tm_z, &full[s], t0, d0, b);
                     uint8_t *bct = st + (GATE ? 3 : 2) * TILE;
                     tma_load_3d(bct, &tm_B, &full[s], t0, 0, b);
-                    if (MODE != 1)
+                    if (OUT)
                         tma_load_3d(bct + Lay::kBCTile, &tm_C, &full[s], t0, 0, b);
                     if (++s == STAGES) {
                         s = 0;
@@ -179,7 +325,7 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                     }
                 }
             }
-            if (ok && mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns)) {
+            if (ok && mbar_wait_backoff(&empty[s], ph ^ 1u, p.timeout_ns)) {
                 info[s] = make_int4(-1, 0, kInfoEnd, 0);
                 mbar_arrive(&full[s]);
             } else {
@@ -192,17 +338,18 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
     }
 
     // ---------------------------------------------------------- consumers
-    const int ch = tid >> 1;     // channel within the tile
-    const int pp = tid & 1;      // state parity held by this lane; token half it prepares
+    const int ch = tid;          // channel within the tile
     const int swz = ch & 7;      // 128-byte swizzle phase of this row
-    uint64_t g[4];               // rescaled states n = pp, pp+2, ..., pp+14 (pairs)
+    uint64_t g[8];               // rescaled states (2k, 2k+1)
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj)
-        g[jj] = pk2(0.f, 0.f);
-    uint64_t apair[4];           // A*log2e of this lane's states, paired (general path)
-    float a0 = 0.f, bias = 0.f, dsk = 0.f, wprev = 1.f;
-    float sdel = 0.f;            // this lane's sum of step sizes in the segment (MODE 1)
+    for (int k = 0; k < 8; ++k)
+        g[k] = pk2(0.f, 0.f);
+    uint64_t apair[8];           // A of this channel, paired (general path)
+    float a0 = 0.f, dsk = 0.f, s_prev = 1.f;
+    uint64_t BL2E2 = 0;          // bias * log2e, paired
+    uint64_t SD = 0;             // sum of step sizes (log2 units) in the segment (MODE 1)
     bool pow_path = true;
+    bool live = false;           // this thread's channel exists (ragged last tile)
     int unit = -1, k = 0, b = 0, d0 = 0, d = 0;
     int prev_t0 = 0, prev_d0 = 0, prev_b = 0;
     int s = 0, it = 0;
@@ -224,50 +371,58 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             b = gg / p.tiles_per_batch;
             d0 = (gg - b * p.tiles_per_batch) * CH;
             d = d0 + ch;
-            const bool live = d < p.dim;
+            live = d < p.dim;
+            // A, h0 and last_state are caller buffers with 4-byte alignment:
+            // scalar accesses only
             const float *arow = p.A + size_t(live ? d : 0) * kDiagN;
-            const float A0 = arow[0];
+            float av[16];
+#pragma unroll
+            for (int n = 0; n < 16; ++n)
+                av[n] = __ldg(arow + n);
             bool ok = true;
-            float al[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int n = 2 * j + pp;  // this lane's states
-                const float an = arow[n];
-                ok = ok && (an == float(n + 1) * A0);
-                al[j] = an * kLog2e;
-            }
+            for (int n = 0; n < 16; ++n)
+                ok = ok && (av[n] == float(n + 1) * av[0]);
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                apair[jj] = pk2(al[2 * jj], al[2 * jj + 1]);
-            a0 = A0 * kLog2e;
+            for (int kk = 0; kk < 8; ++kk)
+                apair[kk] = pk2(av[2 * kk], av[2 * kk + 1]);
+            a0 = av[0];
             pow_path = __all_sync(0xffffffffu, ok);
-            bias = (p.delta_bias && live) ? p.delta_bias[d] : 0.f;
+            const float bias = (p.delta_bias && live) ? p.delta_bias[d] : 0.f;
+            BL2E2 = pk2(bias * kLog2e, bias * kLog2e);
             dsk = (p.Dskip && live) ? p.Dskip[d] : 0.f;
-            wprev = 1.f;  // g starts as h_in (w_{-1} := 1)
-            sdel = 0.f;
-            float hv[8];
+            s_prev = 1.f;  // g starts as h_in (s_{-1} := 1)
+            SD = 0;
+            float hv[16];
+#pragma unroll
+            for (int n = 0; n < 16; ++n)
+                hv[n] = 0.f;
             if (MODE == 1) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    hv[j] = 0.f;
+                // from zero
             } else if (k == 0 || MODE == 2) {
+                if (p.h0 && live) {
+                    const float *src = p.h0 + (size_t(b) * p.dim + d) * kDiagN;
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    hv[j] = (p.h0 && live) ? p.h0[(size_t(b) * p.dim + d) * kDiagN + 2 * j + pp]
-                                           : 0.f;
+                    for (int n = 0; n < 16; ++n)
+                        hv[n] = src[n];
+                }
                 if (MODE == 2) {
                     // h_in = fold over the earlier segments j of this tile:
-                    // h = exp(A * sum(delta_j)) h + E_j
+                    // h = exp(A sum(delta_j)) h + E_j
                     for (int jseg = 0; jseg < k; ++jseg) {
                         const size_t uj = size_t(jseg) * G + gg;
-                        const float sd = __ldcg(p.agg_sd + uj * CH + ch);
+                        const float sd2 = __ldcg(p.agg_sd + uj * CH + ch);
                         const float4 *e = reinterpret_cast<const float4 *>(
-                            p.agg + (uj * CH + ch) * kDiagN + pp * 8);
-                        const float4 e0 = __ldcg(e), e1 = __ldcg(e + 1);
-                        const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                            p.agg + (uj * CH + ch) * kDiagN);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            hv[j] = fmaf(ex2_approx(al[j] * sd), hv[j], ev[j]);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 ev = __ldcg(e + q4);
+                            const float evv[4] = {ev.x, ev.y, ev.z, ev.w};
+#pragma unroll
+                            for (int m = 0; m < 4; ++m)
+                                hv[4 * q4 + m] = fmaf(ex2_approx(av[4 * q4 + m] * sd2),
+                                                      hv[4 * q4 + m], evv[m]);
+                        }
                     }
                 }
             } else {
@@ -280,53 +435,55 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                 if (!got) {
                     if (lane == 0)
                         atomicOr(p.err, kErrTimeoutCarry);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        hv[j] = 0.f;
                 } else {
                     (void)ld_acquire_gpu(flag);
-                    // carry layout: [unit][channel][parity][8]
-                    const float4 *so = reinterpret_cast<const float4 *>(
-                        p.carry + (size_t(prev) * CH + ch) * kDiagN + pp * 8);
-                    const float4 o0 = __ldcg(so), o1 = __ldcg(so + 1);
-                    hv[0] = o0.x; hv[1] = o0.y; hv[2] = o0.z; hv[3] = o0.w;
-                    hv[4] = o1.x; hv[5] = o1.y; hv[6] = o1.z; hv[7] = o1.w;
+                    const float4 *src = reinterpret_cast<const float4 *>(
+                        p.carry + (size_t(prev) * CH + ch) * kDiagN);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 v = __ldcg(src + q4);
+                        hv[4 * q4] = v.x; hv[4 * q4 + 1] = v.y; hv[4 * q4 + 2] = v.z; hv[4 * q4 + 3] = v.w;
+                    }
                 }
             }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                g[jj] = pk2(hv[2 * jj], hv[2 * jj + 1]);
+            for (int kk = 0; kk < 8; ++kk)
+                g[kk] = pk2(hv[2 * kk], hv[2 * kk + 1]);
         }
 
         uint8_t *st = stages + s * Lay::kStage;
         const uint8_t *Bt = st + (GATE ? 3 : 2) * TILE;
         const uint8_t *Ct = Bt + Lay::kBCTile;
-        float *bcb = bcp + (it & 1) * TC * 32;
-        // B, C -> fp32, token-major: [t][parity p][B: X[p], X[p+2], ..., X[p+14]][C: same]
-        for (int q2 = tid; arrived && q2 < TC * (MODE == 1 ? 16 : 32); q2 += CONS) {
-            // MODE 1 stages B only: (token, parity, k8) -> its slot in the
-            // [t][parity][B 8 | C 8] row
-            const int q = MODE == 1
-                              ? ((q2 >> 4) << 5) + (((q2 >> 3) & 1) << 4) + (q2 & 7)
-                              : q2;
-            const int t = q >> 5, rest = q & 31;
-            const int par = rest >> 4, isC = (rest >> 3) & 1, k8 = rest & 7;
-            const int n = 2 * k8 + par;
-            const uint8_t *src = isC ? Ct : Bt;
-            const int chunk = (t * 2) >> 4, within = (t * 2) & 15;
-            const uint16_t v = *reinterpret_cast<const uint16_t *>(
-                src + n * 128 + ((chunk ^ (n & 7)) << 4) + within);
-            bcb[q] = __uint_as_float(uint32_t(v) << 16);
+        float *bcb = bcf + (it & 1) * TC * 32;
+        // B (times ln2) and C of this chunk -> fp32, token-major [t][B 16 | C 16].
+        // Lane r converts row r (B rows 0..15, C rows 16..31), warp w the
+        // 8-token vectors w, w + CW, ...: one 16-byte read, eight 4-byte writes
+        // to consecutive words.
+        if (arrived && (OUT || lane < 16)) {
+            const int isC = lane >> 4, n = lane & 15;
+            const uint8_t *src = (isC ? Ct : Bt) + n * 128;
+            const float sc = isC ? 1.f : kLn2;
+            for (int v = warp; v < 8; v += CW) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(src + ((v ^ (n & 7)) << 4));
+                float f[8];
+                unpack8_bf16(q, f);
+                float *dst = bcb + v * 8 * 32 + lane;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i * 32] = f[i] * sc;
+            }
         }
-        if (tid == 0)
+        if (OUT && tid == 0)
             bulk_wait_read<0>();  // y tile (it & 1) free again
+        if (OUT)
+            fence_proxy_async_smem();  // my y writes of the previous chunk -> its TMA store
         if (named_bar_any(1, CONS, !arrived)) {
             if (tid == 0)
                 atomicOr(p.err, kErrTimeoutPipe);
             *abort_flag = 1;
             break;
         }
-        if (MODE != 1 && tid == 0 && it > 0) {
+        if (OUT && tid == 0 && it > 0) {
             tma_store_3d(&tm_y, ytile + ((it - 1) & 1) * TILE, prev_t0, prev_d0, prev_b);
             bulk_commit();
         }
@@ -337,164 +494,81 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
         uint8_t *y_row = ytile + (it & 1) * TILE + ch * 128;
         const int t0 = inf.y;
 
-        // The 8-token blocks are software-pipelined: while block j runs its
-        // eight steps, the same basic block prepares block j + 1 (softplus,
-        // w, 1/w, decay base: special-function latency) and finishes block
-        // j - 1 (reduce-scatter, D skip, gate, store), so the latencies of
-        // those two phases hide under the step arithmetic.
+        // Block j's eight steps run in the same basic block as the
+        // preparation of block j + 1 and the outputs of block j - 1, so the
+        // special-function and shared-memory latencies of those phases hide
+        // under the step arithmetic.
         auto run = [&](auto pow_tag) {
             constexpr bool POWC = decltype(pow_tag)::value;
-            float rv[4], wv[4], rwv[4], uv[4];  // prepared block (this lane's 4 tokens)
-            float dts[4];                       // its step sizes (aggregate pass)
-            uint2 zq = make_uint2(0, 0);
-            auto prep = [&](int jb) {
-                const int off = ((jb ^ swz) << 4) + pp * 8;
-                const uint2 uq = *reinterpret_cast<const uint2 *>(u_row + off);
-                const uint2 dq = *reinterpret_cast<const uint2 *>(dl_row + off);
-                if (GATE && MODE != 1)
-                    zq = *reinterpret_cast<const uint2 *>(z_row + off);
-                const int tmine = t0 + jb * 8 + pp * 4;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t uw = kk < 2 ? uq.x : uq.y, dw = kk < 2 ? dq.x : dq.y;
-                    uv[kk] = __uint_as_float((kk & 1) ? (uw & 0xffff0000u) : (uw << 16));
-                    const float dv = __uint_as_float((kk & 1) ? (dw & 0xffff0000u) : (dw << 16));
-                    const float x = dv + bias;
-                    float dt = SOFTPLUS ? softplus_fast(x) : x;
-                    dt = (tmine + kk < p.L) ? dt : 0.f;  // padding past L: identity step
-                    dts[kk] = dt;
-                    const float wr = dt * uv[kk];
-                    wv[kk] = copysignf(fmaxf(fabsf(wr), kWMin), wr);
-                    rwv[kk] = rcp_approx(wv[kk]);
-                    rv[kk] = POWC ? ex2_approx(dt * a0) : dt;
-                }
-            };
-            // finished-block state carried into the next iteration
-            float yp_prev[8], w_prev4[4], u_prev4[4];
-            uint2 z_prev = make_uint2(0, 0);
-            int off_prev = 0;
-            auto finish = [&]() {
-                // reduce-scatter: this lane finishes tokens 4pp .. 4pp+3
-                float yo[4];
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const float send = pp ? yp_prev[kk] : yp_prev[4 + kk];
-                    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-                    float v = ((pp ? yp_prev[4 + kk] : yp_prev[kk]) + recv) * w_prev4[kk];
-                    v = fmaf(dsk, u_prev4[kk], v);
-                    if (GATE) {
-                        const uint32_t zw = kk < 2 ? z_prev.x : z_prev.y;
-                        const float zv = __uint_as_float((kk & 1) ? (zw & 0xffff0000u) : (zw << 16));
-                        v *= silu_fast(zv);
-                    }
-                    yo[kk] = v;
-                }
-                *reinterpret_cast<uint2 *>(y_row + off_prev) =
-                    make_uint2(pack2_bf16(yo[0], yo[1]), pack2_bf16(yo[2], yo[3]));
-            };
-            prep(0);
+            PrepBlock cur, nxt;
+            float yp[8], se[8], yp_prev[8], se_prev[8];
+            prep8<SOFTPLUS, POWC, MODE>(cur, u_row, dl_row, swz << 4, t0, p.L, BL2E2, a0);
 #pragma unroll 2
             for (int j = 0; j < TC / 8; ++j) {
-                // both lanes need r, w, 1/w of all 8 tokens of block j
-                float r8[8], w8[8], rw8[8];
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const float ro = __shfl_xor_sync(0xffffffffu, rv[kk], 1);
-                    const float wo = __shfl_xor_sync(0xffffffffu, wv[kk], 1);
-                    const float rwo = __shfl_xor_sync(0xffffffffu, rwv[kk], 1);
-                    r8[kk] = pp ? ro : rv[kk];
-                    r8[4 + kk] = pp ? rv[kk] : ro;
-                    w8[kk] = pp ? wo : wv[kk];
-                    w8[4 + kk] = pp ? wv[kk] : wo;
-                    rw8[kk] = pp ? rwo : rwv[kk];
-                    rw8[4 + kk] = pp ? rwv[kk] : rwo;
-                }
-                float wmine[4], umine[4];
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    wmine[kk] = wv[kk];
-                    umine[kk] = uv[kk];
-                }
-                const uint2 zmine = zq;
+                // channels past dim (zero-filled rows) never ask for the exact form
+                const bool exact = __any_sync(0xffffffffu, cur.tiny && live);
                 if (MODE == 1)
-                    sdel += (dts[0] + dts[1]) + (dts[2] + dts[3]);
-                if (MODE != 1 && j > 0)
-                    finish();            // block j - 1
-                prep((j + 1) & 7);       // block j + 1 (wraps harmlessly after the last)
-                float yp[8];
-                const float *bcb_blk = bcb + j * 8 * 32 + pp * 16;
+                    SD = add2(SD, cur.SD);
+                const int jn = (j + 1) & 7;  // wraps harmlessly after the last block
+                auto body = [&](auto exact_tag) {
+                    constexpr bool EX = decltype(exact_tag)::value;
+                    if (OUT && j > 0)
+                        finish8<GATE>(yp_prev, se_prev, u_row, z_row, y_row,
+                                      ((j - 1) ^ swz) << 4, dsk);
+                    prep8<SOFTPLUS, POWC, MODE>(nxt, u_row, dl_row, (jn ^ swz) << 4,
+                                                t0 + jn * 8, j < 7 ? p.L : 0x7fffffff, BL2E2,
+                                                a0);
+                    steps8<EX, POWC, OUT>(g, cur, s_prev, bcb + j * 8 * 32, yp, se, apair);
+                };
+                if (exact)
+                    body(std::true_type{});
+                else
+                    body(std::false_type{});
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float c = (i == 0 ? wprev : w8[i - 1]) * rw8[i];
-                    const ulonglong2 *bq = reinterpret_cast<const ulonglong2 *>(bcb_blk + i * 32);
-                    const ulonglong2 b01 = bq[0], b23 = bq[1];
-                    uint64_t V[4];
-                    decay_pairs<POWC>(V, r8[i], c, pp, apair);
-                    g[0] = fma2(V[0], g[0], b01.x);
-                    g[1] = fma2(V[1], g[1], b01.y);
-                    g[2] = fma2(V[2], g[2], b23.x);
-                    g[3] = fma2(V[3], g[3], b23.y);
-                    if (MODE == 1) {
-                        yp[i] = 0.f;
-                        continue;
-                    }
-                    const ulonglong2 c01 = bq[2], c23 = bq[3];
-                    uint64_t Ya = mul2(c01.x, g[0]);
-                    uint64_t Yb = mul2(c01.y, g[1]);
-                    Ya = fma2(c23.x, g[2], Ya);
-                    Yb = fma2(c23.y, g[3], Yb);
-                    const uint64_t Y = add2(Ya, Yb);
-                    yp[i] = lo2(Y) + hi2(Y);
-                }
-                wprev = w8[7];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
                     yp_prev[i] = yp[i];
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    w_prev4[kk] = wmine[kk];
-                    u_prev4[kk] = umine[kk];
+                    se_prev[i] = se[i];
                 }
-                z_prev = zmine;
-                off_prev = ((j ^ swz) << 4) + pp * 8;
+                cur = nxt;
             }
-            if (MODE != 1)
-                finish();  // last block
+            if (OUT)
+                finish8<GATE>(yp_prev, se_prev, u_row, z_row, y_row, (7 ^ swz) << 4, dsk);
         };
         if (pow_path)
             run(std::true_type{});
         else
             run(std::false_type{});
 
-        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[s]);
 
         if (inf.z & kInfoLast) {
-            // back to h = w_last * g; continue from h with w_{-1} := 1
-            float hv[8];
+            // back to h = s_last g; continue from h with s_{-1} := 1
+            float hv[16];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                hv[2 * jj] = lo2(g[jj]) * wprev;
-                hv[2 * jj + 1] = hi2(g[jj]) * wprev;
-                g[jj] = pk2(hv[2 * jj], hv[2 * jj + 1]);
+            for (int kk = 0; kk < 8; ++kk) {
+                hv[2 * kk] = lo2(g[kk]) * s_prev;
+                hv[2 * kk + 1] = hi2(g[kk]) * s_prev;
+                g[kk] = pk2(hv[2 * kk], hv[2 * kk + 1]);
             }
-            wprev = 1.f;
+            s_prev = 1.f;
             if (MODE == 1) {
                 // aggregate of this segment: end state from zero, sum of steps
                 const size_t ua = size_t(unit) * CH + ch;
-                float4 *dst = reinterpret_cast<float4 *>(p.agg + ua * kDiagN + pp * 8);
-                __stcg(dst, make_float4(hv[0], hv[1], hv[2], hv[3]));
-                __stcg(dst + 1, make_float4(hv[4], hv[5], hv[6], hv[7]));
-                const float sd = sdel + __shfl_xor_sync(0xffffffffu, sdel, 1);
-                if (pp == 0)
-                    __stcg(p.agg_sd + ua, sd);
+                float4 *dst = reinterpret_cast<float4 *>(p.agg + ua * kDiagN);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    __stcg(dst + q4, make_float4(hv[4 * q4], hv[4 * q4 + 1], hv[4 * q4 + 2],
+                                                 hv[4 * q4 + 3]));
+                __stcg(p.agg_sd + ua, lo2(SD) + hi2(SD));
             } else if (MODE == 0 && k < p.num_segs - 1) {
                 float4 *dst = reinterpret_cast<float4 *>(
-                    p.carry + (size_t(unit) * CH + ch) * kDiagN + pp * 8);
-                dst[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
-                dst[1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
+                    p.carry + (size_t(unit) * CH + ch) * kDiagN);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    dst[q4] = make_float4(hv[4 * q4], hv[4 * q4 + 1], hv[4 * q4 + 2],
+                                          hv[4 * q4 + 3]);
                 __threadfence();
                 __syncwarp();
                 if (lane == 0 && unit != p.dbg_skip_publish)
@@ -502,8 +576,8 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             } else if (p.last_state && d < p.dim && k == p.num_segs - 1) {
                 float *dst = p.last_state + (size_t(b) * p.dim + d) * kDiagN;
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    dst[2 * j + pp] = hv[j];
+                for (int n = 0; n < 16; ++n)
+                    dst[n] = hv[n];
             }
         }
         prev_t0 = inf.y;
@@ -516,9 +590,11 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
         }
     }
 
+    if (OUT)
+        fence_proxy_async_smem();
     named_bar_sync(1, CONS);
     if (tid == 0) {
-        if (MODE != 1 && it > 0 && !*abort_flag) {
+        if (OUT && it > 0 && !*abort_flag) {
             tma_store_3d(&tm_y, ytile + ((it - 1) & 1) * TILE, prev_t0, prev_d0, prev_b);
             bulk_commit();
         }
