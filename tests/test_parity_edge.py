@@ -1,0 +1,185 @@
+"""GPU parity of selscan_fwd on the method's own edge cases, against the fp64
+oracle on the same inputs ("03 -- Modelos de espacio de estados", section "El
+mecanismo selectivo de Mamba": the step size decides whether the state is
+kept or reset, so a zero step keeps it and a large one forgets it).
+
+Each case runs the bf16 kernel in the chained and two-pass forms and the
+fp32 kernel, over 2 x 256 channels and 4096 tokens, so that the special
+stretches cross whole 64-token chunks and time-segment boundaries.  Besides
+the whole-tensor relative L2 (y and last_state separately, 5e-3 bf16 / 1e-5
+fp32) every channel is held to the same bound on its own, so a channel whose
+outputs are small cannot hide behind the others.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 5e-3}
+FORMS = [("bf16", 0), ("bf16", 1), ("f32", -1)]
+FORM_IDS = ["bf16-chained", "bf16-two-pass", "f32"]
+
+
+def rel_l2(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
+
+
+def per_channel_worst(got, ref):
+    """Largest relative L2 over (batch, channel) rows whose reference is non-zero."""
+    got = np.asarray(got, np.float64).reshape(-1, got.shape[-1])
+    ref = np.asarray(ref, np.float64).reshape(-1, ref.shape[-1])
+    num = np.linalg.norm(got - ref, axis=1)
+    den = np.linalg.norm(ref, axis=1)
+    live = den > 0
+    return float(np.max(num[live] / den[live])) if live.any() else 0.0
+
+
+def to_dev(a, dtype):
+    import torch
+    if a is None:
+        return None
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return t.to(torch.bfloat16) if dtype == "bf16" else t.float()
+
+
+def f32dev(a):
+    import torch
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).float().cuda()
+
+
+def run_gpu(inp, mode, L=None):
+    """selscan_fwd through the C ABI, optionally on the first L tokens only."""
+    import selective_state_space_selscan_b200 as ss
+    dt = inp["dtype"]
+    cut = (lambda a: a) if L is None else (lambda a: None if a is None else a[..., :L])
+    ss.debug_diag_mode(mode)
+    try:
+        y, hs = ss.selscan_fwd(to_dev(cut(inp["u"]), dt), to_dev(cut(inp["delta"]), dt),
+                               f32dev(inp["A"]), to_dev(cut(inp["B"]), dt),
+                               to_dev(cut(inp["C"]), dt), D=f32dev(inp["D"]),
+                               z=to_dev(cut(inp["z"]), dt), delta_bias=f32dev(inp["delta_bias"]),
+                               delta_softplus=inp["softplus"])
+        ss.check()
+    finally:
+        ss.debug_diag_mode(-1)
+    return y.float().cpu().numpy(), hs.cpu().numpy()
+
+
+def run_oracle(inp):
+    return oracle.selscan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                          z=inp["z"], delta_bias=inp["delta_bias"],
+                          delta_softplus=inp["softplus"])
+
+
+def store(a, dtype):
+    return synthetic.round_bf16(a) if dtype == "bf16" else np.ascontiguousarray(a, np.float32)
+
+
+def base(dtype, seed, **kw):
+    return synthetic.make_diag(2, 256, 16, 4096, dtype=dtype, seed=seed, **kw)
+
+
+def check(inp, y, hs, what):
+    tol = TOL[inp["dtype"]]
+    y_ref, hs_ref = run_oracle(inp)
+    assert np.isfinite(y).all() and np.isfinite(hs).all(), what
+    ey, eh = rel_l2(y, y_ref), rel_l2(hs, hs_ref)
+    cy, ch = per_channel_worst(y, y_ref), per_channel_worst(hs, hs_ref)
+    assert ey <= tol and eh <= tol, f"{what}: rel L2 y={ey:.3e} state={eh:.3e} (tol {tol})"
+    assert cy <= tol and ch <= tol, f"{what}: worst channel y={cy:.3e} state={ch:.3e}"
+    return y_ref, hs_ref
+
+
+@pytest.mark.parametrize("dtype,mode", FORMS, ids=FORM_IDS)
+def test_zero_input_runs(dtype, mode):
+    """u = 0 over tokens 1000..1599 (whole chunks and segment boundaries),
+    over the first 130 tokens of some channels, and over whole channels
+    (which must give exactly zero output and state)."""
+    inp = base(dtype, 51)
+    u = inp["u"].copy()
+    u[:, :, 1000:1600] = 0.0
+    u[1, 100:108, :130] = 0.0
+    u[0, :8, :] = 0.0
+    inp["u"] = u
+    y, hs = run_gpu(inp, mode)
+    check(inp, y, hs, f"zero runs {dtype} mode {mode}")
+    assert np.all(y[0, :8] == 0.0) and np.all(hs[0, :8] == 0.0), "all-zero channels"
+
+
+@pytest.mark.parametrize("dtype,mode", FORMS, ids=FORM_IDS)
+def test_zero_step_keeps_state(dtype, mode):
+    """Softplus off, no bias, Delta = 0 over the last 704 tokens: the final
+    state equals the state after token 3391 (the scan of the first 3392
+    tokens, a length whose rows stay 16-byte aligned), and the outputs match
+    the oracle throughout."""
+    inp = base(dtype, 52, bias=False)
+    rng = np.random.default_rng(7)
+    delta = np.abs(rng.standard_normal(inp["u"].shape).astype(np.float32)) * 0.05
+    delta[:, :, 3392:] = 0.0
+    inp["delta"] = store(delta, dtype)
+    inp["softplus"] = False
+    y, hs = run_gpu(inp, mode)
+    check(inp, y, hs, f"zero step {dtype} mode {mode}")
+    _, hs_cut = run_gpu(inp, mode, L=3392)
+    e = rel_l2(hs, hs_cut)
+    assert e <= 1e-5, f"state moved over a zero-step run: rel {e:.3e}"
+
+
+@pytest.mark.parametrize("dtype,mode", FORMS, ids=FORM_IDS)
+def test_large_step_resets_state(dtype, mode):
+    """delta |A| >= 50 resets the state to delta B u: softplus off with
+    Delta = 50 on tokens 1500..1503, and (second input) softplus on with a
+    raw Delta of 60 on tokens 2600..2603."""
+    inp = base(dtype, 53, bias=False)
+    rng = np.random.default_rng(8)
+    delta = np.abs(rng.standard_normal(inp["u"].shape).astype(np.float32)) * 0.05
+    delta[:, :, 1500:1504] = 50.0
+    inp["delta"] = store(delta, dtype)
+    inp["softplus"] = False
+    y, hs = run_gpu(inp, mode)
+    check(inp, y, hs, f"reset (plain step) {dtype} mode {mode}")
+    # right after the reset the state is delta B u of the last large step
+    _, hs_cut = run_gpu(inp, mode, L=1504)
+    want = 50.0 * inp["B"][:, None, :, 1503] * inp["u"][:, :, 1503][:, :, None]
+    assert rel_l2(hs_cut, want) <= 1e-5
+
+    inp2 = base(dtype, 54)
+    d2 = inp2["delta"].copy()
+    d2[:, :, 2600:2604] = 60.0
+    inp2["delta"] = store(d2, dtype)
+    y, hs = run_gpu(inp2, mode)
+    check(inp2, y, hs, f"reset (softplus) {dtype} mode {mode}")
+
+
+@pytest.mark.parametrize("dtype,mode", FORMS, ids=FORM_IDS)
+def test_alternating_sign(dtype, mode):
+    """u changes sign at every token."""
+    inp = base(dtype, 55)
+    sgn = np.where(np.arange(4096) % 2 == 0, 1.0, -1.0).astype(np.float32)
+    inp["u"] = store(np.abs(inp["u"]) * sgn, dtype)
+    y, hs = run_gpu(inp, mode)
+    check(inp, y, hs, f"alternating sign {dtype} mode {mode}")
+
+
+@pytest.mark.parametrize("dtype,mode", FORMS, ids=FORM_IDS)
+def test_input_dynamic_range(dtype, mode):
+    """|u| log-uniform over [1e-30, 1e3] token by token (random sign) on half
+    of the channels, and |u| in [1e-25, 1e-20] on every token of 16 channels,
+    so that |delta u| runs from far below 2^-64 to ~1e2 inside one channel."""
+    inp = base(dtype, 56)
+    rng = np.random.default_rng(9)
+    u = inp["u"].copy()
+    mag = 10.0 ** rng.uniform(-30.0, 3.0, size=u[:, ::2].shape)
+    sgn = np.where(rng.random(size=mag.shape) < 0.5, -1.0, 1.0)
+    u[:, ::2] = (mag * sgn).astype(np.float32)
+    tiny = 10.0 ** rng.uniform(-25.0, -20.0, size=u[:, 1:33:2].shape)
+    u[:, 1:33:2] = (tiny * np.sign(u[:, 1:33:2] + 1e-30)).astype(np.float32)
+    inp["u"] = store(u, dtype)
+    y, hs = run_gpu(inp, mode)
+    check(inp, y, hs, f"dynamic range {dtype} mode {mode}")

@@ -88,20 +88,18 @@ def test_empty_sequence():
     assert y.shape == (2, 128, 0) and torch.all(hs == 0)
 
 
-def test_full_size_config4_sampled():
+def test_full_size_config4_whole():
     """Full config (B4 H32 P64 N128 L4096) in the benchmark's launch
-    configuration; the oracle checks three whole heads for every batch."""
+    configuration, compared with the oracle on every head, channel, token and
+    batch row (the oracle runs over head ranges on several host threads).
+    The measured errors are printed (pytest -s) so that the cost of keeping
+    the carried-in state in bf16 for the C h term is visible."""
+    import oracle_par
     inp = synthetic.make_config(4)
     y, hs = run_gpu(inp)
-    P = inp["headdim"]
-    ys, yr, hl, hr = [], [], [], []
-    for h in (0, 15, 31):
-        y_ref, hs_ref = run_oracle(inp, heads=(h, h + 1))
-        ys.append(y[:, h * P:(h + 1) * P]); yr.append(y_ref)
-        hl.append(hs[:, h:h + 1]); hr.append(hs_ref)
-    check(np.concatenate(ys, 1), np.concatenate(hl, 1), np.concatenate(yr, 1),
-          np.concatenate(hr, 1), "config 4")
-    assert np.isfinite(y).all()
+    y_ref, hs_ref = oracle_par.selscan_scalarA(inp)
+    check(y, hs, y_ref, hs_ref, "config 4")
+    print(f"config 4: rel L2 y={rel_l2(y, y_ref):.3e} state={rel_l2(hs, hs_ref):.3e}")
 
 
 @pytest.mark.parametrize("G", [2, 4])
