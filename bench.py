@@ -43,7 +43,7 @@ METRIC = "selective-scan Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU"
 # were taken on; reported as roofline.traffic only for that kernel.
 NCU_TRAFFIC = {
     # config 2 captured at L = 2048, scaled by tokens to L = 4096
-    2: ("scan_diag_bf16_kernel pairs v4", 642.3e6),
+    2: ("scan_diag_bf16_kernel lane-per-channel v5", 644.7e6),
     # config 3 (two-pass form, both kernels of one call) captured at
     # L = 32768, scaled by tokens to L = 131072
     3: ("scan_diag_bf16_kernel two-pass v1", 2679.6e6),
@@ -245,10 +245,67 @@ def oracle_sample(cfg_idx: int, inp: dict, seconds: float = 10.0):
             break
         grow = max(2.0, min(16.0, seconds / max(dt, 1e-3)))
         n = int(min(n * grow, cfg.get("dim") or cfg["nheads"] * cfg["headdim"]))
-    return {"value": done_elems / spent / 1e9, "unit": "Gelem/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{unit} x batch {b} x L {L} = {done_elems} elements, "
-                      f"{spent:.1f} s single-threaded fp64"}
+    out = {"value": done_elems / spent / 1e9, "unit": "Gelem/s", "cores": 1,
+           "kind": "oracle",
+           "sample": f"{unit} x batch {b} x L {L} = {done_elems} elements, "
+                     f"{spent:.1f} s single-threaded fp64",
+           "host": host_cpu()}
+    out["all_cores"] = oracle_all_cores(cfg, inp, n, seconds)
+    return out
+
+
+def host_cpu() -> dict:
+    """Host cores and CPU model of the machine the baseline ran on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+def oracle_all_cores(cfg: dict, inp: dict, n: int, seconds: float) -> dict:
+    """The same unchanged single-threaded oracle, run over channel (or
+    head) ranges on every host core at once: one call per core, side by
+    side (the oracle's C loop runs without the interpreter lock).  The sample
+    is `n` channels per core, capped at the workload's d_inner."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    cores = os.cpu_count() or 1
+    L, b = cfg["L"], cfg["batch"]
+    if cfg["kind"] == "diag":
+        total = min(cfg["dim"], n * cores)
+        edges = np.linspace(0, total, min(cores, total) + 1).astype(int)
+
+        def one(r):
+            oracle.selscan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                           z=inp["z"], delta_bias=inp["delta_bias"],
+                           delta_softplus=inp["softplus"], channels=r)
+        per = 1
+        what = "channels"
+    else:
+        P = cfg["headdim"]
+        total = min(cfg["nheads"], max(1, n // P) * cores)
+        edges = np.linspace(0, total, min(cores, total) + 1).astype(int)
+
+        def one(r):
+            oracle.selscan_scalarA(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], P,
+                                   D=inp["D"], z=inp["z"], heads=r)
+        per = P
+        what = "heads"
+    ranges = [(int(a), int(c)) for a, c in zip(edges[:-1], edges[1:]) if c > a]
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(len(ranges)) as ex:
+        list(ex.map(one, ranges))
+    dt = time.perf_counter() - t0
+    elems = b * total * per * L
+    return {"value": elems / dt / 1e9, "unit": "Gelem/s", "cores": len(ranges),
+            "sample": f"{total} {what} x batch {b} x L {L} = {elems} elements over "
+                      f"{len(ranges)} threads, {dt:.1f} s"}
 
 
 def scan_config(cfg: dict, world: int) -> dict:

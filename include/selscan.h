@@ -182,11 +182,14 @@ SELSCAN_API selscan_status selscan_fwd_scalarA_h0(const selscan_tensor *x,
  * afterwards, and for systems where the stream-ordered allocator (memory
  * pools, which selscan_fwd uses for its scratch) is unavailable.
  *
- * Same arguments, layouts and results as selscan_fwd; the caller passes all
- * inputs and outputs.  Instead of the stream-ordered pool, the look-back scratch
- * (ticket, carry flags, segment carries) lives in one file-scope device
- * array of SELSCAN_NOALLOC_SCRATCH_BYTES per GPU, which every GPU that loads
- * the library holds until the process exits.  The call makes no
+ * Same arguments, layouts and results as selscan_fwd (bit for bit: the same
+ * kernels with the same work decomposition, including the choice between
+ * chained carries and the two-pass form for few channel tiles); the caller
+ * passes all inputs and outputs.  Instead of the stream-ordered pool, the
+ * scratch (tickets, carry flags and segment carries, or the two-pass form's
+ * segment aggregates) lives in one file-scope device array of
+ * SELSCAN_NOALLOC_SCRATCH_BYTES per GPU, which every GPU that loads the
+ * library holds until the process exits.  The call makes no
  * cudaMalloc / cudaFree / allocating call; it clears the part of the array
  * that must start at zero with cudaMemsetAsync on `stream`.
  *   - The first call on a device looks up the array's device address
@@ -196,11 +199,12 @@ SELSCAN_API selscan_status selscan_fwd_scalarA_h0(const selscan_tensor *x,
  *     contents: calls that overlap on the GPU (different streams, no
  *     ordering between them) race on it.  Serialise them.
  *   - A launch whose scratch would exceed the array returns
- *     SELSCAN_ERR_UNSUPPORTED and launches nothing.  The scratch is
- *     256 bytes plus (segments - 1) * tiles * (flags + 128 or 64 carried
- *     channels * 64 bytes); the library's scheduling keeps
- *     (segments - 1) * tiles below 8 * SM count, about 9.7 MiB on a
- *     148-SM B200.
+ *     SELSCAN_ERR_UNSUPPORTED and launches nothing.  The scratch is 256
+ *     bytes plus, per linked unit ((segments - 1) * channel tiles of 128
+ *     bf16 or 64 fp32 channels), the carried states (64 bytes per channel)
+ *     and either a flag per consumer warp (chained) or a step-size sum per
+ *     channel (two-pass form).  The library's scheduling keeps the linked
+ *     units below 8 * SM count: at most about 10.3 MiB on a 148-SM B200.
  */
 #define SELSCAN_NOALLOC_SCRATCH_BYTES (16u << 20)
 SELSCAN_API selscan_status selscan_fwd_noalloc(

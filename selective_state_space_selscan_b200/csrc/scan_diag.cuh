@@ -55,8 +55,6 @@ struct DiagParams {
     float *agg;           // two-pass form: [units][CH][parity][8] segment end states
     float *agg_sd;        // two-pass form: [units][CH] sums of step sizes
     float *last_state;    // (batch, dim, 16) or null
-    void *y;              // output (batch, dim, L), element strides y_bs, y_rs (fast bf16 kernel)
-    long long y_bs, y_rs;
     int softplus;
     unsigned int *ticket;  // zeroed before launch
     unsigned int *flags;   // [total_units][consumer warps], zeroed

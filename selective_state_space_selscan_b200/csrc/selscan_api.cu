@@ -378,9 +378,6 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
     if (units > 0x7fffffffll)
         return SELSCAN_ERR_UNSUPPORTED;
     prm.total_units = int(units);
-    prm.y = y->data;
-    prm.y_bs = y->stride[0];
-    prm.y_rs = y->stride[1];
 
     // Few tiles and several segments: a chain of carries would leave most
     // SMs waiting, so use the two-pass form (aggregates, then output).
@@ -889,7 +886,8 @@ selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor
     if (!ok)
         return SELSCAN_ERR_ALIGN;
 
-    // same work decomposition as selscan_fwd
+    // the work decomposition of selscan_fwd (segments, and the chained or
+    // the two-pass form by the same rule)
     const int tpb = int((dim + CH - 1) / CH);
     const int G = int(batch) * tpb;
     const int ctas_max = sm_count;
@@ -901,6 +899,56 @@ selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor
     const int64_t units = int64_t(G) * S;
     if (units > 0x7fffffffll)
         return SELSCAN_ERR_UNSUPPORTED;
+    prm.tiles_per_batch = tpb;
+    prm.num_tiles = G;
+    prm.seg_len = int(seg_chunks * TC);
+    prm.num_segs = int(S);
+    prm.total_units = int(units);
+    int dev = 0;
+    cudaGetDevice(&dev);
+
+    // Few tiles and several segments: the two-pass form, as selscan_fwd
+    // chooses it, with its aggregates in the static array (there is no
+    // initial state to copy).
+    if constexpr (KIND == 1) {
+    const bool two_pass = g_dbg_diag_mode >= 0 ? (g_dbg_diag_mode == 1 && S > 1)
+                                               : (S > 1 && 2 * int64_t(G) <= sm_count);
+    if (two_pass) {
+        const int64_t agg_units = int64_t(G) * (S - 1);
+        const size_t head = 256;  // two tickets
+        const size_t agg_bytes = size_t(agg_units) * CH * kDiagN * 4;
+        const size_t sd_bytes = ((size_t(agg_units) * CH * 4 + 255) / 256) * 256;
+        if (head + agg_bytes + sd_bytes > size_t(SELSCAN_NOALLOC_SCRATCH_BYTES))
+            return SELSCAN_ERR_UNSUPPORTED;  // the static array is too small for this launch
+        if (cudaMemsetAsync(scratch, 0, head, stream) != cudaSuccess)
+            return SELSCAN_ERR_CUDA;
+        prm.flags = nullptr;
+        prm.carry = nullptr;
+        prm.agg = reinterpret_cast<float *>(scratch + head);
+        prm.agg_sd = reinterpret_cast<float *>(scratch + head + agg_bytes);
+        prm.dbg_skip_publish = -1;
+        DiagParams p1 = prm, p2 = prm;
+        p1.ticket = reinterpret_cast<unsigned int *>(scratch);
+        p1.total_units = int(agg_units);
+        p2.ticket = reinterpret_cast<unsigned int *>(scratch + 64);
+        auto k1 = V::template kernel_mode<1>();
+        auto k2 = V::template kernel_mode<2>();
+        static bool done1[kMaxDevices] = {}, done2[kMaxDevices] = {};
+        if (!ensure_smem(k1, V::template smem_mode<1>(), dev, done1) ||
+            !ensure_smem(k2, V::template smem_mode<2>(), dev, done2))
+            return SELSCAN_ERR_CUDA;
+        k1<<<int(std::min<int64_t>(ctas_max, agg_units)), V::kThreads,
+             V::template smem_mode<1>(), stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, p1);
+        cudaError_t le = counted_launch();
+        if (le == cudaSuccess) {
+            k2<<<int(std::min<int64_t>(ctas_max, units)), V::kThreads,
+                 V::template smem_mode<2>(), stream>>>(tm_u, tm_d, tm_z, tm_B, tm_C, tm_y, p2);
+            le = counted_launch();
+        }
+        return le == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+    }
+    }
+
     // Only units of the first S-1 segments publish a carry and a flag.
     const int64_t linked = int64_t(G) * (S - 1);
     const size_t head = 256;
@@ -908,14 +956,6 @@ selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor
     const size_t carry_bytes = size_t(linked) * CH * kDiagN * 4;
     if (head + flag_bytes + carry_bytes > size_t(SELSCAN_NOALLOC_SCRATCH_BYTES))
         return SELSCAN_ERR_UNSUPPORTED;  // the static array is too small for this launch
-    prm.tiles_per_batch = tpb;
-    prm.num_tiles = G;
-    prm.seg_len = int(seg_chunks * TC);
-    prm.num_segs = int(S);
-    prm.total_units = int(units);
-    prm.y = y->data;
-    prm.y_bs = y->stride[0];
-    prm.y_rs = y->stride[1];
     // the previous call's ticket and flags must not leak into this one
     if (cudaMemsetAsync(scratch, 0, head + flag_bytes, stream) != cudaSuccess)
         return SELSCAN_ERR_CUDA;
@@ -926,8 +966,6 @@ selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor
 
     auto kern = V::kernel();
     static bool attr_set[kMaxDevices] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  V::kSmem) != cudaSuccess)
