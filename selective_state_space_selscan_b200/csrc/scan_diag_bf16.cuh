@@ -29,8 +29,13 @@
 //  * Per-token work that does not depend on the state index (softplus in
 //    log2 units, the decay base, 1/s, the D skip, the gate) runs on pairs of
 //    tokens with packed f32x2 instructions, and is software-pipelined: the
-//    next 8-token block is prepared and the previous one finished in the same
-//    basic block as the current block's eight steps.
+//    next 8-token block is prepared and the previous one finished while the
+//    current block's eight steps run, interleaved token by token in the
+//    source (a pair of the next block's preparation before every even step,
+//    a pair of the previous block's outputs after every odd one), which is
+//    the order the scheduler keeps under full register pressure; with one
+//    warp per scheduler that order decides how much of the special-function
+//    and shared-memory latency hides under the step arithmetic.
 //  * For S4D-real A (A[d,n] = (n+1) A[d,0], checked per channel at run time)
 //    the decays are powers r^(n+1) of r = exp(delta A[d,0]): one ex2 per token
 //    and seven packed multiplies.  Other A take one ex2 per state.
@@ -79,6 +84,49 @@ struct PrepBlock {
     bool tiny;       // some |s| < 2^-64 in the block
 };
 
+// Preparation of token pair k (tokens 2k, 2k + 1) of a block, from the
+// block's u and Delta words; `mn` and `SDa` accumulate over the pairs.
+template <bool SOFTPLUS, bool POW, int MODE>
+__device__ __forceinline__ void prep_pair(PrepBlock &pb, float &mn, uint64_t &SDa, uint32_t uw,
+                                          uint32_t dw, int k, int tfirst, int L, uint64_t BL2E2,
+                                          float a0)
+{
+    const uint64_t L2E2 = pk2(kLog2e, kLog2e);
+    const uint64_t U = bf2_to_f2(uw);
+    uint64_t D2 = fma2(bf2_to_f2(dw), L2E2, BL2E2);  // (Delta + bias) log2e
+    if (SOFTPLUS) {
+        // delta log2e = log2(1 + 2^x): lg2 of 1 + e, or the log1p series
+        // (in log2 units) when e < 2^-6; x itself beyond 2^64.
+        const float xa = lo2(D2), xb = hi2(D2);
+        const uint64_t E = pk2(ex2_approx(fminf(xa, 64.f)), ex2_approx(fminf(xb, 64.f)));
+        const uint64_t T = add2(E, pk2(1.f, 1.f));
+        uint64_t Q = fma2(E, pk2(kLog2e / 3.f, kLog2e / 3.f), pk2(-0.5f * kLog2e, -0.5f * kLog2e));
+        Q = fma2(E, Q, L2E2);
+        Q = mul2(E, Q);
+        float da = lo2(E) < kSmallE ? lo2(Q) : lg2_approx(lo2(T));
+        float db = hi2(E) < kSmallE ? hi2(Q) : lg2_approx(hi2(T));
+        D2 = pk2(fmaxf(da, xa), fmaxf(db, xb));
+    }
+    if (tfirst + 8 > L) {
+        // tokens past the end of the sequence: identity steps
+        const int t = tfirst + 2 * k;
+        D2 = pk2(t < L ? lo2(D2) : 0.f, t + 1 < L ? hi2(D2) : 0.f);
+    }
+    if (MODE == 1)
+        SDa = add2(SDa, D2);
+    if (POW) {
+        const uint64_t X = mul2(D2, pk2(a0, a0));
+        pb.R[k] = pk2(ex2_approx(lo2(X)), ex2_approx(hi2(X)));
+    } else {
+        pb.R[k] = D2;
+    }
+    const uint64_t W = mul2(D2, U);
+    pb.W[k] = W;
+    mn = fminf(mn, fminf(fabsf(lo2(W)), fabsf(hi2(W))));
+    pb.RS[k] = pk2(rcp_approx(lo2(W)), rcp_approx(hi2(W)));
+}
+
+// Preparation of a whole block (the first block of a chunk).
 template <bool SOFTPLUS, bool POW, int MODE>
 __device__ __forceinline__ void prep8(PrepBlock &pb, const uint8_t *u_row, const uint8_t *dl_row,
                                       int off, int tfirst, int L, uint64_t BL2E2, float a0)
@@ -87,60 +135,85 @@ __device__ __forceinline__ void prep8(PrepBlock &pb, const uint8_t *u_row, const
     const uint4 dq = *reinterpret_cast<const uint4 *>(dl_row + off);
     const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
     const uint32_t dw[4] = {dq.x, dq.y, dq.z, dq.w};
-    const uint64_t L2E2 = pk2(kLog2e, kLog2e);
     float mn = 3.0e38f;
     uint64_t SD = pk2(0.f, 0.f);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint64_t U = bf2_to_f2(uw[k]);
-        uint64_t D2 = fma2(bf2_to_f2(dw[k]), L2E2, BL2E2);  // (Delta + bias) log2e
-        if (SOFTPLUS) {
-            // delta log2e = log2(1 + 2^x): lg2 of 1 + e, or the log1p series
-            // (in log2 units) when e < 2^-6; x itself beyond 2^64.
-            const float xa = lo2(D2), xb = hi2(D2);
-            const uint64_t E = pk2(ex2_approx(fminf(xa, 64.f)), ex2_approx(fminf(xb, 64.f)));
-            const uint64_t T = add2(E, pk2(1.f, 1.f));
-            uint64_t Q = fma2(E, pk2(kLog2e / 3.f, kLog2e / 3.f),
-                              pk2(-0.5f * kLog2e, -0.5f * kLog2e));
-            Q = fma2(E, Q, L2E2);
-            Q = mul2(E, Q);
-            float da = lo2(E) < kSmallE ? lo2(Q) : lg2_approx(lo2(T));
-            float db = hi2(E) < kSmallE ? hi2(Q) : lg2_approx(hi2(T));
-            D2 = pk2(fmaxf(da, xa), fmaxf(db, xb));
-        }
-        if (tfirst + 8 > L) {
-            // tokens past the end of the sequence: identity steps
-            const int t = tfirst + 2 * k;
-            D2 = pk2(t < L ? lo2(D2) : 0.f, t + 1 < L ? hi2(D2) : 0.f);
-        }
-        if (MODE == 1)
-            SD = add2(SD, D2);
-        if (POW) {
-            const uint64_t X = mul2(D2, pk2(a0, a0));
-            pb.R[k] = pk2(ex2_approx(lo2(X)), ex2_approx(hi2(X)));
-        } else {
-            pb.R[k] = D2;
-        }
-        const uint64_t W = mul2(D2, U);
-        pb.W[k] = W;
-        mn = fminf(mn, fminf(fabsf(lo2(W)), fabsf(hi2(W))));
-        pb.RS[k] = pk2(rcp_approx(lo2(W)), rcp_approx(hi2(W)));
-    }
+    for (int k = 0; k < 4; ++k)
+        prep_pair<SOFTPLUS, POW, MODE>(pb, mn, SD, uw[k], dw[k], k, tfirst, L, BL2E2, a0);
     pb.SD = SD;
     pb.tiny = mn < kTau;
 }
 
-// Eight recurrence steps of one block.  EXACT: the clamped form for blocks
-// with a tiny |s|.  OUT: also form the outputs (not in the aggregate pass).
-template <bool EXACT, bool POW, bool OUT>
-__device__ __forceinline__ void steps8(uint64_t (&g)[8], const PrepBlock &pb, float &s_prev,
-                                       const float *bct, float (&yp)[8], float (&se)[8],
-                                       const uint64_t (&apair)[8])
+// Outputs of token pair k: y = s (C.g) + D u, times silu(z), packed to bf16.
+template <bool GATE>
+__device__ __forceinline__ uint32_t finish_pair(float y0, float y1, float s0, float s1, uint32_t uw,
+                                                uint32_t zw, float dsk)
 {
+    const uint64_t DU = mul2(bf2_to_f2(uw), pk2(dsk, dsk));
+    uint64_t Y = fma2(pk2(s0, s1), pk2(y0, y1), DU);
+    if (GATE) {
+        // silu(z) = z sigmoid(z) = (z/2) (1 + tanh(z/2))
+        const uint64_t HZ = mul2(bf2_to_f2(zw), pk2(0.5f, 0.5f));
+        const uint64_t TH = pk2(tanh_approx(lo2(HZ)), tanh_approx(hi2(HZ)));
+        Y = mul2(Y, fma2(HZ, TH, HZ));
+    }
+    return pack2_bf16(lo2(Y), hi2(Y));
+}
+
+// Outputs of one block: y = s (C.g) + D u, times silu(z); bf16 into the y tile.
+template <bool GATE>
+__device__ __forceinline__ void finish8(const float (&yp)[8], const float (&se)[8],
+                                        const uint8_t *u_row, const uint8_t *z_row,
+                                        uint8_t *y_row, int off, float dsk)
+{
+    const uint4 uq = *reinterpret_cast<const uint4 *>(u_row + off);
+    uint4 zq = make_uint4(0, 0, 0, 0);
+    if (GATE)
+        zq = *reinterpret_cast<const uint4 *>(z_row + off);
+    const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+    const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        o[k] = finish_pair<GATE>(yp[2 * k], yp[2 * k + 1], se[2 * k], se[2 * k + 1], uw[k], zw[k],
+                                 dsk);
+    *reinterpret_cast<uint4 *>(y_row + off) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// One 8-token block with its neighbours' work interleaved token by token:
+// step i of this block, the preparation of pair i/2 of the next block (even
+// i) and the outputs of pair i/2 of the previous block (odd i, OUT only).
+template <bool EXACT, bool POW, bool OUT, bool SOFTPLUS, bool GATE, int MODE>
+__device__ __forceinline__ void block8(uint64_t (&g)[8], const PrepBlock &pb, PrepBlock &nx,
+                                       float &s_prev, const float *bct, float (&yp)[8],
+                                       float (&se)[8], const uint64_t (&apair)[8],
+                                       const uint8_t *u_row, const uint8_t *dl_row,
+                                       const uint8_t *z_row, uint8_t *y_row, int off_n,
+                                       int tfirst_n, int L_n, uint64_t BL2E2, float a0,
+                                       const float (&yq)[8], const float (&sq)[8], int off_p,
+                                       float dsk)
+{
+    const uint4 uq = *reinterpret_cast<const uint4 *>(u_row + off_n);
+    const uint4 dq = *reinterpret_cast<const uint4 *>(dl_row + off_n);
+    const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+    const uint32_t dw[4] = {dq.x, dq.y, dq.z, dq.w};
+    uint32_t fu[4] = {0, 0, 0, 0}, fz[4] = {0, 0, 0, 0}, o[4];
+    if (OUT) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(u_row + off_p);
+        fu[0] = a.x; fu[1] = a.y; fu[2] = a.z; fu[3] = a.w;
+        if (GATE) {
+            const uint4 c = *reinterpret_cast<const uint4 *>(z_row + off_p);
+            fz[0] = c.x; fz[1] = c.y; fz[2] = c.z; fz[3] = c.w;
+        }
+    }
+    float mn = 3.0e38f;
+    uint64_t SDa = pk2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int k = i >> 1;
         const bool hi = (i & 1) != 0;
+        if (!hi)
+            prep_pair<SOFTPLUS, POW, MODE>(nx, mn, SDa, uw[k], dw[k], k, tfirst_n, L_n, BL2E2, a0);
         const float w = hi ? hi2(pb.W[k]) : lo2(pb.W[k]);
         float s, rs;
         if (EXACT) {
@@ -194,36 +267,14 @@ __device__ __forceinline__ void steps8(uint64_t (&g)[8], const PrepBlock &pb, fl
             acc = fma2(c67.x, g[6], acc);
             acc = fma2(c67.y, g[7], acc);
             yp[i] = lo2(acc) + hi2(acc);
+            if (hi)
+                o[k] = finish_pair<GATE>(yq[i - 1], yq[i], sq[i - 1], sq[i], fu[k], fz[k], dsk);
         }
     }
-}
-
-// Outputs of one block: y = s (C.g) + D u, times silu(z); bf16 into the y tile.
-template <bool GATE>
-__device__ __forceinline__ void finish8(const float (&yp)[8], const float (&se)[8],
-                                        const uint8_t *u_row, const uint8_t *z_row,
-                                        uint8_t *y_row, int off, float dsk)
-{
-    const uint4 uq = *reinterpret_cast<const uint4 *>(u_row + off);
-    uint4 zq = make_uint4(0, 0, 0, 0);
-    if (GATE)
-        zq = *reinterpret_cast<const uint4 *>(z_row + off);
-    const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
-    const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint64_t DU = mul2(bf2_to_f2(uw[k]), pk2(dsk, dsk));
-        uint64_t Y = fma2(pk2(se[2 * k], se[2 * k + 1]), pk2(yp[2 * k], yp[2 * k + 1]), DU);
-        if (GATE) {
-            // silu(z) = z sigmoid(z) = (z/2) (1 + tanh(z/2))
-            const uint64_t HZ = mul2(bf2_to_f2(zw[k]), pk2(0.5f, 0.5f));
-            const uint64_t TH = pk2(tanh_approx(lo2(HZ)), tanh_approx(hi2(HZ)));
-            Y = mul2(Y, fma2(HZ, TH, HZ));
-        }
-        o[k] = pack2_bf16(lo2(Y), hi2(Y));
-    }
-    *reinterpret_cast<uint4 *>(y_row + off) = make_uint4(o[0], o[1], o[2], o[3]);
+    nx.SD = SDa;
+    nx.tiny = mn < kTau;
+    if (OUT)
+        *reinterpret_cast<uint4 *>(y_row + off_p) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // MODE 0: one pass, segments chained through published carries.
@@ -502,6 +553,11 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
             constexpr bool POWC = decltype(pow_tag)::value;
             PrepBlock cur, nxt;
             float yp[8], se[8], yp_prev[8], se_prev[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                yp_prev[i] = 0.f;
+                se_prev[i] = 0.f;
+            }
             prep8<SOFTPLUS, POWC, MODE>(cur, u_row, dl_row, swz << 4, t0, p.L, BL2E2, a0);
 #pragma unroll 2
             for (int j = 0; j < TC / 8; ++j) {
@@ -510,15 +566,14 @@ scan_diag_bf16_kernel(const __grid_constant__ CUtensorMap tm_u,
                 if (MODE == 1)
                     SD = add2(SD, cur.SD);
                 const int jn = (j + 1) & 7;  // wraps harmlessly after the last block
+                // block j - 1's outputs; for j = 0 this writes block 7's slot,
+                // which the last block's outputs overwrite below
                 auto body = [&](auto exact_tag) {
                     constexpr bool EX = decltype(exact_tag)::value;
-                    if (OUT && j > 0)
-                        finish8<GATE>(yp_prev, se_prev, u_row, z_row, y_row,
-                                      ((j - 1) ^ swz) << 4, dsk);
-                    prep8<SOFTPLUS, POWC, MODE>(nxt, u_row, dl_row, (jn ^ swz) << 4,
-                                                t0 + jn * 8, j < 7 ? p.L : 0x7fffffff, BL2E2,
-                                                a0);
-                    steps8<EX, POWC, OUT>(g, cur, s_prev, bcb + j * 8 * 32, yp, se, apair);
+                    block8<EX, POWC, OUT, SOFTPLUS, GATE, MODE>(
+                        g, cur, nxt, s_prev, bcb + j * 8 * 32, yp, se, apair, u_row, dl_row,
+                        z_row, y_row, (jn ^ swz) << 4, t0 + jn * 8, j < 7 ? p.L : 0x7fffffff,
+                        BL2E2, a0, yp_prev, se_prev, (((j - 1) & 7) ^ swz) << 4, dsk);
                 };
                 if (exact)
                     body(std::true_type{});
