@@ -43,15 +43,15 @@ METRIC = "selective-scan Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU"
 # were taken on; reported as roofline.traffic only for that kernel.
 NCU_TRAFFIC = {
     # config 2 captured at L = 2048, scaled by tokens to L = 4096
-    2: ("scan_diag_bf16_kernel lane-per-channel v5", 644.7e6),
+    2: ("scan_diag_bf16_kernel lane-per-channel v6", 640.3e6),
     # config 3 (two-pass form, both kernels of one call) captured at
     # L = 32768, scaled by tokens to L = 131072
     3: ("scan_diag_bf16_kernel two-pass v1", 2679.6e6),
     4: ("ssd_scalarA_kernel v5", 107.9e6),
 }
-KERNEL_TAG = {2: "scan_diag_bf16_kernel lane-per-channel v5",
-              1: "scan_diag_bf16_kernel lane-per-channel v5",
-              3: "scan_diag_bf16_kernel lane-per-channel two-pass v5",
+KERNEL_TAG = {2: "scan_diag_bf16_kernel lane-per-channel v6",
+              1: "scan_diag_bf16_kernel lane-per-channel v6",
+              3: "scan_diag_bf16_kernel lane-per-channel two-pass v6",
               0: "scan_diag_kernel fp32 v3", 4: "ssd_scalarA_kernel v5"}
 HBM_FALLBACK_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # the HGX/DGX nominal figure, reported beside the measured peak
