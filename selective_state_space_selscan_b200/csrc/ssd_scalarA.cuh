@@ -24,25 +24,27 @@
 // (one exponential per row and piece, one per column), and in the pieces
 // that hold a warp's diagonal it is taken per element.
 //
-// Per chunk c, in order (all threads unless noted):
-//   1. x * w for the state product (needs chunk c's x); one thread issues
-//      the state product, which runs during step 2;
-//   2. M from G (tensor memory) and the decays (needs G(c));
-//   3. one thread issues Yd(c) and G(c + 1);
-//   4. the second warpgroup prepares the step sizes of chunk c + 1;
-//   5. y = Yd + 2^cs_t Yo + D x (+ gate), staged in shared memory and written
-//      back by one bulk tensor store;
-//   6. state: h -> bf16 copy for Yo(c + 1), last_state, h *= 2^cs_Q(c + 1);
-//   7. one thread issues Yo(c + 1) and the loads of chunk c + 2.
+// Per chunk c, in order (all threads unless noted), each tensor-core product
+// issued by one thread as soon as its inputs are in place and waited for as
+// late as possible, so that it runs under the next CUDA-core phase:
+//   1. x * w for the state product (needs chunk c's x); issue the state
+//      product h += B (x w)^T, which runs during step 2;
+//   2. the second warpgroup prepares the step sizes of chunk c + 1 (into the
+//      other set of per-token arrays); M from G (tensor memory) and the
+//      decays; issue Yd(c) and G(c + 1), which run during step 3;
+//   3. state: h -> bf16 copy for Yo(c + 1), last_state, h *= 2^cs_Q(c + 1);
+//      issue Yo(c + 1) (into the other Yo columns), which runs during step 4;
+//   4. y = Yd + 2^cs_t Yo + D x (+ gate), staged in shared memory and written
+//      back by one bulk tensor store; issue the loads of chunk c + 2.
 //
 // Operands (bf16, 128-byte swizzle) in shared memory:
 //   C chunk [n][t] and B chunk [n][s] as loaded by the bulk tensor copy,
 //   used MN-major (C^T as A of G and Yo; B as B of G) and K-major (B as A of
 //   the state product); x chunk [p][s] (K-major B of Yd); x * w [p][s]
 //   (K-major B of the state product); M [t][s] (K-major A of Yd); h_prev in
-//   bf16 [n][p] (MN-major B of Yo).  The y tile [p][t] is staged in the M
-//   buffer once Yd has read it.  Accumulators in tensor memory (fp32): G (128
-//   columns), Yd (64), Yo (64), h (64).
+//   bf16 [n][p] (MN-major B of Yo), in the x * w buffer.  The y tile [p][t]
+//   is staged in the M buffer once Yd has read it.  Accumulators in tensor
+//   memory (fp32): G (128 columns), Yd (64), Yo (2 x 64), h (64).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -82,13 +84,19 @@ struct SsdLayout {
     static constexpr int kX = kB + 2 * 32768;      // 2 buffers x [2 slabs][64 p][64 s]
     static constexpr int kXw = kX + 2 * 16384;     // [2 slabs][64 p][64 s]
     static constexpr int kM = kXw + 16384;         // [2 slabs][128 t][64 s]; y tile [2][64 p][64 t]
-    static constexpr int kHs = kM + 32768;         // [128 n][64 p]
-    static constexpr int kBytes = kHs + 16384;
+    // bf16 state [128 n][64 p] for Yo, in the x*w buffer: written once the
+    // state product has read x*w, read by Yo(c+1), which completes before
+    // the next chunk's x*w is written
+    static constexpr int kHs = kXw;
+    static constexpr int kBytes = kM + 32768;
     static constexpr int kAlloc = kBytes + 1024;
 };
 
 constexpr uint32_t kSsdTmemCols = 512;
-constexpr uint32_t kColG = 0, kColYd = 128, kColYo = 192, kColH = 256;
+constexpr uint32_t kColG = 0, kColYd = 128, kColH = 256;
+// Yo of chunk c in columns kColYo + 128 (c % 2): Yo(c + 1) is issued once the
+// state of chunk c is out, while chunk c's epilogue still reads Yo(c)
+constexpr uint32_t kColYo = 192;
 
 __device__ __forceinline__ float ssd_softplus(float x)
 {
@@ -142,7 +150,9 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
     // every pointer derived from it stays in the shared address space
     uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     // per-token values of the chunk being prepared (see cumsum below)
-    __shared__ __align__(16) float s_cs[Q], s_n2[Q], s_sg[Q];
+    // (two sets, by chunk parity: the next chunk's are prepared while this
+    // chunk's are read)
+    __shared__ __align__(16) float s_cs2[2][Q], s_n22[2][Q], s_sg2[2][Q];
     __shared__ float s_wsum[4];
     __shared__ uint64_t bar_tma[2], bar_g, bar_yo, bar_yd, bar_st;
     __shared__ uint32_t s_tbase;
@@ -218,9 +228,9 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
             S += s_wsum[w];
         const float cs = a_l2 * S;
         const float cse = __shfl_sync(0xffffffffu, cs, lane | 15);
-        s_cs[r] = cs;
-        s_n2[r] = lg2_approx(dl) - cs;  // -inf for delta = 0, and 2^-inf = 0
-        s_sg[r] = ex2_approx(cse - cs) * dl;
+        s_cs2[cc & 1][r] = cs;
+        s_n22[cc & 1][r] = lg2_approx(dl) - cs;  // -inf for delta = 0, and 2^-inf = 0
+        s_sg2[cc & 1][r] = ex2_approx(cse - cs) * dl;
     };
 
     // initial state h[n][p] (zero unless given): row n = r, columns p of this
@@ -239,7 +249,7 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
     const uint32_t tb = s_tbase;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;  // this warp's TMEM lanes
     {
-        const float alpha0 = ex2_approx(s_cs[Q - 1]);
+        const float alpha0 = ex2_approx(s_cs2[0][Q - 1]);
         uint8_t *hs = smem + Lay::kHs;
 #pragma unroll
         for (int cc = 0; cc < PW; cc += 16) {
@@ -273,9 +283,10 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
     };
     auto issue_Yo = [&](int c) {
         const uint32_t aC = sbase + Lay::kC + (c & 1) * 32768;
+        const uint32_t col = kColYo + uint32_t(c & 1) * 128u;
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk)
-            umma_bf16(tb + kColYo, umma_desc_mnmajor(aC, N, kk), umma_desc_mnmajor(aHs, N, kk),
+            umma_bf16(tb + col, umma_desc_mnmajor(aC, N, kk), umma_desc_mnmajor(aHs, N, kk),
                       idYo, kk > 0);
         umma_commit(&bar_yo);
     };
@@ -306,7 +317,9 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
 
         // ---- 1. x * w for the state product, w_s = 2^(cs_Q - cs_s) delta_s
         //         = 2^(cs_Q - cs_e) s_sg[s]; units of (p, 8 tokens)
+        const float *s_cs = s_cs2[c & 1], *s_n2 = s_n22[c & 1], *s_sg = s_sg2[c & 1];
         ok = mbar_wait(&bar_tma[buf], tph, p.timeout_ns) && ok;
+        ok = mbar_wait(&bar_yo, ph, p.timeout_ns) && ok;  // Yo(c) has read the bf16 state
         {
             const float csQ = s_cs[Q - 1];
             uint8_t *xw = smem + Lay::kXw;
@@ -336,6 +349,8 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
         // the state product h += B (x w)^T runs while the mask is built
         fence_proxy_async_smem();
         tmem_fence_before_sync();
+        if (tid == 0)
+            bulk_wait_read<0>();  // the previous chunk's y tile has left the M buffer
         __syncthreads();
         if (tid == 0) {
             tmem_fence_after_sync();
@@ -345,9 +360,15 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                           idYd, 1u);
             umma_commit(&bar_st);
         }
-        // ---- 2. M: row t = r, pieces q = wg + NWG * j of 16 columns
+        // ---- 2. the next chunk's step sizes (second warpgroup, into the other
+        //         set), then M: row t = r, pieces q = wg + NWG * j of 16 columns
+        if (c + 1 < p.nchunks) {
+            cumsum(c + 1, dt_next);
+            if (wg == 1)
+                dt_next = (t0 + 2 * Q + r < p.L) ? dt_row[t0 + 2 * Q + r] : 0.f;
+        }
         const float cs_t = s_cs[r];
-        const float ey = ex2_approx(cs_t);  // Yo row scale, used in step 5
+        const float ey = ex2_approx(cs_t);  // Yo row scale, used in step 4
         ok = mbar_wait(&bar_g, ph, p.timeout_ns) && ok;
         tmem_fence_after_sync();
         {
@@ -398,7 +419,7 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
         fence_proxy_async_smem();
         tmem_fence_before_sync();
         __syncthreads();
-        // ---- 3. Yd = M x^T; then the next chunk's C^T B
+        // ---- Yd = M x^T; then the next chunk's C^T B
         if (tid == 0) {
             tmem_fence_after_sync();
 #pragma unroll
@@ -413,58 +434,16 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
                 issue_G(c + 1);
             }
         }
-        // ---- 4. step sizes of the next chunk (the per-token arrays are free
-        //         once every thread has passed the barrier above)
-        if (c + 1 < p.nchunks) {
-            cumsum(c + 1, dt_next);
-            if (wg == 1)
-                dt_next = (t0 + 2 * Q + r < p.L) ? dt_row[t0 + 2 * Q + r] : 0.f;
-        }
-        // ---- 5. y for token t = r, columns p of this warpgroup's slice
-        ok = mbar_wait(&bar_yo, ph, p.timeout_ns) && ok;
-        ok = mbar_wait(&bar_yd, ph, p.timeout_ns) && ok;
-        tmem_fence_after_sync();
-        {
-            uint8_t *ys = smem + Lay::kM;  // Yd has finished reading M
-            const bool valid = t0 + r < p.L;
-            const __nv_bfloat16 *zrow =
-                GATE ? p.z + int64_t(b) * p.z_bs + int64_t(hh * P) * p.z_cs + t0 + r : nullptr;
-#pragma unroll
-            for (int cc = 0; cc < PW; cc += 16) {
-                const int pbase = wg * PW + cc;
-                float yd[16], yo[16];
-                tmem_ld16x2(tb + lane_off + kColYd + pbase, yd, tb + lane_off + kColYo + pbase, yo);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t off = off8[i & 7] + uint32_t(pbase + i) * 128u;
-                    const float xv = __uint_as_float(
-                        uint32_t(*reinterpret_cast<const uint16_t *>(xs + off)) << 16);
-                    float v = fmaf(ey, yo[i], yd[i]);
-                    v = fmaf(dsk, xv, v);
-                    if (GATE) {
-                        const float zv =
-                            valid ? __bfloat162float(zrow[int64_t(pbase + i) * p.z_cs]) : 0.f;
-                        v *= zv / (1.f + __expf(-zv));
-                    }
-                    *reinterpret_cast<__nv_bfloat16 *>(ys + off) = __float2bfloat16_rn(v);
-                }
-            }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_3d(&tm_Y, smem + Lay::kM, t0, hh * P, b);
-            if (t0 + 64 < p.L)
-                tma_store_3d(&tm_Y, smem + Lay::kM + 8192, t0 + 64, hh * P, b);
-            bulk_commit();
-        }
-        // ---- 6. state n = r: bf16 copy for Yo(c+1), final state, decay into chunk c+1
+        // ---- 3. state n = r (while Yd runs): bf16 copy for Yo(c+1) (over
+        //         x*w, which the state product has read), final state, decay
+        //         into chunk c+1
         ok = mbar_wait(&bar_st, ph, p.timeout_ns) && ok;
         tmem_fence_after_sync();
         {
             uint8_t *hs = smem + Lay::kHs;
             const bool last = c == p.nchunks - 1;
-            const float alpha = last ? 1.f : ex2_approx(s_cs[Q - 1]);  // chunk c+1's decay
+            // chunk c+1's decay (its step sizes were prepared in step 2)
+            const float alpha = last ? 1.f : ex2_approx(s_cs2[(c + 1) & 1][Q - 1]);
             float *ls = (p.last_state && last)
                             ? p.last_state + (int64_t(b) * p.H + hh) * P * N + r
                             : nullptr;
@@ -492,14 +471,51 @@ ssd_scalarA_kernel(const __grid_constant__ CUtensorMap tm_C,
         }
         fence_proxy_async_smem();
         tmem_fence_before_sync();
-        if (tid == 0)
-            bulk_wait_read<0>();  // the y tile has left the M buffer
         __syncthreads();
-        // ---- 7. Yo(c+1) from the new bf16 state; chunk c+2 into this buffer
-        if (tid == 0) {
+        if (tid == 0 && c + 1 < p.nchunks) {
             tmem_fence_after_sync();
-            if (c + 1 < p.nchunks)
-                issue_Yo(c + 1);
+            issue_Yo(c + 1);  // runs during this chunk's epilogue
+        }
+        // ---- 4. y for token t = r, columns p of this warpgroup's slice
+        ok = mbar_wait(&bar_yd, ph, p.timeout_ns) && ok;
+        tmem_fence_after_sync();
+        {
+            uint8_t *ys = smem + Lay::kM;  // Yd has finished reading M
+            const bool valid = t0 + r < p.L;
+            const uint32_t colYo = kColYo + uint32_t(c & 1) * 128u;
+            const __nv_bfloat16 *zrow =
+                GATE ? p.z + int64_t(b) * p.z_bs + int64_t(hh * P) * p.z_cs + t0 + r : nullptr;
+#pragma unroll
+            for (int cc = 0; cc < PW; cc += 16) {
+                const int pbase = wg * PW + cc;
+                float yd[16], yo[16];
+                tmem_ld16x2(tb + lane_off + kColYd + pbase, yd, tb + lane_off + colYo + pbase, yo);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t off = off8[i & 7] + uint32_t(pbase + i) * 128u;
+                    const float xv = __uint_as_float(
+                        uint32_t(*reinterpret_cast<const uint16_t *>(xs + off)) << 16);
+                    float v = fmaf(ey, yo[i], yd[i]);
+                    v = fmaf(dsk, xv, v);
+                    if (GATE) {
+                        const float zv =
+                            valid ? __bfloat162float(zrow[int64_t(pbase + i) * p.z_cs]) : 0.f;
+                        v *= zv / (1.f + __expf(-zv));
+                    }
+                    *reinterpret_cast<__nv_bfloat16 *>(ys + off) = __float2bfloat16_rn(v);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tmem_fence_before_sync();
+        __syncthreads();
+        // ---- y out; chunk c+2 into this chunk's buffer (x, B and C of
+        //      chunk c are no longer read: Yd, the state product and Yo(c) are done)
+        if (tid == 0) {
+            tma_store_3d(&tm_Y, smem + Lay::kM, t0, hh * P, b);
+            if (t0 + 64 < p.L)
+                tma_store_3d(&tm_Y, smem + Lay::kM + 8192, t0 + 64, hh * P, b);
+            bulk_commit();
             if (c + 2 < p.nchunks) {
                 fence_proxy_async_smem();
                 issue_loads(c + 2);
