@@ -46,7 +46,7 @@ NCU_TRAFFIC = {
     2: ("scan_diag_bf16_kernel lane-per-channel v6", 640.3e6),
     # config 3 (two-pass form, both kernels of one call) captured at
     # L = 32768, scaled by tokens to L = 131072
-    3: ("scan_diag_bf16_kernel two-pass v1", 2679.6e6),
+    3: ("scan_diag_bf16_kernel lane-per-channel two-pass v6", 2678.5e6),
     4: ("ssd_scalarA_kernel v5", 107.9e6),
 }
 KERNEL_TAG = {2: "scan_diag_bf16_kernel lane-per-channel v6",
