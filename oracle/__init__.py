@@ -279,3 +279,48 @@ def ssd_chunked(x, dt, A, B, C, headdim, chunk, D=None, z=None, dt_bias=None,
         y.ctypes.data_as(_dp), hs.ctypes.data_as(_dp), int(chunk))
     _check(rc)
     return y, hs
+
+
+def selscan_scalarA_bwd(x, dt, A, B, C, headdim, dy, D=None, z=None, dt_bias=None,
+                        dt_softplus=False, h0=None, dlast=None):
+    """Gradients of the scalar-A scan (``selscan_scalarA``) in fp64 for the
+    loss sum(dy * y) + sum(dlast * last_state).
+
+    "Mamba-3: un modelo de espacio de estados centrado en la inferencia",
+    first section: Mamba-2's transition is one scalar per head times the
+    identity.  The scalar-A scan is therefore the diagonal scan with
+    A[d, n] = A[h] for every channel d = h * P + p of head h and every state,
+    the step size dt[b, h, t] (and dt_bias[h], D[h]) repeated over the head's
+    P channels, and B / C of the head's group; its gradients are those of
+    that diagonal problem (``selscan_bwd``) with every repeated parameter's
+    gradient summed over the channels that share it (the chain rule for a
+    copy).  Shapes as in ``selscan_scalarA``; dy like x; dlast like h0
+    (batch, H, P, N).  Returns a dict with dx (like x), ddt (like dt), dA
+    (H,), dB, dC (like B), and dD, dz, ddt_bias, dh0 (None where the input
+    is None)."""
+    x = np.asarray(x)
+    batch, dim, L = x.shape
+    A = np.asarray(A, dtype=np.float64)
+    H = A.shape[0]
+    P = int(headdim)
+    if dim != H * P:
+        raise ValueError("x.shape[1] must equal nheads * headdim")
+    B4 = _bc4(B, batch)
+    N = B4.shape[2]
+    rep = lambda v: None if v is None else np.repeat(np.asarray(v, np.float64), P, axis=0)
+    delta = np.repeat(np.asarray(dt, np.float64), P, axis=1)
+    A_full = np.repeat(A, P)[:, None] * np.ones((1, N))
+    flat = lambda s: None if s is None else np.asarray(s, np.float64).reshape(batch, dim, N)
+    g = selscan_bwd(x, delta, A_full, B, C, dy, D=rep(D), z=z, delta_bias=rep(dt_bias),
+                    delta_softplus=dt_softplus, h0=flat(h0), dlast=flat(dlast))
+    per_head = lambda v: None if v is None else v.reshape(H, P, *v.shape[1:]).sum(axis=1)
+    return {
+        "dx": g["du"],
+        "ddt": g["ddelta"].reshape(batch, H, P, L).sum(axis=2),
+        "dA": g["dA"].reshape(H, P * N).sum(axis=1),
+        "dB": g["dB"], "dC": g["dC"],
+        "dD": per_head(g["dD"]),
+        "dz": g["dz"],
+        "ddt_bias": per_head(g["ddelta_bias"]),
+        "dh0": None if g["dh0"] is None else g["dh0"].reshape(batch, H, P, N),
+    }

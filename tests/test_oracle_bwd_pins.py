@@ -86,3 +86,67 @@ def test_zero_upstream_gradient_gives_zero():
     for k, v in g.items():
         if v is not None:
             assert np.all(v == 0.0), k
+
+
+# ---------------------------------------------------------------- scalar A
+
+def _sa_inputs(rng, batch, H, P, N, L, G, gate, D, bias, h0):
+    f = lambda *s: rng.standard_normal(s)
+    return dict(x=f(batch, H * P, L), dt=np.exp(rng.uniform(-3.0, -0.5, (batch, H, L))),
+                A=-np.exp(rng.uniform(-1.0, 1.0, H)),
+                B=f(batch, G, N, L), C=f(batch, G, N, L),
+                D=f(H) if D else None, z=f(batch, H * P, L) if gate else None,
+                dt_bias=0.3 * f(H) if bias else None,
+                h0=f(batch, H, P, N) if h0 else None)
+
+
+def _sa_loss(inp, P, dy, dlast, softplus):
+    y, hs = oracle.selscan_scalarA(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], P,
+                                   D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"],
+                                   dt_softplus=softplus, h0=inp["h0"])
+    val = float(np.sum(dy * y))
+    if dlast is not None:
+        val += float(np.sum(dlast * hs))
+    return val
+
+
+@pytest.mark.parametrize("gate,softplus,D,bias,h0,G", [
+    (True, True, True, True, True, 1),
+    (False, False, True, False, False, 1),
+    (False, True, False, True, True, 2),
+])
+def test_scalarA_gradients_equal_finite_differences(gate, softplus, D, bias, h0, G):
+    """oracle.selscan_scalarA_bwd against central differences of the
+    scalar-A forward oracle (its own recurrence over heads, not the diagonal
+    code): every entry of every gradient, including the per-head sums that
+    the broadcast reading produces (dt, A, D, dt_bias shared by a head's
+    channels; B, C shared by a group's heads)."""
+    rng = np.random.default_rng(31 + G + 2 * gate + 4 * softplus)
+    batch, H, P, N, L = 2, 2, 2, 3, 5
+    inp = _sa_inputs(rng, batch, H, P, N, L, G, gate, D, bias, h0)
+    dy = rng.standard_normal((batch, H * P, L))
+    dlast = rng.standard_normal((batch, H, P, N)) if h0 else None
+    grads = oracle.selscan_scalarA_bwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], P, dy,
+                                       D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"],
+                                       dt_softplus=softplus, h0=inp["h0"], dlast=dlast)
+    names = {"x": "dx", "dt": "ddt", "A": "dA", "B": "dB", "C": "dC", "D": "dD", "z": "dz",
+             "dt_bias": "ddt_bias", "h0": "dh0"}
+    checked = 0
+    for key, gname in names.items():
+        if inp[key] is None:
+            assert grads[gname] is None
+            continue
+        v = inp[key]
+        fd = np.zeros_like(v)
+        for idx in np.ndindex(v.shape):
+            keep = v[idx]
+            v[idx] = keep + EPS
+            lp = _sa_loss(inp, P, dy, dlast, softplus)
+            v[idx] = keep - EPS
+            lm = _sa_loss(inp, P, dy, dlast, softplus)
+            v[idx] = keep
+            fd[idx] = (lp - lm) / (2 * EPS)
+        got = np.asarray(grads[gname]).reshape(v.shape)
+        np.testing.assert_allclose(got, fd, rtol=1e-6, atol=1e-7, err_msg=gname)
+        checked += v.size
+    assert checked > 100
