@@ -317,6 +317,48 @@ SELSCAN_API selscan_status selscan_bwd(
     selscan_tensor *dh0, cudaStream_t stream);
 
 /*
+ * selscan_bwd_scalarA -- gradients of selscan_fwd_scalarA_h0 (scalar A per
+ * head, Mamba-2 / SSD form) for the loss
+ *     sum(dy * y) + sum(dlast * last_state).
+ * Training differentiates the forward recurrence ("03 -- Modelos de espacio
+ * de estados", sections "Discretizacion" and "Parallel scan"; "P20 --
+ * Mamba", section 5); with one scalar transition per head ("Mamba-3",
+ * first section) the scan of a chunk of tokens is a masked product of
+ * matrices ("Mamba-2 y state-space models", section 4.2), and this call
+ * differentiates that chunked form from the last chunk to the first.  The
+ * result equals the diagonal-A gradients of the same scan with A, the step
+ * size, D and dt_bias repeated over each head's channels, summed back per
+ * head.
+ *
+ * Forward inputs exactly as selscan_fwd_scalarA_h0 (x, dt, dt_bias,
+ * dt_softplus, A, B, C, D, z, headdim, h0; B / C with time stride 1).
+ *   dy         (batch, H*P, L)   BF16, like x: gradient of y
+ *   dlast      (batch, H, P, N)  F32, contiguous; may be NULL (zero)
+ * Outputs (all overwritten):
+ *   dx         (batch, H*P, L)   BF16, like x
+ *   dz         (batch, H*P, L)   BF16; required iff z is given
+ *   ddt        (batch, H, L)     F32, time stride 1 (gradient of the raw dt)
+ *   dA         (H)               F32
+ *   dB, dC     (batch, G, N, L)  F32, contiguous (sums over a group's heads)
+ *   dD, ddt_bias (H)             F32; may be NULL (not computed)
+ *   dh0        (batch, H, P, N)  F32; may be NULL (not computed)
+ * Built for N = 128, P = 64 (as the forward); other sizes return
+ * SELSCAN_ERR_UNSUPPORTED.  Scratch from the stream-ordered pool: the state
+ * at every 32-token chunk start (batch * H * (ceil(L/32) + 1) * 32 KiB) and
+ * 8 partial copies of dB and dC (2 * 8 * batch * G * L * N * 4 bytes).
+ * Sums over heads and batch rows use fp32 atomics, so the last bits of dA,
+ * dB, dC, dD and ddt_bias depend on the order of the additions.
+ */
+SELSCAN_API selscan_status selscan_bwd_scalarA(
+    const selscan_tensor *x, const selscan_tensor *dt, const selscan_tensor *dt_bias,
+    int dt_softplus, const selscan_tensor *A, const selscan_tensor *B, const selscan_tensor *C,
+    const selscan_tensor *D, const selscan_tensor *z, int64_t headdim, const selscan_tensor *h0,
+    const selscan_tensor *dy, const selscan_tensor *dlast, selscan_tensor *dx,
+    selscan_tensor *ddt, selscan_tensor *dA, selscan_tensor *dB, selscan_tensor *dC,
+    selscan_tensor *dD, selscan_tensor *dz, selscan_tensor *ddt_bias, selscan_tensor *dh0,
+    cudaStream_t stream);
+
+/*
  * selscan_check -- synchronise `stream` and report device-side errors that
  * earlier calls recorded (a bounded wait that gave up returns
  * SELSCAN_ERR_TIMEOUT; the record is then cleared).  Returns
@@ -336,7 +378,8 @@ SELSCAN_API int selscan_version(void);
  * or two when it uses the two-pass form (few channel tiles, long
  * sequences); selscan_bwd launches two (three with time segments: the
  * segment aggregates, the gradient walk, the sum of the dB / dC partial
- * copies); the other entry points launch one.  Benchmarks read it around
+ * copies); selscan_bwd_scalarA launches three (chunk states, the chunk
+ * walk, the sum of the dB / dC copies); the other entry points launch one.  Benchmarks read it around
  * a timed region to report how many of the library's kernels ran in it.
  */
 SELSCAN_API unsigned long long selscan_launch_count(void);

@@ -89,6 +89,9 @@ def lib() -> ctypes.CDLL:
                                            ctypes.c_int64, P, ctypes.c_void_p]
         L.selscan_step_scalarA.restype = ctypes.c_int
         L.selscan_bwd.argtypes = [P, P, P, ctypes.c_int] + [P] * 17 + [ctypes.c_void_p]
+        L.selscan_bwd_scalarA.argtypes = ([P, P, P, ctypes.c_int] + [P] * 5 +
+                                          [ctypes.c_int64] + [P] * 12 + [ctypes.c_void_p])
+        L.selscan_bwd_scalarA.restype = ctypes.c_int
         L.selscan_bwd.restype = ctypes.c_int
         L.selscan_release_scratch.argtypes = []
         L.selscan_release_scratch.restype = ctypes.c_int
@@ -313,6 +316,48 @@ def selscan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
                            _stream_handle(stream))
     if rc != 0:
         raise SelscanError(rc, "selscan_bwd")
+    return out
+
+
+def selscan_bwd_scalarA(x, dt, A, B, C, headdim, dy, D=None, z=None, dt_bias=None,
+                        dt_softplus=False, h0=None, dlast=None, need_dh0=None, stream=None):
+    """Gradients of selscan_fwd_scalarA for sum(dy * y) + sum(dlast *
+    last_state).  Returns a dict: dx (like x), dz (like x, or None), ddt
+    (batch, H, L) fp32, dA (H,), dB, dC (batch, G, N, L) fp32, dD, ddt_bias
+    (H,) fp32 or None, dh0 (batch, H, P, N) fp32 or None (computed when h0 is
+    given or need_dh0).  B / C may be (batch, N, L) (one group)."""
+    import torch
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    batch, dim, L = x.shape
+    H = A.shape[0]
+    if B.dim() == 3:
+        B = B.unsqueeze(1)
+        C = C.unsqueeze(1)
+    G, N = B.shape[1], B.shape[2]
+    out = {
+        "dx": torch.empty(x.shape, dtype=x.dtype, device=dev),
+        "dz": torch.empty(x.shape, dtype=x.dtype, device=dev) if z is not None else None,
+        "ddt": torch.empty((batch, H, L), **f32),
+        "dA": torch.empty((H,), **f32),
+        "dB": torch.empty((batch, G, N, L), **f32),
+        "dC": torch.empty((batch, G, N, L), **f32),
+        "dD": torch.empty((H,), **f32) if D is not None else None,
+        "ddt_bias": torch.empty((H,), **f32) if dt_bias is not None else None,
+        "dh0": torch.empty((batch, H, int(headdim), N), **f32)
+        if (h0 is not None or need_dh0) else None,
+    }
+    ins = [describe(t) for t in (x, dt, dt_bias)]
+    mid = [describe(t) for t in (A, B, C, D, z)]
+    tail = [describe(t) for t in (h0, dy, dlast)]
+    outs = [describe(out[k]) for k in ("dx", "ddt", "dA", "dB", "dC", "dD", "dz",
+                                       "ddt_bias", "dh0")]
+    rc = lib().selscan_bwd_scalarA(_ref(ins[0]), _ref(ins[1]), _ref(ins[2]),
+                                   int(bool(dt_softplus)), *[_ref(t) for t in mid],
+                                   ctypes.c_int64(int(headdim)), *[_ref(t) for t in tail],
+                                   *[_ref(t) for t in outs], _stream_handle(stream))
+    if rc != 0:
+        raise SelscanError(rc, "selscan_bwd_scalarA")
     return out
 
 

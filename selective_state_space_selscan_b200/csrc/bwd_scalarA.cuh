@@ -1,0 +1,643 @@
+// bwd_scalarA.cuh -- gradients of the scalar-A (Mamba-2 / SSD) scan, sm_100a.
+//
+// Training differentiates the recurrence of the forward pass ("03 -- Modelos
+// de espacio de estados", sections "Discretizacion" and "Parallel scan";
+// "P20 -- Mamba", section 5).  With a scalar transition per head ("Mamba-3",
+// first section) the forward pass over a chunk of Q tokens has the matrix
+// form of structured state-space duality ("Mamba-2 y state-space models",
+// section 4.2); this file differentiates that form chunk by chunk, from the
+// last chunk to the first.
+//
+// Per head (state h: N x P), chunk tokens t, s = 0 .. Q-1, cs_t = A sum_{r<=t}
+// delta_r (from the chunk start), L[t,s] = e^(cs_t - cs_s) for s <= t, else 0,
+// G = C^T B (G[t,s] = C_t . B_s), h_0 the state entering the chunk, and dh_Q
+// the gradient of the state leaving it:
+//   forward   y~_t = sum_s L[t,s] G[t,s] delta_s x_s + e^cs_t C_t^T h_0
+//             y_t  = (y~_t + D x_t) silu(z_t)
+//             h_Q  = e^cs_Q h_0 + sum_s e^(cs_Q - cs_s) delta_s B_s x_s^T
+//   backward  dout = dy silu(z),  dz = dy (y~ + D x) silu'(z)
+//             u_s  = sum_t L[t,s] G[t,s] dout_t + e^(cs_Q - cs_s) B_s^T dh_Q   (P)
+//             dx_s = delta_s u_s + D dout_s
+//             dC_t = sum_s L[t,s] delta_s (dout_t . x_s) B_s + e^cs_t h_0 dout_t
+//             dB_s = delta_s (sum_t L[t,s] (dout_t . x_s) C_t + e^(cs_Q - cs_s) dh_Q x_s)
+//             dh_0 = e^cs_Q dh_Q + sum_t e^cs_t C_t dout_t^T
+//             dcs_t = dout_t . y~_t - delta_t (x_t . u_t)  [+ <dh_Q, h_Q> for t = Q-1]
+//             ddelta_s = x_s . u_s + A sum_{t>=s} dcs_t,   dA += sum_t dcs_t S_t
+// (S_t = sum_{r<=t} delta_r), then d(dt) = ddelta sigmoid(dt + bias) under the
+// softplus.  Every term is the chain rule of one factor of the forward form:
+// the exponentials carry cs_t with a plus sign where t is the output token
+// and a minus sign where it is the source token, which is what dcs collects.
+//
+// Two kernels, one CTA of 256 threads per (batch, head):
+//   ssd_bwd_states_kernel runs the forward state recurrence chunk by chunk
+//     and stores h at every chunk start (and the final state) in scratch;
+//   ssd_bwd_kernel walks the chunks backwards with dh in registers and
+//     evaluates the products above from shared memory (fp32 CUDA cores;
+//     32-token chunks keep every product's operands on chip).
+// dB and dC sum over the heads of a group: each head adds its chunk terms
+// with 16-byte atomics into one of kSbCopies partial copies ([t][n] rows),
+// and ssd_bwd_reduce_bc sums the copies into (batch, G, N, L).  dA, dD and
+// the bias gradient sum over batch rows: one atomic per CTA.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace selscan {
+
+constexpr int kSbN = 128;       // state size built
+constexpr int kSbP = 64;        // head dimension built
+constexpr int kSbQ = 32;        // tokens per chunk
+constexpr int kSbThreads = 256;
+constexpr int kSbCopies = 8;    // partial copies of dB / dC (head h adds into copy h % 8)
+
+struct SsdBwdParams {
+    int batch, H, L, nchunks, heads_per_group, G;
+    const __nv_bfloat16 *x, *dy, *z;  // (batch, H*P, L), time stride 1
+    int64_t x_bs, x_cs, dy_bs, dy_cs, z_bs, z_cs;
+    const float *dt;                  // (batch, H, L), time stride 1
+    int64_t dt_bs, dt_hs;
+    const float *dt_bias;             // (H) or null
+    int softplus;
+    const float *A, *Dskip;           // (H); Dskip may be null
+    const __nv_bfloat16 *B, *C;       // (batch, G, N, L), time stride 1
+    int64_t B_bs, B_gs, B_ns, C_bs, C_gs, C_ns;
+    const float *h0, *dlast;          // (batch, H, P, N) contiguous, or null
+    __nv_bfloat16 *dx, *dz;           // like x; dz null without gate
+    int64_t dx_bs, dx_cs, dz_bs, dz_cs;
+    float *ddt;                       // (batch, H, L), time stride 1
+    int64_t ddt_bs, ddt_hs;
+    float *dA, *dD, *ddt_bias;        // (H), accumulated; dD / ddt_bias may be null
+    float *dh0;                       // (batch, H, P, N) or null
+    float *pB, *pC;                   // [kSbCopies][batch][G][L][N], zeroed
+    float *states;                    // [batch*H][nchunks+1][256 threads][32]
+};
+
+// Thread ownership of an N x P state matrix: thread tid holds rows
+// n = 4 (tid % 32) + i (i < 4) and columns p = 8 (tid / 32) + j (j < 8).
+struct SbOwn {
+    int nb, pb;
+    __device__ __forceinline__ explicit SbOwn(int tid) : nb(tid & 31), pb(tid >> 5) {}
+};
+
+__device__ __forceinline__ float sb_bf(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Step sizes of a chunk (one warp, lane = token): delta, the raw argument
+// (for the softplus derivative) and the prefix sum S (inclusive).
+__device__ __forceinline__ void sb_steps(const SsdBwdParams &p, int b, int hh, int t0, int valid,
+                                         int lane, float bias, float &raw, float &dl, float &S)
+{
+    raw = 0.f;
+    dl = 0.f;
+    if (lane < valid) {
+        raw = p.dt[int64_t(b) * p.dt_bs + int64_t(hh) * p.dt_hs + t0 + lane] + bias;
+        dl = p.softplus ? (raw > 20.f ? raw : log1pf(expf(raw))) : raw;
+    }
+    S = dl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, S, o);
+        if (lane >= o)
+            S += v;
+    }
+}
+
+// Chunk rows of a (.., N, L) bf16 tensor into smem as fp32 [t][N]: thread
+// tid reads row n = tid / 2, tokens 16 (tid % 2) .. + 15.
+__device__ __forceinline__ void sb_load_nt(float (*dst)[kSbN], const __nv_bfloat16 *row0,
+                                           int64_t ns, int t0, int valid, int tid)
+{
+    const int n = tid >> 1, half = tid & 1;
+    const __nv_bfloat16 *src = row0 + int64_t(n) * ns + t0 + 16 * half;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int t = 16 * half + k;
+        dst[t][n] = t < valid ? sb_bf(src[k]) : 0.f;
+    }
+}
+
+// Chunk rows of a (.., P, L) bf16 tensor (row stride cs) into smem as fp32
+// [t][P]: thread tid reads row p = tid / 4, tokens 8 (tid % 4) .. + 7.
+__device__ __forceinline__ void sb_load_pt(float (*dst)[kSbP], const __nv_bfloat16 *row0,
+                                           int64_t cs, int t0, int valid, int tid)
+{
+    const int pp = tid >> 2, q = tid & 3;
+    const __nv_bfloat16 *src = row0 + int64_t(pp) * cs + t0 + 8 * q;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int t = 8 * q + k;
+        dst[t][pp] = t < valid ? sb_bf(src[k]) : 0.f;
+    }
+}
+
+// ------------------------------------------------------------ forward states
+__global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const SsdBwdParams p)
+{
+    constexpr int Q = kSbQ, N = kSbN, P = kSbP;
+    __shared__ __align__(16) float Bs[Q][N];
+    __shared__ __align__(16) float xs[Q][P];
+    __shared__ __align__(16) float ws[Q];
+    __shared__ float s_decay;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.x, b = bh / p.H, hh = bh - b * p.H;
+    const int g = hh / p.heads_per_group;
+    const SbOwn o(tid);
+    const float A = p.A[hh];
+    const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
+
+    float hs[4][8];
+    {
+        const float *h0 = p.h0 ? p.h0 + (int64_t(b) * p.H + hh) * P * N : nullptr;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                hs[i][j] = h0 ? h0[int64_t(8 * o.pb + j) * N + 4 * o.nb + i] : 0.f;
+    }
+    float4 *st = reinterpret_cast<float4 *>(p.states) +
+                 (int64_t(bh) * (p.nchunks + 1) * kSbThreads + tid) * 8;
+    const int64_t chunk_stride = int64_t(kSbThreads) * 8;  // float4 per chunk entry
+    const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
+    const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
+
+    for (int c = 0; c < p.nchunks; ++c) {
+        float4 *sc = st + int64_t(c) * chunk_stride;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; j += 4)
+                sc[i * 2 + j / 4] = make_float4(hs[i][j], hs[i][j + 1], hs[i][j + 2], hs[i][j + 3]);
+        const int t0 = c * Q, valid = min(Q, p.L - t0);
+        sb_load_nt(Bs, Brow, p.B_ns, t0, valid, tid);
+        sb_load_pt(xs, xrow, p.x_cs, t0, valid, tid);
+        if (warp == 0) {
+            float raw, dl, S;
+            sb_steps(p, b, hh, t0, valid, lane, bias, raw, dl, S);
+            const float SQ = __shfl_sync(0xffffffffu, S, 31);
+            ws[lane] = expf(A * (SQ - S)) * dl;
+            if (lane == 0)
+                s_decay = expf(A * SQ);
+        }
+        __syncthreads();
+        const float dec = s_decay;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                hs[i][j] *= dec;
+        for (int s = 0; s < valid; ++s) {
+            const float4 b4 = *reinterpret_cast<const float4 *>(&Bs[s][4 * o.nb]);
+            const float4 x0 = *reinterpret_cast<const float4 *>(&xs[s][8 * o.pb]);
+            const float4 x1 = *reinterpret_cast<const float4 *>(&xs[s][8 * o.pb + 4]);
+            const float w = ws[s];
+            const float bw[4] = {b4.x * w, b4.y * w, b4.z * w, b4.w * w};
+            const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    hs[i][j] = fmaf(bw[i], xv[j], hs[i][j]);
+        }
+        __syncthreads();
+    }
+    float4 *sc = st + int64_t(p.nchunks) * chunk_stride;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; j += 4)
+            sc[i * 2 + j / 4] = make_float4(hs[i][j], hs[i][j + 1], hs[i][j + 2], hs[i][j + 3]);
+}
+
+// ------------------------------------------------------------ chunk walk
+// Shared memory of the walk (fp32).  Rows are padded (68 / 132 floats, 33
+// for the Q x Q matrices) so that the column groups the threads of a warp
+// read at once fall in distinct banks.
+constexpr int kSbXS = kSbP + 4;   // x, dout, dy silu'(z): [t][p]
+constexpr int kSbNS = kSbN + 4;   // B, C: [t][n]; h_0^T, dh^T: [p][n]
+struct SbSmem {
+    float xs[kSbQ][kSbXS], dos[kSbQ][kSbXS], zf[kSbQ][kSbXS];
+    float Bs[kSbQ][kSbNS], Cs[kSbQ][kSbNS];
+    float h0T[kSbP][kSbNS], dhT[kSbP][kSbNS];
+    float Mm[kSbQ][kSbQ + 1], Md[kSbQ][kSbQ + 1], Wm[kSbQ][kSbQ + 1], Vm[kSbQ][kSbQ + 1];
+    float raw[kSbQ], dl[kSbQ], S[kSbQ], ecs[kSbQ], ecq[kSbQ], ddd[kSbQ], dyy[kSbQ];
+    float red[8];
+    float hqdh, ecQ;
+};
+
+// Block sum of one value per thread (every thread gets the total).
+__device__ __forceinline__ float sb_block_sum(float v, float *red, int tid)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();  // red is free
+    if ((tid & 31) == 0)
+        red[tid >> 5] = v;
+    __syncthreads();
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSbThreads / 32; ++w)
+        t += red[w];
+    return t;
+}
+
+// Sum over the 8 consecutive lanes that share a row (lanes 8r .. 8r + 7).
+__device__ __forceinline__ float sb_sum8(float v)
+{
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    return v;
+}
+
+template <bool GATE>
+__global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdParams p)
+{
+    constexpr int Q = kSbQ, N = kSbN, P = kSbP;
+    extern __shared__ __align__(16) uint8_t sb_raw[];
+    SbSmem &sm = *reinterpret_cast<SbSmem *>(sb_raw);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.x, b = bh / p.H, hh = bh - b * p.H;
+    const int g = hh / p.heads_per_group;
+    const SbOwn o(tid);
+    const int r = tid >> 3, cg = tid & 7;  // row (token) and column group of the product phases
+    const float A = p.A[hh];
+    const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
+    const float dsk = p.Dskip ? p.Dskip[hh] : 0.f;
+
+    // gradient of the state leaving the current chunk, thread-owned
+    float dh[4][8];
+    {
+        const float *dl0 = p.dlast ? p.dlast + (int64_t(b) * p.H + hh) * P * N : nullptr;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                dh[i][j] = dl0 ? dl0[int64_t(8 * o.pb + j) * N + 4 * o.nb + i] : 0.f;
+    }
+    const float4 *st = reinterpret_cast<const float4 *>(p.states) +
+                       (int64_t(bh) * (p.nchunks + 1) * kSbThreads + tid) * 8;
+    const int64_t chunk_stride = int64_t(kSbThreads) * 8;
+    const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
+    const __nv_bfloat16 *Crow = p.C + int64_t(b) * p.C_bs + int64_t(g) * p.C_gs;
+    const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
+    const __nv_bfloat16 *dyrow = p.dy + int64_t(b) * p.dy_bs + int64_t(hh) * P * p.dy_cs;
+    const __nv_bfloat16 *zrow =
+        GATE ? p.z + int64_t(b) * p.z_bs + int64_t(hh) * P * p.z_cs : nullptr;
+    float *pB = p.pB + ((int64_t(hh % kSbCopies) * p.batch + b) * p.G + g) * int64_t(p.L) * N;
+    float *pC = p.pC + ((int64_t(hh % kSbCopies) * p.batch + b) * p.G + g) * int64_t(p.L) * N;
+    float accD = 0.f, accA = 0.f, accBias = 0.f;
+
+    for (int c = p.nchunks - 1; c >= 0; --c) {
+        const int t0 = c * Q, valid = min(Q, p.L - t0);
+        // ---- 1. chunk inputs, h_0 and dh_Q transposed, step sizes
+        {
+            const int pp = tid >> 2, q = tid & 3;
+            const int64_t xo = int64_t(pp) * p.x_cs + t0 + 8 * q;
+            const int64_t yo = int64_t(pp) * p.dy_cs + t0 + 8 * q;
+            const int64_t zo = GATE ? int64_t(pp) * p.z_cs + t0 + 8 * q : 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int t = 8 * q + k;
+                const bool in = t < valid;
+                const float xv = in ? sb_bf(xrow[xo + k]) : 0.f;
+                const float dyv = in ? sb_bf(dyrow[yo + k]) : 0.f;
+                float dout = dyv, zfac = 0.f;
+                if (GATE) {
+                    const float zv = in ? sb_bf(zrow[zo + k]) : 0.f;
+                    const float sg = 1.f / (1.f + expf(-zv));
+                    dout = dyv * zv * sg;
+                    zfac = dyv * (sg * (1.f + zv * (1.f - sg)));
+                }
+                sm.xs[t][pp] = xv;
+                sm.dos[t][pp] = dout;
+                if (GATE)
+                    sm.zf[t][pp] = zfac;
+            }
+        }
+        {
+            const int n = tid >> 1, half = tid & 1;
+            const int64_t bo = int64_t(n) * p.B_ns + t0 + 16 * half;
+            const int64_t co = int64_t(n) * p.C_ns + t0 + 16 * half;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int t = 16 * half + k;
+                const bool in = t < valid;
+                sm.Bs[t][n] = in ? sb_bf(Brow[bo + k]) : 0.f;
+                sm.Cs[t][n] = in ? sb_bf(Crow[co + k]) : 0.f;
+            }
+        }
+        float hq = 0.f;  // <dh_Q, h_Q>, this thread's part
+        {
+            const float4 *s0 = st + int64_t(c) * chunk_stride;
+            const float4 *s1 = st + int64_t(c + 1) * chunk_stride;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 a0 = s0[2 * i], a1 = s0[2 * i + 1];
+                const float4 q0 = s1[2 * i], q1 = s1[2 * i + 1];
+                const float h0v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float hqv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    sm.h0T[8 * o.pb + j][4 * o.nb + i] = h0v[j];
+                    sm.dhT[8 * o.pb + j][4 * o.nb + i] = dh[i][j];
+                    hq = fmaf(dh[i][j], hqv[j], hq);
+                }
+            }
+        }
+        if (warp == 0) {
+            float rw, dl, S;
+            sb_steps(p, b, hh, t0, valid, lane, bias, rw, dl, S);
+            const float SQ = __shfl_sync(0xffffffffu, S, 31);
+            sm.raw[lane] = rw;
+            sm.dl[lane] = dl;
+            sm.S[lane] = S;
+            sm.ecs[lane] = expf(A * S);
+            sm.ecq[lane] = expf(A * (SQ - S));
+            if (lane == 0)
+                sm.ecQ = expf(A * SQ);
+        }
+        hq = sb_block_sum(hq, sm.red, tid);  // (its barriers also publish the loads)
+        if (tid == 0)
+            sm.hqdh = hq;
+        __syncthreads();
+
+        // ---- 2. Q x Q products: row t = r, columns s = cg + 8k
+        {
+            float G4[4] = {0.f, 0.f, 0.f, 0.f}, Y4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int n4 = 0; n4 < N / 4; ++n4) {
+                const float4 cv = *reinterpret_cast<const float4 *>(&sm.Cs[r][4 * n4]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 bv = *reinterpret_cast<const float4 *>(&sm.Bs[cg + 8 * k][4 * n4]);
+                    G4[k] = fmaf(cv.x, bv.x, fmaf(cv.y, bv.y, fmaf(cv.z, bv.z, fmaf(cv.w, bv.w, G4[k]))));
+                }
+            }
+#pragma unroll 4
+            for (int p4 = 0; p4 < P / 4; ++p4) {
+                const float4 dv = *reinterpret_cast<const float4 *>(&sm.dos[r][4 * p4]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 xv = *reinterpret_cast<const float4 *>(&sm.xs[cg + 8 * k][4 * p4]);
+                    Y4[k] = fmaf(dv.x, xv.x, fmaf(dv.y, xv.y, fmaf(dv.z, xv.z, fmaf(dv.w, xv.w, Y4[k]))));
+                }
+            }
+            const float St = sm.S[r];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int s = cg + 8 * k;
+                const float Lts = s <= r ? expf(A * (St - sm.S[s])) : 0.f;
+                const float ds = sm.dl[s];
+                const float m = G4[k] * Lts, v = Y4[k] * Lts;
+                sm.Mm[r][s] = m;
+                sm.Md[r][s] = m * ds;
+                sm.Vm[r][s] = v;
+                sm.Wm[r][s] = v * ds;
+            }
+        }
+        __syncthreads();
+
+        // ---- 3a. y~ (row t = r) and u (row s = r), columns p = cg + 8j
+        float yt[8], uu[8];
+        {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                yt[j] = uu[j] = 0.f;
+            for (int k = 0; k < Q; ++k) {
+                const float md = sm.Md[r][k], mm = sm.Mm[k][r];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    yt[j] = fmaf(md, sm.xs[k][cg + 8 * j], yt[j]);
+                    uu[j] = fmaf(mm, sm.dos[k][cg + 8 * j], uu[j]);
+                }
+            }
+            float y2[8], u2[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                y2[j] = u2[j] = 0.f;
+#pragma unroll 2
+            for (int n4 = 0; n4 < N / 4; ++n4) {
+                const float4 cv = *reinterpret_cast<const float4 *>(&sm.Cs[r][4 * n4]);
+                const float4 bv = *reinterpret_cast<const float4 *>(&sm.Bs[r][4 * n4]);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 hv = *reinterpret_cast<const float4 *>(&sm.h0T[cg + 8 * j][4 * n4]);
+                    const float4 gv = *reinterpret_cast<const float4 *>(&sm.dhT[cg + 8 * j][4 * n4]);
+                    y2[j] = fmaf(cv.x, hv.x, fmaf(cv.y, hv.y, fmaf(cv.z, hv.z, fmaf(cv.w, hv.w, y2[j]))));
+                    u2[j] = fmaf(bv.x, gv.x, fmaf(bv.y, gv.y, fmaf(bv.z, gv.z, fmaf(bv.w, gv.w, u2[j]))));
+                }
+            }
+            const float et = sm.ecs[r], eq = sm.ecq[r];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                yt[j] = fmaf(et, y2[j], yt[j]);
+                uu[j] = fmaf(eq, u2[j], uu[j]);
+            }
+        }
+        // row outputs: dx, dz; sums for ddelta and dcs; dD
+        {
+            const bool in = r < valid;
+            const float ds = sm.dl[r];
+            float xu = 0.f, dyy = 0.f;
+            const int64_t row_t = t0 + r;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int pp = cg + 8 * j;
+                const float xv = sm.xs[r][pp], dv = sm.dos[r][pp];
+                xu = fmaf(xv, uu[j], xu);
+                dyy = fmaf(dv, yt[j], dyy);
+                accD = fmaf(dv, xv, accD);
+                if (in) {
+                    p.dx[int64_t(b) * p.dx_bs + int64_t(hh * P + pp) * p.dx_cs + row_t] =
+                        __float2bfloat16_rn(fmaf(ds, uu[j], dsk * dv));
+                    if (GATE)
+                        p.dz[int64_t(b) * p.dz_bs + int64_t(hh * P + pp) * p.dz_cs + row_t] =
+                            __float2bfloat16_rn(sm.zf[r][pp] * fmaf(dsk, xv, yt[j]));
+                }
+            }
+            xu = sb_sum8(xu);
+            dyy = sb_sum8(dyy);
+            if (cg == 0) {
+                sm.ddd[r] = xu;
+                sm.dyy[r] = dyy;
+            }
+        }
+        // ---- 3b. dC (row t = r) and dB (row s = r), columns n = 4 (cg + 8k) + i
+        {
+            float cacc[4][4], bacc[4][4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    cacc[k][i] = bacc[k][i] = 0.f;
+            for (int q = 0; q < Q; ++q) {
+                const float w = sm.Wm[r][q], v = sm.Vm[q][r];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 bv = *reinterpret_cast<const float4 *>(&sm.Bs[q][4 * (cg + 8 * k)]);
+                    const float4 cv = *reinterpret_cast<const float4 *>(&sm.Cs[q][4 * (cg + 8 * k)]);
+                    cacc[k][0] = fmaf(w, bv.x, cacc[k][0]);
+                    cacc[k][1] = fmaf(w, bv.y, cacc[k][1]);
+                    cacc[k][2] = fmaf(w, bv.z, cacc[k][2]);
+                    cacc[k][3] = fmaf(w, bv.w, cacc[k][3]);
+                    bacc[k][0] = fmaf(v, cv.x, bacc[k][0]);
+                    bacc[k][1] = fmaf(v, cv.y, bacc[k][1]);
+                    bacc[k][2] = fmaf(v, cv.z, bacc[k][2]);
+                    bacc[k][3] = fmaf(v, cv.w, bacc[k][3]);
+                }
+            }
+            float c2[4][4], b2[4][4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    c2[k][i] = b2[k][i] = 0.f;
+#pragma unroll 2
+            for (int pp = 0; pp < P; ++pp) {
+                const float dv = sm.dos[r][pp], xv = sm.xs[r][pp];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 hv = *reinterpret_cast<const float4 *>(&sm.h0T[pp][4 * (cg + 8 * k)]);
+                    const float4 gv = *reinterpret_cast<const float4 *>(&sm.dhT[pp][4 * (cg + 8 * k)]);
+                    c2[k][0] = fmaf(dv, hv.x, c2[k][0]);
+                    c2[k][1] = fmaf(dv, hv.y, c2[k][1]);
+                    c2[k][2] = fmaf(dv, hv.z, c2[k][2]);
+                    c2[k][3] = fmaf(dv, hv.w, c2[k][3]);
+                    b2[k][0] = fmaf(xv, gv.x, b2[k][0]);
+                    b2[k][1] = fmaf(xv, gv.y, b2[k][1]);
+                    b2[k][2] = fmaf(xv, gv.z, b2[k][2]);
+                    b2[k][3] = fmaf(xv, gv.w, b2[k][3]);
+                }
+            }
+            if (r < valid) {
+                const float et = sm.ecs[r], eq = sm.ecq[r], ds = sm.dl[r];
+                float4 *dCr = reinterpret_cast<float4 *>(pC + int64_t(t0 + r) * N);
+                float4 *dBr = reinterpret_cast<float4 *>(pB + int64_t(t0 + r) * N);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 vc = make_float4(fmaf(et, c2[k][0], cacc[k][0]),
+                                                  fmaf(et, c2[k][1], cacc[k][1]),
+                                                  fmaf(et, c2[k][2], cacc[k][2]),
+                                                  fmaf(et, c2[k][3], cacc[k][3]));
+                    const float4 vb = make_float4(ds * fmaf(eq, b2[k][0], bacc[k][0]),
+                                                  ds * fmaf(eq, b2[k][1], bacc[k][1]),
+                                                  ds * fmaf(eq, b2[k][2], bacc[k][2]),
+                                                  ds * fmaf(eq, b2[k][3], bacc[k][3]));
+                    atomicAdd(dCr + cg + 8 * k, vc);
+                    atomicAdd(dBr + cg + 8 * k, vb);
+                }
+            }
+        }
+        // ---- 3c. dh_0 = e^cs_Q dh_Q + sum_t e^cs_t C_t dout_t^T (thread-owned)
+        {
+            const float eQ = sm.ecQ;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    dh[i][j] *= eQ;
+            for (int t = 0; t < valid; ++t) {
+                const float4 cv = *reinterpret_cast<const float4 *>(&sm.Cs[t][4 * o.nb]);
+                const float4 d0 = *reinterpret_cast<const float4 *>(&sm.dos[t][8 * o.pb]);
+                const float4 d1 = *reinterpret_cast<const float4 *>(&sm.dos[t][8 * o.pb + 4]);
+                const float et = sm.ecs[t];
+                const float cc[4] = {cv.x * et, cv.y * et, cv.z * et, cv.w * et};
+                const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dh[i][j] = fmaf(cc[i], dd[j], dh[i][j]);
+            }
+        }
+        __syncthreads();
+        // ---- 4. per-token scalars (one warp, lane = token)
+        if (warp == 0) {
+            const bool in = lane < valid;
+            const float ds = sm.dl[lane];
+            float dcs = sm.dyy[lane] - ds * sm.ddd[lane];
+            if (lane == valid - 1)
+                dcs += sm.hqdh;
+            if (!in)
+                dcs = 0.f;
+            float R = dcs;  // sum over t >= lane
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float v = __shfl_down_sync(0xffffffffu, R, off);
+                if (lane + off < 32)
+                    R += v;
+            }
+            const float dd = sm.ddd[lane] + A * R;
+            const float rw = sm.raw[lane];
+            const float ddt = p.softplus ? dd / (1.f + expf(-rw)) : dd;
+            if (in)
+                p.ddt[int64_t(b) * p.ddt_bs + int64_t(hh) * p.ddt_hs + t0 + lane] = ddt;
+            accA = fmaf(dcs, sm.S[lane], accA);
+            accBias += in ? ddt : 0.f;
+        }
+        __syncthreads();
+    }
+
+    // ---- per-head sums (over this batch row), dh0
+    if (p.dh0) {
+        float *d0 = p.dh0 + (int64_t(b) * p.H + hh) * P * N;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                d0[int64_t(8 * o.pb + j) * N + 4 * o.nb + i] = dh[i][j];
+    }
+    const float sD = sb_block_sum(accD, sm.red, tid);
+    const float sA = sb_block_sum(accA, sm.red, tid);
+    const float sBias = sb_block_sum(accBias, sm.red, tid);
+    if (tid == 0) {
+        atomicAdd(p.dA + hh, sA);
+        if (p.dD)
+            atomicAdd(p.dD + hh, sD);
+        if (p.ddt_bias)
+            atomicAdd(p.ddt_bias + hh, sBias);
+    }
+}
+
+// dB, dC (batch, G, N, L) = sum of the kSbCopies partial copies, each
+// [batch][G][L][N].  A block transposes 32 tokens x 128 states through
+// shared memory so that both the reads and the writes are row-contiguous.
+__global__ void __launch_bounds__(256) ssd_bwd_reduce_bc(const float *pB, const float *pC,
+                                                         float *dB, float *dC, int64_t rows,
+                                                         int L)
+{
+    __shared__ float tile[2][32][kSbN + 1];
+    const int64_t bg = blockIdx.y;             // (batch, group) row
+    const int t0 = blockIdx.x * 32;
+    const int64_t copy = rows * int64_t(L) * kSbN;  // floats per partial copy
+    const int tid = threadIdx.x;
+    for (int e = tid; e < 32 * kSbN; e += 256) {
+        const int t = e / kSbN, n = e - t * kSbN;
+        float sb = 0.f, sc = 0.f;
+        if (t0 + t < L) {
+            const int64_t off = (bg * L + t0 + t) * kSbN + n;
+            for (int k = 0; k < kSbCopies; ++k) {
+                sb += pB[k * copy + off];
+                sc += pC[k * copy + off];
+            }
+        }
+        tile[0][t][n] = sb;
+        tile[1][t][n] = sc;
+    }
+    __syncthreads();
+    for (int e = tid; e < 32 * kSbN; e += 256) {
+        const int n = e / 32, t = e - n * 32;
+        if (t0 + t < L) {
+            const int64_t off = (bg * kSbN + n) * L + t0 + t;
+            dB[off] = tile[0][t][n];
+            dC[off] = tile[1][t][n];
+        }
+    }
+}
+
+}  // namespace selscan

@@ -19,6 +19,7 @@
 #include "ssd_scalarA.cuh"
 #include "step.cuh"
 #include "bwd_diag.cuh"
+#include "bwd_scalarA.cuh"
 
 using namespace selscan;
 
@@ -1528,6 +1529,188 @@ extern "C" selscan_status selscan_bwd(
         const int64_t blocks = std::min<int64_t>((rows + 255) / 256, 8ll * di->sm_count);
         bwd_reduce_bc<<<unsigned(blocks), 256, 0, stream>>>(prm.pB, prm.pC, prm.dB, prm.dC,
                                                             rows, int(L));
+        le = counted_launch();
+    }
+    cudaFreeAsync(ws, stream);
+    return le == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+}
+
+extern "C" selscan_status selscan_bwd_scalarA(
+    const selscan_tensor *x, const selscan_tensor *dt, const selscan_tensor *dt_bias,
+    int dt_softplus, const selscan_tensor *A, const selscan_tensor *B, const selscan_tensor *C,
+    const selscan_tensor *D, const selscan_tensor *z, int64_t headdim, const selscan_tensor *h0,
+    const selscan_tensor *dy, const selscan_tensor *dlast, selscan_tensor *dx,
+    selscan_tensor *ddt, selscan_tensor *dA, selscan_tensor *dB, selscan_tensor *dC,
+    selscan_tensor *dD, selscan_tensor *dz, selscan_tensor *ddt_bias, selscan_tensor *dh0,
+    cudaStream_t stream)
+{
+    if (!present(x) || !present(A) || !dt || !B || !C || !dy || !dx || !ddt || !dA || !dB ||
+        !dC)
+        return SELSCAN_ERR_NULL;
+    if (x->ndim != 3 || A->ndim != 1 || headdim <= 0)
+        return SELSCAN_ERR_SHAPE;
+    if (x->dtype != SELSCAN_BF16)
+        return SELSCAN_ERR_DTYPE;
+    const int64_t batch = x->shape[0], dim = x->shape[1], L = x->shape[2];
+    const int64_t H = A->shape[0];
+    if (batch < 0 || L < 0 || H <= 0 || dim != H * headdim)
+        return SELSCAN_ERR_SHAPE;
+    selscan_status st;
+    for (const selscan_tensor *t : {x, dy, static_cast<const selscan_tensor *>(dx)})
+        if ((st = check_seq(t, batch, dim, L, SELSCAN_BF16)) != SELSCAN_OK) return st;
+    const bool gate = z && z->data;
+    if (gate) {
+        if ((st = check_seq(z, batch, dim, L, SELSCAN_BF16)) != SELSCAN_OK) return st;
+        if ((st = check_seq(dz, batch, dim, L, SELSCAN_BF16)) != SELSCAN_OK) return st;
+    }
+    if ((st = check_seq(dt, batch, H, L, SELSCAN_F32)) != SELSCAN_OK) return st;
+    if ((st = check_seq(ddt, batch, H, L, SELSCAN_F32)) != SELSCAN_OK) return st;
+    for (const selscan_tensor *t : {B, C}) {
+        if (!present(t))
+            return SELSCAN_ERR_NULL;
+        if (t->ndim != 4 || t->shape[0] != batch || t->shape[3] != L)
+            return SELSCAN_ERR_SHAPE;
+        if (t->dtype != SELSCAN_BF16)
+            return SELSCAN_ERR_DTYPE;
+        if (L > 1 && t->stride[3] != 1)
+            return SELSCAN_ERR_STRIDE;
+        if (t->stride[0] < 0 || t->stride[1] < 0 || t->stride[2] < 0)
+            return SELSCAN_ERR_STRIDE;
+    }
+    const int64_t G = B->shape[1], N = B->shape[2];
+    if (C->shape[1] != G || C->shape[2] != N || G <= 0 || H % G != 0)
+        return SELSCAN_ERR_SHAPE;
+    {
+        const int64_t hshape[1] = {H};
+        const int64_t sshape[4] = {batch, H, headdim, N};
+        const int64_t bcshape[4] = {batch, G, N, L};
+        if ((st = check_param(A, 1, hshape, false)) != SELSCAN_OK) return st;
+        if ((st = check_param(dA, 1, hshape, false)) != SELSCAN_OK) return st;
+        if ((st = check_param(dt_bias, 1, hshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(D, 1, hshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(dD, 1, hshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(ddt_bias, 1, hshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(h0, 4, sshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(dlast, 4, sshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(dh0, 4, sshape, true)) != SELSCAN_OK) return st;
+        if ((st = check_param(dB, 4, bcshape, false)) != SELSCAN_OK) return st;
+        if ((st = check_param(dC, 4, bcshape, false)) != SELSCAN_OK) return st;
+    }
+    if (N != kSbN || headdim != kSbP)
+        return SELSCAN_ERR_UNSUPPORTED;
+    if (batch * H > 0x7fffffffll || batch * G > 65535 || L > (int64_t(1) << 30))
+        return SELSCAN_ERR_UNSUPPORTED;
+    auto zero = [&](selscan_tensor *t) {
+        return (!t || !t->data || numel(t) == 0)
+                   ? cudaSuccess
+                   : cudaMemsetAsync(t->data, 0, size_t(numel(t)) * 4, stream);
+    };
+    // per-head sums start at zero; dB and dC sum over heads
+    if (zero(dA) != cudaSuccess || zero(dD) != cudaSuccess || zero(ddt_bias) != cudaSuccess)
+        return SELSCAN_ERR_CUDA;
+    if (batch == 0)
+        return SELSCAN_OK;
+    if (L == 0) {
+        if (dh0 && dh0->data) {
+            const size_t bytes = size_t(batch * H * headdim * N) * 4;
+            const cudaError_t e =
+                (dlast && dlast->data)
+                    ? cudaMemcpyAsync(dh0->data, dlast->data, bytes, cudaMemcpyDeviceToDevice,
+                                      stream)
+                    : cudaMemsetAsync(dh0->data, 0, bytes, stream);
+            return e == cudaSuccess ? SELSCAN_OK : SELSCAN_ERR_CUDA;
+        }
+        return SELSCAN_OK;
+    }
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    if ((st = device_setup(&dev, &di)) != SELSCAN_OK)
+        return st;
+
+    SsdBwdParams prm{};
+    prm.batch = int(batch);
+    prm.H = int(H);
+    prm.L = int(L);
+    prm.nchunks = int((L + kSbQ - 1) / kSbQ);
+    prm.heads_per_group = int(H / G);
+    prm.G = int(G);
+    prm.x = static_cast<const __nv_bfloat16 *>(x->data);
+    prm.x_bs = x->stride[0];
+    prm.x_cs = x->stride[1];
+    prm.dy = static_cast<const __nv_bfloat16 *>(dy->data);
+    prm.dy_bs = dy->stride[0];
+    prm.dy_cs = dy->stride[1];
+    prm.z = gate ? static_cast<const __nv_bfloat16 *>(z->data) : nullptr;
+    prm.z_bs = gate ? z->stride[0] : 0;
+    prm.z_cs = gate ? z->stride[1] : 0;
+    prm.dt = static_cast<const float *>(dt->data);
+    prm.dt_bs = dt->stride[0];
+    prm.dt_hs = dt->stride[1];
+    prm.dt_bias = static_cast<const float *>(opt_data(dt_bias));
+    prm.softplus = dt_softplus ? 1 : 0;
+    prm.A = static_cast<const float *>(A->data);
+    prm.Dskip = static_cast<const float *>(opt_data(D));
+    prm.B = static_cast<const __nv_bfloat16 *>(B->data);
+    prm.B_bs = B->stride[0];
+    prm.B_gs = B->stride[1];
+    prm.B_ns = B->stride[2];
+    prm.C = static_cast<const __nv_bfloat16 *>(C->data);
+    prm.C_bs = C->stride[0];
+    prm.C_gs = C->stride[1];
+    prm.C_ns = C->stride[2];
+    prm.h0 = static_cast<const float *>(opt_data(h0));
+    prm.dlast = static_cast<const float *>(opt_data(dlast));
+    prm.dx = static_cast<__nv_bfloat16 *>(dx->data);
+    prm.dx_bs = dx->stride[0];
+    prm.dx_cs = dx->stride[1];
+    prm.dz = gate ? static_cast<__nv_bfloat16 *>(dz->data) : nullptr;
+    prm.dz_bs = gate ? dz->stride[0] : 0;
+    prm.dz_cs = gate ? dz->stride[1] : 0;
+    prm.ddt = static_cast<float *>(ddt->data);
+    prm.ddt_bs = ddt->stride[0];
+    prm.ddt_hs = ddt->stride[1];
+    prm.dA = static_cast<float *>(dA->data);
+    prm.dD = static_cast<float *>(dD ? dD->data : nullptr);
+    prm.ddt_bias = static_cast<float *>(ddt_bias ? ddt_bias->data : nullptr);
+    prm.dh0 = static_cast<float *>(dh0 ? dh0->data : nullptr);
+
+    // scratch: states at every chunk start [batch*H][nchunks+1][8192] and the
+    // partial copies of dB and dC [kSbCopies][batch][G][L][N] (fp32)
+    const size_t st_bytes = size_t(batch * H) * (prm.nchunks + 1) * kSbN * kSbP * 4;
+    const size_t part = size_t(kSbCopies) * batch * G * L * kSbN;  // floats per tensor
+    void *ws = nullptr;
+    if (scratch_alloc(&ws, st_bytes + 2 * part * 4, stream) != cudaSuccess)
+        return SELSCAN_ERR_CUDA;
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    prm.states = reinterpret_cast<float *>(wsb);
+    prm.pB = reinterpret_cast<float *>(wsb + st_bytes);
+    prm.pC = prm.pB + part;
+    if (cudaMemsetAsync(prm.pB, 0, 2 * part * 4, stream) != cudaSuccess) {
+        cudaFreeAsync(ws, stream);
+        return SELSCAN_ERR_CUDA;
+    }
+    auto kern = gate ? ssd_bwd_kernel<true> : ssd_bwd_kernel<false>;
+    static bool attr_set[2][kMaxDevices] = {};
+    if (!attr_set[gate][dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(sizeof(SbSmem))) != cudaSuccess) {
+            cudaFreeAsync(ws, stream);
+            return SELSCAN_ERR_CUDA;
+        }
+        attr_set[gate][dev] = true;
+    }
+    const unsigned grid = unsigned(batch * H);
+    ssd_bwd_states_kernel<<<grid, kSbThreads, 0, stream>>>(prm);
+    cudaError_t le = counted_launch();
+    if (le == cudaSuccess) {
+        kern<<<grid, kSbThreads, sizeof(SbSmem), stream>>>(prm);
+        le = counted_launch();
+    }
+    if (le == cudaSuccess) {
+        const dim3 rg(unsigned((L + 31) / 32), unsigned(batch * G));
+        ssd_bwd_reduce_bc<<<rg, 256, 0, stream>>>(prm.pB, prm.pC, static_cast<float *>(dB->data),
+                                                  static_cast<float *>(dC->data), batch * G,
+                                                  int(L));
         le = counted_launch();
     }
     cudaFreeAsync(ws, stream);

@@ -1,0 +1,117 @@
+"""GPU parity of the scalar-A backward (selscan_bwd_scalarA, through the C
+ABI) with the fp64 oracle's gradients (oracle.selscan_scalarA_bwd, pinned by
+finite differences of the scalar-A forward oracle) on the same seeded,
+bf16-rounded inputs.
+
+Tolerances, relative L2 per gradient as for the diagonal backward: 5e-3 for
+dx and dz (stored in bf16), 2e-3 for the fp32 gradients (ddt, dA, dB, dC,
+dD, ddt_bias, dh0; fp32 products with the special-function unit's exp)."""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+
+pytestmark = pytest.mark.gpu
+
+P, N = 64, 128
+
+
+def rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def _bf(a):
+    import torch
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda().to(torch.bfloat16)
+
+
+def _f32(a):
+    import torch
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda().float()
+
+
+def make(batch, H, L, G=1, seed=0, gate=False, D=True, softplus=False, bias=False, h0=False):
+    inp = synthetic.make_scalarA(batch, H, P, N, L, ngroups=G, seed=seed, gate=gate, D=D)
+    rng = np.random.default_rng(seed + 1000)
+    if softplus:
+        # raw step arguments around softplus^-1 of the configured range
+        inp["dt"] = (np.log(np.expm1(inp["dt"])) + 0.3 * rng.standard_normal(inp["dt"].shape)
+                     ).astype(np.float32)
+    inp["softplus"] = softplus
+    inp["dt_bias"] = (0.2 * rng.standard_normal(H)).astype(np.float32) if bias else None
+    inp["h0"] = rng.standard_normal((batch, H, P, N)).astype(np.float32) if h0 else None
+    inp["dlast"] = rng.standard_normal((batch, H, P, N)).astype(np.float32) if h0 else None
+    inp["dy"] = synthetic.round_bf16(rng.standard_normal(inp["x"].shape).astype(np.float32))
+    return inp
+
+
+def run_gpu(inp):
+    import selective_state_space_selscan_b200 as ss
+    g = ss.selscan_bwd_scalarA(_bf(inp["x"]), _f32(inp["dt"]), _f32(inp["A"]), _bf(inp["B"]),
+                               _bf(inp["C"]), P, _bf(inp["dy"]), D=_f32(inp["D"]),
+                               z=_bf(inp["z"]), dt_bias=_f32(inp["dt_bias"]),
+                               dt_softplus=inp["softplus"], h0=_f32(inp["h0"]),
+                               dlast=_f32(inp["dlast"]))
+    ss.check()
+    return {k: (None if v is None else v.float().cpu().numpy()) for k, v in g.items()}
+
+
+def run_oracle(inp):
+    return oracle.selscan_scalarA_bwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], P,
+                                      inp["dy"], D=inp["D"], z=inp["z"],
+                                      dt_bias=inp["dt_bias"], dt_softplus=inp["softplus"],
+                                      h0=inp["h0"], dlast=inp["dlast"])
+
+
+def compare(got, want, what):
+    for k, w in want.items():
+        if w is None:
+            assert got[k] is None, (what, k)
+            continue
+        assert np.isfinite(got[k]).all(), (what, k)
+        tol = 5e-3 if k in ("dx", "dz") else 2e-3
+        e = rel(got[k].reshape(w.shape), w)
+        assert e <= tol, f"{what} {k}: rel L2 {e:.3e} > {tol}"
+
+
+@pytest.mark.parametrize("L", [24, 96, 200])
+def test_chunks_and_ragged(L):
+    """One partial chunk (L = 24), whole 32-token chunks (96) and a ragged
+    last chunk (200); two batch rows, three heads, D on."""
+    inp = make(2, 3, L, seed=61 + L)
+    compare(run_gpu(inp), run_oracle(inp), f"L={L}")
+
+
+def test_all_options():
+    """Gate, D, dt_bias, softplus, an initial state and a final-state
+    gradient (dh0 checked)."""
+    inp = make(2, 2, 160, seed=71, gate=True, softplus=True, bias=True, h0=True)
+    compare(run_gpu(inp), run_oracle(inp), "all options")
+
+
+def test_groups_no_D():
+    """Two B/C groups over four heads (dB, dC sum over each group's heads);
+    no D, no gate."""
+    inp = make(1, 4, 136, G=2, seed=72, D=False)
+    compare(run_gpu(inp), run_oracle(inp), "G=2")
+
+
+def test_longer_sequence():
+    """32 chunks of 32 tokens: the reverse walk carries dh across many chunk
+    boundaries; eight heads share one group."""
+    inp = make(1, 8, 1024, seed=73, softplus=True, bias=True)
+    compare(run_gpu(inp), run_oracle(inp), "L=1024")
+
+
+def test_zero_upstream_gradient():
+    """dy = 0 and no final-state gradient: every gradient is exactly zero."""
+    inp = make(1, 2, 64, seed=74, gate=True, h0=True)
+    inp["dy"] = np.zeros_like(inp["dy"])
+    inp["dlast"] = None
+    g = run_gpu(inp)
+    for k, v in g.items():
+        if v is not None:
+            assert np.all(v == 0.0), k
