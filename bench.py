@@ -330,10 +330,15 @@ def step_config(cfg: dict, world: int) -> dict:
             "parallelism": f"dp{world} (independent shards, no collective)"}
 
 
+def cfg_dim(cfg: dict) -> int:
+    """d_inner of a config (channels; heads x headdim for scalar A)."""
+    return cfg["dim"] if cfg["kind"] == "diag" else cfg["nheads"] * cfg["headdim"]
+
+
 def bwd_config(cfg: dict, world: int) -> dict:
     """The ``config`` object of a backward line (both arms)."""
     return {"workload": "backward of " + cfg["name"], "batch": cfg["batch"],
-            "d_inner": cfg["dim"], "d_state": cfg["N"], "seq_len": cfg["L"],
+            "d_inner": cfg_dim(cfg), "d_state": cfg["N"], "seq_len": cfg["L"],
             "global_batch": cfg["batch"] * world,
             "l2": "inputs larger than L2 (no flush)" if bwd_bytes(cfg) > 126e6 else
                   "inputs smaller than L2",
@@ -449,11 +454,22 @@ def run_reference_bwd(args, world: int):
     one whole channel (all batches, all tokens) of the workload."""
     cfg = synthetic.CONFIGS[args.config]
     inp = synthetic.make_config(args.config)
-    dy = np.random.default_rng(cfg["seed"] + 500).standard_normal(inp["u"].shape,
-                                                                     dtype=np.float32)
+    scalar = cfg["kind"] == "scalarA"
+    dy = np.random.default_rng(cfg["seed"] + 500).standard_normal(
+        inp["x" if scalar else "u"].shape, dtype=np.float32)
     import oracle
 
     def one(i):
+        if scalar:
+            # one head (its P channels, all batches, all tokens) per step
+            P, hh = cfg["headdim"], i % cfg["nheads"]
+            g = hh // (cfg["nheads"] // cfg["ngroups"])
+            ch = lambda x: None if x is None else x[:, hh * P:(hh + 1) * P]
+            hv = lambda x: None if x is None else x[hh:hh + 1]
+            oracle.selscan_scalarA_bwd(ch(inp["x"]), inp["dt"][:, hh:hh + 1], hv(inp["A"]),
+                                       inp["B"][:, g:g + 1], inp["C"][:, g:g + 1], P,
+                                       ch(dy), D=hv(inp["D"]), z=ch(inp["z"]))
+            return
         c = i % cfg["dim"]
         sl = lambda x: None if x is None else x[:, c:c + 1]
         vec = lambda x: None if x is None else x[c:c + 1]
@@ -471,7 +487,8 @@ def run_reference_bwd(args, world: int):
         if time.perf_counter() - t0 > 150.0:
             break
     dt = time.perf_counter() - t0
-    val = done * cfg["batch"] * cfg["L"] / dt / 1e9
+    per_step = cfg["headdim"] if scalar else 1  # channels per step
+    val = done * per_step * cfg["batch"] * cfg["L"] / dt / 1e9
     print(json.dumps({
         "impl": "reference",
         "metric": "selective-scan backward Gelem/s (B·D·L) and % of B200 HBM roofline, 1 GPU",
@@ -479,9 +496,10 @@ def run_reference_bwd(args, world: int):
         "warmup": args.warmup, "ms_per_step": dt / done * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(bwd_config(cfg, world),
-                       sample_per_step="one channel (all batches, all tokens)"),
+                       sample_per_step=("one head" if scalar else "one channel") +
+                       " (all batches, all tokens)"),
         "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{done} steps x one channel"},
+                         "sample": f"{done} steps x one " + ("head" if scalar else "channel")},
         "e2e": {"value": val, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -848,7 +866,17 @@ def run_step(args, rank: int, world: int, local: int):
 def bwd_bytes(cfg: dict) -> int:
     """Bytes one backward call must move: u, delta, z, dy read and du,
     ddelta, dz written once, B and C read and dB, dC (fp32) written once,
-    the per-channel parameters and their gradients."""
+    the per-channel parameters and their gradients.  Scalar A: x, z, dy read
+    and dx, dz written (bf16), dt read and ddt written (fp32, per head), B
+    and C read (bf16) and dB, dC written (fp32) per group."""
+    if cfg["kind"] == "scalarA":
+        b, H, P, N, L = cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["N"], cfg["L"]
+        G = cfg["ngroups"]
+        total = b * H * P * L * 2 * ((2 if cfg["gate"] else 1) * 2 + 1)   # x, z in+grad; dy
+        total += b * H * L * 8                                             # dt in, ddt out
+        total += 2 * b * G * N * L * (2 + 4)                               # B, C in; dB, dC out
+        total += 4 * H * 4                                                 # A, dA, D, dD
+        return total
     es = 2 if cfg["dtype"] == "bf16" else 4
     b, dim, N, L = cfg["batch"], cfg["dim"], cfg["N"], cfg["L"]
     per_elem = es * (3 if cfg["gate"] else 2) * 2 + es           # (u, delta, z) in+grad, dy
@@ -880,18 +908,26 @@ def run_bwd(args, rank: int, world: int, local: int):
     import selective_state_space_selscan_b200 as ss
     torch.cuda.set_device(local)
     cfg = synthetic.CONFIGS[args.config]
-    if cfg["kind"] != "diag":
-        raise SystemExit("--op bwd runs the diagonal configs (0-3)")
+    scalar = cfg["kind"] == "scalarA"
     inp = synthetic.make_config(args.config, seed=shard_seed(cfg, rank))
     dt = cfg["dtype"]
     stream = torch.cuda.current_stream()
     rng = np.random.default_rng(shard_seed(cfg, rank) + 500)
-    dy_host = rng.standard_normal(inp["u"].shape, dtype=np.float32)
-    dev = {k: to_dev(inp[k], dt, torch) for k in ("u", "delta", "B", "C", "z")}
+    xk = "x" if scalar else "u"
+    dy_host = rng.standard_normal(inp[xk].shape, dtype=np.float32)
+    if scalar:
+        dev = {k: to_dev(inp[k], dt, torch) for k in ("x", "B", "C", "z")}
+        dev["dt"] = to_dev(inp["dt"], "f32", torch)
+        par = {k: to_dev(inp[k], "f32", torch) for k in ("A", "D")}
+    else:
+        dev = {k: to_dev(inp[k], dt, torch) for k in ("u", "delta", "B", "C", "z")}
+        par = {k: to_dev(inp[k], "f32", torch) for k in ("A", "D", "delta_bias")}
     dev["dy"] = to_dev(dy_host, dt, torch)
-    par = {k: to_dev(inp[k], "f32", torch) for k in ("A", "D", "delta_bias")}
 
     def call():
+        if scalar:
+            return ss.selscan_bwd_scalarA(dev["x"], dev["dt"], par["A"], dev["B"], dev["C"],
+                                          inp["headdim"], dev["dy"], D=par["D"], z=dev["z"])
         return ss.selscan_bwd(dev["u"], dev["delta"], par["A"], dev["B"], dev["C"], dev["dy"],
                               D=par["D"], z=dev["z"], delta_bias=par["delta_bias"])
 
@@ -939,14 +975,14 @@ def run_bwd(args, rank: int, world: int, local: int):
     clock_info = clocks.stop(t_wall0, t_wall1) if clocks else None
     total_ms, avg_launch_ms = max_over_ranks([total_ms, avg_launch_ms])
     ms_per_step = total_ms / args.steps
-    elems = cfg["batch"] * cfg["dim"] * cfg["L"]
+    elems = cfg["batch"] * cfg_dim(cfg) * cfg["L"]
     value = aggregate_rate(world, elems, ms_per_step) / 1e9
 
     # end to end: inputs and dy from pinned host memory in, every gradient out
-    host_keys = ("u", "delta", "B", "C", "z", "dy")
+    host_keys = ("x", "dt", "B", "C", "z", "dy") if scalar else ("u", "delta", "B", "C", "z", "dy")
     src = dict(inp, dy=dy_host)
     pinned = {k: torch.from_numpy(np.ascontiguousarray(src[k])).to(
-        torch.bfloat16 if dt == "bf16" else torch.float32).pin_memory()
+        torch.bfloat16 if (dt == "bf16" and k != "dt") else torch.float32).pin_memory()
         for k in host_keys if src.get(k) is not None}
     outs = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
             for k, v in grads.items() if v is not None}
@@ -1003,10 +1039,28 @@ def run_bwd(args, rank: int, world: int, local: int):
 
 def oracle_bwd_sample(cfg: dict, inp: dict, dy: np.ndarray, seconds: float = 10.0):
     """The fp64 oracle's backward on whole channels of the workload (all
-    batches, all tokens), grown until about `seconds` of work; Gelem/s."""
+    batches, all tokens; whole heads for scalar A), grown until about
+    `seconds` of work; Gelem/s."""
     import oracle
     n, spent = 1, 0.0
     b, L = cfg["batch"], cfg["L"]
+    if cfg["kind"] == "scalarA":
+        P, per = cfg["headdim"], cfg["nheads"] // cfg["ngroups"]
+        while True:
+            ch = lambda x: None if x is None else x[:, :n * P]
+            hv = lambda x: None if x is None else x[:n]
+            t0 = time.perf_counter()
+            oracle.selscan_scalarA_bwd(ch(inp["x"]), inp["dt"][:, :n], inp["A"][:n],
+                                       inp["B"][:, :1], inp["C"][:, :1], P, dy[:, :n * P],
+                                       D=hv(inp["D"]), z=ch(inp["z"]))
+            spent = time.perf_counter() - t0
+            if spent >= seconds * 0.5 or n >= per:
+                break
+            n = int(min(per, n * max(2.0, min(16.0, seconds / max(spent, 1e-3)))))
+        return {"value": b * n * P * L / spent / 1e9, "unit": "Gelem/s", "cores": 1,
+                "kind": "oracle",
+                "sample": f"{n} head(s) x {P} channels x batch {b} x L {L}, {spent:.1f} s "
+                          "single-threaded fp64"}
     while True:
         sl = lambda x: None if x is None else x[:, :n]
         vec = lambda x: None if x is None else x[:n]
