@@ -28,12 +28,13 @@
 // the exponentials carry cs_t with a plus sign where t is the output token
 // and a minus sign where it is the source token, which is what dcs collects.
 //
-// Two kernels, one CTA of 256 threads per (batch, head):
-//   ssd_bwd_states_kernel runs the forward state recurrence chunk by chunk
-//     and stores h at every chunk start (and the final state) in scratch;
-//   ssd_bwd_kernel walks the chunks backwards with dh in registers and
-//     evaluates the products above from shared memory (fp32 CUDA cores;
-//     32-token chunks keep every product's operands on chip).
+// Two kernels, one CTA per (batch, head):
+//   ssd_bwd_states_kernel (256 threads) runs the forward state recurrence
+//     chunk by chunk and stores h at every chunk start (and the final state)
+//     in scratch;
+//   ssd_bwd_kernel (512 threads) walks the chunks backwards with dh in
+//     registers and evaluates the products above from shared memory (fp32
+//     CUDA cores; 32-token chunks keep every product's operands on chip).
 // dB and dC sum over the heads of a group: each head adds its chunk terms
 // with 16-byte atomics into one of kSbCopies partial copies ([t][n] rows),
 // and ssd_bwd_reduce_bc sums the copies into (batch, G, N, L).  dA, dD and
@@ -212,18 +213,23 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
 }
 
 // ------------------------------------------------------------ chunk walk
-// Shared memory of the walk (fp32).  Rows are padded (68 / 132 floats, 33
-// for the Q x Q matrices) so that the column groups the threads of a warp
-// read at once fall in distinct banks.
+// 512 threads (16 warps per SM to hide the shared-memory latency of the
+// products).  Shared memory of the walk (fp32); rows are padded (68 / 132 /
+// 36 floats) so that the column groups a warp reads at once fall in distinct
+// banks and every row stays 16-byte aligned.
+constexpr int kSbWalk = 512;
 constexpr int kSbXS = kSbP + 4;   // x, dout, dy silu'(z): [t][p]
 constexpr int kSbNS = kSbN + 4;   // B, C: [t][n]; h_0^T, dh^T: [p][n]
+constexpr int kSbTS = kSbQ + 4;   // x^T, dout^T: [p][t]; the Q x Q matrices
 struct SbSmem {
     float xs[kSbQ][kSbXS], dos[kSbQ][kSbXS], zf[kSbQ][kSbXS];
+    float xsT[kSbP][kSbTS], dosT[kSbP][kSbTS];
     float Bs[kSbQ][kSbNS], Cs[kSbQ][kSbNS];
     float h0T[kSbP][kSbNS], dhT[kSbP][kSbNS];
-    float Mm[kSbQ][kSbQ + 1], Md[kSbQ][kSbQ + 1], Wm[kSbQ][kSbQ + 1], Vm[kSbQ][kSbQ + 1];
+    // L.G.delta_s [t][s], (L.G)^T [s][t], L.delta_s.(dout x^T) [t][s], (L.(dout x^T))^T [s][t]
+    float Md[kSbQ][kSbTS], MmT[kSbQ][kSbTS], Wm[kSbQ][kSbTS], VmT[kSbQ][kSbTS];
     float raw[kSbQ], dl[kSbQ], S[kSbQ], ecs[kSbQ], ecq[kSbQ], ddd[kSbQ], dyy[kSbQ];
-    float red[8];
+    float red[kSbWalk / 32];
     float hqdh, ecQ;
 };
 
@@ -239,22 +245,34 @@ __device__ __forceinline__ float sb_block_sum(float v, float *red, int tid)
     __syncthreads();
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < kSbThreads / 32; ++w)
+    for (int w = 0; w < kSbWalk / 32; ++w)
         t += red[w];
     return t;
 }
 
-// Sum over the 8 consecutive lanes that share a row (lanes 8r .. 8r + 7).
-__device__ __forceinline__ float sb_sum8(float v)
+// Sum over the 16 consecutive lanes that share a row (lanes 16r .. 16r + 15).
+__device__ __forceinline__ float sb_sum16(float v)
 {
     v += __shfl_xor_sync(0xffffffffu, v, 1);
     v += __shfl_xor_sync(0xffffffffu, v, 2);
     v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
     return v;
 }
 
+__device__ __forceinline__ float sb_dot4(float4 a, float4 b, float acc)
+{
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+}
+
+template <typename T>
+__device__ __forceinline__ float4 sb_ld4(const T &ref)
+{
+    return *reinterpret_cast<const float4 *>(&ref);
+}
+
 template <bool GATE>
-__global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdParams p)
+__global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams p)
 {
     constexpr int Q = kSbQ, N = kSbN, P = kSbP;
     extern __shared__ __align__(16) uint8_t sb_raw[];
@@ -263,24 +281,26 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bh = blockIdx.x, b = bh / p.H, hh = bh - b * p.H;
     const int g = hh / p.heads_per_group;
-    const SbOwn o(tid);
-    const int r = tid >> 3, cg = tid & 7;  // row (token) and column group of the product phases
+    // state ownership: half (ih) of the 4 x 8 block of states-kernel thread u
+    const int u = tid >> 1, ih = tid & 1;
+    const int nb = u & 31, pb = u >> 5;
+    const int n0 = 4 * nb + 2 * ih;        // rows n0, n0 + 1; columns 8 pb + j
+    const int r = tid >> 4, cg = tid & 15;  // row (token) and column group of the products
     const float A = p.A[hh];
     const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
     const float dsk = p.Dskip ? p.Dskip[hh] : 0.f;
 
-    // gradient of the state leaving the current chunk, thread-owned
-    float dh[4][8];
+    float dh[2][8];  // gradient of the state leaving the current chunk
     {
         const float *dl0 = p.dlast ? p.dlast + (int64_t(b) * p.H + hh) * P * N : nullptr;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                dh[i][j] = dl0 ? dl0[int64_t(8 * o.pb + j) * N + 4 * o.nb + i] : 0.f;
+            for (int i = 0; i < 2; ++i)
+                dh[i][j] = dl0 ? dl0[int64_t(8 * pb + j) * N + n0 + i] : 0.f;
     }
     const float4 *st = reinterpret_cast<const float4 *>(p.states) +
-                       (int64_t(bh) * (p.nchunks + 1) * kSbThreads + tid) * 8;
+                       (int64_t(bh) * (p.nchunks + 1) * kSbThreads + u) * 8 + 4 * ih;
     const int64_t chunk_stride = int64_t(kSbThreads) * 8;
     const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
     const __nv_bfloat16 *Crow = p.C + int64_t(b) * p.C_bs + int64_t(g) * p.C_gs;
@@ -294,15 +314,16 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
 
     for (int c = p.nchunks - 1; c >= 0; --c) {
         const int t0 = c * Q, valid = min(Q, p.L - t0);
-        // ---- 1. chunk inputs, h_0 and dh_Q transposed, step sizes
+        // ---- 1. chunk inputs (and transposed copies), h_0^T, dh_Q^T, step sizes
         {
-            const int pp = tid >> 2, q = tid & 3;
-            const int64_t xo = int64_t(pp) * p.x_cs + t0 + 8 * q;
-            const int64_t yo = int64_t(pp) * p.dy_cs + t0 + 8 * q;
-            const int64_t zo = GATE ? int64_t(pp) * p.z_cs + t0 + 8 * q : 0;
+            const int pp = tid >> 3, q = tid & 7;  // row p, tokens 4q .. 4q + 3
+            const int64_t xo = int64_t(pp) * p.x_cs + t0 + 4 * q;
+            const int64_t yo = int64_t(pp) * p.dy_cs + t0 + 4 * q;
+            const int64_t zo = GATE ? int64_t(pp) * p.z_cs + t0 + 4 * q : 0;
+            float xv4[4], dv4[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int t = 8 * q + k;
+            for (int k = 0; k < 4; ++k) {
+                const int t = 4 * q + k;
                 const bool in = t < valid;
                 const float xv = in ? sb_bf(xrow[xo + k]) : 0.f;
                 const float dyv = in ? sb_bf(dyrow[yo + k]) : 0.f;
@@ -317,15 +338,21 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
                 sm.dos[t][pp] = dout;
                 if (GATE)
                     sm.zf[t][pp] = zfac;
+                xv4[k] = xv;
+                dv4[k] = dout;
             }
+            *reinterpret_cast<float4 *>(&sm.xsT[pp][4 * q]) =
+                make_float4(xv4[0], xv4[1], xv4[2], xv4[3]);
+            *reinterpret_cast<float4 *>(&sm.dosT[pp][4 * q]) =
+                make_float4(dv4[0], dv4[1], dv4[2], dv4[3]);
         }
         {
-            const int n = tid >> 1, half = tid & 1;
-            const int64_t bo = int64_t(n) * p.B_ns + t0 + 16 * half;
-            const int64_t co = int64_t(n) * p.C_ns + t0 + 16 * half;
+            const int n = tid >> 2, q = tid & 3;  // row n, tokens 8q .. 8q + 7
+            const int64_t bo = int64_t(n) * p.B_ns + t0 + 8 * q;
+            const int64_t co = int64_t(n) * p.C_ns + t0 + 8 * q;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int t = 16 * half + k;
+            for (int k = 0; k < 8; ++k) {
+                const int t = 8 * q + k;
                 const bool in = t < valid;
                 sm.Bs[t][n] = in ? sb_bf(Brow[bo + k]) : 0.f;
                 sm.Cs[t][n] = in ? sb_bf(Crow[co + k]) : 0.f;
@@ -336,15 +363,15 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
             const float4 *s0 = st + int64_t(c) * chunk_stride;
             const float4 *s1 = st + int64_t(c + 1) * chunk_stride;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 2; ++i) {
                 const float4 a0 = s0[2 * i], a1 = s0[2 * i + 1];
                 const float4 q0 = s1[2 * i], q1 = s1[2 * i + 1];
                 const float h0v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                 const float hqv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    sm.h0T[8 * o.pb + j][4 * o.nb + i] = h0v[j];
-                    sm.dhT[8 * o.pb + j][4 * o.nb + i] = dh[i][j];
+                    sm.h0T[8 * pb + j][n0 + i] = h0v[j];
+                    sm.dhT[8 * pb + j][n0 + i] = dh[i][j];
                     hq = fmaf(dh[i][j], hqv[j], hq);
                 }
             }
@@ -366,75 +393,66 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
             sm.hqdh = hq;
         __syncthreads();
 
-        // ---- 2. Q x Q products: row t = r, columns s = cg + 8k
+        // ---- 2. Q x Q matrices: row t = r, columns s = cg, cg + 16
         {
-            float G4[4] = {0.f, 0.f, 0.f, 0.f}, Y4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+            float G2[2] = {0.f, 0.f}, Y2[2] = {0.f, 0.f};
+#pragma unroll 8
             for (int n4 = 0; n4 < N / 4; ++n4) {
-                const float4 cv = *reinterpret_cast<const float4 *>(&sm.Cs[r][4 * n4]);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 bv = *reinterpret_cast<const float4 *>(&sm.Bs[cg + 8 * k][4 * n4]);
-                    G4[k] = fmaf(cv.x, bv.x, fmaf(cv.y, bv.y, fmaf(cv.z, bv.z, fmaf(cv.w, bv.w, G4[k]))));
-                }
+                const float4 cv = sb_ld4(sm.Cs[r][4 * n4]);
+                G2[0] = sb_dot4(cv, sb_ld4(sm.Bs[cg][4 * n4]), G2[0]);
+                G2[1] = sb_dot4(cv, sb_ld4(sm.Bs[cg + 16][4 * n4]), G2[1]);
             }
-#pragma unroll 4
+#pragma unroll 8
             for (int p4 = 0; p4 < P / 4; ++p4) {
-                const float4 dv = *reinterpret_cast<const float4 *>(&sm.dos[r][4 * p4]);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 xv = *reinterpret_cast<const float4 *>(&sm.xs[cg + 8 * k][4 * p4]);
-                    Y4[k] = fmaf(dv.x, xv.x, fmaf(dv.y, xv.y, fmaf(dv.z, xv.z, fmaf(dv.w, xv.w, Y4[k]))));
-                }
+                const float4 dv = sb_ld4(sm.dos[r][4 * p4]);
+                Y2[0] = sb_dot4(dv, sb_ld4(sm.xs[cg][4 * p4]), Y2[0]);
+                Y2[1] = sb_dot4(dv, sb_ld4(sm.xs[cg + 16][4 * p4]), Y2[1]);
             }
             const float St = sm.S[r];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int s = cg + 8 * k;
+            for (int k = 0; k < 2; ++k) {
+                const int s = cg + 16 * k;
                 const float Lts = s <= r ? expf(A * (St - sm.S[s])) : 0.f;
                 const float ds = sm.dl[s];
-                const float m = G4[k] * Lts, v = Y4[k] * Lts;
-                sm.Mm[r][s] = m;
+                const float m = G2[k] * Lts, v = Y2[k] * Lts;
                 sm.Md[r][s] = m * ds;
-                sm.Vm[r][s] = v;
+                sm.MmT[s][r] = m;
                 sm.Wm[r][s] = v * ds;
+                sm.VmT[s][r] = v;
             }
         }
         __syncthreads();
 
-        // ---- 3a. y~ (row t = r) and u (row s = r), columns p = cg + 8j
-        float yt[8], uu[8];
+        // ---- 3a. y~ (row t = r) and u (row s = r), columns p = cg + 16 j
+        float yt[4], uu[4];
         {
+            float y2[4], u2[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                yt[j] = uu[j] = 0.f;
-            for (int k = 0; k < Q; ++k) {
-                const float md = sm.Md[r][k], mm = sm.Mm[k][r];
+            for (int j = 0; j < 4; ++j)
+                yt[j] = uu[j] = y2[j] = u2[j] = 0.f;
+#pragma unroll 4
+            for (int k4 = 0; k4 < Q / 4; ++k4) {
+                const float4 md = sb_ld4(sm.Md[r][4 * k4]);
+                const float4 mm = sb_ld4(sm.MmT[r][4 * k4]);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    yt[j] = fmaf(md, sm.xs[k][cg + 8 * j], yt[j]);
-                    uu[j] = fmaf(mm, sm.dos[k][cg + 8 * j], uu[j]);
+                for (int j = 0; j < 4; ++j) {
+                    yt[j] = sb_dot4(md, sb_ld4(sm.xsT[cg + 16 * j][4 * k4]), yt[j]);
+                    uu[j] = sb_dot4(mm, sb_ld4(sm.dosT[cg + 16 * j][4 * k4]), uu[j]);
                 }
             }
-            float y2[8], u2[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                y2[j] = u2[j] = 0.f;
-#pragma unroll 2
+#pragma unroll 4
             for (int n4 = 0; n4 < N / 4; ++n4) {
-                const float4 cv = *reinterpret_cast<const float4 *>(&sm.Cs[r][4 * n4]);
-                const float4 bv = *reinterpret_cast<const float4 *>(&sm.Bs[r][4 * n4]);
+                const float4 cv = sb_ld4(sm.Cs[r][4 * n4]);
+                const float4 bv = sb_ld4(sm.Bs[r][4 * n4]);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 hv = *reinterpret_cast<const float4 *>(&sm.h0T[cg + 8 * j][4 * n4]);
-                    const float4 gv = *reinterpret_cast<const float4 *>(&sm.dhT[cg + 8 * j][4 * n4]);
-                    y2[j] = fmaf(cv.x, hv.x, fmaf(cv.y, hv.y, fmaf(cv.z, hv.z, fmaf(cv.w, hv.w, y2[j]))));
-                    u2[j] = fmaf(bv.x, gv.x, fmaf(bv.y, gv.y, fmaf(bv.z, gv.z, fmaf(bv.w, gv.w, u2[j]))));
+                for (int j = 0; j < 4; ++j) {
+                    y2[j] = sb_dot4(cv, sb_ld4(sm.h0T[cg + 16 * j][4 * n4]), y2[j]);
+                    u2[j] = sb_dot4(bv, sb_ld4(sm.dhT[cg + 16 * j][4 * n4]), u2[j]);
                 }
             }
             const float et = sm.ecs[r], eq = sm.ecq[r];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 4; ++j) {
                 yt[j] = fmaf(et, y2[j], yt[j]);
                 uu[j] = fmaf(eq, u2[j], uu[j]);
             }
@@ -446,8 +464,8 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
             float xu = 0.f, dyy = 0.f;
             const int64_t row_t = t0 + r;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int pp = cg + 8 * j;
+            for (int j = 0; j < 4; ++j) {
+                const int pp = cg + 16 * j;
                 const float xv = sm.xs[r][pp], dv = sm.dos[r][pp];
                 xu = fmaf(xv, uu[j], xu);
                 dyy = fmaf(dv, yt[j], dyy);
@@ -460,58 +478,53 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
                             __float2bfloat16_rn(sm.zf[r][pp] * fmaf(dsk, xv, yt[j]));
                 }
             }
-            xu = sb_sum8(xu);
-            dyy = sb_sum8(dyy);
+            xu = sb_sum16(xu);
+            dyy = sb_sum16(dyy);
             if (cg == 0) {
                 sm.ddd[r] = xu;
                 sm.dyy[r] = dyy;
             }
         }
-        // ---- 3b. dC (row t = r) and dB (row s = r), columns n = 4 (cg + 8k) + i
+        // ---- 3b. dC (row t = r) and dB (row s = r), columns n = 4 (cg + 16 k) + i
         {
-            float cacc[4][4], bacc[4][4];
+            float4 ca[2], ba[2], c2[2], b2[2];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 2; ++k)
+                ca[k] = ba[k] = c2[k] = b2[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            auto axpy = [](float a, float4 x, float4 &y) {
+                y.x = fmaf(a, x.x, y.x);
+                y.y = fmaf(a, x.y, y.y);
+                y.z = fmaf(a, x.z, y.z);
+                y.w = fmaf(a, x.w, y.w);
+            };
+#pragma unroll 2
+            for (int q4 = 0; q4 < Q / 4; ++q4) {
+                const float4 w4 = sb_ld4(sm.Wm[r][4 * q4]);
+                const float4 v4 = sb_ld4(sm.VmT[r][4 * q4]);
+                const float wv[4] = {w4.x, w4.y, w4.z, w4.w}, vv[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    cacc[k][i] = bacc[k][i] = 0.f;
-            for (int q = 0; q < Q; ++q) {
-                const float w = sm.Wm[r][q], v = sm.Vm[q][r];
+                for (int m = 0; m < 4; ++m) {
+                    const int q = 4 * q4 + m;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 bv = *reinterpret_cast<const float4 *>(&sm.Bs[q][4 * (cg + 8 * k)]);
-                    const float4 cv = *reinterpret_cast<const float4 *>(&sm.Cs[q][4 * (cg + 8 * k)]);
-                    cacc[k][0] = fmaf(w, bv.x, cacc[k][0]);
-                    cacc[k][1] = fmaf(w, bv.y, cacc[k][1]);
-                    cacc[k][2] = fmaf(w, bv.z, cacc[k][2]);
-                    cacc[k][3] = fmaf(w, bv.w, cacc[k][3]);
-                    bacc[k][0] = fmaf(v, cv.x, bacc[k][0]);
-                    bacc[k][1] = fmaf(v, cv.y, bacc[k][1]);
-                    bacc[k][2] = fmaf(v, cv.z, bacc[k][2]);
-                    bacc[k][3] = fmaf(v, cv.w, bacc[k][3]);
+                    for (int k = 0; k < 2; ++k) {
+                        axpy(wv[m], sb_ld4(sm.Bs[q][4 * (cg + 16 * k)]), ca[k]);
+                        axpy(vv[m], sb_ld4(sm.Cs[q][4 * (cg + 16 * k)]), ba[k]);
+                    }
                 }
             }
-            float c2[4][4], b2[4][4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    c2[k][i] = b2[k][i] = 0.f;
 #pragma unroll 2
-            for (int pp = 0; pp < P; ++pp) {
-                const float dv = sm.dos[r][pp], xv = sm.xs[r][pp];
+            for (int p4 = 0; p4 < P / 4; ++p4) {
+                const float4 d4 = sb_ld4(sm.dos[r][4 * p4]);
+                const float4 x4 = sb_ld4(sm.xs[r][4 * p4]);
+                const float dv[4] = {d4.x, d4.y, d4.z, d4.w}, xv[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 hv = *reinterpret_cast<const float4 *>(&sm.h0T[pp][4 * (cg + 8 * k)]);
-                    const float4 gv = *reinterpret_cast<const float4 *>(&sm.dhT[pp][4 * (cg + 8 * k)]);
-                    c2[k][0] = fmaf(dv, hv.x, c2[k][0]);
-                    c2[k][1] = fmaf(dv, hv.y, c2[k][1]);
-                    c2[k][2] = fmaf(dv, hv.z, c2[k][2]);
-                    c2[k][3] = fmaf(dv, hv.w, c2[k][3]);
-                    b2[k][0] = fmaf(xv, gv.x, b2[k][0]);
-                    b2[k][1] = fmaf(xv, gv.y, b2[k][1]);
-                    b2[k][2] = fmaf(xv, gv.z, b2[k][2]);
-                    b2[k][3] = fmaf(xv, gv.w, b2[k][3]);
+                for (int m = 0; m < 4; ++m) {
+                    const int pp = 4 * p4 + m;
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        axpy(dv[m], sb_ld4(sm.h0T[pp][4 * (cg + 16 * k)]), c2[k]);
+                        axpy(xv[m], sb_ld4(sm.dhT[pp][4 * (cg + 16 * k)]), b2[k]);
+                    }
                 }
             }
             if (r < valid) {
@@ -519,17 +532,17 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
                 float4 *dCr = reinterpret_cast<float4 *>(pC + int64_t(t0 + r) * N);
                 float4 *dBr = reinterpret_cast<float4 *>(pB + int64_t(t0 + r) * N);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 vc = make_float4(fmaf(et, c2[k][0], cacc[k][0]),
-                                                  fmaf(et, c2[k][1], cacc[k][1]),
-                                                  fmaf(et, c2[k][2], cacc[k][2]),
-                                                  fmaf(et, c2[k][3], cacc[k][3]));
-                    const float4 vb = make_float4(ds * fmaf(eq, b2[k][0], bacc[k][0]),
-                                                  ds * fmaf(eq, b2[k][1], bacc[k][1]),
-                                                  ds * fmaf(eq, b2[k][2], bacc[k][2]),
-                                                  ds * fmaf(eq, b2[k][3], bacc[k][3]));
-                    atomicAdd(dCr + cg + 8 * k, vc);
-                    atomicAdd(dBr + cg + 8 * k, vb);
+                for (int k = 0; k < 2; ++k) {
+                    const float4 vc = make_float4(fmaf(et, c2[k].x, ca[k].x),
+                                                  fmaf(et, c2[k].y, ca[k].y),
+                                                  fmaf(et, c2[k].z, ca[k].z),
+                                                  fmaf(et, c2[k].w, ca[k].w));
+                    const float4 vb = make_float4(ds * fmaf(eq, b2[k].x, ba[k].x),
+                                                  ds * fmaf(eq, b2[k].y, ba[k].y),
+                                                  ds * fmaf(eq, b2[k].z, ba[k].z),
+                                                  ds * fmaf(eq, b2[k].w, ba[k].w));
+                    atomicAdd(dCr + cg + 16 * k, vc);
+                    atomicAdd(dBr + cg + 16 * k, vb);
                 }
             }
         }
@@ -537,19 +550,19 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
         {
             const float eQ = sm.ecQ;
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 2; ++i)
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     dh[i][j] *= eQ;
             for (int t = 0; t < valid; ++t) {
-                const float4 cv = *reinterpret_cast<const float4 *>(&sm.Cs[t][4 * o.nb]);
-                const float4 d0 = *reinterpret_cast<const float4 *>(&sm.dos[t][8 * o.pb]);
-                const float4 d1 = *reinterpret_cast<const float4 *>(&sm.dos[t][8 * o.pb + 4]);
+                const float2 cv = *reinterpret_cast<const float2 *>(&sm.Cs[t][n0]);
+                const float4 d0 = sb_ld4(sm.dos[t][8 * pb]);
+                const float4 d1 = sb_ld4(sm.dos[t][8 * pb + 4]);
                 const float et = sm.ecs[t];
-                const float cc[4] = {cv.x * et, cv.y * et, cv.z * et, cv.w * et};
+                const float cc[2] = {cv.x * et, cv.y * et};
                 const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < 2; ++i)
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
                         dh[i][j] = fmaf(cc[i], dd[j], dh[i][j]);
@@ -589,8 +602,8 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_kernel(const SsdBwdPara
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                d0[int64_t(8 * o.pb + j) * N + 4 * o.nb + i] = dh[i][j];
+            for (int i = 0; i < 2; ++i)
+                d0[int64_t(8 * pb + j) * N + n0 + i] = dh[i][j];
     }
     const float sD = sb_block_sum(accD, sm.red, tid);
     const float sA = sb_block_sum(accA, sm.red, tid);

@@ -1703,7 +1703,7 @@ extern "C" selscan_status selscan_bwd_scalarA(
     ssd_bwd_states_kernel<<<grid, kSbThreads, 0, stream>>>(prm);
     cudaError_t le = counted_launch();
     if (le == cudaSuccess) {
-        kern<<<grid, kSbThreads, sizeof(SbSmem), stream>>>(prm);
+        kern<<<grid, kSbWalk, sizeof(SbSmem), stream>>>(prm);
         le = counted_launch();
     }
     if (le == cudaSuccess) {
