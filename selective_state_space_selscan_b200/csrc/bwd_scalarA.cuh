@@ -271,6 +271,86 @@ __device__ __forceinline__ float4 sb_ld4(const T &ref)
     return *reinterpret_cast<const float4 *>(&ref);
 }
 
+// ---- warp-level tensor-core products (mma.sync m16n8k8, tf32 inputs, fp32
+// accumulators).  Fragment coordinates, with g = lane / 4 and q = lane % 4:
+// A (16 x 8): a0 (g, q), a1 (g + 8, q), a2 (g, q + 4), a3 (g + 8, q + 4);
+// B (8 x 8):  b0 (q, g), b1 (q + 4, g);
+// D (16 x 8): d0 (g, 2q), d1 (g, 2q + 1), d2 (g + 8, 2q), d3 (g + 8, 2q + 1).
+__device__ __forceinline__ uint32_t sb_tf32(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void sb_mma(float (&d)[4], const uint32_t (&a)[4],
+                                       const uint32_t (&b)[2])
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// x = hi + lo with hi, lo both tf32 (hi the rounded value, lo the rounded rest).
+__device__ __forceinline__ void sb_split(float x, uint32_t &hi, uint32_t &lo)
+{
+    hi = sb_tf32(x);
+    lo = sb_tf32(x - __uint_as_float(hi));
+}
+
+// D[NT tiles] += sum_{k < K} A(m0 + row, k) B(k, n0 + 8 t + col): one A
+// fragment per k step serves NT output tiles.  fa(m, k) and fb(k, n) read
+// the operands from shared memory in whatever layout they are kept.  SPLIT:
+// each operand as the sum of two tf32 numbers and three products (hi hi, hi
+// lo, lo hi), which carries about the 21 leading bits of fp32 into the
+// products that feed the differences of the step-size gradients.
+template <int K, int NT, bool SPLIT, typename FA, typename FB>
+__device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, FA fa, FB fb,
+                                        int lane)
+{
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const float av[4] = {fa(m0 + g, k0 + q), fa(m0 + g + 8, k0 + q), fa(m0 + g, k0 + q + 4),
+                             fa(m0 + g + 8, k0 + q + 4)};
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (SPLIT)
+                sb_split(av[i], ah[i], al[i]);
+            else
+                ah[i] = sb_tf32(av[i]);
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const float bv[2] = {fb(k0 + q, n0 + 8 * t + g), fb(k0 + q + 4, n0 + 8 * t + g)};
+            uint32_t bh[2], bl[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if (SPLIT)
+                    sb_split(bv[i], bh[i], bl[i]);
+                else
+                    bh[i] = sb_tf32(bv[i]);
+            }
+            if (SPLIT) {
+                sb_mma(d[t], al, bh);
+                sb_mma(d[t], ah, bl);
+            }
+            sb_mma(d[t], ah, bh);
+        }
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void sb_zero(float (&d)[NT][4])
+{
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+        d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+}
+
 template <bool GATE>
 __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams p)
 {
@@ -279,29 +359,48 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
     SbSmem &sm = *reinterpret_cast<SbSmem *>(sb_raw);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g8 = lane >> 2, q4 = lane & 3;  // fragment row / column of this lane
     const int bh = blockIdx.x, b = bh / p.H, hh = bh - b * p.H;
     const int g = hh / p.heads_per_group;
-    // state ownership: half (ih) of the 4 x 8 block of states-kernel thread u
-    const int u = tid >> 1, ih = tid & 1;
-    const int nb = u & 31, pb = u >> 5;
-    const int n0 = 4 * nb + 2 * ih;        // rows n0, n0 + 1; columns 8 pb + j
-    const int r = tid >> 4, cg = tid & 15;  // row (token) and column group of the products
     const float A = p.A[hh];
     const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
     const float dsk = p.Dskip ? p.Dskip[hh] : 0.f;
 
-    float dh[2][8];  // gradient of the state leaving the current chunk
+    // dh (N x P) in accumulator fragments: warp w holds rows 16 (w / 2) .. + 15,
+    // columns 32 (w % 2) .. + 31 (four 16 x 8 tiles)
+    const int dm0 = 16 * (warp >> 1), dn0 = 32 * (warp & 1);
+    float dh[4][4];
     {
         const float *dl0 = p.dlast ? p.dlast + (int64_t(b) * p.H + hh) * P * N : nullptr;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
-                dh[i][j] = dl0 ? dl0[int64_t(8 * pb + j) * N + n0 + i] : 0.f;
+            for (int e = 0; e < 4; ++e) {
+                const int n = dm0 + g8 + 8 * (e >> 1), pp = dn0 + 8 * t + 2 * q4 + (e & 1);
+                dh[t][e] = dl0 ? dl0[int64_t(pp) * N + n] : 0.f;
+            }
     }
-    const float4 *st = reinterpret_cast<const float4 *>(p.states) +
-                       (int64_t(bh) * (p.nchunks + 1) * kSbThreads + u) * 8 + 4 * ih;
+    const float4 *st_base = reinterpret_cast<const float4 *>(p.states) +
+                            int64_t(bh) * (p.nchunks + 1) * kSbThreads * 8;
     const int64_t chunk_stride = int64_t(kSbThreads) * 8;
+    // <dlast, final state> for the last chunk: states-kernel layout, read by
+    // thread halves (u = tid / 2 owns rows 4 (u % 32) + i, columns 8 (u / 32) + j)
+    float hq_next = 0.f;
+    if (p.dlast) {
+        const int u = tid >> 1, ih = tid & 1;
+        const float4 *sf = st_base + int64_t(p.nchunks) * chunk_stride + u * 8 + 4 * ih;
+        const float *dl0 = p.dlast + (int64_t(b) * p.H + hh) * P * N;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float4 a0 = sf[2 * i], a1 = sf[2 * i + 1];
+            const float hv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const int n = 4 * (u & 31) + 2 * ih + i;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                hq_next = fmaf(dl0[int64_t(8 * (u >> 5) + j) * N + n], hv[j], hq_next);
+        }
+    }
+    hq_next = sb_block_sum(hq_next, sm.red, tid);
     const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
     const __nv_bfloat16 *Crow = p.C + int64_t(b) * p.C_bs + int64_t(g) * p.C_gs;
     const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
@@ -358,24 +457,24 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
                 sm.Cs[t][n] = in ? sb_bf(Crow[co + k]) : 0.f;
             }
         }
-        float hq = 0.f;  // <dh_Q, h_Q>, this thread's part
         {
-            const float4 *s0 = st + int64_t(c) * chunk_stride;
-            const float4 *s1 = st + int64_t(c + 1) * chunk_stride;
+            const int u = tid >> 1, ih = tid & 1;
+            const float4 *s0 = st_base + int64_t(c) * chunk_stride + u * 8 + 4 * ih;
+            const int n0 = 4 * (u & 31) + 2 * ih, pb = u >> 5;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const float4 a0 = s0[2 * i], a1 = s0[2 * i + 1];
-                const float4 q0 = s1[2 * i], q1 = s1[2 * i + 1];
                 const float h0v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const float hqv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 8; ++j)
                     sm.h0T[8 * pb + j][n0 + i] = h0v[j];
-                    sm.dhT[8 * pb + j][n0 + i] = dh[i][j];
-                    hq = fmaf(dh[i][j], hqv[j], hq);
-                }
             }
         }
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                sm.dhT[dn0 + 8 * t + 2 * q4 + (e & 1)][dm0 + g8 + 8 * (e >> 1)] = dh[t][e];
         if (warp == 0) {
             float rw, dl, S;
             sb_steps(p, b, hh, t0, valid, lane, bias, rw, dl, S);
@@ -385,197 +484,153 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             sm.S[lane] = S;
             sm.ecs[lane] = expf(A * S);
             sm.ecq[lane] = expf(A * (SQ - S));
+            sm.ddd[lane] = 0.f;
+            sm.dyy[lane] = 0.f;
             if (lane == 0)
                 sm.ecQ = expf(A * SQ);
         }
-        hq = sb_block_sum(hq, sm.red, tid);  // (its barriers also publish the loads)
-        if (tid == 0)
-            sm.hqdh = hq;
         __syncthreads();
 
-        // ---- 2. Q x Q matrices: row t = r, columns s = cg, cg + 16
+        // ---- 2. Q x Q matrices: warps 0-7 G = C B^T, warps 8-15 dout x^T;
+        //         one 16 x 8 tile each, then the mask and the step sizes
         {
-            float G2[2] = {0.f, 0.f}, Y2[2] = {0.f, 0.f};
-#pragma unroll 8
-            for (int n4 = 0; n4 < N / 4; ++n4) {
-                const float4 cv = sb_ld4(sm.Cs[r][4 * n4]);
-                G2[0] = sb_dot4(cv, sb_ld4(sm.Bs[cg][4 * n4]), G2[0]);
-                G2[1] = sb_dot4(cv, sb_ld4(sm.Bs[cg + 16][4 * n4]), G2[1]);
-            }
-#pragma unroll 8
-            for (int p4 = 0; p4 < P / 4; ++p4) {
-                const float4 dv = sb_ld4(sm.dos[r][4 * p4]);
-                Y2[0] = sb_dot4(dv, sb_ld4(sm.xs[cg][4 * p4]), Y2[0]);
-                Y2[1] = sb_dot4(dv, sb_ld4(sm.xs[cg + 16][4 * p4]), Y2[1]);
-            }
-            const float St = sm.S[r];
+            const int w8 = warp & 7, m0 = 16 * (w8 >> 2), n0 = 8 * (w8 & 3);
+            float acc[1][4];
+            sb_zero(acc);
+            if (warp < 8)
+                sb_gemm<N, 1, true>(acc, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
+                              [&](int k, int n) { return sm.Bs[n][k]; }, lane);
+            else
+                sb_gemm<P, 1, true>(acc, m0, n0, [&](int m, int k) { return sm.dos[m][k]; },
+                              [&](int k, int n) { return sm.xs[n][k]; }, lane);
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int s = cg + 16 * k;
-                const float Lts = s <= r ? expf(A * (St - sm.S[s])) : 0.f;
-                const float ds = sm.dl[s];
-                const float m = G2[k] * Lts, v = Y2[k] * Lts;
-                sm.Md[r][s] = m * ds;
-                sm.MmT[s][r] = m;
-                sm.Wm[r][s] = v * ds;
-                sm.VmT[s][r] = v;
+            for (int e = 0; e < 4; ++e) {
+                const int t = m0 + g8 + 8 * (e >> 1), s_ = n0 + 2 * q4 + (e & 1);
+                const float Lts = s_ <= t ? expf(A * (sm.S[t] - sm.S[s_])) : 0.f;
+                const float v = acc[0][e] * Lts, ds = sm.dl[s_];
+                if (warp < 8) {
+                    sm.Md[t][s_] = v * ds;
+                    sm.MmT[s_][t] = v;
+                } else {
+                    sm.Wm[t][s_] = v * ds;
+                    sm.VmT[s_][t] = v;
+                }
             }
         }
         __syncthreads();
 
-        // ---- 3a. y~ (row t = r) and u (row s = r), columns p = cg + 16 j
-        float yt[4], uu[4];
+        // ---- 3a. y~ (rows t) and u (rows s): 32 x 64 each; warp w holds the
+        //          16 x 8 tile (16 (w / 8), 8 (w % 8)) of both
         {
-            float y2[4], u2[4];
+            const int m0 = 16 * (warp >> 3), n0 = 8 * (warp & 7);
+            float y1[1][4], y2[1][4], u1[1][4], u2[1][4];
+            sb_zero(y1);
+            sb_zero(y2);
+            sb_zero(u1);
+            sb_zero(u2);
+            sb_gemm<Q, 1, true>(y1, m0, n0, [&](int m, int k) { return sm.Md[m][k]; },
+                          [&](int k, int n) { return sm.xsT[n][k]; }, lane);
+            sb_gemm<N, 1, true>(y2, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
+                          [&](int k, int n) { return sm.h0T[n][k]; }, lane);
+            sb_gemm<Q, 1, true>(u1, m0, n0, [&](int m, int k) { return sm.MmT[m][k]; },
+                          [&](int k, int n) { return sm.dosT[n][k]; }, lane);
+            sb_gemm<N, 1, true>(u2, m0, n0, [&](int m, int k) { return sm.Bs[m][k]; },
+                          [&](int k, int n) { return sm.dhT[n][k]; }, lane);
+            float xu[2] = {0.f, 0.f}, dyy[2] = {0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                yt[j] = uu[j] = y2[j] = u2[j] = 0.f;
-#pragma unroll 4
-            for (int k4 = 0; k4 < Q / 4; ++k4) {
-                const float4 md = sb_ld4(sm.Md[r][4 * k4]);
-                const float4 mm = sb_ld4(sm.MmT[r][4 * k4]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    yt[j] = sb_dot4(md, sb_ld4(sm.xsT[cg + 16 * j][4 * k4]), yt[j]);
-                    uu[j] = sb_dot4(mm, sb_ld4(sm.dosT[cg + 16 * j][4 * k4]), uu[j]);
-                }
-            }
-#pragma unroll 4
-            for (int n4 = 0; n4 < N / 4; ++n4) {
-                const float4 cv = sb_ld4(sm.Cs[r][4 * n4]);
-                const float4 bv = sb_ld4(sm.Bs[r][4 * n4]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    y2[j] = sb_dot4(cv, sb_ld4(sm.h0T[cg + 16 * j][4 * n4]), y2[j]);
-                    u2[j] = sb_dot4(bv, sb_ld4(sm.dhT[cg + 16 * j][4 * n4]), u2[j]);
-                }
-            }
-            const float et = sm.ecs[r], eq = sm.ecq[r];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                yt[j] = fmaf(et, y2[j], yt[j]);
-                uu[j] = fmaf(eq, u2[j], uu[j]);
-            }
-        }
-        // row outputs: dx, dz; sums for ddelta and dcs; dD
-        {
-            const bool in = r < valid;
-            const float ds = sm.dl[r];
-            float xu = 0.f, dyy = 0.f;
-            const int64_t row_t = t0 + r;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int pp = cg + 16 * j;
+            for (int e = 0; e < 4; ++e) {
+                const int hr = e >> 1, r = m0 + g8 + 8 * hr, pp = n0 + 2 * q4 + (e & 1);
+                const float yt = fmaf(sm.ecs[r], y2[0][e], y1[0][e]);
+                const float uu = fmaf(sm.ecq[r], u2[0][e], u1[0][e]);
                 const float xv = sm.xs[r][pp], dv = sm.dos[r][pp];
-                xu = fmaf(xv, uu[j], xu);
-                dyy = fmaf(dv, yt[j], dyy);
+                xu[hr] = fmaf(xv, uu, xu[hr]);
+                dyy[hr] = fmaf(dv, yt, dyy[hr]);
                 accD = fmaf(dv, xv, accD);
-                if (in) {
+                if (r < valid) {
+                    const int64_t row_t = t0 + r;
                     p.dx[int64_t(b) * p.dx_bs + int64_t(hh * P + pp) * p.dx_cs + row_t] =
-                        __float2bfloat16_rn(fmaf(ds, uu[j], dsk * dv));
+                        __float2bfloat16_rn(fmaf(sm.dl[r], uu, dsk * dv));
                     if (GATE)
                         p.dz[int64_t(b) * p.dz_bs + int64_t(hh * P + pp) * p.dz_cs + row_t] =
-                            __float2bfloat16_rn(sm.zf[r][pp] * fmaf(dsk, xv, yt[j]));
+                            __float2bfloat16_rn(sm.zf[r][pp] * fmaf(dsk, xv, yt));
                 }
             }
-            xu = sb_sum16(xu);
-            dyy = sb_sum16(dyy);
-            if (cg == 0) {
-                sm.ddd[r] = xu;
-                sm.dyy[r] = dyy;
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                xu[hr] += __shfl_xor_sync(0xffffffffu, xu[hr], 1);
+                xu[hr] += __shfl_xor_sync(0xffffffffu, xu[hr], 2);
+                dyy[hr] += __shfl_xor_sync(0xffffffffu, dyy[hr], 1);
+                dyy[hr] += __shfl_xor_sync(0xffffffffu, dyy[hr], 2);
+                if (q4 == 0) {
+                    atomicAdd(&sm.ddd[m0 + g8 + 8 * hr], xu[hr]);
+                    atomicAdd(&sm.dyy[m0 + g8 + 8 * hr], dyy[hr]);
+                }
             }
         }
-        // ---- 3b. dC (row t = r) and dB (row s = r), columns n = 4 (cg + 16 k) + i
+        // ---- 3b. dC (warps 0-7) and dB (warps 8-15): 32 x 128 each; warp
+        //          holds rows 16 ((w / 4) % 2), columns 32 (w % 4) .. + 31
         {
-            float4 ca[2], ba[2], c2[2], b2[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k)
-                ca[k] = ba[k] = c2[k] = b2[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            auto axpy = [](float a, float4 x, float4 &y) {
-                y.x = fmaf(a, x.x, y.x);
-                y.y = fmaf(a, x.y, y.y);
-                y.z = fmaf(a, x.z, y.z);
-                y.w = fmaf(a, x.w, y.w);
-            };
-#pragma unroll 2
-            for (int q4 = 0; q4 < Q / 4; ++q4) {
-                const float4 w4 = sb_ld4(sm.Wm[r][4 * q4]);
-                const float4 v4 = sb_ld4(sm.VmT[r][4 * q4]);
-                const float wv[4] = {w4.x, w4.y, w4.z, w4.w}, vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int q = 4 * q4 + m;
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        axpy(wv[m], sb_ld4(sm.Bs[q][4 * (cg + 16 * k)]), ca[k]);
-                        axpy(vv[m], sb_ld4(sm.Cs[q][4 * (cg + 16 * k)]), ba[k]);
-                    }
-                }
+            const int m0 = 16 * ((warp >> 2) & 1), n0 = 32 * (warp & 3);
+            float a1[4][4], a2[4][4];
+            sb_zero(a1);
+            sb_zero(a2);
+            if (warp < 8) {
+                sb_gemm<Q, 4, false>(a1, m0, n0, [&](int m, int k) { return sm.Wm[m][k]; },
+                              [&](int k, int n) { return sm.Bs[k][n]; }, lane);
+                sb_gemm<P, 4, false>(a2, m0, n0, [&](int m, int k) { return sm.dos[m][k]; },
+                              [&](int k, int n) { return sm.h0T[k][n]; }, lane);
+            } else {
+                sb_gemm<Q, 4, false>(a1, m0, n0, [&](int m, int k) { return sm.VmT[m][k]; },
+                              [&](int k, int n) { return sm.Cs[k][n]; }, lane);
+                sb_gemm<P, 4, false>(a2, m0, n0, [&](int m, int k) { return sm.xs[m][k]; },
+                              [&](int k, int n) { return sm.dhT[k][n]; }, lane);
             }
-#pragma unroll 2
-            for (int p4 = 0; p4 < P / 4; ++p4) {
-                const float4 d4 = sb_ld4(sm.dos[r][4 * p4]);
-                const float4 x4 = sb_ld4(sm.xs[r][4 * p4]);
-                const float dv[4] = {d4.x, d4.y, d4.z, d4.w}, xv[4] = {x4.x, x4.y, x4.z, x4.w};
+            float *dst = warp < 8 ? pC : pB;
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int pp = 4 * p4 + m;
+            for (int hr = 0; hr < 2; ++hr) {
+                const int r = m0 + g8 + 8 * hr;
+                if (r < valid) {
+                    const float sc = warp < 8 ? sm.ecs[r] : sm.ecq[r];
+                    const float pre = warp < 8 ? 1.f : sm.dl[r];
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        axpy(dv[m], sb_ld4(sm.h0T[pp][4 * (cg + 16 * k)]), c2[k]);
-                        axpy(xv[m], sb_ld4(sm.dhT[pp][4 * (cg + 16 * k)]), b2[k]);
+                    for (int t = 0; t < 4; ++t) {
+                        const int n = n0 + 8 * t + 2 * q4;
+                        const float2 v = make_float2(
+                            pre * fmaf(sc, a2[t][2 * hr], a1[t][2 * hr]),
+                            pre * fmaf(sc, a2[t][2 * hr + 1], a1[t][2 * hr + 1]));
+                        atomicAdd(reinterpret_cast<float2 *>(dst + int64_t(t0 + r) * N + n), v);
                     }
-                }
-            }
-            if (r < valid) {
-                const float et = sm.ecs[r], eq = sm.ecq[r], ds = sm.dl[r];
-                float4 *dCr = reinterpret_cast<float4 *>(pC + int64_t(t0 + r) * N);
-                float4 *dBr = reinterpret_cast<float4 *>(pB + int64_t(t0 + r) * N);
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const float4 vc = make_float4(fmaf(et, c2[k].x, ca[k].x),
-                                                  fmaf(et, c2[k].y, ca[k].y),
-                                                  fmaf(et, c2[k].z, ca[k].z),
-                                                  fmaf(et, c2[k].w, ca[k].w));
-                    const float4 vb = make_float4(ds * fmaf(eq, b2[k].x, ba[k].x),
-                                                  ds * fmaf(eq, b2[k].y, ba[k].y),
-                                                  ds * fmaf(eq, b2[k].z, ba[k].z),
-                                                  ds * fmaf(eq, b2[k].w, ba[k].w));
-                    atomicAdd(dCr + cg + 16 * k, vc);
-                    atomicAdd(dBr + cg + 16 * k, vb);
                 }
             }
         }
-        // ---- 3c. dh_0 = e^cs_Q dh_Q + sum_t e^cs_t C_t dout_t^T (thread-owned)
+        // ---- 3c. dh_0 = e^cs_Q dh_Q + C^T (e^cs dout): rows n, columns p
         {
             const float eQ = sm.ecQ;
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int t = 0; t < 4; ++t)
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    dh[i][j] *= eQ;
-            for (int t = 0; t < valid; ++t) {
-                const float2 cv = *reinterpret_cast<const float2 *>(&sm.Cs[t][n0]);
-                const float4 d0 = sb_ld4(sm.dos[t][8 * pb]);
-                const float4 d1 = sb_ld4(sm.dos[t][8 * pb + 4]);
-                const float et = sm.ecs[t];
-                const float cc[2] = {cv.x * et, cv.y * et};
-                const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        dh[i][j] = fmaf(cc[i], dd[j], dh[i][j]);
-            }
+                for (int e = 0; e < 4; ++e)
+                    dh[t][e] *= eQ;
+            sb_gemm<Q, 4, true>(dh, dm0, dn0, [&](int m, int k) { return sm.Cs[k][m]; },
+                          [&](int k, int n) { return sm.ecs[k] * sm.dos[k][n]; }, lane);
         }
-        __syncthreads();
+        // <dh_0, h_0> of this chunk: the <dh_Q, h_Q> term of the next one
+        float hq = 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                hq = fmaf(dh[t][e],
+                          sm.h0T[dn0 + 8 * t + 2 * q4 + (e & 1)][dm0 + g8 + 8 * (e >> 1)], hq);
+        const float hq_this = hq_next;
+        hq_next = sb_block_sum(hq, sm.red, tid);  // (its barriers also order 3a-3c before 4)
         // ---- 4. per-token scalars (one warp, lane = token)
         if (warp == 0) {
             const bool in = lane < valid;
             const float ds = sm.dl[lane];
             float dcs = sm.dyy[lane] - ds * sm.ddd[lane];
             if (lane == valid - 1)
-                dcs += sm.hqdh;
+                dcs += hq_this;
             if (!in)
                 dcs = 0.f;
             float R = dcs;  // sum over t >= lane
@@ -600,10 +655,11 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
     if (p.dh0) {
         float *d0 = p.dh0 + (int64_t(b) * p.H + hh) * P * N;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
-                d0[int64_t(8 * pb + j) * N + n0 + i] = dh[i][j];
+            for (int e = 0; e < 4; ++e)
+                d0[int64_t(dn0 + 8 * t + 2 * q4 + (e & 1)) * N + dm0 + g8 + 8 * (e >> 1)] =
+                    dh[t][e];
     }
     const float sD = sb_block_sum(accD, sm.red, tid);
     const float sA = sb_block_sum(accA, sm.red, tid);
