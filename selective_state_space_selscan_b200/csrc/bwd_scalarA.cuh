@@ -33,8 +33,13 @@
 //     chunk by chunk and stores h at every chunk start (and the final state)
 //     in scratch;
 //   ssd_bwd_kernel (512 threads) walks the chunks backwards with dh in
-//     registers and evaluates the products above from shared memory (fp32
-//     CUDA cores; 32-token chunks keep every product's operands on chip).
+//     accumulator fragments and evaluates the products above from shared
+//     memory (32-token chunks keep every product's operands on chip).
+// Every product runs on the tensor cores as warp-level m16n8k8 tiles with
+// tf32 operands and fp32 accumulation; the products whose results feed the
+// step-size gradients (differences of nearly equal sums) and the two state
+// recurrences split each operand into two tf32 parts (three products), which
+// keeps about 21 bits of every operand.
 // dB and dC sum over the heads of a group: each head adds its chunk terms
 // with 16-byte atomics into one of kSbCopies partial copies ([t][n] rows),
 // and ssd_bwd_reduce_bc sums the copies into (batch, G, N, L).  dA, dD and
@@ -73,14 +78,7 @@ struct SsdBwdParams {
     float *dA, *dD, *ddt_bias;        // (H), accumulated; dD / ddt_bias may be null
     float *dh0;                       // (batch, H, P, N) or null
     float *pB, *pC;                   // [kSbCopies][batch][G][L][N], zeroed
-    float *states;                    // [batch*H][nchunks+1][256 threads][32]
-};
-
-// Thread ownership of an N x P state matrix: thread tid holds rows
-// n = 4 (tid % 32) + i (i < 4) and columns p = 8 (tid / 32) + j (j < 8).
-struct SbOwn {
-    int nb, pb;
-    __device__ __forceinline__ explicit SbOwn(int tid) : nb(tid & 31), pb(tid >> 5) {}
+    float *states;                    // [batch*H][nchunks+1][256 threads][32] (sb_state_coord)
 };
 
 __device__ __forceinline__ float sb_bf(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -103,172 +101,6 @@ __device__ __forceinline__ void sb_steps(const SsdBwdParams &p, int b, int hh, i
         if (lane >= o)
             S += v;
     }
-}
-
-// Chunk rows of a (.., N, L) bf16 tensor into smem as fp32 [t][N]: thread
-// tid reads row n = tid / 2, tokens 16 (tid % 2) .. + 15.
-__device__ __forceinline__ void sb_load_nt(float (*dst)[kSbN], const __nv_bfloat16 *row0,
-                                           int64_t ns, int t0, int valid, int tid)
-{
-    const int n = tid >> 1, half = tid & 1;
-    const __nv_bfloat16 *src = row0 + int64_t(n) * ns + t0 + 16 * half;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const int t = 16 * half + k;
-        dst[t][n] = t < valid ? sb_bf(src[k]) : 0.f;
-    }
-}
-
-// Chunk rows of a (.., P, L) bf16 tensor (row stride cs) into smem as fp32
-// [t][P]: thread tid reads row p = tid / 4, tokens 8 (tid % 4) .. + 7.
-__device__ __forceinline__ void sb_load_pt(float (*dst)[kSbP], const __nv_bfloat16 *row0,
-                                           int64_t cs, int t0, int valid, int tid)
-{
-    const int pp = tid >> 2, q = tid & 3;
-    const __nv_bfloat16 *src = row0 + int64_t(pp) * cs + t0 + 8 * q;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int t = 8 * q + k;
-        dst[t][pp] = t < valid ? sb_bf(src[k]) : 0.f;
-    }
-}
-
-// ------------------------------------------------------------ forward states
-__global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const SsdBwdParams p)
-{
-    constexpr int Q = kSbQ, N = kSbN, P = kSbP;
-    __shared__ __align__(16) float Bs[Q][N];
-    __shared__ __align__(16) float xs[Q][P];
-    __shared__ __align__(16) float ws[Q];
-    __shared__ float s_decay;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = blockIdx.x, b = bh / p.H, hh = bh - b * p.H;
-    const int g = hh / p.heads_per_group;
-    const SbOwn o(tid);
-    const float A = p.A[hh];
-    const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
-
-    float hs[4][8];
-    {
-        const float *h0 = p.h0 ? p.h0 + (int64_t(b) * p.H + hh) * P * N : nullptr;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                hs[i][j] = h0 ? h0[int64_t(8 * o.pb + j) * N + 4 * o.nb + i] : 0.f;
-    }
-    float4 *st = reinterpret_cast<float4 *>(p.states) +
-                 (int64_t(bh) * (p.nchunks + 1) * kSbThreads + tid) * 8;
-    const int64_t chunk_stride = int64_t(kSbThreads) * 8;  // float4 per chunk entry
-    const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
-    const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
-
-    for (int c = 0; c < p.nchunks; ++c) {
-        float4 *sc = st + int64_t(c) * chunk_stride;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; j += 4)
-                sc[i * 2 + j / 4] = make_float4(hs[i][j], hs[i][j + 1], hs[i][j + 2], hs[i][j + 3]);
-        const int t0 = c * Q, valid = min(Q, p.L - t0);
-        sb_load_nt(Bs, Brow, p.B_ns, t0, valid, tid);
-        sb_load_pt(xs, xrow, p.x_cs, t0, valid, tid);
-        if (warp == 0) {
-            float raw, dl, S;
-            sb_steps(p, b, hh, t0, valid, lane, bias, raw, dl, S);
-            const float SQ = __shfl_sync(0xffffffffu, S, 31);
-            ws[lane] = expf(A * (SQ - S)) * dl;
-            if (lane == 0)
-                s_decay = expf(A * SQ);
-        }
-        __syncthreads();
-        const float dec = s_decay;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                hs[i][j] *= dec;
-        for (int s = 0; s < valid; ++s) {
-            const float4 b4 = *reinterpret_cast<const float4 *>(&Bs[s][4 * o.nb]);
-            const float4 x0 = *reinterpret_cast<const float4 *>(&xs[s][8 * o.pb]);
-            const float4 x1 = *reinterpret_cast<const float4 *>(&xs[s][8 * o.pb + 4]);
-            const float w = ws[s];
-            const float bw[4] = {b4.x * w, b4.y * w, b4.z * w, b4.w * w};
-            const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    hs[i][j] = fmaf(bw[i], xv[j], hs[i][j]);
-        }
-        __syncthreads();
-    }
-    float4 *sc = st + int64_t(p.nchunks) * chunk_stride;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; j += 4)
-            sc[i * 2 + j / 4] = make_float4(hs[i][j], hs[i][j + 1], hs[i][j + 2], hs[i][j + 3]);
-}
-
-// ------------------------------------------------------------ chunk walk
-// 512 threads (16 warps per SM to hide the shared-memory latency of the
-// products).  Shared memory of the walk (fp32); rows are padded (68 / 132 /
-// 36 floats) so that the column groups a warp reads at once fall in distinct
-// banks and every row stays 16-byte aligned.
-constexpr int kSbWalk = 512;
-constexpr int kSbXS = kSbP + 4;   // x, dout, dy silu'(z): [t][p]
-constexpr int kSbNS = kSbN + 4;   // B, C: [t][n]; h_0^T, dh^T: [p][n]
-constexpr int kSbTS = kSbQ + 4;   // x^T, dout^T: [p][t]; the Q x Q matrices
-struct SbSmem {
-    float xs[kSbQ][kSbXS], dos[kSbQ][kSbXS], zf[kSbQ][kSbXS];
-    float xsT[kSbP][kSbTS], dosT[kSbP][kSbTS];
-    float Bs[kSbQ][kSbNS], Cs[kSbQ][kSbNS];
-    float h0T[kSbP][kSbNS], dhT[kSbP][kSbNS];
-    // L.G.delta_s [t][s], (L.G)^T [s][t], L.delta_s.(dout x^T) [t][s], (L.(dout x^T))^T [s][t]
-    float Md[kSbQ][kSbTS], MmT[kSbQ][kSbTS], Wm[kSbQ][kSbTS], VmT[kSbQ][kSbTS];
-    float raw[kSbQ], dl[kSbQ], S[kSbQ], ecs[kSbQ], ecq[kSbQ], ddd[kSbQ], dyy[kSbQ];
-    float red[kSbWalk / 32];
-    float hqdh, ecQ;
-};
-
-// Block sum of one value per thread (every thread gets the total).
-__device__ __forceinline__ float sb_block_sum(float v, float *red, int tid)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    __syncthreads();  // red is free
-    if ((tid & 31) == 0)
-        red[tid >> 5] = v;
-    __syncthreads();
-    float t = 0.f;
-#pragma unroll
-    for (int w = 0; w < kSbWalk / 32; ++w)
-        t += red[w];
-    return t;
-}
-
-// Sum over the 16 consecutive lanes that share a row (lanes 16r .. 16r + 15).
-__device__ __forceinline__ float sb_sum16(float v)
-{
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    return v;
-}
-
-__device__ __forceinline__ float sb_dot4(float4 a, float4 b, float acc)
-{
-    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
-}
-
-template <typename T>
-__device__ __forceinline__ float4 sb_ld4(const T &ref)
-{
-    return *reinterpret_cast<const float4 *>(&ref);
 }
 
 // ---- warp-level tensor-core products (mma.sync m16n8k8, tf32 inputs, fp32
@@ -351,6 +183,158 @@ __device__ __forceinline__ void sb_zero(float (&d)[NT][4])
         d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
 }
 
+// ------------------------------------------------------------ forward states
+// Scratch layout of the stored states: per (batch, head) and chunk entry, 256
+// threads x 32 floats, thread-contiguous.  Thread u = 32 w + l holds the
+// accumulator fragments of rows 16 w .. 16 w + 15 (n) and all 64 columns (p)
+// in eight 16 x 8 tiles: float 4 t + e is element e of tile t, at row
+// n = 16 w + l / 4 + 8 (e / 2) and column p = 8 t + 2 (l % 4) + e % 2.
+__device__ __forceinline__ void sb_state_coord(int u, int f, int &n, int &pp)
+{
+    const int w = u >> 5, l = u & 31, t = f >> 2, e = f & 3;
+    n = 16 * w + (l >> 2) + 8 * (e >> 1);
+    pp = 8 * t + 2 * (l & 3) + (e & 1);
+}
+
+__global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const SsdBwdParams p)
+{
+    constexpr int Q = kSbQ, N = kSbN, P = kSbP;
+    __shared__ __align__(16) float Bs[Q][N + 4];
+    __shared__ __align__(16) float xs[Q][P + 4];
+    __shared__ __align__(16) float ws[Q];
+    __shared__ float s_decay;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.x, b = bh / p.H, hh = bh - b * p.H;
+    const int g = hh / p.heads_per_group;
+    const float A = p.A[hh];
+    const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
+
+    float hs[8][4];
+    {
+        const float *h0 = p.h0 ? p.h0 + (int64_t(b) * p.H + hh) * P * N : nullptr;
+#pragma unroll
+        for (int f = 0; f < 32; ++f) {
+            int n, pp;
+            sb_state_coord(tid, f, n, pp);
+            hs[f >> 2][f & 3] = h0 ? h0[int64_t(pp) * N + n] : 0.f;
+        }
+    }
+    float4 *st = reinterpret_cast<float4 *>(p.states) +
+                 (int64_t(bh) * (p.nchunks + 1) * kSbThreads + tid) * 8;
+    const int64_t chunk_stride = int64_t(kSbThreads) * 8;  // float4 per chunk entry
+    const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
+    const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
+
+    for (int c = 0; c < p.nchunks; ++c) {
+        float4 *sc = st + int64_t(c) * chunk_stride;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+            sc[t] = make_float4(hs[t][0], hs[t][1], hs[t][2], hs[t][3]);
+        const int t0 = c * Q, valid = min(Q, p.L - t0);
+        {
+            const int n = tid >> 1, half = tid & 1;  // row n, tokens 16 half .. + 15
+            const __nv_bfloat16 *src = Brow + int64_t(n) * p.B_ns + t0 + 16 * half;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int t = 16 * half + k;
+                Bs[t][n] = t < valid ? sb_bf(src[k]) : 0.f;
+            }
+        }
+        {
+            const int pp = tid >> 2, q = tid & 3;  // row p, tokens 8q .. 8q + 7
+            const __nv_bfloat16 *src = xrow + int64_t(pp) * p.x_cs + t0 + 8 * q;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int t = 8 * q + k;
+                xs[t][pp] = t < valid ? sb_bf(src[k]) : 0.f;
+            }
+        }
+        if (warp == 0) {
+            float raw, dl, S;
+            sb_steps(p, b, hh, t0, valid, lane, bias, raw, dl, S);
+            const float SQ = __shfl_sync(0xffffffffu, S, 31);
+            ws[lane] = expf(A * (SQ - S)) * dl;
+            if (lane == 0)
+                s_decay = expf(A * SQ);
+        }
+        __syncthreads();
+        // h = e^cs_Q h + sum_s (w_s B_s) x_s^T on the tensor cores
+        const float dec = s_decay;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                hs[t][e] *= dec;
+        sb_gemm<Q, 8, true>(hs, 16 * warp, 0, [&](int m, int k) { return ws[k] * Bs[k][m]; },
+                            [&](int k, int n) { return xs[k][n]; }, lane);
+        __syncthreads();
+    }
+    float4 *sc = st + int64_t(p.nchunks) * chunk_stride;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+        sc[t] = make_float4(hs[t][0], hs[t][1], hs[t][2], hs[t][3]);
+}
+
+// ------------------------------------------------------------ chunk walk
+// 512 threads (16 warps per SM to hide the shared-memory latency of the
+// products).  Shared memory of the walk (fp32); rows are padded (68 / 132 /
+// 36 floats) so that the column groups a warp reads at once fall in distinct
+// banks and every row stays 16-byte aligned.
+constexpr int kSbWalk = 512;
+constexpr int kSbXS = kSbP + 4;   // x, dout, dy silu'(z): [t][p]
+constexpr int kSbNS = kSbN + 4;   // B, C: [t][n]; h_0^T, dh^T: [p][n]
+constexpr int kSbTS = kSbQ + 4;   // x^T, dout^T: [p][t]; the Q x Q matrices
+struct SbSmem {
+    float xs[kSbQ][kSbXS], dos[kSbQ][kSbXS], zf[kSbQ][kSbXS];
+    float xsT[kSbP][kSbTS], dosT[kSbP][kSbTS];
+    float Bs[kSbQ][kSbNS], Cs[kSbQ][kSbNS];
+    float h0T[kSbP][kSbNS], dhT[kSbP][kSbNS];
+    // L.G.delta_s [t][s], (L.G)^T [s][t], L.delta_s.(dout x^T) [t][s], (L.(dout x^T))^T [s][t]
+    float Md[kSbQ][kSbTS], MmT[kSbQ][kSbTS], Wm[kSbQ][kSbTS], VmT[kSbQ][kSbTS];
+    float raw[kSbQ], dl[kSbQ], S[kSbQ], ecs[kSbQ], ecq[kSbQ], ddd[kSbQ], dyy[kSbQ];
+    float red[kSbWalk / 32];
+    float hqdh, ecQ;
+};
+
+// Block sum of one value per thread (every thread gets the total).
+__device__ __forceinline__ float sb_block_sum(float v, float *red, int tid)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();  // red is free
+    if ((tid & 31) == 0)
+        red[tid >> 5] = v;
+    __syncthreads();
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSbWalk / 32; ++w)
+        t += red[w];
+    return t;
+}
+
+// Sum over the 16 consecutive lanes that share a row (lanes 16r .. 16r + 15).
+__device__ __forceinline__ float sb_sum16(float v)
+{
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    return v;
+}
+
+__device__ __forceinline__ float sb_dot4(float4 a, float4 b, float acc)
+{
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+}
+
+template <typename T>
+__device__ __forceinline__ float4 sb_ld4(const T &ref)
+{
+    return *reinterpret_cast<const float4 *>(&ref);
+}
+
 template <bool GATE>
 __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams p)
 {
@@ -387,17 +371,19 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
     // thread halves (u = tid / 2 owns rows 4 (u % 32) + i, columns 8 (u / 32) + j)
     float hq_next = 0.f;
     if (p.dlast) {
-        const int u = tid >> 1, ih = tid & 1;
+        const int u = tid >> 1, ih = tid & 1;  // floats 16 ih .. 16 ih + 15 of thread u
         const float4 *sf = st_base + int64_t(p.nchunks) * chunk_stride + u * 8 + 4 * ih;
         const float *dl0 = p.dlast + (int64_t(b) * p.H + hh) * P * N;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float4 a0 = sf[2 * i], a1 = sf[2 * i + 1];
-            const float hv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const int n = 4 * (u & 31) + 2 * ih + i;
+        for (int v = 0; v < 4; ++v) {
+            const float4 a = sf[v];
+            const float hv[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                hq_next = fmaf(dl0[int64_t(8 * (u >> 5) + j) * N + n], hv[j], hq_next);
+            for (int e = 0; e < 4; ++e) {
+                int n, pp;
+                sb_state_coord(u, 16 * ih + 4 * v + e, n, pp);
+                hq_next = fmaf(dl0[int64_t(pp) * N + n], hv[e], hq_next);
+            }
         }
     }
     hq_next = sb_block_sum(hq_next, sm.red, tid);
@@ -458,16 +444,18 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             }
         }
         {
-            const int u = tid >> 1, ih = tid & 1;
+            const int u = tid >> 1, ih = tid & 1;  // floats 16 ih .. 16 ih + 15 of thread u
             const float4 *s0 = st_base + int64_t(c) * chunk_stride + u * 8 + 4 * ih;
-            const int n0 = 4 * (u & 31) + 2 * ih, pb = u >> 5;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const float4 a0 = s0[2 * i], a1 = s0[2 * i + 1];
-                const float h0v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            for (int v = 0; v < 4; ++v) {
+                const float4 a = s0[v];
+                const float hv[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    sm.h0T[8 * pb + j][n0 + i] = h0v[j];
+                for (int e = 0; e < 4; ++e) {
+                    int n, pp;
+                    sb_state_coord(u, 16 * ih + 4 * v + e, n, pp);
+                    sm.h0T[pp][n] = hv[e];
+                }
             }
         }
 #pragma unroll
