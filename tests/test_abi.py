@@ -232,6 +232,46 @@ def test_bwd_rejects(over, expect):
     assert _bwd(**over) == C[expect]
 
 
+def _bwd_sa(**over):
+    b, H, P, N, L, G = 2, 4, 64, 128, 64, 1
+    f32 = ss.SELSCAN_F32
+    args = dict(x=_t((b, H * P, L)), dt=_t((b, H, L), f32), bias=None, A=_t((H,), f32),
+                B=_t((b, G, N, L)), C=_t((b, G, N, L)), Dv=None, z=None, P=P, h0=None,
+                dy=_t((b, H * P, L)), dlast=None, dx=_t((b, H * P, L)), ddt=_t((b, H, L), f32),
+                dA=_t((H,), f32), dB=_t((b, G, N, L), f32), dC=_t((b, G, N, L), f32),
+                dD=None, dz=None, dbias=None, dh0=None)
+    args.update(over)
+    r = lambda x: None if x is None else ctypes.byref(x)
+    mid = ("A", "B", "C", "Dv", "z")
+    tail = ("h0", "dy", "dlast", "dx", "ddt", "dA", "dB", "dC", "dD", "dz", "dbias", "dh0")
+    return ss.lib().selscan_bwd_scalarA(r(args["x"]), r(args["dt"]), r(args["bias"]), 0,
+                                        *[r(args[k]) for k in mid], args["P"],
+                                        *[r(args[k]) for k in tail], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(x=None), "SELSCAN_ERR_NULL"),
+    (dict(dy=None), "SELSCAN_ERR_NULL"),
+    (dict(ddt=None), "SELSCAN_ERR_NULL"),
+    (dict(dB=None), "SELSCAN_ERR_NULL"),
+    (dict(z=_t((2, 256, 64))), "SELSCAN_ERR_NULL"),           # gate given, dz missing
+    (dict(P=48), "SELSCAN_ERR_SHAPE"),
+    (dict(x=_t((2, 256, 64), ss.SELSCAN_F32)), "SELSCAN_ERR_DTYPE"),
+    (dict(dt=_t((2, 4, 64))), "SELSCAN_ERR_DTYPE"),             # bf16 step sizes
+    (dict(ddt=_t((2, 4, 63), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(dB=_t((2, 1, 128, 64))), "SELSCAN_ERR_DTYPE"),        # bf16 gradient of B
+    (dict(dC=_t((2, 2, 128, 64), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(dh0=_t((2, 4, 64, 64), ss.SELSCAN_F32)), "SELSCAN_ERR_SHAPE"),
+    (dict(B=_t((2, 3, 128, 64)), C=_t((2, 3, 128, 64))), "SELSCAN_ERR_SHAPE"),  # 3 does not divide 4
+    (dict(B=_t((2, 1, 128, 64), strides=(128 * 128, 128 * 128, 128, 2))), "SELSCAN_ERR_STRIDE"),
+    (dict(dx=_t((2, 256, 64), data=FAKE + 8)), "SELSCAN_ERR_ALIGN"),
+    (dict(B=_t((2, 1, 64, 64)), C=_t((2, 1, 64, 64)), dB=_t((2, 1, 64, 64), ss.SELSCAN_F32),
+          dC=_t((2, 1, 64, 64), ss.SELSCAN_F32)), "SELSCAN_ERR_UNSUPPORTED"),
+])
+def test_bwd_scalarA_rejects(over, expect):
+    assert _bwd_sa(**over) == C[expect]
+
+
 def test_backward_segment_plan():
     """The backward's choice of time segments (host arithmetic, no GPU):
     ceil(units / slots) / S is minimised over at most four waves, with at
