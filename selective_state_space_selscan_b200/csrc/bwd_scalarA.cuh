@@ -507,52 +507,56 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
         }
         __syncthreads();
 
-        // ---- 3a. y~ (rows t) and u (rows s): 32 x 64 each; warp w holds the
-        //          16 x 8 tile (16 (w / 8), 8 (w % 8)) of both
+        // ---- 3a. y~ (rows t, warps 0-7) and u (rows s, warps 8-15), 32 x 64
+        //          each; warp w holds rows 16 ((w / 4) % 2), columns 16 (w % 4) .. + 15
         {
-            const int m0 = 16 * (warp >> 3), n0 = 8 * (warp & 7);
-            float y1[1][4], y2[1][4], u1[1][4], u2[1][4];
-            sb_zero(y1);
-            sb_zero(y2);
-            sb_zero(u1);
-            sb_zero(u2);
-            sb_gemm<Q, 1, true>(y1, m0, n0, [&](int m, int k) { return sm.Md[m][k]; },
-                          [&](int k, int n) { return sm.xsT[n][k]; }, lane);
-            sb_gemm<N, 1, true>(y2, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
-                          [&](int k, int n) { return sm.h0T[n][k]; }, lane);
-            sb_gemm<Q, 1, true>(u1, m0, n0, [&](int m, int k) { return sm.MmT[m][k]; },
-                          [&](int k, int n) { return sm.dosT[n][k]; }, lane);
-            sb_gemm<N, 1, true>(u2, m0, n0, [&](int m, int k) { return sm.Bs[m][k]; },
-                          [&](int k, int n) { return sm.dhT[n][k]; }, lane);
-            float xu[2] = {0.f, 0.f}, dyy[2] = {0.f, 0.f};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int hr = e >> 1, r = m0 + g8 + 8 * hr, pp = n0 + 2 * q4 + (e & 1);
-                const float yt = fmaf(sm.ecs[r], y2[0][e], y1[0][e]);
-                const float uu = fmaf(sm.ecq[r], u2[0][e], u1[0][e]);
-                const float xv = sm.xs[r][pp], dv = sm.dos[r][pp];
-                xu[hr] = fmaf(xv, uu, xu[hr]);
-                dyy[hr] = fmaf(dv, yt, dyy[hr]);
-                accD = fmaf(dv, xv, accD);
-                if (r < valid) {
-                    const int64_t row_t = t0 + r;
-                    p.dx[int64_t(b) * p.dx_bs + int64_t(hh * P + pp) * p.dx_cs + row_t] =
-                        __float2bfloat16_rn(fmaf(sm.dl[r], uu, dsk * dv));
-                    if (GATE)
-                        p.dz[int64_t(b) * p.dz_bs + int64_t(hh * P + pp) * p.dz_cs + row_t] =
-                            __float2bfloat16_rn(sm.zf[r][pp] * fmaf(dsk, xv, yt));
-                }
+            const bool isy = warp < 8;
+            const int m0 = 16 * ((warp >> 2) & 1), n0 = 16 * (warp & 3);
+            float v1[2][4], v2[2][4];
+            sb_zero(v1);
+            sb_zero(v2);
+            if (isy) {
+                sb_gemm<Q, 2, true>(v1, m0, n0, [&](int m, int k) { return sm.Md[m][k]; },
+                                    [&](int k, int n) { return sm.xsT[n][k]; }, lane);
+                sb_gemm<N, 2, true>(v2, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
+                                    [&](int k, int n) { return sm.h0T[n][k]; }, lane);
+            } else {
+                sb_gemm<Q, 2, true>(v1, m0, n0, [&](int m, int k) { return sm.MmT[m][k]; },
+                                    [&](int k, int n) { return sm.dosT[n][k]; }, lane);
+                sb_gemm<N, 2, true>(v2, m0, n0, [&](int m, int k) { return sm.Bs[m][k]; },
+                                    [&](int k, int n) { return sm.dhT[n][k]; }, lane);
             }
+            float rs[2] = {0.f, 0.f};  // x.u (u warps) or dout.y~ (y~ warps) per row
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int hr = e >> 1, r = m0 + g8 + 8 * hr;
+                    const int pp = n0 + 8 * t + 2 * q4 + (e & 1);
+                    const float xv = sm.xs[r][pp], dv = sm.dos[r][pp];
+                    const int64_t col = int64_t(hh * P + pp);
+                    if (isy) {
+                        const float yt = fmaf(sm.ecs[r], v2[t][e], v1[t][e]);
+                        rs[hr] = fmaf(dv, yt, rs[hr]);
+                        accD = fmaf(dv, xv, accD);
+                        if (GATE && r < valid)
+                            p.dz[int64_t(b) * p.dz_bs + col * p.dz_cs + t0 + r] =
+                                __float2bfloat16_rn(sm.zf[r][pp] * fmaf(dsk, xv, yt));
+                    } else {
+                        const float uu = fmaf(sm.ecq[r], v2[t][e], v1[t][e]);
+                        rs[hr] = fmaf(xv, uu, rs[hr]);
+                        if (r < valid)
+                            p.dx[int64_t(b) * p.dx_bs + col * p.dx_cs + t0 + r] =
+                                __float2bfloat16_rn(fmaf(sm.dl[r], uu, dsk * dv));
+                    }
+                }
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
-                xu[hr] += __shfl_xor_sync(0xffffffffu, xu[hr], 1);
-                xu[hr] += __shfl_xor_sync(0xffffffffu, xu[hr], 2);
-                dyy[hr] += __shfl_xor_sync(0xffffffffu, dyy[hr], 1);
-                dyy[hr] += __shfl_xor_sync(0xffffffffu, dyy[hr], 2);
-                if (q4 == 0) {
-                    atomicAdd(&sm.ddd[m0 + g8 + 8 * hr], xu[hr]);
-                    atomicAdd(&sm.dyy[m0 + g8 + 8 * hr], dyy[hr]);
-                }
+                rs[hr] += __shfl_xor_sync(0xffffffffu, rs[hr], 1);
+                rs[hr] += __shfl_xor_sync(0xffffffffu, rs[hr], 2);
+                if (q4 == 0)
+                    atomicAdd(isy ? &sm.dyy[m0 + g8 + 8 * hr] : &sm.ddd[m0 + g8 + 8 * hr],
+                              rs[hr]);
             }
         }
         // ---- 3b. dC (warps 0-7) and dB (warps 8-15): 32 x 128 each; warp
