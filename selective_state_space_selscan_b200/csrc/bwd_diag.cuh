@@ -440,7 +440,10 @@ bwd_agg_kernel(const BwdParams p)
             if (fwd) {
                 bwd_vals<T, KV>(st[buf].u, lane, uv);
                 bwd_bc_to_smem<T, KV>(st[buf], sm, lane, false);
-                bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane, dts);
+                if (valid == kBwdT)  // a constant token count for whole chunks
+                    bwd_forward_chunk<T, false>(p, ch, sm, kBwdT, uv, dv, h2, lane, dts);
+                else
+                    bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane, dts);
             }
             __syncwarp();
             buf ^= 1;
@@ -474,25 +477,33 @@ bwd_agg_kernel(const BwdParams p)
             bwd_vals<T, KV>(st[buf].dy, lane, yv);
             if (p.z)
                 bwd_vals<T, KV>(st[buf].z, lane, zv);
+            auto walk = [&](auto full_tag) {
+                const int vld = decltype(full_tag)::value ? kBwdT : valid;
 #pragma unroll
-            for (int i = kBwdT - 1; i >= 0; --i) {
-                if (i >= valid)
-                    continue;
-                const float dt = bwd_step<FAST>(dv[i] + ch.bias, p.softplus);
-                float dout = live ? yv[i] : 0.f;
-                if (p.z)
-                    dout *= zv[i] / (1.f + __expf(-zv[i]));
-                const uint64_t DO = pk2(dout, dout);
-                uint64_t a2[8];
-                bwd_decays<FAST>(dt, ch.al, ch.pow_path, a2);
-                const float4 *cq = reinterpret_cast<const float4 *>(sm.bc[i][1]);
+                for (int i = kBwdT - 1; i >= 0; --i) {
+                    if (i >= vld)
+                        continue;
+                    const float dt = bwd_step<FAST>(dv[i] + ch.bias, p.softplus);
+                    float dout = live ? yv[i] : 0.f;
+                    if (p.z)
+                        dout *= zv[i] / (1.f + __expf(-zv[i]));
+                    const uint64_t DO = pk2(dout, dout);
+                    uint64_t a2[8];
+                    bwd_decays<FAST>(dt, ch.al, ch.pow_path, a2);
+                    const float4 *cq = reinterpret_cast<const float4 *>(sm.bc[i][1]);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 cc = cq[q];
-                    g2[2 * q] = mul2(a2[2 * q], fma2(DO, pk2(cc.x, cc.y), g2[2 * q]));
-                    g2[2 * q + 1] = mul2(a2[2 * q + 1], fma2(DO, pk2(cc.z, cc.w), g2[2 * q + 1]));
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 cc = cq[q];
+                        g2[2 * q] = mul2(a2[2 * q], fma2(DO, pk2(cc.x, cc.y), g2[2 * q]));
+                        g2[2 * q + 1] =
+                            mul2(a2[2 * q + 1], fma2(DO, pk2(cc.z, cc.w), g2[2 * q + 1]));
+                    }
                 }
-            }
+            };
+            if (valid == kBwdT)  // a constant token count for whole chunks
+                walk(std::true_type{});
+            else
+                walk(std::false_type{});
             __syncwarp();
             buf ^= 1;
         }
@@ -591,7 +602,10 @@ selscan_bwd_kernel(const BwdParams p)
             bwd_vals<T, KV>(st[buf].u, lane, uv);
             bwd_vals<T, KV>(st[buf].dl, lane, dv);
             bwd_bc_to_smem<T, KV>(st[buf], sm, lane, false);
-            bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane, dts);
+            if (valid == TC)  // a constant token count for whole chunks
+                bwd_forward_chunk<T, false>(p, ch, sm, TC, uv, dv, h2, lane, dts);
+            else
+                bwd_forward_chunk<T, false>(p, ch, sm, valid, uv, dv, h2, lane, dts);
             __syncwarp();
             buf ^= 1;
         }
@@ -620,138 +634,149 @@ selscan_bwd_kernel(const BwdParams p)
                              t0 - TC, TC, lane, whatB, ck + (c - 1) * N);
         cp_async_commit();
         cp_async_wait<1>();
-        const BwdStage<KV> &cur = st[bufB];
-        uint64_t hc2[8];  // state before the chunk
+        // whole chunks (all but a ragged last one) take a copy of the walk in
+        // which the number of tokens is a constant, so the unrolled token loop
+        // keeps its registers in place from one token to the next
+        auto chunk = [&](auto full_tag) {
+            constexpr bool FULL = decltype(full_tag)::value;
+            const int vld = FULL ? TC : valid;
+            const BwdStage<KV> &cur = st[bufB];
+            uint64_t hc2[8];  // state before the chunk
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 v = live ? cur.ck[q][lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-            hc2[2 * q] = pk2(v.x, v.y);
-            hc2[2 * q + 1] = pk2(v.z, v.w);
-        }
-        float uv[8], dv[8], yv[8], zv[8], dts[8];
-        bwd_vals<T, KV>(cur.u, lane, uv);
-        bwd_vals<T, KV>(cur.dl, lane, dv);
-        bwd_vals<T, KV>(cur.dy, lane, yv);
-        if (p.z)
-            bwd_vals<T, KV>(cur.z, lane, zv);
-        bwd_bc_to_smem<T, KV>(cur, sm, lane, true);
-        {
-            uint64_t hr[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                hr[j] = hc2[j];
-            bwd_forward_chunk<T, true>(p, ch, sm, valid, uv, dv, hr, lane, dts);
-        }
-        __syncwarp();
-        // output gradient through the gate and the factor of dz, per token
-        float dov[8], fzv[8];
-#pragma unroll
-        for (int i = 0; i < TC; ++i) {
-            const float dyv = (live && i < valid) ? yv[i] : 0.f;
-            float dout = dyv, f = 0.f;
-            if (p.z) {
-                const float zz = zv[i];
-                const float sg = 1.f / (1.f + __expf(-zz));
-                f = dyv * (sg * (1.f + zz * (1.f - sg)));
-                dout = dyv * zz * sg;
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = live ? cur.ck[q][lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+                hc2[2 * q] = pk2(v.x, v.y);
+                hc2[2 * q + 1] = pk2(v.z, v.w);
             }
-            dov[i] = dout;
-            fzv[i] = f;
-            sm.dout[i][lane] = dout;
-        }
-        __syncwarp();
-        // dC of the chunk: lane -> token ri, states 4 rc .. 4 rc + 3
-        const int ri = lane >> 2, rc = lane & 3;
-        const float4 dCv = bwd_piece_sum<true>(sm, ri, rc);
-        __syncwarp();  // all rows read before the walk overwrites them
-        float o_du[8], o_dd[8], o_dz[8];
-#pragma unroll
-        for (int i = 0; i < TC; ++i)
-            o_du[i] = o_dd[i] = o_dz[i] = 0.f;
-        uint64_t ht2[8];  // state after token i, carried down from token i + 1
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            ht2[j] = pk2(0.f, 0.f);
-#pragma unroll
-        for (int i = TC - 1; i >= 0; --i) {
-            if (i >= valid)
-                continue;
-            if (i == valid - 1)
-                bwd_get_row(sm, i, lane, ht2);
-            uint64_t hp2[8];
-            if (i > 0) {
-                bwd_get_row(sm, i - 1, lane, hp2);
-            } else {
+            float uv[8], dv[8], yv[8], zv[8], dts[8];
+            bwd_vals<T, KV>(cur.u, lane, uv);
+            bwd_vals<T, KV>(cur.dl, lane, dv);
+            bwd_vals<T, KV>(cur.dy, lane, yv);
+            if (p.z)
+                bwd_vals<T, KV>(cur.z, lane, zv);
+            bwd_bc_to_smem<T, KV>(cur, sm, lane, true);
+            {
+                uint64_t hr[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    hp2[j] = hc2[j];
+                    hr[j] = hc2[j];
+                bwd_forward_chunk<T, true>(p, ch, sm, vld, uv, dv, hr, lane, dts);
             }
-            const float raw = dv[i] + ch.bias;
-            const float dt = dts[i];
-            const float x = uv[i];
-            uint64_t a2[8];
-            bwd_decays<FAST>(dt, ch.al, ch.pow_path, a2);
-            uint64_t B2[8], C2[8];
-            {
-                const float4 *bq = reinterpret_cast<const float4 *>(sm.bc[i][0]);
-                const float4 *cq = reinterpret_cast<const float4 *>(sm.bc[i][1]);
+            __syncwarp();
+            // output gradient through the gate and the factor of dz, per token
+            float dov[8], fzv[8];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 bb = bq[q], cc = cq[q];
-                    B2[2 * q] = pk2(bb.x, bb.y);
-                    B2[2 * q + 1] = pk2(bb.z, bb.w);
-                    C2[2 * q] = pk2(cc.x, cc.y);
-                    C2[2 * q + 1] = pk2(cc.z, cc.w);
+            for (int i = 0; i < TC; ++i) {
+                const float dyv = (live && i < vld) ? yv[i] : 0.f;
+                float dout = dyv, f = 0.f;
+                if (p.z) {
+                    const float zz = zv[i];
+                    const float sg = 1.f / (1.f + __expf(-zz));
+                    f = dyv * (sg * (1.f + zz * (1.f - sg)));
+                    dout = dyv * zz * sg;
                 }
+                dov[i] = dout;
+                fzv[i] = f;
+                sm.dout[i][lane] = dout;
             }
-            if (p.z) {
-                uint64_t Y2 = mul2(C2[0], ht2[0]);
+            __syncwarp();
+            // dC of the chunk: lane -> token ri, states 4 rc .. 4 rc + 3
+            const int ri = lane >> 2, rc = lane & 3;
+            const float4 dCv = bwd_piece_sum<true>(sm, ri, rc);
+            __syncwarp();  // all rows read before the walk overwrites them
+            float o_du[8], o_dd[8], o_dz[8];
 #pragma unroll
-                for (int j = 1; j < 8; ++j)
-                    Y2 = fma2(C2[j], ht2[j], Y2);
-                o_dz[i] = fzv[i] * fmaf(ch.dsk, x, lo2(Y2) + hi2(Y2));
-            }
-            const float dout = dov[i];
-            gD = fmaf(dout, x, gD);
-            // with g after adding dout C:  du = dt sum g B + D dout,
-            // ddelta = sum g A abar h_prev + u sum g B,  dA += dt g abar h_prev
-            const uint64_t DO = pk2(dout, dout), DT = pk2(dt, dt);
-            const uint64_t DTX = pk2(dt * x, dt * x);
-            uint64_t gB2 = pk2(0.f, 0.f), gAh2 = pk2(0.f, 0.f), vb[8];
+            for (int i = 0; i < TC; ++i)
+                o_du[i] = o_dd[i] = o_dz[i] = 0.f;
+            uint64_t ht2[8];  // state after token i, carried down from token i + 1
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                g2[j] = fma2(DO, C2[j], g2[j]);
-                vb[j] = mul2(g2[j], DTX);
-                gB2 = fma2(g2[j], B2[j], gB2);
-                const uint64_t gah = mul2(g2[j], mul2(a2[j], hp2[j]));
-                gAh2 = fma2(ch.An2[j], gah, gAh2);
-                gA2[j] = fma2(DT, gah, gA2[j]);
-                g2[j] = mul2(g2[j], a2[j]);
-                ht2[j] = hp2[j];
+            for (int j = 0; j < 8; ++j)
+                ht2[j] = pk2(0.f, 0.f);
+#pragma unroll
+            for (int i = TC - 1; i >= 0; --i) {
+                if (i >= vld)
+                    continue;
+                if (i == vld - 1)
+                    bwd_get_row(sm, i, lane, ht2);
+                uint64_t hp2[8];
+                if (i > 0) {
+                    bwd_get_row(sm, i - 1, lane, hp2);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        hp2[j] = hc2[j];
+                }
+                const float raw = dv[i] + ch.bias;
+                const float dt = dts[i];
+                const float x = uv[i];
+                uint64_t a2[8];
+                bwd_decays<FAST>(dt, ch.al, ch.pow_path, a2);
+                uint64_t B2[8], C2[8];
+                {
+                    const float4 *bq = reinterpret_cast<const float4 *>(sm.bc[i][0]);
+                    const float4 *cq = reinterpret_cast<const float4 *>(sm.bc[i][1]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 bb = bq[q], cc = cq[q];
+                        B2[2 * q] = pk2(bb.x, bb.y);
+                        B2[2 * q + 1] = pk2(bb.z, bb.w);
+                        C2[2 * q] = pk2(cc.x, cc.y);
+                        C2[2 * q + 1] = pk2(cc.z, cc.w);
+                    }
+                }
+                if (p.z) {
+                    uint64_t Y2 = mul2(C2[0], ht2[0]);
+#pragma unroll
+                    for (int j = 1; j < 8; ++j)
+                        Y2 = fma2(C2[j], ht2[j], Y2);
+                    o_dz[i] = fzv[i] * fmaf(ch.dsk, x, lo2(Y2) + hi2(Y2));
+                }
+                const float dout = dov[i];
+                gD = fmaf(dout, x, gD);
+                // with g after adding dout C:  du = dt sum g B + D dout,
+                // ddelta = sum g A abar h_prev + u sum g B,  dA += dt g abar h_prev
+                const uint64_t DO = pk2(dout, dout), DT = pk2(dt, dt);
+                const uint64_t DTX = pk2(dt * x, dt * x);
+                uint64_t gB2 = pk2(0.f, 0.f), gAh2 = pk2(0.f, 0.f), vb[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    g2[j] = fma2(DO, C2[j], g2[j]);
+                    vb[j] = mul2(g2[j], DTX);
+                    gB2 = fma2(g2[j], B2[j], gB2);
+                    const uint64_t gah = mul2(g2[j], mul2(a2[j], hp2[j]));
+                    gAh2 = fma2(ch.An2[j], gah, gAh2);
+                    gA2[j] = fma2(DT, gah, gA2[j]);
+                    g2[j] = mul2(g2[j], a2[j]);
+                    ht2[j] = hp2[j];
+                }
+                bwd_put_row(sm, i, lane, vb);  // this lane's dB terms of token i
+                const float gB = lo2(gB2) + hi2(gB2);
+                const float dx = fmaf(dout, ch.dsk, dt * gB);
+                const float ddt = fmaf(x, gB, lo2(gAh2) + hi2(gAh2));
+                const float dDelta = p.softplus ? ddt / (1.f + __expf(-raw)) : ddt;
+                gbias += dDelta;
+                o_du[i] = dx;
+                o_dd[i] = dDelta;
             }
-            bwd_put_row(sm, i, lane, vb);  // this lane's dB terms of token i
-            const float gB = lo2(gB2) + hi2(gB2);
-            const float dx = fmaf(dout, ch.dsk, dt * gB);
-            const float ddt = fmaf(x, gB, lo2(gAh2) + hi2(gAh2));
-            const float dDelta = p.softplus ? ddt / (1.f + __expf(-raw)) : ddt;
-            gbias += dDelta;
-            o_du[i] = dx;
-            o_dd[i] = dDelta;
-        }
-        __syncwarp();
-        const float4 dBv = bwd_piece_sum<false>(sm, ri, rc);
-        if (live) {
-            bwd_st8(p.du, ch.row_du + t0, valid, o_du, tag);
-            bwd_st8(p.ddelta, ch.row_dd + t0, valid, o_dd, tag);
-            if (p.z)
-                bwd_st8(p.dz, ch.row_dz + t0, valid, o_dz, tag);
-        }
-        if (ri < valid) {
-            const int64_t off = ((int64_t(tile % kBwdCopies) * p.batch + b) * p.L + t0 + ri) * N +
-                                4 * rc;
-            atomicAdd(reinterpret_cast<float4 *>(p.pB + off), dBv);
-            atomicAdd(reinterpret_cast<float4 *>(p.pC + off), dCv);
-        }
+            __syncwarp();
+            const float4 dBv = bwd_piece_sum<false>(sm, ri, rc);
+            if (live) {
+                bwd_st8(p.du, ch.row_du + t0, vld, o_du, tag);
+                bwd_st8(p.ddelta, ch.row_dd + t0, vld, o_dd, tag);
+                if (p.z)
+                    bwd_st8(p.dz, ch.row_dz + t0, vld, o_dz, tag);
+            }
+            if (ri < vld) {
+                const int64_t off = ((int64_t(tile % kBwdCopies) * p.batch + b) * p.L + t0 + ri) * N +
+                                    4 * rc;
+                atomicAdd(reinterpret_cast<float4 *>(p.pB + off), dBv);
+                atomicAdd(reinterpret_cast<float4 *>(p.pC + off), dCv);
+            }
+        };
+        if (valid == TC)
+            chunk(std::true_type{});
+        else
+            chunk(std::false_type{});
         __syncwarp();
         bufB ^= 1;
     }
