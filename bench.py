@@ -888,7 +888,7 @@ def bwd_bytes(cfg: dict) -> int:
 
 # DRAM bytes per backward call (ncu, profiles/selscan_bwd_config2.md): captured
 # at L = 1024 on the B4 D5120 layer, scaled by tokens to L = 4096
-BWD_NCU_TRAFFIC = {2: ("selscan_bwd_kernel v4", 4 * 622.3e6)}
+BWD_NCU_TRAFFIC = {2: ("selscan_bwd_kernel v5", 4 * 687.2e6)}
 BWD_KERNEL_TAG = "selscan_bwd_kernel v5"
 
 
