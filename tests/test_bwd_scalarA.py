@@ -115,3 +115,48 @@ def test_zero_upstream_gradient():
     for k, v in g.items():
         if v is not None:
             assert np.all(v == 0.0), k
+
+
+def test_full_size_config4_sampled_heads():
+    """The benchmark's workload (B4 H32 P64 N128 G1 L4096) in its launch
+    configuration, with an upstream gradient that is zero outside two heads
+    (5 and 26): every other head then contributes exactly zero to every
+    gradient, so the oracle run on those two heads alone gives the whole
+    expected dB and dC, and dx, ddt, dA, dD of the two heads; the other heads'
+    dx, ddt, dA and dD must be exactly zero.  The two heads' oracle runs go on
+    two host threads (ctypes releases the interpreter lock)."""
+    from concurrent.futures import ThreadPoolExecutor
+    inp = synthetic.make_config(4)
+    H = inp["A"].shape[0]
+    heads = (5, 26)
+    rng = np.random.default_rng(404)
+    dy = np.zeros(inp["x"].shape, np.float32)
+    for h in heads:
+        dy[:, h * P:(h + 1) * P] = synthetic.round_bf16(
+            rng.standard_normal((inp["x"].shape[0], P, inp["x"].shape[2])).astype(np.float32))
+    inp.update(softplus=False, dt_bias=None, h0=None, dlast=None, dy=dy)
+    got = run_gpu(inp)
+
+    def one(h):
+        ch = slice(h * P, (h + 1) * P)
+        return oracle.selscan_scalarA_bwd(inp["x"][:, ch], inp["dt"][:, h:h + 1],
+                                          inp["A"][h:h + 1], inp["B"], inp["C"], P, dy[:, ch],
+                                          D=inp["D"][h:h + 1])
+
+    with ThreadPoolExecutor(len(heads)) as ex:
+        want = list(ex.map(one, heads))
+    others = [h for h in range(H) if h not in heads]
+    for h, w in zip(heads, want):
+        ch = slice(h * P, (h + 1) * P)
+        assert rel(got["dx"][:, ch], w["dx"]) <= 5e-3, ("dx", h)
+        assert rel(got["ddt"][:, h:h + 1], w["ddt"]) <= 2e-3, ("ddt", h)
+        assert abs(got["dA"][h] - w["dA"][0]) <= 2e-3 * abs(w["dA"][0]), ("dA", h)
+        assert abs(got["dD"][h] - w["dD"][0]) <= 2e-3 * abs(w["dD"][0]), ("dD", h)
+    for k in ("dB", "dC"):
+        total = want[0][k] + want[1][k]
+        e = rel(got[k].reshape(total.shape), total)
+        assert e <= 2e-3, (k, e)
+    oc = np.concatenate([np.arange(h * P, (h + 1) * P) for h in others])
+    assert np.all(got["dx"][:, oc] == 0.0)
+    assert np.all(got["ddt"][:, others] == 0.0)
+    assert np.all(got["dA"][others] == 0.0) and np.all(got["dD"][others] == 0.0)
