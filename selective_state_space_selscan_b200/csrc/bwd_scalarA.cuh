@@ -36,10 +36,11 @@
 //     accumulator fragments and evaluates the products above from shared
 //     memory (32-token chunks keep every product's operands on chip).
 // Every product runs on the tensor cores as warp-level m16n8k8 tiles with
-// tf32 operands and fp32 accumulation; the products whose results feed the
-// step-size gradients (differences of nearly equal sums) and the two state
-// recurrences split each operand into two tf32 parts (three products), which
-// keeps about 21 bits of every operand.
+// tf32 operands and fp32 accumulation.  In the products whose results feed
+// the step-size gradients (differences of nearly equal sums) and in the two
+// state recurrences, every operand that is not a bf16 input is split into two
+// tf32 parts (one extra product each), which keeps about 21 bits of it; bf16
+// inputs are exact in tf32.
 // dB and dC sum over the heads of a group: each head adds its chunk terms
 // with 16-byte atomics into one of kSbCopies partial copies ([t][n] rows),
 // and ssd_bwd_reduce_bc sums the copies into (batch, G, N, L).  dA, dD and
@@ -134,11 +135,12 @@ __device__ __forceinline__ void sb_split(float x, uint32_t &hi, uint32_t &lo)
 
 // D[NT tiles] += sum_{k < K} A(m0 + row, k) B(k, n0 + 8 t + col): one A
 // fragment per k step serves NT output tiles.  fa(m, k) and fb(k, n) read
-// the operands from shared memory in whatever layout they are kept.  SPLIT:
-// each operand as the sum of two tf32 numbers and three products (hi hi, hi
-// lo, lo hi), which carries about the 21 leading bits of fp32 into the
-// products that feed the differences of the step-size gradients.
-template <int K, int NT, bool SPLIT, typename FA, typename FB>
+// the operands from shared memory in whatever layout they are kept.  SA / SB:
+// that operand is taken as the sum of two tf32 numbers, with one extra
+// product per split operand (hi hi, then lo hi and / or hi lo), which keeps
+// about 21 bits of it; an operand that holds bf16 values (x, B, C, dy) is
+// exact in tf32 and is not split.
+template <int K, int NT, bool SA, bool SB, typename FA, typename FB>
 __device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, FA fa, FB fb,
                                         int lane)
 {
@@ -150,7 +152,7 @@ __device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, FA fa
         uint32_t ah[4], al[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            if (SPLIT)
+            if (SA)
                 sb_split(av[i], ah[i], al[i]);
             else
                 ah[i] = sb_tf32(av[i]);
@@ -161,15 +163,15 @@ __device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, FA fa
             uint32_t bh[2], bl[2];
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-                if (SPLIT)
+                if (SB)
                     sb_split(bv[i], bh[i], bl[i]);
                 else
                     bh[i] = sb_tf32(bv[i]);
             }
-            if (SPLIT) {
+            if (SA)
                 sb_mma(d[t], al, bh);
+            if (SB)
                 sb_mma(d[t], ah, bl);
-            }
             sb_mma(d[t], ah, bh);
         }
     }
@@ -266,7 +268,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 hs[t][e] *= dec;
-        sb_gemm<Q, 8, true>(hs, 16 * warp, 0, [&](int m, int k) { return ws[k] * Bs[k][m]; },
+        sb_gemm<Q, 8, true, false>(hs, 16 * warp, 0, [&](int m, int k) { return ws[k] * Bs[k][m]; },
                             [&](int k, int n) { return xs[k][n]; }, lane);
         __syncthreads();
     }
@@ -486,10 +488,10 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             float acc[1][4];
             sb_zero(acc);
             if (warp < 8)
-                sb_gemm<N, 1, true>(acc, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
+                sb_gemm<N, 1, false, false>(acc, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
                               [&](int k, int n) { return sm.Bs[n][k]; }, lane);
             else
-                sb_gemm<P, 1, true>(acc, m0, n0, [&](int m, int k) { return sm.dos[m][k]; },
+                sb_gemm<P, 1, GATE, false>(acc, m0, n0, [&](int m, int k) { return sm.dos[m][k]; },
                               [&](int k, int n) { return sm.xs[n][k]; }, lane);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -516,14 +518,14 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             sb_zero(v1);
             sb_zero(v2);
             if (isy) {
-                sb_gemm<Q, 2, true>(v1, m0, n0, [&](int m, int k) { return sm.Md[m][k]; },
+                sb_gemm<Q, 2, true, false>(v1, m0, n0, [&](int m, int k) { return sm.Md[m][k]; },
                                     [&](int k, int n) { return sm.xsT[n][k]; }, lane);
-                sb_gemm<N, 2, true>(v2, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
+                sb_gemm<N, 2, false, true>(v2, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
                                     [&](int k, int n) { return sm.h0T[n][k]; }, lane);
             } else {
-                sb_gemm<Q, 2, true>(v1, m0, n0, [&](int m, int k) { return sm.MmT[m][k]; },
+                sb_gemm<Q, 2, true, GATE>(v1, m0, n0, [&](int m, int k) { return sm.MmT[m][k]; },
                                     [&](int k, int n) { return sm.dosT[n][k]; }, lane);
-                sb_gemm<N, 2, true>(v2, m0, n0, [&](int m, int k) { return sm.Bs[m][k]; },
+                sb_gemm<N, 2, false, true>(v2, m0, n0, [&](int m, int k) { return sm.Bs[m][k]; },
                                     [&](int k, int n) { return sm.dhT[n][k]; }, lane);
             }
             float rs[2] = {0.f, 0.f};  // x.u (u warps) or dout.y~ (y~ warps) per row
@@ -567,14 +569,14 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             sb_zero(a1);
             sb_zero(a2);
             if (warp < 8) {
-                sb_gemm<Q, 4, false>(a1, m0, n0, [&](int m, int k) { return sm.Wm[m][k]; },
+                sb_gemm<Q, 4, false, false>(a1, m0, n0, [&](int m, int k) { return sm.Wm[m][k]; },
                               [&](int k, int n) { return sm.Bs[k][n]; }, lane);
-                sb_gemm<P, 4, false>(a2, m0, n0, [&](int m, int k) { return sm.dos[m][k]; },
+                sb_gemm<P, 4, false, false>(a2, m0, n0, [&](int m, int k) { return sm.dos[m][k]; },
                               [&](int k, int n) { return sm.h0T[k][n]; }, lane);
             } else {
-                sb_gemm<Q, 4, false>(a1, m0, n0, [&](int m, int k) { return sm.VmT[m][k]; },
+                sb_gemm<Q, 4, false, false>(a1, m0, n0, [&](int m, int k) { return sm.VmT[m][k]; },
                               [&](int k, int n) { return sm.Cs[k][n]; }, lane);
-                sb_gemm<P, 4, false>(a2, m0, n0, [&](int m, int k) { return sm.xs[m][k]; },
+                sb_gemm<P, 4, false, false>(a2, m0, n0, [&](int m, int k) { return sm.xs[m][k]; },
                               [&](int k, int n) { return sm.dhT[k][n]; }, lane);
             }
             float *dst = warp < 8 ? pC : pB;
@@ -603,7 +605,7 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     dh[t][e] *= eQ;
-            sb_gemm<Q, 4, true>(dh, dm0, dn0, [&](int m, int k) { return sm.Cs[k][m]; },
+            sb_gemm<Q, 4, false, true>(dh, dm0, dn0, [&](int m, int k) { return sm.Cs[k][m]; },
                           [&](int k, int n) { return sm.ecs[k] * sm.dos[k][n]; }, lane);
         }
         // <dh_0, h_0> of this chunk: the <dh_Q, h_Q> term of the next one
