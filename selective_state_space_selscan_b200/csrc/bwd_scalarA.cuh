@@ -133,14 +133,29 @@ __device__ __forceinline__ void sb_split(float x, uint32_t &hi, uint32_t &lo)
     lo = sb_tf32(x - __uint_as_float(hi));
 }
 
+// How an operand enters a product: kSbRound rounds it to tf32; kSbExact
+// passes its bits as they are (values of bf16 inputs: x, B, C, ungated dy,
+// which tf32 holds exactly); kSbSplit takes it as the sum of two tf32
+// numbers, with one extra product (hi hi, then lo hi and / or hi lo), which
+// keeps about 21 bits of it.
+constexpr int kSbRound = 0, kSbExact = 1, kSbSplit = 2;
+
+template <int MODE>
+__device__ __forceinline__ void sb_operand(float x, uint32_t &hi, uint32_t &lo)
+{
+    if (MODE == kSbSplit)
+        sb_split(x, hi, lo);
+    else if (MODE == kSbExact)
+        hi = __float_as_uint(x);
+    else
+        hi = sb_tf32(x);
+}
+
 // D[NT tiles] += sum_{k < K} A(m0 + row, k) B(k, n0 + 8 t + col): one A
 // fragment per k step serves NT output tiles.  fa(m, k) and fb(k, n) read
-// the operands from shared memory in whatever layout they are kept.  SA / SB:
-// that operand is taken as the sum of two tf32 numbers, with one extra
-// product per split operand (hi hi, then lo hi and / or hi lo), which keeps
-// about 21 bits of it; an operand that holds bf16 values (x, B, C, dy) is
-// exact in tf32 and is not split.
-template <int K, int NT, bool SA, bool SB, typename FA, typename FB>
+// the operands from shared memory in whatever layout they are kept; MA / MB
+// say how each enters the products (kSbRound / kSbExact / kSbSplit).
+template <int K, int NT, int MA, int MB, typename FA, typename FB>
 __device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, FA fa, FB fb,
                                         int lane)
 {
@@ -151,26 +166,18 @@ __device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, FA fa
                              fa(m0 + g + 8, k0 + q + 4)};
         uint32_t ah[4], al[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (SA)
-                sb_split(av[i], ah[i], al[i]);
-            else
-                ah[i] = sb_tf32(av[i]);
-        }
+        for (int i = 0; i < 4; ++i)
+            sb_operand<MA>(av[i], ah[i], al[i]);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             const float bv[2] = {fb(k0 + q, n0 + 8 * t + g), fb(k0 + q + 4, n0 + 8 * t + g)};
             uint32_t bh[2], bl[2];
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                if (SB)
-                    sb_split(bv[i], bh[i], bl[i]);
-                else
-                    bh[i] = sb_tf32(bv[i]);
-            }
-            if (SA)
+            for (int i = 0; i < 2; ++i)
+                sb_operand<MB>(bv[i], bh[i], bl[i]);
+            if (MA == kSbSplit)
                 sb_mma(d[t], al, bh);
-            if (SB)
+            if (MB == kSbSplit)
                 sb_mma(d[t], ah, bl);
             sb_mma(d[t], ah, bh);
         }
@@ -268,7 +275,8 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 hs[t][e] *= dec;
-        sb_gemm<Q, 8, true, false>(hs, 16 * warp, 0, [&](int m, int k) { return ws[k] * Bs[k][m]; },
+        sb_gemm<Q, 8, kSbSplit, kSbExact>(hs, 16 * warp, 0,
+            [&](int m, int k) { return ws[k] * Bs[k][m]; },
                             [&](int k, int n) { return xs[k][n]; }, lane);
         __syncthreads();
     }
@@ -488,10 +496,12 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             float acc[1][4];
             sb_zero(acc);
             if (warp < 8)
-                sb_gemm<N, 1, false, false>(acc, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
+                sb_gemm<N, 1, kSbExact, kSbExact>(acc, m0, n0,
+                    [&](int m, int k) { return sm.Cs[m][k]; },
                               [&](int k, int n) { return sm.Bs[n][k]; }, lane);
             else
-                sb_gemm<P, 1, GATE, false>(acc, m0, n0, [&](int m, int k) { return sm.dos[m][k]; },
+                sb_gemm<P, 1, (GATE ? kSbSplit : kSbExact), kSbExact>(acc, m0, n0,
+                    [&](int m, int k) { return sm.dos[m][k]; },
                               [&](int k, int n) { return sm.xs[n][k]; }, lane);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -518,14 +528,18 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             sb_zero(v1);
             sb_zero(v2);
             if (isy) {
-                sb_gemm<Q, 2, true, false>(v1, m0, n0, [&](int m, int k) { return sm.Md[m][k]; },
+                sb_gemm<Q, 2, kSbSplit, kSbExact>(v1, m0, n0,
+                    [&](int m, int k) { return sm.Md[m][k]; },
                                     [&](int k, int n) { return sm.xsT[n][k]; }, lane);
-                sb_gemm<N, 2, false, true>(v2, m0, n0, [&](int m, int k) { return sm.Cs[m][k]; },
+                sb_gemm<N, 2, kSbExact, kSbSplit>(v2, m0, n0,
+                    [&](int m, int k) { return sm.Cs[m][k]; },
                                     [&](int k, int n) { return sm.h0T[n][k]; }, lane);
             } else {
-                sb_gemm<Q, 2, true, GATE>(v1, m0, n0, [&](int m, int k) { return sm.MmT[m][k]; },
+                sb_gemm<Q, 2, kSbSplit, (GATE ? kSbSplit : kSbExact)>(v1, m0, n0,
+                    [&](int m, int k) { return sm.MmT[m][k]; },
                                     [&](int k, int n) { return sm.dosT[n][k]; }, lane);
-                sb_gemm<N, 2, false, true>(v2, m0, n0, [&](int m, int k) { return sm.Bs[m][k]; },
+                sb_gemm<N, 2, kSbExact, kSbSplit>(v2, m0, n0,
+                    [&](int m, int k) { return sm.Bs[m][k]; },
                                     [&](int k, int n) { return sm.dhT[n][k]; }, lane);
             }
             float rs[2] = {0.f, 0.f};  // x.u (u warps) or dout.y~ (y~ warps) per row
@@ -569,14 +583,18 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             sb_zero(a1);
             sb_zero(a2);
             if (warp < 8) {
-                sb_gemm<Q, 4, false, false>(a1, m0, n0, [&](int m, int k) { return sm.Wm[m][k]; },
+                sb_gemm<Q, 4, kSbRound, kSbExact>(a1, m0, n0,
+                    [&](int m, int k) { return sm.Wm[m][k]; },
                               [&](int k, int n) { return sm.Bs[k][n]; }, lane);
-                sb_gemm<P, 4, false, false>(a2, m0, n0, [&](int m, int k) { return sm.dos[m][k]; },
+                sb_gemm<P, 4, (GATE ? kSbRound : kSbExact), kSbRound>(a2, m0, n0,
+                    [&](int m, int k) { return sm.dos[m][k]; },
                               [&](int k, int n) { return sm.h0T[k][n]; }, lane);
             } else {
-                sb_gemm<Q, 4, false, false>(a1, m0, n0, [&](int m, int k) { return sm.VmT[m][k]; },
+                sb_gemm<Q, 4, kSbRound, kSbExact>(a1, m0, n0,
+                    [&](int m, int k) { return sm.VmT[m][k]; },
                               [&](int k, int n) { return sm.Cs[k][n]; }, lane);
-                sb_gemm<P, 4, false, false>(a2, m0, n0, [&](int m, int k) { return sm.xs[m][k]; },
+                sb_gemm<P, 4, kSbExact, kSbRound>(a2, m0, n0,
+                    [&](int m, int k) { return sm.xs[m][k]; },
                               [&](int k, int n) { return sm.dhT[k][n]; }, lane);
             }
             float *dst = warp < 8 ? pC : pB;
@@ -605,7 +623,8 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     dh[t][e] *= eQ;
-            sb_gemm<Q, 4, false, true>(dh, dm0, dn0, [&](int m, int k) { return sm.Cs[k][m]; },
+            sb_gemm<Q, 4, kSbExact, kSbSplit>(dh, dm0, dn0,
+                [&](int m, int k) { return sm.Cs[k][m]; },
                           [&](int k, int n) { return sm.ecs[k] * sm.dos[k][n]; }, lane);
         }
         // <dh_0, h_0> of this chunk: the <dh_Q, h_Q> term of the next one
