@@ -50,6 +50,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "f32x2.cuh"
 #include "ptx.cuh"
 
 namespace selscan {
@@ -83,6 +84,37 @@ struct SsdBwdParams {
 };
 
 __device__ __forceinline__ float sb_bf(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Tokens t .. t + 7 (t .. t + 3) of a bf16 row as fp32, zero from token
+// `valid` on: one 16-byte (8-byte) load when all of them are in the
+// sequence (rows are 16-byte aligned and t a multiple of 8 (4)).
+__device__ __forceinline__ void sb_ld8(const __nv_bfloat16 *src, int t, int valid,
+                                       float (&v)[8])
+{
+    if (t + 8 <= valid) {
+        unpack8_bf16(*reinterpret_cast<const uint4 *>(src), v);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            v[k] = t + k < valid ? sb_bf(src[k]) : 0.f;
+    }
+}
+
+__device__ __forceinline__ void sb_ld4(const __nv_bfloat16 *src, int t, int valid,
+                                       float (&v)[4])
+{
+    if (t + 4 <= valid) {
+        const uint2 q = *reinterpret_cast<const uint2 *>(src);
+        v[0] = __uint_as_float(q.x << 16);
+        v[1] = __uint_as_float(q.x & 0xffff0000u);
+        v[2] = __uint_as_float(q.y << 16);
+        v[3] = __uint_as_float(q.y & 0xffff0000u);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            v[k] = t + k < valid ? sb_bf(src[k]) : 0.f;
+    }
+}
 
 // Step sizes of a chunk (one warp, lane = token): delta, the raw argument
 // (for the softplus derivative) and the prefix sum S (inclusive).
@@ -244,20 +276,22 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
         {
             const int n = tid >> 1, half = tid & 1;  // row n, tokens 16 half .. + 15
             const __nv_bfloat16 *src = Brow + int64_t(n) * p.B_ns + t0 + 16 * half;
+            float v[8];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int t = 16 * half + k;
-                Bs[t][n] = t < valid ? sb_bf(src[k]) : 0.f;
+            for (int h8 = 0; h8 < 2; ++h8) {
+                sb_ld8(src + 8 * h8, 16 * half + 8 * h8, valid, v);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    Bs[16 * half + 8 * h8 + k][n] = v[k];
             }
         }
         {
             const int pp = tid >> 2, q = tid & 3;  // row p, tokens 8q .. 8q + 7
-            const __nv_bfloat16 *src = xrow + int64_t(pp) * p.x_cs + t0 + 8 * q;
+            float v[8];
+            sb_ld8(xrow + int64_t(pp) * p.x_cs + t0 + 8 * q, 8 * q, valid, v);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int t = 8 * q + k;
-                xs[t][pp] = t < valid ? sb_bf(src[k]) : 0.f;
-            }
+            for (int k = 0; k < 8; ++k)
+                xs[8 * q + k][pp] = v[k];
         }
         if (warp == 0) {
             float raw, dl, S;
@@ -415,16 +449,19 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             const int64_t xo = int64_t(pp) * p.x_cs + t0 + 4 * q;
             const int64_t yo = int64_t(pp) * p.dy_cs + t0 + 4 * q;
             const int64_t zo = GATE ? int64_t(pp) * p.z_cs + t0 + 4 * q : 0;
-            float xv4[4], dv4[4];
+            float xv4[4], dv4[4], xl[4], yl[4], zl[4];
+            sb_ld4(xrow + xo, 4 * q, valid, xl);
+            sb_ld4(dyrow + yo, 4 * q, valid, yl);
+            if (GATE)
+                sb_ld4(zrow + zo, 4 * q, valid, zl);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int t = 4 * q + k;
-                const bool in = t < valid;
-                const float xv = in ? sb_bf(xrow[xo + k]) : 0.f;
-                const float dyv = in ? sb_bf(dyrow[yo + k]) : 0.f;
+                const float xv = xl[k];
+                const float dyv = yl[k];
                 float dout = dyv, zfac = 0.f;
                 if (GATE) {
-                    const float zv = in ? sb_bf(zrow[zo + k]) : 0.f;
+                    const float zv = zl[k];
                     const float sg = 1.f / (1.f + expf(-zv));
                     dout = dyv * zv * sg;
                     zfac = dyv * (sg * (1.f + zv * (1.f - sg)));
@@ -443,14 +480,13 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
         }
         {
             const int n = tid >> 2, q = tid & 3;  // row n, tokens 8q .. 8q + 7
-            const int64_t bo = int64_t(n) * p.B_ns + t0 + 8 * q;
-            const int64_t co = int64_t(n) * p.C_ns + t0 + 8 * q;
+            float bv[8], cv[8];
+            sb_ld8(Brow + int64_t(n) * p.B_ns + t0 + 8 * q, 8 * q, valid, bv);
+            sb_ld8(Crow + int64_t(n) * p.C_ns + t0 + 8 * q, 8 * q, valid, cv);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const int t = 8 * q + k;
-                const bool in = t < valid;
-                sm.Bs[t][n] = in ? sb_bf(Brow[bo + k]) : 0.f;
-                sm.Cs[t][n] = in ? sb_bf(Crow[co + k]) : 0.f;
+                sm.Bs[8 * q + k][n] = bv[k];
+                sm.Cs[8 * q + k][n] = cv[k];
             }
         }
         {

@@ -1576,6 +1576,10 @@ extern "C" selscan_status selscan_bwd_scalarA(
             return SELSCAN_ERR_STRIDE;
         if (t->stride[0] < 0 || t->stride[1] < 0 || t->stride[2] < 0)
             return SELSCAN_ERR_STRIDE;
+        // rows are read with 16-byte loads
+        if (L > 0 && (!aligned16(t->data) || ((t->stride[0] * 2) & 15) ||
+                      ((t->stride[1] * 2) & 15) || ((t->stride[2] * 2) & 15)))
+            return SELSCAN_ERR_ALIGN;
     }
     const int64_t G = B->shape[1], N = B->shape[2];
     if (C->shape[1] != G || C->shape[2] != N || G <= 0 || H % G != 0)
