@@ -331,7 +331,8 @@ SELSCAN_API selscan_status selscan_bwd(
  * head.
  *
  * Forward inputs exactly as selscan_fwd_scalarA_h0 (x, dt, dt_bias,
- * dt_softplus, A, B, C, D, z, headdim, h0; B / C with time stride 1).
+ * dt_softplus, A, B, C, D, z, headdim, h0; B / C with time stride 1 and
+ * 16-byte aligned rows, as there).
  *   dy         (batch, H*P, L)   BF16, like x: gradient of y
  *   dlast      (batch, H, P, N)  F32, contiguous; may be NULL (zero)
  * Outputs (all overwritten):
