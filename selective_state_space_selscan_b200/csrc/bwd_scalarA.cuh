@@ -141,11 +141,12 @@ __device__ __forceinline__ void sb_steps(const SsdBwdParams &p, int b, int hh, i
 // A (16 x 8): a0 (g, q), a1 (g + 8, q), a2 (g, q + 4), a3 (g + 8, q + 4);
 // B (8 x 8):  b0 (q, g), b1 (q + 4, g);
 // D (16 x 8): d0 (g, 2q), d1 (g, 2q + 1), d2 (g + 8, 2q), d3 (g + 8, 2q + 1).
+// x rounded to tf32 (10 mantissa bits), to nearest with ties away from
+// zero: add half a unit of the 13 dropped bits to the magnitude, then clear
+// them (a carry into the exponent gives the next power of two, or infinity).
 __device__ __forceinline__ uint32_t sb_tf32(float x)
 {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return (__float_as_uint(x) + 0x1000u) & 0xffffe000u;
 }
 
 __device__ __forceinline__ void sb_mma(float (&d)[4], const uint32_t (&a)[4],
@@ -267,41 +268,62 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
     const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
     const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
 
+    // the next chunk's B and x values and raw step sizes are read into
+    // registers while the current chunk's products run
+    const int bn = tid >> 1, bhalf = tid & 1;  // B row n, tokens 16 bhalf .. + 15
+    const int xp = tid >> 2, xq = tid & 3;     // x row p, tokens 8 xq .. + 7
+    float bv[16], xv[8], dtv = 0.f;
+    auto fetch = [&](int c) {
+        const int t0 = c * Q, valid = min(Q, p.L - t0);
+        const __nv_bfloat16 *bsrc = Brow + int64_t(bn) * p.B_ns + t0 + 16 * bhalf;
+        float v8[8];
+        sb_ld8(bsrc, 16 * bhalf, valid, v8);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            bv[k] = v8[k];
+        sb_ld8(bsrc + 8, 16 * bhalf + 8, valid, v8);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            bv[8 + k] = v8[k];
+        sb_ld8(xrow + int64_t(xp) * p.x_cs + t0 + 8 * xq, 8 * xq, valid, xv);
+        dtv = (warp == 0 && lane < valid)
+                  ? p.dt[int64_t(b) * p.dt_bs + int64_t(hh) * p.dt_hs + t0 + lane]
+                  : 0.f;
+    };
+    if (p.nchunks > 0)
+        fetch(0);
     for (int c = 0; c < p.nchunks; ++c) {
         float4 *sc = st + int64_t(c) * chunk_stride;
 #pragma unroll
         for (int t = 0; t < 8; ++t)
             sc[t] = make_float4(hs[t][0], hs[t][1], hs[t][2], hs[t][3]);
         const int t0 = c * Q, valid = min(Q, p.L - t0);
-        {
-            const int n = tid >> 1, half = tid & 1;  // row n, tokens 16 half .. + 15
-            const __nv_bfloat16 *src = Brow + int64_t(n) * p.B_ns + t0 + 16 * half;
-            float v[8];
 #pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-                sb_ld8(src + 8 * h8, 16 * half + 8 * h8, valid, v);
+        for (int k = 0; k < 16; ++k)
+            Bs[16 * bhalf + k][bn] = bv[k];
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    Bs[16 * half + 8 * h8 + k][n] = v[k];
-            }
-        }
-        {
-            const int pp = tid >> 2, q = tid & 3;  // row p, tokens 8q .. 8q + 7
-            float v[8];
-            sb_ld8(xrow + int64_t(pp) * p.x_cs + t0 + 8 * q, 8 * q, valid, v);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                xs[8 * q + k][pp] = v[k];
-        }
+        for (int k = 0; k < 8; ++k)
+            xs[8 * xq + k][xp] = xv[k];
         if (warp == 0) {
-            float raw, dl, S;
-            sb_steps(p, b, hh, t0, valid, lane, bias, raw, dl, S);
+            // the same step sizes as sb_steps computes in the walk
+            const float raw = lane < valid ? dtv + bias : 0.f;
+            const float dl =
+                lane < valid ? (p.softplus ? (raw > 20.f ? raw : log1pf(expf(raw))) : raw) : 0.f;
+            float S = dl;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, S, o);
+                if (lane >= o)
+                    S += v;
+            }
             const float SQ = __shfl_sync(0xffffffffu, S, 31);
             ws[lane] = expf(A * (SQ - S)) * dl;
             if (lane == 0)
                 s_decay = expf(A * SQ);
         }
         __syncthreads();
+        if (c + 1 < p.nchunks)
+            fetch(c + 1);
         // h = e^cs_Q h + sum_s (w_s B_s) x_s^T on the tensor cores
         const float dec = s_decay;
 #pragma unroll
