@@ -193,7 +193,7 @@ __device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, FA fa
                                         int lane)
 {
     const int g = lane >> 2, q = lane & 3;
-#pragma unroll 2
+#pragma unroll
     for (int k0 = 0; k0 < K; k0 += 8) {
         const float av[4] = {fa(m0 + g, k0 + q), fa(m0 + g + 8, k0 + q), fa(m0 + g, k0 + q + 4),
                              fa(m0 + g + 8, k0 + q + 4)};
