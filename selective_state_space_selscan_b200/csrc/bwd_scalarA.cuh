@@ -36,13 +36,14 @@
 //     accumulator fragments and evaluates the products above from shared
 //     memory (32-token chunks keep every product's operands on chip).
 // Every product runs on the tensor cores as warp-level m16n8k8 tiles with
-// tf32 operands and fp32 accumulation.  In the products whose results feed
-// the step-size gradients (differences of nearly equal sums) and in the two
-// state recurrences, every operand that is not a bf16 input is split into two
-// tf32 parts (one extra product each), which keeps about 21 bits of it; bf16
-// inputs are exact in tf32.
+// tf32 operands and fp32 accumulation, read from shared-memory tiles laid out
+// so that no fragment load meets a bank conflict (sb_off).  In the products
+// whose results feed the step-size gradients (differences of nearly equal
+// sums) and in the two state recurrences, every operand that is not a bf16
+// input is split into two tf32 parts (one extra product each), which keeps
+// about 21 bits of it; bf16 inputs are exact in tf32.
 // dB and dC sum over the heads of a group: each head adds its chunk terms
-// with 16-byte atomics into one of kSbCopies partial copies ([t][n] rows),
+// with 8-byte atomics into one of kSbCopies partial copies ([t][n] rows),
 // and ssd_bwd_reduce_bc sums the copies into (batch, G, N, L).  dA, dD and
 // the bias gradient sum over batch rows: one atomic per CTA.
 #pragma once
@@ -80,40 +81,78 @@ struct SsdBwdParams {
     float *dA, *dD, *ddt_bias;        // (H), accumulated; dD / ddt_bias may be null
     float *dh0;                       // (batch, H, P, N) or null
     float *pB, *pC;                   // [kSbCopies][batch][G][L][N], zeroed
-    float *states;                    // [batch*H][nchunks+1][256 threads][32] (sb_state_coord)
+    float *states;                    // [batch*H][nchunks+1][P][N]: h^T at every chunk start
 };
 
-__device__ __forceinline__ float sb_bf(__nv_bfloat16 v) { return __bfloat162float(v); }
-
-// Tokens t .. t + 7 (t .. t + 3) of a bf16 row as fp32, zero from token
-// `valid` on: one 16-byte (8-byte) load when all of them are in the
-// sequence (rows are 16-byte aligned and t a multiple of 8 (4)).
-__device__ __forceinline__ void sb_ld8(const __nv_bfloat16 *src, int t, int valid,
-                                       float (&v)[8])
+// Tokens t .. t + 7 (t .. t + 3) of a bf16 row as raw bits, two tokens per
+// word in token order, zero from token `valid` on: one 16-byte (8-byte) load
+// when all of them are in the sequence (rows are 16-byte aligned and t a
+// multiple of 8 (4)).
+__device__ __forceinline__ uint4 sb_raw8(const __nv_bfloat16 *src, int t, int valid)
 {
-    if (t + 8 <= valid) {
-        unpack8_bf16(*reinterpret_cast<const uint4 *>(src), v);
-    } else {
+    if (t + 8 <= valid)
+        return *reinterpret_cast<const uint4 *>(src);
+    const unsigned short *s = reinterpret_cast<const unsigned short *>(src);
+    uint32_t w[4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            v[k] = t + k < valid ? sb_bf(src[k]) : 0.f;
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = t + 2 * k < valid ? s[2 * k] : 0u;
+        const uint32_t hi = t + 2 * k + 1 < valid ? s[2 * k + 1] : 0u;
+        w[k] = lo | (hi << 16);
     }
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ void sb_ld4(const __nv_bfloat16 *src, int t, int valid,
-                                       float (&v)[4])
+__device__ __forceinline__ uint2 sb_raw4(const __nv_bfloat16 *src, int t, int valid)
 {
-    if (t + 4 <= valid) {
-        const uint2 q = *reinterpret_cast<const uint2 *>(src);
-        v[0] = __uint_as_float(q.x << 16);
-        v[1] = __uint_as_float(q.x & 0xffff0000u);
-        v[2] = __uint_as_float(q.y << 16);
-        v[3] = __uint_as_float(q.y & 0xffff0000u);
-    } else {
+    if (t + 4 <= valid)
+        return *reinterpret_cast<const uint2 *>(src);
+    const unsigned short *s = reinterpret_cast<const unsigned short *>(src);
+    uint32_t w[2];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-            v[k] = t + k < valid ? sb_bf(src[k]) : 0.f;
+    for (int k = 0; k < 2; ++k) {
+        const uint32_t lo = t + 2 * k < valid ? s[2 * k] : 0u;
+        const uint32_t hi = t + 2 * k + 1 < valid ? s[2 * k + 1] : 0u;
+        w[k] = lo | (hi << 16);
     }
+    return make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ void sb_unpack4(uint2 v, float (&f)[4])
+{
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xffff0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xffff0000u);
+}
+
+// f[i] = token i ^ r of the eight packed in v (r = 0 .. 3): bit 0 of r swaps
+// the two tokens of every word, bit 1 swaps neighbouring words.
+__device__ __forceinline__ void sb_unpack8_xor(uint4 v, int r, float (&f)[8])
+{
+    const uint32_t sel = (r & 1) ? 0x1032u : 0x3210u;
+    uint32_t w[4] = {__byte_perm(v.x, 0u, sel), __byte_perm(v.y, 0u, sel),
+                     __byte_perm(v.z, 0u, sel), __byte_perm(v.w, 0u, sel)};
+    if (r & 2) {
+        const uint32_t a = w[0], c = w[2];
+        w[0] = w[1];
+        w[1] = a;
+        w[2] = w[3];
+        w[3] = c;
+    }
+    unpack8_bf16(make_uint4(w[0], w[1], w[2], w[3]), f);
+}
+
+// o[i] = v[i ^ r] (r = 0 .. 3)
+__device__ __forceinline__ void sb_xor4(const float (&v)[4], int r, float (&o)[4])
+{
+    const bool b0 = r & 1, b1 = r & 2;
+    const float a0 = b1 ? v[2] : v[0], a1 = b1 ? v[3] : v[1];
+    const float a2 = b1 ? v[0] : v[2], a3 = b1 ? v[1] : v[3];
+    o[0] = b0 ? a1 : a0;
+    o[1] = b0 ? a0 : a1;
+    o[2] = b0 ? a3 : a2;
+    o[3] = b0 ? a2 : a3;
 }
 
 // Step sizes of a chunk (one warp, lane = token): delta, the raw argument
@@ -135,6 +174,21 @@ __device__ __forceinline__ void sb_steps(const SsdBwdParams &p, int b, int hh, i
             S += v;
     }
 }
+
+// ---- shared-memory tiles.  A tile of rows of R floats (R = 32, 64 or 128)
+// has row stride R + 8 and keeps element (r, c) at r (R + 8) + (c ^ (r & 4)):
+// bit 2 of the column flips with bit 2 of the row.  With m16n8k8 fragments
+// two read patterns occur: rows 8 apart by lane / 4 and columns by lane % 4
+// (an operand whose summed index runs along the row), and rows by lane % 4
+// and columns by lane / 4 (summed index down the column).  The stride of 8
+// mod 32 words spreads the first over all 32 banks; the flip keeps the
+// second, whose rows 0-3 and 4-7 would otherwise share banks, conflict-free
+// as well.  Column blocks of 4 stay contiguous and 16-byte aligned.
+constexpr int kSbSX = kSbP + 8;   // rows of P floats
+constexpr int kSbSN = kSbN + 8;   // rows of N floats
+constexpr int kSbST = kSbQ + 8;   // rows of Q floats
+
+__device__ __forceinline__ int sb_off(int S, int r, int c) { return r * S + (c ^ (r & 4)); }
 
 // ---- warp-level tensor-core products (mma.sync m16n8k8, tf32 inputs, fp32
 // accumulators).  Fragment coordinates, with g = lane / 4 and q = lane % 4:
@@ -184,26 +238,69 @@ __device__ __forceinline__ void sb_operand(float x, uint32_t &hi, uint32_t &lo)
         hi = sb_tf32(x);
 }
 
+// Where an operand lives: kSbAlong, the summed index k runs along the tile's
+// rows (A(m, k) at tile (m, k); B(k, n) at tile (n, k)); kSbDown, it runs
+// down the columns (A(m, k) at tile (k, m); B(k, n) at tile (k, n)).
+constexpr int kSbAlong = 0, kSbDown = 1;
+
+// Offset of the element (i, k) of an operand (i = m for A, n for B) for the
+// lanes' i = i0 + lane / 4 and k = lane % 4 + 4 h (h = 0, 1), relative to
+// the k-step k0 and the tile i0 (i0 and k0 multiples of 8).
+template <int O, int S>
+__device__ __forceinline__ int sb_lane_off(int i0, int g, int q, int h)
+{
+    return O == kSbAlong ? (i0 + g) * S + ((q + 4 * h) ^ (g & 4))
+                         : (q + 4 * h) * S + i0 + (g ^ (4 * h));
+}
+
+// Step between k-steps (8 k) and between row blocks 8 apart in i.
+template <int O, int S> struct SbStep {
+    static constexpr int k8 = O == kSbAlong ? 8 : 8 * S;
+    static constexpr int i8 = O == kSbAlong ? 8 * S : 8;
+};
+
 // D[NT tiles] += sum_{k < K} A(m0 + row, k) B(k, n0 + 8 t + col): one A
-// fragment per k step serves NT output tiles.  fa(m, k) and fb(k, n) read
-// the operands from shared memory in whatever layout they are kept; MA / MB
-// say how each enters the products (kSbRound / kSbExact / kSbSplit).
-template <int K, int NT, int MA, int MB, typename FA, typename FB>
-__device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, FA fa, FB fb,
+// fragment per k step serves NT output tiles.  A and B are tiles in the sb_off
+// layout with row strides SA, SB and orientations OA, OB; as / bs, when not
+// null, scale A(., k) and B(k, .) by as[k], bs[k]; MA / MB say how each
+// operand enters the products (kSbRound / kSbExact / kSbSplit).
+template <int K, int NT, int MA, int OA, int SA, int MB, int OB, int SB>
+__device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, const float *a,
+                                        const float *as, const float *b, const float *bs,
                                         int lane)
 {
     const int g = lane >> 2, q = lane & 3;
+    const int ao0 = sb_lane_off<OA, SA>(m0, g, q, 0), ao1 = sb_lane_off<OA, SA>(m0, g, q, 1);
+    const int bo0 = sb_lane_off<OB, SB>(n0, g, q, 0), bo1 = sb_lane_off<OB, SB>(n0, g, q, 1);
+    constexpr int AK = SbStep<OA, SA>::k8, AI = SbStep<OA, SA>::i8;
+    constexpr int BK = SbStep<OB, SB>::k8, BI = SbStep<OB, SB>::i8;
 #pragma unroll
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        const float av[4] = {fa(m0 + g, k0 + q), fa(m0 + g + 8, k0 + q), fa(m0 + g, k0 + q + 4),
-                             fa(m0 + g + 8, k0 + q + 4)};
+    for (int ks = 0; ks < K / 8; ++ks) {
+        float av[4] = {a[ao0 + ks * AK], a[ao0 + ks * AK + AI], a[ao1 + ks * AK],
+                       a[ao1 + ks * AK + AI]};
+        if (as) {
+            const float s0 = as[8 * ks + q], s1 = as[8 * ks + q + 4];
+            av[0] *= s0;
+            av[1] *= s0;
+            av[2] *= s1;
+            av[3] *= s1;
+        }
         uint32_t ah[4], al[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             sb_operand<MA>(av[i], ah[i], al[i]);
+        float s0 = 1.f, s1 = 1.f;
+        if (bs) {
+            s0 = bs[8 * ks + q];
+            s1 = bs[8 * ks + q + 4];
+        }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-            const float bv[2] = {fb(k0 + q, n0 + 8 * t + g), fb(k0 + q + 4, n0 + 8 * t + g)};
+            float bv[2] = {b[bo0 + ks * BK + t * BI], b[bo1 + ks * BK + t * BI]};
+            if (bs) {
+                bv[0] *= s0;
+                bv[1] *= s1;
+            }
             uint32_t bh[2], bl[2];
 #pragma unroll
             for (int i = 0; i < 2; ++i)
@@ -226,66 +323,64 @@ __device__ __forceinline__ void sb_zero(float (&d)[NT][4])
 }
 
 // ------------------------------------------------------------ forward states
-// Scratch layout of the stored states: per (batch, head) and chunk entry, 256
-// threads x 32 floats, thread-contiguous.  Thread u = 32 w + l holds the
-// accumulator fragments of rows 16 w .. 16 w + 15 (n) and all 64 columns (p)
-// in eight 16 x 8 tiles: float 4 t + e is element e of tile t, at row
-// n = 16 w + l / 4 + 8 (e / 2) and column p = 8 t + 2 (l % 4) + e % 2.
-__device__ __forceinline__ void sb_state_coord(int u, int f, int &n, int &pp)
-{
-    const int w = u >> 5, l = u & 31, t = f >> 2, e = f & 3;
-    n = 16 * w + (l >> 2) + 8 * (e >> 1);
-    pp = 8 * t + 2 * (l & 3) + (e & 1);
-}
-
+// The states are kept transposed, h^T (P x N), as accumulator fragments:
+// warp w holds rows p = 16 (w % 4) .. + 15 and columns n = 64 (w / 4) .. + 63
+// (eight 16 x 8 tiles).  Each chunk entry of the scratch is h^T at the chunk
+// start, row-major [p][n], so the walk reads it back with contiguous loads.
+//
+// Loads of a chunk (shared by both kernels): B, C rows n as 8 tokens per
+// thread (thread (n, qq), tokens 8 qq .. + 7) and x, dy, z rows p as 4 tokens
+// per thread (thread (p, q), tokens 4 q .. + 3).  A warp stores them to the
+// token-major tiles one token per thread per instruction; each thread takes
+// its tokens in an order rotated by its lane (token 8 qq + (i ^ qq), resp.
+// 4 q + (i ^ ((q / 2) % 4)), at store i), which puts the 32 stores of an
+// instruction in 32 different banks.
 __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const SsdBwdParams p)
 {
     constexpr int Q = kSbQ, N = kSbN, P = kSbP;
-    __shared__ __align__(16) float Bs[Q][N + 4];
-    __shared__ __align__(16) float xs[Q][P + 4];
+    __shared__ __align__(16) float Bs[Q * kSbSN];
+    __shared__ __align__(16) float xs[Q * kSbSX];
     __shared__ __align__(16) float ws[Q];
     __shared__ float s_decay;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g8 = lane >> 2, q4 = lane & 3;
     const int bh = blockIdx.x, b = bh / p.H, hh = bh - b * p.H;
     const int g = hh / p.heads_per_group;
     const float A = p.A[hh];
     const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
+    const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
 
     float hs[8][4];
     {
         const float *h0 = p.h0 ? p.h0 + (int64_t(b) * p.H + hh) * P * N : nullptr;
 #pragma unroll
-        for (int f = 0; f < 32; ++f) {
-            int n, pp;
-            sb_state_coord(tid, f, n, pp);
-            hs[f >> 2][f & 3] = h0 ? h0[int64_t(pp) * N + n] : 0.f;
-        }
+        for (int t = 0; t < 8; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int pp = m0 + g8 + 8 * (e >> 1), n = n0 + 8 * t + 2 * q4 + (e & 1);
+                hs[t][e] = h0 ? h0[pp * N + n] : 0.f;
+            }
     }
-    float4 *st = reinterpret_cast<float4 *>(p.states) +
-                 (int64_t(bh) * (p.nchunks + 1) * kSbThreads + tid) * 8;
-    const int64_t chunk_stride = int64_t(kSbThreads) * 8;  // float4 per chunk entry
+    float *st = p.states + int64_t(bh) * (p.nchunks + 1) * P * N;
     const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
     const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
 
     // the next chunk's B and x values and raw step sizes are read into
-    // registers while the current chunk's products run
-    const int bn = tid >> 1, bhalf = tid & 1;  // B row n, tokens 16 bhalf .. + 15
-    const int xp = tid >> 2, xq = tid & 3;     // x row p, tokens 8 xq .. + 7
-    float bv[16], xv[8], dtv = 0.f;
+    // registers while the current chunk's products run (two rows per thread)
+    const int bn = tid >> 2, bq = tid & 3;  // B rows bn, bn + 64, tokens 8 bq .. + 7
+    const int xp = tid >> 3, xq = tid & 7;  // x rows xp, xp + 32, tokens 4 xq .. + 3
+    const int xr = (xq >> 1) & 3;
+    uint4 bv[2];
+    uint2 xv[2];
+    float dtv = 0.f;
     auto fetch = [&](int c) {
         const int t0 = c * Q, valid = min(Q, p.L - t0);
-        const __nv_bfloat16 *bsrc = Brow + int64_t(bn) * p.B_ns + t0 + 16 * bhalf;
-        float v8[8];
-        sb_ld8(bsrc, 16 * bhalf, valid, v8);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            bv[k] = v8[k];
-        sb_ld8(bsrc + 8, 16 * bhalf + 8, valid, v8);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-            bv[8 + k] = v8[k];
-        sb_ld8(xrow + int64_t(xp) * p.x_cs + t0 + 8 * xq, 8 * xq, valid, xv);
+        for (int j = 0; j < 2; ++j) {
+            bv[j] = sb_raw8(Brow + int64_t(bn + 64 * j) * p.B_ns + t0 + 8 * bq, 8 * bq, valid);
+            xv[j] = sb_raw4(xrow + int64_t(xp + 32 * j) * p.x_cs + t0 + 4 * xq, 4 * xq, valid);
+        }
         dtv = (warp == 0 && lane < valid)
                   ? p.dt[int64_t(b) * p.dt_bs + int64_t(hh) * p.dt_hs + t0 + lane]
                   : 0.f;
@@ -293,17 +388,28 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
     if (p.nchunks > 0)
         fetch(0);
     for (int c = 0; c < p.nchunks; ++c) {
-        float4 *sc = st + int64_t(c) * chunk_stride;
+        float *sc = st + int64_t(c) * P * N;
 #pragma unroll
         for (int t = 0; t < 8; ++t)
-            sc[t] = make_float4(hs[t][0], hs[t][1], hs[t][2], hs[t][3]);
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+                *reinterpret_cast<float2 *>(sc + (m0 + g8 + 8 * hr) * N + n0 + 8 * t + 2 * q4) =
+                    make_float2(hs[t][2 * hr], hs[t][2 * hr + 1]);
         const int t0 = c * Q, valid = min(Q, p.L - t0);
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-            Bs[16 * bhalf + k][bn] = bv[k];
+        for (int j = 0; j < 2; ++j) {
+            float f[8];
+            sb_unpack8_xor(bv[j], bq, f);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            xs[8 * xq + k][xp] = xv[k];
+            for (int i = 0; i < 8; ++i)
+                Bs[sb_off(kSbSN, 8 * bq + (i ^ bq), bn + 64 * j)] = f[i];
+            float v[4], o[4];
+            sb_unpack4(xv[j], v);
+            sb_xor4(v, xr, o);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                xs[sb_off(kSbSX, 4 * xq + (i ^ xr), xp + 32 * j)] = o[i];
+        }
         if (warp == 0) {
             // the same step sizes as sb_steps computes in the walk
             const float raw = lane < valid ? dtv + bias : 0.f;
@@ -324,43 +430,41 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
         __syncthreads();
         if (c + 1 < p.nchunks)
             fetch(c + 1);
-        // h = e^cs_Q h + sum_s (w_s B_s) x_s^T on the tensor cores
+        // h^T = e^cs_Q h^T + sum_s x_s (w_s B_s)^T on the tensor cores
         const float dec = s_decay;
 #pragma unroll
         for (int t = 0; t < 8; ++t)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 hs[t][e] *= dec;
-        sb_gemm<Q, 8, kSbSplit, kSbExact>(hs, 16 * warp, 0,
-            [&](int m, int k) { return ws[k] * Bs[k][m]; },
-                            [&](int k, int n) { return xs[k][n]; }, lane);
+        sb_gemm<Q, 8, kSbExact, kSbDown, kSbSX, kSbSplit, kSbDown, kSbSN>(
+            hs, m0, n0, xs, nullptr, Bs, ws, lane);
         __syncthreads();
     }
-    float4 *sc = st + int64_t(p.nchunks) * chunk_stride;
+    float *sc = st + int64_t(p.nchunks) * P * N;
 #pragma unroll
     for (int t = 0; t < 8; ++t)
-        sc[t] = make_float4(hs[t][0], hs[t][1], hs[t][2], hs[t][3]);
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr)
+            *reinterpret_cast<float2 *>(sc + (m0 + g8 + 8 * hr) * N + n0 + 8 * t + 2 * q4) =
+                make_float2(hs[t][2 * hr], hs[t][2 * hr + 1]);
 }
 
 // ------------------------------------------------------------ chunk walk
 // 512 threads (16 warps per SM to hide the shared-memory latency of the
-// products).  Shared memory of the walk (fp32); rows are padded (68 / 132 /
-// 36 floats) so that the column groups a warp reads at once fall in distinct
-// banks and every row stays 16-byte aligned.
+// products).  Shared memory of the walk (fp32), every tile in the sb_off
+// layout.
 constexpr int kSbWalk = 512;
-constexpr int kSbXS = kSbP + 4;   // x, dout, dy silu'(z): [t][p]
-constexpr int kSbNS = kSbN + 4;   // B, C: [t][n]; h_0^T, dh^T: [p][n]
-constexpr int kSbTS = kSbQ + 4;   // x^T, dout^T: [p][t]; the Q x Q matrices
 struct SbSmem {
-    float xs[kSbQ][kSbXS], dos[kSbQ][kSbXS], zf[kSbQ][kSbXS];
-    float xsT[kSbP][kSbTS], dosT[kSbP][kSbTS];
-    float Bs[kSbQ][kSbNS], Cs[kSbQ][kSbNS];
-    float h0T[kSbP][kSbNS], dhT[kSbP][kSbNS];
+    float xs[kSbQ * kSbSX], dos[kSbQ * kSbSX], zf[kSbQ * kSbSX];  // x, dout, dy silu'(z): [t][p]
+    float xsT[kSbP * kSbST], dosT[kSbP * kSbST];                  // x, dout: [p][t]
+    float Bs[kSbQ * kSbSN], Cs[kSbQ * kSbSN];                     // [t][n]
+    float h0T[kSbP * kSbSN], dhT[kSbP * kSbSN];                   // h_0^T, dh_Q^T: [p][n]
     // L.G.delta_s [t][s], (L.G)^T [s][t], L.delta_s.(dout x^T) [t][s], (L.(dout x^T))^T [s][t]
-    float Md[kSbQ][kSbTS], MmT[kSbQ][kSbTS], Wm[kSbQ][kSbTS], VmT[kSbQ][kSbTS];
+    float Md[kSbQ * kSbST], MmT[kSbQ * kSbST], Wm[kSbQ * kSbST], VmT[kSbQ * kSbST];
     float raw[kSbQ], dl[kSbQ], S[kSbQ], ecs[kSbQ], ecq[kSbQ], ddd[kSbQ], dyy[kSbQ];
     float red[kSbWalk / 32];
-    float hqdh, ecQ;
+    float ecQ;
 };
 
 // Block sum of one value per thread (every thread gets the total).
@@ -380,25 +484,9 @@ __device__ __forceinline__ float sb_block_sum(float v, float *red, int tid)
     return t;
 }
 
-// Sum over the 16 consecutive lanes that share a row (lanes 16r .. 16r + 15).
-__device__ __forceinline__ float sb_sum16(float v)
+__device__ __forceinline__ float2 sb_ld2(const float *tile, int off)
 {
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    return v;
-}
-
-__device__ __forceinline__ float sb_dot4(float4 a, float4 b, float acc)
-{
-    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
-}
-
-template <typename T>
-__device__ __forceinline__ float4 sb_ld4(const T &ref)
-{
-    return *reinterpret_cast<const float4 *>(&ref);
+    return *reinterpret_cast<const float2 *>(tile + off);
 }
 
 template <bool GATE>
@@ -416,9 +504,10 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
     const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
     const float dsk = p.Dskip ? p.Dskip[hh] : 0.f;
 
-    // dh (N x P) in accumulator fragments: warp w holds rows 16 (w / 2) .. + 15,
-    // columns 32 (w % 2) .. + 31 (four 16 x 8 tiles)
-    const int dm0 = 16 * (warp >> 1), dn0 = 32 * (warp & 1);
+    // dh^T (P x N) in accumulator fragments: warp w holds rows p = 16 (w % 4) .. + 15,
+    // columns n = 32 (w / 4) .. + 31 (four 16 x 8 tiles); element 2 hr + e of
+    // tile t is (p, n) = (dm0 + g8 + 8 hr, dn0 + 8 t + 2 q4 + e)
+    const int dm0 = 16 * (warp & 3), dn0 = 32 * (warp >> 2);
     float dh[4][4];
     {
         const float *dl0 = p.dlast ? p.dlast + (int64_t(b) * p.H + hh) * P * N : nullptr;
@@ -426,31 +515,18 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
         for (int t = 0; t < 4; ++t)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int n = dm0 + g8 + 8 * (e >> 1), pp = dn0 + 8 * t + 2 * q4 + (e & 1);
-                dh[t][e] = dl0 ? dl0[int64_t(pp) * N + n] : 0.f;
+                const int pp = dm0 + g8 + 8 * (e >> 1), n = dn0 + 8 * t + 2 * q4 + (e & 1);
+                dh[t][e] = dl0 ? dl0[pp * N + n] : 0.f;
             }
     }
-    const float4 *st_base = reinterpret_cast<const float4 *>(p.states) +
-                            int64_t(bh) * (p.nchunks + 1) * kSbThreads * 8;
-    const int64_t chunk_stride = int64_t(kSbThreads) * 8;
-    // <dlast, final state> for the last chunk: states-kernel layout, read by
-    // thread halves (u = tid / 2 owns rows 4 (u % 32) + i, columns 8 (u / 32) + j)
+    const float *st_base = p.states + int64_t(bh) * (p.nchunks + 1) * P * N;
+    // <dlast, final state> for the last chunk (both [p][n])
     float hq_next = 0.f;
     if (p.dlast) {
-        const int u = tid >> 1, ih = tid & 1;  // floats 16 ih .. 16 ih + 15 of thread u
-        const float4 *sf = st_base + int64_t(p.nchunks) * chunk_stride + u * 8 + 4 * ih;
+        const float *sf = st_base + int64_t(p.nchunks) * P * N;
         const float *dl0 = p.dlast + (int64_t(b) * p.H + hh) * P * N;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const float4 a = sf[v];
-            const float hv[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                int n, pp;
-                sb_state_coord(u, 16 * ih + 4 * v + e, n, pp);
-                hq_next = fmaf(dl0[int64_t(pp) * N + n], hv[e], hq_next);
-            }
-        }
+        for (int i = tid; i < P * N; i += kSbWalk)
+            hq_next = fmaf(dl0[i], sf[i], hq_next);
     }
     hq_next = sb_block_sum(hq_next, sm.red, tid);
     const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
@@ -462,75 +538,80 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
     float *pB = p.pB + ((int64_t(hh % kSbCopies) * p.batch + b) * p.G + g) * int64_t(p.L) * N;
     float *pC = p.pC + ((int64_t(hh % kSbCopies) * p.batch + b) * p.G + g) * int64_t(p.L) * N;
     float accD = 0.f, accA = 0.f, accBias = 0.f;
+    // chunk loads: x, dy, z row xp, tokens 4 xq .. + 3 (stored in the order
+    // rotated by xr); B, C row bn, tokens 8 bq .. + 7 (rotated by bq)
+    const int xp = tid >> 3, xq = tid & 7, xr = (xq >> 1) & 3;
+    const int bn = tid >> 2, bq = tid & 3;
 
     for (int c = p.nchunks - 1; c >= 0; --c) {
         const int t0 = c * Q, valid = min(Q, p.L - t0);
         // ---- 1. chunk inputs (and transposed copies), h_0^T, dh_Q^T, step sizes
         {
-            const int pp = tid >> 3, q = tid & 7;  // row p, tokens 4q .. 4q + 3
-            const int64_t xo = int64_t(pp) * p.x_cs + t0 + 4 * q;
-            const int64_t yo = int64_t(pp) * p.dy_cs + t0 + 4 * q;
-            const int64_t zo = GATE ? int64_t(pp) * p.z_cs + t0 + 4 * q : 0;
-            float xv4[4], dv4[4], xl[4], yl[4], zl[4];
-            sb_ld4(xrow + xo, 4 * q, valid, xl);
-            sb_ld4(dyrow + yo, 4 * q, valid, yl);
+            float xl[4], yl[4], zl[4], dv[4], zv[4];
+            sb_unpack4(sb_raw4(xrow + int64_t(xp) * p.x_cs + t0 + 4 * xq, 4 * xq, valid), xl);
+            sb_unpack4(sb_raw4(dyrow + int64_t(xp) * p.dy_cs + t0 + 4 * xq, 4 * xq, valid), yl);
             if (GATE)
-                sb_ld4(zrow + zo, 4 * q, valid, zl);
+                sb_unpack4(sb_raw4(zrow + int64_t(xp) * p.z_cs + t0 + 4 * xq, 4 * xq, valid), zl);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int t = 4 * q + k;
-                const float xv = xl[k];
-                const float dyv = yl[k];
-                float dout = dyv, zfac = 0.f;
+                dv[k] = yl[k];
+                zv[k] = 0.f;
                 if (GATE) {
-                    const float zv = zl[k];
-                    const float sg = 1.f / (1.f + expf(-zv));
-                    dout = dyv * zv * sg;
-                    zfac = dyv * (sg * (1.f + zv * (1.f - sg)));
+                    const float sg = 1.f / (1.f + expf(-zl[k]));
+                    dv[k] = yl[k] * zl[k] * sg;
+                    zv[k] = yl[k] * (sg * (1.f + zl[k] * (1.f - sg)));
                 }
-                sm.xs[t][pp] = xv;
-                sm.dos[t][pp] = dout;
-                if (GATE)
-                    sm.zf[t][pp] = zfac;
-                xv4[k] = xv;
-                dv4[k] = dout;
             }
-            *reinterpret_cast<float4 *>(&sm.xsT[pp][4 * q]) =
-                make_float4(xv4[0], xv4[1], xv4[2], xv4[3]);
-            *reinterpret_cast<float4 *>(&sm.dosT[pp][4 * q]) =
-                make_float4(dv4[0], dv4[1], dv4[2], dv4[3]);
-        }
-        {
-            const int n = tid >> 2, q = tid & 3;  // row n, tokens 8q .. 8q + 7
-            float bv[8], cv[8];
-            sb_ld8(Brow + int64_t(n) * p.B_ns + t0 + 8 * q, 8 * q, valid, bv);
-            sb_ld8(Crow + int64_t(n) * p.C_ns + t0 + 8 * q, 8 * q, valid, cv);
+            *reinterpret_cast<float4 *>(&sm.xsT[sb_off(kSbST, xp, 4 * xq)]) =
+                make_float4(xl[0], xl[1], xl[2], xl[3]);
+            *reinterpret_cast<float4 *>(&sm.dosT[sb_off(kSbST, xp, 4 * xq)]) =
+                make_float4(dv[0], dv[1], dv[2], dv[3]);
+            float o[4];
+            sb_xor4(xl, xr, o);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                sm.Bs[8 * q + k][n] = bv[k];
-                sm.Cs[8 * q + k][n] = cv[k];
+            for (int i = 0; i < 4; ++i)
+                sm.xs[sb_off(kSbSX, 4 * xq + (i ^ xr), xp)] = o[i];
+            sb_xor4(dv, xr, o);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                sm.dos[sb_off(kSbSX, 4 * xq + (i ^ xr), xp)] = o[i];
+            if (GATE) {
+                sb_xor4(zv, xr, o);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    sm.zf[sb_off(kSbSX, 4 * xq + (i ^ xr), xp)] = o[i];
             }
         }
         {
-            const int u = tid >> 1, ih = tid & 1;  // floats 16 ih .. 16 ih + 15 of thread u
-            const float4 *s0 = st_base + int64_t(c) * chunk_stride + u * 8 + 4 * ih;
+            float f[8];
+            sb_unpack8_xor(sb_raw8(Brow + int64_t(bn) * p.B_ns + t0 + 8 * bq, 8 * bq, valid), bq,
+                           f);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float4 a = s0[v];
-                const float hv[4] = {a.x, a.y, a.z, a.w};
+            for (int i = 0; i < 8; ++i)
+                sm.Bs[sb_off(kSbSN, 8 * bq + (i ^ bq), bn)] = f[i];
+            sb_unpack8_xor(sb_raw8(Crow + int64_t(bn) * p.C_ns + t0 + 8 * bq, 8 * bq, valid), bq,
+                           f);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    int n, pp;
-                    sb_state_coord(u, 16 * ih + 4 * v + e, n, pp);
-                    sm.h0T[pp][n] = hv[e];
-                }
+            for (int i = 0; i < 8; ++i)
+                sm.Cs[sb_off(kSbSN, 8 * bq + (i ^ bq), bn)] = f[i];
+        }
+        {
+            // h_0^T: 64 rows of 128 floats in 16-byte pieces, consecutive threads
+            // on consecutive pieces
+            const float4 *s0 = reinterpret_cast<const float4 *>(st_base + int64_t(c) * P * N);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int f = tid + kSbWalk * i, pp = f >> 5, n = 4 * (f & 31);
+                *reinterpret_cast<float4 *>(&sm.h0T[sb_off(kSbSN, pp, n)]) = s0[f];
             }
         }
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                sm.dhT[dn0 + 8 * t + 2 * q4 + (e & 1)][dm0 + g8 + 8 * (e >> 1)] = dh[t][e];
+            for (int hr = 0; hr < 2; ++hr)
+                *reinterpret_cast<float2 *>(
+                    &sm.dhT[sb_off(kSbSN, dm0 + g8 + 8 * hr, dn0 + 8 * t + 2 * q4)]) =
+                    make_float2(dh[t][2 * hr], dh[t][2 * hr + 1]);
         if (warp == 0) {
             float rw, dl, S;
             sb_steps(p, b, hh, t0, valid, lane, bias, rw, dl, S);
@@ -554,25 +635,25 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             float acc[1][4];
             sb_zero(acc);
             if (warp < 8)
-                sb_gemm<N, 1, kSbExact, kSbExact>(acc, m0, n0,
-                    [&](int m, int k) { return sm.Cs[m][k]; },
-                              [&](int k, int n) { return sm.Bs[n][k]; }, lane);
+                sb_gemm<N, 1, kSbExact, kSbAlong, kSbSN, kSbExact, kSbAlong, kSbSN>(
+                    acc, m0, n0, sm.Cs, nullptr, sm.Bs, nullptr, lane);
             else
-                sb_gemm<P, 1, (GATE ? kSbSplit : kSbExact), kSbExact>(acc, m0, n0,
-                    [&](int m, int k) { return sm.dos[m][k]; },
-                              [&](int k, int n) { return sm.xs[n][k]; }, lane);
+                sb_gemm<P, 1, (GATE ? kSbSplit : kSbExact), kSbAlong, kSbSX, kSbExact, kSbAlong,
+                        kSbSX>(acc, m0, n0, sm.dos, nullptr, sm.xs, nullptr, lane);
+            float *Mr = warp < 8 ? sm.Md : sm.Wm;    // [t][s], times delta_s
+            float *Mc = warp < 8 ? sm.MmT : sm.VmT;  // [s][t]
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int t = m0 + g8 + 8 * (e >> 1), s_ = n0 + 2 * q4 + (e & 1);
-                const float Lts = s_ <= t ? expf(A * (sm.S[t] - sm.S[s_])) : 0.f;
-                const float v = acc[0][e] * Lts, ds = sm.dl[s_];
-                if (warp < 8) {
-                    sm.Md[t][s_] = v * ds;
-                    sm.MmT[s_][t] = v;
-                } else {
-                    sm.Wm[t][s_] = v * ds;
-                    sm.VmT[s_][t] = v;
+            for (int hr = 0; hr < 2; ++hr) {
+                const int t = m0 + g8 + 8 * hr, s_ = n0 + 2 * q4;
+                float v[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float Lts = s_ + e <= t ? expf(A * (sm.S[t] - sm.S[s_ + e])) : 0.f;
+                    v[e] = acc[0][2 * hr + e] * Lts;
+                    Mc[sb_off(kSbST, s_ + e, t)] = v[e];
                 }
+                *reinterpret_cast<float2 *>(&Mr[sb_off(kSbST, t, s_)]) =
+                    make_float2(v[0] * sm.dl[s_], v[1] * sm.dl[s_ + 1]);
             }
         }
         __syncthreads();
@@ -586,42 +667,46 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             sb_zero(v1);
             sb_zero(v2);
             if (isy) {
-                sb_gemm<Q, 2, kSbSplit, kSbExact>(v1, m0, n0,
-                    [&](int m, int k) { return sm.Md[m][k]; },
-                                    [&](int k, int n) { return sm.xsT[n][k]; }, lane);
-                sb_gemm<N, 2, kSbExact, kSbSplit>(v2, m0, n0,
-                    [&](int m, int k) { return sm.Cs[m][k]; },
-                                    [&](int k, int n) { return sm.h0T[n][k]; }, lane);
+                sb_gemm<Q, 2, kSbSplit, kSbAlong, kSbST, kSbExact, kSbAlong, kSbST>(
+                    v1, m0, n0, sm.Md, nullptr, sm.xsT, nullptr, lane);
+                sb_gemm<N, 2, kSbExact, kSbAlong, kSbSN, kSbSplit, kSbAlong, kSbSN>(
+                    v2, m0, n0, sm.Cs, nullptr, sm.h0T, nullptr, lane);
             } else {
-                sb_gemm<Q, 2, kSbSplit, (GATE ? kSbSplit : kSbExact)>(v1, m0, n0,
-                    [&](int m, int k) { return sm.MmT[m][k]; },
-                                    [&](int k, int n) { return sm.dosT[n][k]; }, lane);
-                sb_gemm<N, 2, kSbExact, kSbSplit>(v2, m0, n0,
-                    [&](int m, int k) { return sm.Bs[m][k]; },
-                                    [&](int k, int n) { return sm.dhT[n][k]; }, lane);
+                sb_gemm<Q, 2, kSbSplit, kSbAlong, kSbST, (GATE ? kSbSplit : kSbExact), kSbAlong,
+                        kSbST>(v1, m0, n0, sm.MmT, nullptr, sm.dosT, nullptr, lane);
+                sb_gemm<N, 2, kSbExact, kSbAlong, kSbSN, kSbSplit, kSbAlong, kSbSN>(
+                    v2, m0, n0, sm.Bs, nullptr, sm.dhT, nullptr, lane);
             }
             float rs[2] = {0.f, 0.f};  // x.u (u warps) or dout.y~ (y~ warps) per row
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int hr = e >> 1, r = m0 + g8 + 8 * hr;
-                    const int pp = n0 + 8 * t + 2 * q4 + (e & 1);
-                    const float xv = sm.xs[r][pp], dv = sm.dos[r][pp];
-                    const int64_t col = int64_t(hh * P + pp);
-                    if (isy) {
-                        const float yt = fmaf(sm.ecs[r], v2[t][e], v1[t][e]);
-                        rs[hr] = fmaf(dv, yt, rs[hr]);
-                        accD = fmaf(dv, xv, accD);
-                        if (GATE && r < valid)
-                            p.dz[int64_t(b) * p.dz_bs + col * p.dz_cs + t0 + r] =
-                                __float2bfloat16_rn(sm.zf[r][pp] * fmaf(dsk, xv, yt));
-                    } else {
-                        const float uu = fmaf(sm.ecq[r], v2[t][e], v1[t][e]);
-                        rs[hr] = fmaf(xv, uu, rs[hr]);
-                        if (r < valid)
-                            p.dx[int64_t(b) * p.dx_bs + col * p.dx_cs + t0 + r] =
-                                __float2bfloat16_rn(fmaf(sm.dl[r], uu, dsk * dv));
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int r = m0 + g8 + 8 * hr, p0 = n0 + 8 * t + 2 * q4;
+                    const int off = sb_off(kSbSX, r, p0);
+                    const float2 x2 = sb_ld2(sm.xs, off), d2 = sb_ld2(sm.dos, off);
+                    float2 z2 = make_float2(0.f, 0.f);
+                    if (GATE && isy)
+                        z2 = sb_ld2(sm.zf, off);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float xv = e ? x2.y : x2.x, dv = e ? d2.y : d2.x;
+                        const float v1e = v1[t][2 * hr + e], v2e = v2[t][2 * hr + e];
+                        const int64_t col = int64_t(hh * P + p0 + e);
+                        if (isy) {
+                            const float yt = fmaf(sm.ecs[r], v2e, v1e);
+                            rs[hr] = fmaf(dv, yt, rs[hr]);
+                            accD = fmaf(dv, xv, accD);
+                            if (GATE && r < valid)
+                                p.dz[int64_t(b) * p.dz_bs + col * p.dz_cs + t0 + r] =
+                                    __float2bfloat16_rn((e ? z2.y : z2.x) * fmaf(dsk, xv, yt));
+                        } else {
+                            const float uu = fmaf(sm.ecq[r], v2e, v1e);
+                            rs[hr] = fmaf(xv, uu, rs[hr]);
+                            if (r < valid)
+                                p.dx[int64_t(b) * p.dx_bs + col * p.dx_cs + t0 + r] =
+                                    __float2bfloat16_rn(fmaf(sm.dl[r], uu, dsk * dv));
+                        }
                     }
                 }
 #pragma unroll
@@ -641,19 +726,15 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             sb_zero(a1);
             sb_zero(a2);
             if (warp < 8) {
-                sb_gemm<Q, 4, kSbRound, kSbExact>(a1, m0, n0,
-                    [&](int m, int k) { return sm.Wm[m][k]; },
-                              [&](int k, int n) { return sm.Bs[k][n]; }, lane);
-                sb_gemm<P, 4, (GATE ? kSbRound : kSbExact), kSbRound>(a2, m0, n0,
-                    [&](int m, int k) { return sm.dos[m][k]; },
-                              [&](int k, int n) { return sm.h0T[k][n]; }, lane);
+                sb_gemm<Q, 4, kSbRound, kSbAlong, kSbST, kSbExact, kSbDown, kSbSN>(
+                    a1, m0, n0, sm.Wm, nullptr, sm.Bs, nullptr, lane);
+                sb_gemm<P, 4, (GATE ? kSbRound : kSbExact), kSbAlong, kSbSX, kSbRound, kSbDown,
+                        kSbSN>(a2, m0, n0, sm.dos, nullptr, sm.h0T, nullptr, lane);
             } else {
-                sb_gemm<Q, 4, kSbRound, kSbExact>(a1, m0, n0,
-                    [&](int m, int k) { return sm.VmT[m][k]; },
-                              [&](int k, int n) { return sm.Cs[k][n]; }, lane);
-                sb_gemm<P, 4, kSbExact, kSbRound>(a2, m0, n0,
-                    [&](int m, int k) { return sm.xs[m][k]; },
-                              [&](int k, int n) { return sm.dhT[k][n]; }, lane);
+                sb_gemm<Q, 4, kSbRound, kSbAlong, kSbST, kSbExact, kSbDown, kSbSN>(
+                    a1, m0, n0, sm.VmT, nullptr, sm.Cs, nullptr, lane);
+                sb_gemm<P, 4, kSbExact, kSbAlong, kSbSX, kSbRound, kSbDown, kSbSN>(
+                    a2, m0, n0, sm.xs, nullptr, sm.dhT, nullptr, lane);
             }
             float *dst = warp < 8 ? pC : pB;
 #pragma unroll
@@ -673,7 +754,7 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
                 }
             }
         }
-        // ---- 3c. dh_0 = e^cs_Q dh_Q + C^T (e^cs dout): rows n, columns p
+        // ---- 3c. dh_0^T = e^cs_Q dh_Q^T + sum_t (e^cs_t dout_t) C_t^T: rows p, columns n
         {
             const float eQ = sm.ecQ;
 #pragma unroll
@@ -681,18 +762,19 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     dh[t][e] *= eQ;
-            sb_gemm<Q, 4, kSbExact, kSbSplit>(dh, dm0, dn0,
-                [&](int m, int k) { return sm.Cs[k][m]; },
-                          [&](int k, int n) { return sm.ecs[k] * sm.dos[k][n]; }, lane);
+            sb_gemm<Q, 4, kSbSplit, kSbDown, kSbSX, kSbExact, kSbDown, kSbSN>(
+                dh, dm0, dn0, sm.dos, sm.ecs, sm.Cs, nullptr, lane);
         }
         // <dh_0, h_0> of this chunk: the <dh_Q, h_Q> term of the next one
         float hq = 0.f;
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                hq = fmaf(dh[t][e],
-                          sm.h0T[dn0 + 8 * t + 2 * q4 + (e & 1)][dm0 + g8 + 8 * (e >> 1)], hq);
+            for (int hr = 0; hr < 2; ++hr) {
+                const float2 h2 =
+                    sb_ld2(sm.h0T, sb_off(kSbSN, dm0 + g8 + 8 * hr, dn0 + 8 * t + 2 * q4));
+                hq = fmaf(dh[t][2 * hr], h2.x, fmaf(dh[t][2 * hr + 1], h2.y, hq));
+            }
         const float hq_this = hq_next;
         hq_next = sb_block_sum(hq, sm.red, tid);  // (its barriers also order 3a-3c before 4)
         // ---- 4. per-token scalars (one warp, lane = token)
@@ -729,8 +811,7 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
         for (int t = 0; t < 4; ++t)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                d0[int64_t(dn0 + 8 * t + 2 * q4 + (e & 1)) * N + dm0 + g8 + 8 * (e >> 1)] =
-                    dh[t][e];
+                d0[(dm0 + g8 + 8 * (e >> 1)) * N + dn0 + 8 * t + 2 * q4 + (e & 1)] = dh[t][e];
     }
     const float sD = sb_block_sum(accD, sm.red, tid);
     const float sA = sb_block_sum(accA, sm.red, tid);
