@@ -259,15 +259,17 @@ template <int O, int S> struct SbStep {
     static constexpr int i8 = O == kSbAlong ? 8 * S : 8;
 };
 
-// D[NT tiles] += sum_{k < K} A(m0 + row, k) B(k, n0 + 8 t + col): one A
-// fragment per k step serves NT output tiles.  A and B are tiles in the sb_off
-// layout with row strides SA, SB and orientations OA, OB; as / bs, when not
-// null, scale A(., k) and B(k, .) by as[k], bs[k]; MA / MB say how each
-// operand enters the products (kSbRound / kSbExact / kSbSplit).
-template <int K, int NT, int MA, int OA, int SA, int MB, int OB, int SB>
-__device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, const float *a,
-                                        const float *as, const float *b, const float *bs,
-                                        int lane)
+// D[MT row blocks][NT tiles] += sum_{k < K} A(m0 + 16 mt + row, k)
+// B(k, n0 + 8 t + col): per k step the B fragments of the NT tiles are read
+// (and split) once and serve all MT row blocks, and each A fragment serves
+// the NT tiles.  A and B are tiles in the sb_off layout with row strides SA,
+// SB and orientations OA, OB; as / bs, when not null, scale A(., k) and
+// B(k, .) by as[k], bs[k]; MA / MB say how each operand enters the products
+// (kSbRound / kSbExact / kSbSplit).
+template <int K, int MT, int NT, int MA, int OA, int SA, int MB, int OB, int SB>
+__device__ __forceinline__ void sb_gemm_mt(float (&d)[MT][NT][4], int m0, int n0, const float *a,
+                                           const float *as, const float *b, const float *bs,
+                                           int lane)
 {
     const int g = lane >> 2, q = lane & 3;
     const int ao0 = sb_lane_off<OA, SA>(m0, g, q, 0), ao1 = sb_lane_off<OA, SA>(m0, g, q, 1);
@@ -276,42 +278,60 @@ __device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, const
     constexpr int BK = SbStep<OB, SB>::k8, BI = SbStep<OB, SB>::i8;
 #pragma unroll
     for (int ks = 0; ks < K / 8; ++ks) {
-        float av[4] = {a[ao0 + ks * AK], a[ao0 + ks * AK + AI], a[ao1 + ks * AK],
-                       a[ao1 + ks * AK + AI]};
-        if (as) {
-            const float s0 = as[8 * ks + q], s1 = as[8 * ks + q + 4];
-            av[0] *= s0;
-            av[1] *= s0;
-            av[2] *= s1;
-            av[3] *= s1;
-        }
-        uint32_t ah[4], al[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            sb_operand<MA>(av[i], ah[i], al[i]);
-        float s0 = 1.f, s1 = 1.f;
-        if (bs) {
-            s0 = bs[8 * ks + q];
-            s1 = bs[8 * ks + q + 4];
-        }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            float bv[2] = {b[bo0 + ks * BK + t * BI], b[bo1 + ks * BK + t * BI]};
+        uint32_t bh[NT][2], bl[NT][2];
+        {
+            float s0 = 1.f, s1 = 1.f;
             if (bs) {
-                bv[0] *= s0;
-                bv[1] *= s1;
+                s0 = bs[8 * ks + q];
+                s1 = bs[8 * ks + q + 4];
             }
-            uint32_t bh[2], bl[2];
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
-                sb_operand<MB>(bv[i], bh[i], bl[i]);
-            if (MA == kSbSplit)
-                sb_mma(d[t], al, bh);
-            if (MB == kSbSplit)
-                sb_mma(d[t], ah, bl);
-            sb_mma(d[t], ah, bh);
+            for (int t = 0; t < NT; ++t) {
+                float bv[2] = {b[bo0 + ks * BK + t * BI], b[bo1 + ks * BK + t * BI]};
+                if (bs) {
+                    bv[0] *= s0;
+                    bv[1] *= s1;
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    sb_operand<MB>(bv[i], bh[t][i], bl[t][i]);
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int ro = 2 * mt * AI + ks * AK;
+            float av[4] = {a[ao0 + ro], a[ao0 + ro + AI], a[ao1 + ro], a[ao1 + ro + AI]};
+            if (as) {
+                const float s0 = as[8 * ks + q], s1 = as[8 * ks + q + 4];
+                av[0] *= s0;
+                av[1] *= s0;
+                av[2] *= s1;
+                av[3] *= s1;
+            }
+            uint32_t ah[4], al[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                sb_operand<MA>(av[i], ah[i], al[i]);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                if (MA == kSbSplit)
+                    sb_mma(d[mt][t], al, bh[t]);
+                if (MB == kSbSplit)
+                    sb_mma(d[mt][t], ah, bl[t]);
+                sb_mma(d[mt][t], ah, bh[t]);
+            }
         }
     }
+}
+
+// One row block (MT = 1).
+template <int K, int NT, int MA, int OA, int SA, int MB, int OB, int SB>
+__device__ __forceinline__ void sb_gemm(float (&d)[NT][4], int m0, int n0, const float *a,
+                                        const float *as, const float *b, const float *bs,
+                                        int lane)
+{
+    sb_gemm_mt<K, 1, NT, MA, OA, SA, MB, OB, SB>(reinterpret_cast<float(&)[1][NT][4]>(d), m0,
+                                                 n0, a, as, b, bs, lane);
 }
 
 template <int NT>
@@ -322,10 +342,18 @@ __device__ __forceinline__ void sb_zero(float (&d)[NT][4])
         d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
 }
 
+template <int MT, int NT>
+__device__ __forceinline__ void sb_zero(float (&d)[MT][NT][4])
+{
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+        sb_zero(d[mt]);
+}
+
 // ------------------------------------------------------------ forward states
 // The states are kept transposed, h^T (P x N), as accumulator fragments:
-// warp w holds rows p = 16 (w % 4) .. + 15 and columns n = 64 (w / 4) .. + 63
-// (eight 16 x 8 tiles).  Each chunk entry of the scratch is h^T at the chunk
+// warp w holds all 64 rows p and columns n = 16 w .. + 15 (four row blocks of
+// two 16 x 8 tiles), so that each split operand (w_s B_s) is split by one warp.  Each chunk entry of the scratch is h^T at the chunk
 // start, row-major [p][n], so the walk reads it back with contiguous loads.
 //
 // Loads of a chunk (shared by both kernels): B, C rows n as 8 tokens per
@@ -349,19 +377,33 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
     const int g = hh / p.heads_per_group;
     const float A = p.A[hh];
     const float bias = p.dt_bias ? p.dt_bias[hh] : 0.f;
-    const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
+    const int n0 = 16 * warp;
 
-    float hs[8][4];
+    float hs[4][2][4];
     {
         const float *h0 = p.h0 ? p.h0 + (int64_t(b) * p.H + hh) * P * N : nullptr;
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
+        for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int pp = m0 + g8 + 8 * (e >> 1), n = n0 + 8 * t + 2 * q4 + (e & 1);
-                hs[t][e] = h0 ? h0[pp * N + n] : 0.f;
-            }
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int pp = 16 * mt + g8 + 8 * (e >> 1), n = n0 + 8 * t + 2 * q4 + (e & 1);
+                    hs[mt][t][e] = h0 ? h0[pp * N + n] : 0.f;
+                }
     }
+    // h^T fragments to a [p][n] entry of the scratch
+    auto store_state = [&](float *sc) {
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr)
+                    *reinterpret_cast<float2 *>(sc + (16 * mt + g8 + 8 * hr) * N + n0 + 8 * t +
+                                                2 * q4) =
+                        make_float2(hs[mt][t][2 * hr], hs[mt][t][2 * hr + 1]);
+    };
     float *st = p.states + int64_t(bh) * (p.nchunks + 1) * P * N;
     const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
     const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
@@ -388,13 +430,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
     if (p.nchunks > 0)
         fetch(0);
     for (int c = 0; c < p.nchunks; ++c) {
-        float *sc = st + int64_t(c) * P * N;
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr)
-                *reinterpret_cast<float2 *>(sc + (m0 + g8 + 8 * hr) * N + n0 + 8 * t + 2 * q4) =
-                    make_float2(hs[t][2 * hr], hs[t][2 * hr + 1]);
+        store_state(st + int64_t(c) * P * N);
         const int t0 = c * Q, valid = min(Q, p.L - t0);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -433,21 +469,17 @@ __global__ void __launch_bounds__(kSbThreads, 1) ssd_bwd_states_kernel(const Ssd
         // h^T = e^cs_Q h^T + sum_s x_s (w_s B_s)^T on the tensor cores
         const float dec = s_decay;
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
+        for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                hs[t][e] *= dec;
-        sb_gemm<Q, 8, kSbExact, kSbDown, kSbSX, kSbSplit, kSbDown, kSbSN>(
-            hs, m0, n0, xs, nullptr, Bs, ws, lane);
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    hs[mt][t][e] *= dec;
+        sb_gemm_mt<Q, 4, 2, kSbExact, kSbDown, kSbSX, kSbSplit, kSbDown, kSbSN>(
+            hs, 0, n0, xs, nullptr, Bs, ws, lane);
         __syncthreads();
     }
-    float *sc = st + int64_t(p.nchunks) * P * N;
-#pragma unroll
-    for (int t = 0; t < 8; ++t)
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr)
-            *reinterpret_cast<float2 *>(sc + (m0 + g8 + 8 * hr) * N + n0 + 8 * t + 2 * q4) =
-                make_float2(hs[t][2 * hr], hs[t][2 * hr + 1]);
+    store_state(st + int64_t(p.nchunks) * P * N);
 }
 
 // ------------------------------------------------------------ chunk walk
@@ -462,7 +494,11 @@ struct SbSmem {
     float h0T[kSbP * kSbSN], dhT[kSbP * kSbSN];                   // h_0^T, dh_Q^T: [p][n]
     // L.G.delta_s [t][s], (L.G)^T [s][t], L.delta_s.(dout x^T) [t][s], (L.(dout x^T))^T [s][t]
     float Md[kSbQ * kSbST], MmT[kSbQ * kSbST], Wm[kSbQ * kSbST], VmT[kSbQ * kSbST];
-    float raw[kSbQ], dl[kSbQ], S[kSbQ], ecs[kSbQ], ecq[kSbQ], ddd[kSbQ], dyy[kSbQ];
+    float ecs[kSbQ], ecq[kSbQ];
+    // per-token values read by the per-token pass, which runs one chunk late:
+    // two copies, chunk c in copy c % 2
+    float raw[2][kSbQ], dl[2][kSbQ], S[2][kSbQ], ddd[2][kSbQ], dyy[2][kSbQ];
+    float hqp[2][kSbWalk / 32];  // per-warp parts of <dh_0, h_0>
     float red[kSbWalk / 32];
     float ecQ;
 };
@@ -521,14 +557,14 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
     }
     const float *st_base = p.states + int64_t(bh) * (p.nchunks + 1) * P * N;
     // <dlast, final state> for the last chunk (both [p][n])
-    float hq_next = 0.f;
+    float hq_next = 0.f;  // <dlast, final state>
     if (p.dlast) {
         const float *sf = st_base + int64_t(p.nchunks) * P * N;
         const float *dl0 = p.dlast + (int64_t(b) * p.H + hh) * P * N;
         for (int i = tid; i < P * N; i += kSbWalk)
             hq_next = fmaf(dl0[i], sf[i], hq_next);
     }
-    hq_next = sb_block_sum(hq_next, sm.red, tid);
+    const float hq_last = sb_block_sum(hq_next, sm.red, tid);
     const __nv_bfloat16 *Brow = p.B + int64_t(b) * p.B_bs + int64_t(g) * p.B_gs;
     const __nv_bfloat16 *Crow = p.C + int64_t(b) * p.C_bs + int64_t(g) * p.C_gs;
     const __nv_bfloat16 *xrow = p.x + int64_t(b) * p.x_bs + int64_t(hh) * P * p.x_cs;
@@ -543,8 +579,46 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
     const int xp = tid >> 3, xq = tid & 7, xr = (xq >> 1) & 3;
     const int bn = tid >> 2, bq = tid & 3;
 
+    // ---- 4. per-token scalars of chunk cc (one warp, lane = token), given
+    //         <dh_Q, h_Q> of that chunk
+    auto per_token = [&](int cc, float hq_this) {
+        const int tt0 = cc * Q, vv = min(Q, p.L - tt0), cb = cc & 1;
+        const bool in = lane < vv;
+        const float ds = sm.dl[cb][lane];
+        float dcs = sm.dyy[cb][lane] - ds * sm.ddd[cb][lane];
+        if (lane == vv - 1)
+            dcs += hq_this;
+        if (!in)
+            dcs = 0.f;
+        float R = dcs;  // sum over t >= lane
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float v = __shfl_down_sync(0xffffffffu, R, off);
+            if (lane + off < 32)
+                R += v;
+        }
+        const float dd = sm.ddd[cb][lane] + A * R;
+        const float rw = sm.raw[cb][lane];
+        const float ddt = p.softplus ? dd / (1.f + expf(-rw)) : dd;
+        if (in)
+            p.ddt[int64_t(b) * p.ddt_bs + int64_t(hh) * p.ddt_hs + tt0 + lane] = ddt;
+        accA = fmaf(dcs, sm.S[cb][lane], accA);
+        accBias += in ? ddt : 0.f;
+    };
+    // <dh_0, h_0> of chunk cc + 1 (summed from its warps' parts), or of the end
+    auto hq_after = [&](int cc) {
+        if (cc + 1 >= p.nchunks)
+            return hq_last;
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSbWalk / 32; ++w)
+            t += sm.hqp[(cc + 1) & 1][w];
+        return t;
+    };
+    constexpr int kTokenWarp = 8;  // a warp with half a tile in phase 2
+
     for (int c = p.nchunks - 1; c >= 0; --c) {
-        const int t0 = c * Q, valid = min(Q, p.L - t0);
+        const int t0 = c * Q, valid = min(Q, p.L - t0), cb = c & 1;
         // ---- 1. chunk inputs (and transposed copies), h_0^T, dh_Q^T, step sizes
         {
             float xl[4], yl[4], zl[4], dv[4], zv[4];
@@ -616,13 +690,13 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
             float rw, dl, S;
             sb_steps(p, b, hh, t0, valid, lane, bias, rw, dl, S);
             const float SQ = __shfl_sync(0xffffffffu, S, 31);
-            sm.raw[lane] = rw;
-            sm.dl[lane] = dl;
-            sm.S[lane] = S;
+            sm.raw[cb][lane] = rw;
+            sm.dl[cb][lane] = dl;
+            sm.S[cb][lane] = S;
             sm.ecs[lane] = expf(A * S);
             sm.ecq[lane] = expf(A * (SQ - S));
-            sm.ddd[lane] = 0.f;
-            sm.dyy[lane] = 0.f;
+            sm.ddd[cb][lane] = 0.f;
+            sm.dyy[cb][lane] = 0.f;
             if (lane == 0)
                 sm.ecQ = expf(A * SQ);
         }
@@ -648,13 +722,25 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
                 float v[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float Lts = s_ + e <= t ? expf(A * (sm.S[t] - sm.S[s_ + e])) : 0.f;
+                    const float Lts = s_ + e <= t ? expf(A * (sm.S[cb][t] - sm.S[cb][s_ + e])) : 0.f;
                     v[e] = acc[0][2 * hr + e] * Lts;
-                    Mc[sb_off(kSbST, s_ + e, t)] = v[e];
                 }
-                *reinterpret_cast<float2 *>(&Mr[sb_off(kSbST, t, s_)]) =
-                    make_float2(v[0] * sm.dl[s_], v[1] * sm.dl[s_ + 1]);
+                float w0 = v[0] * sm.dl[cb][s_], w1 = v[1] * sm.dl[cb][s_ + 1];
+                if (warp >= 8) {
+                    // Wm and VmT enter their products rounded to tf32: round once here
+                    v[0] = __uint_as_float(sb_tf32(v[0]));
+                    v[1] = __uint_as_float(sb_tf32(v[1]));
+                    w0 = __uint_as_float(sb_tf32(w0));
+                    w1 = __uint_as_float(sb_tf32(w1));
+                }
+                Mc[sb_off(kSbST, s_, t)] = v[0];
+                Mc[sb_off(kSbST, s_ + 1, t)] = v[1];
+                *reinterpret_cast<float2 *>(&Mr[sb_off(kSbST, t, s_)]) = make_float2(w0, w1);
             }
+            // the per-token pass of the chunk after this one: its products all
+            // finished before the barrier above
+            if (warp == kTokenWarp && c + 1 < p.nchunks)
+                per_token(c + 1, hq_after(c + 1));
         }
         __syncthreads();
 
@@ -705,7 +791,7 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
                             rs[hr] = fmaf(xv, uu, rs[hr]);
                             if (r < valid)
                                 p.dx[int64_t(b) * p.dx_bs + col * p.dx_cs + t0 + r] =
-                                    __float2bfloat16_rn(fmaf(sm.dl[r], uu, dsk * dv));
+                                    __float2bfloat16_rn(fmaf(sm.dl[cb][r], uu, dsk * dv));
                         }
                     }
                 }
@@ -714,45 +800,48 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
                 rs[hr] += __shfl_xor_sync(0xffffffffu, rs[hr], 1);
                 rs[hr] += __shfl_xor_sync(0xffffffffu, rs[hr], 2);
                 if (q4 == 0)
-                    atomicAdd(isy ? &sm.dyy[m0 + g8 + 8 * hr] : &sm.ddd[m0 + g8 + 8 * hr],
+                    atomicAdd(isy ? &sm.dyy[cb][m0 + g8 + 8 * hr] : &sm.ddd[cb][m0 + g8 + 8 * hr],
                               rs[hr]);
             }
         }
         // ---- 3b. dC (warps 0-7) and dB (warps 8-15): 32 x 128 each; warp
-        //          holds rows 16 ((w / 4) % 2), columns 32 (w % 4) .. + 31
+        //          holds all 32 rows, columns 16 (w % 8) .. + 15
         {
-            const int m0 = 16 * ((warp >> 2) & 1), n0 = 32 * (warp & 3);
-            float a1[4][4], a2[4][4];
+            const int n0 = 16 * (warp & 7);
+            float a1[2][2][4], a2[2][2][4];
             sb_zero(a1);
             sb_zero(a2);
             if (warp < 8) {
-                sb_gemm<Q, 4, kSbRound, kSbAlong, kSbST, kSbExact, kSbDown, kSbSN>(
-                    a1, m0, n0, sm.Wm, nullptr, sm.Bs, nullptr, lane);
-                sb_gemm<P, 4, (GATE ? kSbRound : kSbExact), kSbAlong, kSbSX, kSbRound, kSbDown,
-                        kSbSN>(a2, m0, n0, sm.dos, nullptr, sm.h0T, nullptr, lane);
+                sb_gemm_mt<Q, 2, 2, kSbExact, kSbAlong, kSbST, kSbExact, kSbDown, kSbSN>(
+                    a1, 0, n0, sm.Wm, nullptr, sm.Bs, nullptr, lane);
+                sb_gemm_mt<P, 2, 2, (GATE ? kSbRound : kSbExact), kSbAlong, kSbSX, kSbRound,
+                           kSbDown, kSbSN>(a2, 0, n0, sm.dos, nullptr, sm.h0T, nullptr, lane);
             } else {
-                sb_gemm<Q, 4, kSbRound, kSbAlong, kSbST, kSbExact, kSbDown, kSbSN>(
-                    a1, m0, n0, sm.VmT, nullptr, sm.Cs, nullptr, lane);
-                sb_gemm<P, 4, kSbExact, kSbAlong, kSbSX, kSbRound, kSbDown, kSbSN>(
-                    a2, m0, n0, sm.xs, nullptr, sm.dhT, nullptr, lane);
+                sb_gemm_mt<Q, 2, 2, kSbExact, kSbAlong, kSbST, kSbExact, kSbDown, kSbSN>(
+                    a1, 0, n0, sm.VmT, nullptr, sm.Cs, nullptr, lane);
+                sb_gemm_mt<P, 2, 2, kSbExact, kSbAlong, kSbSX, kSbRound, kSbDown, kSbSN>(
+                    a2, 0, n0, sm.xs, nullptr, sm.dhT, nullptr, lane);
             }
             float *dst = warp < 8 ? pC : pB;
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int r = m0 + g8 + 8 * hr;
-                if (r < valid) {
-                    const float sc = warp < 8 ? sm.ecs[r] : sm.ecq[r];
-                    const float pre = warp < 8 ? 1.f : sm.dl[r];
+            for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const int n = n0 + 8 * t + 2 * q4;
-                        const float2 v = make_float2(
-                            pre * fmaf(sc, a2[t][2 * hr], a1[t][2 * hr]),
-                            pre * fmaf(sc, a2[t][2 * hr + 1], a1[t][2 * hr + 1]));
-                        atomicAdd(reinterpret_cast<float2 *>(dst + int64_t(t0 + r) * N + n), v);
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int r = 16 * mt + g8 + 8 * hr;
+                    if (r < valid) {
+                        const float sc = warp < 8 ? sm.ecs[r] : sm.ecq[r];
+                        const float pre = warp < 8 ? 1.f : sm.dl[cb][r];
+#pragma unroll
+                        for (int t = 0; t < 2; ++t) {
+                            const int n = n0 + 8 * t + 2 * q4;
+                            const float2 v = make_float2(
+                                pre * fmaf(sc, a2[mt][t][2 * hr], a1[mt][t][2 * hr]),
+                                pre * fmaf(sc, a2[mt][t][2 * hr + 1], a1[mt][t][2 * hr + 1]));
+                            atomicAdd(reinterpret_cast<float2 *>(dst + int64_t(t0 + r) * N + n),
+                                      v);
+                        }
                     }
                 }
-            }
         }
         // ---- 3c. dh_0^T = e^cs_Q dh_Q^T + sum_t (e^cs_t dout_t) C_t^T: rows p, columns n
         {
@@ -775,34 +864,15 @@ __global__ void __launch_bounds__(kSbWalk, 1) ssd_bwd_kernel(const SsdBwdParams 
                     sb_ld2(sm.h0T, sb_off(kSbSN, dm0 + g8 + 8 * hr, dn0 + 8 * t + 2 * q4));
                 hq = fmaf(dh[t][2 * hr], h2.x, fmaf(dh[t][2 * hr + 1], h2.y, hq));
             }
-        const float hq_this = hq_next;
-        hq_next = sb_block_sum(hq, sm.red, tid);  // (its barriers also order 3a-3c before 4)
-        // ---- 4. per-token scalars (one warp, lane = token)
-        if (warp == 0) {
-            const bool in = lane < valid;
-            const float ds = sm.dl[lane];
-            float dcs = sm.dyy[lane] - ds * sm.ddd[lane];
-            if (lane == valid - 1)
-                dcs += hq_this;
-            if (!in)
-                dcs = 0.f;
-            float R = dcs;  // sum over t >= lane
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float v = __shfl_down_sync(0xffffffffu, R, off);
-                if (lane + off < 32)
-                    R += v;
-            }
-            const float dd = sm.ddd[lane] + A * R;
-            const float rw = sm.raw[lane];
-            const float ddt = p.softplus ? dd / (1.f + expf(-rw)) : dd;
-            if (in)
-                p.ddt[int64_t(b) * p.ddt_bs + int64_t(hh) * p.ddt_hs + t0 + lane] = ddt;
-            accA = fmaf(dcs, sm.S[lane], accA);
-            accBias += in ? ddt : 0.f;
-        }
-        __syncthreads();
+        for (int o = 16; o > 0; o >>= 1)
+            hq += __shfl_xor_sync(0xffffffffu, hq, o);
+        if (lane == 0)
+            sm.hqp[cb][warp] = hq;
+        __syncthreads();  // the tiles are free for the next chunk
     }
+    if (warp == kTokenWarp && p.nchunks > 0)
+        per_token(0, hq_after(0));
 
     // ---- per-head sums (over this batch row), dh0
     if (p.dh0) {
