@@ -101,6 +101,24 @@ def ssd_flops(cfg: dict, Q: int = 128) -> float:
     return float(b * nch * per_chunk)
 
 
+def ssd_bwd_flops(cfg: dict, Q: int = 32) -> float:
+    """Tensor-core FLOPs of the chunked scalar-A backward per call at chunk
+    length Q (the kernels' Q = 32), counting each product once (the extra
+    products of split operands are not counted): C.B^T once per batch, group
+    and chunk; per head and chunk dout.x^T, the two products of y~ and of u,
+    the two of dC and of dB, the dh recurrence and the forward state
+    recurrence."""
+    b, L = cfg["batch"], cfg["L"]
+    H, P, N, G = cfg["nheads"], cfg["headdim"], cfg["N"], cfg["ngroups"]
+    nch = (L + Q - 1) // Q
+    per_head = 6 * Q * Q * P + 4 * Q * Q * N + 12 * Q * P * N
+    return float(b * nch * (G * 2 * Q * Q * N + H * per_head))
+
+
+# nominal dense tensor throughput of tf32 relative to bf16 on B200 (1.1 / 2.25 PFLOP/s)
+TF32_PER_BF16 = 1.1 / 2.25
+
+
 # ------------------------------------------------------------ ranks
 @contextlib.contextmanager
 def gc_paused(collect: bool = True):
@@ -886,17 +904,19 @@ def bwd_bytes(cfg: dict) -> int:
     return total
 
 
-# DRAM bytes per backward call (ncu, profiles/selscan_bwd_config2.md): captured
-# at L = 1024 on the B4 D5120 layer, scaled by tokens to L = 4096
-BWD_NCU_TRAFFIC = {2: ("selscan_bwd_kernel v5", 4 * 687.2e6)}
-BWD_KERNEL_TAG = "selscan_bwd_kernel v5"
+# DRAM bytes per launch of the backward's dominant kernel (ncu): captured at
+# L = 1024 and scaled by tokens to L = 4096 (profiles/selscan_bwd_config2.md,
+# profiles/ssd_bwd_scalarA_config4.md)
+BWD_NCU_TRAFFIC = {2: ("selscan_bwd_kernel v5", 4 * 687.2e6),
+                   4: ("ssd_bwd_kernel v7", 4 * 235.8e6)}
+BWD_KERNEL_TAG = {2: "selscan_bwd_kernel v5", 4: "ssd_bwd_kernel v7"}
 
 
 def bwd_traffic(args, cfg):
     if args.traffic is not None:
         return args.traffic
     ent = BWD_NCU_TRAFFIC.get(args.config)
-    if ent and ent[0] == BWD_KERNEL_TAG and cfg == BASE_CONFIGS[args.config]:
+    if ent and ent[0] == BWD_KERNEL_TAG.get(args.config) and cfg == BASE_CONFIGS[args.config]:
         return ent[1]
     return None
 
@@ -1032,6 +1052,14 @@ def run_bwd(args, rank: int, world: int, local: int):
         "gpu_launches": n_launch,
         "clocks": clock_info,
     }
+    if scalar:
+        fl = ssd_bwd_flops(cfg)
+        peak = peaks.get("bf16_tflops", 1590.0) * TF32_PER_BF16
+        line["roofline"]["tensor"] = {
+            "flops_per_launch": fl, "dtype": "tf32",
+            "achieved_tflops": fl / (avg_launch_ms * 1e-3) / 1e12, "peak_tflops": peak,
+            "peak_source": f"{peaks_src} bf16 GEMM x nominal tf32/bf16 ratio {TF32_PER_BF16:.3f}",
+            "frac": fl / (avg_launch_ms * 1e-3) / 1e12 / peak}
     if not args.no_cpu_baseline and world == 1:  # the oracle baseline: rank 0 at N = 1
         line["cpu_baseline"] = oracle_bwd_sample(cfg, inp, dy_host, seconds=args.cpu_seconds)
     print(json.dumps(line), flush=True)
