@@ -40,8 +40,8 @@
 // so that no fragment load meets a bank conflict (sb_off).  In the products
 // whose results feed the step-size gradients (differences of nearly equal
 // sums) and in the two state recurrences, every operand that is not a bf16
-// input is split into two tf32 parts (one extra product each), which keeps
-// about 21 bits of it; bf16 inputs are exact in tf32.
+// input is split into two parts (one extra product each), which keeps about
+// 20 bits of it; bf16 inputs are exact in tf32.
 // dB and dC sum over the heads of a group: each head adds its chunk terms
 // with 8-byte atomics into one of kSbCopies partial copies ([t][n] rows),
 // and ssd_bwd_reduce_bc sums the copies into (batch, G, N, L).  dA, dD and
@@ -213,18 +213,21 @@ __device__ __forceinline__ void sb_mma(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// x = hi + lo with hi, lo both tf32 (hi the rounded value, lo the rounded rest).
+// x = hi + lo: hi is x with its 13 low mantissa bits cleared (a tf32
+// value), lo = x - hi exactly (an fp32 value below 2^-10 of |x|).  A tf32
+// product reads only the top 19 bits of each operand, so lo enters it
+// truncated to tf32, which leaves an error below 2^-20 |x|.
 __device__ __forceinline__ void sb_split(float x, uint32_t &hi, uint32_t &lo)
 {
-    hi = sb_tf32(x);
-    lo = sb_tf32(x - __uint_as_float(hi));
+    hi = __float_as_uint(x) & 0xffffe000u;
+    lo = __float_as_uint(x - __uint_as_float(hi));
 }
 
 // How an operand enters a product: kSbRound rounds it to tf32; kSbExact
 // passes its bits as they are (values of bf16 inputs: x, B, C, ungated dy,
-// which tf32 holds exactly); kSbSplit takes it as the sum of two tf32
-// numbers, with one extra product (hi hi, then lo hi and / or hi lo), which
-// keeps about 21 bits of it.
+// which tf32 holds exactly); kSbSplit takes it as the sum of two parts
+// (sb_split), with one extra product (hi hi, then lo hi and / or hi lo),
+// which keeps about 20 bits of it.
 constexpr int kSbRound = 0, kSbExact = 1, kSbSplit = 2;
 
 template <int MODE>
