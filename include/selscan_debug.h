@@ -45,6 +45,15 @@ SELSCAN_API void selscan_debug_diag_mode(int mode);
 SELSCAN_API void selscan_debug_bwd_segments(int segs);
 
 /*
+ * Number of time segments per channel tile in subsequent selscan_fwd calls
+ * (0, the default, = the library's choice).  Capped at the number of 64-token
+ * chunks and rounded to whole chunks per segment.  Every segment count gives
+ * the same result up to the order of the chained fold; the hook lets the
+ * choice be timed and lets tests cover many-segment chains on small inputs.
+ */
+SELSCAN_API void selscan_debug_fwd_segments(int segs);
+
+/*
  * The number of time segments per channel tile that selscan_bwd would pick
  * for `tiles` tiles of (batch row, 32 channels), `nchunks` 8-token
  * checkpoint chunks and `slots` warps resident at once (blocks per SM x
@@ -52,6 +61,16 @@ SELSCAN_API void selscan_debug_bwd_segments(int segs);
  * no CUDA call.  Lets the choice be tested without a GPU.
  */
 SELSCAN_API long long selscan_debug_bwd_plan(long long tiles, long long nchunks, long long slots);
+
+/*
+ * The time segments per channel tile that selscan_fwd would pick in its
+ * automatic mode (bf16) for `tiles` tiles of 128 channels, `chunks` 64-token
+ * chunks and `ctas` persistent CTAs, before rounding to whole chunks per
+ * segment: positive for the one-pass form with chained carries, negative
+ * (minus the count) for the two-pass form.  Host arithmetic only: no CUDA
+ * call.  Lets the choice be tested without a GPU.
+ */
+SELSCAN_API long long selscan_debug_fwd_plan(long long tiles, long long chunks, long long ctas);
 
 #ifdef __cplusplus
 }

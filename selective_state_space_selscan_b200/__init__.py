@@ -101,6 +101,10 @@ def lib() -> ctypes.CDLL:
         L.selscan_debug_diag_mode.restype = None
         L.selscan_debug_bwd_segments.argtypes = [ctypes.c_int]
         L.selscan_debug_bwd_segments.restype = None
+        L.selscan_debug_fwd_segments.argtypes = [ctypes.c_int]
+        L.selscan_debug_fwd_segments.restype = None
+        L.selscan_debug_fwd_plan.argtypes = [ctypes.c_longlong] * 3
+        L.selscan_debug_fwd_plan.restype = ctypes.c_longlong
         L.selscan_debug_bwd_plan.argtypes = [ctypes.c_longlong] * 3
         L.selscan_debug_bwd_plan.restype = ctypes.c_longlong
         _lib = L
@@ -376,6 +380,18 @@ def debug_diag_mode(mode: int) -> None:
 def debug_bwd_segments(segs: int) -> None:
     """Test hook: time segments per channel tile in selscan_bwd (0: automatic)."""
     lib().selscan_debug_bwd_segments(int(segs))
+
+
+def debug_fwd_segments(segs: int) -> None:
+    """Test hook: time segments per channel tile in selscan_fwd (0: automatic)."""
+    lib().selscan_debug_fwd_segments(int(segs))
+
+
+def debug_fwd_plan(tiles: int, chunks: int, ctas: int) -> int:
+    """Test hook: selscan_fwd's automatic segment count for ``tiles`` tiles,
+    ``chunks`` 64-token chunks and ``ctas`` CTAs (negative: the two-pass
+    form).  Host arithmetic only."""
+    return int(lib().selscan_debug_fwd_plan(int(tiles), int(chunks), int(ctas)))
 
 
 def debug_bwd_plan(tiles: int, nchunks: int, slots: int) -> int:

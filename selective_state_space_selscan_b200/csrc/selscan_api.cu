@@ -166,6 +166,45 @@ int64_t bwd_segments(int64_t tiles, int64_t nchunks, int64_t slots)
     return S ? S : S_any;
 }
 
+// Time segments per channel tile of the forward pass: `tiles` tiles of CH
+// channels, `chunks` 64-token chunks, `ctas` persistent CTAs (one per SM);
+// `forced_mode` is the test hook's form (-1: automatic).  Returns the segment
+// count before rounding to whole chunks per segment; *two_pass tells the
+// form.  The spread rule gives about 8 units per CTA with at least 4 chunks
+// per segment.
+//  - Few tiles (2 tiles <= ctas) and a spread of more than one segment: the
+//    two-pass form, whose segments do not wait for one another.
+//  - The chained form with tiles <= ctas: one segment per tile.  A tile's
+//    segments run one after another (each waits for its predecessor's
+//    carry), so the call cannot be shorter than one tile's whole sequence,
+//    and every extra segment adds its start and carry hand-off to that
+//    chain: B8 D1536 L2048 1 segment 0.168 ms (2: 0.173, 8: 0.191), B4 D4096
+//    L4096 0.327 ms (8: 0.350, 10: 0.371), B2 D5120 L4096 0.323 ms (15:
+//    0.354).
+//  - The chained form with more tiles than CTAs: the spread rule, which
+//    balances the units over the CTAs (B4 D5120 L4096: 8 segments 0.388 ms,
+//    4: 0.411, 16: 0.413; B16 D2560 L1024: 4 segments 0.215 ms, 1: 0.249).
+//  A forced form keeps the spread rule, so that tests of either form cover
+//  multi-segment chains and folds.
+int64_t fwd_segments(int64_t tiles, int64_t chunks, int64_t ctas, int forced_mode,
+                     bool can_two_pass, bool *two_pass)
+{
+    *two_pass = false;
+    if (tiles < 1 || chunks < 1 || ctas < 1)
+        return 1;
+    const int64_t spread = std::max<int64_t>(
+        1, std::min<int64_t>((8 * ctas + tiles - 1) / tiles, (chunks + 3) / 4));
+    if (forced_mode >= 0) {
+        *two_pass = can_two_pass && forced_mode == 1 && spread > 1;
+        return spread;
+    }
+    if (can_two_pass && spread > 1 && 2 * tiles <= ctas) {
+        *two_pass = true;
+        return spread;
+    }
+    return tiles <= ctas ? 1 : spread;
+}
+
 size_t elem_size(int32_t dt) { return dt == SELSCAN_BF16 ? 2 : 4; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -320,6 +359,7 @@ bool ensure_smem(K kern, int bytes, int dev, bool (&done)[kMaxDevices])
 
 int g_dbg_diag_mode = -1;  // test hook, see selscan_debug_diag_mode
 int g_dbg_bwd_segs = 0;     // test hook, see selscan_debug_bwd_segments
+int g_dbg_fwd_segs = 0;     // test hook, see selscan_debug_fwd_segments
 
 template <int KIND, typename T, int CH, int STAGES, bool GATE, bool SOFTPLUS>
 selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
@@ -365,10 +405,10 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
     const int G = int(batch) * tpb;
     const int ctas_max = sm_count;  // one persistent CTA per SM
     const int64_t chunks = (L + TC - 1) / TC;
-    // aim for about 8 units per CTA so the tail is short, segments >= 4 chunks
-    int64_t want_units = 8ll * ctas_max;
-    int64_t S = (want_units + G - 1) / G;
-    S = std::max<int64_t>(1, std::min<int64_t>(S, (chunks + 3) / 4));
+    bool two_pass_plan = false;
+    int64_t S = fwd_segments(G, chunks, ctas_max, g_dbg_diag_mode, KIND == 1, &two_pass_plan);
+    if (g_dbg_fwd_segs > 0)
+        S = std::min<int64_t>(g_dbg_fwd_segs, std::max<int64_t>(1, chunks));
     int64_t seg_chunks = (chunks + S - 1) / S;
     S = (chunks + seg_chunks - 1) / seg_chunks;
     prm.tiles_per_batch = tpb;
@@ -383,8 +423,7 @@ selscan_status launch_diag(const selscan_tensor *u, const selscan_tensor *delta,
     // Few tiles and several segments: a chain of carries would leave most
     // SMs waiting, so use the two-pass form (aggregates, then output).
     if constexpr (KIND == 1) {
-    const bool two_pass = g_dbg_diag_mode >= 0 ? (g_dbg_diag_mode == 1 && S > 1)
-                                               : (S > 1 && 2 * int64_t(G) <= sm_count);
+    const bool two_pass = two_pass_plan && S > 1;
     if (two_pass) {
         int dev = 0;
         cudaGetDevice(&dev);
@@ -518,10 +557,18 @@ selscan_status selscan_release_scratch(void)
 void selscan_debug_diag_mode(int mode) { g_dbg_diag_mode = mode; }
 
 void selscan_debug_bwd_segments(int segs) { g_dbg_bwd_segs = segs < 0 ? 0 : segs; }
+void selscan_debug_fwd_segments(int segs) { g_dbg_fwd_segs = segs < 0 ? 0 : segs; }
 
 long long selscan_debug_bwd_plan(long long tiles, long long nchunks, long long slots)
 {
     return bwd_segments(tiles, nchunks, slots);
+}
+
+long long selscan_debug_fwd_plan(long long tiles, long long chunks, long long ctas)
+{
+    bool two_pass = false;
+    const int64_t S = fwd_segments(tiles, chunks, ctas, -1, true, &two_pass);
+    return two_pass ? -S : S;
 }
 
 void selscan_debug_withhold_carry(int unit) { g_dbg_skip_publish = unit; }
@@ -893,8 +940,10 @@ selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor
     const int G = int(batch) * tpb;
     const int ctas_max = sm_count;
     const int64_t chunks = (L + TC - 1) / TC;
-    int64_t S = (8ll * ctas_max + G - 1) / G;
-    S = std::max<int64_t>(1, std::min<int64_t>(S, (chunks + 3) / 4));
+    bool two_pass_plan = false;
+    int64_t S = fwd_segments(G, chunks, ctas_max, g_dbg_diag_mode, KIND == 1, &two_pass_plan);
+    if (g_dbg_fwd_segs > 0)
+        S = std::min<int64_t>(g_dbg_fwd_segs, std::max<int64_t>(1, chunks));
     const int64_t seg_chunks = (chunks + S - 1) / S;
     S = (chunks + seg_chunks - 1) / seg_chunks;
     const int64_t units = int64_t(G) * S;
@@ -912,8 +961,7 @@ selscan_status launch_diag_noalloc(const selscan_tensor *u, const selscan_tensor
     // chooses it, with its aggregates in the static array (there is no
     // initial state to copy).
     if constexpr (KIND == 1) {
-    const bool two_pass = g_dbg_diag_mode >= 0 ? (g_dbg_diag_mode == 1 && S > 1)
-                                               : (S > 1 && 2 * int64_t(G) <= sm_count);
+    const bool two_pass = two_pass_plan && S > 1;
     if (two_pass) {
         const int64_t agg_units = int64_t(G) * (S - 1);
         const size_t head = 256;  // two tickets

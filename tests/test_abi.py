@@ -272,6 +272,35 @@ def test_bwd_scalarA_rejects(over, expect):
     assert _bwd_sa(**over) == C[expect]
 
 
+def test_forward_segment_plan():
+    """The forward's choice of time segments and form (host arithmetic, no
+    GPU): few tiles (2 tiles <= CTAs) with a spread of more than one
+    segment take the two-pass form; otherwise the chained form takes one
+    segment when the tiles fit on the CTAs (a tile's segments run one after
+    another, so more segments only lengthen that chain) and the spread rule
+    (about 8 units per CTA, segments of at least 4 chunks) when they do not.
+    Negative values denote the two-pass form."""
+    plan = ss.debug_fwd_plan
+    assert plan(160, 64, 148) == 8         # B4 D5120 L4096: 8 segments
+    assert plan(96, 32, 148) == 1          # B8 D1536 L2048: one segment per tile
+    assert plan(128, 64, 148) == 1         # B4 D4096 L4096
+    assert plan(75, 64, 148) == 1          # 2 x 75 > 148: still chained
+    assert plan(74, 64, 148) == -16        # 2 x 74 <= 148: two-pass, 16 chunks max
+    assert plan(16, 2048, 148) == -74      # B1 D2048 L131072: two-pass
+    assert plan(320, 16, 148) == 4         # B16 D2560 L1024: spread, capped at 16 / 4
+    assert plan(169, 32, 148) == 8         # the largest chained scratch
+    assert plan(1, 4, 148) == 1            # one chunk group: nothing to split
+    assert plan(0, 10, 10) == 1 and plan(10, 0, 10) == 1 and plan(10, 10, 0) == 1
+    for tiles in (1, 7, 74, 75, 148, 149, 640, 3000):
+        for chunks in (1, 3, 4, 64, 2048):
+            s = plan(tiles, chunks, 148)
+            assert 1 <= abs(s) <= max(1, (chunks + 3) // 4)
+            if s < 0:
+                assert 2 * tiles <= 148 and s < -1
+            elif tiles <= 148:
+                assert s == 1 or 2 * tiles <= 148
+
+
 def test_backward_segment_plan():
     """The backward's choice of time segments (host arithmetic, no GPU):
     ceil(units / slots) / S is minimised over at most four waves, with at
