@@ -275,18 +275,23 @@ def test_bwd_scalarA_rejects(over, expect):
 def test_forward_segment_plan():
     """The forward's choice of time segments and form (host arithmetic, no
     GPU): few tiles (2 tiles <= CTAs) with a spread of more than one
-    segment take the two-pass form; otherwise the chained form takes one
-    segment when the tiles fit on the CTAs (a tile's segments run one after
-    another, so more segments only lengthen that chain) and the spread rule
-    (about 8 units per CTA, segments of at least 4 chunks) when they do not.
-    Negative values denote the two-pass form."""
+    segment take the two-pass form, with the count (at most the spread)
+    that minimises whole waves of units per pass plus the folds of earlier
+    segments; otherwise the chained form takes one segment when the tiles
+    fit on the CTAs (a tile's segments run one after another, so more
+    segments only lengthen that chain) and the spread rule (about 8 units
+    per CTA, segments of at least 4 chunks) when they do not.  Negative
+    values denote the two-pass form."""
     plan = ss.debug_fwd_plan
     assert plan(160, 64, 148) == 8         # B4 D5120 L4096: 8 segments
     assert plan(96, 32, 148) == 1          # B8 D1536 L2048: one segment per tile
     assert plan(128, 64, 148) == 1         # B4 D4096 L4096
     assert plan(75, 64, 148) == 1          # 2 x 75 > 148: still chained
-    assert plan(74, 64, 148) == -16        # 2 x 74 <= 148: two-pass, 16 chunks max
-    assert plan(16, 2048, 148) == -74      # B1 D2048 L131072: two-pass
+    assert plan(74, 64, 148) == -2         # 2 x 74 <= 148: two-pass, one wave of units
+    assert plan(16, 2048, 148) == -37      # B1 D2048 L131072: 4 waves of 56 chunks
+    assert plan(1, 4736, 148) == -148      # one tile, long: one wave (the spread: 1184)
+    assert plan(2, 1024, 148) == -74       # B1 D256 L65536: one wave
+    assert plan(32, 512, 148) == -9        # B2 D2048 L32768
     assert plan(320, 16, 148) == 4         # B16 D2560 L1024: spread, capped at 16 / 4
     assert plan(169, 32, 148) == 8         # the largest chained scratch
     assert plan(1, 4, 148) == 1            # one chunk group: nothing to split
@@ -297,6 +302,8 @@ def test_forward_segment_plan():
             assert 1 <= abs(s) <= max(1, (chunks + 3) // 4)
             if s < 0:
                 assert 2 * tiles <= 148 and s < -1
+                spread = min(-(-8 * 148 // tiles), (chunks + 3) // 4)
+                assert -s <= spread
             elif tiles <= 148:
                 assert s == 1 or 2 * tiles <= 148
 
