@@ -46,12 +46,12 @@ NCU_TRAFFIC = {
     2: ("scan_diag_bf16_kernel lane-per-channel v6", 640.3e6),
     # config 3 (two-pass form, both kernels of one call) captured at
     # L = 32768, scaled by tokens to L = 131072
-    3: ("scan_diag_bf16_kernel lane-per-channel two-pass v6", 2678.5e6),
+    3: ("scan_diag_bf16_kernel lane-per-channel two-pass v7", 2484.5e6),
     4: ("ssd_scalarA_kernel v6", 108.1e6),
 }
 KERNEL_TAG = {2: "scan_diag_bf16_kernel lane-per-channel v6",
               1: "scan_diag_bf16_kernel lane-per-channel v6",
-              3: "scan_diag_bf16_kernel lane-per-channel two-pass v6",
+              3: "scan_diag_bf16_kernel lane-per-channel two-pass v7",
               0: "scan_diag_kernel fp32 v3", 4: "ssd_scalarA_kernel v6"}
 HBM_FALLBACK_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # the HGX/DGX nominal figure, reported beside the measured peak
