@@ -908,8 +908,8 @@ def bwd_bytes(cfg: dict) -> int:
 # L = 1024 and scaled by tokens to L = 4096 (profiles/selscan_bwd_config2.md,
 # profiles/ssd_bwd_scalarA_config4.md)
 BWD_NCU_TRAFFIC = {2: ("selscan_bwd_kernel v5", 4 * 687.2e6),
-                   4: ("ssd_bwd_kernel v8", 4 * 232.6e6)}
-BWD_KERNEL_TAG = {2: "selscan_bwd_kernel v5", 4: "ssd_bwd_kernel v8"}
+                   4: ("ssd_bwd_kernel v9", 4 * 185.6e6)}
+BWD_KERNEL_TAG = {2: "selscan_bwd_kernel v5", 4: "ssd_bwd_kernel v9"}
 
 
 def bwd_traffic(args, cfg):

@@ -43,8 +43,8 @@
 // input is split into two parts (one extra product each), which keeps about
 // 20 bits of it; bf16 inputs are exact in tf32.
 // dB and dC sum over the heads of a group: each head adds its chunk terms
-// with 8-byte atomics into one of kSbCopies partial copies ([t][n] rows),
-// and ssd_bwd_reduce_bc sums the copies into (batch, G, N, L).  dA, dD and
+// with 8-byte atomics into a token-major accumulation buffer ([t][n] rows),
+// and ssd_bwd_reduce_bc transposes it into (batch, G, N, L).  dA, dD and
 // the bias gradient sum over batch rows: one atomic per CTA.
 #pragma once
 
@@ -60,7 +60,11 @@ constexpr int kSbN = 128;       // state size built
 constexpr int kSbP = 64;        // head dimension built
 constexpr int kSbQ = 32;        // tokens per chunk
 constexpr int kSbThreads = 256;
-constexpr int kSbCopies = 8;    // partial copies of dB / dC (head h adds into copy h % 8)
+// Accumulation copies of dB / dC (head h adds into copy h % kSbCopies).  One
+// copy measured fastest on B4 H32 G1 L4096 (1.493 ms; 2, 4, 8, 16 copies:
+// 1.499, 1.506, 1.529, 1.607 ms): zeroing and summing more copies costs more
+// than the contention of 32 heads' atomics on one.
+constexpr int kSbCopies = 1;
 
 struct SsdBwdParams {
     int batch, H, L, nchunks, heads_per_group, G;
