@@ -62,3 +62,73 @@ def selscan_scalarA(inp, parts=None, dt_softplus=False, dt_bias=None, h0=None):
         res = list(ex.map(one, rs))
     return (np.concatenate([r[0] for r in res], axis=1),
             np.concatenate([r[1] for r in res], axis=1))
+
+
+def selscan_bwd(inp, dy, parts=None, delta_softplus=True):
+    """oracle.selscan_bwd over every channel of a diagonal-A input dict with
+    one B/C group, split into channel ranges run in parallel.  The gradients
+    of per-channel quantities (du, ddelta, dz, dA, dD, ddelta_bias) are those
+    of each range, concatenated; dB and dC, sums over all channels, are the
+    sums of the ranges' dB and dC (the loss is a sum over channels)."""
+    u = np.asarray(inp["u"])
+    batch, dim, _ = u.shape
+    B = np.asarray(inp["B"])
+    assert B.ndim == 3 or B.shape[1] == 1, "one B/C group (channel ranges keep no group map)"
+    rs = _ranges(dim, parts or workers())
+
+    def one(r):
+        d0, d1 = r
+        seq = lambda a: None if a is None else np.ascontiguousarray(np.asarray(a)[:, d0:d1])
+        par = lambda a: None if a is None else np.ascontiguousarray(np.asarray(a)[d0:d1])
+        return oracle.selscan_bwd(seq(inp["u"]), seq(inp["delta"]), par(inp["A"]), inp["B"],
+                                  inp["C"], seq(dy), D=par(inp["D"]), z=seq(inp["z"]),
+                                  delta_bias=par(inp["delta_bias"]),
+                                  delta_softplus=delta_softplus)
+
+    with ThreadPoolExecutor(len(rs)) as ex:
+        res = list(ex.map(one, rs))
+    out = {}
+    for k, v in res[0].items():
+        if v is None:
+            out[k] = None
+        elif k in ("dB", "dC"):
+            out[k] = np.sum([r[k] for r in res], axis=0)
+        elif k in ("du", "ddelta", "dz", "dh0"):
+            out[k] = np.concatenate([r[k] for r in res], axis=1)
+        else:
+            out[k] = np.concatenate([r[k] for r in res], axis=0)
+    return out
+
+
+def selscan_scalarA_bwd(inp, dy, parts=None, dt_softplus=False, dt_bias=None):
+    """oracle.selscan_scalarA_bwd over every head of a scalar-A input dict with
+    one B/C group, split into head ranges run in parallel: per-head
+    gradients concatenated, dB and dC summed over the ranges."""
+    H = np.asarray(inp["A"]).shape[0]
+    P = inp["headdim"]
+    B = np.asarray(inp["B"])
+    assert B.ndim == 3 or B.shape[1] == 1, "one B/C group (head ranges keep no group map)"
+    rs = _ranges(H, parts or workers())
+
+    def one(r):
+        h0, h1 = r
+        ch = lambda a: None if a is None else np.ascontiguousarray(np.asarray(a)[:, h0 * P:h1 * P])
+        hd = lambda a: None if a is None else np.ascontiguousarray(np.asarray(a)[:, h0:h1])
+        par = lambda a: None if a is None else np.ascontiguousarray(np.asarray(a)[h0:h1])
+        return oracle.selscan_scalarA_bwd(ch(inp["x"]), hd(inp["dt"]), par(inp["A"]), inp["B"],
+                                          inp["C"], P, ch(dy), D=par(inp["D"]), z=ch(inp["z"]),
+                                          dt_bias=par(dt_bias), dt_softplus=dt_softplus)
+
+    with ThreadPoolExecutor(len(rs)) as ex:
+        res = list(ex.map(one, rs))
+    out = {}
+    for k, v in res[0].items():
+        if v is None:
+            out[k] = None
+        elif k in ("dB", "dC"):
+            out[k] = np.sum([r[k] for r in res], axis=0)
+        elif k in ("dx", "dz", "ddt", "dh0"):
+            out[k] = np.concatenate([r[k] for r in res], axis=1)
+        else:
+            out[k] = np.concatenate([r[k] for r in res], axis=0)
+    return out

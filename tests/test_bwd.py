@@ -167,6 +167,19 @@ def test_full_size_config2_sampled():
     assert not got["du"][:, others].any() and not got["dA"][others].any()
 
 
+def test_full_size_config2_whole():
+    """The benchmark's workload over the whole tensor: every gradient of
+    every channel and token against the oracle, which runs on channel ranges
+    side by side (oracle_par.selscan_bwd; dB and dC are the sums of the
+    ranges' parts)."""
+    import oracle_par
+    inp = synthetic.make_config(2)
+    dy = _dy(inp, 94)
+    got = run(inp, dy, "bf16")
+    want = oracle_par.selscan_bwd(inp, dy)
+    compare(got, want, "bf16")
+
+
 @pytest.mark.parametrize("segs", [1, 3, 16])
 def test_forced_segment_counts(segs):
     """The same gradients whatever the number of time segments per tile:

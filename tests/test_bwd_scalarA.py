@@ -160,3 +160,18 @@ def test_full_size_config4_sampled_heads():
     assert np.all(got["dx"][:, oc] == 0.0)
     assert np.all(got["ddt"][:, others] == 0.0)
     assert np.all(got["dA"][others] == 0.0) and np.all(got["dD"][others] == 0.0)
+
+
+def test_full_size_config4_whole():
+    """The benchmark's workload over the whole tensor: every gradient of
+    every head, channel and token against the oracle, which runs on head
+    ranges side by side (oracle_par.selscan_scalarA_bwd; dB and dC are the
+    sums of the ranges' parts)."""
+    import oracle_par
+    inp = synthetic.make_config(4)
+    rng = np.random.default_rng(405)
+    inp.update(softplus=False, dt_bias=None, h0=None, dlast=None,
+               dy=synthetic.round_bf16(rng.standard_normal(inp["x"].shape).astype(np.float32)))
+    got = run_gpu(inp)
+    want = oracle_par.selscan_scalarA_bwd(inp, inp["dy"])
+    compare(got, want, "config 4 whole")
