@@ -167,14 +167,16 @@ def test_full_size_config2_sampled():
     assert not got["du"][:, others].any() and not got["dA"][others].any()
 
 
-def test_full_size_config2_whole():
-    """The benchmark's workload over the whole tensor: every gradient of
-    every channel and token against the oracle, which runs on channel ranges
-    side by side (oracle_par.selscan_bwd; dB and dC are the sums of the
-    ranges' parts)."""
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_full_size_config_whole(cfg):
+    """Configs 1-3 (B8 D1536 L2048, the benchmark's B4 D5120 L4096, B1 D2048
+    L131072) over the whole tensor, in the launch configurations the library
+    picks for them: every gradient of every channel and token against the
+    oracle, which runs on channel ranges side by side (oracle_par.selscan_bwd;
+    dB and dC are the sums of the ranges' parts)."""
     import oracle_par
-    inp = synthetic.make_config(2)
-    dy = _dy(inp, 94)
+    inp = synthetic.make_config(cfg)
+    dy = _dy(inp, 94 + cfg)
     got = run(inp, dy, "bf16")
     want = oracle_par.selscan_bwd(inp, dy)
     compare(got, want, "bf16")
