@@ -531,6 +531,60 @@ def to_dev(a, dtype, torch):
     return (t.to(torch.bfloat16) if dtype == "bf16" else t.float()).cuda()
 
 
+def pipelined_e2e(torch, stream, steps, pinned, dev_sets, compute, host_outs):
+    """End-to-end steps through the public API, pipelined as a loader drives
+    the call: every step copies its inputs from pinned host memory (``pinned``,
+    name -> tensor) into one of two device buffer sets (``dev_sets``), runs
+    ``compute(j)`` on set j on ``stream`` (it returns the device tensors of
+    the step's results) and copies those results into pinned host memory
+    (``host_outs[j]``, in the same order).  The copies in, the compute and the
+    copies out run on three streams, so step i + 1's inputs go in while step
+    i computes and step i - 1's results come out (PCIe carries both
+    directions at once); events keep a buffer set from being refilled before
+    the step that used it has computed and copied its results out.  Returns
+    the milliseconds per step, from the first copy in to the last copy out,
+    after two untimed steps."""
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+
+    def run(n):
+        for i in range(n):
+            j = i & 1
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_comp[j])  # the step that last read set j has computed
+                for k, t in pinned.items():
+                    dev_sets[j][k].copy_(t, non_blocking=True)
+                ev_in[j].record(s_in)
+            stream.wait_event(ev_in[j])
+            stream.wait_event(ev_out[j])     # set j's previous results are out
+            res = compute(j)
+            ev_comp[j].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[j])
+                for src, dst in zip(res, host_outs[j]):
+                    dst.copy_(src, non_blocking=True)
+                    src.record_stream(s_out)  # keep pooled memory until the copy is done
+                ev_out[j].record(s_out)
+
+    run(2)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with gc_paused():
+        e0.record(s_in)
+        run(steps)
+        stream.wait_event(ev_out[(steps - 1) & 1])
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def second_set(torch, dev, keys):
+    """A second device buffer set for the keys copied in every step."""
+    return {k: (torch.empty_like(v) if (k in keys and v is not None) else v)
+            for k, v in dev.items()}
+
+
 def run_gpu(args, rank: int, world: int, local: int):
     import torch
     import selective_state_space_selscan_b200 as ss
@@ -546,10 +600,10 @@ def run_gpu(args, rank: int, world: int, local: int):
         hs = torch.empty((cfg["batch"], cfg["dim"], cfg["N"]), dtype=torch.float32,
                          device="cuda")
 
-        def call():
-            ss.selscan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
-                           z=dev["z"], delta_bias=dev["delta_bias"], delta_softplus=True,
-                           out=y, last_state=hs)
+        def call_on(d, yy, hh):
+            ss.selscan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"],
+                           z=d["z"], delta_bias=d["delta_bias"], delta_softplus=True,
+                           out=yy, last_state=hh)
         host_in = ("u", "delta", "B", "C", "z", "A", "D", "delta_bias")
     else:
         dev = {k: to_dev(inp[k], dt, torch) for k in ("x", "B", "C", "z")}
@@ -558,11 +612,14 @@ def run_gpu(args, rank: int, world: int, local: int):
         hs = torch.empty((cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["N"]),
                          dtype=torch.float32, device="cuda")
 
-        def call():
-            ss.selscan_fwd_scalarA(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"],
-                                   cfg["headdim"], D=dev["D"], z=dev["z"], out=y,
-                                   last_state=hs)
+        def call_on(d, yy, hh):
+            ss.selscan_fwd_scalarA(d["x"], d["dt"], d["A"], d["B"], d["C"],
+                                   cfg["headdim"], D=d["D"], z=d["z"], out=yy,
+                                   last_state=hh)
         host_in = ("x", "dt", "B", "C", "z", "A", "D")
+
+    def call():
+        call_on(dev, y, hs)
 
     elems = synthetic.elements(args.config)
     dist = world > 1
@@ -613,36 +670,28 @@ def run_gpu(args, rank: int, world: int, local: int):
     ms_per_step = total_ms / args.steps
     value = aggregate_rate(world, elems, ms_per_step) / 1e9
 
-    # end to end through the public API: pinned host inputs -> device,
-    # scan, result back to the host, every step
+    # end to end through the public API, every step: inputs from pinned host
+    # memory in, the scan, y and the final state out (pipelined_e2e)
     pinned = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(
         torch.bfloat16 if (dt == "bf16" and k not in ("A", "D", "delta_bias", "dt")) else
         torch.float32).pin_memory() for k in host_in if inp.get(k) is not None}
-    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    hs_host = torch.empty(hs.shape, dtype=hs.dtype).pin_memory()
+    sets = [(dev, y, hs), (second_set(torch, dev, pinned), torch.empty_like(y),
+                           torch.empty_like(hs))]
+    host_out = [(torch.empty(y.shape, dtype=y.dtype).pin_memory(),
+                 torch.empty(hs.shape, dtype=hs.dtype).pin_memory()) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = y_host.numel() * y_host.element_size() + hs_host.numel() * hs_host.element_size()
-    e2e_steps = max(1, min(args.steps, 10))
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
+    e2e_steps = max(2, min(args.steps, 10))
 
-    def e2e_step():
-        for k, t in pinned.items():
-            dev[k].copy_(t, non_blocking=True)
-        call()
-        y_host.copy_(y, non_blocking=True)
-        hs_host.copy_(hs, non_blocking=True)
+    def compute(j):
+        d, yy, hh = sets[j]
+        call_on(d, yy, hh)
+        return (yy, hh)
 
-    e2e_step()
-    torch.cuda.synchronize()
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with gc_paused():
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
+    e2e_ms = pipelined_e2e(torch, stream, e2e_steps, pinned, [st[0] for st in sets], compute,
+                           host_out)
+    e2e_ms = max_over_ranks([e2e_ms])[0]
     barrier()
     if rank != 0:
         return
@@ -762,14 +811,17 @@ def run_step(args, rank: int, world: int, local: int):
     y = torch.empty(first.shape, dtype=first.dtype, device="cuda")
 
     if cfg["kind"] == "diag":
-        def call():
-            ss.selscan_step(state, dev["u"], dev["delta"], par["A"], dev["B"], dev["C"],
-                            D=par.get("D"), z=dev.get("z"), delta_bias=par.get("delta_bias"),
-                            out=y)
+        def call_on(d, yy):
+            ss.selscan_step(state, d["u"], d["delta"], par["A"], d["B"], d["C"],
+                            D=par.get("D"), z=d.get("z"), delta_bias=par.get("delta_bias"),
+                            out=yy)
     else:
-        def call():
-            ss.selscan_step_scalarA(state, dev["x"], dev["dt"], par["A"], dev["B"], dev["C"],
-                                    cfg["headdim"], D=par.get("D"), z=dev.get("z"), out=y)
+        def call_on(d, yy):
+            ss.selscan_step_scalarA(state, d["x"], d["dt"], par["A"], d["B"], d["C"],
+                                    cfg["headdim"], D=par.get("D"), z=d.get("z"), out=yy)
+
+    def call():
+        call_on(dev, y)
 
     dist = world > 1
     if dist:
@@ -817,34 +869,26 @@ def run_step(args, rank: int, world: int, local: int):
     ms_per_step = total_ms / args.steps
     value = aggregate_rate(world, batch, ms_per_step)
 
-    # end to end: the token's inputs from pinned host memory, y back; the
-    # state stays resident on the device, as a decoding server keeps it
+    # end to end: the token's inputs from pinned host memory, y back, every
+    # step (pipelined_e2e); the state stays resident on the device, as a
+    # decoding server keeps it, and is updated in place step after step
     pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(
         torch.float32 if (k == "dt" or dt == "f32") else torch.bfloat16).pin_memory()
         for k, v in host.items()}
-    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    sets = [dev, second_set(torch, dev, pinned)]
+    ys = [y, torch.empty_like(y)]
+    host_out = [(torch.empty(y.shape, dtype=y.dtype).pin_memory(),) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = y_host.numel() * y_host.element_size()
-    e2e_steps = max(1, min(args.steps, 100))
+    d2h = host_out[0][0].numel() * host_out[0][0].element_size()
+    e2e_steps = max(2, min(args.steps, 100))
 
-    def e2e_step():
-        for k, t in pinned.items():
-            dev[k].copy_(t, non_blocking=True)
-        call()
-        y_host.copy_(y, non_blocking=True)
+    def compute(j):
+        call_on(sets[j], ys[j])
+        return (ys[j],)
 
-    e2e_step()
-    torch.cuda.synchronize()
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with gc_paused():
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
+    e2e_ms = pipelined_e2e(torch, stream, e2e_steps, pinned, sets, compute, host_out)
+    e2e_ms = max_over_ranks([e2e_ms])[0]
     barrier()
     if rank != 0:
         return
@@ -944,12 +988,15 @@ def run_bwd(args, rank: int, world: int, local: int):
         par = {k: to_dev(inp[k], "f32", torch) for k in ("A", "D", "delta_bias")}
     dev["dy"] = to_dev(dy_host, dt, torch)
 
-    def call():
+    def call_on(d):
         if scalar:
-            return ss.selscan_bwd_scalarA(dev["x"], dev["dt"], par["A"], dev["B"], dev["C"],
-                                          inp["headdim"], dev["dy"], D=par["D"], z=dev["z"])
-        return ss.selscan_bwd(dev["u"], dev["delta"], par["A"], dev["B"], dev["C"], dev["dy"],
-                              D=par["D"], z=dev["z"], delta_bias=par["delta_bias"])
+            return ss.selscan_bwd_scalarA(d["x"], d["dt"], par["A"], d["B"], d["C"],
+                                          inp["headdim"], d["dy"], D=par["D"], z=d["z"])
+        return ss.selscan_bwd(d["u"], d["delta"], par["A"], d["B"], d["C"], d["dy"],
+                              D=par["D"], z=d["z"], delta_bias=par["delta_bias"])
+
+    def call():
+        return call_on(dev)
 
     dist = world > 1
     if dist:
@@ -998,37 +1045,28 @@ def run_bwd(args, rank: int, world: int, local: int):
     elems = cfg["batch"] * cfg_dim(cfg) * cfg["L"]
     value = aggregate_rate(world, elems, ms_per_step) / 1e9
 
-    # end to end: inputs and dy from pinned host memory in, every gradient out
+    # end to end: inputs and dy from pinned host memory in, every gradient out,
+    # every step (pipelined_e2e)
     host_keys = ("x", "dt", "B", "C", "z", "dy") if scalar else ("u", "delta", "B", "C", "z", "dy")
     src = dict(inp, dy=dy_host)
     pinned = {k: torch.from_numpy(np.ascontiguousarray(src[k])).to(
         torch.bfloat16 if (dt == "bf16" and k != "dt") else torch.float32).pin_memory()
         for k in host_keys if src.get(k) is not None}
-    outs = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
-            for k, v in grads.items() if v is not None}
+    out_keys = [k for k, v in grads.items() if v is not None]
+    host_out = [tuple(torch.empty(grads[k].shape, dtype=grads[k].dtype).pin_memory()
+                      for k in out_keys) for _ in range(2)]
+    sets = [dev, second_set(torch, dev, pinned)]
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs.values())
-    e2e_steps = max(1, min(args.steps, 10))
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
+    e2e_steps = max(2, min(args.steps, 10))
 
-    def e2e_step():
-        for k, t in pinned.items():
-            dev[k].copy_(t, non_blocking=True)
-        g = call()
-        for k, t in outs.items():
-            t.copy_(g[k], non_blocking=True)
+    def compute(j):
+        g = call_on(sets[j])
+        return tuple(g[k] for k in out_keys)
 
-    e2e_step()
-    torch.cuda.synchronize()
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with gc_paused():
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps])[0]
+    e2e_ms = pipelined_e2e(torch, stream, e2e_steps, pinned, sets, compute, host_out)
+    e2e_ms = max_over_ranks([e2e_ms])[0]
     barrier()
     if rank != 0:
         return
